@@ -1,0 +1,338 @@
+/*
+ * dsa_oracle.c -- plain, slow fp64 CPU oracle for DeepSeek Sparse Attention.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing in the product path may link, load or
+ * call this file; only the tests, __graft_entry__.smoke() and the benchmark's
+ * CPU-baseline leg do.  It shares no code, header, table or constant with the
+ * CUDA library.
+ *
+ * What it computes, stage by stage (the plain definition, no blocking, no
+ * fusion, no reordering):
+ *
+ *  1. Lightning indexer ("DeepSeek-V3.2-Exp DSA 技术深度解析", section 1: a
+ *     light indexer with few heads, low-dimensional FP8 query/key and ReLU
+ *     scores every history token of a query):
+ *        I[t,s] = sum_h w[t,h] * max(0, sum_j qhat[t,h,j] * khat[s,j]),  0 <= s <= t
+ *     with qhat = e4m3(q8) * sq[t], khat = e4m3(k8) * sk[s] (per-token fp32
+ *     scales; fp32 inputs are used as they are).
+ *  2. Top-k selector (same section; the "fine-grained selector" of the hotdry
+ *     page): the min(k, t+1) positions s <= t with the largest I[t,s], ties
+ *     to the lower s, emitted in ascending s and padded with -1.
+ *  3. Main attention over the selected set only (same section; O(L^2) ->
+ *     O(L k)):  z_j = sm * q[t,h] . K[j],  p = softmax(z),  o = sum_j p_j V[j],
+ *     lse = max z + log sum exp(z - max z), natural log.
+ *  4. Decode: stages 1-3 for one query per sequence whose context (already
+ *     holding the current token) lives in paged caches.
+ *
+ * Number formats are decoded from their published definitions:
+ *   E4M3 (OCP 8-bit floating point, "E4M3FN"): 1 sign, 4 exponent (bias 7),
+ *   3 mantissa bits, subnormals when the exponent field is 0, no infinities,
+ *   S.1111.111 is NaN; largest finite magnitude 448.
+ *   bfloat16: the upper 16 bits of an IEEE-754 binary32.
+ *
+ * Build: gcc -O2 -fopenmp -shared -fPIC (no fast-math: every sum is taken in
+ * the order written here, in double precision).
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+enum { OR_F32 = 0, OR_BF16 = 1, OR_E4M3 = 2 };
+
+/* ---------------- number formats ---------------- */
+
+double dsa_or_e4m3(uint8_t code)
+{
+    int sign = (code >> 7) & 1;
+    int e = (code >> 3) & 0xF;
+    int m = code & 0x7;
+    double mag;
+    if (e == 0xF && m == 0x7) return NAN;             /* the only NaN pattern */
+    if (e == 0) mag = ldexp((double)m / 8.0, 1 - 7);   /* subnormal: 0.m * 2^(1-bias) */
+    else mag = ldexp(1.0 + (double)m / 8.0, e - 7);    /* normal: 1.m * 2^(e-bias) */
+    return sign ? -mag : mag;
+}
+
+double dsa_or_bf16(uint16_t bits)
+{
+    uint32_t u = (uint32_t)bits << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return (double)f;
+}
+
+static double load_elem(const void *p, int dtype, int64_t i)
+{
+    switch (dtype) {
+    case OR_F32: return (double)((const float *)p)[i];
+    case OR_BF16: return dsa_or_bf16(((const uint16_t *)p)[i]);
+    case OR_E4M3: return dsa_or_e4m3(((const uint8_t *)p)[i]);
+    }
+    return NAN;
+}
+
+/* ---------------- stage 1: indexer scores ---------------- */
+
+/* One score I[t,s].  q_row: the H*D dequantised query values of token t;
+ * k_row: the D dequantised key values of token s; w_row: H weights. */
+static double index_score(const double *q_row, const double *k_row, const double *w_row,
+                          int H, int D)
+{
+    double total = 0.0;
+    for (int h = 0; h < H; ++h) {
+        double dot = 0.0;
+        for (int j = 0; j < D; ++j) dot += q_row[(int64_t)h * D + j] * k_row[j];
+        double relu = dot > 0.0 ? dot : 0.0;
+        total += w_row[h] * relu;
+    }
+    return total;
+}
+
+/* Dequantise the whole key matrix once: khat[s,j] = value(k[s,j]) * sk[s]. */
+static double *dequant_keys(const void *k_idx, const float *k_scale, int kdt, int64_t T, int D)
+{
+    double *khat = (double *)malloc(sizeof(double) * (size_t)T * D);
+    if (!khat) return NULL;
+#pragma omp parallel for schedule(static)
+    for (int64_t s = 0; s < T; ++s) {
+        double sc = k_scale ? (double)k_scale[s] : 1.0;
+        for (int j = 0; j < D; ++j) khat[s * D + j] = load_elem(k_idx, kdt, s * D + j) * sc;
+    }
+    return khat;
+}
+
+/* qhat / w for one query token t. */
+static void dequant_query(const void *q_idx, const float *q_scale, int qdt, const void *w, int wdt,
+                          int64_t t, int H, int D, double *q_row, double *w_row)
+{
+    double sc = q_scale ? (double)q_scale[t] : 1.0;
+    for (int64_t i = 0; i < (int64_t)H * D; ++i)
+        q_row[i] = load_elem(q_idx, qdt, t * H * D + i) * sc;
+    for (int h = 0; h < H; ++h) w_row[h] = load_elem(w, wdt, t * H + h);
+}
+
+/*
+ * Scores of the query rows rows[0..nrows) against every key 0..T-1:
+ * out[r*T + s] = I[rows[r], s] for s <= rows[r], -inf for s > rows[r].
+ * idx_dtype: OR_F32 (q/k fp32, no scales) or OR_E4M3 (q/k bytes + scales);
+ * w_dtype: OR_F32 or OR_BF16.  Returns 0, or -1 on allocation failure.
+ */
+int dsa_or_index_scores(const void *q_idx, const float *q_scale, const void *k_idx,
+                        const float *k_scale, const void *w, int idx_dtype, int w_dtype,
+                        int64_t T, int H, int D, const int64_t *rows, int64_t nrows, double *out)
+{
+    double *khat = dequant_keys(k_idx, k_scale, idx_dtype, T, D);
+    if (!khat) return -1;
+    int err = 0;
+#pragma omp parallel
+    {
+        double *q_row = (double *)malloc(sizeof(double) * (size_t)H * D);
+        double *w_row = (double *)malloc(sizeof(double) * (size_t)H);
+        if (!q_row || !w_row) {
+#pragma omp atomic write
+            err = -1;
+        } else {
+#pragma omp for schedule(dynamic, 1)
+            for (int64_t r = 0; r < nrows; ++r) {
+                int64_t t = rows[r];
+                dequant_query(q_idx, q_scale, idx_dtype, w, w_dtype, t, H, D, q_row, w_row);
+                for (int64_t s = 0; s < T; ++s)
+                    out[r * T + s] = (s <= t) ? index_score(q_row, khat + s * D, w_row, H, D)
+                                              : -INFINITY;
+            }
+        }
+        free(q_row);
+        free(w_row);
+    }
+    free(khat);
+    return err;
+}
+
+/* ---------------- stage 2: top-k ---------------- */
+
+typedef struct { double score; int64_t pos; } cand_t;
+
+/* (score descending, position ascending): the selector's total order. */
+static int cand_cmp(const void *a, const void *b)
+{
+    const cand_t *x = (const cand_t *)a, *y = (const cand_t *)b;
+    if (x->score > y->score) return -1;
+    if (x->score < y->score) return 1;
+    return (x->pos < y->pos) ? -1 : (x->pos > y->pos);
+}
+
+static int pos_cmp(const void *a, const void *b)
+{
+    int32_t x = *(const int32_t *)a, y = *(const int32_t *)b;
+    return (x > y) - (x < y);
+}
+
+/* Select from scores[0..n) (n = t+1 candidates) the min(k,n) best positions. */
+static int select_row(const double *scores, int64_t n, int k, int32_t *out, cand_t *buf)
+{
+    for (int64_t s = 0; s < n; ++s) { buf[s].score = scores[s]; buf[s].pos = s; }
+    qsort(buf, (size_t)n, sizeof(cand_t), cand_cmp);
+    int64_t m = n < k ? n : k;
+    for (int64_t i = 0; i < m; ++i) out[i] = (int32_t)buf[i].pos;
+    qsort(out, (size_t)m, sizeof(int32_t), pos_cmp);
+    for (int64_t i = m; i < k; ++i) out[i] = -1;
+    return 0;
+}
+
+/*
+ * Top-k of each score row: row r holds the scores of query position rows[r]
+ * (entries 0..rows[r] are candidates, the rest is ignored), with leading
+ * dimension ld.  idx_out[r*k + i]: selected positions ascending, -1 padded.
+ */
+int dsa_or_topk(const double *scores, int64_t ld, const int64_t *rows, int64_t nrows, int k,
+                int32_t *idx_out)
+{
+    int err = 0;
+#pragma omp parallel
+    {
+        int64_t maxn = 0;
+        for (int64_t r = 0; r < nrows; ++r) if (rows[r] + 1 > maxn) maxn = rows[r] + 1;
+        cand_t *buf = (cand_t *)malloc(sizeof(cand_t) * (size_t)(maxn > 0 ? maxn : 1));
+        if (!buf) {
+#pragma omp atomic write
+            err = -1;
+        } else {
+#pragma omp for schedule(dynamic, 4)
+            for (int64_t r = 0; r < nrows; ++r)
+                select_row(scores + r * ld, rows[r] + 1, k, idx_out + r * k, buf);
+        }
+        free(buf);
+    }
+    return err;
+}
+
+/* ---------------- stage 3: attention over the selected set ---------------- */
+
+/* Attention of one query token (H heads of dimension D) over the rows listed
+ * in sel[0..k) (-1 = unused).  krow(j)/vrow(j) give the key / value element
+ * offsets of cache row j.  Writes o[H*D] and lse[H] (lse = -inf, o = 0 when
+ * nothing is selected). */
+static void attend_one(const void *q, int64_t q_off, const void *K, const void *V, int dtype,
+                       const int64_t *koff, int64_t nsel, int H, int D, double sm,
+                       double *o, double *lse, double *z)
+{
+    for (int h = 0; h < H; ++h) {
+        double zmax = -INFINITY;
+        for (int64_t j = 0; j < nsel; ++j) {
+            double dot = 0.0;
+            for (int c = 0; c < D; ++c)
+                dot += load_elem(q, dtype, q_off + (int64_t)h * D + c) * load_elem(K, dtype, koff[j] + c);
+            z[j] = sm * dot;
+            if (z[j] > zmax) zmax = z[j];
+        }
+        double l = 0.0;
+        for (int64_t j = 0; j < nsel; ++j) { z[j] = exp(z[j] - zmax); l += z[j]; }
+        for (int c = 0; c < D; ++c) {
+            double acc = 0.0;
+            for (int64_t j = 0; j < nsel; ++j) acc += z[j] * load_elem(V, dtype, koff[j] + c);
+            o[(int64_t)h * D + c] = nsel > 0 ? acc / l : 0.0;
+        }
+        lse[h] = nsel > 0 ? zmax + log(l) : -INFINITY;
+    }
+}
+
+/*
+ * Sparse attention for query rows rows[0..nrows): q [T,H,D], K/V [T,D] of
+ * dtype OR_F32 or OR_BF16; idx [nrows, k] (row r = query position rows[r]),
+ * entries -1 ignored.  out [nrows, H, D], lse [nrows, H] (nullable).
+ */
+int dsa_or_sparse_attn(const void *q, const void *K, const void *V, int dtype, const int32_t *idx,
+                       const int64_t *rows, int64_t nrows, int k, int H, int D, double sm,
+                       double *out, double *lse)
+{
+    int err = 0;
+#pragma omp parallel
+    {
+        int64_t *koff = (int64_t *)malloc(sizeof(int64_t) * (size_t)k);
+        double *z = (double *)malloc(sizeof(double) * (size_t)k);
+        double *l = (double *)malloc(sizeof(double) * (size_t)H);
+        if (!koff || !z || !l) {
+#pragma omp atomic write
+            err = -1;
+        } else {
+#pragma omp for schedule(dynamic, 1)
+            for (int64_t r = 0; r < nrows; ++r) {
+                int64_t n = 0;
+                for (int i = 0; i < k; ++i) {
+                    int32_t j = idx[r * k + i];
+                    if (j >= 0) koff[n++] = (int64_t)j * D;
+                }
+                attend_one(q, rows[r] * H * D, K, V, dtype, koff, n, H, D, sm,
+                           out + r * H * D, l, z);
+                if (lse) for (int h = 0; h < H; ++h) lse[r * H + h] = l[h];
+            }
+        }
+        free(koff); free(z); free(l);
+    }
+    return err;
+}
+
+/* ---------------- stage 4: decode over paged caches ---------------- */
+
+/*
+ * One decode step for B sequences.  Sequence b has n = ctx[b] cached tokens
+ * (the current token included) at positions 0..n-1; position s lives in
+ * physical page bt[b*max_pages + s/ps], slot s%ps.
+ *   q_idx  e4m3 [B,H_I,D_I], q_scale [B], w bf16 [B,H_I], q bf16 [B,H_q,D]
+ *   kidx   e4m3 [P,ps,D_I], kscale f32 [P,ps], kc/vc bf16 [P,ps,D]
+ * Outputs: scores_out [B, ld] (nullable; entries s < n), idx_out [B,k]
+ * (positions, ascending, -1 padded), out [B,H_q,D], lse [B,H_q] (nullable).
+ */
+int dsa_or_decode(const uint8_t *q_idx, const float *q_scale, const uint16_t *w,
+                  const uint16_t *q, const uint8_t *kidx, const float *kscale,
+                  const uint16_t *kc, const uint16_t *vc, const int32_t *bt,
+                  const int32_t *ctx, int B, int max_pages, int ps, int H_I, int D_I,
+                  int H_q, int D, int k, double sm, double *scores_out, int64_t ld,
+                  int32_t *idx_out, double *out, double *lse)
+{
+    int err = 0;
+    for (int b = 0; b < B && !err; ++b) {
+        int64_t n = ctx[b];
+        double *sc = (double *)malloc(sizeof(double) * (size_t)(n > 0 ? n : 1));
+        double *q_row = (double *)malloc(sizeof(double) * (size_t)H_I * D_I);
+        double *w_row = (double *)malloc(sizeof(double) * (size_t)H_I);
+        cand_t *buf = (cand_t *)malloc(sizeof(cand_t) * (size_t)(n > 0 ? n : 1));
+        int64_t *koff = (int64_t *)malloc(sizeof(int64_t) * (size_t)k);
+        double *z = (double *)malloc(sizeof(double) * (size_t)k);
+        if (!sc || !q_row || !w_row || !buf || !koff || !z) err = -1;
+        if (!err) {
+            double sq = q_scale[b];
+            for (int64_t i = 0; i < (int64_t)H_I * D_I; ++i)
+                q_row[i] = dsa_or_e4m3(q_idx[(int64_t)b * H_I * D_I + i]) * sq;
+            for (int h = 0; h < H_I; ++h) w_row[h] = dsa_or_bf16(w[(int64_t)b * H_I + h]);
+#pragma omp parallel
+            {
+                double k_row[1024];
+#pragma omp for schedule(static)
+                for (int64_t s = 0; s < n; ++s) {
+                    int64_t page = bt[(int64_t)b * max_pages + s / ps];
+                    int64_t slot = page * ps + s % ps;
+                    double sk = kscale[slot];
+                    for (int j = 0; j < D_I; ++j) k_row[j] = dsa_or_e4m3(kidx[slot * D_I + j]) * sk;
+                    sc[s] = index_score(q_row, k_row, w_row, H_I, D_I);
+                }
+            }
+            if (scores_out) for (int64_t s = 0; s < n; ++s) scores_out[(int64_t)b * ld + s] = sc[s];
+            int32_t *sel = idx_out + (int64_t)b * k;
+            select_row(sc, n, k, sel, buf);
+            int64_t m = 0;
+            for (int i = 0; i < k; ++i) {
+                if (sel[i] < 0) continue;
+                int64_t page = bt[(int64_t)b * max_pages + sel[i] / ps];
+                koff[m++] = (page * ps + sel[i] % ps) * D;
+            }
+            double l[1024];
+            attend_one(q, (int64_t)b * H_q * D, kc, vc, OR_BF16, koff, m, H_q, D, sm,
+                       out + (int64_t)b * H_q * D, l, z);
+            if (lse) for (int h = 0; h < H_q; ++h) lse[(int64_t)b * H_q + h] = l[h];
+        }
+        free(sc); free(q_row); free(w_row); free(buf); free(koff); free(z);
+    }
+    return err;
+}
