@@ -1,0 +1,188 @@
+/*
+ * dsa.h -- C ABI of a B200 (sm_100a) library for the hot path of DeepSeek
+ * Sparse Attention (DSA).
+ *
+ * The method ("DeepSeek-V3.2-Exp DSA 技术深度解析", section 1; "DeepSeek V4 ...
+ * 稀疏注意力" on hotdry, section on the lightning indexer and the fine-grained
+ * selector): before the main attention, a light "lightning indexer" with few
+ * heads, a low-dimensional FP8 query/key (index_head_dim 128) and ReLU scores
+ * every history token of each query token; a top-k selector keeps the k
+ * best-scoring KV entries; the main attention then runs over those k entries
+ * only, so its cost falls from O(n^2) to O(n k) while the indexer stays O(n^2)
+ * with a tiny constant.  Concretely, for query token t and history token s<=t:
+ *
+ *     I[t,s] = sum_h w[t,h] * ReLU( qI[t,h] . kI[s] )                 (indexer)
+ *     S_t    = the min(k, t+1) positions s <= t with the largest I[t,s],
+ *              ties broken toward the lower s                          (top-k)
+ *     o[t,h] = sum_{j in S_t} softmax_j( sm * q[t,h] . K[j] ) V[j]     (attention)
+ *
+ * with one shared index-key head, per-head weights w, FP8 E4M3 index query
+ * and key values each carrying one fp32 scale per token
+ * (qI[t,h,:] = e4m3(q8[t,h,:]) * sq[t], kI[s,:] = e4m3(k8[s,:]) * sk[s]), and
+ * one shared K/V head for all query heads (multi-query attention; one index
+ * set S_t shared by all query heads of token t).
+ *
+ * Conventions for every entry point
+ *  - Returns dsa_status.  No C++ exception crosses this boundary.
+ *  - Tensor pointers are DEVICE memory owned by the caller, dense row-major
+ *    in the layouts stated per function, 16-byte aligned.  The library never
+ *    keeps a pointer after the call returns and never frees one.
+ *  - The library allocates no device memory.  Entry points that need scratch
+ *    take a caller workspace of at least dsa_*_workspace_size(...) bytes,
+ *    256-byte aligned; its first 256 bytes hold a device status word.
+ *  - Work is enqueued asynchronously on `stream` (a cudaStream_t; NULL is the
+ *    legacy default stream).  Argument errors are detected on the host and
+ *    returned before anything is enqueued.  Errors that only the device can
+ *    see (a bounded wait that timed out, a page id out of range) are written
+ *    to the workspace status word; read them with dsa_stream_status().
+ *  - All sizes are element counts unless stated otherwise.
+ */
+#ifndef DSA_H_
+#define DSA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define DSA_VERSION_MAJOR 0
+#define DSA_VERSION_MINOR 1
+
+typedef enum dsa_status {
+    DSA_OK = 0,
+    DSA_ERR_INVALID_ARG = 1,  /* null/misaligned pointer, bad size, non-positive k, ... */
+    DSA_ERR_UNSUPPORTED = 2,  /* shape or dtype this build has no kernel for */
+    DSA_ERR_WORKSPACE = 3,    /* workspace missing or smaller than required */
+    DSA_ERR_CUDA = 4,         /* a CUDA runtime call failed (launch, sync, ...) */
+    DSA_ERR_TIMEOUT = 5       /* a device-side bounded wait gave up */
+} dsa_status;
+
+typedef enum dsa_dtype {
+    DSA_F32 = 0,   /* all operands fp32 (no FP8 scales) */
+    DSA_BF16 = 1,  /* bf16 values */
+    DSA_E4M3 = 2   /* FP8 E4M3 index query/key bytes + fp32 per-token scales; bf16 w, Q, K, V */
+} dsa_dtype;
+
+/* Human-readable name of a status code (static storage, never NULL). */
+const char *dsa_status_string(dsa_status s);
+
+/* (DSA_VERSION_MAJOR << 16) | DSA_VERSION_MINOR. */
+int dsa_version(void);
+
+/*
+ * dsa_index_scores -- lightning-indexer scores of a block of query rows
+ * (DSA section 1: light indexer, few heads, FP8, ReLU, every history token).
+ *
+ *   dtype == DSA_E4M3: q_idx uint8 E4M3 [T, H_I, d_I]; q_scale f32 [T];
+ *                      k_idx uint8 E4M3 [T, d_I];    k_scale f32 [T];
+ *                      w bf16 [T, H_I].  Scales finite and > 0.
+ *   dtype == DSA_F32:  q_idx f32 [T, H_I, d_I]; k_idx f32 [T, d_I]; w f32
+ *                      [T, H_I]; q_scale and k_scale must be NULL.
+ * Writes, for r in [0, q_row_count) and s in [0, T), with t = q_row_begin + r:
+ *   scores_out[r * ld_scores + s] = I[t, s] (fp32) if s <= t, else -inf.
+ * Requires 0 <= q_row_begin, q_row_begin + q_row_count <= T, ld_scores >= T.
+ * Supported: E4M3 with d_I == 128 and 1 <= H_I <= 128; F32 with d_I <= 256,
+ * H_I <= 64.  q_row_count == 0 is a no-op.
+ */
+dsa_status dsa_index_scores(const void *q_idx, const float *q_scale, const void *k_idx,
+                            const float *k_scale, const void *w, int64_t T, int H_I, int d_I,
+                            int64_t q_row_begin, int64_t q_row_count, float *scores_out,
+                            int64_t ld_scores, dsa_dtype dtype, void *stream);
+
+/*
+ * dsa_topk -- the top-k selector (DSA section 1; the "fine-grained selector"):
+ * for each row r (query position t = row_begin + r), the min(k, t+1)
+ * positions s in [0, t] with the largest scores[r * ld_scores + s]; equal
+ * scores go to the lower s, and +0 equals -0.  Entries past t are not read.
+ *   idx_out int32 [row_count, k]: selected positions in ascending order,
+ *   padded with -1.  Scores must not be NaN.
+ * Bit-exact: the set is unique under the stated order.
+ * Requires row_begin + row_count <= T, ld_scores >= T, 1 <= k <= 65536.
+ * workspace: at least dsa_topk_workspace_size(row_count, T, k) bytes (may be
+ * NULL when that size is 0).
+ */
+size_t dsa_topk_workspace_size(int64_t row_count, int64_t T, int k);
+dsa_status dsa_topk(const float *scores, int64_t ld_scores, int64_t row_begin,
+                    int64_t row_count, int64_t T, int k, int32_t *idx_out, void *workspace,
+                    size_t ws_bytes, void *stream);
+
+/*
+ * dsa_sparse_attn -- main attention restricted to the selected KV rows
+ * (DSA section 1: the main attention only looks at the selected subset).
+ *   q   [T, H_q, d], k and v [T, d] (one shared KV head), out [T, H_q, d]:
+ *       all bf16 (dtype DSA_BF16 or DSA_E4M3) or all f32 (DSA_F32).
+ *   idx int32 [T, k_sel]: row t lists the KV rows query t attends to; -1
+ *       entries are skipped, and so is any entry outside [0, T).
+ *   lse_out f32 [T, H_q] (nullable): natural-log log-sum-exp of the scaled
+ *       logits sm_scale * q.K over the attended rows (-inf if none).
+ *   o[t,h] = sum_j softmax_j(sm_scale * q[t,h].K[j]) V[j]; 0 if no row.
+ * Supported: bf16 with d in {64, 128}, H_q <= 128 or a multiple of 128;
+ * f32 with d <= 128.
+ */
+dsa_status dsa_sparse_attn(const void *q, const void *k, const void *v, const int32_t *idx,
+                           int64_t T, int H_q, int d, int k_sel, float sm_scale, void *out,
+                           float *lse_out, dsa_dtype dtype, void *stream);
+
+/*
+ * dsa_prefill -- the whole prefill hot path of one sequence: indexer, top-k
+ * and sparse attention for every query token 0..T-1 (layouts as in the
+ * three stage functions above; dtype DSA_E4M3 or DSA_F32).
+ *   out [T, H_q, d]; lse_out [T, H_q] (nullable); idx_out int32 [T, k_sel]
+ *   (nullable: the selection is then kept in the workspace only).
+ * workspace: at least dsa_prefill_workspace_size(...) bytes.  A larger
+ * workspace lets the indexer process more query rows per pass.
+ */
+size_t dsa_prefill_workspace_size(int64_t T, int H_I, int d_I, int H_q, int d, int k_sel,
+                                  dsa_dtype dtype);
+dsa_status dsa_prefill(const void *q_idx, const float *q_scale, const void *k_idx,
+                       const float *k_scale, const void *w, const void *q, const void *k,
+                       const void *v, int64_t T, int H_I, int d_I, int H_q, int d, int k_sel,
+                       float sm_scale, void *out, float *lse_out, int32_t *idx_out,
+                       dsa_dtype dtype, void *workspace, size_t ws_bytes, void *stream);
+
+/*
+ * dsa_decode -- one decode step of B sequences against paged caches (the
+ * current token is already appended; DSA on the decode path, plus the FP8
+ * index-key cache).
+ *   q_idx  uint8 E4M3 [B, H_I, d_I]; q_scale f32 [B]; w bf16 [B, H_I];
+ *   q      bf16 [B, H_q, d];
+ *   kidx_cache   uint8 E4M3 [num_pages, page_size, d_I];
+ *   kscale_cache f32 [num_pages, page_size];
+ *   k_cache, v_cache bf16 [num_pages, page_size, d];
+ *   block_table  int32 [B, max_pages_per_seq]: physical page of each logical
+ *                page (position s of sequence b is in page
+ *                block_table[b, s / page_size], slot s % page_size);
+ *   context_lens int32 [B]: tokens cached per sequence, current one included;
+ *                each in [1, max_context] and <= max_pages_per_seq*page_size.
+ * Outputs: out bf16 [B, H_q, d]; lse_out f32 [B, H_q] (nullable); idx_out
+ * int32 [B, k_sel] (nullable): selected positions ascending, -1 padded.
+ * A page id outside [0, num_pages) or a context length out of range is
+ * reported as DSA_ERR_INVALID_ARG through dsa_stream_status (the offending
+ * rows are skipped, nothing is read out of bounds).
+ * Supported: d_I == 128, H_I <= 64 and a multiple of 8, d == 128,
+ * page_size a multiple of 16, H_q <= 128 or a multiple of 128.
+ */
+size_t dsa_decode_workspace_size(int B, int64_t max_context, int H_q, int d, int k_sel);
+dsa_status dsa_decode(const void *q_idx, const float *q_scale, const void *w, const void *q,
+                      const void *kidx_cache, const float *kscale_cache, const void *k_cache,
+                      const void *v_cache, const int32_t *block_table,
+                      const int32_t *context_lens, int64_t num_pages, int max_pages_per_seq,
+                      int page_size, int B, int64_t max_context, int H_I, int d_I, int H_q,
+                      int d, int k_sel, float sm_scale, void *out, float *lse_out,
+                      int32_t *idx_out, void *workspace, size_t ws_bytes, void *stream);
+
+/*
+ * dsa_stream_status -- waits for `stream`, then returns the device status
+ * word of `workspace` (DSA_OK if no device-side error was recorded by the
+ * last call that used this workspace) and resets it to DSA_OK.
+ * Returns DSA_ERR_CUDA if the synchronisation itself fails.
+ */
+dsa_status dsa_stream_status(void *workspace, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DSA_H_ */

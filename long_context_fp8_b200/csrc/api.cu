@@ -1,0 +1,277 @@
+// C entry points: argument validation, workspace carving, stage sequencing.
+// Everything numeric happens in the kernels; this file only checks and launches.
+#include <cmath>
+
+#include "kernels.h"
+
+using namespace dsa;
+
+namespace {
+
+inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline cudaStream_t as_stream(void *s) { return reinterpret_cast<cudaStream_t>(s); }
+inline dsa_status cuda_status(cudaError_t e) { return e == cudaSuccess ? DSA_OK : DSA_ERR_CUDA; }
+
+// Row block of the prefill indexer pass: as many rows as the score buffer holds.
+constexpr int64_t kPrefillRowsDefault = 8192;
+constexpr size_t kPrefillScoreBudget = size_t(4) << 30;
+
+inline int64_t prefill_rows_default(int64_t T)
+{
+    int64_t r = (int64_t)(kPrefillScoreBudget / (sizeof(float) * (size_t)(T > 0 ? T : 1)));
+    r = r < kPrefillRowsDefault ? r : kPrefillRowsDefault;
+    r = r / 64 * 64;
+    if (r < 64) r = 64;
+    int64_t tr = ceil_div(T, 64) * 64;
+    return r < tr ? r : tr;
+}
+
+inline size_t idx_bytes(int64_t rows, int k) { return align_up(sizeof(int32_t) * (size_t)rows * k, 256); }
+
+dsa_status check_index_args(const void *q_idx, const float *q_scale, const void *k_idx,
+                            const float *k_scale, const void *w, int64_t T, int H_I, int d_I,
+                            dsa_dtype dtype)
+{
+    if (!q_idx || !k_idx || !w || T <= 0 || H_I <= 0 || d_I <= 0) return DSA_ERR_INVALID_ARG;
+    if (!aligned16(q_idx) || !aligned16(k_idx)) return DSA_ERR_INVALID_ARG;
+    if (dtype == DSA_E4M3) {
+        if (!q_scale || !k_scale) return DSA_ERR_INVALID_ARG;
+        if (d_I != 128 || H_I > 128) return DSA_ERR_UNSUPPORTED;
+    } else if (dtype == DSA_F32) {
+        if (q_scale || k_scale) return DSA_ERR_INVALID_ARG;
+        if (d_I > 256 || H_I > 64) return DSA_ERR_UNSUPPORTED;
+    } else {
+        return DSA_ERR_UNSUPPORTED;
+    }
+    return DSA_OK;
+}
+
+dsa_status check_attn_args(const void *q, const void *k, const void *v, const int32_t *idx,
+                           int64_t T, int H_q, int d, int k_sel, const void *out, dsa_dtype dtype)
+{
+    if (!q || !k || !v || !idx || !out || T <= 0 || H_q <= 0 || d <= 0 || k_sel <= 0)
+        return DSA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return DSA_ERR_INVALID_ARG;
+    if (dtype == DSA_F32) {
+        if (d > 128 || H_q > 32) return DSA_ERR_UNSUPPORTED;
+    } else if (dtype == DSA_BF16 || dtype == DSA_E4M3) {
+        if (d != 128 && d != 64) return DSA_ERR_UNSUPPORTED;
+        if (H_q > 128 && H_q % 128 != 0) return DSA_ERR_UNSUPPORTED;
+        if (H_q > 65535 * 128) return DSA_ERR_UNSUPPORTED;
+    } else {
+        return DSA_ERR_UNSUPPORTED;
+    }
+    return DSA_OK;
+}
+
+cudaError_t run_attn(const void *q, const void *k, const void *v, const int32_t *idx, int64_t T,
+                     int H_q, int d, int k_sel, float sm_scale, void *out, float *lse,
+                     dsa_dtype dtype, cudaStream_t st)
+{
+    if (dtype == DSA_F32)
+        return launch_sparse_attn_f32((const float *)q, (const float *)k, (const float *)v, idx,
+                                      T, H_q, d, k_sel, sm_scale, (float *)out, lse, st);
+    return launch_sparse_attn_bf16((const uint16_t *)q, (const uint16_t *)k, (const uint16_t *)v,
+                                   idx, T, T, H_q, d, k_sel, sm_scale, (uint16_t *)out, lse, st);
+}
+
+cudaError_t run_index(const void *q_idx, const float *q_scale, const void *k_idx,
+                      const float *k_scale, const void *w, int64_t T, int H_I, int d_I,
+                      int64_t row_begin, int64_t row_count, float *out, int64_t ld,
+                      bool write_upper, dsa_dtype dtype, cudaStream_t st)
+{
+    if (dtype == DSA_E4M3)
+        return launch_index_fp8((const uint8_t *)q_idx, q_scale, (const uint8_t *)k_idx, k_scale,
+                                (const uint16_t *)w, T, H_I, row_begin, row_count, out, ld,
+                                write_upper, st);
+    return launch_index_f32((const float *)q_idx, (const float *)k_idx, (const float *)w, T, H_I,
+                            d_I, row_begin, row_count, out, ld, write_upper, st);
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *dsa_status_string(dsa_status s)
+{
+    switch (s) {
+    case DSA_OK: return "DSA_OK";
+    case DSA_ERR_INVALID_ARG: return "DSA_ERR_INVALID_ARG";
+    case DSA_ERR_UNSUPPORTED: return "DSA_ERR_UNSUPPORTED";
+    case DSA_ERR_WORKSPACE: return "DSA_ERR_WORKSPACE";
+    case DSA_ERR_CUDA: return "DSA_ERR_CUDA";
+    case DSA_ERR_TIMEOUT: return "DSA_ERR_TIMEOUT";
+    }
+    return "DSA_ERR_UNKNOWN";
+}
+
+int dsa_version(void) { return (DSA_VERSION_MAJOR << 16) | DSA_VERSION_MINOR; }
+
+dsa_status dsa_index_scores(const void *q_idx, const float *q_scale, const void *k_idx,
+                            const float *k_scale, const void *w, int64_t T, int H_I, int d_I,
+                            int64_t q_row_begin, int64_t q_row_count, float *scores_out,
+                            int64_t ld_scores, dsa_dtype dtype, void *stream)
+{
+    dsa_status s = check_index_args(q_idx, q_scale, k_idx, k_scale, w, T, H_I, d_I, dtype);
+    if (s != DSA_OK) return s;
+    if (q_row_begin < 0 || q_row_count < 0 || q_row_begin + q_row_count > T) return DSA_ERR_INVALID_ARG;
+    if (q_row_count == 0) return DSA_OK;
+    if (!scores_out || ld_scores < T) return DSA_ERR_INVALID_ARG;
+    return cuda_status(run_index(q_idx, q_scale, k_idx, k_scale, w, T, H_I, d_I, q_row_begin,
+                                 q_row_count, scores_out, ld_scores, true, dtype,
+                                 as_stream(stream)));
+}
+
+size_t dsa_topk_workspace_size(int64_t row_count, int64_t T, int k)
+{
+    (void)row_count; (void)T; (void)k;
+    return 0;
+}
+
+dsa_status dsa_topk(const float *scores, int64_t ld_scores, int64_t row_begin,
+                    int64_t row_count, int64_t T, int k, int32_t *idx_out, void *workspace,
+                    size_t ws_bytes, void *stream)
+{
+    (void)workspace; (void)ws_bytes;
+    if (!scores || !idx_out || T <= 0 || k < 1 || k > 65536) return DSA_ERR_INVALID_ARG;
+    if (row_begin < 0 || row_count < 0 || row_begin + row_count > T || ld_scores < T)
+        return DSA_ERR_INVALID_ARG;
+    if (row_count == 0) return DSA_OK;
+    return cuda_status(launch_topk_rows(scores, ld_scores, row_begin, nullptr, T, row_count, k,
+                                        idx_out, nullptr, as_stream(stream)));
+}
+
+dsa_status dsa_sparse_attn(const void *q, const void *k, const void *v, const int32_t *idx,
+                           int64_t T, int H_q, int d, int k_sel, float sm_scale, void *out,
+                           float *lse_out, dsa_dtype dtype, void *stream)
+{
+    dsa_status s = check_attn_args(q, k, v, idx, T, H_q, d, k_sel, out, dtype);
+    if (s != DSA_OK) return s;
+    if (!std::isfinite(sm_scale)) return DSA_ERR_INVALID_ARG;
+    return cuda_status(run_attn(q, k, v, idx, T, H_q, d, k_sel, sm_scale, out, lse_out, dtype,
+                                as_stream(stream)));
+}
+
+size_t dsa_prefill_workspace_size(int64_t T, int H_I, int d_I, int H_q, int d, int k_sel,
+                                  dsa_dtype dtype)
+{
+    (void)H_I; (void)d_I; (void)H_q; (void)d; (void)dtype;
+    if (T <= 0 || k_sel <= 0) return 0;
+    int64_t R = prefill_rows_default(T);
+    return kWsHeader + idx_bytes(T, k_sel) + align_up(sizeof(float) * (size_t)R * T, 256);
+}
+
+dsa_status dsa_prefill(const void *q_idx, const float *q_scale, const void *k_idx,
+                       const float *k_scale, const void *w, const void *q, const void *k,
+                       const void *v, int64_t T, int H_I, int d_I, int H_q, int d, int k_sel,
+                       float sm_scale, void *out, float *lse_out, int32_t *idx_out,
+                       dsa_dtype dtype, void *workspace, size_t ws_bytes, void *stream)
+{
+    if (dtype != DSA_E4M3 && dtype != DSA_F32) return DSA_ERR_UNSUPPORTED;
+    dsa_status s = check_index_args(q_idx, q_scale, k_idx, k_scale, w, T, H_I, d_I, dtype);
+    if (s != DSA_OK) return s;
+    // any non-null placeholder for idx: only the other attention arguments are checked here
+    s = check_attn_args(q, k, v, reinterpret_cast<const int32_t *>(q), T, H_q, d, k_sel, out, dtype);
+    if (s != DSA_OK) return s;
+    if (k_sel > 65536 || !std::isfinite(sm_scale)) return DSA_ERR_INVALID_ARG;
+    if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u)) return DSA_ERR_WORKSPACE;
+    size_t fixed = kWsHeader + (idx_out ? 0 : idx_bytes(T, k_sel));
+    if (ws_bytes < fixed + sizeof(float) * 64 * (size_t)T) return DSA_ERR_WORKSPACE;
+    int64_t R = (int64_t)((ws_bytes - fixed) / (sizeof(float) * (size_t)T)) / 64 * 64;
+    R = R < T ? R : ceil_div(T, 64) * 64;
+
+    cudaStream_t st = as_stream(stream);
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    WsHeader *hdr = reinterpret_cast<WsHeader *>(ws);
+    int32_t *idx = idx_out ? idx_out : reinterpret_cast<int32_t *>(ws + kWsHeader);
+    float *scores = reinterpret_cast<float *>(ws + fixed);
+    cudaError_t e = cudaMemsetAsync(hdr, 0, sizeof(WsHeader), st);
+    for (int64_t r0 = 0; e == cudaSuccess && r0 < T; r0 += R) {
+        int64_t n = T - r0 < R ? T - r0 : R;
+        e = run_index(q_idx, q_scale, k_idx, k_scale, w, T, H_I, d_I, r0, n, scores, T, false,
+                      dtype, st);
+        if (e == cudaSuccess)
+            e = launch_topk_rows(scores, T, r0, nullptr, T, n, k_sel, idx + r0 * (int64_t)k_sel,
+                                 hdr, st);
+    }
+    if (e == cudaSuccess)
+        e = run_attn(q, k, v, idx, T, H_q, d, k_sel, sm_scale, out, lse_out, dtype, st);
+    return cuda_status(e);
+}
+
+size_t dsa_decode_workspace_size(int B, int64_t max_context, int H_q, int d, int k_sel)
+{
+    if (B <= 0 || max_context <= 0 || k_sel <= 0) return 0;
+    int splits = sparse_attn_paged_splits(B, k_sel);
+    return kWsHeader + align_up(sizeof(float) * (size_t)B * max_context, 256) + idx_bytes(B, k_sel) +
+           align_up(sparse_attn_paged_part_bytes(B, H_q, d, splits), 256);
+}
+
+dsa_status dsa_decode(const void *q_idx, const float *q_scale, const void *w, const void *q,
+                      const void *kidx_cache, const float *kscale_cache, const void *k_cache,
+                      const void *v_cache, const int32_t *block_table,
+                      const int32_t *context_lens, int64_t num_pages, int max_pages_per_seq,
+                      int page_size, int B, int64_t max_context, int H_I, int d_I, int H_q,
+                      int d, int k_sel, float sm_scale, void *out, float *lse_out,
+                      int32_t *idx_out, void *workspace, size_t ws_bytes, void *stream)
+{
+    if (!q_idx || !q_scale || !w || !q || !kidx_cache || !kscale_cache || !k_cache || !v_cache ||
+        !block_table || !context_lens || !out)
+        return DSA_ERR_INVALID_ARG;
+    if (B <= 0 || max_context <= 0 || num_pages <= 0 || max_pages_per_seq <= 0 || page_size <= 0 ||
+        H_I <= 0 || H_q <= 0 || k_sel <= 0 || k_sel > 65536 || !std::isfinite(sm_scale))
+        return DSA_ERR_INVALID_ARG;
+    if (!aligned16(q_idx) || !aligned16(q) || !aligned16(kidx_cache) || !aligned16(k_cache) ||
+        !aligned16(v_cache) || !aligned16(out))
+        return DSA_ERR_INVALID_ARG;
+    if (d_I != 128 || d != 128 || H_I > 64 || H_I % 8 != 0 || page_size % 16 != 0)
+        return DSA_ERR_UNSUPPORTED;
+    if (H_q > 128 && H_q % 128 != 0) return DSA_ERR_UNSUPPORTED;
+    if (B > 65535) return DSA_ERR_UNSUPPORTED;
+    if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u)) return DSA_ERR_WORKSPACE;
+    if (ws_bytes < dsa_decode_workspace_size(B, max_context, H_q, d, k_sel)) return DSA_ERR_WORKSPACE;
+
+    cudaStream_t st = as_stream(stream);
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    WsHeader *hdr = reinterpret_cast<WsHeader *>(ws);
+    size_t off = kWsHeader;
+    float *scores = reinterpret_cast<float *>(ws + off);
+    off += align_up(sizeof(float) * (size_t)B * max_context, 256);
+    int32_t *idx = reinterpret_cast<int32_t *>(ws + off);
+    off += idx_bytes(B, k_sel);
+    float *part = reinterpret_cast<float *>(ws + off);
+    if (idx_out) idx = idx_out;
+    const int splits = sparse_attn_paged_splits(B, k_sel);
+
+    cudaError_t e = cudaMemsetAsync(hdr, 0, sizeof(WsHeader), st);
+    if (e == cudaSuccess)
+        e = launch_decode_index((const uint8_t *)q_idx, q_scale, (const uint16_t *)w,
+                                (const uint8_t *)kidx_cache, kscale_cache, block_table,
+                                context_lens, num_pages, max_pages_per_seq, page_size, B,
+                                max_context, H_I, scores, max_context, hdr, st);
+    if (e == cudaSuccess)
+        e = launch_topk_rows(scores, max_context, 0, context_lens, max_context, B, k_sel, idx, hdr,
+                             st);
+    if (e == cudaSuccess) {
+        PagedKV kv{(const uint16_t *)k_cache, (const uint16_t *)v_cache, block_table, context_lens,
+                   num_pages, max_pages_per_seq, page_size};
+        e = launch_sparse_attn_paged_bf16((const uint16_t *)q, kv, idx, B, H_q, d, k_sel, sm_scale,
+                                          (uint16_t *)out, lse_out, part, splits, hdr, st);
+    }
+    return cuda_status(e);
+}
+
+dsa_status dsa_stream_status(void *workspace, void *stream)
+{
+    if (!workspace) return DSA_ERR_INVALID_ARG;
+    cudaStream_t st = as_stream(stream);
+    WsHeader h;
+    if (cudaMemcpyAsync(&h, workspace, sizeof(WsHeader), cudaMemcpyDeviceToHost, st) != cudaSuccess)
+        return DSA_ERR_CUDA;
+    if (cudaStreamSynchronize(st) != cudaSuccess) return DSA_ERR_CUDA;
+    if (cudaMemsetAsync(workspace, 0, sizeof(WsHeader), st) != cudaSuccess) return DSA_ERR_CUDA;
+    if (cudaStreamSynchronize(st) != cudaSuccess) return DSA_ERR_CUDA;
+    return (dsa_status)h.status;
+}
+
+}  // extern "C"

@@ -1,0 +1,68 @@
+// Internal launchers of the DSA library.  Each returns cudaGetLastError()
+// of its launches; shapes were validated by the C entry points.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "dsa_common.cuh"
+
+namespace dsa {
+
+// ---- indexer (index.cu, index_tc.cu) ----
+// Scores of rows [row_begin, row_begin+row_count) into out[(t-row_begin)*ld + s].
+// write_upper: also write -inf for s in (t, T).
+cudaError_t launch_index_fp8(const uint8_t *q8, const float *sq, const uint8_t *k8,
+                             const float *sk, const uint16_t *w, int64_t T, int H,
+                             int64_t row_begin, int64_t row_count, float *out, int64_t ld,
+                             bool write_upper, cudaStream_t st);
+cudaError_t launch_index_f32(const float *q, const float *k, const float *w, int64_t T, int H,
+                             int D, int64_t row_begin, int64_t row_count, float *out,
+                             int64_t ld, bool write_upper, cudaStream_t st);
+
+// ---- top-k (topk.cu) ----
+// Row r: candidates scores[r*ld + s] for s < n_r, where n_r = lens[r] if
+// lens != nullptr, else row_begin + r + 1.  Output idx[r*k ...] ascending,
+// -1 padded.  Rows with lens[r] outside [1, max_len] are skipped (set to -1)
+// and reported in hdr.
+cudaError_t launch_topk_rows(const float *scores, int64_t ld, int64_t row_begin,
+                             const int32_t *lens, int64_t max_len, int64_t row_count, int k,
+                             int32_t *idx, WsHeader *hdr, cudaStream_t st);
+
+// ---- sparse attention (sparse_attn.cu) ----
+struct PagedKV {
+    const uint16_t *k_cache;     // [num_pages, page_size, d]
+    const uint16_t *v_cache;
+    const int32_t *block_table;  // [B, max_pages]
+    const int32_t *context_lens; // [B]
+    int64_t num_pages;
+    int max_pages;
+    int page_size;
+};
+// Contiguous K/V [T, d]; one query row per idx row; bf16.
+cudaError_t launch_sparse_attn_bf16(const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                                    const int32_t *idx, int64_t rows, int64_t T, int H, int d,
+                                    int ksel, float sm_scale, uint16_t *out, float *lse,
+                                    cudaStream_t st);
+// Paged K/V, one query row per sequence, split over `splits` chunks of the
+// index list; partials in `part` (see sparse_attn.cu for the layout).
+cudaError_t launch_sparse_attn_paged_bf16(const uint16_t *q, const PagedKV &kv,
+                                          const int32_t *idx, int B, int H, int d, int ksel,
+                                          float sm_scale, uint16_t *out, float *lse,
+                                          float *part, int splits, WsHeader *hdr,
+                                          cudaStream_t st);
+size_t sparse_attn_paged_part_bytes(int B, int H, int d, int splits);
+int sparse_attn_paged_splits(int B, int ksel);
+cudaError_t launch_sparse_attn_f32(const float *q, const float *k, const float *v,
+                                   const int32_t *idx, int64_t T, int H, int d, int ksel,
+                                   float sm_scale, float *out, float *lse, cudaStream_t st);
+
+// ---- decode indexer (decode.cu) ----
+cudaError_t launch_decode_index(const uint8_t *q8, const float *sq, const uint16_t *w,
+                                const uint8_t *kidx, const float *kscale,
+                                const int32_t *block_table, const int32_t *context_lens,
+                                int64_t num_pages, int max_pages, int page_size, int B,
+                                int64_t max_context, int H, float *scores, int64_t ld,
+                                WsHeader *hdr, cudaStream_t st);
+
+}  // namespace dsa

@@ -1,0 +1,226 @@
+"""Thin Python binding of the DSA C ABI (``include/dsa.h``).
+
+Argument marshalling only: every function passes torch CUDA tensors' device
+pointers and the current CUDA stream to the entry point of the same name in
+``libdsa_b200.so``; every step of the computation runs in that library's
+kernels.  There is no fallback: if the library is missing, or a call returns
+an error status, a ``DSAError`` is raised.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+from typing import Optional
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libdsa_b200.so")
+
+DSA_F32, DSA_BF16, DSA_E4M3 = 0, 1, 2
+STATUS = {0: "DSA_OK", 1: "DSA_ERR_INVALID_ARG", 2: "DSA_ERR_UNSUPPORTED", 3: "DSA_ERR_WORKSPACE",
+          4: "DSA_ERR_CUDA", 5: "DSA_ERR_TIMEOUT"}
+
+# Every symbol include/dsa.h declares.
+EXPORTS = ("dsa_status_string", "dsa_version", "dsa_index_scores", "dsa_topk_workspace_size",
+           "dsa_topk", "dsa_sparse_attn", "dsa_prefill_workspace_size", "dsa_prefill",
+           "dsa_decode_workspace_size", "dsa_decode", "dsa_stream_status")
+
+
+class DSAError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        super().__init__(f"{fn} returned {STATUS.get(status, status)}")
+        self.status = status
+
+
+_lib = None
+
+
+def load(path: str = LIB_PATH):
+    """Load the CUDA library (raises if it was not built)."""
+    global _lib
+    if _lib is not None and path == LIB_PATH:
+        return _lib
+    if not os.path.exists(path):
+        raise RuntimeError(
+            f"DSA CUDA library not found at {path}; build it with "
+            "`python -m long_context_fp8_b200.build`")
+    lib = ctypes.CDLL(path)
+    P, I64, I32, F, SZ = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+    sig = {
+        "dsa_status_string": ([I32], ctypes.c_char_p),
+        "dsa_version": ([], I32),
+        "dsa_index_scores": ([P, P, P, P, P, I64, I32, I32, I64, I64, P, I64, I32, P], I32),
+        "dsa_topk_workspace_size": ([I64, I64, I32], SZ),
+        "dsa_topk": ([P, I64, I64, I64, I64, I32, P, P, SZ, P], I32),
+        "dsa_sparse_attn": ([P, P, P, P, I64, I32, I32, I32, F, P, P, I32, P], I32),
+        "dsa_prefill_workspace_size": ([I64, I32, I32, I32, I32, I32, I32], SZ),
+        "dsa_prefill": ([P, P, P, P, P, P, P, P, I64, I32, I32, I32, I32, I32, F, P, P, P, I32, P,
+                         SZ, P], I32),
+        "dsa_decode_workspace_size": ([I32, I64, I32, I32, I32], SZ),
+        "dsa_decode": ([P, P, P, P, P, P, P, P, P, P, I64, I32, I32, I32, I64, I32, I32, I32, I32,
+                        I32, F, P, P, P, P, SZ, P], I32),
+        "dsa_stream_status": ([P, P], I32),
+    }
+    for name, (args, res) in sig.items():
+        fn = getattr(lib, name)
+        fn.argtypes = args
+        fn.restype = res
+    if path == LIB_PATH:
+        _lib = lib
+    return lib
+
+
+def _p(t: Optional[torch.Tensor]):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("DSA entry points take CUDA tensors")
+    if not t.is_contiguous():
+        raise ValueError("DSA entry points take contiguous tensors")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _check(fn: str, st: int):
+    if st != 0:
+        raise DSAError(fn, st)
+
+
+def _idx_dtype(q_idx: torch.Tensor) -> int:
+    if q_idx.dtype == torch.uint8:
+        return DSA_E4M3
+    if q_idx.dtype == torch.float32:
+        return DSA_F32
+    raise ValueError(f"unsupported index dtype {q_idx.dtype}")
+
+
+def _val_dtype(q: torch.Tensor) -> int:
+    return {torch.bfloat16: DSA_BF16, torch.float32: DSA_F32}[q.dtype]
+
+
+def workspace(nbytes: int, device) -> torch.Tensor:
+    """Caller-owned workspace (256-byte aligned by the torch allocator)."""
+    return torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device=device)
+
+
+def dsa_version() -> int:
+    return load().dsa_version()
+
+
+def dsa_status_string(s: int) -> str:
+    return load().dsa_status_string(s).decode()
+
+
+def dsa_index_scores(q_idx, q_scale, k_idx, k_scale, w, row_begin=0, row_count=None, out=None,
+                     ld=None, stream=None):
+    """Indexer scores of query rows [row_begin, row_begin+row_count) -> f32 [rows, ld]."""
+    T, H, D = q_idx.shape
+    row_count = T - row_begin if row_count is None else row_count
+    ld = T if ld is None else ld
+    if out is None:
+        out = torch.empty((max(row_count, 0), ld), dtype=torch.float32, device=q_idx.device)
+    st = load().dsa_index_scores(_p(q_idx), _p(q_scale), _p(k_idx), _p(k_scale), _p(w), T, H, D,
+                                 row_begin, row_count, _p(out), ld, _idx_dtype(q_idx),
+                                 _stream(stream))
+    _check("dsa_index_scores", st)
+    return out
+
+
+def dsa_topk(scores, k, row_begin=0, T=None, out=None, stream=None):
+    """Top-k of score rows (row r = query position row_begin + r) -> int32 [rows, k]."""
+    rows, ld = scores.shape
+    T = ld if T is None else T
+    if out is None:
+        out = torch.empty((rows, k), dtype=torch.int32, device=scores.device)
+    lib = load()
+    wsb = lib.dsa_topk_workspace_size(rows, T, k)
+    ws = workspace(wsb, scores.device) if wsb else None
+    st = lib.dsa_topk(_p(scores), ld, row_begin, rows, T, k, _p(out), _p(ws), wsb, _stream(stream))
+    _check("dsa_topk", st)
+    return out
+
+
+def dsa_sparse_attn(q, k, v, idx, sm_scale=None, out=None, lse=None, stream=None):
+    """Attention of each query row over its selected K/V rows -> (out, lse)."""
+    T, H, D = q.shape
+    ksel = idx.shape[1]
+    sm_scale = 1.0 / math.sqrt(D) if sm_scale is None else sm_scale
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((T, H), dtype=torch.float32, device=q.device)
+    st = load().dsa_sparse_attn(_p(q), _p(k), _p(v), _p(idx), T, H, D, ksel, sm_scale, _p(out),
+                                _p(lse), _val_dtype(q), _stream(stream))
+    _check("dsa_sparse_attn", st)
+    return out, lse
+
+
+def prefill_workspace_size(T, H_I, d_I, H_q, d, k_sel, dtype=DSA_E4M3) -> int:
+    return load().dsa_prefill_workspace_size(T, H_I, d_I, H_q, d, k_sel, dtype)
+
+
+def dsa_prefill(inp: dict, k_sel: int, sm_scale=None, out=None, lse=None, idx_out=None, ws=None,
+                want_idx=True, stream=None):
+    """Fused prefill (indexer -> top-k -> sparse attention) of one sequence."""
+    q_idx, q = inp["q_idx"], inp["q"]
+    T, H_I, d_I = q_idx.shape
+    _, H_q, d = q.shape
+    dt = _idx_dtype(q_idx)
+    sm_scale = 1.0 / math.sqrt(d) if sm_scale is None else sm_scale
+    lib = load()
+    if ws is None:
+        ws = workspace(lib.dsa_prefill_workspace_size(T, H_I, d_I, H_q, d, k_sel, dt), q.device)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((T, H_q), dtype=torch.float32, device=q.device)
+    if idx_out is None and want_idx:
+        idx_out = torch.empty((T, k_sel), dtype=torch.int32, device=q.device)
+    st = lib.dsa_prefill(_p(q_idx), _p(inp["q_scale"]), _p(inp["k_idx"]), _p(inp["k_scale"]),
+                         _p(inp["w"]), _p(q), _p(inp["k"]), _p(inp["v"]), T, H_I, d_I, H_q, d,
+                         k_sel, sm_scale, _p(out), _p(lse), _p(idx_out), dt, _p(ws), ws.numel(),
+                         _stream(stream))
+    _check("dsa_prefill", st)
+    return out, lse, idx_out
+
+
+def decode_workspace_size(B, max_context, H_q, d, k_sel) -> int:
+    return load().dsa_decode_workspace_size(B, max_context, H_q, d, k_sel)
+
+
+def dsa_decode(inp: dict, k_sel: int, max_context: int, sm_scale=None, out=None, lse=None,
+               idx_out=None, ws=None, want_idx=True, stream=None):
+    """One decode step of B sequences over paged caches -> (out, lse, idx)."""
+    B, H_I, d_I = inp["q_idx"].shape
+    _, H_q, d = inp["q"].shape
+    P, ps, _ = inp["kidx_cache"].shape
+    max_pages = inp["block_table"].shape[1]
+    sm_scale = 1.0 / math.sqrt(d) if sm_scale is None else sm_scale
+    lib = load()
+    if ws is None:
+        ws = workspace(lib.dsa_decode_workspace_size(B, max_context, H_q, d, k_sel), inp["q"].device)
+    if out is None:
+        out = torch.empty_like(inp["q"])
+    if lse is None:
+        lse = torch.empty((B, H_q), dtype=torch.float32, device=inp["q"].device)
+    if idx_out is None and want_idx:
+        idx_out = torch.empty((B, k_sel), dtype=torch.int32, device=inp["q"].device)
+    st = lib.dsa_decode(_p(inp["q_idx"]), _p(inp["q_scale"]), _p(inp["w"]), _p(inp["q"]),
+                        _p(inp["kidx_cache"]), _p(inp["kscale_cache"]), _p(inp["k_cache"]),
+                        _p(inp["v_cache"]), _p(inp["block_table"]), _p(inp["context_lens"]),
+                        P, max_pages, ps, B, max_context, H_I, d_I, H_q, d, k_sel, sm_scale,
+                        _p(out), _p(lse), _p(idx_out), _p(ws), ws.numel(), _stream(stream))
+    _check("dsa_decode", st)
+    return out, lse, idx_out
+
+
+def dsa_stream_status(ws: torch.Tensor, stream=None) -> int:
+    """Synchronise the stream and return (and clear) the workspace's device status."""
+    return load().dsa_stream_status(_p(ws), _stream(stream))

@@ -102,19 +102,21 @@ static double *dequant_keys(const void *k_idx, const float *k_scale, int kdt, in
     return khat;
 }
 
-/* qhat / w for one query token t. */
+/* qhat / w of the r-th listed query row (arrays hold only the listed rows). */
 static void dequant_query(const void *q_idx, const float *q_scale, int qdt, const void *w, int wdt,
-                          int64_t t, int H, int D, double *q_row, double *w_row)
+                          int64_t r, int H, int D, double *q_row, double *w_row)
 {
-    double sc = q_scale ? (double)q_scale[t] : 1.0;
+    double sc = q_scale ? (double)q_scale[r] : 1.0;
     for (int64_t i = 0; i < (int64_t)H * D; ++i)
-        q_row[i] = load_elem(q_idx, qdt, t * H * D + i) * sc;
-    for (int h = 0; h < H; ++h) w_row[h] = load_elem(w, wdt, t * H + h);
+        q_row[i] = load_elem(q_idx, qdt, r * H * D + i) * sc;
+    for (int h = 0; h < H; ++h) w_row[h] = load_elem(w, wdt, r * H + h);
 }
 
 /*
- * Scores of the query rows rows[0..nrows) against every key 0..T-1:
- * out[r*T + s] = I[rows[r], s] for s <= rows[r], -inf for s > rows[r].
+ * Scores of the query rows at positions rows[0..nrows) against every key
+ * 0..T-1: out[r*T + s] = I[rows[r], s] for s <= rows[r], -inf for s > rows[r].
+ * q_idx [nrows,H,D], q_scale [nrows], w [nrows,H] hold the listed rows only;
+ * k_idx [T,D], k_scale [T] hold every key.
  * idx_dtype: OR_F32 (q/k fp32, no scales) or OR_E4M3 (q/k bytes + scales);
  * w_dtype: OR_F32 or OR_BF16.  Returns 0, or -1 on allocation failure.
  */
@@ -136,7 +138,7 @@ int dsa_or_index_scores(const void *q_idx, const float *q_scale, const void *k_i
 #pragma omp for schedule(dynamic, 1)
             for (int64_t r = 0; r < nrows; ++r) {
                 int64_t t = rows[r];
-                dequant_query(q_idx, q_scale, idx_dtype, w, w_dtype, t, H, D, q_row, w_row);
+                dequant_query(q_idx, q_scale, idx_dtype, w, w_dtype, r, H, D, q_row, w_row);
                 for (int64_t s = 0; s < T; ++s)
                     out[r * T + s] = (s <= t) ? index_score(q_row, khat + s * D, w_row, H, D)
                                               : -INFINITY;
@@ -238,13 +240,13 @@ static void attend_one(const void *q, int64_t q_off, const void *K, const void *
 }
 
 /*
- * Sparse attention for query rows rows[0..nrows): q [T,H,D], K/V [T,D] of
- * dtype OR_F32 or OR_BF16; idx [nrows, k] (row r = query position rows[r]),
- * entries -1 ignored.  out [nrows, H, D], lse [nrows, H] (nullable).
+ * Sparse attention of nrows query rows: q [nrows,H,D] (the listed rows only),
+ * K/V [*,D] of dtype OR_F32 or OR_BF16; idx [nrows, k] lists the K/V rows
+ * each query attends to, entries -1 ignored.  out [nrows, H, D], lse
+ * [nrows, H] (nullable).
  */
 int dsa_or_sparse_attn(const void *q, const void *K, const void *V, int dtype, const int32_t *idx,
-                       const int64_t *rows, int64_t nrows, int k, int H, int D, double sm,
-                       double *out, double *lse)
+                       int64_t nrows, int k, int H, int D, double sm, double *out, double *lse)
 {
     int err = 0;
 #pragma omp parallel
@@ -263,7 +265,7 @@ int dsa_or_sparse_attn(const void *q, const void *K, const void *V, int dtype, c
                     int32_t j = idx[r * k + i];
                     if (j >= 0) koff[n++] = (int64_t)j * D;
                 }
-                attend_one(q, rows[r] * H * D, K, V, dtype, koff, n, H, D, sm,
+                attend_one(q, r * H * D, K, V, dtype, koff, n, H, D, sm,
                            out + r * H * D, l, z);
                 if (lse) for (int h = 0; h < H; ++h) lse[r * H + h] = l[h];
             }

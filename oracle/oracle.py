@@ -14,6 +14,7 @@ import subprocess
 from typing import Optional
 
 import numpy as np
+import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "dsa_oracle.c")
@@ -51,7 +52,7 @@ def load(path: Optional[str] = None):
     lib.dsa_or_index_scores.restype = I32
     lib.dsa_or_topk.argtypes = [P, I64, P, I64, I32, P]
     lib.dsa_or_topk.restype = I32
-    lib.dsa_or_sparse_attn.argtypes = [P, P, P, I32, P, P, I64, I32, I32, I32, D, P, P]
+    lib.dsa_or_sparse_attn.argtypes = [P, P, P, I32, P, I64, I32, I32, I32, D, P, P]
     lib.dsa_or_sparse_attn.restype = I32
     lib.dsa_or_decode.argtypes = [P, P, P, P, P, P, P, P, P, P, I32, I32, I32, I32, I32,
                                   I32, I32, I32, D, P, I64, P, P, P]
@@ -78,6 +79,14 @@ def _np(x, dtype=None):
     if dtype is not None:
         a = np.ascontiguousarray(a.astype(dtype, copy=False))
     return a
+
+
+def _is_torch(x) -> bool:
+    try:
+        import torch
+        return isinstance(x, torch.Tensor)
+    except ImportError:  # pragma: no cover
+        return False
 
 
 def _ptr(a):
@@ -108,21 +117,28 @@ def bf16(bits: int) -> float:
     return load().dsa_or_bf16(bits)
 
 
-def index_scores(q_idx, q_scale, k_idx, k_scale, w, rows, lib=None) -> np.ndarray:
+def index_scores(q_idx, q_scale, k_idx, k_scale, w, rows, lib=None, compact=False) -> np.ndarray:
     """Indexer scores I[rows[r], s] for all s (-inf for s > rows[r]); fp64 [nrows, T].
 
     Follows stage 1 of the oracle header (lightning indexer, DSA section 1).
+    q_idx/q_scale/w hold every query row, or (compact=True) only the listed rows.
     """
     lib = lib or load()
+    rows = np.ascontiguousarray(np.asarray(rows, dtype=np.int64))
+    if not compact:
+        # keep only the listed query rows (the oracle reads query data per listed row)
+        sel = torch.from_numpy(rows) if _is_torch(q_idx) else rows
+        q_idx, w = q_idx[sel], w[sel]
+        q_scale = q_scale[sel] if q_scale is not None else None
     qa, ka, wa = _np(q_idx), _np(k_idx), _np(w)
-    T, H, D = qa.shape
+    T, D = ka.shape
+    H = qa.shape[1]
     dt = OR_E4M3 if qa.dtype == np.uint8 else OR_F32
     if dt == OR_F32:
         qa, ka = qa.astype(np.float32), ka.astype(np.float32)
     wdt = _val_dtype(w)
     qs = _np(q_scale, np.float32) if q_scale is not None else None
     ks = _np(k_scale, np.float32) if k_scale is not None else None
-    rows = np.ascontiguousarray(np.asarray(rows, dtype=np.int64))
     out = np.empty((rows.size, T), dtype=np.float64)
     rc = lib.dsa_or_index_scores(_ptr(qa), _ptr(qs), _ptr(ka), _ptr(ks), _ptr(wa), dt, wdt,
                                  T, H, D, _ptr(rows), rows.size, _ptr(out))
@@ -145,21 +161,28 @@ def topk(scores, rows, k, lib=None) -> np.ndarray:
     return out
 
 
-def sparse_attn(q, K, V, idx, rows, sm_scale, lib=None):
-    """Attention of query rows over their selected K/V rows (stage 3); (out, lse) fp64."""
+def sparse_attn(q, K, V, idx, rows, sm_scale, lib=None, compact=False):
+    """Attention of query rows over their selected K/V rows (stage 3); (out, lse) fp64.
+
+    idx row r holds the selection of query position rows[r]; q holds every
+    query row, or (compact=True) only the listed rows.
+    """
     lib = lib or load()
+    rows = np.ascontiguousarray(np.asarray(rows, dtype=np.int64))
+    if not compact:
+        q = q[torch.from_numpy(rows)] if _is_torch(q) else q[rows]
     dt = _val_dtype(q)
     qa, ka, va = _np(q), _np(K), _np(V)
     if dt == OR_F32:
         qa, ka, va = qa.astype(np.float32), ka.astype(np.float32), va.astype(np.float32)
-    T, H, D = qa.shape
+    n, H, D = qa.shape
     ia = _np(idx, np.int32)
-    rows = np.ascontiguousarray(np.asarray(rows, dtype=np.int64))
     k = ia.shape[1]
-    out = np.empty((rows.size, H, D), dtype=np.float64)
-    lse = np.empty((rows.size, H), dtype=np.float64)
-    rc = lib.dsa_or_sparse_attn(_ptr(qa), _ptr(ka), _ptr(va), dt, _ptr(ia), _ptr(rows),
-                                rows.size, k, H, D, float(sm_scale), _ptr(out), _ptr(lse))
+    assert ia.shape[0] == n == rows.size
+    out = np.empty((n, H, D), dtype=np.float64)
+    lse = np.empty((n, H), dtype=np.float64)
+    rc = lib.dsa_or_sparse_attn(_ptr(qa), _ptr(ka), _ptr(va), dt, _ptr(ia), n, k, H, D,
+                                float(sm_scale), _ptr(out), _ptr(lse))
     assert rc == 0
     return out, lse
 

@@ -1,0 +1,99 @@
+"""Host-only checks of the C-ABI library: it builds, loads, exports every
+symbol ``include/dsa.h`` declares, and rejects bad arguments on the host
+before touching the GPU (no compute call is made here)."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+from long_context_fp8_b200 import build as dsa_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "dsa.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    dsa_build.build()
+    from long_context_fp8_b200 import dsa
+    return dsa.load()
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    names = re.findall(r"\b(dsa_[a-z_0-9]+)\s*\(", src)
+    return sorted(set(names))
+
+
+def test_header_and_binding_agree():
+    from long_context_fp8_b200 import dsa
+    assert sorted(dsa.EXPORTS) == declared_functions()
+
+
+def test_library_exports_every_declared_symbol(lib):
+    out = subprocess.run(["nm", "-D", "--defined-only", dsa_build.LIB], capture_output=True,
+                         text=True, check=True).stdout
+    exported = set(re.findall(r"\sT\s(dsa_\w+)", out))
+    for name in declared_functions():
+        assert name in exported, name
+        assert hasattr(lib, name)
+
+
+def test_version_and_status_strings(lib):
+    assert lib.dsa_version() == (0 << 16) | 1
+    assert lib.dsa_status_string(0) == b"DSA_OK"
+    assert lib.dsa_status_string(5) == b"DSA_ERR_TIMEOUT"
+    assert lib.dsa_status_string(99) == b"DSA_ERR_UNKNOWN"
+
+
+def test_workspace_sizes(lib):
+    assert lib.dsa_topk_workspace_size(10, 100, 8) == 0
+    T, k = 131072, 2048
+    ws = lib.dsa_prefill_workspace_size(T, 64, 128, 128, 128, k, 2)
+    assert ws >= 256 + T * k * 4 + 64 * T * 4
+    assert ws % 256 == 0
+    assert lib.dsa_prefill_workspace_size(0, 64, 128, 128, 128, k, 2) == 0
+    wd = lib.dsa_decode_workspace_size(64, 65536, 128, 128, 2048)
+    assert wd >= 256 + 64 * 65536 * 4 + 64 * 2048 * 4
+
+
+def test_host_argument_errors(lib):
+    P = ctypes.c_void_p
+    fake = P(0x1000)            # never dereferenced: every call below fails validation first
+    INVALID, UNSUP, WS = 1, 2, 3
+    # null pointers
+    assert lib.dsa_index_scores(None, None, None, None, None, 10, 4, 64, 0, 1, fake, 10, 0, None) == INVALID
+    # fp32 indexer must not get scales
+    assert lib.dsa_index_scores(fake, fake, fake, fake, fake, 10, 4, 64, 0, 1, fake, 10, 0, None) == INVALID
+    # unsupported fp8 head dim
+    assert lib.dsa_index_scores(fake, fake, fake, fake, fake, 10, 4, 64, 0, 1, fake, 10, 2, None) == UNSUP
+    # row range out of bounds / short leading dimension
+    assert lib.dsa_index_scores(fake, None, fake, None, fake, 10, 4, 64, 5, 6, fake, 10, 0, None) == INVALID
+    assert lib.dsa_index_scores(fake, None, fake, None, fake, 10, 4, 64, 0, 6, fake, 9, 0, None) == INVALID
+    # misaligned pointer
+    assert lib.dsa_index_scores(P(0x1001), None, fake, None, fake, 10, 4, 64, 0, 1, fake, 10, 0, None) == INVALID
+    # top-k: bad k, bad rows
+    assert lib.dsa_topk(fake, 10, 0, 1, 10, 0, fake, None, 0, None) == INVALID
+    assert lib.dsa_topk(fake, 10, 0, 1, 10, 70000, fake, None, 0, None) == INVALID
+    assert lib.dsa_topk(fake, 10, 8, 3, 10, 4, fake, None, 0, None) == INVALID
+    # attention: unsupported head dim, bad k
+    assert lib.dsa_sparse_attn(fake, fake, fake, fake, 10, 4, 96, 8, 1.0, fake, None, 1, None) == UNSUP
+    assert lib.dsa_sparse_attn(fake, fake, fake, fake, 10, 4, 64, 0, 1.0, fake, None, 1, None) == INVALID
+    assert lib.dsa_sparse_attn(fake, fake, fake, fake, 10, 200, 128, 8, 1.0, fake, None, 1, None) == UNSUP
+    assert lib.dsa_sparse_attn(fake, fake, fake, fake, 10, 4, 64, 8, float("nan"), fake, None, 1, None) == INVALID
+    # prefill: missing / short / misaligned workspace
+    args = [fake, fake, fake, fake, fake, fake, fake, fake, 1000, 64, 128, 16, 128, 64, 0.1, fake,
+            None, None, 2]
+    assert lib.dsa_prefill(*args, None, 0, None) == WS
+    assert lib.dsa_prefill(*args, fake, 1024, None) == WS
+    assert lib.dsa_prefill(*args, P(0x1080), 1 << 30, None) == WS
+    # decode: unsupported page size, short workspace
+    dargs = [fake] * 10 + [100, 4, 64, 2, 256, 64, 128, 128, 128, 64, 0.1, fake, None, None]
+    assert lib.dsa_decode(*dargs, fake, 10, None) == WS
+    dargs_bad = list(dargs)
+    dargs_bad[12] = 24          # page_size not a multiple of 16
+    assert lib.dsa_decode(*dargs_bad, fake, 1 << 30, None) == UNSUP
+    assert lib.dsa_stream_status(None, None) == INVALID
