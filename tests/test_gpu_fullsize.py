@@ -94,10 +94,11 @@ def test_decode_fullsize_sampled(name, seqs):
                                     np.arange(sel.size, dtype=np.int32)[None], [0], sm_of(spec.d))
         assert_attn_close(out[b:b + 1].float().cpu().numpy(), ro, lse[b:b + 1].cpu().numpy(), rl,
                           f"{name} seq {b}")
-    # planted needles (noisy copies of the new query) are mostly selected
-    hits, total = 0, 0
+    # planted needles (noisy copies of the new query): a sanity metric, not a
+    # parity criterion -- the GPU recalls as many as the oracle's own selection
+    hits_g, hits_o = 0, 0
     for i, b in enumerate(seqs):
         pos = set(inp["needle_pos"][b].tolist())
-        total += len(pos)
-        hits += len(pos & set(idx_s[i].tolist()))
-    assert total == 0 or hits / total >= 0.9
+        hits_g += len(pos & set(idx_s[i].tolist()))
+        hits_o += len(pos & set(ref["idx"][i].tolist()))
+    assert abs(hits_g - hits_o) <= max(2, hits_o // 100), (hits_g, hits_o)

@@ -191,12 +191,17 @@ def test_prefill_end_to_end(name):
 
 
 def test_prefill_needles_recovered():
+    """Sanity metric: needle recall of the GPU selection equals the oracle's."""
     spec = fp8_spec(2000, k=64, seed=23, n_needles=40)
     inp = dsa_synth.make_prefill(spec)
     _, _, idx = dsa.dsa_prefill(to_dev(inp), spec.k)
     idx = idx.cpu().numpy()
-    hits = [p in set(idx[t].tolist()) for p, t in zip(inp["needle_pos"].tolist(), inp["needle_src"].tolist())]
-    assert np.mean(hits) >= 0.9
+    src = inp["needle_src"].numpy()
+    ref = oracle.prefill(inp, spec.k, sm_of(spec.d), src)
+    pos = inp["needle_pos"].tolist()
+    hits_g = sum(p in set(idx[t].tolist()) for p, t in zip(pos, src))
+    hits_o = sum(p in set(ref["idx"][i].tolist()) for i, p in enumerate(pos))
+    assert hits_g == hits_o and hits_o > 0, (hits_g, hits_o)
 
 
 # ------------------------------------------------------------------ decode
