@@ -1,0 +1,528 @@
+"""Benchmark of the DSA hot path on B200.
+
+Default run (1 GPU): the 128K-token prefill (indexer -> top-k -> sparse
+attention, k = 2048, 64 FP8 indexer heads, 128 query heads) timed through
+``dsa_prefill``, plus the 64 x 64K-context decode step through ``dsa_decode``
+reported in the same JSON line.  Inputs are seeded synthetic tensors already
+resident in HBM; L2 is flushed between timed steps; each step is timed with
+CUDA events on the stream the library launches on.
+
+``--impl reference`` times the fp64 CPU oracle on a bounded sample of the same
+workload instead (rank 0 only).
+
+Multi-GPU (torchrun): every rank runs its own independent sequence (weak
+scaling, no data-path collective); the step time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import dsa_synth  # noqa: E402
+
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+L2_FLUSH_BYTES = 256 << 20
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(PEAKS_FALLBACK), "fallback"
+
+
+# ----------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.dev = device_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.dev}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            time.sleep(0.25)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        rows = []
+        if self.path and os.path.exists(self.path):
+            for line in open(self.path):
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    rows.append(dict(sm=float(parts[1]), smax=float(parts[2]),
+                                     power=float(parts[3]) if parts[3] not in ("[N/A]", "") else 0.0,
+                                     hw=parts[5], hwt=parts[6], swt=parts[7], swp=parts[8]))
+                except ValueError:
+                    continue
+            os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        busy = [r for r in rows if r["power"] > 250.0] or rows
+        reasons = set()
+        for r in busy:
+            for key, name in (("hw", "hw_slowdown"), ("hwt", "hw_thermal_slowdown"),
+                              ("swt", "sw_thermal_slowdown"), ("swp", "sw_power_cap")):
+                if r[key].lower().startswith("active"):
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(r["sm"] for r in busy),
+                "sm_max_mhz": max(r["smax"] for r in rows), "reasons": sorted(reasons),
+                "samples": len(busy)}
+
+
+# ----------------------------------------------------------------------------- helpers
+
+def dist_setup():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if ws > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                             device_id=torch.device("cuda", local))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(local)
+    return ws, rank, local
+
+
+def barrier(ws):
+    if ws > 1:
+        torch.distributed.barrier()
+
+
+def max_over_ranks(x: float, ws: int) -> float:
+    if ws == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def timed_steps(fn, steps, warmup, flush):
+    """Warm-up, then `steps` calls each bracketed by CUDA events on the current
+    stream, L2 flushed before each; returns per-step milliseconds."""
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    times = []
+    stream = torch.cuda.current_stream()
+    for _ in range(steps):
+        flush.zero_()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        fn()
+        b.record(stream)
+        times.append((a, b))
+    torch.cuda.synchronize()
+    return [a.elapsed_time(b) for a, b in times]
+
+
+def count_launches(fn):
+    """Kernels of this library (namespace dsa::) launched by one call of fn,
+    from the CUPTI kernel trace of torch.profiler; returns (count, per-name)."""
+    from torch.profiler import ProfilerActivity, profile
+    torch.cuda.synchronize()
+    with profile(activities=[ProfilerActivity.CUDA]) as prof:
+        fn()
+        torch.cuda.synchronize()
+    per = {}
+    for ev in prof.key_averages():
+        if "dsa::" in ev.key and ev.count > 0:
+            name = ev.key.replace("(anonymous namespace)::", "").replace("void ", "")
+            name = name.split("(")[0].split("<")[0].replace("dsa::", "")
+            per[name] = per.get(name, 0) + int(ev.count)
+    return sum(per.values()), per
+
+
+
+
+# ----------------------------------------------------------------------------- prefill
+
+def prefill_stage_breakdown(dsa, inp, spec, ws, flush, reps=2):
+    """Per-kernel time of the prefill's stages, each stage entry point timed
+    with CUDA events on the current stream (same kernels, same row passes)."""
+    T, k = spec.L, spec.k
+    R = ws["rows_per_pass"]
+    scores = ws["scores"]
+    idx = ws["idx"]
+    stream = torch.cuda.current_stream()
+    idx_ms, topk_ms, attn_ms = 0.0, 0.0, 0.0
+    per_launch = []
+    for rep in range(reps):
+        flush.zero_()
+        for r0 in range(0, T, R):
+            n = min(R, T - r0)
+            ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+            ev[0].record(stream)
+            dsa.dsa_index_scores(inp["q_idx"], inp["q_scale"], inp["k_idx"], inp["k_scale"], inp["w"],
+                                 row_begin=r0, row_count=n, out=scores[:n * T].view(n, T), ld=T)
+            ev[1].record(stream)
+            dsa.dsa_topk(scores[:n * T].view(n, T), k, row_begin=r0, T=T, out=idx[r0:r0 + n])
+            ev[2].record(stream)
+            per_launch.append((ev, r0, n))
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        dsa.dsa_sparse_attn(inp["q"], inp["k"], inp["v"], idx, 1.0 / math.sqrt(spec.d),
+                            out=ws["out"], lse=ws["lse"])
+        b.record(stream)
+        per_launch.append(((a, b), None, None))
+    torch.cuda.synchronize()
+    idx_launch_ms, idx_launch_flop = [], []
+    for ev, r0, n in per_launch:
+        if r0 is None:
+            attn_ms += ev[0].elapsed_time(ev[1])
+        else:
+            t_i = ev[0].elapsed_time(ev[1])
+            idx_ms += t_i
+            topk_ms += ev[1].elapsed_time(ev[2])
+            idx_launch_ms.append(t_i)
+            pairs = sum_pairs(r0, n)
+            idx_launch_flop.append(2.0 * spec.H_I * spec.d_I * pairs)
+    return dict(indexer_ms=idx_ms / reps, topk_ms=topk_ms / reps, attn_ms=attn_ms / reps,
+                indexer_launch_ms=idx_launch_ms, indexer_launch_flop=idx_launch_flop)
+
+
+def sum_pairs(r0, n):
+    """Causal (t, s<=t) pairs of query rows [r0, r0+n)."""
+    return n * (r0 + 1) + n * (n - 1) / 2
+
+
+def bench_prefill(args, dsa, spec, peaks, peak_kind, ws_n, rank):
+    dev = torch.device("cuda")
+    inp = dsa_synth.make_prefill(dataclass_replace_seed(spec, rank), device=dev)
+    torch.cuda.synchronize()
+    T, k, H_q, d = spec.L, spec.k, spec.H_q, spec.d
+    sm = 1.0 / math.sqrt(d)
+    lib = dsa.load()
+    wsb = lib.dsa_prefill_workspace_size(T, spec.H_I, spec.d_I, H_q, d, k, dsa.DSA_E4M3)
+    ws = dsa.workspace(wsb, dev)
+    out = torch.empty_like(inp["q"])
+    lse = torch.empty((T, H_q), dtype=torch.float32, device=dev)
+    idx = torch.empty((T, k), dtype=torch.int32, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+
+    def step():
+        dsa.dsa_prefill(inp, k, sm, out=out, lse=lse, idx_out=idx, ws=ws)
+
+    step()
+    torch.cuda.synchronize()
+    n_launch, per_kernel = count_launches(step)
+
+    barrier(ws_n)
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        ms = timed_steps(step, args.steps, args.warmup, flush)
+    clocks = clk.summary()
+    step_ms = sum(ms) / len(ms)
+    step_ms_max = max_over_ranks(step_ms, ws_n)
+
+    # stage breakdown (same kernels as dsa_prefill's passes) for the roofline
+    rows_per_pass = rows_per_pass_of(wsb, T, k)
+    scores_buf = torch.empty(rows_per_pass * T, dtype=torch.float32, device=dev)
+    br = prefill_stage_breakdown(dsa, inp, spec,
+                                 dict(rows_per_pass=rows_per_pass, scores=scores_buf, idx=idx,
+                                      out=out, lse=lse), flush)
+    del scores_buf
+    flops = dsa_synth.prefill_flops(spec)
+    fp8_peak = peaks["bf16_tflops"] * 2.0           # nominal fp8:bf16 ratio 2 on B200
+    idx_achieved = sum(br["indexer_launch_flop"]) / (sum(br["indexer_launch_ms"]) * 1e-3) / 1e12
+    attn_tflops = flops["attn_flop"] / (br["attn_ms"] * 1e-3) / 1e12
+
+    e2e = None
+    if not args.no_e2e:
+        e2e = prefill_e2e(dsa, inp, spec, out, lse, idx, ws, flush, args, ws_n)
+
+    del inp, ws, out, lse, idx
+    torch.cuda.empty_cache()
+    return dict(step_ms=step_ms_max, ms=ms, clocks=clocks, launches=n_launch, per_kernel=per_kernel,
+                breakdown=br, flops=flops, fp8_peak=fp8_peak, idx_tflops=idx_achieved,
+                attn_tflops=attn_tflops, e2e=e2e, rows_per_pass=rows_per_pass)
+
+
+def rows_per_pass_of(wsb, T, k):
+    fixed = 256  # idx_out is passed, so only the header precedes the score buffer
+    R = ((wsb - fixed) // (4 * T)) // 64 * 64
+    return min(R, ((T + 63) // 64) * 64)
+
+
+def dataclass_replace_seed(spec, rank):
+    from dataclasses import replace
+    return replace(spec, seed=spec.seed + 1000 * rank) if rank else spec
+
+
+def prefill_e2e(dsa, inp, spec, out, lse, idx, ws, flush, args, ws_n):
+    """End to end through the public API: pinned host inputs copied in, the
+    prefill, and the output read back, all inside the timed region."""
+    keys = ("q_idx", "q_scale", "k_idx", "k_scale", "w", "q", "k", "v")
+    host = {key: torch.empty(inp[key].shape, dtype=inp[key].dtype, pin_memory=True) for key in keys}
+    for key in keys:
+        host[key].copy_(inp[key])
+    out_h = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+    h2d = sum(host[key].numel() * host[key].element_size() for key in keys)
+    d2h = out_h.numel() * out_h.element_size()
+    sm = 1.0 / math.sqrt(spec.d)
+
+    def step():
+        for key in keys:
+            inp[key].copy_(host[key], non_blocking=True)
+        dsa.dsa_prefill(inp, spec.k, sm, out=out, lse=lse, idx_out=idx, ws=ws)
+        out_h.copy_(out, non_blocking=True)
+
+    steps = max(2, min(args.steps, 3))
+    ms = timed_steps(step, steps, 1, flush)
+    step_ms = max_over_ranks(sum(ms) / len(ms), ws_n)
+    del host, out_h
+    return dict(step_ms=step_ms, h2d=h2d, d2h=d2h)
+
+
+# ----------------------------------------------------------------------------- decode
+
+def decode_hbm_bytes(spec):
+    """Algorithmic HBM bytes of one decode step (what the method must move)."""
+    B, n = spec.B, sum(spec.context_lens)
+    sel = sum(min(spec.k, c) for c in spec.context_lens)
+    return dict(index_keys=n * spec.d_I, key_scales=n * 4, kv_gather=sel * spec.d * 2 * 2,
+                q=B * spec.H_q * spec.d * 2, out=B * spec.H_q * spec.d * 2,
+                q_idx=B * spec.H_I * spec.d_I + B * 4 + B * spec.H_I * 2, idx=B * spec.k * 4)
+
+
+def bench_decode(args, dsa, spec, peaks, ws_n, rank):
+    dev = torch.device("cuda")
+    from dataclasses import replace
+    inp = dsa_synth.make_decode(replace(spec, seed=spec.seed + 1000 * rank) if rank else spec,
+                                device=dev)
+    inp.pop("needle_pos")
+    torch.cuda.synchronize()
+    maxc = max(spec.context_lens)
+    lib = dsa.load()
+    ws = dsa.workspace(lib.dsa_decode_workspace_size(spec.B, maxc, spec.H_q, spec.d, spec.k), dev)
+    out = torch.empty_like(inp["q"])
+    lse = torch.empty((spec.B, spec.H_q), dtype=torch.float32, device=dev)
+    idx = torch.empty((spec.B, spec.k), dtype=torch.int32, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    sm = 1.0 / math.sqrt(spec.d)
+
+    def step():
+        dsa.dsa_decode(inp, spec.k, maxc, sm, out=out, lse=lse, idx_out=idx, ws=ws)
+
+    step()
+    torch.cuda.synchronize()
+    n_launch, per_kernel = count_launches(step)
+    barrier(ws_n)
+    ms = timed_steps(step, max(args.steps, 20), args.warmup, flush)
+    step_ms = max_over_ranks(sum(ms) / len(ms), ws_n)
+    status = dsa.dsa_stream_status(ws)
+    by = decode_hbm_bytes(spec)
+    total = sum(by.values())
+    del inp, ws
+    torch.cuda.empty_cache()
+    return dict(step_ms=step_ms, launches=n_launch, per_kernel=per_kernel, bytes=total,
+                bytes_detail=by, status=status)
+
+
+# ----------------------------------------------------------------------------- CPU oracle
+
+def cpu_prefill_sample(spec, inp, budget_s):
+    """Oracle throughput (tokens/s) on uniformly spaced query rows of the workload.
+
+    ``inp`` holds the workload's tensors (on any device); only the sampled
+    query rows and the key/value tensors are brought to the host, outside the
+    timed oracle calls."""
+    from oracle import oracle
+    L = spec.L
+    sm = 1.0 / math.sqrt(spec.d)
+    keys = {k: inp[k].cpu() for k in ("k_idx", "k_scale", "k", "v")}
+
+    def run(rows):
+        rows = np.asarray(rows, dtype=np.int64)
+        rt = torch.from_numpy(rows).to(inp["q_idx"].device)
+        q_idx, q_scale, w, q = (inp[k][rt].cpu() for k in ("q_idx", "q_scale", "w", "q"))
+        t0 = time.perf_counter()
+        sc = oracle.index_scores(q_idx, q_scale, keys["k_idx"], keys["k_scale"], w, rows, compact=True)
+        sel = oracle.topk(sc, rows, spec.k)
+        del sc
+        oracle.sparse_attn(q, keys["k"], keys["v"], sel, rows, sm, compact=True)
+        return time.perf_counter() - t0
+
+    probe = np.linspace(L // 4, 3 * L // 4, 8).astype(np.int64)
+    t_probe = run(probe) / len(probe)       # mid rows cost the average row
+    n = int(max(4, min(512, budget_s / max(t_probe, 1e-6))))
+    rows = np.unique(np.linspace(0, L - 1, n).astype(np.int64))
+    dt = run(rows)
+    return dict(value=len(rows) / dt, seconds=dt, rows=len(rows))
+
+
+def cpu_inputs_for(spec, device="cuda"):
+    return dsa_synth.make_prefill(spec, device=device)
+
+
+def oracle_threads():
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:  # pragma: no cover
+        return os.cpu_count() or 1
+
+
+# ----------------------------------------------------------------------------- main
+
+def workload_config(spec, dspec, rows_per_pass=None):
+    cfg = {"workload": f"dsa_prefill_L{spec.L}_HI{spec.H_I}_dI{spec.d_I}_k{spec.k}_Hq{spec.H_q}_d{spec.d}",
+           "L": spec.L, "index_heads": spec.H_I, "index_head_dim": spec.d_I, "top_k": spec.k,
+           "query_heads": spec.H_q, "kv_heads": 1, "head_dim": spec.d, "index_dtype": "e4m3",
+           "value_dtype": "bf16", "batch": 1, "l2": "flushed between timed steps",
+           "decode_workload": f"dsa_decode_B{dspec.B}_ctx{dspec.context_lens[0]}_k{dspec.k}_Hq{dspec.H_q}"}
+    return cfg
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="dsa", choices=["dsa", "reference"])
+    ap.add_argument("--workload", default="p128k", choices=["p128k", "p16k"])
+    ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=15.0)
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3) if args.impl == "dsa" else args.warmup
+
+    ws_n, rank, local = dist_setup()
+    spec = dsa_synth.prefill_spec(args.workload)
+    dspec = dsa_synth.decode_spec("dec64x64k")
+    metric = "DSA prefill tokens/s @128K; decode steps/s @64K ctx x64 seqs; % of roofline"
+
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        os.environ.setdefault("OMP_NUM_THREADS", str(oracle_threads()))
+        inp_cpu = cpu_inputs_for(spec, "cuda" if torch.cuda.is_available() else "cpu")
+        per_step = max(2.0, 60.0 / max(1, args.steps + args.warmup))
+        for _ in range(args.warmup):
+            cpu_prefill_sample(spec, inp_cpu, per_step / 4)
+        vals, secs, nrows = [], 0.0, 0
+        for _ in range(args.steps):
+            r = cpu_prefill_sample(spec, inp_cpu, per_step)
+            vals.append(r["value"]); secs += r["seconds"]; nrows += r["rows"]
+        v = nrows / secs
+        line = {"metric": metric, "value": v, "unit": "tokens/s", "n_gpus": args.gpus,
+                "steps": args.steps, "warmup": args.warmup,
+                "ms_per_step": 1000.0 * spec.L / v, "higher_is_better": True, "scaling": "weak",
+                "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+                "config": workload_config(spec, dspec), "impl": "reference",
+                "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": oracle_threads(),
+                                 "kind": "oracle",
+                                 "sample": f"{nrows} uniformly spaced query rows of the {spec.L}-token "
+                                           f"prefill over {args.steps} steps (indexer, top-k and "
+                                           f"attention per row, fp64)"},
+                "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                        "d2h_bytes_per_step": 0}}
+        print(json.dumps(line), flush=True)
+        return
+
+    from long_context_fp8_b200 import dsa
+    dsa.load()
+    peaks, peak_kind = load_peaks()
+
+    pre = bench_prefill(args, dsa, spec, peaks, peak_kind, ws_n, rank)
+    dec = None if args.no_decode else bench_decode(args, dsa, dspec, peaks, ws_n, rank)
+
+    T = spec.L
+    value = ws_n * T / (pre["step_ms"] * 1e-3)
+    br = pre["breakdown"]
+    idx_peak = pre["fp8_peak"]
+    roofline = {"bound": "tensor", "kernel": "indexer (FP8 e4m3 x e4m3 -> fp32)",
+                "achieved": round(pre["idx_tflops"], 2), "peak": round(idx_peak, 1),
+                "unit": "TFLOP/s", "frac": round(pre["idx_tflops"] / idx_peak, 4),
+                "peak_source": f"{peak_kind} bf16 dense x 2 (fp8:bf16 nominal ratio)",
+                "traffic": None}
+    stages = {
+        "indexer_ms": round(br["indexer_ms"], 3), "topk_ms": round(br["topk_ms"], 3),
+        "attention_ms": round(br["attn_ms"], 3),
+        "attention_tflops": round(pre["attn_tflops"], 2),
+        "attention_frac_bf16": round(pre["attn_tflops"] / peaks["bf16_tflops"], 4),
+        "topk_hbm_gbs": round((pre["flops"]["pairs"] * 4 + T * spec.k * 4) / (br["topk_ms"] * 1e-3) / 1e9, 1),
+        "indexer_passes": len(br["indexer_launch_ms"]), "rows_per_pass": pre["rows_per_pass"],
+    }
+    line = {"metric": metric, "value": round(value, 1), "unit": "tokens/s", "n_gpus": ws_n,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(pre["step_ms"], 3),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "e4m3/bf16",
+            "data": "synthetic (seeded; planted needles)",
+            "config": dict(workload_config(spec, dspec), parallelism=f"replicas{ws_n}"),
+            "roofline": roofline, "stages": stages, "clocks": pre["clocks"],
+            "gpu_launches": pre["launches"] * args.steps,
+            "gpu_launches_per_step": pre["per_kernel"]}
+    if pre["e2e"]:
+        e = pre["e2e"]
+        line["e2e"] = {"value": round(ws_n * T / (e["step_ms"] * 1e-3), 1), "unit": "tokens/s",
+                       "h2d_bytes_per_step": e["h2d"], "d2h_bytes_per_step": e["d2h"],
+                       "ms_per_step": round(e["step_ms"], 3)}
+    if dec:
+        us = dec["step_ms"] * 1e3
+        gbs = dec["bytes"] / (dec["step_ms"] * 1e-3) / 1e9
+        line["decode"] = {"value": round(ws_n * 1e3 / dec["step_ms"], 1), "unit": "steps/s",
+                          "us_per_step": round(us, 2),
+                          "roofline": {"bound": "hbm", "achieved": round(gbs, 1),
+                                       "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                                       "frac": round(gbs / peaks["hbm_gbs"], 4),
+                                       "algorithmic_bytes": dec["bytes"]},
+                          "gpu_launches_per_step": dec["per_kernel"], "device_status": dec["status"]}
+    if rank == 0 and ws_n == 1 and not args.no_cpu:
+        os.environ.setdefault("OMP_NUM_THREADS", str(oracle_threads()))
+        inp_cpu = cpu_inputs_for(spec)
+        r = cpu_prefill_sample(spec, inp_cpu, args.cpu_budget)
+        line["cpu_baseline"] = {"value": round(r["value"], 3), "unit": "tokens/s",
+                                "cores": oracle_threads(), "kind": "oracle",
+                                "sample": f"{r['rows']} uniformly spaced query rows of the {T}-token "
+                                          f"prefill (indexer, top-k, attention; fp64), {r['seconds']:.1f} s"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if ws_n > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()
