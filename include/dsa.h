@@ -174,6 +174,41 @@ dsa_status dsa_decode(const void *q_idx, const float *q_scale, const void *w, co
                       int32_t *idx_out, void *workspace, size_t ws_bytes, void *stream);
 
 /*
+ * dsa_decode_noalloc -- dsa_decode without a caller workspace.  The paper has
+ * no counterpart: this entry point exists for callers that cannot allocate
+ * device memory for the library -- for example a plugin whose host process
+ * has reserved all device memory in its own pool, or code on a
+ * latency-critical path where a device allocation (which can synchronise the
+ * device) is not allowed.  It calls no cudaMalloc, cudaFree or other
+ * allocating routine.
+ *
+ * Arguments and results are those of dsa_decode, minus workspace/ws_bytes,
+ * plus status_out: nullable DEVICE pointer to one uint32_t that receives the
+ * step's device status word (a dsa_status) on `stream` after the step.
+ *
+ * The scratch is a fixed device array of DSA_DECODE_NOALLOC_SCRATCH_BYTES
+ * (64 MiB) inside the library; every GPU that loads the library holds it
+ * until the process exits.  A problem whose dsa_decode_workspace_size()
+ * exceeds that size is rejected with DSA_ERR_WORKSPACE before any launch
+ * (64 sequences x 64K context x k 2048 x 128 heads needs about 37 MiB).
+ * The first call on each device looks up the array's device address with
+ * that device current; make that first call before any stream capture.
+ * Every call on a device shares the one array and leaves its contents behind
+ * (the status word is cleared at the start of each call): calls whose GPU
+ * work overlaps -- on different streams, or from different host threads --
+ * race and must be serialised by the caller.
+ */
+#define DSA_DECODE_NOALLOC_SCRATCH_BYTES (64u << 20)
+dsa_status dsa_decode_noalloc(const void *q_idx, const float *q_scale, const void *w, const void *q,
+                              const void *kidx_cache, const float *kscale_cache,
+                              const void *k_cache, const void *v_cache,
+                              const int32_t *block_table, const int32_t *context_lens,
+                              int64_t num_pages, int max_pages_per_seq, int page_size, int B,
+                              int64_t max_context, int H_I, int d_I, int H_q, int d, int k_sel,
+                              float sm_scale, void *out, float *lse_out, int32_t *idx_out,
+                              uint32_t *status_out, void *stream);
+
+/*
  * dsa_stream_status -- waits for `stream`, then returns the device status
  * word of `workspace` (DSA_OK if no device-side error was recorded by the
  * last call that used this workspace) and resets it to DSA_OK.

@@ -25,7 +25,7 @@ STATUS = {0: "DSA_OK", 1: "DSA_ERR_INVALID_ARG", 2: "DSA_ERR_UNSUPPORTED", 3: "D
 # Every symbol include/dsa.h declares.
 EXPORTS = ("dsa_status_string", "dsa_version", "dsa_index_scores", "dsa_topk_workspace_size",
            "dsa_topk", "dsa_sparse_attn", "dsa_prefill_workspace_size", "dsa_prefill",
-           "dsa_decode_workspace_size", "dsa_decode", "dsa_stream_status")
+           "dsa_decode_workspace_size", "dsa_decode", "dsa_decode_noalloc", "dsa_stream_status")
 
 
 class DSAError(RuntimeError):
@@ -61,6 +61,8 @@ def load(path: str = LIB_PATH):
         "dsa_decode_workspace_size": ([I32, I64, I32, I32, I32], SZ),
         "dsa_decode": ([P, P, P, P, P, P, P, P, P, P, I64, I32, I32, I32, I64, I32, I32, I32, I32,
                         I32, F, P, P, P, P, SZ, P], I32),
+        "dsa_decode_noalloc": ([P, P, P, P, P, P, P, P, P, P, I64, I32, I32, I32, I64, I32, I32, I32,
+                                I32, I32, F, P, P, P, P, P], I32),
         "dsa_stream_status": ([P, P], I32),
     }
     for name, (args, res) in sig.items():
@@ -218,6 +220,29 @@ def dsa_decode(inp: dict, k_sel: int, max_context: int, sm_scale=None, out=None,
                         P, max_pages, ps, B, max_context, H_I, d_I, H_q, d, k_sel, sm_scale,
                         _p(out), _p(lse), _p(idx_out), _p(ws), ws.numel(), _stream(stream))
     _check("dsa_decode", st)
+    return out, lse, idx_out
+
+
+NOALLOC_SCRATCH_BYTES = 64 << 20
+
+
+def dsa_decode_noalloc(inp: dict, k_sel: int, max_context: int, sm_scale=None, out=None, lse=None,
+                       idx_out=None, status_out=None, stream=None):
+    """dsa_decode with the library's fixed internal scratch instead of a
+    caller workspace (for callers that cannot allocate device memory)."""
+    B, H_I, d_I = inp["q_idx"].shape
+    _, H_q, d = inp["q"].shape
+    P, ps, _ = inp["kidx_cache"].shape
+    max_pages = inp["block_table"].shape[1]
+    sm_scale = 1.0 / math.sqrt(d) if sm_scale is None else sm_scale
+    if out is None:
+        out = torch.empty_like(inp["q"])
+    st = load().dsa_decode_noalloc(_p(inp["q_idx"]), _p(inp["q_scale"]), _p(inp["w"]), _p(inp["q"]),
+                                   _p(inp["kidx_cache"]), _p(inp["kscale_cache"]), _p(inp["k_cache"]),
+                                   _p(inp["v_cache"]), _p(inp["block_table"]), _p(inp["context_lens"]),
+                                   P, max_pages, ps, B, max_context, H_I, d_I, H_q, d, k_sel, sm_scale,
+                                   _p(out), _p(lse), _p(idx_out), _p(status_out), _stream(stream))
+    _check("dsa_decode_noalloc", st)
     return out, lse, idx_out
 
 
