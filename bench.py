@@ -196,7 +196,8 @@ def prefill_stage_breakdown(dsa, inp, spec, ws, flush, reps=2):
             ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
             ev[0].record(stream)
             dsa.dsa_index_scores(inp["q_idx"], inp["q_scale"], inp["k_idx"], inp["k_scale"], inp["w"],
-                                 row_begin=r0, row_count=n, out=scores[:n * T].view(n, T), ld=T)
+                                 row_begin=r0, row_count=n, out=scores[:n * T].view(n, T), ld=T,
+                                 fill_upper=False)
             ev[1].record(stream)
             dsa.dsa_topk(scores[:n * T].view(n, T), k, row_begin=r0, T=T, out=idx[r0:r0 + n])
             ev[2].record(stream)

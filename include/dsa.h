@@ -80,16 +80,19 @@ int dsa_version(void);
  *                      w bf16 [T, H_I].  Scales finite and > 0.
  *   dtype == DSA_F32:  q_idx f32 [T, H_I, d_I]; k_idx f32 [T, d_I]; w f32
  *                      [T, H_I]; q_scale and k_scale must be NULL.
- * Writes, for r in [0, q_row_count) and s in [0, T), with t = q_row_begin + r:
- *   scores_out[r * ld_scores + s] = I[t, s] (fp32) if s <= t, else -inf.
+ * Writes, for r in [0, q_row_count) and s in [0, t], with t = q_row_begin + r:
+ *   scores_out[r * ld_scores + s] = I[t, s] (fp32);
+ * and, if fill_upper != 0, -inf for s in (t, T); with fill_upper == 0 the
+ * entries above the diagonal are left untouched (saves their bandwidth).
  * Requires 0 <= q_row_begin, q_row_begin + q_row_count <= T, ld_scores >= T.
- * Supported: E4M3 with d_I == 128 and 1 <= H_I <= 128; F32 with d_I <= 256,
- * H_I <= 64.  q_row_count == 0 is a no-op.
+ * Supported: E4M3 with d_I == 128 and 1 <= H_I <= 128 (H_I <= 64 runs on the
+ * tcgen05 tensor-core kernel); F32 with d_I <= 256, H_I <= 64.
+ * q_row_count == 0 is a no-op.
  */
 dsa_status dsa_index_scores(const void *q_idx, const float *q_scale, const void *k_idx,
                             const float *k_scale, const void *w, int64_t T, int H_I, int d_I,
                             int64_t q_row_begin, int64_t q_row_count, float *scores_out,
-                            int64_t ld_scores, dsa_dtype dtype, void *stream);
+                            int64_t ld_scores, int fill_upper, dsa_dtype dtype, void *stream);
 
 /*
  * dsa_topk -- the top-k selector (DSA section 1; the "fine-grained selector"):

@@ -80,10 +80,18 @@ cudaError_t run_index(const void *q_idx, const float *q_scale, const void *k_idx
                       int64_t row_begin, int64_t row_count, float *out, int64_t ld,
                       bool write_upper, dsa_dtype dtype, cudaStream_t st)
 {
-    if (dtype == DSA_E4M3)
+    if (dtype == DSA_E4M3) {
+        // tcgen05 tensor-core indexer where the shape allows, else mma.sync
+        if (index_tc_supported(H_I) && T < ((int64_t)1 << 31)) {
+            cudaError_t e = launch_index_tc((const uint8_t *)q_idx, q_scale, (const uint8_t *)k_idx,
+                                            k_scale, (const uint16_t *)w, T, H_I, row_begin,
+                                            row_count, out, ld, write_upper, nullptr, st);
+            if (e != cudaErrorNotSupported) return e;
+        }
         return launch_index_fp8((const uint8_t *)q_idx, q_scale, (const uint8_t *)k_idx, k_scale,
                                 (const uint16_t *)w, T, H_I, row_begin, row_count, out, ld,
                                 write_upper, st);
+    }
     return launch_index_f32((const float *)q_idx, (const float *)k_idx, (const float *)w, T, H_I,
                             d_I, row_begin, row_count, out, ld, write_upper, st);
 }
@@ -110,7 +118,7 @@ int dsa_version(void) { return (DSA_VERSION_MAJOR << 16) | DSA_VERSION_MINOR; }
 dsa_status dsa_index_scores(const void *q_idx, const float *q_scale, const void *k_idx,
                             const float *k_scale, const void *w, int64_t T, int H_I, int d_I,
                             int64_t q_row_begin, int64_t q_row_count, float *scores_out,
-                            int64_t ld_scores, dsa_dtype dtype, void *stream)
+                            int64_t ld_scores, int fill_upper, dsa_dtype dtype, void *stream)
 {
     dsa_status s = check_index_args(q_idx, q_scale, k_idx, k_scale, w, T, H_I, d_I, dtype);
     if (s != DSA_OK) return s;
@@ -118,7 +126,7 @@ dsa_status dsa_index_scores(const void *q_idx, const float *q_scale, const void 
     if (q_row_count == 0) return DSA_OK;
     if (!scores_out || ld_scores < T) return DSA_ERR_INVALID_ARG;
     return cuda_status(run_index(q_idx, q_scale, k_idx, k_scale, w, T, H_I, d_I, q_row_begin,
-                                 q_row_count, scores_out, ld_scores, true, dtype,
+                                 q_row_count, scores_out, ld_scores, fill_upper != 0, dtype,
                                  as_stream(stream)));
 }
 
@@ -244,11 +252,20 @@ dsa_status dsa_decode(const void *q_idx, const float *q_scale, const void *w, co
     const int splits = sparse_attn_paged_splits(B, k_sel);
 
     cudaError_t e = cudaMemsetAsync(hdr, 0, sizeof(WsHeader), st);
-    if (e == cudaSuccess)
-        e = launch_decode_index((const uint8_t *)q_idx, q_scale, (const uint16_t *)w,
-                                (const uint8_t *)kidx_cache, kscale_cache, block_table,
-                                context_lens, num_pages, max_pages_per_seq, page_size, B,
-                                max_context, H_I, scores, max_context, hdr, st);
+    if (e == cudaSuccess) {
+        // tensor-core (tcgen05 + TMA) indexer where the shape allows, else mma.sync
+        if (decode_index_tc_supported(H_I, page_size) &&
+            (int64_t)num_pages * page_size < ((int64_t)1 << 31))
+            e = launch_decode_index_tc((const uint8_t *)q_idx, q_scale, (const uint16_t *)w,
+                                       (const uint8_t *)kidx_cache, kscale_cache, block_table,
+                                       context_lens, num_pages, max_pages_per_seq, page_size, B,
+                                       max_context, H_I, scores, max_context, hdr, st);
+        else
+            e = launch_decode_index((const uint8_t *)q_idx, q_scale, (const uint16_t *)w,
+                                    (const uint8_t *)kidx_cache, kscale_cache, block_table,
+                                    context_lens, num_pages, max_pages_per_seq, page_size, B,
+                                    max_context, H_I, scores, max_context, hdr, st);
+    }
     if (e == cudaSuccess)
         e = launch_topk_rows(scores, max_context, 0, context_lens, max_context, B, k_sel, idx, hdr,
                              st);

@@ -1,0 +1,348 @@
+// Lightning-indexer scores on the 5th-generation tensor cores (tcgen05).
+//
+//   I[t,s] = sk[s] * sum_h c[t,h] * ReLU(q8[t,h,:] . k8[s,:]),  c[t,h] = w[t,h] * sq[t]
+// ("DeepSeek-V3.2-Exp 稀疏注意力机制(DSA)技术深度解析", section 1: few heads,
+// index_head_dim 128, FP8, ReLU; the indexer is O(n^2) but cheap per pair).
+//
+// Persistent, warp-specialised CTA (one per SM) sweeping the causal
+// (128 query rows x 256 keys) work tiles:
+//   warp 0    TMA producer: the key tile (256 x 128 B, kept for all heads,
+//             double-buffered across work tiles) and one 128 x 128 B query
+//             tile per head through a 4-stage ring (128-byte swizzle);
+//   warp 1    MMA issuer (one thread): per head, 4 x tcgen05.mma kind::f8f6f4
+//             (M = 128 query rows, N = 256 keys, K = 32) into one of two
+//             256-column fp32 accumulators in tensor memory;
+//   warps 2-9 epilogue: TMEM lane = query row; each warp reads half the
+//             columns of its lane quarter and folds c[t,h] * ReLU(acc) into
+//             128 running scores held in registers, so the per-head products
+//             never leave the SM; after the last head the key scales are
+//             applied and the causal part of the tile is stored.
+// Every mbarrier wait is bounded; a timeout records DSA_ERR_TIMEOUT, makes
+// every role stop at its next wait, and the CTA still frees its tensor memory.
+#include <algorithm>
+
+#include "kernels.h"
+#include "sm100.cuh"
+
+namespace dsa {
+namespace {
+
+using namespace sm100;
+
+constexpr int IT_BM = 128;                    // query rows per work tile (UMMA M)
+constexpr int IT_BN = 256;                    // keys per work tile (UMMA N)
+constexpr int IT_QSTAGES = 4;
+constexpr int IT_KSTAGES = 2;
+constexpr int IT_EPI_WARPS = 8;
+constexpr int IT_THREADS = 32 * (2 + IT_EPI_WARPS);
+constexpr int IT_QBYTES = IT_BM * 128;        // 16 KB
+constexpr int IT_KBYTES = IT_BN * 128;        // 32 KB
+constexpr int IT_CS_STRIDE = IT_BM + 1;       // padded row of the c table (bank spread)
+constexpr int IT_MAX_H = 64;
+
+struct IdxTcArgs {
+    const float *sq;
+    const float *sk;
+    const uint16_t *w;
+    int64_t T;
+    int H;
+    int64_t row_begin, row_count;
+    int64_t n_rb;                // 128-row blocks in [row_begin, row_begin + row_count)
+    float *out;
+    int64_t ld;
+    int vec_store;               // ld % 4 == 0 and out 16-byte aligned
+    WsHeader *hdr;
+};
+
+struct SmemLayout {
+    static constexpr size_t k_off = 0;
+    static constexpr size_t q_off = k_off + (size_t)IT_KSTAGES * IT_KBYTES;
+    static constexpr size_t c_off = q_off + (size_t)IT_QSTAGES * IT_QBYTES;
+    static constexpr size_t sk_off = c_off + sizeof(float) * IT_MAX_H * IT_CS_STRIDE;
+    static constexpr size_t bar_off = sk_off + sizeof(float) * IT_BN;
+    static constexpr int n_bars = 2 * IT_KSTAGES + 2 * IT_QSTAGES + 4;
+    static constexpr size_t slot_off = bar_off + 8 * n_bars;
+    static constexpr size_t total = slot_off + 16 + 1024;   // + alignment slack
+};
+
+// Walks the causal work tiles of the row range in (row block, key tile) order.
+struct TileWalk {
+    int64_t rb = 0, kt = 0;
+    __device__ __forceinline__ static int64_t tiles_of(const IdxTcArgs &a, int64_t rb)
+    {
+        int64_t last = min(a.row_begin + rb * IT_BM + IT_BM - 1, a.row_begin + a.row_count - 1);
+        return last / IT_BN + 1;
+    }
+    __device__ __forceinline__ bool normalise(const IdxTcArgs &a)
+    {
+        while (rb < a.n_rb) {
+            int64_t nk = tiles_of(a, rb);
+            if (kt < nk) return true;
+            kt -= nk;
+            ++rb;
+        }
+        return false;
+    }
+    __device__ __forceinline__ bool start(const IdxTcArgs &a, int64_t idx) { rb = 0; kt = idx; return normalise(a); }
+    __device__ __forceinline__ bool next(const IdxTcArgs &a, int64_t step) { kt += step; return normalise(a); }
+};
+
+// Bounded wait that also gives up as soon as another role has aborted.
+__device__ __forceinline__ bool wait_or_abort(uint64_t *bar, uint32_t parity, volatile int *abort)
+{
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = globaltimer_ns();
+    while (true) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if (*abort) return false;
+        if (globaltimer_ns() - t0 > kWaitLimitNs) {
+            *abort = 1;
+            return false;
+        }
+    }
+}
+
+__device__ __forceinline__ void epi_bar_sync() { asm volatile("bar.sync 1, %0;" :: "n"(32 * IT_EPI_WARPS) : "memory"); }
+
+__global__ void __launch_bounds__(IT_THREADS, 1)
+index_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap kmap,
+                const IdxTcArgs a)
+{
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *Ks = smem + SmemLayout::k_off;
+    uint8_t *Qs = smem + SmemLayout::q_off;
+    float *Cs = reinterpret_cast<float *>(smem + SmemLayout::c_off);
+    float *Sk = reinterpret_cast<float *>(smem + SmemLayout::sk_off);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + SmemLayout::bar_off);
+    uint64_t *kfull = bars, *kempty = bars + IT_KSTAGES;
+    uint64_t *qfull = bars + 2 * IT_KSTAGES, *qempty = qfull + IT_QSTAGES;
+    uint64_t *tfull = qempty + IT_QSTAGES, *tempty = tfull + 2;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + SmemLayout::slot_off);
+    __shared__ volatile int abort_flag;
+    // progress of the producer and the MMA issuer, for the wind-down after an abort
+    __shared__ int q_issued, k_issued, q_consumed, k_consumed, mma_heads;
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int H = a.H;
+    const int64_t row_end = a.row_begin + a.row_count;
+
+    if (warp == 0) {
+        tmem_alloc(tmem_slot, 512);
+        tmem_relinquish();
+    }
+    if (tid == 0) {
+        for (int i = 0; i < IT_KSTAGES; ++i) { mbar_init(&kfull[i], 1); mbar_init(&kempty[i], 1); }
+        for (int i = 0; i < IT_QSTAGES; ++i) { mbar_init(&qfull[i], 1); mbar_init(&qempty[i], 1); }
+        for (int i = 0; i < 2; ++i) { mbar_init(&tfull[i], 1); mbar_init(&tempty[i], IT_EPI_WARPS); }
+        abort_flag = 0;
+        q_issued = k_issued = q_consumed = k_consumed = mma_heads = 0;
+        fence_mbar_init();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 0) {
+        // ------------------------------------------------ TMA producer
+        if (lane == 0) {
+            tma_prefetch_desc(&qmap);
+            tma_prefetch_desc(&kmap);
+            TileWalk tw;
+            int lt = 0;
+            for (bool ok = tw.start(a, blockIdx.x); ok; ok = tw.next(a, gridDim.x), ++lt) {
+                const int kb = lt & 1;
+                if (!wait_or_abort(&kempty[kb], ((lt >> 1) & 1) ^ 1, &abort_flag)) break;
+                mbar_arrive_expect_tx(&kfull[kb], IT_KBYTES);
+                tma_load_2d(Ks + kb * IT_KBYTES, &kmap, &kfull[kb], 0, (int)(tw.kt * IT_BN));
+                k_issued = lt + 1;
+                const int t0 = (int)(a.row_begin + tw.rb * IT_BM);
+                bool stop = false;
+                for (int h = 0; h < H; ++h) {
+                    const int g = lt * H + h, st = g % IT_QSTAGES;
+                    if (!wait_or_abort(&qempty[st], ((g / IT_QSTAGES) & 1) ^ 1, &abort_flag)) { stop = true; break; }
+                    mbar_arrive_expect_tx(&qfull[st], IT_QBYTES);
+                    tma_load_3d(Qs + st * IT_QBYTES, &qmap, &qfull[st], 0, h, t0);
+                    q_issued = g + 1;
+                }
+                if (stop) break;
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t idesc = umma_idesc_e4m3_f32(IT_BM, IT_BN);
+            TileWalk tw;
+            int lt = 0;
+            for (bool ok = tw.start(a, blockIdx.x); ok; ok = tw.next(a, gridDim.x), ++lt) {
+                const int kb = lt & 1;
+                if (!wait_or_abort(&kfull[kb], (lt >> 1) & 1, &abort_flag)) break;
+                k_consumed = lt + 1;
+                const uint64_t bdesc = umma_desc_k_sw128(smem_u32(Ks + kb * IT_KBYTES));
+                bool stop = false;
+                for (int h = 0; h < H; ++h) {
+                    const int g = lt * H + h, st = g % IT_QSTAGES, acc = g & 1;
+                    if (!wait_or_abort(&qfull[st], (g / IT_QSTAGES) & 1, &abort_flag)) { stop = true; break; }
+                    q_consumed = g + 1;
+                    if (!wait_or_abort(&tempty[acc], ((g >> 1) & 1) ^ 1, &abort_flag)) { stop = true; break; }
+                    tc_fence_after();
+                    const uint64_t adesc = umma_desc_k_sw128(smem_u32(Qs + st * IT_QBYTES));
+                    const uint32_t d = tmem + (uint32_t)(acc * IT_BN);
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) umma_f8f6f4(d, adesc + 2 * k, bdesc + 2 * k, idesc, k > 0);
+                    umma_commit(&qempty[st]);
+                    umma_commit(&tfull[acc]);
+                    mma_heads = g + 1;
+                }
+                if (stop) break;
+                umma_commit(&kempty[kb]);
+            }
+        }
+    } else {
+        // ------------------------------------------------ epilogue (8 warps)
+        const int et = tid - 64;                     // 0..255
+        const int quarter = warp & 3;                // TMEM lane quarter this warp may access
+        const int half = (warp - 2) >> 2;            // column half: 0 for warps 2-5, 1 for 6-9
+        const int row = quarter * 32 + lane;         // query row within the tile = TMEM lane
+        const uint32_t tlane = tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(half * 128);
+        TileWalk tw;
+        int lt = 0;
+        bool dead = false;   // after an abort: keep walking the tiles (so every epilogue warp
+                             // meets every named barrier) but do no work
+        for (bool ok = tw.start(a, blockIdx.x); ok; ok = tw.next(a, gridDim.x), ++lt) {
+            const int64_t t0 = a.row_begin + tw.rb * IT_BM;
+            const int64_t s0 = tw.kt * IT_BN;
+            epi_bar_sync();                          // the previous tile is done with Cs / Sk
+            dead = dead || abort_flag;
+            if (!dead) {
+                for (int i = et; i < IT_BM * H; i += 32 * IT_EPI_WARPS) {
+                    const int r = i / H, h = i % H;
+                    const int64_t t = t0 + r;
+                    Cs[h * IT_CS_STRIDE + r] = t < row_end ? bf16_to_f32(a.w[t * H + h]) * a.sq[t] : 0.f;
+                }
+                for (int i = et; i < IT_BN; i += 32 * IT_EPI_WARPS)
+                    Sk[i] = s0 + i < a.T ? a.sk[s0 + i] : 0.f;
+            }
+            epi_bar_sync();
+            if (dead) continue;
+
+            float score[128];
+#pragma unroll
+            for (int i = 0; i < 128; ++i) score[i] = 0.f;
+            for (int h = 0; h < H; ++h) {
+                const int g = lt * H + h, acc = g & 1;
+                if (!wait_or_abort(&tfull[acc], (g >> 1) & 1, &abort_flag)) { dead = true; break; }
+                tc_fence_after();
+                const float c = Cs[h * IT_CS_STRIDE + row];
+#pragma unroll
+                for (int c4 = 0; c4 < 4; ++c4) {
+                    uint32_t v[32];
+                    tmem_ld32(tlane + (uint32_t)(acc * IT_BN + c4 * 32), v);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int i = 0; i < 32; ++i)
+                        score[c4 * 32 + i] = fmaf(c, fmaxf(__uint_as_float(v[i]), 0.f), score[c4 * 32 + i]);
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&tempty[acc]);
+            }
+            if (dead) continue;
+            // key scales, causal mask, store
+            const int64_t t = t0 + row;
+            if (t < row_end) {
+                float *orow = a.out + (t - a.row_begin) * a.ld;
+                const int64_t sb = s0 + half * 128;
+                const float *skh = Sk + half * 128;
+#pragma unroll
+                for (int j4 = 0; j4 < 32; ++j4) {
+                    const int64_t s = sb + j4 * 4;
+                    if (a.vec_store && s + 3 <= t && s + 3 < a.T) {
+                        float4 o4 = make_float4(score[j4 * 4] * skh[j4 * 4], score[j4 * 4 + 1] * skh[j4 * 4 + 1],
+                                                score[j4 * 4 + 2] * skh[j4 * 4 + 2], score[j4 * 4 + 3] * skh[j4 * 4 + 3]);
+                        *reinterpret_cast<float4 *>(orow + s) = o4;
+                    } else {
+#pragma unroll
+                        for (int e = 0; e < 4; ++e)
+                            if (s + e <= t && s + e < a.T) orow[s + e] = score[j4 * 4 + e] * skh[j4 * 4 + e];
+                    }
+                }
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (abort_flag && tid == 0) {
+        record_error(a.hdr, DSA_ERR_TIMEOUT, blockIdx.x);
+        // let the TMA copies and MMAs still in flight land before the shared and
+        // tensor memory are released (each wait bounded)
+        for (int g = q_consumed; g < q_issued; ++g) mbar_wait(&qfull[g % IT_QSTAGES], (g / IT_QSTAGES) & 1);
+        for (int l = k_consumed; l < k_issued; ++l) mbar_wait(&kfull[l & 1], (l >> 1) & 1);
+        if (mma_heads > 0) mbar_wait(&tfull[(mma_heads - 1) & 1], ((mma_heads - 1) >> 1) & 1);
+    }
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 0) tmem_dealloc(tmem, 512);
+}
+
+// -inf above the diagonal of the stage output (s > t, s < T).
+__global__ void fill_upper_kernel(float *out, int64_t ld, int64_t T, int64_t row_begin)
+{
+    const int64_t r = blockIdx.y;
+    const int64_t t = row_begin + r;
+    for (int64_t s = t + 1 + (int64_t)blockIdx.x * blockDim.x + threadIdx.x; s < T;
+         s += (int64_t)gridDim.x * blockDim.x)
+        out[r * ld + s] = -INFINITY;
+}
+
+}  // namespace
+
+bool index_tc_supported(int H) { return H >= 1 && H <= IT_MAX_H; }
+
+cudaError_t launch_index_tc(const uint8_t *q8, const float *sq, const uint8_t *k8, const float *sk,
+                            const uint16_t *w, int64_t T, int H, int64_t row_begin,
+                            int64_t row_count, float *out, int64_t ld, bool write_upper,
+                            WsHeader *hdr, cudaStream_t st)
+{
+    if (row_count <= 0) return cudaSuccess;
+    if (!index_tc_supported(H) || T >= ((int64_t)1 << 31)) return cudaErrorNotSupported;
+    CUtensorMap qmap, kmap;
+    uint64_t qd[3] = {128, (uint64_t)H, (uint64_t)T}, qs[2] = {128, (uint64_t)H * 128};
+    uint32_t qb[3] = {128, 1, (uint32_t)IT_BM};
+    uint64_t kd[2] = {128, (uint64_t)T}, ks[1] = {128};
+    uint32_t kb[2] = {128, (uint32_t)IT_BN};
+    if (!make_tmap_u8(&qmap, q8, 3, qd, qs, qb) || !make_tmap_u8(&kmap, k8, 2, kd, ks, kb))
+        return cudaErrorNotSupported;
+    IdxTcArgs a{};
+    a.sq = sq; a.sk = sk; a.w = w; a.T = T; a.H = H; a.row_begin = row_begin; a.row_count = row_count;
+    a.n_rb = ceil_div(row_count, IT_BM);
+    a.out = out; a.ld = ld;
+    a.vec_store = (ld % 4 == 0) && ((reinterpret_cast<uintptr_t>(out) & 15u) == 0);
+    a.hdr = hdr;
+    // number of work tiles, to size the persistent grid
+    int64_t tiles = 0;
+    for (int64_t rb = 0; rb < a.n_rb; ++rb) {
+        int64_t last = std::min(row_begin + rb * IT_BM + IT_BM - 1, row_begin + row_count - 1);
+        tiles += last / IT_BN + 1;
+    }
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const unsigned grid = (unsigned)std::min<int64_t>(tiles, sms);
+    const size_t smem = SmemLayout::total;
+    cudaError_t e = cudaFuncSetAttribute(index_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem);
+    if (e != cudaSuccess) return e;
+    if (write_upper) {
+        for (int64_t r0 = 0; r0 < row_count; r0 += 65535) {
+            int64_t n = std::min<int64_t>(row_count - r0, 65535);
+            fill_upper_kernel<<<dim3(8, (unsigned)n), 256, 0, st>>>(out + r0 * ld, ld, T, row_begin + r0);
+        }
+    }
+    index_tc_kernel<<<grid, IT_THREADS, smem, st>>>(qmap, kmap, a);
+    return cudaGetLastError();
+}
+
+}  // namespace dsa

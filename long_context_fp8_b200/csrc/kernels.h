@@ -16,6 +16,11 @@ cudaError_t launch_index_fp8(const uint8_t *q8, const float *sq, const uint8_t *
                              const float *sk, const uint16_t *w, int64_t T, int H,
                              int64_t row_begin, int64_t row_count, float *out, int64_t ld,
                              bool write_upper, cudaStream_t st);
+bool index_tc_supported(int H);
+cudaError_t launch_index_tc(const uint8_t *q8, const float *sq, const uint8_t *k8, const float *sk,
+                            const uint16_t *w, int64_t T, int H, int64_t row_begin,
+                            int64_t row_count, float *out, int64_t ld, bool write_upper,
+                            WsHeader *hdr, cudaStream_t st);
 cudaError_t launch_index_f32(const float *q, const float *k, const float *w, int64_t T, int H,
                              int D, int64_t row_begin, int64_t row_count, float *out,
                              int64_t ld, bool write_upper, cudaStream_t st);
@@ -57,7 +62,14 @@ cudaError_t launch_sparse_attn_f32(const float *q, const float *k, const float *
                                    const int32_t *idx, int64_t T, int H, int d, int ksel,
                                    float sm_scale, float *out, float *lse, cudaStream_t st);
 
-// ---- decode indexer (decode.cu) ----
+// ---- decode indexer (decode_tc.cu: tcgen05 + TMA; decode.cu: mma.sync) ----
+bool decode_index_tc_supported(int H, int page_size);
+cudaError_t launch_decode_index_tc(const uint8_t *q8, const float *sq, const uint16_t *w,
+                                   const uint8_t *kidx, const float *kscale,
+                                   const int32_t *block_table, const int32_t *context_lens,
+                                   int64_t num_pages, int max_pages, int page_size, int B,
+                                   int64_t max_context, int H, float *scores, int64_t ld,
+                                   WsHeader *hdr, cudaStream_t st);
 cudaError_t launch_decode_index(const uint8_t *q8, const float *sq, const uint16_t *w,
                                 const uint8_t *kidx, const float *kscale,
                                 const int32_t *block_table, const int32_t *context_lens,

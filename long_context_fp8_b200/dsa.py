@@ -51,7 +51,7 @@ def load(path: str = LIB_PATH):
     sig = {
         "dsa_status_string": ([I32], ctypes.c_char_p),
         "dsa_version": ([], I32),
-        "dsa_index_scores": ([P, P, P, P, P, I64, I32, I32, I64, I64, P, I64, I32, P], I32),
+        "dsa_index_scores": ([P, P, P, P, P, I64, I32, I32, I64, I64, P, I64, I32, I32, P], I32),
         "dsa_topk_workspace_size": ([I64, I64, I32], SZ),
         "dsa_topk": ([P, I64, I64, I64, I64, I32, P, P, SZ, P], I32),
         "dsa_sparse_attn": ([P, P, P, P, I64, I32, I32, I32, F, P, P, I32, P], I32),
@@ -121,16 +121,17 @@ def dsa_status_string(s: int) -> str:
 
 
 def dsa_index_scores(q_idx, q_scale, k_idx, k_scale, w, row_begin=0, row_count=None, out=None,
-                     ld=None, stream=None):
-    """Indexer scores of query rows [row_begin, row_begin+row_count) -> f32 [rows, ld]."""
+                     ld=None, fill_upper=True, stream=None):
+    """Indexer scores of query rows [row_begin, row_begin+row_count) -> f32 [rows, ld]
+    (-inf above the diagonal when fill_upper, else those entries untouched)."""
     T, H, D = q_idx.shape
     row_count = T - row_begin if row_count is None else row_count
     ld = T if ld is None else ld
     if out is None:
         out = torch.empty((max(row_count, 0), ld), dtype=torch.float32, device=q_idx.device)
     st = load().dsa_index_scores(_p(q_idx), _p(q_scale), _p(k_idx), _p(k_scale), _p(w), T, H, D,
-                                 row_begin, row_count, _p(out), ld, _idx_dtype(q_idx),
-                                 _stream(stream))
+                                 row_begin, row_count, _p(out), ld, int(bool(fill_upper)),
+                                 _idx_dtype(q_idx), _stream(stream))
     _check("dsa_index_scores", st)
     return out
 

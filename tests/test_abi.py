@@ -65,16 +65,16 @@ def test_host_argument_errors(lib):
     fake = P(0x1000)            # never dereferenced: every call below fails validation first
     INVALID, UNSUP, WS = 1, 2, 3
     # null pointers
-    assert lib.dsa_index_scores(None, None, None, None, None, 10, 4, 64, 0, 1, fake, 10, 0, None) == INVALID
+    assert lib.dsa_index_scores(None, None, None, None, None, 10, 4, 64, 0, 1, fake, 10, 1, 0, None) == INVALID
     # fp32 indexer must not get scales
-    assert lib.dsa_index_scores(fake, fake, fake, fake, fake, 10, 4, 64, 0, 1, fake, 10, 0, None) == INVALID
+    assert lib.dsa_index_scores(fake, fake, fake, fake, fake, 10, 4, 64, 0, 1, fake, 10, 1, 0, None) == INVALID
     # unsupported fp8 head dim
-    assert lib.dsa_index_scores(fake, fake, fake, fake, fake, 10, 4, 64, 0, 1, fake, 10, 2, None) == UNSUP
+    assert lib.dsa_index_scores(fake, fake, fake, fake, fake, 10, 4, 64, 0, 1, fake, 10, 1, 2, None) == UNSUP
     # row range out of bounds / short leading dimension
-    assert lib.dsa_index_scores(fake, None, fake, None, fake, 10, 4, 64, 5, 6, fake, 10, 0, None) == INVALID
-    assert lib.dsa_index_scores(fake, None, fake, None, fake, 10, 4, 64, 0, 6, fake, 9, 0, None) == INVALID
+    assert lib.dsa_index_scores(fake, None, fake, None, fake, 10, 4, 64, 5, 6, fake, 10, 1, 0, None) == INVALID
+    assert lib.dsa_index_scores(fake, None, fake, None, fake, 10, 4, 64, 0, 6, fake, 9, 1, 0, None) == INVALID
     # misaligned pointer
-    assert lib.dsa_index_scores(P(0x1001), None, fake, None, fake, 10, 4, 64, 0, 1, fake, 10, 0, None) == INVALID
+    assert lib.dsa_index_scores(P(0x1001), None, fake, None, fake, 10, 4, 64, 0, 1, fake, 10, 1, 0, None) == INVALID
     # top-k: bad k, bad rows
     assert lib.dsa_topk(fake, 10, 0, 1, 10, 0, fake, None, 0, None) == INVALID
     assert lib.dsa_topk(fake, 10, 0, 1, 10, 70000, fake, None, 0, None) == INVALID

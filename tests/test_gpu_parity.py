@@ -231,7 +231,10 @@ def decode_reference_attention(inp, idx, sm):
 
 @pytest.mark.parametrize("lens,k,H_q,ps", [((1000, 64, 1, 2049, 777), 128, 16, 64),
                                            ((5000, 3000), 512, 128, 16),
-                                           ((300,) * 9, 64, 32, 32)])
+                                           ((300,) * 9, 64, 32, 32),
+                                           ((1500, 129, 640), 100, 16, 128),
+                                           ((700, 300), 64, 16, 256),
+                                           ((900, 17), 64, 16, 48)])      # 48: mma.sync indexer
 def test_decode_end_to_end(lens, k, H_q, ps):
     spec = small_decode_spec(lens, k, H_q, seed=len(lens) + k, ps=ps)
     inp = dsa_synth.make_decode(spec)
@@ -260,3 +263,19 @@ def test_decode_bad_page_reported_not_faulted():
     out, _, _ = dsa.dsa_decode(dev, 64, 500, ws=ws)
     assert dsa.dsa_stream_status(ws) == 0
     assert torch.isfinite(out.float()).all()
+
+
+def test_index_scores_fill_upper_off_leaves_upper_untouched():
+    inp = dsa_synth.make_prefill(fp8_spec(700, seed=41))
+    dev = to_dev(inp)
+    out = torch.full((300, 700), 5.0, device="cuda")
+    dsa.dsa_index_scores(dev["q_idx"], dev["q_scale"], dev["k_idx"], dev["k_scale"], dev["w"],
+                         row_begin=257, row_count=300, out=out, ld=700, fill_upper=False)
+    o = out.cpu().numpy()
+    ref = oracle.index_scores(inp["q_idx"], inp["q_scale"], inp["k_idx"], inp["k_scale"], inp["w"],
+                              np.arange(257, 557))
+    for r in range(300):
+        t = 257 + r
+        assert np.all(o[r, t + 1:] == 5.0)
+        o[r, t + 1:] = -np.inf
+    assert_scores_close(o, ref, "fill_upper=False")
