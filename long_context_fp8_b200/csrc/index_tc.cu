@@ -12,7 +12,7 @@
 //   warp 1    MMA issuer (one thread): per head, 4 x tcgen05.mma kind::f8f6f4
 //             (M = 128 query rows, N = 256 keys, K = 32) into one of two
 //             256-column fp32 accumulators in tensor memory;
-//   warps 2-9 epilogue: TMEM lane = query row; each warp reads half the
+//   warps 4-11 epilogue: TMEM lane = query row; each warp reads half the
 //             columns of its lane quarter and folds c[t,h] * ReLU(acc) into
 //             128 running scores held in registers, so the per-head products
 //             never leave the SM; after the last head the key scales are
@@ -34,7 +34,14 @@ constexpr int IT_BN = 256;                    // keys per work tile (UMMA N)
 constexpr int IT_QSTAGES = 4;
 constexpr int IT_KSTAGES = 2;
 constexpr int IT_EPI_WARPS = 8;
-constexpr int IT_THREADS = 32 * (2 + IT_EPI_WARPS);
+constexpr int IT_THREADS = 32 * (4 + IT_EPI_WARPS);   // warpgroup 0: producer, MMA, 2 idle
+// Register split (setmaxnreg): the kernel is built for 168 registers x 384
+// threads = 64512; warpgroup 0 gives up to 40 and the two epilogue warpgroups
+// take 232: 128 x 40 + 256 x 232 = 64512, the launch's own total.
+constexpr int IT_LAUNCH_REGS = 168;
+constexpr int IT_REGS_LOW = 40;
+constexpr int IT_REGS_HIGH = 232;
+static_assert(128 * IT_REGS_LOW + 256 * IT_REGS_HIGH <= IT_LAUNCH_REGS * IT_THREADS, "register split");
 constexpr int IT_QBYTES = IT_BM * 128;        // 16 KB
 constexpr int IT_KBYTES = IT_BN * 128;        // 32 KB
 constexpr int IT_CS_STRIDE = IT_BM + 1;       // padded row of the c table (bank spread)
@@ -143,67 +150,71 @@ index_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant_
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-
-    if (warp == 0) {
-        // ------------------------------------------------ TMA producer
-        if (lane == 0) {
-            tma_prefetch_desc(&qmap);
-            tma_prefetch_desc(&kmap);
-            TileWalk tw;
-            int lt = 0;
-            for (bool ok = tw.start(a, blockIdx.x); ok; ok = tw.next(a, gridDim.x), ++lt) {
-                const int kb = lt & 1;
-                if (!wait_or_abort(&kempty[kb], ((lt >> 1) & 1) ^ 1, &abort_flag)) break;
-                mbar_arrive_expect_tx(&kfull[kb], IT_KBYTES);
-                tma_load_2d(Ks + kb * IT_KBYTES, &kmap, &kfull[kb], 0, (int)(tw.kt * IT_BN));
-                k_issued = lt + 1;
-                const int t0 = (int)(a.row_begin + tw.rb * IT_BM);
-                bool stop = false;
-                for (int h = 0; h < H; ++h) {
-                    const int g = lt * H + h, st = g % IT_QSTAGES;
-                    if (!wait_or_abort(&qempty[st], ((g / IT_QSTAGES) & 1) ^ 1, &abort_flag)) { stop = true; break; }
-                    mbar_arrive_expect_tx(&qfull[st], IT_QBYTES);
-                    tma_load_3d(Qs + st * IT_QBYTES, &qmap, &qfull[st], 0, h, t0);
-                    q_issued = g + 1;
+    if (warp < 4) {
+        // warpgroup 0 (warps 0-3): producer, MMA issuer, two idle warps
+        regs_dec<IT_REGS_LOW>();
+        if (warp == 0) {
+            // ------------------------------------------------ TMA producer
+            if (lane == 0) {
+                tma_prefetch_desc(&qmap);
+                tma_prefetch_desc(&kmap);
+                TileWalk tw;
+                int lt = 0;
+                for (bool ok = tw.start(a, blockIdx.x); ok; ok = tw.next(a, gridDim.x), ++lt) {
+                    const int kb = lt & 1;
+                    if (!wait_or_abort(&kempty[kb], ((lt >> 1) & 1) ^ 1, &abort_flag)) break;
+                    mbar_arrive_expect_tx(&kfull[kb], IT_KBYTES);
+                    tma_load_2d(Ks + kb * IT_KBYTES, &kmap, &kfull[kb], 0, (int)(tw.kt * IT_BN));
+                    k_issued = lt + 1;
+                    const int t0 = (int)(a.row_begin + tw.rb * IT_BM);
+                    bool stop = false;
+                    for (int h = 0; h < H; ++h) {
+                        const int g = lt * H + h, st = g % IT_QSTAGES;
+                        if (!wait_or_abort(&qempty[st], ((g / IT_QSTAGES) & 1) ^ 1, &abort_flag)) { stop = true; break; }
+                        mbar_arrive_expect_tx(&qfull[st], IT_QBYTES);
+                        tma_load_3d(Qs + st * IT_QBYTES, &qmap, &qfull[st], 0, h, t0);
+                        q_issued = g + 1;
+                    }
+                    if (stop) break;
                 }
-                if (stop) break;
             }
-        }
-    } else if (warp == 1) {
-        // ------------------------------------------------ MMA issuer
-        if (lane == 0) {
-            constexpr uint32_t idesc = umma_idesc_e4m3_f32(IT_BM, IT_BN);
-            TileWalk tw;
-            int lt = 0;
-            for (bool ok = tw.start(a, blockIdx.x); ok; ok = tw.next(a, gridDim.x), ++lt) {
-                const int kb = lt & 1;
-                if (!wait_or_abort(&kfull[kb], (lt >> 1) & 1, &abort_flag)) break;
-                k_consumed = lt + 1;
-                const uint64_t bdesc = umma_desc_k_sw128(smem_u32(Ks + kb * IT_KBYTES));
-                bool stop = false;
-                for (int h = 0; h < H; ++h) {
-                    const int g = lt * H + h, st = g % IT_QSTAGES, acc = g & 1;
-                    if (!wait_or_abort(&qfull[st], (g / IT_QSTAGES) & 1, &abort_flag)) { stop = true; break; }
-                    q_consumed = g + 1;
-                    if (!wait_or_abort(&tempty[acc], ((g >> 1) & 1) ^ 1, &abort_flag)) { stop = true; break; }
-                    tc_fence_after();
-                    const uint64_t adesc = umma_desc_k_sw128(smem_u32(Qs + st * IT_QBYTES));
-                    const uint32_t d = tmem + (uint32_t)(acc * IT_BN);
-#pragma unroll
-                    for (int k = 0; k < 4; ++k) umma_f8f6f4(d, adesc + 2 * k, bdesc + 2 * k, idesc, k > 0);
-                    umma_commit(&qempty[st]);
-                    umma_commit(&tfull[acc]);
-                    mma_heads = g + 1;
+        } else if (warp == 1) {
+            // ------------------------------------------------ MMA issuer
+            if (lane == 0) {
+                constexpr uint32_t idesc = umma_idesc_e4m3_f32(IT_BM, IT_BN);
+                TileWalk tw;
+                int lt = 0;
+                for (bool ok = tw.start(a, blockIdx.x); ok; ok = tw.next(a, gridDim.x), ++lt) {
+                    const int kb = lt & 1;
+                    if (!wait_or_abort(&kfull[kb], (lt >> 1) & 1, &abort_flag)) break;
+                    k_consumed = lt + 1;
+                    const uint64_t bdesc = umma_desc_k_sw128(smem_u32(Ks + kb * IT_KBYTES));
+                    bool stop = false;
+                    for (int h = 0; h < H; ++h) {
+                        const int g = lt * H + h, st = g % IT_QSTAGES, acc = g & 1;
+                        if (!wait_or_abort(&qfull[st], (g / IT_QSTAGES) & 1, &abort_flag)) { stop = true; break; }
+                        q_consumed = g + 1;
+                        if (!wait_or_abort(&tempty[acc], ((g >> 1) & 1) ^ 1, &abort_flag)) { stop = true; break; }
+                        tc_fence_after();
+                        const uint64_t adesc = umma_desc_k_sw128(smem_u32(Qs + st * IT_QBYTES));
+                        const uint32_t d = tmem + (uint32_t)(acc * IT_BN);
+    #pragma unroll
+                        for (int k = 0; k < 4; ++k) umma_f8f6f4(d, adesc + 2 * k, bdesc + 2 * k, idesc, k > 0);
+                        umma_commit(&qempty[st]);
+                        umma_commit(&tfull[acc]);
+                        mma_heads = g + 1;
+                    }
+                    if (stop) break;
+                    umma_commit(&kempty[kb]);
                 }
-                if (stop) break;
-                umma_commit(&kempty[kb]);
             }
         }
     } else {
+        regs_inc<IT_REGS_HIGH>();
         // ------------------------------------------------ epilogue (8 warps)
-        const int et = tid - 64;                     // 0..255
+        const int et = tid - 128;                    // 0..255
         const int quarter = warp & 3;                // TMEM lane quarter this warp may access
-        const int half = (warp - 2) >> 2;            // column half: 0 for warps 2-5, 1 for 6-9
+        const int half = (warp - 4) >> 2;            // column half: 0 for warps 4-7, 1 for 8-11
         const int row = quarter * 32 + lane;         // query row within the tile = TMEM lane
         const uint32_t tlane = tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(half * 128);
         TileWalk tw;
@@ -227,22 +238,36 @@ index_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant_
             epi_bar_sync();
             if (dead) continue;
 
-            float score[128];
+            uint64_t sc[64];                         // running scores, column pairs (2i, 2i+1)
 #pragma unroll
-            for (int i = 0; i < 128; ++i) score[i] = 0.f;
+            for (int i = 0; i < 64; ++i) sc[i] = 0ull;
             for (int h = 0; h < H; ++h) {
                 const int g = lt * H + h, acc = g & 1;
                 if (!wait_or_abort(&tfull[acc], (g >> 1) & 1, &abort_flag)) { dead = true; break; }
                 tc_fence_after();
                 const float c = Cs[h * IT_CS_STRIDE + row];
+                const uint64_t cc = f2_pack(c, c);
+                const uint32_t base = tlane + (uint32_t)(acc * IT_BN);
+                // 8 chunks of 16 columns; the load of chunk i+1 overlaps the math of chunk i
+                uint32_t va[16], vb[16];
+                tmem_ld16(base, va);
+                tmem_wait_ld_dep16(va);
 #pragma unroll
-                for (int c4 = 0; c4 < 4; ++c4) {
-                    uint32_t v[32];
-                    tmem_ld32(tlane + (uint32_t)(acc * IT_BN + c4 * 32), v);
-                    tmem_wait_ld();
+                for (int ch = 0; ch < 8; ch += 2) {
+                    tmem_ld16(base + (uint32_t)((ch + 1) * 16), vb);
 #pragma unroll
-                    for (int i = 0; i < 32; ++i)
-                        score[c4 * 32 + i] = fmaf(c, fmaxf(__uint_as_float(v[i]), 0.f), score[c4 * 32 + i]);
+                    for (int i = 0; i < 8; ++i)
+                        sc[ch * 8 + i] = f2_fma(cc, f2_pack(fmaxf(__uint_as_float(va[2 * i]), 0.f),
+                                                            fmaxf(__uint_as_float(va[2 * i + 1]), 0.f)),
+                                                sc[ch * 8 + i]);
+                    tmem_wait_ld_dep16(vb);
+                    if (ch + 2 < 8) tmem_ld16(base + (uint32_t)((ch + 2) * 16), va);
+#pragma unroll
+                    for (int i = 0; i < 8; ++i)
+                        sc[(ch + 1) * 8 + i] = f2_fma(cc, f2_pack(fmaxf(__uint_as_float(vb[2 * i]), 0.f),
+                                                                  fmaxf(__uint_as_float(vb[2 * i + 1]), 0.f)),
+                                                      sc[(ch + 1) * 8 + i]);
+                    if (ch + 2 < 8) tmem_wait_ld_dep16(va);
                 }
                 tc_fence_before();
                 __syncwarp();
@@ -258,14 +283,17 @@ index_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant_
 #pragma unroll
                 for (int j4 = 0; j4 < 32; ++j4) {
                     const int64_t s = sb + j4 * 4;
+                    float v0, v1, v2, v3;
+                    f2_unpack(sc[2 * j4], v0, v1);
+                    f2_unpack(sc[2 * j4 + 1], v2, v3);
+                    v0 *= skh[j4 * 4]; v1 *= skh[j4 * 4 + 1]; v2 *= skh[j4 * 4 + 2]; v3 *= skh[j4 * 4 + 3];
                     if (a.vec_store && s + 3 <= t && s + 3 < a.T) {
-                        float4 o4 = make_float4(score[j4 * 4] * skh[j4 * 4], score[j4 * 4 + 1] * skh[j4 * 4 + 1],
-                                                score[j4 * 4 + 2] * skh[j4 * 4 + 2], score[j4 * 4 + 3] * skh[j4 * 4 + 3]);
-                        *reinterpret_cast<float4 *>(orow + s) = o4;
+                        *reinterpret_cast<float4 *>(orow + s) = make_float4(v0, v1, v2, v3);
                     } else {
-#pragma unroll
-                        for (int e = 0; e < 4; ++e)
-                            if (s + e <= t && s + e < a.T) orow[s + e] = score[j4 * 4 + e] * skh[j4 * 4 + e];
+                        if (s <= t && s < a.T) orow[s] = v0;
+                        if (s + 1 <= t && s + 1 < a.T) orow[s + 1] = v1;
+                        if (s + 2 <= t && s + 2 < a.T) orow[s + 2] = v2;
+                        if (s + 3 <= t && s + 3 < a.T) orow[s + 3] = v3;
                     }
                 }
             }
@@ -332,8 +360,13 @@ cudaError_t launch_index_tc(const uint8_t *q8, const float *sq, const uint8_t *k
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     const unsigned grid = (unsigned)std::min<int64_t>(tiles, sms);
     const size_t smem = SmemLayout::total;
-    cudaError_t e = cudaFuncSetAttribute(index_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)smem);
+    // the warpgroups' register split adds up to the launch's total only if the
+    // kernel was built for exactly IT_LAUNCH_REGS registers per thread
+    cudaFuncAttributes fa;
+    cudaError_t e = cudaFuncGetAttributes(&fa, index_tc_kernel);
+    if (e != cudaSuccess) return e;
+    if (fa.numRegs != IT_LAUNCH_REGS) return cudaErrorNotSupported;
+    e = cudaFuncSetAttribute(index_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     if (write_upper) {
         for (int64_t r0 = 0; r0 < row_count; r0 += 65535) {
