@@ -212,7 +212,8 @@ size_t dsa_decode_workspace_size(int B, int64_t max_context, int H_q, int d, int
     if (B <= 0 || max_context <= 0 || k_sel <= 0) return 0;
     int splits = sparse_attn_paged_splits(B, k_sel);
     return kWsHeader + align_up(sizeof(float) * (size_t)B * max_context, 256) + idx_bytes(B, k_sel) +
-           align_up(sparse_attn_paged_part_bytes(B, H_q, d, splits), 256);
+           align_up(sparse_attn_paged_part_bytes(B, H_q, d, splits), 256) +
+           align_up(topk_split_ws_bytes(B, max_context), 256);
 }
 
 dsa_status dsa_decode(const void *q_idx, const float *q_scale, const void *w, const void *q,
@@ -248,6 +249,8 @@ dsa_status dsa_decode(const void *q_idx, const float *q_scale, const void *w, co
     int32_t *idx = reinterpret_cast<int32_t *>(ws + off);
     off += idx_bytes(B, k_sel);
     float *part = reinterpret_cast<float *>(ws + off);
+    off += align_up(sparse_attn_paged_part_bytes(B, H_q, d, sparse_attn_paged_splits(B, k_sel)), 256);
+    void *topk_ws = ws + off;
     if (idx_out) idx = idx_out;
     const int splits = sparse_attn_paged_splits(B, k_sel);
 
@@ -255,7 +258,8 @@ dsa_status dsa_decode(const void *q_idx, const float *q_scale, const void *w, co
     if (e == cudaSuccess) {
         // tensor-core (tcgen05 + TMA) indexer where the shape allows, else mma.sync
         if (decode_index_tc_supported(H_I, page_size) &&
-            (int64_t)num_pages * page_size < ((int64_t)1 << 31))
+            (int64_t)num_pages * page_size < ((int64_t)1 << 31) &&
+            (reinterpret_cast<uintptr_t>(kscale_cache) & 15u) == 0)
             e = launch_decode_index_tc((const uint8_t *)q_idx, q_scale, (const uint16_t *)w,
                                        (const uint8_t *)kidx_cache, kscale_cache, block_table,
                                        context_lens, num_pages, max_pages_per_seq, page_size, B,
@@ -267,8 +271,8 @@ dsa_status dsa_decode(const void *q_idx, const float *q_scale, const void *w, co
                                     max_context, H_I, scores, max_context, hdr, st);
     }
     if (e == cudaSuccess)
-        e = launch_topk_rows(scores, max_context, 0, context_lens, max_context, B, k_sel, idx, hdr,
-                             st);
+        e = launch_topk_split(scores, max_context, context_lens, max_context, B, k_sel, idx, topk_ws,
+                              hdr, st);
     if (e == cudaSuccess) {
         PagedKV kv{(const uint16_t *)k_cache, (const uint16_t *)v_cache, block_table, context_lens,
                    num_pages, max_pages_per_seq, page_size};

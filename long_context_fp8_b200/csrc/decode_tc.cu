@@ -11,10 +11,15 @@
 // memory (tcgen05.mma kind::f8f6f4, M = 128, N = H, K = 4 x 32).  Each
 // epilogue thread owns one key (one TMEM lane), reads its H head products,
 // and folds them as sum_h c_h * ReLU(.) with c_h = w[h] * sq, then applies
-// the key's scale.  A 4-stage TMA ring keeps the HBM stream going while the
-// epilogue of the previous tile runs.  Every mbarrier wait is bounded; on a
-// timeout the CTA records DSA_ERR_TIMEOUT, drains its outstanding copies
-// (again bounded), frees its tensor memory and returns.
+// the key's scale.  Persistent and warp-specialised: one CTA per SM takes a
+// contiguous share of the (sequence, tile) items; a producer warp keeps an
+// 8-stage TMA ring of key tiles in flight, one thread issues the MMAs into
+// two alternating TMEM accumulators, and four epilogue warps drain them, so
+// the HBM stream never waits on the epilogue.  Every mbarrier wait is
+// bounded; on a timeout every role stops, the CTA records DSA_ERR_TIMEOUT,
+// waits (bounded) for its copies in flight, frees its tensor memory and returns.
+#include <algorithm>
+
 #include "kernels.h"
 #include "sm100.cuh"
 
@@ -23,11 +28,11 @@ namespace {
 
 using namespace sm100;
 
-constexpr int DT_STAGES = 4;
+constexpr int DT_STAGES = 8;
 constexpr int DT_TILE = 128;                 // keys per tile = UMMA M
 constexpr int DT_TILE_BYTES = DT_TILE * 128;
-constexpr int DT_TPC = 16;                   // tiles per CTA
-constexpr int DT_THREADS = 128;
+constexpr int DT_EPI_WARPS = 4;
+constexpr int DT_THREADS = 32 * (2 + DT_EPI_WARPS);
 constexpr int DT_TMEM_COLS = 128;            // two 64-column accumulators
 
 struct DecTcArgs {
@@ -40,6 +45,7 @@ struct DecTcArgs {
     int max_pages;
     int page_size;
     int box_rows;            // rows per TMA box: min(page_size, 128)
+    int B;
     int64_t max_context;
     float *scores;
     int64_t ld;
@@ -48,170 +54,299 @@ struct DecTcArgs {
 
 constexpr size_t dt_smem_bytes()
 {
-    return 1024 /*align slack*/ + 8192 /*q*/ + (size_t)DT_STAGES * DT_TILE_BYTES + 64 * 4 /*c*/ +
-           (DT_STAGES + 3) * 8 + 16;
+    return 1024 /*align slack*/ + 2 * 8192 /*q, double-buffered*/ + (size_t)DT_STAGES * DT_TILE_BYTES +
+           (size_t)DT_STAGES * DT_TILE * 4 /*key scales*/ + DT_STAGES * 4 /*segment masks*/ +
+           2 * 64 * 4 /*c*/ + (2 * DT_STAGES + 8) * 8 + 16;
 }
 
+// Context length of sequence b if valid, else 0 (the caller records the error).
+__device__ __forceinline__ int64_t seq_len(const DecTcArgs &a, int b)
+{
+    int64_t n = a.context_lens[b];
+    if (n < 1 || n > a.max_context || n > (int64_t)a.max_pages * a.page_size) return 0;
+    return n;
+}
+
+// Walks this CTA's contiguous share of the (sequence, 128-key tile) items.
+struct ItemWalk {
+    int b = 0;
+    int64_t tile = 0, left = 0, n = 0;
+    __device__ bool start(const DecTcArgs &a, int64_t first, int64_t count)
+    {
+        left = count;
+        b = 0;
+        tile = first;
+        while (b < a.B) {
+            n = seq_len(a, b);
+            int64_t nt = (n + DT_TILE - 1) / DT_TILE;
+            if (tile < nt) return left > 0;
+            tile -= nt;
+            ++b;
+        }
+        return false;
+    }
+    __device__ bool next(const DecTcArgs &a)
+    {
+        if (--left <= 0) return false;
+        ++tile;
+        while (b < a.B) {
+            int64_t nt = (n + DT_TILE - 1) / DT_TILE;
+            if (tile < nt) return true;
+            tile = 0;
+            if (++b < a.B) n = seq_len(a, b);
+        }
+        return false;
+    }
+};
+
+__device__ __forceinline__ bool wait_or_abort(uint64_t *bar, uint32_t parity, volatile int *abort)
+{
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = globaltimer_ns();
+    while (true) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if (*abort) return false;
+        if (globaltimer_ns() - t0 > kWaitLimitNs) {
+            *abort = 1;
+            return false;
+        }
+    }
+}
+
+__device__ __forceinline__ void epi_sync() { asm volatile("bar.sync 1, %0;" :: "n"(32 * DT_EPI_WARPS) : "memory"); }
+
 template <int H>
-__global__ void __launch_bounds__(DT_THREADS)
+__global__ void __launch_bounds__(DT_THREADS, 1)
 decode_index_tc_kernel(const __grid_constant__ CUtensorMap kmap,
                        const __grid_constant__ CUtensorMap qmap, const DecTcArgs a)
 {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint8_t *qs = smem;                                         // H x 128 B
-    uint8_t *ks = qs + 8192;                                    // stages x 128 x 128 B
-    float *cw = reinterpret_cast<float *>(ks + DT_STAGES * DT_TILE_BYTES);
-    uint64_t *full = reinterpret_cast<uint64_t *>(cw + 64);
-    uint64_t *qbar = full + DT_STAGES;
-    uint64_t *mbar = qbar + 1;                                  // [2]: one per accumulator
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(mbar + 2);
+    uint8_t *qs = smem;                                         // [2] x H x 128 B
+    uint8_t *ks = qs + 2 * 8192;                                // stages x 128 x 128 B
+    float *kss = reinterpret_cast<float *>(ks + DT_STAGES * DT_TILE_BYTES);  // [stages][128] key scales
+    uint32_t *kmask = reinterpret_cast<uint32_t *>(kss + DT_STAGES * DT_TILE); // [stages] loaded segments
+    float *cw = reinterpret_cast<float *>(kmask + DT_STAGES);                   // [2][64]
+    uint64_t *kfull = reinterpret_cast<uint64_t *>(cw + 128);
+    uint64_t *kempty = kfull + DT_STAGES;
+    uint64_t *qfull = kempty + DT_STAGES, *qempty = qfull + 2;
+    uint64_t *tfull = qempty + 2, *tempty = tfull + 2;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(tempty + 2);
+    __shared__ volatile int abort_flag;
+    __shared__ int k_issued, k_consumed, mma_items;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int b = blockIdx.y;
     const int ps = a.page_size;
-    const int64_t n = a.context_lens[b];
-    if (n < 1 || n > a.max_context || n > (int64_t)a.max_pages * ps) {
-        if (blockIdx.x == 0 && tid == 0) record_error(a.hdr, DSA_ERR_INVALID_ARG, (unsigned)b);
-        return;
+
+    // this CTA's share of the work items
+    int64_t total = 0;
+    for (int b = 0; b < a.B; ++b) {
+        int64_t n = seq_len(a, b);
+        if (n == 0 && blockIdx.x == 0 && tid == 0) record_error(a.hdr, DSA_ERR_INVALID_ARG, (unsigned)b);
+        total += (n + DT_TILE - 1) / DT_TILE;
     }
-    const int64_t tiles = (n + DT_TILE - 1) / DT_TILE;
-    const int64_t t_begin = (int64_t)blockIdx.x * DT_TPC;
-    if (t_begin >= tiles) return;
-    const int nt = (int)min((int64_t)DT_TPC, tiles - t_begin);
-    const int32_t *bt = a.block_table + (int64_t)b * a.max_pages;
+    const int64_t per = (total + gridDim.x - 1) / gridDim.x;
+    const int64_t first = (int64_t)blockIdx.x * per;
+    const int64_t count = min(per, total - first);
+    if (count <= 0) return;
 
     if (warp == 0) {
         tmem_alloc(tmem_slot, DT_TMEM_COLS);
         tmem_relinquish();
     }
     if (tid == 0) {
-        for (int s = 0; s < DT_STAGES; ++s) mbar_init(&full[s], 1);
-        mbar_init(qbar, 1);
-        mbar_init(&mbar[0], 1);
-        mbar_init(&mbar[1], 1);
+        // a stage is free once its MMA has completed and the epilogue warps have read its scales
+        for (int s = 0; s < DT_STAGES; ++s) { mbar_init(&kfull[s], 1); mbar_init(&kempty[s], 1 + DT_EPI_WARPS); }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&qfull[i], 1); mbar_init(&qempty[i], 1);
+            mbar_init(&tfull[i], 1); mbar_init(&tempty[i], DT_EPI_WARPS);
+        }
+        abort_flag = 0;
+        k_issued = k_consumed = mma_items = 0;
         fence_mbar_init();
     }
-    if (tid < H) cw[tid] = bf16_to_f32(a.w[(int64_t)b * H + tid]) * a.sq[b];
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
-    // Producer (thread 0): one tile = 128 / box_rows TMA boxes, one per page segment.
-    int issued = 0;
-    auto issue_tile = [&](int j) {
-        const int s = j % DT_STAGES;
-        const int64_t p0 = (t_begin + j) * DT_TILE;
-        const int nseg = DT_TILE / a.box_rows;
-        uint32_t bytes = 0;
-        for (int seg = 0; seg < nseg; ++seg) {
-            int64_t pos = p0 + (int64_t)seg * a.box_rows;
-            if (pos >= n) break;
-            int page = bt[pos / ps];
-            if (page >= 0 && page < a.num_pages) bytes += (uint32_t)a.box_rows * 128;
+    if (warp == 0) {
+        // ------------------------------------------------ TMA producer (whole warp)
+        // The 32 lanes resolve the page ids of 32 consecutive items at once (one
+        // memory latency per 32 tiles); lane 0 then issues their copies in order.
+        if (lane == 0) {
+            tma_prefetch_desc(&kmap);
+            tma_prefetch_desc(&qmap);
         }
-        mbar_arrive_expect_tx(&full[s], bytes);
-        for (int seg = 0; seg < nseg; ++seg) {
-            int64_t pos = p0 + (int64_t)seg * a.box_rows;
-            if (pos >= n) break;
-            int page = bt[pos / ps];
-            if (page < 0 || page >= a.num_pages) {
-                record_error(a.hdr, DSA_ERR_INVALID_ARG, (unsigned)b);
-                continue;
+        const int nseg = DT_TILE / a.box_rows;           // <= 8 page segments per tile
+        int seg = -1, prev_b = -1;
+        bool stop = false;
+        for (int64_t j0 = 0; j0 < count && !stop; j0 += 32) {
+            // this lane's item j0 + lane
+            ItemWalk mine;
+            const bool have = j0 + lane < count && mine.start(a, first + j0 + lane, count - j0 - lane);
+            int my_b = have ? mine.b : -1;
+            uint32_t my_mask = 0;
+            int my_slot[8];
+#pragma unroll
+            for (int g = 0; g < 8; ++g) my_slot[g] = 0;
+            if (have) {
+                const int32_t *bt = a.block_table + (int64_t)mine.b * a.max_pages;
+                const int64_t p0 = mine.tile * DT_TILE;
+#pragma unroll
+                for (int g = 0; g < 8; ++g) {
+                    const int64_t pos = p0 + (int64_t)g * a.box_rows;
+                    if (g < nseg && pos < mine.n) {
+                        const int page = bt[pos / ps];
+                        if (page >= 0 && page < a.num_pages) {
+                            my_mask |= 1u << g;
+                            my_slot[g] = (int)((int64_t)page * ps + pos % ps);
+                        } else {
+                            record_error(a.hdr, DSA_ERR_INVALID_ARG, (unsigned)mine.b);
+                        }
+                    }
+                }
             }
-            tma_load_2d(ks + s * DT_TILE_BYTES + seg * a.box_rows * 128, &kmap, &full[s], 0,
-                        (int)((int64_t)page * ps + pos % ps));
+            const int nb = (int)min((int64_t)32, count - j0);
+            for (int i = 0; i < nb; ++i) {
+                const int b = __shfl_sync(0xffffffffu, my_b, i);
+                const uint32_t mask = __shfl_sync(0xffffffffu, my_mask, i);
+                int slot[8];
+#pragma unroll
+                for (int g = 0; g < 8; ++g) slot[g] = __shfl_sync(0xffffffffu, my_slot[g], i);
+                if (lane == 0) {
+                    const int64_t j = j0 + i;
+                    if (b != prev_b) {                       // a new sequence: its query heads
+                        ++seg;
+                        prev_b = b;
+                        if (!wait_or_abort(&qempty[seg & 1], ((seg >> 1) & 1) ^ 1, &abort_flag)) stop = true;
+                        else {
+                            mbar_arrive_expect_tx(&qfull[seg & 1], H * 128);
+                            tma_load_2d(qs + (seg & 1) * 8192, &qmap, &qfull[seg & 1], 0, b * H);
+                        }
+                    }
+                    const int s = (int)(j % DT_STAGES);
+                    if (!stop && !wait_or_abort(&kempty[s], (uint32_t)((j / DT_STAGES) & 1) ^ 1, &abort_flag))
+                        stop = true;
+                    if (!stop) {
+                        kmask[s] = mask;                     // published by the arrive below
+                        mbar_arrive_expect_tx(&kfull[s], (uint32_t)__popc(mask) * a.box_rows * (128 + 4));
+#pragma unroll
+                        for (int g = 0; g < 8; ++g) {
+                            if ((mask >> g) & 1u) {
+                                tma_load_2d(ks + s * DT_TILE_BYTES + g * a.box_rows * 128, &kmap, &kfull[s], 0,
+                                            slot[g]);
+                                bulk_load(kss + s * DT_TILE + g * a.box_rows, a.kscale + slot[g],
+                                          (uint32_t)a.box_rows * 4, &kfull[s]);
+                            }
+                        }
+                        k_issued = (int)j + 1;
+                    }
+                }
+                stop = __shfl_sync(0xffffffffu, stop, 0);
+                if (stop) break;
+            }
         }
-        ++issued;
-    };
-    if (tid == 0) {
-        tma_prefetch_desc(&kmap);
-        tma_prefetch_desc(&qmap);
-        mbar_arrive_expect_tx(qbar, H * 128);
-        tma_load_2d(qs, &qmap, qbar, 0, b * H);
-        for (int j = 0; j < nt && j < DT_STAGES; ++j) issue_tile(j);
+    } else if (warp == 1) {
+        // ------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t idesc = umma_idesc_e4m3_f32(DT_TILE, H);
+            ItemWalk it;
+            int j = 0, seg = -1, prev_b = -1;
+            uint64_t bdesc = 0;
+            for (bool ok = it.start(a, first, count); ok; ok = it.next(a), ++j) {
+                if (it.b != prev_b) {
+                    if (seg >= 0) umma_commit(&qempty[seg & 1]);   // previous query heads are free
+                    ++seg;
+                    prev_b = it.b;
+                    if (!wait_or_abort(&qfull[seg & 1], (seg >> 1) & 1, &abort_flag)) break;
+                    bdesc = umma_desc_k_sw128(smem_u32(qs + (seg & 1) * 8192));
+                }
+                const int s = j % DT_STAGES, acc = j & 1;
+                if (!wait_or_abort(&kfull[s], (j / DT_STAGES) & 1, &abort_flag)) break;
+                k_consumed = j + 1;
+                if (!wait_or_abort(&tempty[acc], ((j >> 1) & 1) ^ 1, &abort_flag)) break;
+                tc_fence_after();
+                const uint64_t adesc = umma_desc_k_sw128(smem_u32(ks + s * DT_TILE_BYTES));
+                const uint32_t d = tmem + (uint32_t)(acc * 64);
+#pragma unroll
+                for (int k = 0; k < 4; ++k) umma_f8f6f4(d, adesc + 2 * k, bdesc + 2 * k, idesc, k > 0);
+                umma_commit(&kempty[s]);
+                umma_commit(&tfull[acc]);
+                mma_items = j + 1;
+            }
+        }
+    } else {
+        // ------------------------------------------------ epilogue (4 warps, one key per thread)
+        const int q4 = warp & 3;                       // TMEM lane quarter
+        const int et = tid - 64;
+        ItemWalk it;
+        int j = 0, seg = -1, prev_b = -1;
+        bool dead = false;
+        for (bool ok = it.start(a, first, count); ok; ok = it.next(a), ++j) {
+            if (it.b != prev_b) {                       // per-sequence head weights c_h = w[b,h] * sq[b]
+                ++seg;
+                prev_b = it.b;
+                epi_sync();
+                if (et < H) cw[(seg & 1) * 64 + et] = bf16_to_f32(a.w[(int64_t)it.b * H + et]) * a.sq[it.b];
+                epi_sync();
+            }
+            if (dead) continue;
+            // this thread's key (TMEM lane), its scale and whether its page was loaded
+            const int s = j % DT_STAGES, acc = j & 1;
+            const int r = q4 * 32 + lane;
+            const int64_t pos = it.tile * DT_TILE + r;
+            if (!wait_or_abort(&kfull[s], (j / DT_STAGES) & 1, &abort_flag)) { dead = true; continue; }
+            const bool live = pos < it.n && ((kmask[s] >> (r / a.box_rows)) & 1u);
+            const float ksc = kss[s * DT_TILE + r];
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&kempty[s]);
+            if (!wait_or_abort(&tfull[acc], (j >> 1) & 1, &abort_flag)) { dead = true; continue; }
+            tc_fence_after();
+            const uint32_t trow = tmem + ((uint32_t)(q4 * 32) << 16) + (uint32_t)(acc * 64);
+            const float *c = cw + (seg & 1) * 64;
+            uint64_t s2 = 0ull;
+            if constexpr (H % 32 == 0) {
+#pragma unroll
+                for (int c0 = 0; c0 < H; c0 += 32) {
+                    uint32_t v[32];
+                    tmem_ld32(trow + c0, v);
+                    tmem_wait_ld_dep32(v);
+#pragma unroll
+                    for (int i = 0; i < 32; i += 2)
+                        s2 = f2_fma(f2_pack(c[c0 + i], c[c0 + i + 1]),
+                                    f2_pack(fmaxf(__uint_as_float(v[i]), 0.f), fmaxf(__uint_as_float(v[i + 1]), 0.f)), s2);
+                }
+            } else {
+#pragma unroll
+                for (int c0 = 0; c0 < H; c0 += 16) {
+                    uint32_t v[16];
+                    tmem_ld16(trow + c0, v);
+                    tmem_wait_ld_dep16(v);
+#pragma unroll
+                    for (int i = 0; i < 16; i += 2)
+                        s2 = f2_fma(f2_pack(c[c0 + i], c[c0 + i + 1]),
+                                    f2_pack(fmaxf(__uint_as_float(v[i]), 0.f), fmaxf(__uint_as_float(v[i + 1]), 0.f)), s2);
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&tempty[acc]);
+            float lo, hi;
+            f2_unpack(s2, lo, hi);
+            if (live) a.scores[(int64_t)it.b * a.ld + pos] = (lo + hi) * ksc;
+        }
     }
 
-    constexpr uint32_t idesc = umma_idesc_e4m3_f32(DT_TILE, H);
-    const uint64_t bdesc = umma_desc_k_sw128(smem_u32(qs));
-    // thread 0: wait for tile j's keys, then run its MMA into accumulator j & 1
-    int consumed = 0, mma_issued = 0;
-    auto mma_tile = [&](int j) -> bool {
-        const int s = j % DT_STAGES;
-        if (!mbar_wait(&full[s], (j / DT_STAGES) & 1)) return false;
-        consumed = j + 1;
-        tc_fence_after();
-        const uint64_t adesc = umma_desc_k_sw128(smem_u32(ks + s * DT_TILE_BYTES));
-        const uint32_t d = tmem + (uint32_t)((j & 1) * 64);
-#pragma unroll
-        for (int k = 0; k < 4; ++k) umma_f8f6f4(d, adesc + 2 * k, bdesc + 2 * k, idesc, k > 0);
-        umma_commit(&mbar[j & 1]);
-        mma_issued = j + 1;
-        return true;
-    };
-    int bad = 0;
-    if (tid == 0) bad = !(mbar_wait(qbar, 0) && mma_tile(0));
-    bool failed = __syncthreads_or(bad);
-    for (int j = 0; j < nt && !failed; ++j) {
-        // this thread's key of tile j, and its scale, fetched while the MMA runs
-        const int64_t pos = (t_begin + j) * DT_TILE + warp * 32 + lane;
-        float ksc = 0.f;
-        bool live = false;
-        if (pos < n) {
-            int page = bt[pos / ps];
-            if (page >= 0 && page < a.num_pages) {
-                ksc = a.kscale[(int64_t)page * ps + pos % ps];
-                live = true;
-            }
-        }
-        bad = 0;
-        if (tid == 0 && j + 1 < nt) bad = !mma_tile(j + 1);
-        bad |= !mbar_wait(&mbar[j & 1], (j >> 1) & 1);
-        if (__syncthreads_or(bad)) { failed = true; break; }
-        tc_fence_after();
-        // tile j's MMA is done with its stage: refill it
-        if (tid == 0 && j + DT_STAGES < nt) issue_tile(j + DT_STAGES);
-
-        // epilogue: this thread's key = TMEM lane 32*warp + lane, accumulator j & 1
-        const uint32_t trow = tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)((j & 1) * 64);
-        float acc = 0.f;
-        if constexpr (H % 32 == 0) {
-#pragma unroll
-            for (int c0 = 0; c0 < H; c0 += 32) {
-                uint32_t v[32];
-                tmem_ld32(trow + c0, v);
-                tmem_wait_ld();
-#pragma unroll
-                for (int i = 0; i < 32; ++i) acc = fmaf(cw[c0 + i], fmaxf(__uint_as_float(v[i]), 0.f), acc);
-            }
-        } else {
-#pragma unroll
-            for (int c0 = 0; c0 < H; c0 += 16) {
-                uint32_t v[16];
-                tmem_ld16(trow + c0, v);
-                tmem_wait_ld();
-#pragma unroll
-                for (int i = 0; i < 16; ++i) acc = fmaf(cw[c0 + i], fmaxf(__uint_as_float(v[i]), 0.f), acc);
-            }
-        }
-        if (live) a.scores[(int64_t)b * a.ld + pos] = acc * ksc;
-        tc_fence_before();
-        __syncthreads();          // accumulator j & 1 is free for tile j + 2
+    tc_fence_before();
+    __syncthreads();
+    if (abort_flag && tid == 0) {
+        record_error(a.hdr, DSA_ERR_TIMEOUT, blockIdx.x);
+        // let copies and MMAs still in flight land before shared and tensor memory go
+        for (int j = k_consumed; j < k_issued; ++j) mbar_wait(&kfull[j % DT_STAGES], (j / DT_STAGES) & 1);
+        if (mma_items > 0) mbar_wait(&tfull[(mma_items - 1) & 1], ((mma_items - 1) >> 1) & 1);
     }
-
-    if (failed) {
-        // wind down: let copies and MMAs already in flight land before the CTA's
-        // shared and tensor memory are released (bounded again)
-        if (tid == 0) {
-            record_error(a.hdr, DSA_ERR_TIMEOUT, (unsigned)b);
-            for (int j = consumed; j < issued; ++j) mbar_wait(&full[j % DT_STAGES], (j / DT_STAGES) & 1);
-            for (int j = (mma_issued >= 2 ? mma_issued - 2 : 0); j < mma_issued; ++j)
-                mbar_wait(&mbar[j & 1], (j >> 1) & 1);
-        }
-        tc_fence_before();
-        __syncthreads();
-    }
+    __syncthreads();
     tc_fence_after();
     if (warp == 0) tmem_dealloc(tmem, DT_TMEM_COLS);
 }
@@ -246,9 +381,12 @@ cudaError_t launch_decode_index_tc(const uint8_t *q8, const float *sq, const uin
     if (!make_tmap_u8(&kmap, kidx, 2, kd, kst, kb) || !make_tmap_u8(&qmap, q8, 2, qd, qst, qb))
         return cudaErrorNotSupported;
     DecTcArgs a{sq, w, kscale, block_table, context_lens, num_pages, max_pages, page_size, box_rows,
-                max_context, scores, ld, hdr};
-    const int64_t tiles = ceil_div(max_context, DT_TILE);
-    dim3 grid((unsigned)ceil_div(tiles, DT_TPC), (unsigned)B);
+                B, max_context, scores, ld, hdr};
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int64_t max_items = (int64_t)B * ceil_div(max_context, DT_TILE);
+    dim3 grid((unsigned)std::min<int64_t>(max_items, sms));
     const size_t smem = dt_smem_bytes();
     cudaError_t e;
 #define DT_CASE(HV)                                                                              \

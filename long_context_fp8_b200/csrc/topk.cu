@@ -1,16 +1,21 @@
-// Top-k selector ("DeepSeek-V3.2-Exp DSA 技术深度解析", section 1: keep only
-// the k best-scoring KV per query token; the hotdry page's "fine-grained
-// selector").  Exact: the min(k, n) largest scores of a row, ties toward the
-// lower position, emitted in ascending position order.
+// Top-k selector ("DeepSeek-V3.2-Exp 稀疏注意力机制(DSA)技术深度解析", section 1:
+// keep only the k best-scoring KV per query token; the hotdry page's
+// "fine-grained selector").  Exact: the min(k, n) largest scores of a row, ties
+// toward the lower position, emitted in ascending position order.
 //
-// One CTA per row.  The fp32 scores are mapped to order-preserving uint32
-// keys (-0 folded onto +0) and the k-th largest key is found by a three-pass
-// radix select (11 + 11 + 10 bits) with shared-memory histograms; the pass
-// after the first only counts keys that share the digits found so far.  A
-// final pass streams the row in position order and keeps every key above the
-// threshold plus the first `need` keys equal to it; one packed block scan per
-// 4096 positions gives each kept position its output slot, so the output is
-// ascending by construction and needs no sort.
+// One CTA per row.  Scores are mapped to order-preserving uint32 keys (-0
+// folded onto +0).  Two passes over the row:
+//   1. a histogram of the top 11 key bits (16-byte loads, warp-aggregated
+//      shared-memory atomics: neighbouring scores share their top bits),
+//      which fixes the bin b1 holding the k-th largest key;
+//   2. an ordered compaction that copies every (key, position) whose top bits
+//      are >= b1 into shared memory -- the keys above b1 are selected for
+//      sure, those in b1 are the only ones left to decide.
+// The remaining 21 bits are resolved by two more histogram passes over the
+// candidates in shared memory, and a last ordered compaction over them emits
+// the selection in ascending position order (no sort needed).  If the
+// candidates do not fit in shared memory, the row falls back to the same
+// radix select run over the row in global memory.
 #include "kernels.h"
 
 namespace dsa {
@@ -18,10 +23,19 @@ namespace {
 
 constexpr int TK_THREADS = 512;
 constexpr int TK_WARPS = TK_THREADS / 32;
-constexpr int TK_ITEMS = 8;           // consecutive positions per thread in the output pass
+constexpr int TK_ITEMS = 8;                          // consecutive positions per thread per step
+constexpr int TK_STEP = TK_THREADS * TK_ITEMS;       // positions per block-wide step
+constexpr int TK_CAP = 12288;                        // shared-memory candidate capacity
 
-// Exclusive block-wide prefix sum of `v`; returns the exclusive prefix and
-// writes the block total to *total.  All threads must call it.
+struct TopkSmem {
+    uint32_t hist[2048];
+    uint32_t warp_buf[32];
+    uint32_t sh_bin, sh_above, sh_count, sh_overflow;
+    uint32_t ckey[TK_CAP];
+    int32_t cpos[TK_CAP];
+};
+
+// Exclusive block-wide prefix sum of `v`; the block total goes to *total.
 __device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t *warp_buf, uint32_t *total)
 {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -40,7 +54,7 @@ __device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t *warp_b
             uint32_t y = __shfl_up_sync(0xffffffffu, s, o);
             if (lane >= o) s += y;
         }
-        if (lane < TK_WARPS) warp_buf[lane] = s;    // inclusive warp-total prefix
+        if (lane < TK_WARPS) warp_buf[lane] = s;
     }
     __syncthreads();
     uint32_t before = (warp > 0 ? warp_buf[warp - 1] : 0u) + x - v;
@@ -49,14 +63,178 @@ __device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t *warp_b
     return before;
 }
 
+// Keys of positions [s, s + 8) of a row (bit i of *valid set when s + i < n).
+__device__ __forceinline__ void load8(const float *row, int64_t n, int64_t s, bool vec,
+                                      uint32_t (&key)[TK_ITEMS], uint32_t &valid)
+{
+    valid = 0;
+    if (vec && s + TK_ITEMS <= n) {
+        float4 a = __ldg(reinterpret_cast<const float4 *>(row + s));
+        float4 b = __ldg(reinterpret_cast<const float4 *>(row + s + 4));
+        key[0] = float_key(a.x); key[1] = float_key(a.y); key[2] = float_key(a.z); key[3] = float_key(a.w);
+        key[4] = float_key(b.x); key[5] = float_key(b.y); key[6] = float_key(b.z); key[7] = float_key(b.w);
+        valid = 0xffu;
+    } else {
+#pragma unroll
+        for (int i = 0; i < TK_ITEMS; ++i) {
+            key[i] = 0;
+            if (s + i < n) { key[i] = float_key(row[s + i]); valid |= 1u << i; }
+        }
+    }
+}
+
+// Bin holding the `remaining`-th largest count (from the top), and how many
+// counts lie strictly above it.  All threads call it; results in smem.
+__device__ __forceinline__ void find_bin(TopkSmem &sm, int nb, uint32_t remaining)
+{
+    const int tid = threadIdx.x;
+    const int bpt = nb / TK_THREADS;
+    uint32_t local = 0;
+    for (int j = 0; j < bpt; ++j) local += sm.hist[nb - 1 - (tid * bpt + j)];
+    uint32_t tot;
+    uint32_t cum = block_excl_scan(local, sm.warp_buf, &tot);
+    for (int j = 0; j < bpt; ++j) {
+        int b = nb - 1 - (tid * bpt + j);
+        uint32_t c = sm.hist[b];
+        if (cum < remaining && remaining <= cum + c) { sm.sh_bin = (uint32_t)b; sm.sh_above = cum; }
+        cum += c;
+    }
+    __syncthreads();
+}
+
+// Ordered compaction of a key sequence given by get(i) for i in [0, n):
+// emits pos(i) for keys above thr and for the first `need` keys equal to thr.
+template <class GetKey, class GetPos>
+__device__ __forceinline__ void emit_selected(TopkSmem &sm, int64_t n, uint32_t thr, uint32_t need,
+                                              int k, int32_t *out, GetKey get, GetPos pos_of)
+{
+    const int tid = threadIdx.x;
+    uint32_t base_gt = 0, base_eq = 0;
+    for (int64_t c0 = 0; c0 < n; c0 += TK_STEP) {
+        const int64_t i0 = c0 + (int64_t)tid * TK_ITEMS;
+        uint32_t flags_gt = 0, flags_eq = 0, n_gt = 0, n_eq = 0;
+        uint32_t keys[TK_ITEMS], valid;
+        get(i0, keys, valid);
+#pragma unroll
+        for (int i = 0; i < TK_ITEMS; ++i) {
+            if ((valid >> i) & 1u) {
+                if (keys[i] > thr) { flags_gt |= 1u << i; ++n_gt; }
+                else if (keys[i] == thr) { flags_eq |= 1u << i; ++n_eq; }
+            }
+        }
+        uint32_t tot;
+        uint32_t ex = block_excl_scan((n_gt << 16) | n_eq, sm.warp_buf, &tot);
+        uint32_t gt_before = base_gt + (ex >> 16), eq_before = base_eq + (ex & 0xffffu);
+#pragma unroll
+        for (int i = 0; i < TK_ITEMS; ++i) {
+            bool gt = (flags_gt >> i) & 1u, eq = (flags_eq >> i) & 1u;
+            if (gt || (eq && eq_before < need)) {
+                uint32_t p = gt_before + min(eq_before, need);
+                if (p < (uint32_t)k) out[p] = pos_of(i0 + i);
+            }
+            gt_before += gt;
+            eq_before += eq;
+        }
+        base_gt += tot >> 16;
+        base_eq += tot & 0xffffu;
+    }
+}
+
+// Given the candidates (every key whose top 11 bits are >= b1, in ascending
+// position order) in shared memory, resolve the remaining 21 bits of the
+// threshold on chip and emit the selection in position order.
+__device__ void select_on_chip(TopkSmem &sm, uint32_t ncand, uint32_t b1, uint32_t remaining, int k,
+                               int32_t *out)
+{
+    const int tid = threadIdx.x;
+    uint32_t prefix = b1 << 21, pmask = 0x7FFu << 21;
+#pragma unroll 1
+    for (int pass = 0; pass < 2; ++pass) {
+        const int shift = pass == 0 ? 10 : 0;
+        const int nb = pass == 0 ? 2048 : 1024;
+        const uint32_t bmask = (uint32_t)nb - 1u;
+        for (int i = tid; i < nb; i += TK_THREADS) sm.hist[i] = 0u;
+        __syncthreads();
+        for (uint32_t j = tid; j < ncand; j += TK_THREADS) {
+            uint32_t key = sm.ckey[j];
+            if ((key & pmask) == prefix) atomicAdd(&sm.hist[(key >> shift) & bmask], 1u);
+        }
+        __syncthreads();
+        find_bin(sm, nb, remaining);
+        remaining -= sm.sh_above;
+        prefix |= sm.sh_bin << shift;
+        pmask |= bmask << shift;
+        __syncthreads();
+    }
+    emit_selected(
+        sm, ncand, prefix, remaining, k, out,
+        [&](int64_t i0, uint32_t (&keys)[TK_ITEMS], uint32_t &valid) {
+            valid = 0;
+#pragma unroll
+            for (int i = 0; i < TK_ITEMS; ++i) {
+                keys[i] = 0;
+                if (i0 + i < (int64_t)ncand) { keys[i] = sm.ckey[i0 + i]; valid |= 1u << i; }
+            }
+        },
+        [&](int64_t i) { return sm.cpos[i]; });
+}
+
+// Radix select run over the whole row in global memory (candidates did not fit).
+__device__ void select_global(TopkSmem &sm, const float *row, int64_t n, bool vec, int k, int32_t *out)
+{
+    const int tid = threadIdx.x;
+    auto row_keys = [&](int64_t s, uint32_t (&keys)[TK_ITEMS], uint32_t &valid) {
+        load8(row, n, s, vec, keys, valid);
+    };
+    uint32_t prefix = 0, pmask = 0, remaining = (uint32_t)k;
+#pragma unroll 1
+    for (int pass = 0; pass < 3; ++pass) {
+        const int shift = pass == 0 ? 21 : (pass == 1 ? 10 : 0);
+        const int nb = pass == 2 ? 1024 : 2048;
+        const uint32_t bmask = (uint32_t)nb - 1u;
+        for (int i = tid; i < nb; i += TK_THREADS) sm.hist[i] = 0u;
+        __syncthreads();
+        for (int64_t c0 = 0; c0 < n; c0 += TK_STEP) {
+            uint32_t keys[TK_ITEMS], valid;
+            row_keys(c0 + (int64_t)tid * TK_ITEMS, keys, valid);
+#pragma unroll
+            for (int i = 0; i < TK_ITEMS; ++i)
+                if (((valid >> i) & 1u) && (keys[i] & pmask) == prefix)
+                    atomicAdd(&sm.hist[(keys[i] >> shift) & bmask], 1u);
+        }
+        __syncthreads();
+        find_bin(sm, nb, remaining);
+        remaining -= sm.sh_above;
+        prefix |= sm.sh_bin << shift;
+        pmask |= bmask << shift;
+        __syncthreads();
+    }
+    emit_selected(sm, n, prefix, remaining, k, out, row_keys, [&](int64_t i) { return (int32_t)i; });
+}
+
+// Warp-aggregated histogram of the top 11 bits of keys[valid].
+__device__ __forceinline__ void hist_top11(uint32_t *hist, const uint32_t (&keys)[TK_ITEMS], uint32_t valid)
+{
+    const int lane = threadIdx.x & 31;
+#pragma unroll
+    for (int i = 0; i < TK_ITEMS; ++i) {
+        const bool v = (valid >> i) & 1u;
+        const unsigned act = __ballot_sync(0xffffffffu, v);
+        if (v) {
+            const uint32_t bin = keys[i] >> 21;
+            const unsigned same = __match_any_sync(act, bin);
+            if (lane == __ffs(same) - 1) atomicAdd(&hist[bin], (uint32_t)__popc(same));
+        }
+    }
+}
+
 __global__ void __launch_bounds__(TK_THREADS)
 topk_rows_kernel(const float *__restrict__ scores, int64_t ld, int64_t row_begin,
                  const int32_t *__restrict__ lens, int64_t max_len, int k,
-                 int32_t *__restrict__ idx, WsHeader *hdr)
+                 int32_t *__restrict__ idx, WsHeader *hdr, int vec_ok)
 {
-    __shared__ uint32_t hist[2048];
-    __shared__ uint32_t warp_buf[32];
-    __shared__ uint32_t sh_bin, sh_above;
+    extern __shared__ __align__(16) uint8_t smem_raw[];
+    TopkSmem &sm = *reinterpret_cast<TopkSmem *>(smem_raw);
 
     const int64_t r = blockIdx.x;
     const int tid = threadIdx.x;
@@ -77,72 +255,193 @@ topk_rows_kernel(const float *__restrict__ scores, int64_t ld, int64_t row_begin
         for (int i = tid; i < k; i += TK_THREADS) out[i] = i < n ? i : -1;
         return;
     }
+    const bool vec = vec_ok != 0;
+    auto row_keys = [&](int64_t s, uint32_t (&keys)[TK_ITEMS], uint32_t &valid) {
+        load8(row, n, s, vec, keys, valid);
+    };
 
-    // ---- radix select of the k-th largest key ----
-    uint32_t prefix = 0, pmask = 0, remaining = (uint32_t)k;
-#pragma unroll 1
-    for (int pass = 0; pass < 3; ++pass) {
-        const int shift = pass == 0 ? 21 : (pass == 1 ? 10 : 0);
-        const int width = pass == 2 ? 10 : 11;
-        const int nb = 1 << width;
-        const uint32_t bmask = (uint32_t)nb - 1u;
-        for (int i = tid; i < nb; i += TK_THREADS) hist[i] = 0u;
-        __syncthreads();
-        for (int64_t s = tid; s < n; s += TK_THREADS) {
-            uint32_t key = float_key(row[s]);
-            if ((key & pmask) == prefix) atomicAdd(&hist[(key >> shift) & bmask], 1u);
-        }
-        __syncthreads();
-        // suffix counts from the top bin down: thread i owns reverse positions [i*bpt, (i+1)*bpt)
-        const int bpt = nb / TK_THREADS;
-        uint32_t local = 0;
-        for (int j = 0; j < bpt; ++j) local += hist[nb - 1 - (tid * bpt + j)];
-        uint32_t tot;
-        uint32_t cum = block_excl_scan(local, warp_buf, &tot);
-        for (int j = 0; j < bpt; ++j) {
-            int b = nb - 1 - (tid * bpt + j);
-            uint32_t c = hist[b];
-            if (cum < remaining && remaining <= cum + c) { sh_bin = (uint32_t)b; sh_above = cum; }
-            cum += c;
-        }
-        __syncthreads();
-        remaining -= sh_above;
-        prefix |= sh_bin << shift;
-        pmask |= bmask << shift;
-        __syncthreads();
+    // ---- pass 1: histogram of the top 11 bits over the row ----
+    for (int i = tid; i < 2048; i += TK_THREADS) sm.hist[i] = 0u;
+    if (tid == 0) { sm.sh_count = 0; sm.sh_overflow = 0; }
+    __syncthreads();
+    for (int64_t c0 = 0; c0 < n; c0 += TK_STEP) {
+        uint32_t keys[TK_ITEMS], valid;
+        row_keys(c0 + (int64_t)tid * TK_ITEMS, keys, valid);
+        hist_top11(sm.hist, keys, valid);
     }
-    const uint32_t thr = prefix;          // the k-th largest key
-    const uint32_t need = remaining;      // how many keys equal to thr are kept (lowest positions)
+    __syncthreads();
+    find_bin(sm, 2048, (uint32_t)k);
+    const uint32_t b1 = sm.sh_bin;
+    uint32_t remaining = (uint32_t)k - sm.sh_above;
 
-    // ---- ordered compaction ----
-    uint32_t base_gt = 0, base_eq = 0;
-    for (int64_t c0 = 0; c0 < n; c0 += (int64_t)TK_THREADS * TK_ITEMS) {
-        const int64_t s_first = c0 + (int64_t)tid * TK_ITEMS;
-        uint32_t flags_gt = 0, flags_eq = 0, n_gt = 0, n_eq = 0;
+    // ---- pass 2: ordered copy of every key with top bits >= b1 ----
+    uint32_t base = 0;
+    for (int64_t c0 = 0; c0 < n; c0 += TK_STEP) {
+        const int64_t s0 = c0 + (int64_t)tid * TK_ITEMS;
+        uint32_t keys[TK_ITEMS], valid, flags = 0, cnt = 0;
+        row_keys(s0, keys, valid);
 #pragma unroll
-        for (int i = 0; i < TK_ITEMS; ++i) {
-            int64_t s = s_first + i;
-            if (s < n) {
-                uint32_t key = float_key(row[s]);
-                if (key > thr) { flags_gt |= 1u << i; ++n_gt; }
-                else if (key == thr) { flags_eq |= 1u << i; ++n_eq; }
-            }
-        }
+        for (int i = 0; i < TK_ITEMS; ++i)
+            if (((valid >> i) & 1u) && (keys[i] >> 21) >= b1) { flags |= 1u << i; ++cnt; }
         uint32_t tot;
-        uint32_t ex = block_excl_scan((n_gt << 16) | n_eq, warp_buf, &tot);
-        uint32_t gt_before = base_gt + (ex >> 16), eq_before = base_eq + (ex & 0xffffu);
+        uint32_t off = base + block_excl_scan(cnt, sm.warp_buf, &tot);
 #pragma unroll
         for (int i = 0; i < TK_ITEMS; ++i) {
-            bool gt = (flags_gt >> i) & 1u, eq = (flags_eq >> i) & 1u;
-            if (gt || (eq && eq_before < need)) {
-                uint32_t pos = gt_before + min(eq_before, need);
-                if (pos < (uint32_t)k) out[pos] = (int32_t)(s_first + i);
+            if ((flags >> i) & 1u) {
+                if (off < TK_CAP) { sm.ckey[off] = keys[i]; sm.cpos[off] = (int32_t)(s0 + i); }
+                ++off;
             }
-            gt_before += gt;
-            eq_before += eq;
         }
-        base_gt += tot >> 16;
-        base_eq += tot & 0xffffu;
+        base += tot;
+    }
+    const uint32_t ncand = base;
+
+    if (ncand <= TK_CAP) select_on_chip(sm, ncand, b1, remaining, k, out);
+    else select_global(sm, row, n, vec, k, out);
+}
+
+
+// ---------------------------------------------------------------- long rows, split over CTAs
+// Workspace per row: hist[2048] (zeroed by the launcher), cnt[chunks], then
+// per chunk a fixed slot of TL_SLOT (key, position) candidates.
+
+constexpr int TL_CHUNK = 32768;            // positions per CTA
+constexpr int TL_SLOT = 8192;              // candidate slot per chunk (more: the row falls back)
+
+struct SplitWs {
+    uint32_t *hist;      // [rows][2048]
+    uint32_t *cnt;       // [rows][chunks]
+    uint32_t *ckey;      // [rows][chunks][TL_SLOT]
+    int32_t *cpos;       // [rows][chunks][TL_SLOT]
+    int chunks;
+};
+
+__device__ __forceinline__ int64_t split_len(const int32_t *lens, int64_t max_len, int64_t r)
+{
+    int64_t n = lens[r];
+    return (n < 1 || n > max_len) ? -1 : n;
+}
+
+// Pass 1: histogram of the top 11 bits of one chunk, added into the row's.
+__global__ void __launch_bounds__(TK_THREADS)
+topk_split_hist_kernel(const float *__restrict__ scores, int64_t ld, const int32_t *__restrict__ lens,
+                       int64_t max_len, int k, SplitWs ws, int vec_ok)
+{
+    __shared__ uint32_t hist[2048];
+    const int64_t r = blockIdx.y;
+    const int64_t n = split_len(lens, max_len, r);
+    const int64_t c0 = (int64_t)blockIdx.x * TL_CHUNK;
+    if (n <= k || c0 >= n) return;                  // short or invalid rows: the final kernel handles them
+    const int64_t c1 = min(n, c0 + TL_CHUNK);
+    const float *row = scores + r * ld;
+    for (int i = threadIdx.x; i < 2048; i += TK_THREADS) hist[i] = 0u;
+    __syncthreads();
+    for (int64_t s0 = c0; s0 < c1; s0 += TK_STEP) {
+        uint32_t keys[TK_ITEMS], valid;
+        load8(row, c1, s0 + (int64_t)threadIdx.x * TK_ITEMS, vec_ok != 0, keys, valid);
+        hist_top11(hist, keys, valid);
+    }
+    __syncthreads();
+    uint32_t *gh = ws.hist + r * 2048;
+    for (int i = threadIdx.x; i < 2048; i += TK_THREADS)
+        if (hist[i]) atomicAdd(&gh[i], hist[i]);
+}
+
+// Pass 2: ordered copy of the chunk's keys whose top 11 bits are >= the row's
+// threshold bin into the chunk's candidate slot.
+__global__ void __launch_bounds__(TK_THREADS)
+topk_split_collect_kernel(const float *__restrict__ scores, int64_t ld, const int32_t *__restrict__ lens,
+                          int64_t max_len, int k, SplitWs ws, int vec_ok)
+{
+    extern __shared__ __align__(16) uint8_t smem_raw[];
+    TopkSmem &sm = *reinterpret_cast<TopkSmem *>(smem_raw);
+    const int64_t r = blockIdx.y;
+    const int64_t n = split_len(lens, max_len, r);
+    const int64_t c0 = (int64_t)blockIdx.x * TL_CHUNK;
+    if (n <= k || c0 >= n) return;
+    const int64_t c1 = min(n, c0 + TL_CHUNK);
+    const float *row = scores + r * ld;
+    for (int i = threadIdx.x; i < 2048; i += TK_THREADS) sm.hist[i] = ws.hist[r * 2048 + i];
+    __syncthreads();
+    find_bin(sm, 2048, (uint32_t)k);
+    const uint32_t b1 = sm.sh_bin;
+    const int64_t slot = (r * ws.chunks + blockIdx.x) * (int64_t)TL_SLOT;
+    uint32_t base = 0;
+    for (int64_t s0 = c0; s0 < c1; s0 += TK_STEP) {
+        const int64_t s = s0 + (int64_t)threadIdx.x * TK_ITEMS;
+        uint32_t keys[TK_ITEMS], valid, flags = 0, cnt = 0;
+        load8(row, c1, s, vec_ok != 0, keys, valid);
+#pragma unroll
+        for (int i = 0; i < TK_ITEMS; ++i)
+            if (((valid >> i) & 1u) && (keys[i] >> 21) >= b1) { flags |= 1u << i; ++cnt; }
+        uint32_t tot;
+        uint32_t off = base + block_excl_scan(cnt, sm.warp_buf, &tot);
+#pragma unroll
+        for (int i = 0; i < TK_ITEMS; ++i) {
+            if ((flags >> i) & 1u) {
+                if (off < TL_SLOT) {
+                    ws.ckey[slot + off] = keys[i];
+                    ws.cpos[slot + off] = (int32_t)(s + i);
+                }
+                ++off;
+            }
+        }
+        base += tot;
+    }
+    if (threadIdx.x == 0) ws.cnt[r * ws.chunks + blockIdx.x] = base;
+}
+
+// Pass 3: one CTA per row joins the chunks' candidates in chunk order (so in
+// position order), finishes the select on chip, or falls back to the row.
+__global__ void __launch_bounds__(TK_THREADS)
+topk_split_final_kernel(const float *__restrict__ scores, int64_t ld, const int32_t *__restrict__ lens,
+                        int64_t max_len, int k, SplitWs ws, int32_t *__restrict__ idx, WsHeader *hdr,
+                        int vec_ok)
+{
+    extern __shared__ __align__(16) uint8_t smem_raw[];
+    TopkSmem &sm = *reinterpret_cast<TopkSmem *>(smem_raw);
+    const int64_t r = blockIdx.x;
+    const int tid = threadIdx.x;
+    int32_t *out = idx + r * (int64_t)k;
+    const int64_t n = split_len(lens, max_len, r);
+    if (n < 0) {
+        if (tid == 0) record_error(hdr, DSA_ERR_INVALID_ARG, (unsigned)r);
+        for (int i = tid; i < k; i += TK_THREADS) out[i] = -1;
+        return;
+    }
+    if (n <= k) {
+        for (int i = tid; i < k; i += TK_THREADS) out[i] = i < n ? i : -1;
+        return;
+    }
+    const float *row = scores + r * ld;
+    for (int i = tid; i < 2048; i += TK_THREADS) sm.hist[i] = ws.hist[r * 2048 + i];
+    __syncthreads();
+    find_bin(sm, 2048, (uint32_t)k);
+    const uint32_t b1 = sm.sh_bin;
+    const uint32_t remaining = (uint32_t)k - sm.sh_above;
+    const int nch = (int)((n + TL_CHUNK - 1) / TL_CHUNK);
+    uint32_t total = 0;
+    bool fits = true;
+    for (int c = 0; c < nch; ++c) {
+        const uint32_t m = ws.cnt[r * ws.chunks + c];
+        total += m;
+        fits = fits && m <= TL_SLOT;
+    }
+    if (fits && total <= TK_CAP) {
+        uint32_t off = 0;
+        for (int c = 0; c < nch; ++c) {
+            const uint32_t m = ws.cnt[r * ws.chunks + c];
+            const int64_t slot = (r * ws.chunks + c) * (int64_t)TL_SLOT;
+            for (uint32_t i = tid; i < m; i += TK_THREADS) {
+                sm.ckey[off + i] = ws.ckey[slot + i];
+                sm.cpos[off + i] = ws.cpos[slot + i];
+            }
+            off += m;
+        }
+        __syncthreads();
+        select_on_chip(sm, total, b1, remaining, k, out);
+    } else {
+        select_global(sm, row, n, vec_ok != 0, k, out);
     }
 }
 
@@ -153,8 +452,53 @@ cudaError_t launch_topk_rows(const float *scores, int64_t ld, int64_t row_begin,
                              int32_t *idx, WsHeader *hdr, cudaStream_t st)
 {
     if (row_count <= 0) return cudaSuccess;
-    topk_rows_kernel<<<(unsigned)row_count, TK_THREADS, 0, st>>>(scores, ld, row_begin, lens,
-                                                                  max_len, k, idx, hdr);
+    const size_t smem = sizeof(TopkSmem);
+    cudaError_t e = cudaFuncSetAttribute(topk_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem);
+    if (e != cudaSuccess) return e;
+    const int vec_ok = (ld % 4 == 0) && ((reinterpret_cast<uintptr_t>(scores) & 15u) == 0);
+    topk_rows_kernel<<<(unsigned)row_count, TK_THREADS, smem, st>>>(scores, ld, row_begin, lens,
+                                                                     max_len, k, idx, hdr, vec_ok);
+    return cudaGetLastError();
+}
+
+size_t topk_split_ws_bytes(int64_t rows, int64_t max_len)
+{
+    const int64_t chunks = ceil_div(max_len, TL_CHUNK);
+    return align_up(sizeof(uint32_t) * (size_t)rows * 2048, 256) +
+           align_up(sizeof(uint32_t) * (size_t)rows * chunks, 256) +
+           2 * align_up(sizeof(uint32_t) * (size_t)rows * chunks * TL_SLOT, 256);
+}
+
+cudaError_t launch_topk_split(const float *scores, int64_t ld, const int32_t *lens, int64_t max_len,
+                              int64_t rows, int k, int32_t *idx, void *ws_base, WsHeader *hdr,
+                              cudaStream_t st)
+{
+    if (rows <= 0) return cudaSuccess;
+    const int64_t chunks = ceil_div(max_len, TL_CHUNK);
+    uint8_t *p = static_cast<uint8_t *>(ws_base);
+    SplitWs ws;
+    ws.chunks = (int)chunks;
+    ws.hist = reinterpret_cast<uint32_t *>(p);
+    p += align_up(sizeof(uint32_t) * (size_t)rows * 2048, 256);
+    ws.cnt = reinterpret_cast<uint32_t *>(p);
+    p += align_up(sizeof(uint32_t) * (size_t)rows * chunks, 256);
+    ws.ckey = reinterpret_cast<uint32_t *>(p);
+    p += align_up(sizeof(uint32_t) * (size_t)rows * chunks * TL_SLOT, 256);
+    ws.cpos = reinterpret_cast<int32_t *>(p);
+    const int vec_ok = (ld % 4 == 0) && ((reinterpret_cast<uintptr_t>(scores) & 15u) == 0);
+    const size_t smem = sizeof(TopkSmem);
+    cudaError_t e = cudaMemsetAsync(ws.hist, 0, sizeof(uint32_t) * (size_t)rows * 2048, st);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(topk_split_collect_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(topk_split_final_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    dim3 grid((unsigned)chunks, (unsigned)rows);
+    topk_split_hist_kernel<<<grid, TK_THREADS, 0, st>>>(scores, ld, lens, max_len, k, ws, vec_ok);
+    topk_split_collect_kernel<<<grid, TK_THREADS, smem, st>>>(scores, ld, lens, max_len, k, ws, vec_ok);
+    topk_split_final_kernel<<<(unsigned)rows, TK_THREADS, smem, st>>>(scores, ld, lens, max_len, k, ws, idx,
+                                                                      hdr, vec_ok);
     return cudaGetLastError();
 }
 

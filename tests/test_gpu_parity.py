@@ -279,3 +279,32 @@ def test_index_scores_fill_upper_off_leaves_upper_untouched():
         assert np.all(o[r, t + 1:] == 5.0)
         o[r, t + 1:] = -np.inf
     assert_scores_close(o, ref, "fill_upper=False")
+
+
+def test_topk_candidate_overflow_falls_back_exactly():
+    """Rows whose threshold bin holds more keys than fit on chip take the
+    global-memory path; the result is still exact."""
+    T, k = 30000, 100
+    rng = np.random.default_rng(9)
+    sc = np.zeros((4, T), np.float32)                       # 30000 equal keys
+    sc[1] = np.float32(3.0) + np.float32(2 ** -20) * rng.integers(0, 4, T)   # 4 distinct, huge bins
+    sc[2] = rng.standard_normal(T).astype(np.float32)       # ordinary row (on-chip path)
+    sc[3, ::2] = 1.0                                         # 15000 ties at the top
+    _topk_check(sc, k, row_begin=T - 4)
+
+
+def test_decode_all_equal_scores_take_the_lowest_positions():
+    """Every index key zero: all scores tie at 0, the selection is the k lowest
+    positions; long rows overflow the on-chip candidate slots and take the
+    global-memory path."""
+    spec = small_decode_spec((40000, 9000, 100), k=300, H_q=16, seed=3)
+    inp = dsa_synth.make_decode(spec)
+    inp["kidx_cache"].zero_()
+    dev = to_dev(inp)
+    _, _, idx = dsa.dsa_decode(dev, spec.k, 40000, sm_of(128))
+    idx = idx.cpu().numpy()
+    for b, n in enumerate(spec.context_lens):
+        expect = list(range(min(n, spec.k))) + [-1] * (spec.k - min(n, spec.k))
+        assert idx[b].tolist() == expect
+    ref = oracle.decode(inp, spec.k, sm_of(128))
+    np.testing.assert_array_equal(idx, ref["idx"])
