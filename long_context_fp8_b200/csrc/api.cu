@@ -71,6 +71,14 @@ cudaError_t run_attn(const void *q, const void *k, const void *v, const int32_t 
     if (dtype == DSA_F32)
         return launch_sparse_attn_f32((const float *)q, (const float *)k, (const float *)v, idx,
                                       T, H_q, d, k_sel, sm_scale, (float *)out, lse, st);
+    if (sparse_attn_tc_supported(H_q, d)) {
+        // tcgen05 kernel: the 128 query heads of a token are the MMA's M dimension
+        cudaError_t e = launch_sparse_attn_tc((const uint16_t *)q, (const uint16_t *)k,
+                                              (const uint16_t *)v, T, T, nullptr, nullptr, 0, 0, 0,
+                                              idx, T, H_q, d, k_sel, sm_scale, (uint16_t *)out, lse,
+                                              nullptr, 1, nullptr, st);
+        if (e != cudaErrorNotSupported) return e;
+    }
     return launch_sparse_attn_bf16((const uint16_t *)q, (const uint16_t *)k, (const uint16_t *)v,
                                    idx, T, T, H_q, d, k_sel, sm_scale, (uint16_t *)out, lse, st);
 }
@@ -257,7 +265,7 @@ dsa_status dsa_decode(const void *q_idx, const float *q_scale, const void *w, co
     cudaError_t e = cudaMemsetAsync(hdr, 0, sizeof(WsHeader), st);
     if (e == cudaSuccess) {
         // tensor-core (tcgen05 + TMA) indexer where the shape allows, else mma.sync
-        if (decode_index_tc_supported(H_I, page_size) &&
+        if (decode_index_tc_supported(H_I, page_size) && B <= 4096 &&
             (int64_t)num_pages * page_size < ((int64_t)1 << 31) &&
             (reinterpret_cast<uintptr_t>(kscale_cache) & 15u) == 0)
             e = launch_decode_index_tc((const uint8_t *)q_idx, q_scale, (const uint16_t *)w,
@@ -274,10 +282,25 @@ dsa_status dsa_decode(const void *q_idx, const float *q_scale, const void *w, co
         e = launch_topk_split(scores, max_context, context_lens, max_context, B, k_sel, idx, topk_ws,
                               hdr, st);
     if (e == cudaSuccess) {
-        PagedKV kv{(const uint16_t *)k_cache, (const uint16_t *)v_cache, block_table, context_lens,
-                   num_pages, max_pages_per_seq, page_size};
-        e = launch_sparse_attn_paged_bf16((const uint16_t *)q, kv, idx, B, H_q, d, k_sel, sm_scale,
-                                          (uint16_t *)out, lse_out, part, splits, hdr, st);
+        bool done = false;
+        if (sparse_attn_tc_supported(H_q, d) && (int64_t)num_pages * page_size < ((int64_t)1 << 31)) {
+            // tcgen05 kernel over the paged caches, the index list split in 128-row blocks
+            const int chunk = (int)(ceil_div(ceil_div(k_sel, splits), 128) * 128);
+            const int tc_splits = (int)ceil_div(k_sel, chunk);
+            e = launch_sparse_attn_tc((const uint16_t *)q, (const uint16_t *)k_cache,
+                                      (const uint16_t *)v_cache, num_pages * page_size, 0,
+                                      block_table, context_lens, num_pages, max_pages_per_seq,
+                                      page_size, idx, B, H_q, d, k_sel, sm_scale, (uint16_t *)out,
+                                      lse_out, part, tc_splits, hdr, st);
+            if (e == cudaSuccess) e = launch_merge_splits(part, B, tc_splits, H_q, d, (uint16_t *)out, lse_out, st);
+            done = e != cudaErrorNotSupported;
+        }
+        if (!done) {
+            PagedKV kv{(const uint16_t *)k_cache, (const uint16_t *)v_cache, block_table, context_lens,
+                       num_pages, max_pages_per_seq, page_size};
+            e = launch_sparse_attn_paged_bf16((const uint16_t *)q, kv, idx, B, H_q, d, k_sel, sm_scale,
+                                              (uint16_t *)out, lse_out, part, splits, hdr, st);
+        }
     }
     return cuda_status(e);
 }

@@ -34,6 +34,7 @@ constexpr int DT_TILE_BYTES = DT_TILE * 128;
 constexpr int DT_EPI_WARPS = 4;
 constexpr int DT_THREADS = 32 * (2 + DT_EPI_WARPS);
 constexpr int DT_TMEM_COLS = 128;            // two 64-column accumulators
+constexpr int DT_MAX_B = 4096;               // sequences the per-CTA item table can hold
 
 struct DecTcArgs {
     const float *sq;
@@ -56,7 +57,8 @@ constexpr size_t dt_smem_bytes()
 {
     return 1024 /*align slack*/ + 2 * 8192 /*q, double-buffered*/ + (size_t)DT_STAGES * DT_TILE_BYTES +
            (size_t)DT_STAGES * DT_TILE * 4 /*key scales*/ + DT_STAGES * 4 /*segment masks*/ +
-           2 * 64 * 4 /*c*/ + (2 * DT_STAGES + 8) * 8 + 16;
+           2 * 64 * 4 /*c*/ + (2 * DT_STAGES + 8) * 8 + 16 +
+           (size_t)(2 * DT_MAX_B + 1) * 4 /*per-sequence lengths and tile prefix*/;
 }
 
 // Context length of sequence b if valid, else 0 (the caller records the error).
@@ -67,35 +69,42 @@ __device__ __forceinline__ int64_t seq_len(const DecTcArgs &a, int b)
     return n;
 }
 
+// Per-CTA table of the sequences' lengths and of the prefix sums of their
+// 128-key tiles (filled once from context_lens), so that locating an item is
+// a binary search in shared memory.
+struct SeqTable {
+    const int32_t *n;        // [B]
+    const int32_t *prefix;   // [B + 1]
+    int B;
+};
+
 // Walks this CTA's contiguous share of the (sequence, 128-key tile) items.
 struct ItemWalk {
     int b = 0;
     int64_t tile = 0, left = 0, n = 0;
-    __device__ bool start(const DecTcArgs &a, int64_t first, int64_t count)
+    __device__ bool start(const SeqTable &t, int64_t first, int64_t count)
     {
         left = count;
-        b = 0;
-        tile = first;
-        while (b < a.B) {
-            n = seq_len(a, b);
-            int64_t nt = (n + DT_TILE - 1) / DT_TILE;
-            if (tile < nt) return left > 0;
-            tile -= nt;
-            ++b;
+        if (count <= 0 || first >= t.prefix[t.B]) return false;
+        int lo = 0, hi = t.B - 1;                        // last b with prefix[b] <= first
+        while (lo < hi) {
+            int mid = (lo + hi + 1) >> 1;
+            if (t.prefix[mid] <= first) lo = mid; else hi = mid - 1;
         }
-        return false;
+        b = lo;
+        tile = first - t.prefix[b];
+        n = t.n[b];
+        return true;
     }
-    __device__ bool next(const DecTcArgs &a)
+    __device__ bool next(const SeqTable &t)
     {
         if (--left <= 0) return false;
         ++tile;
-        while (b < a.B) {
-            int64_t nt = (n + DT_TILE - 1) / DT_TILE;
-            if (tile < nt) return true;
+        while (b < t.B && tile >= t.prefix[b + 1] - t.prefix[b]) {
             tile = 0;
-            if (++b < a.B) n = seq_len(a, b);
+            if (++b < t.B) n = t.n[b];
         }
-        return false;
+        return b < t.B;
     }
 };
 
@@ -132,19 +141,41 @@ decode_index_tc_kernel(const __grid_constant__ CUtensorMap kmap,
     uint64_t *qfull = kempty + DT_STAGES, *qempty = qfull + 2;
     uint64_t *tfull = qempty + 2, *tempty = tfull + 2;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(tempty + 2);
+    int32_t *tab_n = reinterpret_cast<int32_t *>(tmem_slot + 4);     // [DT_MAX_B]
+    int32_t *tab_prefix = tab_n + DT_MAX_B;                            // [DT_MAX_B + 1]
     __shared__ volatile int abort_flag;
     __shared__ int k_issued, k_consumed, mma_items;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int ps = a.page_size;
 
-    // this CTA's share of the work items
-    int64_t total = 0;
-    for (int b = 0; b < a.B; ++b) {
-        int64_t n = seq_len(a, b);
-        if (n == 0 && blockIdx.x == 0 && tid == 0) record_error(a.hdr, DSA_ERR_INVALID_ARG, (unsigned)b);
-        total += (n + DT_TILE - 1) / DT_TILE;
+    // per-sequence lengths and tile prefix sums (warp 0: lane l scans a block of sequences)
+    if (warp == 0) {
+        const int per_lane = (a.B + 31) / 32;
+        const int b0 = min(a.B, lane * per_lane), b1 = min(a.B, b0 + per_lane);
+        int32_t local = 0;
+        for (int b = b0; b < b1; ++b) {
+            const int64_t n = seq_len(a, b);
+            if (n == 0 && blockIdx.x == 0) record_error(a.hdr, DSA_ERR_INVALID_ARG, (unsigned)b);
+            tab_n[b] = (int32_t)n;
+            local += (int32_t)((n + DT_TILE - 1) / DT_TILE);
+        }
+        int32_t incl = local;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            int32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += y;
+        }
+        int32_t run = incl - local;
+        for (int b = b0; b < b1; ++b) {
+            tab_prefix[b] = run;
+            run += (tab_n[b] + DT_TILE - 1) / DT_TILE;
+        }
+        if (lane == 31) tab_prefix[a.B] = incl;
     }
+    __syncthreads();
+    const SeqTable tab{tab_n, tab_prefix, a.B};
+    const int64_t total = tab_prefix[a.B];
     const int64_t per = (total + gridDim.x - 1) / gridDim.x;
     const int64_t first = (int64_t)blockIdx.x * per;
     const int64_t count = min(per, total - first);
@@ -184,7 +215,7 @@ decode_index_tc_kernel(const __grid_constant__ CUtensorMap kmap,
         for (int64_t j0 = 0; j0 < count && !stop; j0 += 32) {
             // this lane's item j0 + lane
             ItemWalk mine;
-            const bool have = j0 + lane < count && mine.start(a, first + j0 + lane, count - j0 - lane);
+            const bool have = j0 + lane < count && mine.start(tab, first + j0 + lane, count - j0 - lane);
             int my_b = have ? mine.b : -1;
             uint32_t my_mask = 0;
             int my_slot[8];
@@ -254,7 +285,7 @@ decode_index_tc_kernel(const __grid_constant__ CUtensorMap kmap,
             ItemWalk it;
             int j = 0, seg = -1, prev_b = -1;
             uint64_t bdesc = 0;
-            for (bool ok = it.start(a, first, count); ok; ok = it.next(a), ++j) {
+            for (bool ok = it.start(tab, first, count); ok; ok = it.next(tab), ++j) {
                 if (it.b != prev_b) {
                     if (seg >= 0) umma_commit(&qempty[seg & 1]);   // previous query heads are free
                     ++seg;
@@ -283,7 +314,7 @@ decode_index_tc_kernel(const __grid_constant__ CUtensorMap kmap,
         ItemWalk it;
         int j = 0, seg = -1, prev_b = -1;
         bool dead = false;
-        for (bool ok = it.start(a, first, count); ok; ok = it.next(a), ++j) {
+        for (bool ok = it.start(tab, first, count); ok; ok = it.next(tab), ++j) {
             if (it.b != prev_b) {                       // per-sequence head weights c_h = w[b,h] * sq[b]
                 ++seg;
                 prev_b = it.b;
@@ -296,12 +327,19 @@ decode_index_tc_kernel(const __grid_constant__ CUtensorMap kmap,
             const int s = j % DT_STAGES, acc = j & 1;
             const int r = q4 * 32 + lane;
             const int64_t pos = it.tile * DT_TILE + r;
-            if (!wait_or_abort(&kfull[s], (j / DT_STAGES) & 1, &abort_flag)) { dead = true; continue; }
+            if (!__all_sync(0xffffffffu, wait_or_abort(&kfull[s], (j / DT_STAGES) & 1, &abort_flag))) {
+                dead = true;
+                continue;
+            }
             const bool live = pos < it.n && ((kmask[s] >> (r / a.box_rows)) & 1u);
             const float ksc = kss[s * DT_TILE + r];
             __syncwarp();
             if (lane == 0) mbar_arrive(&kempty[s]);
-            if (!wait_or_abort(&tfull[acc], (j >> 1) & 1, &abort_flag)) { dead = true; continue; }
+            // warp-uniform outcome: the TMEM loads below are warp-collective
+            if (!__all_sync(0xffffffffu, wait_or_abort(&tfull[acc], (j >> 1) & 1, &abort_flag))) {
+                dead = true;
+                continue;
+            }
             tc_fence_after();
             const uint32_t trow = tmem + ((uint32_t)(q4 * 32) << 16) + (uint32_t)(acc * 64);
             const float *c = cw + (seg & 1) * 64;
@@ -369,7 +407,7 @@ cudaError_t launch_decode_index_tc(const uint8_t *q8, const float *sq, const uin
                                    WsHeader *hdr, cudaStream_t st)
 {
     if (B <= 0) return cudaSuccess;
-    if (!decode_index_tc_supported(H, page_size)) return cudaErrorNotSupported;
+    if (!decode_index_tc_supported(H, page_size) || B > DT_MAX_B) return cudaErrorNotSupported;
     if ((int64_t)num_pages * page_size >= ((int64_t)1 << 31) || (int64_t)B * H >= ((int64_t)1 << 31))
         return cudaErrorNotSupported;
     CUtensorMap kmap, qmap;

@@ -225,7 +225,7 @@ index_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant_
             const int64_t t0 = a.row_begin + tw.rb * IT_BM;
             const int64_t s0 = tw.kt * IT_BN;
             epi_bar_sync();                          // the previous tile is done with Cs / Sk
-            dead = dead || abort_flag;
+            dead = __any_sync(0xffffffffu, dead || abort_flag);
             if (!dead) {
                 for (int i = et; i < IT_BM * H; i += 32 * IT_EPI_WARPS) {
                     const int r = i / H, h = i % H;
@@ -243,7 +243,9 @@ index_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant_
             for (int i = 0; i < 64; ++i) sc[i] = 0ull;
             for (int h = 0; h < H; ++h) {
                 const int g = lt * H + h, acc = g & 1;
-                if (!wait_or_abort(&tfull[acc], (g >> 1) & 1, &abort_flag)) { dead = true; break; }
+                // warp-uniform outcome: the TMEM loads below are warp-collective
+                const bool ok = wait_or_abort(&tfull[acc], (g >> 1) & 1, &abort_flag);
+                if (!__all_sync(0xffffffffu, ok)) { dead = true; break; }
                 tc_fence_after();
                 const float c = Cs[h * IT_CS_STRIDE + row];
                 const uint64_t cc = f2_pack(c, c);

@@ -64,10 +64,22 @@ cudaError_t launch_sparse_attn_paged_bf16(const uint16_t *q, const PagedKV &kv,
                                           float *part, int splits, WsHeader *hdr,
                                           cudaStream_t st);
 size_t sparse_attn_paged_part_bytes(int B, int H, int d, int splits);
+cudaError_t launch_merge_splits(const float *part, int rows, int splits, int H, int d, uint16_t *out,
+                               float *lse, cudaStream_t st);
 int sparse_attn_paged_splits(int B, int ksel);
 cudaError_t launch_sparse_attn_f32(const float *q, const float *k, const float *v,
                                    const int32_t *idx, int64_t T, int H, int d, int ksel,
                                    float sm_scale, float *out, float *lse, cudaStream_t st);
+
+// tcgen05 attention (sparse_attn_tc.cu): H a multiple of 128, d == 128.
+// Contiguous K/V when block_table is null (positions < T), else paged.
+bool sparse_attn_tc_supported(int H, int d);
+cudaError_t launch_sparse_attn_tc(const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                                  int64_t kv_rows, int64_t T, const int32_t *block_table,
+                                  const int32_t *context_lens, int64_t num_pages, int max_pages,
+                                  int page_size, const int32_t *idx, int64_t rows, int H, int d,
+                                  int ksel, float sm_scale, uint16_t *out, float *lse, float *part,
+                                  int splits, WsHeader *hdr, cudaStream_t st);
 
 // ---- decode indexer (decode_tc.cu: tcgen05 + TMA; decode.cu: mma.sync) ----
 bool decode_index_tc_supported(int H, int page_size);

@@ -106,6 +106,25 @@ __device__ __forceinline__ void bulk_load(void *smem_dst, const void *gsrc, uint
         :: "r"(smem_u32(smem_dst)), "l"(gsrc), "r"(bytes), "r"(smem_u32(bar)) : "memory");
 }
 
+// Four rows (y0..y3) of a 2-D tensor map, one box each, starting at column x.
+__device__ __forceinline__ void tma_gather4(void *smem_dst, const CUtensorMap *map, uint64_t *bar, int x,
+                                            int y0, int y1, int y2, int y3)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];"
+        :: "r"(smem_u32(smem_dst)), "l"(map), "r"(smem_u32(bar)), "r"(x), "r"(y0), "r"(y1), "r"(y2),
+           "r"(y3)
+        : "memory");
+}
+
+// Order this thread's generic-proxy shared-memory writes before later
+// async-proxy (tensor core, TMA) accesses.
+__device__ __forceinline__ void fence_proxy_async_smem()
+{
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
 // ---------------------------------------------------------------- UMMA
 
 // Shared-memory matrix descriptor of a K-major operand stored as rows of 128
@@ -124,6 +143,32 @@ __device__ __forceinline__ uint64_t umma_desc_k_sw128(uint32_t smem_addr)
     return d;
 }
 
+// Descriptor of an MN-major operand in the 128-byte swizzle: rows of 128 bytes
+// (64 16-bit elements along M/N) for successive K indices, 8-row groups `sbo`
+// bytes apart along K, 64-element groups `lbo` bytes apart along M/N.
+__device__ __forceinline__ uint64_t umma_desc_mn_sw128(uint32_t smem_addr, uint32_t lbo, uint32_t sbo)
+{
+    uint64_t d = 0;
+    d |= (uint64_t)((smem_addr & 0x3FFFFu) >> 4);
+    d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
+    d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
+    d |= (uint64_t)1 << 46;
+    d |= (uint64_t)2 << 61;
+    return d;
+}
+
+// K-major, 128-byte swizzle, with an explicit stride between 8-row groups.
+__device__ __forceinline__ uint64_t umma_desc_k_sw128_sbo(uint32_t smem_addr, uint32_t sbo)
+{
+    uint64_t d = 0;
+    d |= (uint64_t)((smem_addr & 0x3FFFFu) >> 4);
+    d |= (uint64_t)1 << 16;
+    d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
+    d |= (uint64_t)1 << 46;
+    d |= (uint64_t)2 << 61;
+    return d;
+}
+
 // Instruction descriptor: E4M3 x E4M3 -> fp32, both operands K-major.
 __host__ __device__ constexpr uint32_t umma_idesc_e4m3_f32(int M, int N)
 {
@@ -133,11 +178,12 @@ __host__ __device__ constexpr uint32_t umma_idesc_e4m3_f32(int M, int N)
            | ((uint32_t)(M >> 4) << 24);   // M / 16
 }
 
-// Instruction descriptor: bf16 x bf16 -> fp32, both operands K-major.
-__host__ __device__ constexpr uint32_t umma_idesc_bf16_f32(int M, int N)
+// Instruction descriptor: bf16 x bf16 -> fp32; A K-major; B K-major or (b_mn)
+// MN-major.
+__host__ __device__ constexpr uint32_t umma_idesc_bf16_f32(int M, int N, bool b_mn = false)
 {
-    return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) |
-           ((uint32_t)(M >> 4) << 24);
+    return (1u << 4) | (1u << 7) | (1u << 10) | ((b_mn ? 1u : 0u) << 16) |
+           ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
 
 __device__ __forceinline__ void umma_f8f6f4(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc,
@@ -215,6 +261,22 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&v)[16])
 
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
+// 32 lanes x 32 columns store (the inverse of tmem_ld32); complete with tmem_wait_st.
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&v)[32])
+{
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+        "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+        "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};"
+        :: "r"(taddr), "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]),
+           "r"(v[7]), "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]),
+           "r"(v[14]), "r"(v[15]), "r"(v[16]), "r"(v[17]), "r"(v[18]), "r"(v[19]), "r"(v[20]),
+           "r"(v[21]), "r"(v[22]), "r"(v[23]), "r"(v[24]), "r"(v[25]), "r"(v[26]), "r"(v[27]),
+           "r"(v[28]), "r"(v[29]), "r"(v[30]), "r"(v[31])
+        : "memory");
+}
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
 // Wait for this thread's outstanding tensor-memory loads, naming the 16
 // registers the last load wrote so that no use of them is scheduled earlier.
 __device__ __forceinline__ void tmem_wait_ld_dep16(uint32_t (&v)[16])
@@ -272,5 +334,8 @@ __device__ __forceinline__ uint32_t elect_one_lane() { return (threadIdx.x & 31)
 // or returns false if the driver entry point is unavailable or rejects it.
 bool make_tmap_u8(CUtensorMap *map, const void *base, int rank, const uint64_t *dims,
                   const uint64_t *strides_bytes, const uint32_t *box);
+// Same for a 2-D bf16 tensor (dims/box in elements).
+bool make_tmap_bf16_2d(CUtensorMap *map, const void *base, uint64_t cols, uint64_t rows,
+                       uint64_t row_stride_bytes, uint32_t box_cols, uint32_t box_rows);
 
 }  // namespace dsa

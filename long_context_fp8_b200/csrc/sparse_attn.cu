@@ -409,6 +409,16 @@ cudaError_t launch_sparse_attn_paged_bf16(const uint16_t *q, const PagedKV &kv,
     return cudaGetLastError();
 }
 
+cudaError_t launch_merge_splits(const float *part, int rows, int splits, int H, int d, uint16_t *out,
+                               float *lse, cudaStream_t st)
+{
+    if (rows <= 0 || splits <= 1) return cudaSuccess;
+    if (d != 128) return cudaErrorNotSupported;
+    dim3 mg((unsigned)rows, (unsigned)H);
+    merge_splits_kernel<128><<<mg, 128, 0, st>>>(part, rows, splits, H, out, lse);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_sparse_attn_f32(const float *q, const float *k, const float *v,
                                    const int32_t *idx, int64_t T, int H, int d, int ksel,
                                    float sm_scale, float *out, float *lse, cudaStream_t st)

@@ -308,3 +308,27 @@ def test_decode_all_equal_scores_take_the_lowest_positions():
         assert idx[b].tolist() == expect
     ref = oracle.decode(inp, spec.k, sm_of(128))
     np.testing.assert_array_equal(idx, ref["idx"])
+
+
+def test_sparse_attn_running_max_jump_per_head():
+    """A key whose logit is huge for one head only, placed in a later 128-row
+    block: that head's running max jumps (its output is rescaled) while the
+    other heads of the same warp keep theirs."""
+    T, H, d, k = 400, 128, 128, 1024
+    g = torch.Generator().manual_seed(77)
+    q = torch.randn((T, H, d), generator=g).to(torch.bfloat16)
+    K = torch.randn((T, d), generator=g).to(torch.bfloat16)
+    V = torch.randn((T, d), generator=g).to(torch.bfloat16)
+    rng = np.random.default_rng(77)
+    idx = np.full((T, k), -1, np.int32)
+    for t in range(T):
+        n = min(k, t + 1)
+        idx[t, :n] = np.arange(n)
+    # row t >= 300: key 290 (third block) aligned with head t % H, scaled up
+    for t in range(300, T, 7):
+        K[290] = (q[t, t % H].float() * 3.0).to(torch.bfloat16)
+        break
+    out, lse = dsa.dsa_sparse_attn(q.cuda(), K.cuda(), V.cuda(), torch.from_numpy(idx).cuda(), sm_of(d))
+    ref, ref_lse = oracle.sparse_attn(q, K, V, idx, np.arange(T), sm_of(d))
+    assert_attn_close(out.float().cpu().numpy(), ref, lse.cpu().numpy(), ref_lse, "max jump")
+    assert np.max(ref_lse) > 20.0      # the jump did happen for some (row, head)
