@@ -222,14 +222,21 @@ sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_con
             if (warp == 5) stop = stop || abort_flag;
             ++qi;
             const int32_t *irow = a.idx + item.row * a.ksel;
-            int e = item.e0 + pt;
+            // warp (w - 4) copies rows 32 (w - 4) .. +31 of each block; lane l copies
+            // 16-byte chunk l % 16 of the row's K (l < 16) or V (l >= 16), so one
+            // instruction moves one whole row pair (two 256-byte runs).  Lane l also
+            // resolves row 32 (w - 4) + l of the block, broadcast by shuffles.
+            const int rbase = (warp - 4) * 32;
+            int e = item.e0 + rbase + lane;
             int p_next = e < item.e1 ? __ldg(irow + e) : -1;
+            const int chunk = lane & 15;
+            const bool is_v = lane >= 16;
             for (int b = 0; b < item.nblk && !stop; ++b, ++g) {
                 const int st = g % AT_STAGES;
                 const int p = p_next;
                 e += AT_BLK;                          // prefetch the next block's index
                 p_next = (b + 1 < item.nblk && e < item.e1) ? __ldg(irow + e) : -1;
-                // warp-uniform outcome: the ballot below needs every lane
+                // warp-uniform outcome: the ballot and shuffles below need every lane
                 const bool ok = __all_sync(0xffffffffu,
                                            wait_or_abort(&kvempty[st], ((g / AT_STAGES) & 1) ^ 1, &abort_flag));
                 if (!ok) { stop = true; break; }
@@ -251,13 +258,16 @@ sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_con
                 }
                 const unsigned vw = __ballot_sync(0xffffffffu, v);
                 if (lane == 0) valid[st * 2 + (warp - 4)] = vw;
-                uint8_t *kt = KVs + st * AT_STAGE, *vt = kt + AT_KTILE;
-                const uint16_t *ksrc = a.k + (v ? r : 0) * AT_D, *vsrc = a.v + (v ? r : 0) * AT_D;
-#pragma unroll
-                for (int c = 0; c < 16; ++c) {
-                    const int off = (c >> 3) * AT_KHALF + pt * 128 + (((c & 7) ^ (pt & 7)) << 4);
-                    cp_async_16(kt + off, ksrc + c * 8, v);
-                    cp_async_16(vt + off, vsrc + c * 8, v);
+                uint8_t *tile = KVs + st * AT_STAGE + (is_v ? AT_KTILE : 0);
+                const uint16_t *base = is_v ? a.v : a.k;
+                const int coff = (chunk >> 3) * AT_KHALF;
+#pragma unroll 4
+                for (int i = 0; i < 32; ++i) {
+                    const int j = rbase + i;          // row of the block
+                    const int64_t ri = __shfl_sync(0xffffffffu, r, i);
+                    const bool vi = (vw >> i) & 1u;
+                    cp_async_16(tile + coff + j * 128 + (((chunk & 7) ^ (j & 7)) << 4),
+                                base + ri * AT_D + chunk * 8, vi);
                 }
                 cp_async_commit();
                 if (pt == 0) kv_issued = g + 1;

@@ -4,18 +4,18 @@
 // toward the lower position, emitted in ascending position order.
 //
 // One CTA per row.  Scores are mapped to order-preserving uint32 keys (-0
-// folded onto +0).  Two passes over the row:
-//   1. a histogram of the top 11 key bits (16-byte loads, warp-aggregated
-//      shared-memory atomics: neighbouring scores share their top bits),
-//      which fixes the bin b1 holding the k-th largest key;
-//   2. an ordered compaction that copies every (key, position) whose top bits
-//      are >= b1 into shared memory -- the keys above b1 are selected for
-//      sure, those in b1 are the only ones left to decide.
-// The remaining 21 bits are resolved by two more histogram passes over the
-// candidates in shared memory, and a last ordered compaction over them emits
-// the selection in ascending position order (no sort needed).  If the
-// candidates do not fit in shared memory, the row falls back to the same
-// radix select run over the row in global memory.
+// folded onto +0).  Normally one pass over the row: a threshold tau is guessed
+// from 2048 evenly spaced samples (the sample rank that should leave about
+// 1.5 k keys of the row at or above it), and an ordered compaction copies
+// every (key, position) with key >= tau into shared memory.  If that yields at
+// least k and at most the buffer's capacity, the selection is among them:
+// an exact radix select over the candidates on chip and a last ordered
+// compaction emit it in ascending position order (no sort needed).  Rows
+// short enough to fit are copied whole.  Otherwise the row falls back to two
+// passes: a histogram of the top 11 key bits (warp-aggregated atomics) fixes
+// the bin holding the k-th largest key, the keys in or above it go on chip;
+// and if even those do not fit, a radix select runs over the row in global
+// memory.  Every path is exact; the guess only decides which one is taken.
 #include "kernels.h"
 
 namespace dsa {
@@ -27,10 +27,13 @@ constexpr int TK_ITEMS = 8;                          // consecutive positions pe
 constexpr int TK_STEP = TK_THREADS * TK_ITEMS;       // positions per block-wide step
 constexpr int TK_CAP = 12288;                        // shared-memory candidate capacity
 
+constexpr int TK_SAMPLE = 2048;                     // evenly spaced samples for the threshold guess
+
 struct TopkSmem {
     uint32_t hist[2048];
     uint32_t warp_buf[32];
     uint32_t sh_bin, sh_above, sh_count, sh_overflow;
+    uint32_t sample[TK_SAMPLE];
     uint32_t ckey[TK_CAP];
     int32_t cpos[TK_CAP];
 };
@@ -179,6 +182,92 @@ __device__ void select_on_chip(TopkSmem &sm, uint32_t ncand, uint32_t b1, uint32
         [&](int64_t i) { return sm.cpos[i]; });
 }
 
+// Full 32-bit radix select over keys[0..n) in shared memory: the `rank`-th
+// largest key (*thr) and how many keys equal to it rank within the first
+// `rank` (*need).
+__device__ void radix_select_smem(TopkSmem &sm, const uint32_t *keys, uint32_t n, uint32_t rank,
+                                  uint32_t *thr, uint32_t *need)
+{
+    const int tid = threadIdx.x;
+    uint32_t prefix = 0, pmask = 0, remaining = rank;
+#pragma unroll 1
+    for (int pass = 0; pass < 3; ++pass) {
+        const int shift = pass == 0 ? 21 : (pass == 1 ? 10 : 0);
+        const int nb = pass == 2 ? 1024 : 2048;
+        const uint32_t bmask = (uint32_t)nb - 1u;
+        for (int i = tid; i < nb; i += TK_THREADS) sm.hist[i] = 0u;
+        __syncthreads();
+        for (uint32_t j = tid; j < n; j += TK_THREADS) {
+            const uint32_t key = keys[j];
+            if ((key & pmask) == prefix) atomicAdd(&sm.hist[(key >> shift) & bmask], 1u);
+        }
+        __syncthreads();
+        find_bin(sm, nb, remaining);
+        remaining -= sm.sh_above;
+        prefix |= sm.sh_bin << shift;
+        pmask |= bmask << shift;
+        __syncthreads();
+    }
+    *thr = prefix;
+    *need = remaining;
+}
+
+// Exact select among the candidates in shared memory (every key that could
+// be selected, in ascending position order), emitted in position order.
+__device__ void select_candidates(TopkSmem &sm, uint32_t ncand, int k, int32_t *out)
+{
+    uint32_t thr, need;
+    radix_select_smem(sm, sm.ckey, ncand, (uint32_t)k, &thr, &need);
+    emit_selected(
+        sm, ncand, thr, need, k, out,
+        [&](int64_t i0, uint32_t (&keys)[TK_ITEMS], uint32_t &valid) {
+            valid = 0;
+#pragma unroll
+            for (int i = 0; i < TK_ITEMS; ++i) {
+                keys[i] = 0;
+                if (i0 + i < (int64_t)ncand) { keys[i] = sm.ckey[i0 + i]; valid |= 1u << i; }
+            }
+        },
+        [&](int64_t i) { return sm.cpos[i]; });
+}
+
+// Ordered copy of every key of the row that passes `keep` into the candidate
+// buffer; returns the total count (entries past TK_CAP are counted, not
+// stored).  Each thread takes 8 consecutive positions per step (two 16-byte
+// loads), one block scan per 4K positions.
+template <class Keep>
+__device__ uint32_t collect_candidates(TopkSmem &sm, const float *row, int64_t n, bool vec, Keep keep)
+{
+    constexpr int G = 1;                                   // groups of TK_ITEMS per thread per step
+    const int tid = threadIdx.x;
+    uint32_t base = 0;
+    for (int64_t c0 = 0; c0 < n; c0 += (int64_t)TK_STEP * G) {
+        const int64_t s0 = c0 + (int64_t)tid * TK_ITEMS * G;
+        uint32_t keys[G][TK_ITEMS], valid[G];
+#pragma unroll
+        for (int q = 0; q < G; ++q) load8(row, n, s0 + q * TK_ITEMS, vec, keys[q], valid[q]);
+        uint32_t flags = 0, cnt = 0;
+#pragma unroll
+        for (int q = 0; q < G; ++q)
+#pragma unroll
+            for (int i = 0; i < TK_ITEMS; ++i)
+                if (((valid[q] >> i) & 1u) && keep(keys[q][i])) { flags |= 1u << (q * TK_ITEMS + i); ++cnt; }
+        uint32_t tot;
+        uint32_t off = base + block_excl_scan(cnt, sm.warp_buf, &tot);
+#pragma unroll
+        for (int q = 0; q < G; ++q)
+#pragma unroll
+            for (int i = 0; i < TK_ITEMS; ++i) {
+                if ((flags >> (q * TK_ITEMS + i)) & 1u) {
+                    if (off < TK_CAP) { sm.ckey[off] = keys[q][i]; sm.cpos[off] = (int32_t)(s0 + q * TK_ITEMS + i); }
+                    ++off;
+                }
+            }
+        base += tot;
+    }
+    return base;
+}
+
 // Radix select run over the whole row in global memory (candidates did not fit).
 __device__ void select_global(TopkSmem &sm, const float *row, int64_t n, bool vec, int k, int32_t *out)
 {
@@ -256,46 +345,46 @@ topk_rows_kernel(const float *__restrict__ scores, int64_t ld, int64_t row_begin
         return;
     }
     const bool vec = vec_ok != 0;
-    auto row_keys = [&](int64_t s, uint32_t (&keys)[TK_ITEMS], uint32_t &valid) {
-        load8(row, n, s, vec, keys, valid);
-    };
-
-    // ---- pass 1: histogram of the top 11 bits over the row ----
-    for (int i = tid; i < 2048; i += TK_THREADS) sm.hist[i] = 0u;
     if (tid == 0) { sm.sh_count = 0; sm.sh_overflow = 0; }
+
+    // ---- short rows: every key is a candidate ----
+    if (n <= TK_CAP) {
+        const uint32_t c = collect_candidates(sm, row, n, vec, [](uint32_t) { return true; });
+        select_candidates(sm, c, k, out);
+        return;
+    }
+
+    // ---- guess a threshold from evenly spaced samples: about 1.5 k keys of the
+    // row should lie at or above it; then one ordered pass collects them ----
+    {
+        for (int i = tid; i < TK_SAMPLE; i += TK_THREADS)
+            sm.sample[i] = float_key(row[(int64_t)i * n / TK_SAMPLE]);
+        __syncthreads();
+        const double want = 1.5 * (double)k * TK_SAMPLE / (double)n;
+        const uint32_t rank = (uint32_t)min((double)TK_SAMPLE, max(1.0, ceil(want)));
+        uint32_t tau, unused;
+        radix_select_smem(sm, sm.sample, TK_SAMPLE, rank, &tau, &unused);
+        const uint32_t c = collect_candidates(sm, row, n, vec, [tau](uint32_t key) { return key >= tau; });
+        if (c >= (uint32_t)k && c <= TK_CAP) {        // the selection lies among the candidates
+            select_candidates(sm, c, k, out);
+            return;
+        }
+    }
+
+    // ---- fallback: histogram of the top 11 bits, then the keys in or above the
+    // threshold bin on chip (or, if too many, the radix select in global memory) ----
+    for (int i = tid; i < 2048; i += TK_THREADS) sm.hist[i] = 0u;
     __syncthreads();
     for (int64_t c0 = 0; c0 < n; c0 += TK_STEP) {
         uint32_t keys[TK_ITEMS], valid;
-        row_keys(c0 + (int64_t)tid * TK_ITEMS, keys, valid);
+        load8(row, n, c0 + (int64_t)tid * TK_ITEMS, vec, keys, valid);
         hist_top11(sm.hist, keys, valid);
     }
     __syncthreads();
     find_bin(sm, 2048, (uint32_t)k);
     const uint32_t b1 = sm.sh_bin;
-    uint32_t remaining = (uint32_t)k - sm.sh_above;
-
-    // ---- pass 2: ordered copy of every key with top bits >= b1 ----
-    uint32_t base = 0;
-    for (int64_t c0 = 0; c0 < n; c0 += TK_STEP) {
-        const int64_t s0 = c0 + (int64_t)tid * TK_ITEMS;
-        uint32_t keys[TK_ITEMS], valid, flags = 0, cnt = 0;
-        row_keys(s0, keys, valid);
-#pragma unroll
-        for (int i = 0; i < TK_ITEMS; ++i)
-            if (((valid >> i) & 1u) && (keys[i] >> 21) >= b1) { flags |= 1u << i; ++cnt; }
-        uint32_t tot;
-        uint32_t off = base + block_excl_scan(cnt, sm.warp_buf, &tot);
-#pragma unroll
-        for (int i = 0; i < TK_ITEMS; ++i) {
-            if ((flags >> i) & 1u) {
-                if (off < TK_CAP) { sm.ckey[off] = keys[i]; sm.cpos[off] = (int32_t)(s0 + i); }
-                ++off;
-            }
-        }
-        base += tot;
-    }
-    const uint32_t ncand = base;
-
+    const uint32_t remaining = (uint32_t)k - sm.sh_above;
+    const uint32_t ncand = collect_candidates(sm, row, n, vec, [b1](uint32_t key) { return (key >> 21) >= b1; });
     if (ncand <= TK_CAP) select_on_chip(sm, ncand, b1, remaining, k, out);
     else select_global(sm, row, n, vec, k, out);
 }
