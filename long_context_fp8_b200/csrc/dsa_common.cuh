@@ -55,6 +55,12 @@ __device__ __forceinline__ void cp_async_16(void *smem, const void *gmem, bool v
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n"
                  :: "r"(smem_u32(smem)), "l"(gmem), "r"(n) : "memory");
 }
+// Arrive on `bar` (asynchronously) once every cp.async this thread issued so
+// far has completed; counts toward the barrier's expected arrivals.
+__device__ __forceinline__ void cp_async_arrive_noinc(uint64_t *bar)
+{
+    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];\n" :: "r"(smem_u32(bar)) : "memory");
+}
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
 template <int N>
 __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;\n" :: "n"(N) : "memory"); }

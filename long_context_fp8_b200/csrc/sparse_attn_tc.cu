@@ -42,7 +42,7 @@ constexpr int AT_BLK = 64;             // selected rows per block (UMMA N of S, 
 constexpr int AT_STAGES = 4;           // K/V gather ring depth
 constexpr int AT_THREADS = 224;        // 4 softmax warps, 2 producer warps, MMA warp
 constexpr int AT_PRODUCERS = 64;       // producer threads: one selected row each per block
-constexpr int AT_LAG = 2;              // blocks a producer keeps in flight before publishing
+
 constexpr int AT_QHALF = AT_HEADS * 128;     // one 64-column half of Q (16 KB)
 constexpr int AT_QTILE = 2 * AT_QHALF;       // Q of one item (32 KB)
 constexpr int AT_KHALF = AT_BLK * 128;       // one 64-column half of a 64-row K or V tile (8 KB)
@@ -161,7 +161,9 @@ sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_con
             mbar_init(&pfull[i], 4); mbar_init(&pempty[i], 1);
             mbar_init(&ofull[i], 1); mbar_init(&oempty[i], 4);
         }
-        for (int i = 0; i < AT_STAGES; ++i) { mbar_init(&kvfull[i], AT_PRODUCERS); mbar_init(&kvempty[i], 1); }
+        // kvfull: one asynchronous arrival per producer thread when its copies land,
+        // plus one ordinary arrival per producer warp publishing the validity bits
+        for (int i = 0; i < AT_STAGES; ++i) { mbar_init(&kvfull[i], AT_PRODUCERS + 2); mbar_init(&kvempty[i], 1); }
         abort_flag = 0;
         kv_issued = kv_consumed = q_issued = q_consumed = mma_blocks = 0;
         fence_mbar_init();
@@ -176,21 +178,15 @@ sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_con
         // ------------------------------------------------ producers (2 warps, one row per thread)
         // Thread p copies selected row p of each 64-row block (its K and V rows,
         // 16 x 16 bytes each) with cp.async into the 128-byte-swizzled tiles.
-        // Completion is published two blocks later: after cp.async.wait_group and
-        // a proxy fence (the tensor cores read through the async proxy), every
-        // producer arrives on the block's kvfull barrier.
+        // Each thread's copies signal the block's kvfull barrier asynchronously when
+        // they land (cp.async.mbarrier.arrive.noinc); the MMA issuer fences the
+        // generic-proxy writes for the tensor cores' async-proxy reads.
         const int pt = tid - 128;                     // 0..63: row of the block
         if (pt == 0) {
             tma_prefetch_desc(&qmap);
         }
-        int qi = 0, g = 0, published = 0;
+        int qi = 0, g = 0;
         bool stop = false;
-        auto publish = [&](int upto) {                // blocks [published, upto) have landed
-            for (; published < upto; ++published) {
-                fence_proxy_async_smem();
-                mbar_arrive(&kvfull[published % AT_STAGES]);
-            }
-        };
         for (int64_t it = it_begin; it < it_end && !stop; ++it) {
             Item item;
             item.set(a, it);
@@ -199,13 +195,6 @@ sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_con
             if (paged) {
                 ctx = a.context_lens[item.row];
                 if (ctx < 0 || (int64_t)ctx > (int64_t)a.max_pages * a.page_size) ctx = 0;
-            }
-            // The Q buffer of this item is freed by the last PV of item qi - 2, which
-            // may need blocks this thread copied but has not published yet: publish
-            // everything first (otherwise the wait below could never end).
-            if (qi >= 2 && published < g) {
-                cp_async_wait<0>();
-                publish(g);
             }
             if (pt == 0) {
                 const int qb = qi & 1;
@@ -257,7 +246,10 @@ sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_con
                     v = true;
                 }
                 const unsigned vw = __ballot_sync(0xffffffffu, v);
-                if (lane == 0) valid[st * 2 + (warp - 4)] = vw;
+                if (lane == 0) {
+                    valid[st * 2 + (warp - 4)] = vw;
+                    mbar_arrive(&kvfull[st]);          // releases the validity bits
+                }
                 uint8_t *tile = KVs + st * AT_STAGE + (is_v ? AT_KTILE : 0);
                 const uint16_t *base = is_v ? a.v : a.k;
                 const int coff = (chunk >> 3) * AT_KHALF;
@@ -269,15 +261,11 @@ sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_con
                     cp_async_16(tile + coff + j * 128 + (((chunk & 7) ^ (j & 7)) << 4),
                                 base + ri * AT_D + chunk * 8, vi);
                 }
-                cp_async_commit();
+                cp_async_arrive_noinc(&kvfull[st]);   // fires when this thread's copies land
                 if (pt == 0) kv_issued = g + 1;
-                // publish the block issued AT_LAG blocks ago
-                cp_async_wait<AT_LAG>();
-                publish(g + 1 - AT_LAG);
             }
         }
-        cp_async_wait<0>();
-        publish(stop ? published : g);
+        cp_async_wait<0>();                           // nothing in flight when the CTA retires
     } else if (warp == 6) {
         // ------------------------------------------------ MMA issuer: S(g), then PV(g - 1)
         if (lane == 0) {
@@ -323,6 +311,7 @@ sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_con
                     if (!wait_or_abort(&kvfull[st], (g / AT_STAGES) & 1, &abort_flag) ||
                         !wait_or_abort(&sempty[sb], ((g >> 1) & 1) ^ 1, &abort_flag)) { ok = false; break; }
                     kv_consumed = g + 1;
+                    fence_proxy_async_smem();         // cp.async wrote the tiles; the MMA reads them
                     tc_fence_after();
                     const uint32_t ka = smem_u32(KVs + st * AT_STAGE);
 #pragma unroll
