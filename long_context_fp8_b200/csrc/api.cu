@@ -266,8 +266,7 @@ dsa_status dsa_decode(const void *q_idx, const float *q_scale, const void *w, co
     if (e == cudaSuccess) {
         // tensor-core (tcgen05 + TMA) indexer where the shape allows, else mma.sync
         if (decode_index_tc_supported(H_I, page_size) && B <= 4096 &&
-            (int64_t)num_pages * page_size < ((int64_t)1 << 31) &&
-            (reinterpret_cast<uintptr_t>(kscale_cache) & 15u) == 0)
+            (int64_t)num_pages * page_size < ((int64_t)1 << 31) && aligned16(kscale_cache))
             e = launch_decode_index_tc((const uint8_t *)q_idx, q_scale, (const uint16_t *)w,
                                        (const uint8_t *)kidx_cache, kscale_cache, block_table,
                                        context_lens, num_pages, max_pages_per_seq, page_size, B,

@@ -12,12 +12,14 @@
 // epilogue thread owns one key (one TMEM lane), reads its H head products,
 // and folds them as sum_h c_h * ReLU(.) with c_h = w[h] * sq, then applies
 // the key's scale.  Persistent and warp-specialised: one CTA per SM takes a
-// contiguous share of the (sequence, tile) items; a producer warp keeps an
-// 8-stage TMA ring of key tiles in flight, one thread issues the MMAs into
-// two alternating TMEM accumulators, and four epilogue warps drain them, so
-// the HBM stream never waits on the epilogue.  Every mbarrier wait is
-// bounded; on a timeout every role stops, the CTA records DSA_ERR_TIMEOUT,
-// waits (bounded) for its copies in flight, frees its tensor memory and returns.
+// contiguous share of the (sequence, 256-key item) work; a producer warp
+// keeps a 4-stage TMA ring of items in flight, one thread issues each item's
+// two 128-key MMAs into one of two rotating TMEM accumulator pairs, and two
+// groups of four epilogue warps (one per 128-key half) drain them.  Items of
+// 256 keys halve the per-item hand-offs between the roles, which bound the
+// throughput at 128-key items.  Every mbarrier wait is bounded; on a
+// timeout every role stops, the CTA records DSA_ERR_TIMEOUT, waits (bounded)
+// for its copies in flight, frees its tensor memory and returns.
 #include <algorithm>
 
 #include "kernels.h"
@@ -28,13 +30,21 @@ namespace {
 
 using namespace sm100;
 
-constexpr int DT_STAGES = 8;
-constexpr int DT_TILE = 128;                 // keys per tile = UMMA M
+constexpr int DT_TILE = 128;                 // keys per UMMA tile = UMMA M
 constexpr int DT_TILE_BYTES = DT_TILE * 128;
-constexpr int DT_EPI_WARPS = 4;
+constexpr int DT_SUB = 2;                    // UMMA tiles per item
+constexpr int DT_ITEM = DT_TILE * DT_SUB;    // keys per item (one pipeline stage)
+constexpr int DT_STAGE_BYTES = DT_ITEM * 128;
+constexpr int DT_STAGES = 4;
+constexpr int DT_MAXSEG = DT_ITEM / 16;      // page segments per item (pages hold >= 16 keys)
+constexpr int DT_EPI_WARPS = 4 * DT_SUB;     // four warps (the 128 TMEM lanes) per UMMA tile
 constexpr int DT_THREADS = 32 * (2 + DT_EPI_WARPS);
-constexpr int DT_TMEM_COLS = 128;            // two 64-column accumulators
+constexpr int DT_ACC = 2;                    // item accumulators (DT_SUB x 64 columns each) in rotation
+constexpr int DT_TMEM_COLS = 64 * DT_SUB * DT_ACC;
 constexpr int DT_MAX_B = 4096;               // sequences the per-CTA item table can hold
+static_assert(DT_STAGE_BYTES % 1024 == 0, "stages keep the 1024-byte swizzle alignment");
+static_assert(DT_TMEM_COLS >= 32 && DT_TMEM_COLS <= 512 && (DT_TMEM_COLS & (DT_TMEM_COLS - 1)) == 0,
+              "tensor memory is allocated in powers of two columns");
 
 struct DecTcArgs {
     const float *sq;
@@ -55,11 +65,15 @@ struct DecTcArgs {
 
 constexpr size_t dt_smem_bytes()
 {
-    return 1024 /*align slack*/ + 2 * 8192 /*q, double-buffered*/ + (size_t)DT_STAGES * DT_TILE_BYTES +
-           (size_t)DT_STAGES * DT_TILE * 4 /*key scales*/ + DT_STAGES * 4 /*segment masks*/ +
-           2 * 64 * 4 /*c*/ + (2 * DT_STAGES + 8) * 8 + 16 +
+    return 1024 /*align slack*/ + 2 * 8192 /*q, double-buffered*/ + (size_t)DT_STAGES * DT_STAGE_BYTES +
+           (size_t)DT_STAGES * (DT_ITEM + 1) * 4 /*key scales, segment masks*/ +
+           64 * (DT_MAXSEG + 2) * 4 /*producer batches*/ +
+           2 * 64 * 4 /*c*/ + (2 * DT_STAGES + 4 + 2 * DT_ACC) * 8 + 16 +
            (size_t)(2 * DT_MAX_B + 1) * 4 /*per-sequence lengths and tile prefix*/;
 }
+static_assert(dt_smem_bytes() <= 232448 - 64, "dynamic shared memory per CTA");
+static_assert(((2 * DT_STAGES + 4 + 2 * DT_ACC) * 8 + 16) % 16 == 0,
+              "the key-scale stages (bulk-copy targets) start 16-byte aligned");
 
 // Context length of sequence b if valid, else 0 (the caller records the error).
 __device__ __forceinline__ int64_t seq_len(const DecTcArgs &a, int b)
@@ -70,7 +84,7 @@ __device__ __forceinline__ int64_t seq_len(const DecTcArgs &a, int b)
 }
 
 // Per-CTA table of the sequences' lengths and of the prefix sums of their
-// 128-key tiles (filled once from context_lens), so that locating an item is
+// 256-key items (filled once from context_lens), so that locating an item is
 // a binary search in shared memory.
 struct SeqTable {
     const int32_t *n;        // [B]
@@ -78,7 +92,8 @@ struct SeqTable {
     int B;
 };
 
-// Walks this CTA's contiguous share of the (sequence, 128-key tile) items.
+// Walks this CTA's contiguous share of the (sequence, 256-key item) work; `tile`
+// is the item's index within its sequence.
 struct ItemWalk {
     int b = 0;
     int64_t tile = 0, left = 0, n = 0;
@@ -132,17 +147,22 @@ decode_index_tc_kernel(const __grid_constant__ CUtensorMap kmap,
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *qs = smem;                                         // [2] x H x 128 B
-    uint8_t *ks = qs + 2 * 8192;                                // stages x 128 x 128 B
-    float *kss = reinterpret_cast<float *>(ks + DT_STAGES * DT_TILE_BYTES);  // [stages][128] key scales
-    uint32_t *kmask = reinterpret_cast<uint32_t *>(kss + DT_STAGES * DT_TILE); // [stages] loaded segments
-    float *cw = reinterpret_cast<float *>(kmask + DT_STAGES);                   // [2][64]
-    uint64_t *kfull = reinterpret_cast<uint64_t *>(cw + 128);
+    uint8_t *ks = qs + 2 * 8192;                                // stages x 256 x 128 B
+    // the mbarriers first: they follow a 1024-byte-aligned region, so they stay
+    // 8-byte aligned whatever the sizes of the 4-byte arrays after them
+    uint64_t *kfull = reinterpret_cast<uint64_t *>(ks + DT_STAGES * DT_STAGE_BYTES);
     uint64_t *kempty = kfull + DT_STAGES;
     uint64_t *qfull = kempty + DT_STAGES, *qempty = qfull + 2;
-    uint64_t *tfull = qempty + 2, *tempty = tfull + 2;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(tempty + 2);
-    int32_t *tab_n = reinterpret_cast<int32_t *>(tmem_slot + 4);     // [DT_MAX_B]
-    int32_t *tab_prefix = tab_n + DT_MAX_B;                            // [DT_MAX_B + 1]
+    uint64_t *tfull = qempty + 2, *tempty = tfull + DT_ACC;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(tempty + DT_ACC);
+    float *kss = reinterpret_cast<float *>(tmem_slot + 4);                         // [stages][ITEM] key scales
+    uint32_t *kmask = reinterpret_cast<uint32_t *>(kss + DT_STAGES * DT_ITEM);     // [stages] loaded segments
+    int32_t *pt_b = reinterpret_cast<int32_t *>(kmask + DT_STAGES);               // producer's batches: [2][32] sequences
+    uint32_t *pt_mask = reinterpret_cast<uint32_t *>(pt_b + 64);                   // [2][32] segment masks
+    int32_t *pt_slot = reinterpret_cast<int32_t *>(pt_mask + 64);                  // [2][32][MAXSEG] segment cache rows
+    float *cw = reinterpret_cast<float *>(pt_slot + 64 * DT_MAXSEG);               // [2][64]
+    int32_t *tab_n = reinterpret_cast<int32_t *>(cw + 128);                        // [DT_MAX_B]
+    int32_t *tab_prefix = tab_n + DT_MAX_B;                                         // [DT_MAX_B + 1]
     __shared__ volatile int abort_flag;
     __shared__ int k_issued, k_consumed, mma_items;
 
@@ -158,7 +178,7 @@ decode_index_tc_kernel(const __grid_constant__ CUtensorMap kmap,
             const int64_t n = seq_len(a, b);
             if (n == 0 && blockIdx.x == 0) record_error(a.hdr, DSA_ERR_INVALID_ARG, (unsigned)b);
             tab_n[b] = (int32_t)n;
-            local += (int32_t)((n + DT_TILE - 1) / DT_TILE);
+            local += (int32_t)((n + DT_ITEM - 1) / DT_ITEM);
         }
         int32_t incl = local;
 #pragma unroll
@@ -169,7 +189,7 @@ decode_index_tc_kernel(const __grid_constant__ CUtensorMap kmap,
         int32_t run = incl - local;
         for (int b = b0; b < b1; ++b) {
             tab_prefix[b] = run;
-            run += (tab_n[b] + DT_TILE - 1) / DT_TILE;
+            run += (tab_n[b] + DT_ITEM - 1) / DT_ITEM;
         }
         if (lane == 31) tab_prefix[a.B] = incl;
     }
@@ -186,12 +206,11 @@ decode_index_tc_kernel(const __grid_constant__ CUtensorMap kmap,
         tmem_relinquish();
     }
     if (tid == 0) {
-        // a stage is free once its MMA has completed and the epilogue warps have read its scales
+        // a stage is free once its MMAs have completed and every epilogue warp has
+        // read its key scales
         for (int s = 0; s < DT_STAGES; ++s) { mbar_init(&kfull[s], 1); mbar_init(&kempty[s], 1 + DT_EPI_WARPS); }
-        for (int i = 0; i < 2; ++i) {
-            mbar_init(&qfull[i], 1); mbar_init(&qempty[i], 1);
-            mbar_init(&tfull[i], 1); mbar_init(&tempty[i], DT_EPI_WARPS);
-        }
+        for (int i = 0; i < 2; ++i) { mbar_init(&qfull[i], 1); mbar_init(&qempty[i], 1); }
+        for (int i = 0; i < DT_ACC; ++i) { mbar_init(&tfull[i], 1); mbar_init(&tempty[i], DT_EPI_WARPS); }
         abort_flag = 0;
         k_issued = k_consumed = mma_items = 0;
         fence_mbar_init();
@@ -203,80 +222,94 @@ decode_index_tc_kernel(const __grid_constant__ CUtensorMap kmap,
 
     if (warp == 0) {
         // ------------------------------------------------ TMA producer (whole warp)
-        // The 32 lanes resolve the page ids of 32 consecutive items at once (one
-        // memory latency per 32 tiles); lane 0 then issues their copies in order.
+        // The 32 lanes resolve the page ids of the 32 items of a batch at once,
+        // one batch ahead, so that the block-table reads are in flight while the
+        // current batch is issued.  Per item, lane 0 claims the stage and lane g
+        // copies page segment g: its keys by tensor TMA, its scales by bulk copy.
         if (lane == 0) {
             tma_prefetch_desc(&kmap);
             tma_prefetch_desc(&qmap);
         }
-        const int nseg = DT_TILE / a.box_rows;           // <= 8 page segments per tile
+        const int nseg = DT_ITEM / a.box_rows;           // <= DT_MAXSEG page segments per item
         int seg = -1, prev_b = -1;
         bool stop = false;
-        for (int64_t j0 = 0; j0 < count && !stop; j0 += 32) {
-            // this lane's item j0 + lane
-            ItemWalk mine;
-            const bool have = j0 + lane < count && mine.start(tab, first + j0 + lane, count - j0 - lane);
-            int my_b = have ? mine.b : -1;
-            uint32_t my_mask = 0;
-            int my_slot[8];
+        ItemWalk mine;                                   // this lane's item of the batch being fetched
+        bool have = false;
+        int pgs[DT_MAXSEG];                              // its page ids, loads in flight
+        auto fetch = [&](int64_t j0) {
+            have = j0 + lane < count && mine.start(tab, first + j0 + lane, count - j0 - lane);
+            const int64_t p0 = mine.tile * DT_ITEM;
 #pragma unroll
-            for (int g = 0; g < 8; ++g) my_slot[g] = 0;
-            if (have) {
-                const int32_t *bt = a.block_table + (int64_t)mine.b * a.max_pages;
-                const int64_t p0 = mine.tile * DT_TILE;
+            for (int g = 0; g < DT_MAXSEG; ++g) {
+                const int64_t pos = p0 + (int64_t)g * a.box_rows;
+                pgs[g] = have && g < nseg && pos < mine.n
+                             ? __ldg(a.block_table + (int64_t)mine.b * a.max_pages + pos / ps) : -1;
+            }
+        };
+        auto publish = [&](int t) {                      // batch table t <- this lane's item
+            uint32_t m = 0;
+            const int64_t p0 = mine.tile * DT_ITEM;
 #pragma unroll
-                for (int g = 0; g < 8; ++g) {
-                    const int64_t pos = p0 + (int64_t)g * a.box_rows;
-                    if (g < nseg && pos < mine.n) {
-                        const int page = bt[pos / ps];
-                        if (page >= 0 && page < a.num_pages) {
-                            my_mask |= 1u << g;
-                            my_slot[g] = (int)((int64_t)page * ps + pos % ps);
-                        } else {
-                            record_error(a.hdr, DSA_ERR_INVALID_ARG, (unsigned)mine.b);
-                        }
+            for (int g = 0; g < DT_MAXSEG; ++g) {
+                const int64_t pos = p0 + (int64_t)g * a.box_rows;
+                int slot = 0;
+                if (have && g < nseg && pos < mine.n) {
+                    if (pgs[g] >= 0 && pgs[g] < a.num_pages) {
+                        m |= 1u << g;
+                        slot = (int)((int64_t)pgs[g] * ps + pos % ps);
+                    } else {
+                        record_error(a.hdr, DSA_ERR_INVALID_ARG, (unsigned)mine.b);
                     }
                 }
+                if (g < nseg) pt_slot[(t * 32 + lane) * DT_MAXSEG + g] = slot;
             }
+            pt_b[t * 32 + lane] = have ? mine.b : -1;
+            pt_mask[t * 32 + lane] = m;
+        };
+        fetch(0);
+        int t = 0;
+        for (int64_t j0 = 0; j0 < count && !stop; j0 += 32, t ^= 1) {
+            publish(t);
+            fetch(j0 + 32);
+            __syncwarp();
             const int nb = (int)min((int64_t)32, count - j0);
             for (int i = 0; i < nb; ++i) {
-                const int b = __shfl_sync(0xffffffffu, my_b, i);
-                const uint32_t mask = __shfl_sync(0xffffffffu, my_mask, i);
-                int slot[8];
-#pragma unroll
-                for (int g = 0; g < 8; ++g) slot[g] = __shfl_sync(0xffffffffu, my_slot[g], i);
+                const int64_t j = j0 + i;
+                const int s = (int)(j % DT_STAGES);
+                const uint32_t mask = pt_mask[t * 32 + i];
+                bool ok = true;
                 if (lane == 0) {
-                    const int64_t j = j0 + i;
+                    const int b = pt_b[t * 32 + i];
                     if (b != prev_b) {                       // a new sequence: its query heads
                         ++seg;
                         prev_b = b;
-                        if (!wait_or_abort(&qempty[seg & 1], ((seg >> 1) & 1) ^ 1, &abort_flag)) stop = true;
-                        else {
+                        ok = wait_or_abort(&qempty[seg & 1], ((seg >> 1) & 1) ^ 1, &abort_flag);
+                        if (ok) {
                             mbar_arrive_expect_tx(&qfull[seg & 1], H * 128);
                             tma_load_2d(qs + (seg & 1) * 8192, &qmap, &qfull[seg & 1], 0, b * H);
                         }
                     }
-                    const int s = (int)(j % DT_STAGES);
-                    if (!stop && !wait_or_abort(&kempty[s], (uint32_t)((j / DT_STAGES) & 1) ^ 1, &abort_flag))
-                        stop = true;
-                    if (!stop) {
+                    if (ok) ok = wait_or_abort(&kempty[s], (uint32_t)((j / DT_STAGES) & 1) ^ 1, &abort_flag);
+                    if (ok) {
                         kmask[s] = mask;                     // published by the arrive below
                         mbar_arrive_expect_tx(&kfull[s], (uint32_t)__popc(mask) * a.box_rows * (128 + 4));
-#pragma unroll
-                        for (int g = 0; g < 8; ++g) {
-                            if ((mask >> g) & 1u) {
-                                tma_load_2d(ks + s * DT_TILE_BYTES + g * a.box_rows * 128, &kmap, &kfull[s], 0,
-                                            slot[g]);
-                                bulk_load(kss + s * DT_TILE + g * a.box_rows, a.kscale + slot[g],
-                                          (uint32_t)a.box_rows * 4, &kfull[s]);
-                            }
-                        }
-                        k_issued = (int)j + 1;
                     }
                 }
-                stop = __shfl_sync(0xffffffffu, stop, 0);
-                if (stop) break;
+                // after lane 0's claim of the stage (the shuffle orders the warp behind it)
+                if (!__shfl_sync(0xffffffffu, ok, 0)) {
+                    stop = true;
+                    break;
+                }
+                __syncwarp();
+                if (lane < nseg && ((mask >> lane) & 1u)) {
+                    const int slot = pt_slot[(t * 32 + i) * DT_MAXSEG + lane];
+                    tma_load_2d(ks + s * DT_STAGE_BYTES + lane * a.box_rows * 128, &kmap, &kfull[s], 0, slot);
+                    bulk_load(kss + s * DT_ITEM + lane * a.box_rows, a.kscale + slot, (uint32_t)a.box_rows * 4,
+                              &kfull[s]);
+                }
+                if (lane == 0) k_issued = (int)j + 1;
             }
+            __syncwarp();                                    // batch table t is rewritten two batches on
         }
     } else if (warp == 1) {
         // ------------------------------------------------ MMA issuer
@@ -293,27 +326,33 @@ decode_index_tc_kernel(const __grid_constant__ CUtensorMap kmap,
                     if (!wait_or_abort(&qfull[seg & 1], (seg >> 1) & 1, &abort_flag)) break;
                     bdesc = umma_desc_k_sw128(smem_u32(qs + (seg & 1) * 8192));
                 }
-                const int s = j % DT_STAGES, acc = j & 1;
+                const int s = j % DT_STAGES, acc = j % DT_ACC;
                 if (!wait_or_abort(&kfull[s], (j / DT_STAGES) & 1, &abort_flag)) break;
                 k_consumed = j + 1;
-                if (!wait_or_abort(&tempty[acc], ((j >> 1) & 1) ^ 1, &abort_flag)) break;
+                if (!wait_or_abort(&tempty[acc], ((j / DT_ACC) & 1) ^ 1, &abort_flag)) break;
                 tc_fence_after();
-                const uint64_t adesc = umma_desc_k_sw128(smem_u32(ks + s * DT_TILE_BYTES));
-                const uint32_t d = tmem + (uint32_t)(acc * 64);
 #pragma unroll
-                for (int k = 0; k < 4; ++k) umma_f8f6f4(d, adesc + 2 * k, bdesc + 2 * k, idesc, k > 0);
+                for (int sub = 0; sub < DT_SUB; ++sub) {
+                    const uint64_t adesc = umma_desc_k_sw128(smem_u32(ks + s * DT_STAGE_BYTES + sub * DT_TILE_BYTES));
+                    const uint32_t d = tmem + (uint32_t)((acc * DT_SUB + sub) * 64);
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) umma_f8f6f4(d, adesc + 2 * k, bdesc + 2 * k, idesc, k > 0);
+                }
                 umma_commit(&kempty[s]);
                 umma_commit(&tfull[acc]);
                 mma_items = j + 1;
             }
         }
     } else {
-        // ------------------------------------------------ epilogue (4 warps, one key per thread)
+        // ------------------------------------------------ epilogue (4 warps per UMMA tile, one key per thread)
         const int q4 = warp & 3;                       // TMEM lane quarter
         const int et = tid - 64;
-        ItemWalk it;
+        const int sub = (warp - 2) >> 2;               // this warp's UMMA tile of every item
+        const int r = sub * DT_TILE + q4 * 32 + lane;   // this thread's key within every item
         int j = 0, seg = -1, prev_b = -1;
         bool dead = false;
+        uint64_t cpk[H / 2];                           // this sequence's c_h, packed in pairs
+        ItemWalk it;
         for (bool ok = it.start(tab, first, count); ok; ok = it.next(tab), ++j) {
             if (it.b != prev_b) {                       // per-sequence head weights c_h = w[b,h] * sq[b]
                 ++seg;
@@ -321,39 +360,45 @@ decode_index_tc_kernel(const __grid_constant__ CUtensorMap kmap,
                 epi_sync();
                 if (et < H) cw[(seg & 1) * 64 + et] = bf16_to_f32(a.w[(int64_t)it.b * H + et]) * a.sq[it.b];
                 epi_sync();
+#pragma unroll
+                for (int i = 0; i < H / 2; ++i) cpk[i] = f2_pack(cw[(seg & 1) * 64 + 2 * i], cw[(seg & 1) * 64 + 2 * i + 1]);
             }
             if (dead) continue;
-            // this thread's key (TMEM lane), its scale and whether its page was loaded
-            const int s = j % DT_STAGES, acc = j & 1;
-            const int r = q4 * 32 + lane;
-            const int64_t pos = it.tile * DT_TILE + r;
+            const int s = j % DT_STAGES, acc = j % DT_ACC;
+            const int64_t pos = it.tile * DT_ITEM + r;
+            // warp-uniform outcome: the TMEM loads below are warp-collective
+            if (!__all_sync(0xffffffffu, wait_or_abort(&tfull[acc], (j / DT_ACC) & 1, &abort_flag))) {
+                dead = true;
+                continue;
+            }
+            tc_fence_after();
+            // the stage's copies landed before its MMAs ran: this wait only orders the
+            // scale reads behind the copies
             if (!__all_sync(0xffffffffu, wait_or_abort(&kfull[s], (j / DT_STAGES) & 1, &abort_flag))) {
                 dead = true;
                 continue;
             }
             const bool live = pos < it.n && ((kmask[s] >> (r / a.box_rows)) & 1u);
-            const float ksc = kss[s * DT_TILE + r];
+            const float ksc = kss[s * DT_ITEM + r];
             __syncwarp();
             if (lane == 0) mbar_arrive(&kempty[s]);
-            // warp-uniform outcome: the TMEM loads below are warp-collective
-            if (!__all_sync(0xffffffffu, wait_or_abort(&tfull[acc], (j >> 1) & 1, &abort_flag))) {
-                dead = true;
-                continue;
-            }
-            tc_fence_after();
-            const uint32_t trow = tmem + ((uint32_t)(q4 * 32) << 16) + (uint32_t)(acc * 64);
-            const float *c = cw + (seg & 1) * 64;
-            uint64_t s2 = 0ull;
-            if constexpr (H % 32 == 0) {
+            const uint32_t trow = tmem + ((uint32_t)(q4 * 32) << 16) + (uint32_t)((acc * DT_SUB + sub) * 64);
+            // all of this key's H head products in one round trip, four independent sums
+            uint64_t s4[4] = {0ull, 0ull, 0ull, 0ull};
+            if constexpr (H == 64) {
+                uint32_t va[32], vb[32];
+                tmem_ld32(trow, va);
+                tmem_ld32(trow + 32, vb);
+                tmem_wait_ld_dep32(vb);
+                tmem_wait_ld_dep32(va);
 #pragma unroll
-                for (int c0 = 0; c0 < H; c0 += 32) {
-                    uint32_t v[32];
-                    tmem_ld32(trow + c0, v);
-                    tmem_wait_ld_dep32(v);
-#pragma unroll
-                    for (int i = 0; i < 32; i += 2)
-                        s2 = f2_fma(f2_pack(c[c0 + i], c[c0 + i + 1]),
-                                    f2_pack(fmaxf(__uint_as_float(v[i]), 0.f), fmaxf(__uint_as_float(v[i + 1]), 0.f)), s2);
+                for (int i = 0; i < 32; i += 2) {
+                    s4[(i >> 1) & 3] = f2_fma(cpk[i >> 1],
+                                              f2_pack(fmaxf(__uint_as_float(va[i]), 0.f), fmaxf(__uint_as_float(va[i + 1]), 0.f)),
+                                              s4[(i >> 1) & 3]);
+                    s4[(i >> 1) & 3] = f2_fma(cpk[16 + (i >> 1)],
+                                              f2_pack(fmaxf(__uint_as_float(vb[i]), 0.f), fmaxf(__uint_as_float(vb[i + 1]), 0.f)),
+                                              s4[(i >> 1) & 3]);
                 }
             } else {
 #pragma unroll
@@ -363,16 +408,21 @@ decode_index_tc_kernel(const __grid_constant__ CUtensorMap kmap,
                     tmem_wait_ld_dep16(v);
 #pragma unroll
                     for (int i = 0; i < 16; i += 2)
-                        s2 = f2_fma(f2_pack(c[c0 + i], c[c0 + i + 1]),
-                                    f2_pack(fmaxf(__uint_as_float(v[i]), 0.f), fmaxf(__uint_as_float(v[i + 1]), 0.f)), s2);
+                        s4[(i >> 1) & 3] = f2_fma(cpk[(c0 + i) >> 1],
+                                                  f2_pack(fmaxf(__uint_as_float(v[i]), 0.f), fmaxf(__uint_as_float(v[i + 1]), 0.f)),
+                                                  s4[(i >> 1) & 3]);
                 }
+            }
+            float lo, hi, acc_sum = 0.f;
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                f2_unpack(s4[q], lo, hi);
+                acc_sum += lo + hi;
             }
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&tempty[acc]);
-            float lo, hi;
-            f2_unpack(s2, lo, hi);
-            if (live) a.scores[(int64_t)it.b * a.ld + pos] = (lo + hi) * ksc;
+            if (live) a.scores[(int64_t)it.b * a.ld + pos] = acc_sum * ksc;
         }
     }
 
@@ -382,7 +432,7 @@ decode_index_tc_kernel(const __grid_constant__ CUtensorMap kmap,
         record_error(a.hdr, DSA_ERR_TIMEOUT, blockIdx.x);
         // let copies and MMAs still in flight land before shared and tensor memory go
         for (int j = k_consumed; j < k_issued; ++j) mbar_wait(&kfull[j % DT_STAGES], (j / DT_STAGES) & 1);
-        if (mma_items > 0) mbar_wait(&tfull[(mma_items - 1) & 1], ((mma_items - 1) >> 1) & 1);
+        if (mma_items > 0) mbar_wait(&tfull[(mma_items - 1) % DT_ACC], ((mma_items - 1) / DT_ACC) & 1);
     }
     __syncthreads();
     tc_fence_after();
@@ -423,7 +473,7 @@ cudaError_t launch_decode_index_tc(const uint8_t *q8, const float *sq, const uin
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    const int64_t max_items = (int64_t)B * ceil_div(max_context, DT_TILE);
+    const int64_t max_items = (int64_t)B * ceil_div(max_context, DT_ITEM);
     dim3 grid((unsigned)std::min<int64_t>(max_items, sms));
     const size_t smem = dt_smem_bytes();
     cudaError_t e;
