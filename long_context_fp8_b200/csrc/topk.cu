@@ -25,14 +25,15 @@ constexpr int TK_THREADS = 512;
 constexpr int TK_WARPS = TK_THREADS / 32;
 constexpr int TK_ITEMS = 8;                          // consecutive positions per thread per step
 constexpr int TK_STEP = TK_THREADS * TK_ITEMS;       // positions per block-wide step
-constexpr int TK_CAP = 12288;                        // shared-memory candidate capacity
+constexpr int TK_CAP = 8192;                         // shared-memory candidate capacity (two CTAs fit an SM)
 
 constexpr int TK_SAMPLE = 2048;                     // evenly spaced samples for the threshold guess
 
 struct TopkSmem {
     uint32_t hist[2048];
     uint32_t warp_buf[32];
-    uint32_t sh_bin, sh_above, sh_count, sh_overflow;
+    uint32_t sh_bin, sh_above, sh_count, sh_overflow, sh_diff;
+    uint32_t wcnt[TK_WARPS], wbefore[TK_WARPS + 1];
     uint32_t sample[TK_SAMPLE];
     uint32_t ckey[TK_CAP];
     int32_t cpos[TK_CAP];
@@ -66,24 +67,40 @@ __device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t *warp_b
     return before;
 }
 
+// Raw scores of positions [s, s + 8) of a row (0 past n).  Kept apart from
+// the key conversion so that a loop can issue the next step's loads before it
+// works on the current step's values.
+__device__ __forceinline__ void load_raw8(const float *row, int64_t n, int64_t s, bool vec, float (&v)[TK_ITEMS])
+{
+    if (vec && s + TK_ITEMS <= n) {
+        const float4 a = __ldg(reinterpret_cast<const float4 *>(row + s));
+        const float4 b = __ldg(reinterpret_cast<const float4 *>(row + s + 4));
+        v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+    } else {
+#pragma unroll
+        for (int i = 0; i < TK_ITEMS; ++i) v[i] = s + i < n ? row[s + i] : 0.f;
+    }
+}
+
+// Keys of raw scores of positions [s, s + 8) (bit i of *valid set when s + i < n).
+__device__ __forceinline__ void keys_of(const float (&v)[TK_ITEMS], int64_t n, int64_t s,
+                                        uint32_t (&key)[TK_ITEMS], uint32_t &valid)
+{
+    valid = 0;
+#pragma unroll
+    for (int i = 0; i < TK_ITEMS; ++i) {
+        key[i] = float_key(v[i]);
+        if (s + i < n) valid |= 1u << i;
+    }
+}
+
 // Keys of positions [s, s + 8) of a row (bit i of *valid set when s + i < n).
 __device__ __forceinline__ void load8(const float *row, int64_t n, int64_t s, bool vec,
                                       uint32_t (&key)[TK_ITEMS], uint32_t &valid)
 {
-    valid = 0;
-    if (vec && s + TK_ITEMS <= n) {
-        float4 a = __ldg(reinterpret_cast<const float4 *>(row + s));
-        float4 b = __ldg(reinterpret_cast<const float4 *>(row + s + 4));
-        key[0] = float_key(a.x); key[1] = float_key(a.y); key[2] = float_key(a.z); key[3] = float_key(a.w);
-        key[4] = float_key(b.x); key[5] = float_key(b.y); key[6] = float_key(b.z); key[7] = float_key(b.w);
-        valid = 0xffu;
-    } else {
-#pragma unroll
-        for (int i = 0; i < TK_ITEMS; ++i) {
-            key[i] = 0;
-            if (s + i < n) { key[i] = float_key(row[s + i]); valid |= 1u << i; }
-        }
-    }
+    float v[TK_ITEMS];
+    load_raw8(row, n, s, vec, v);
+    keys_of(v, n, s, key, valid);
 }
 
 // Bin holding the `remaining`-th largest count (from the top), and how many
@@ -91,13 +108,17 @@ __device__ __forceinline__ void load8(const float *row, int64_t n, int64_t s, bo
 __device__ __forceinline__ void find_bin(TopkSmem &sm, int nb, uint32_t remaining)
 {
     const int tid = threadIdx.x;
-    const int bpt = nb / TK_THREADS;
+    const int bpt = nb > TK_THREADS ? nb / TK_THREADS : 1;     // nb: a power of two
     uint32_t local = 0;
-    for (int j = 0; j < bpt; ++j) local += sm.hist[nb - 1 - (tid * bpt + j)];
+    for (int j = 0; j < bpt; ++j) {
+        const int b = nb - 1 - (tid * bpt + j);
+        if (b >= 0) local += sm.hist[b];
+    }
     uint32_t tot;
     uint32_t cum = block_excl_scan(local, sm.warp_buf, &tot);
     for (int j = 0; j < bpt; ++j) {
-        int b = nb - 1 - (tid * bpt + j);
+        const int b = nb - 1 - (tid * bpt + j);
+        if (b < 0) break;
         uint32_t c = sm.hist[b];
         if (cum < remaining && remaining <= cum + c) { sm.sh_bin = (uint32_t)b; sm.sh_above = cum; }
         cum += c;
@@ -146,7 +167,7 @@ __device__ __forceinline__ void emit_selected(TopkSmem &sm, int64_t n, uint32_t 
 // Given the candidates (every key whose top 11 bits are >= b1, in ascending
 // position order) in shared memory, resolve the remaining 21 bits of the
 // threshold on chip and emit the selection in position order.
-__device__ void select_on_chip(TopkSmem &sm, uint32_t ncand, uint32_t b1, uint32_t remaining, int k,
+__device__ __noinline__ void select_on_chip(TopkSmem &sm, uint32_t ncand, uint32_t b1, uint32_t remaining, int k,
                                int32_t *out)
 {
     const int tid = threadIdx.x;
@@ -182,18 +203,40 @@ __device__ void select_on_chip(TopkSmem &sm, uint32_t ncand, uint32_t b1, uint32
         [&](int64_t i) { return sm.cpos[i]; });
 }
 
-// Full 32-bit radix select over keys[0..n) in shared memory: the `rank`-th
+// Radix select over keys[0..n) in shared memory (n >= 1): the `rank`-th
 // largest key (*thr) and how many keys equal to it rank within the first
-// `rank` (*need).
+// `rank` (*need).  The digits start below the bits that all keys share (found
+// by an OR-reduction of key ^ keys[0]), so that the first histogram spreads
+// over the keys' actual range instead of piling onto one bin of the top bits.
+// With passes = 3 the result is exact; with fewer, the bits not yet resolved
+// are zero in *thr (a threshold at or below the exact key).
 __device__ void radix_select_smem(TopkSmem &sm, const uint32_t *keys, uint32_t n, uint32_t rank,
-                                  uint32_t *thr, uint32_t *need)
+                                  uint32_t *thr, uint32_t *need, int passes = 3)
 {
     const int tid = threadIdx.x;
-    uint32_t prefix = 0, pmask = 0, remaining = rank;
+    const uint32_t first = keys[0];
+    if (tid == 0) sm.sh_diff = 0u;
+    __syncthreads();
+    uint32_t diff = 0;
+    for (uint32_t j = tid; j < n; j += TK_THREADS) diff |= keys[j] ^ first;
+    diff = __reduce_or_sync(0xffffffffu, diff);
+    if ((tid & 31) == 0 && diff) atomicOr(&sm.sh_diff, diff);
+    __syncthreads();
+    diff = sm.sh_diff;
+    uint32_t remaining = rank;
+    if (diff == 0u) {                                     // every key equal
+        *thr = first;
+        *need = remaining;
+        return;
+    }
+    int lo = 32 - __clz(diff);                            // bits [0, lo) still to resolve
+    uint32_t pmask = lo == 32 ? 0u : ~((1u << lo) - 1u);
+    uint32_t prefix = first & pmask;
 #pragma unroll 1
-    for (int pass = 0; pass < 3; ++pass) {
-        const int shift = pass == 0 ? 21 : (pass == 1 ? 10 : 0);
-        const int nb = pass == 2 ? 1024 : 2048;
+    for (int pass = 0; pass < passes && lo > 0; ++pass) {
+        const int width = lo < 11 ? lo : 11;
+        const int shift = lo - width;
+        const int nb = 1 << width;
         const uint32_t bmask = (uint32_t)nb - 1u;
         for (int i = tid; i < nb; i += TK_THREADS) sm.hist[i] = 0u;
         __syncthreads();
@@ -206,6 +249,7 @@ __device__ void radix_select_smem(TopkSmem &sm, const uint32_t *keys, uint32_t n
         remaining -= sm.sh_above;
         prefix |= sm.sh_bin << shift;
         pmask |= bmask << shift;
+        lo = shift;
         __syncthreads();
     }
     *thr = prefix;
@@ -238,38 +282,149 @@ __device__ void select_candidates(TopkSmem &sm, uint32_t ncand, int k, int32_t *
 template <class Keep>
 __device__ uint32_t collect_candidates(TopkSmem &sm, const float *row, int64_t n, bool vec, Keep keep)
 {
-    constexpr int G = 1;                                   // groups of TK_ITEMS per thread per step
+    constexpr int D = 2;                                   // steps of loads in flight
     const int tid = threadIdx.x;
     uint32_t base = 0;
-    for (int64_t c0 = 0; c0 < n; c0 += (int64_t)TK_STEP * G) {
-        const int64_t s0 = c0 + (int64_t)tid * TK_ITEMS * G;
-        uint32_t keys[G][TK_ITEMS], valid[G];
+    float ring[D][TK_ITEMS];
 #pragma unroll
-        for (int q = 0; q < G; ++q) load8(row, n, s0 + q * TK_ITEMS, vec, keys[q], valid[q]);
-        uint32_t flags = 0, cnt = 0;
+    for (int q = 0; q < D; ++q)
+        if ((int64_t)q * TK_STEP < n) load_raw8(row, n, (int64_t)q * TK_STEP + (int64_t)tid * TK_ITEMS, vec, ring[q]);
+    for (int64_t c0 = 0; c0 < n; c0 += (int64_t)D * TK_STEP) {
 #pragma unroll
-        for (int q = 0; q < G; ++q)
+        for (int q = 0; q < D; ++q) {
+            const int64_t cq = c0 + (int64_t)q * TK_STEP;
+            if (cq >= n) break;                            // block-uniform
+            const int64_t s0 = cq + (int64_t)tid * TK_ITEMS;
+            uint32_t keys[TK_ITEMS], valid;
+            keys_of(ring[q], n, s0, keys, valid);
+            if (cq + (int64_t)D * TK_STEP < n) load_raw8(row, n, s0 + (int64_t)D * TK_STEP, vec, ring[q]);
+            uint32_t flags = 0, cnt = 0;
 #pragma unroll
             for (int i = 0; i < TK_ITEMS; ++i)
-                if (((valid[q] >> i) & 1u) && keep(keys[q][i])) { flags |= 1u << (q * TK_ITEMS + i); ++cnt; }
-        uint32_t tot;
-        uint32_t off = base + block_excl_scan(cnt, sm.warp_buf, &tot);
-#pragma unroll
-        for (int q = 0; q < G; ++q)
+                if (((valid >> i) & 1u) && keep(keys[i])) { flags |= 1u << i; ++cnt; }
+            uint32_t tot;
+            uint32_t off = base + block_excl_scan(cnt, sm.warp_buf, &tot);
 #pragma unroll
             for (int i = 0; i < TK_ITEMS; ++i) {
-                if ((flags >> (q * TK_ITEMS + i)) & 1u) {
-                    if (off < TK_CAP) { sm.ckey[off] = keys[q][i]; sm.cpos[off] = (int32_t)(s0 + q * TK_ITEMS + i); }
+                if ((flags >> i) & 1u) {
+                    if (off < TK_CAP) { sm.ckey[off] = keys[i]; sm.cpos[off] = (int32_t)(s0 + i); }
                     ++off;
                 }
             }
-        base += tot;
+            base += tot;
+        }
     }
     return base;
 }
 
+// Float of an order-preserving key (the inverse of float_key on non-negative
+// zero): x >= key_float(t) exactly when float_key(x) >= t, for every non-NaN x.
+__device__ __forceinline__ float key_float(uint32_t key)
+{
+    return __uint_as_float((key & 0x80000000u) ? (key & 0x7fffffffu) : ~key);
+}
+
+constexpr int TK_WCAP = TK_CAP / TK_WARPS;          // candidate slots per warp
+
+// Candidates x >= tau_f of the row, in ascending position order, into
+// sm.ckey / sm.cpos[0, count).  Each warp scans its own contiguous chunk of
+// the row (four steps of 256 scores in flight, warp-level ordered
+// compaction, no block barrier) into its own TK_WCAP slots; one barrier, then
+// the warps' lists are packed in warp order.  Returns the count, or
+// 0xffffffff if a warp's chunk held more than TK_WCAP candidates (the caller
+// falls back).
+__device__ uint32_t collect_above_warp(TopkSmem &sm, const float *row, int64_t n, bool vec, float tau_f)
+{
+    constexpr int D = 4;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int64_t per = ((n + TK_WARPS - 1) / TK_WARPS + 255) / 256 * 256;
+    const int64_t w0 = (int64_t)warp * per, w1 = min(n, w0 + per);
+    uint32_t *wk = sm.ckey + warp * TK_WCAP;
+    int32_t *wp = sm.cpos + warp * TK_WCAP;
+    uint32_t cnt = 0;                                      // warp-uniform
+    float ring[D][TK_ITEMS];
+#pragma unroll
+    for (int q = 0; q < D; ++q)
+        if (w0 + q * 256 < w1) load_raw8(row, w1, w0 + q * 256 + lane * TK_ITEMS, vec, ring[q]);
+    for (int64_t c0 = w0; c0 < w1; c0 += D * 256) {
+#pragma unroll
+        for (int q = 0; q < D; ++q) {
+            const int64_t cq = c0 + q * 256;
+            if (cq >= w1) break;                           // warp-uniform
+            const int64_t s0 = cq + lane * TK_ITEMS;
+            float v[TK_ITEMS];
+#pragma unroll
+            for (int i = 0; i < TK_ITEMS; ++i) v[i] = ring[q][i];
+            if (cq + D * 256 < w1) load_raw8(row, w1, s0 + D * 256, vec, ring[q]);
+            uint32_t flags = 0;
+#pragma unroll
+            for (int i = 0; i < TK_ITEMS; ++i)
+                if (s0 + i < w1 && v[i] >= tau_f) flags |= 1u << i;
+            const uint32_t c = (uint32_t)__popc(flags);
+            uint32_t x = c;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
+                if (lane >= o) x += y;
+            }
+            uint32_t off = cnt + x - c;
+            while (flags) {
+                const int i = __ffs(flags) - 1;
+                flags &= flags - 1;
+                if (off < TK_WCAP) { wk[off] = float_key(v[i]); wp[off] = (int32_t)(s0 + i); }
+                ++off;
+            }
+            cnt += __shfl_sync(0xffffffffu, x, 31);
+        }
+    }
+    if (lane == 0) sm.wcnt[warp] = cnt;
+    __syncthreads();
+    if (warp == 0) {                                       // exclusive prefix of the warps' counts
+        const uint32_t c = lane < TK_WARPS ? sm.wcnt[lane] : 0u;
+        uint32_t x = c;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
+            if (lane >= o) x += y;
+        }
+        const bool over = __any_sync(0xffffffffu, c > TK_WCAP);
+        if (lane <= TK_WARPS) sm.wbefore[lane] = over ? 0xffffffffu : x - c;
+    }
+    __syncthreads();
+    const uint32_t total = sm.wbefore[TK_WARPS];
+    if (total == 0xffffffffu) return total;                // a warp overflowed (block-uniform)
+    // Pack in rounds of TK_THREADS * 4 entries in increasing order: an entry only
+    // moves down, so a round's targets never hold a later round's sources; each
+    // round reads all its sources before it writes.
+    for (uint32_t r0 = 0; r0 < total; r0 += TK_THREADS * 4) {
+        uint32_t kk[4];
+        int32_t pp[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const uint32_t i = r0 + tid + q * TK_THREADS;
+            if (i < total) {
+                int w = 0;                                 // last warp with wbefore[w] <= i
+#pragma unroll
+                for (int step = TK_WARPS / 2; step > 0; step >>= 1)
+                    if (sm.wbefore[w + step] <= i) w += step;
+                const uint32_t src = w * TK_WCAP + (i - sm.wbefore[w]);
+                kk[q] = sm.ckey[src];
+                pp[q] = sm.cpos[src];
+            }
+        }
+        __syncthreads();
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const uint32_t i = r0 + tid + q * TK_THREADS;
+            if (i < total) { sm.ckey[i] = kk[q]; sm.cpos[i] = pp[q]; }
+        }
+        __syncthreads();
+    }
+    return total;
+}
+
 // Radix select run over the whole row in global memory (candidates did not fit).
-__device__ void select_global(TopkSmem &sm, const float *row, int64_t n, bool vec, int k, int32_t *out)
+__device__ __noinline__ void select_global(TopkSmem &sm, const float *row, int64_t n, bool vec, int k, int32_t *out)
 {
     const int tid = threadIdx.x;
     auto row_keys = [&](int64_t s, uint32_t (&keys)[TK_ITEMS], uint32_t &valid) {
@@ -317,7 +472,7 @@ __device__ __forceinline__ void hist_top11(uint32_t *hist, const uint32_t (&keys
     }
 }
 
-__global__ void __launch_bounds__(TK_THREADS)
+__global__ void __launch_bounds__(TK_THREADS, 2)
 topk_rows_kernel(const float *__restrict__ scores, int64_t ld, int64_t row_begin,
                  const int32_t *__restrict__ lens, int64_t max_len, int k,
                  int32_t *__restrict__ idx, WsHeader *hdr, int vec_ok)
@@ -357,14 +512,18 @@ topk_rows_kernel(const float *__restrict__ scores, int64_t ld, int64_t row_begin
     // ---- guess a threshold from evenly spaced samples: about 1.5 k keys of the
     // row should lie at or above it; then one ordered pass collects them ----
     {
-        for (int i = tid; i < TK_SAMPLE; i += TK_THREADS)
-            sm.sample[i] = float_key(row[(int64_t)i * n / TK_SAMPLE]);
+        float sv[TK_SAMPLE / TK_THREADS];                 // all loads issued before any is used
+#pragma unroll
+        for (int q = 0; q < TK_SAMPLE / TK_THREADS; ++q)
+            sv[q] = __ldg(row + (int64_t)(tid + q * TK_THREADS) * n / TK_SAMPLE);
+#pragma unroll
+        for (int q = 0; q < TK_SAMPLE / TK_THREADS; ++q) sm.sample[tid + q * TK_THREADS] = float_key(sv[q]);
         __syncthreads();
         const double want = 1.5 * (double)k * TK_SAMPLE / (double)n;
         const uint32_t rank = (uint32_t)min((double)TK_SAMPLE, max(1.0, ceil(want)));
         uint32_t tau, unused;
-        radix_select_smem(sm, sm.sample, TK_SAMPLE, rank, &tau, &unused);
-        const uint32_t c = collect_candidates(sm, row, n, vec, [tau](uint32_t key) { return key >= tau; });
+        radix_select_smem(sm, sm.sample, TK_SAMPLE, rank, &tau, &unused, 2);
+        const uint32_t c = collect_above_warp(sm, row, n, vec, key_float(tau));
         if (c >= (uint32_t)k && c <= TK_CAP) {        // the selection lies among the candidates
             select_candidates(sm, c, k, out);
             return;

@@ -234,7 +234,8 @@ def decode_reference_attention(inp, idx, sm):
                                            ((300,) * 9, 64, 32, 32),
                                            ((1500, 129, 640), 100, 16, 128),
                                            ((700, 300), 64, 16, 256),
-                                           ((900, 17), 64, 16, 48)])      # 48: mma.sync indexer
+                                           ((900, 17), 64, 16, 48),       # 48: mma.sync indexer
+                                           ((3000, 1000, 5000) * 6, 256, 16, 64)])   # 18 rows: one CTA per row
 def test_decode_end_to_end(lens, k, H_q, ps):
     spec = small_decode_spec(lens, k, H_q, seed=len(lens) + k, ps=ps)
     inp = dsa_synth.make_decode(spec)
