@@ -367,10 +367,13 @@ cudaError_t launch_sparse_attn_bf16(const uint16_t *q, const uint16_t *k, const 
     return cudaGetLastError();
 }
 
+// Index-list splits per decode sequence: as many as keep B x splits items
+// within one wave of the B200's 148 SMs (a second, partial wave of items cost
+// more than the smaller merge it saves).
 int sparse_attn_paged_splits(int B, int ksel)
 {
     int max_splits = (ksel + AT_BK - 1) / AT_BK;
-    int want = (2 * 148 + B - 1) / B;
+    int want = 148 / B;
     int s = want < max_splits ? want : max_splits;
     return s < 1 ? 1 : s;
 }

@@ -15,10 +15,13 @@
 //             tiles of a 4-stage ring (many small loads in flight per SM: the
 //             rows are scattered); one thread also brings the next item's Q
 //             with TMA into a second Q buffer;
-//   warp 6    MMA issuer: S = Q K^T (kind::f16, M 128 heads, N 64 rows,
-//             K = 128 = 8 x 16) into one of two TMEM buffers, then
-//             O += P V of the previous block (V read MN-major straight from
-//             the gathered rows) into one of two TMEM O buffers (per item);
+//   warp 6    S issuer: S = Q K^T (kind::f16, M 128 heads, N 64 rows,
+//             K = 128 = 8 x 16) into one of two TMEM buffers, as soon as the
+//             K tile is in and the softmax has read that buffer's last S;
+//   warp 7    PV issuer: O += P V (V read MN-major straight from the gathered
+//             rows) into one of two TMEM O buffers (per item), as soon as P
+//             is written.  Two issuing threads keep the S MMAs from queueing
+//             behind the PV MMAs, which wait for the softmax;
 //   warps 0-3 softmax: thread = head row.  Reads its S row from TMEM, masks
 //             unused slots, keeps the running max m and sum l in registers,
 //             writes P (bf16) to one of two shared buffers for the PV MMA.  O is rescaled
@@ -40,8 +43,16 @@ constexpr int AT_HEADS = 128;          // UMMA M: query heads per item
 constexpr int AT_D = 128;              // head dim
 constexpr int AT_BLK = 64;             // selected rows per block (UMMA N of S, K of PV)
 constexpr int AT_STAGES = 4;           // K/V gather ring depth
-constexpr int AT_THREADS = 224;        // 4 softmax warps, 2 producer warps, MMA warp
+constexpr int AT_THREADS = 384;        // 2 x 4 softmax warps, 2 producer warps, S and PV issuer warps
 constexpr int AT_PRODUCERS = 64;       // producer threads: one selected row each per block
+// Register split by warpgroup: producers and issuers (warps 4-7) give theirs to
+// the two softmax sets (warps 0-3 and 8-11).  The split adds up to the launch's
+// total only for a kernel built with exactly AT_LAUNCH_REGS per thread (checked
+// before every launch).
+constexpr int AT_LAUNCH_REGS = 168;
+constexpr int AT_REGS_LOW = 96;
+constexpr int AT_REGS_HIGH = 200;
+static_assert(128 * AT_REGS_LOW + 256 * AT_REGS_HIGH <= AT_LAUNCH_REGS * 384, "register split");
 
 constexpr int AT_QHALF = AT_HEADS * 128;     // one 64-column half of Q (16 KB)
 constexpr int AT_QTILE = 2 * AT_QHALF;       // Q of one item (32 KB)
@@ -81,8 +92,9 @@ struct AtSmem {
     static constexpr size_t kv_off = q_off + 2 * AT_QTILE;                // [stages] K, V tiles
     static constexpr size_t p_off = kv_off + (size_t)AT_STAGES * AT_STAGE; // [2] P tiles
     static constexpr size_t valid_off = p_off + 2 * AT_PTILE;            // [stages][2] validity bits
-    static constexpr size_t bar_off = valid_off + AT_STAGES * 2 * 4;
-    // qfull[2] qempty[2] kvfull[S] kvempty[S] sfull[2] sempty[2] pfull[2] pempty[2] ofull[2] oempty[2]
+    static constexpr size_t ml_off = valid_off + AT_STAGES * 2 * 4;      // set 1's (m, l) per head
+    static constexpr size_t bar_off = ml_off + 2 * AT_HEADS * 4;
+    // qfull[2] qempty[2] kvfull[S] kvempty[S] sfull[2] sempty[2] pfull[2] pempty[2] ofull oempty mlfull mlempty
     static constexpr int n_bars = 2 * AT_STAGES + 16;
     static constexpr size_t slot_off = bar_off + 8 * n_bars;
     static constexpr size_t total = slot_off + 16 + 1024;
@@ -100,6 +112,15 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t *bar, uint32_t parity, vo
             return false;
         }
     }
+}
+
+// 2^x by the SFU's approximate base-2 exponential (results below 2^-126 flush
+// to zero; P is rounded to bf16 right after, so neither matters).
+__device__ __forceinline__ float ex2_sfu(float x)
+{
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
 }
 
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi)
@@ -138,10 +159,11 @@ sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_con
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + AtSmem::bar_off);
     uint64_t *qfull = bars, *qempty = bars + 2, *kvfull = bars + 4, *kvempty = kvfull + AT_STAGES;
     uint64_t *sfull = kvempty + AT_STAGES, *sempty = sfull + 2, *pfull = sempty + 2, *pempty = pfull + 2;
-    uint64_t *ofull = pempty + 2, *oempty = ofull + 2;
+    uint64_t *ofull = pempty + 2, *oempty = ofull + 1, *mlfull = oempty + 1, *mlempty = mlfull + 1;
+    float *mls = reinterpret_cast<float *>(smem + AtSmem::ml_off);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + AtSmem::slot_off);
     __shared__ volatile int abort_flag;
-    __shared__ int kv_issued, kv_consumed, q_issued, q_consumed, mma_blocks;
+    __shared__ int kv_issued, kv_consumed, q_issued, q_consumed, pv_last, s_last;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int64_t per = (a.items + gridDim.x - 1) / gridDim.x;
@@ -157,15 +179,16 @@ sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_con
     if (tid == 0) {
         for (int i = 0; i < 2; ++i) {
             mbar_init(&qfull[i], 1); mbar_init(&qempty[i], 1);
-            mbar_init(&sfull[i], 1); mbar_init(&sempty[i], 4);
+            mbar_init(&sfull[i], 1); mbar_init(&sempty[i], 4);   // [x]: the 4 warps of softmax set x
             mbar_init(&pfull[i], 4); mbar_init(&pempty[i], 1);
-            mbar_init(&ofull[i], 1); mbar_init(&oempty[i], 4);
         }
+        mbar_init(ofull, 1); mbar_init(oempty, 4);                // oempty: set 0 read O_0 and O_1
+        mbar_init(mlfull, 4); mbar_init(mlempty, 4);              // set 1 -> set 0 hand-off of (m, l)
         // kvfull: one asynchronous arrival per producer thread when its copies land,
         // plus one ordinary arrival per producer warp publishing the validity bits
         for (int i = 0; i < AT_STAGES; ++i) { mbar_init(&kvfull[i], AT_PRODUCERS + 2); mbar_init(&kvempty[i], 1); }
         abort_flag = 0;
-        kv_issued = kv_consumed = q_issued = q_consumed = mma_blocks = 0;
+        kv_issued = kv_consumed = q_issued = q_consumed = pv_last = s_last = 0;
         fence_mbar_init();
     }
     tc_fence_before();
@@ -174,239 +197,289 @@ sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_con
     const uint32_t tmem = *tmem_slot;
     const uint32_t tS = tmem, tO = tmem + 2 * AT_BLK;    // S [0,128), O [128,384)
 
-    if (warp == 4 || warp == 5) {
-        // ------------------------------------------------ producers (2 warps, one row per thread)
-        // Thread p copies selected row p of each 64-row block (its K and V rows,
-        // 16 x 16 bytes each) with cp.async into the 128-byte-swizzled tiles.
-        // Each thread's copies signal the block's kvfull barrier asynchronously when
-        // they land (cp.async.mbarrier.arrive.noinc); the MMA issuer fences the
-        // generic-proxy writes for the tensor cores' async-proxy reads.
-        const int pt = tid - 128;                     // 0..63: row of the block
-        if (pt == 0) {
-            tma_prefetch_desc(&qmap);
-        }
-        int qi = 0, g = 0;
-        bool stop = false;
-        for (int64_t it = it_begin; it < it_end && !stop; ++it) {
-            Item item;
-            item.set(a, it);
-            if (item.nblk == 0) continue;
-            int ctx = 0;
-            if (paged) {
-                ctx = a.context_lens[item.row];
-                if (ctx < 0 || (int64_t)ctx > (int64_t)a.max_pages * a.page_size) ctx = 0;
-            }
+    if (warp >= 4 && warp < 8) {
+        regs_dec<AT_REGS_LOW>();
+        if (warp == 4 || warp == 5) {
+            // ------------------------------------------------ producers (2 warps, one row per thread)
+            // Thread p copies selected row p of each 64-row block (its K and V rows,
+            // 16 x 16 bytes each) with cp.async into the 128-byte-swizzled tiles.
+            // Each thread's copies signal the block's kvfull barrier asynchronously when
+            // they land (cp.async.mbarrier.arrive.noinc); the MMA issuer fences the
+            // generic-proxy writes for the tensor cores' async-proxy reads.
+            const int pt = tid - 128;                     // 0..63: row of the block
             if (pt == 0) {
-                const int qb = qi & 1;
-                if (!wait_or_abort(&qempty[qb], ((qi >> 1) & 1) ^ 1, &abort_flag)) stop = true;
-                else {
-                    mbar_arrive_expect_tx(&qfull[qb], AT_QTILE);
-                    const int qrow = (int)(item.row * a.H + item.hg * AT_HEADS);
-                    tma_load_2d(Qs + qb * AT_QTILE, &qmap, &qfull[qb], 0, qrow);
-                    tma_load_2d(Qs + qb * AT_QTILE + AT_QHALF, &qmap, &qfull[qb], 64, qrow);
-                    q_issued = qi + 1;
-                }
+                tma_prefetch_desc(&qmap);
             }
-            stop = __shfl_sync(0xffffffffu, stop, 0) || __any_sync(0xffffffffu, stop);
-            if (warp == 5) stop = stop || abort_flag;
-            ++qi;
-            const int32_t *irow = a.idx + item.row * a.ksel;
-            // warp (w - 4) copies rows 32 (w - 4) .. +31 of each block; lane l copies
-            // 16-byte chunk l % 16 of the row's K (l < 16) or V (l >= 16), so one
-            // instruction moves one whole row pair (two 256-byte runs).  Lane l also
-            // resolves row 32 (w - 4) + l of the block, broadcast by shuffles.
-            const int rbase = (warp - 4) * 32;
-            int e = item.e0 + rbase + lane;
-            int p_next = e < item.e1 ? __ldg(irow + e) : -1;
-            const int chunk = lane & 15;
-            const bool is_v = lane >= 16;
-            for (int b = 0; b < item.nblk && !stop; ++b, ++g) {
-                const int st = g % AT_STAGES;
-                const int p = p_next;
-                e += AT_BLK;                          // prefetch the next block's index
-                p_next = (b + 1 < item.nblk && e < item.e1) ? __ldg(irow + e) : -1;
-                // warp-uniform outcome: the ballot and shuffles below need every lane
-                const bool ok = __all_sync(0xffffffffu,
-                                           wait_or_abort(&kvempty[st], ((g / AT_STAGES) & 1) ^ 1, &abort_flag));
-                if (!ok) { stop = true; break; }
-                int64_t r = 0;
-                bool v = false;
-                if (paged) {
-                    if (p >= 0 && p < ctx) {
-                        const int page = a.block_table[item.row * a.max_pages + p / a.page_size];
-                        if (page >= 0 && page < a.num_pages) {
-                            r = (int64_t)page * a.page_size + p % a.page_size;
-                            v = true;
-                        } else {
-                            record_error(a.hdr, DSA_ERR_INVALID_ARG, (unsigned)item.row);
-                        }
-                    }
-                } else if (p >= 0 && p < a.T) {
-                    r = p;
-                    v = true;
-                }
-                const unsigned vw = __ballot_sync(0xffffffffu, v);
-                if (lane == 0) {
-                    valid[st * 2 + (warp - 4)] = vw;
-                    mbar_arrive(&kvfull[st]);          // releases the validity bits
-                }
-                uint8_t *tile = KVs + st * AT_STAGE + (is_v ? AT_KTILE : 0);
-                const uint16_t *base = is_v ? a.v : a.k;
-                const int coff = (chunk >> 3) * AT_KHALF;
-#pragma unroll 4
-                for (int i = 0; i < 32; ++i) {
-                    const int j = rbase + i;          // row of the block
-                    const int64_t ri = __shfl_sync(0xffffffffu, r, i);
-                    const bool vi = (vw >> i) & 1u;
-                    cp_async_16(tile + coff + j * 128 + (((chunk & 7) ^ (j & 7)) << 4),
-                                base + ri * AT_D + chunk * 8, vi);
-                }
-                cp_async_arrive_noinc(&kvfull[st]);   // fires when this thread's copies land
-                if (pt == 0) kv_issued = g + 1;
-            }
-        }
-        cp_async_wait<0>();                           // nothing in flight when the CTA retires
-    } else if (warp == 6) {
-        // ------------------------------------------------ MMA issuer: S(g), then PV(g - 1)
-        if (lane == 0) {
-            constexpr uint32_t idesc_s = umma_idesc_bf16_f32(AT_HEADS, AT_BLK, false);
-            constexpr uint32_t idesc_o = umma_idesc_bf16_f32(AT_HEADS, AT_D, true);
-            // the pending PV: block gp of the item with Q/O buffer slot qp, first/last flags
-            int gp = -1, qp = 0;
-            bool p_first = false, p_last = false;
-            auto issue_pv = [&]() -> bool {
-                const int st = gp % AT_STAGES, pb = gp & 1, ob = qp & 1;
-                if (!wait_or_abort(&pfull[pb], (gp >> 1) & 1, &abort_flag)) return false;
-                if (p_first && !wait_or_abort(&oempty[ob], ((qp >> 1) & 1) ^ 1, &abort_flag)) return false;
-                tc_fence_after();
-                const uint32_t pa = smem_u32(Ps + pb * AT_PTILE);
-                const uint32_t va = smem_u32(KVs + st * AT_STAGE + AT_KTILE);
-#pragma unroll
-                for (int kk = 0; kk < AT_BLK / 16; ++kk) {
-                    const uint64_t ad = umma_desc_k_sw128_sbo(pa + kk * 32, 1024);
-                    const uint64_t bd = umma_desc_mn_sw128(va + kk * 2048, AT_KHALF, 1024);
-                    umma_f16(tO + ob * AT_D, ad, bd, idesc_o, (!p_first || kk > 0) ? 1u : 0u);
-                }
-                umma_commit(&kvempty[st]);
-                umma_commit(&pempty[pb]);
-                if (p_last) {
-                    umma_commit(&ofull[ob]);
-                    umma_commit(&qempty[ob]);
-                }
-                mma_blocks = gp + 1;
-                return true;
-            };
             int qi = 0, g = 0;
-            bool ok = true;
-            for (int64_t it = it_begin; it < it_end && ok; ++it) {
+            bool stop = false;
+            for (int64_t it = it_begin; it < it_end && !stop; ++it) {
                 Item item;
                 item.set(a, it);
                 if (item.nblk == 0) continue;
-                const int qb = qi & 1;
-                if (!wait_or_abort(&qfull[qb], (qi >> 1) & 1, &abort_flag)) { ok = false; break; }
-                q_consumed = qi + 1;
-                const uint32_t qa = smem_u32(Qs + qb * AT_QTILE);
-                for (int b = 0; b < item.nblk; ++b, ++g) {
-                    const int st = g % AT_STAGES, sb = g & 1;
-                    if (!wait_or_abort(&kvfull[st], (g / AT_STAGES) & 1, &abort_flag) ||
-                        !wait_or_abort(&sempty[sb], ((g >> 1) & 1) ^ 1, &abort_flag)) { ok = false; break; }
-                    kv_consumed = g + 1;
-                    fence_proxy_async_smem();         // cp.async wrote the tiles; the MMA reads them
-                    tc_fence_after();
-                    const uint32_t ka = smem_u32(KVs + st * AT_STAGE);
-#pragma unroll
-                    for (int kk = 0; kk < AT_D / 16; ++kk) {
-                        umma_f16(tS + sb * AT_BLK,
-                                 umma_desc_k_sw128_sbo(qa + (kk >> 2) * AT_QHALF + (kk & 3) * 32, 1024),
-                                 umma_desc_k_sw128_sbo(ka + (kk >> 2) * AT_KHALF + (kk & 3) * 32, 1024),
-                                 idesc_s, kk > 0 ? 1u : 0u);
-                    }
-                    umma_commit(&sfull[sb]);
-                    if (gp >= 0 && !issue_pv()) { ok = false; break; }
-                    gp = g; qp = qi; p_first = b == 0; p_last = b == item.nblk - 1;
+                int ctx = 0;
+                if (paged) {
+                    ctx = a.context_lens[item.row];
+                    if (ctx < 0 || (int64_t)ctx > (int64_t)a.max_pages * a.page_size) ctx = 0;
                 }
+                if (pt == 0) {
+                    const int qb = qi & 1;
+                    if (!wait_or_abort(&qempty[qb], ((qi >> 1) & 1) ^ 1, &abort_flag)) stop = true;
+                    else {
+                        mbar_arrive_expect_tx(&qfull[qb], AT_QTILE);
+                        const int qrow = (int)(item.row * a.H + item.hg * AT_HEADS);
+                        tma_load_2d(Qs + qb * AT_QTILE, &qmap, &qfull[qb], 0, qrow);
+                        tma_load_2d(Qs + qb * AT_QTILE + AT_QHALF, &qmap, &qfull[qb], 64, qrow);
+                        q_issued = qi + 1;
+                    }
+                }
+                stop = __shfl_sync(0xffffffffu, stop, 0) || __any_sync(0xffffffffu, stop);
+                if (warp == 5) stop = stop || abort_flag;
                 ++qi;
+                const int32_t *irow = a.idx + item.row * a.ksel;
+                // warp (w - 4) copies rows 32 (w - 4) .. +31 of each block; lane l copies
+                // 16-byte chunk l % 16 of the row's K (l < 16) or V (l >= 16), so one
+                // instruction moves one whole row pair (two 256-byte runs).  Lane l also
+                // resolves row 32 (w - 4) + l of the block, broadcast by shuffles.
+                const int rbase = (warp - 4) * 32;
+                const int32_t *brow = paged ? a.block_table + item.row * a.max_pages : nullptr;
+                // Lane l's selected position in blocks b + 1 and b + 2 and, for the
+                // paged caches, the page id of block b + 1: the index and block-table
+                // reads run ahead of the copies, so their latency is not paid per block.
+                int e = item.e0 + rbase + lane;
+                int p1 = e < item.e1 ? __ldg(irow + e) : -1;
+                int pg1 = paged && p1 >= 0 && p1 < ctx ? __ldg(brow + p1 / a.page_size) : -1;
+                e += AT_BLK;
+                int p2 = (1 < item.nblk && e < item.e1) ? __ldg(irow + e) : -1;
+                const int chunk = lane & 15;
+                const bool is_v = lane >= 16;
+                for (int b = 0; b < item.nblk && !stop; ++b, ++g) {
+                    const int st = g % AT_STAGES;
+                    const int p = p1, pg = pg1;
+                    p1 = p2;
+                    pg1 = paged && p1 >= 0 && p1 < ctx ? __ldg(brow + p1 / a.page_size) : -1;
+                    e += AT_BLK;
+                    p2 = (b + 2 < item.nblk && e < item.e1) ? __ldg(irow + e) : -1;
+                    // warp-uniform outcome: the ballot and shuffles below need every lane
+                    const bool ok = __all_sync(0xffffffffu,
+                                               wait_or_abort(&kvempty[st], ((g / AT_STAGES) & 1) ^ 1, &abort_flag));
+                    if (!ok) { stop = true; break; }
+                    int r = 0;                            // K/V row (kv_rows < 2^31)
+                    bool v = false;
+                    if (paged) {
+                        if (p >= 0 && p < ctx) {
+                            if (pg >= 0 && pg < a.num_pages) {
+                                r = pg * a.page_size + p % a.page_size;
+                                v = true;
+                            } else {
+                                record_error(a.hdr, DSA_ERR_INVALID_ARG, (unsigned)item.row);
+                            }
+                        }
+                    } else if (p >= 0 && p < a.T) {
+                        r = p;
+                        v = true;
+                    }
+                    const unsigned vw = __ballot_sync(0xffffffffu, v);
+                    if (lane == 0) {
+                        valid[st * 2 + (warp - 4)] = vw;
+                        mbar_arrive(&kvfull[st]);          // releases the validity bits
+                    }
+                    uint8_t *tile = KVs + st * AT_STAGE + (is_v ? AT_KTILE : 0) + (chunk >> 3) * AT_KHALF + rbase * 128;
+                    const uint16_t *base = (is_v ? a.v : a.k) + chunk * 8;
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) {        // row rbase + i of the block (rbase % 8 == 0)
+                        const int ri = __shfl_sync(0xffffffffu, r, i);
+                        cp_async_16(tile + i * 128 + (((chunk ^ i) & 7) << 4), base + (int64_t)ri * AT_D, (vw >> i) & 1u);
+                    }
+                    cp_async_arrive_noinc(&kvfull[st]);   // fires when this thread's copies land
+                    if (pt == 0) kv_issued = g + 1;
+                }
             }
-            if (ok && gp >= 0) issue_pv();
+            cp_async_wait<0>();                           // nothing in flight when the CTA retires
+        } else if (warp == 6) {
+            // ------------------------------------------------ S issuer: S(b) = Q K(b)^T
+            // Block b of an item belongs to softmax set b % 2 and its S buffer; S(b)
+            // waits only for its K tile and for that set to have read its last S.
+            if (lane == 0) {
+                constexpr uint32_t idesc_s = umma_idesc_bf16_f32(AT_HEADS, AT_BLK, false);
+                int qi = 0, g = 0, cnt[2] = {0, 0};
+                bool ok = true;
+                for (int64_t it = it_begin; it < it_end && ok; ++it) {
+                    Item item;
+                    item.set(a, it);
+                    if (item.nblk == 0) continue;
+                    const int qb = qi & 1;
+                    if (!wait_or_abort(&qfull[qb], (qi >> 1) & 1, &abort_flag)) { ok = false; break; }
+                    q_consumed = qi + 1;
+                    const uint32_t qa = smem_u32(Qs + qb * AT_QTILE);
+                    for (int b = 0; b < item.nblk; ++b, ++g) {
+                        const int st = g % AT_STAGES, x = b & 1, k = cnt[x]++;
+                        if (!wait_or_abort(&kvfull[st], (g / AT_STAGES) & 1, &abort_flag) ||
+                            !wait_or_abort(&sempty[x], (k & 1) ^ 1, &abort_flag)) { ok = false; break; }
+                        kv_consumed = g + 1;
+                        fence_proxy_async_smem();         // cp.async wrote the tiles; the MMA reads them
+                        tc_fence_after();
+                        const uint32_t ka = smem_u32(KVs + st * AT_STAGE);
+#pragma unroll
+                        for (int kk = 0; kk < AT_D / 16; ++kk) {
+                            umma_f16(tS + x * AT_BLK,
+                                     umma_desc_k_sw128_sbo(qa + (kk >> 2) * AT_QHALF + (kk & 3) * 32, 1024),
+                                     umma_desc_k_sw128_sbo(ka + (kk >> 2) * AT_KHALF + (kk & 3) * 32, 1024),
+                                     idesc_s, kk > 0 ? 1u : 0u);
+                        }
+                        umma_commit(&sfull[x]);
+                        s_last = x | ((k & 1) << 1) | 4;
+                    }
+                    if (ok) umma_commit(&qempty[qb]);     // Q is read by this item's S MMAs only
+                    ++qi;
+                }
+            }
+        } else {
+            // ------------------------------------------------ PV issuer: O_x += P(b) V(b), x = b % 2
+            if (lane == 0) {
+                constexpr uint32_t idesc_o = umma_idesc_bf16_f32(AT_HEADS, AT_D, true);
+                int qi = 0, g = 0, cnt[2] = {0, 0};
+                bool ok = true;
+                for (int64_t it = it_begin; it < it_end && ok; ++it) {
+                    Item item;
+                    item.set(a, it);
+                    if (item.nblk == 0) continue;
+                    for (int b = 0; b < item.nblk; ++b, ++g) {
+                        const int st = g % AT_STAGES, x = b & 1, k = cnt[x]++;
+                        // kvfull (long complete) orders this thread's V reads behind the copies;
+                        // oempty: the previous item's O_0 and O_1 have been read
+                        if (!wait_or_abort(&pfull[x], k & 1, &abort_flag) ||
+                            !wait_or_abort(&kvfull[st], (g / AT_STAGES) & 1, &abort_flag) ||
+                            (b == 0 && !wait_or_abort(oempty, (qi & 1) ^ 1, &abort_flag))) {
+                            ok = false;
+                            break;
+                        }
+                        fence_proxy_async_smem();
+                        tc_fence_after();
+                        const uint32_t pa = smem_u32(Ps + x * AT_PTILE);
+                        const uint32_t va = smem_u32(KVs + st * AT_STAGE + AT_KTILE);
+#pragma unroll
+                        for (int kk = 0; kk < AT_BLK / 16; ++kk) {
+                            const uint64_t ad = umma_desc_k_sw128_sbo(pa + kk * 32, 1024);
+                            const uint64_t bd = umma_desc_mn_sw128(va + kk * 2048, AT_KHALF, 1024);
+                            umma_f16(tO + x * AT_D, ad, bd, idesc_o, (b > 1 || kk > 0) ? 1u : 0u);
+                        }
+                        umma_commit(&kvempty[st]);        // S(b) completed before P(b) existed
+                        umma_commit(&pempty[x]);
+                        if (b == item.nblk - 1) umma_commit(ofull);
+                        pv_last = x | ((k & 1) << 1) | 4;
+                    }
+                    ++qi;
+                }
+            }
         }
     } else {
-        // ------------------------------------------------ softmax (thread = head row)
-        const int h = warp * 32 + lane;
-        const uint32_t trow = (uint32_t)(warp * 32) << 16;
-        int qi = 0, g = 0;
+        regs_inc<AT_REGS_HIGH>();
+        // ------------------------------------------------ softmax sets (thread = head row)
+        // Set x (warps 0-3: x = 0; warps 8-11: x = 1) takes blocks b = x, x + 2, ...
+        // of every item, with its own S, P and O buffers and its own running max m
+        // and sum l; two sets keep two softmax warps on every SM sub-partition, so
+        // one's TMEM and memory latencies hide behind the other's arithmetic.  At
+        // the end of an item set 1 hands (m, l) to set 0, which merges O_0 and O_1:
+        //   O = (2^(m0 - m) O_0 + 2^(m1 - m) O_1) / (2^(m0 - m) l0 + 2^(m1 - m) l1).
+        const int x = warp >> 3;
+        const int q4 = warp & 3;
+        const int h = q4 * 32 + lane;
+        const uint32_t trow = (uint32_t)(q4 * 32) << 16;
+        const uint32_t tSx = tS + x * AT_BLK, tOx = tO + x * AT_D;
+        uint8_t *Px = Ps + x * AT_PTILE;
+        int qi = 0, g = 0, k = 0, mi = 0;   // items, blocks before this item, this set's blocks, merged items
         bool dead = false;
         for (int64_t it = it_begin; it < it_end; ++it) {
             Item item;
             item.set(a, it);
             float m = -INFINITY, l = 0.f;
-            const int ob = qi & 1;
-            bool have = item.nblk > 0;
-            for (int b = 0; b < item.nblk && !dead; ++b, ++g) {
-                const int st = g % AT_STAGES, sb = g & 1;
-                // kvfull: acquire the producer's validity bits; sfull: S of block g is in TMEM.
+            for (int b = x; b < item.nblk && !dead; b += 2, ++k) {
+                const int gb = g + b, st = gb % AT_STAGES;
+                // kvfull: acquire the producer's validity bits; sfull: S of block b is in TMEM.
                 // Outcomes are made warp-uniform: the TMEM accesses below are warp-collective.
-                bool ok = wait_or_abort(&kvfull[st], (g / AT_STAGES) & 1, &abort_flag) &&
-                          wait_or_abort(&sfull[sb], (g >> 1) & 1, &abort_flag);
+                bool ok = wait_or_abort(&kvfull[st], (gb / AT_STAGES) & 1, &abort_flag) &&
+                          wait_or_abort(&sfull[x], k & 1, &abort_flag);
                 if (!__all_sync(0xffffffffu, ok)) { dead = true; break; }
                 tc_fence_after();
-                float sv[AT_BLK];
+                // both halves of the S row in one TMEM round trip
+                uint32_t va[32], vb[32];
+                tmem_ld32(tSx + trow, va);
+                tmem_ld32(tSx + trow + 32, vb);
+                tmem_wait_ld_dep32(va);
+                tmem_wait_ld_dep32(vb);
+                float sv[AT_BLK];                     // raw q.k; unused slots -inf
 #pragma unroll
-                for (int c = 0; c < AT_BLK / 32; ++c) {
-                    uint32_t v[32];
-                    tmem_ld32(tS + trow + sb * AT_BLK + c * 32, v);
-                    tmem_wait_ld_dep32(v);
-                    const uint32_t vw = valid[st * 2 + c];
-#pragma unroll
-                    for (int i = 0; i < 32; ++i)
-                        sv[c * 32 + i] = ((vw >> i) & 1u) ? __uint_as_float(v[i]) * a.scale_log2 : -INFINITY;
-                }
+                for (int i = 0; i < 32; ++i) { sv[i] = __uint_as_float(va[i]); sv[32 + i] = __uint_as_float(vb[i]); }
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&sempty[sb]);
-                float mb = -INFINITY;
+                if (lane == 0) mbar_arrive(&sempty[x]);
+                const uint32_t vw0 = valid[st * 2], vw1 = valid[st * 2 + 1];
+                if ((vw0 & vw1) != 0xffffffffu) {     // block-uniform: only blocks with unused slots mask
 #pragma unroll
-                for (int i = 0; i < AT_BLK; ++i) mb = fmaxf(mb, sv[i]);
+                    for (int i = 0; i < 32; ++i) {
+                        if (!((vw0 >> i) & 1u)) sv[i] = -INFINITY;
+                        if (!((vw1 >> i) & 1u)) sv[32 + i] = -INFINITY;
+                    }
+                }
+                float mx[8];                          // eight independent max chains
+#pragma unroll
+                for (int i = 0; i < 8; ++i) mx[i] = sv[i];
+#pragma unroll
+                for (int i = 8; i < AT_BLK; ++i) mx[i & 7] = fmaxf(mx[i & 7], sv[i]);
+                const float mr = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                                       fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+                const float mb = mr * a.scale_log2;   // the scale is positive: max commutes with it
                 float m_new = m, alpha = 1.f;
                 if (mb > m + kRescaleThreshold || (m == -INFINITY && mb != -INFINITY)) {
                     m_new = mb;
                     alpha = m == -INFINITY ? 0.f : exp2f(m - m_new);
                 }
                 const float base = m_new == -INFINITY ? 0.f : m_new;
-                float rs = 0.f;
+                // p = 2^(s * scale - base): one packed FMA per pair for the exponent,
+                // four packed partial sums
+                const uint64_t sc2 = f2_pack(a.scale_log2, a.scale_log2), nb2 = f2_pack(-base, -base);
+                const uint64_t one2 = f2_pack(1.f, 1.f);
+                uint64_t rs2[4] = {0ull, 0ull, 0ull, 0ull};
                 uint32_t pk[AT_BLK / 2];
 #pragma unroll
                 for (int i = 0; i < AT_BLK / 2; ++i) {
-                    const float p0 = exp2f(sv[2 * i] - base), p1 = exp2f(sv[2 * i + 1] - base);
-                    rs += p0 + p1;
+                    float x0, x1;
+                    f2_unpack(f2_fma(f2_pack(sv[2 * i], sv[2 * i + 1]), sc2, nb2), x0, x1);
+                    const float p0 = ex2_sfu(x0), p1 = ex2_sfu(x1);
+                    rs2[i & 3] = f2_fma(f2_pack(p0, p1), one2, rs2[i & 3]);
                     pk[i] = pack_bf16(p0, p1);
                 }
-                l = l * alpha + rs;
+                float rsum = 0.f;
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    float lo, hi;
+                    f2_unpack(rs2[q], lo, hi);
+                    rsum += lo + hi;
+                }
+                l = l * alpha + rsum;
                 m = m_new;
-                // P buffer sb is free once PV(g - 2) has completed
-                ok = wait_or_abort(&pempty[sb], ((g >> 1) & 1) ^ 1, &abort_flag);
+                // P_x is free and O_x up to date once this set's previous PV has completed
+                ok = wait_or_abort(&pempty[x], (k & 1) ^ 1, &abort_flag);
                 if (!__all_sync(0xffffffffu, ok)) { dead = true; break; }
-                // Rescale O rows whose max moved (needs PV(g - 1) done).  tcgen05.ld/st are
-                // warp-collective: the whole warp takes the branch if any of its rows needs
-                // it, the others multiply by 1.
-                const bool need = b > 0 && alpha != 1.f;
+                // Rescale O_x rows whose max moved.  tcgen05.ld/st are warp-collective: the
+                // whole warp takes the branch if any of its rows needs it, the others multiply by 1.
+                const bool need = b > x && alpha != 1.f;
                 if (__any_sync(0xffffffffu, need)) {
-                    ok = wait_or_abort(&pempty[(g - 1) & 1], ((g - 1) >> 1) & 1, &abort_flag);
-                    if (!__all_sync(0xffffffffu, ok)) { dead = true; break; }
                     const float f = need ? alpha : 1.f;
                     tc_fence_after();
 #pragma unroll
                     for (int c = 0; c < AT_D / 32; ++c) {
                         uint32_t v[32];
-                        tmem_ld32(tO + trow + ob * AT_D + c * 32, v);
+                        tmem_ld32(tOx + trow + c * 32, v);
                         tmem_wait_ld_dep32(v);
 #pragma unroll
                         for (int i = 0; i < 32; ++i) v[i] = __float_as_uint(__uint_as_float(v[i]) * f);
-                        tmem_st32(tO + trow + ob * AT_D + c * 32, v);
+                        tmem_st32(tOx + trow + c * 32, v);
                     }
                     tmem_wait_st();
                 }
                 // P row h: 64 keys = 128 bytes, 16-byte chunks swizzled by h % 8
-                uint8_t *prow = Ps + sb * AT_PTILE + h * 128;
+                uint8_t *prow = Px + h * 128;
 #pragma unroll
                 for (int c = 0; c < 8; ++c)
                     *reinterpret_cast<uint4 *>(prow + ((c ^ (h & 7)) << 4)) =
@@ -414,57 +487,101 @@ sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_con
                 fence_proxy_async_smem();
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&pfull[sb]);
+                if (lane == 0) mbar_arrive(&pfull[x]);
             }
-            // ---- item epilogue: O / l and the log-sum-exp ----
-            float o[AT_D];
+            g += item.nblk;
+            if (item.nblk == 0 && x == 1) continue;
+            const bool two = item.nblk >= 2;
+            if (x == 1) {
+                // ---- set 1: hand its running max and sum to set 0 ----
+                if (two) {
+                    bool ok = !dead && wait_or_abort(mlempty, (mi & 1) ^ 1, &abort_flag);
+                    if (__all_sync(0xffffffffu, ok)) {
+                        mls[h] = m;
+                        mls[AT_HEADS + h] = l;
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(mlfull);
+                    } else {
+                        dead = true;
+                    }
+                    ++mi;
+                }
+                continue;
+            }
+            // ---- set 0: merge the two sets, O / l and the log-sum-exp ----
+            bool have = item.nblk > 0;
+            float m1 = -INFINITY, l1 = 0.f;
+            if (two) {
+                bool ok = !dead && wait_or_abort(mlfull, mi & 1, &abort_flag);
+                if (__all_sync(0xffffffffu, ok)) {
+                    m1 = mls[h];
+                    l1 = mls[AT_HEADS + h];
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(mlempty);
+                } else {
+                    dead = true;
+                }
+                ++mi;
+            }
             if (have) {
-                bool ok = !dead && wait_or_abort(&ofull[ob], (qi >> 1) & 1, &abort_flag);
+                bool ok = !dead && wait_or_abort(ofull, qi & 1, &abort_flag);
                 have = __all_sync(0xffffffffu, ok);
                 dead = dead || !have;
             }
-            if (have) {
-                tc_fence_after();
+            const float mt = fmaxf(m, m1);
+            const float f0 = (have && m != -INFINITY) ? exp2f(m - mt) : 0.f;
+            const float f1 = (have && m1 != -INFINITY) ? exp2f(m1 - mt) : 0.f;
+            const float lt = l * f0 + l1 * f1;
+            const float inv = lt > 0.f ? 1.f / lt : 0.f;
+            const float lse = lt > 0.f ? mt * kLn2 + logf(lt) : -INFINITY;
+            const float g0 = f0 * inv, g1 = f1 * inv;
+            const int64_t hh = (int64_t)item.hg * AT_HEADS + h;
+            if (have) tc_fence_after();
 #pragma unroll
-                for (int c = 0; c < AT_D / 32; ++c) {
-                    uint32_t v[32];
-                    tmem_ld32(tO + trow + ob * AT_D + c * 32, v);
-                    tmem_wait_ld_dep32(v);
+            for (int c = 0; c < AT_D / 32; ++c) {
+                float o[32];
+                if (have) {
+                    uint32_t v0[32], v1[32];
+                    tmem_ld32(tO + trow + c * 32, v0);
+                    if (two) tmem_ld32(tO + AT_D + trow + c * 32, v1);
+                    tmem_wait_ld_dep32(v0);
+                    if (two) {
+                        tmem_wait_ld_dep32(v1);
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) o[c * 32 + i] = __uint_as_float(v[i]);
+                        for (int i = 0; i < 32; ++i) o[i] = __uint_as_float(v0[i]) * g0 + __uint_as_float(v1[i]) * g1;
+                    } else {
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) o[i] = __uint_as_float(v0[i]) * g0;
+                    }
+                } else {
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) o[i] = 0.f;
                 }
+                if (a.splits == 1) {
+                    uint16_t *orow = a.out + (item.row * a.H + hh) * AT_D + c * 32;
+#pragma unroll
+                    for (int u = 0; u < 4; ++u)
+                        *reinterpret_cast<uint4 *>(orow + u * 8) =
+                            make_uint4(pack_bf16(o[u * 8], o[u * 8 + 1]), pack_bf16(o[u * 8 + 2], o[u * 8 + 3]),
+                                       pack_bf16(o[u * 8 + 4], o[u * 8 + 5]), pack_bf16(o[u * 8 + 6], o[u * 8 + 7]));
+                } else {
+                    float *po = a.part + ((item.row * a.splits + item.split) * a.H + hh) * (int64_t)AT_D + c * 32;
+#pragma unroll
+                    for (int u = 0; u < 8; ++u)
+                        *reinterpret_cast<float4 *>(po + u * 4) = make_float4(o[u * 4], o[u * 4 + 1], o[u * 4 + 2], o[u * 4 + 3]);
+                }
+            }
+            if (have) {
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&oempty[ob]);
-            } else {
-#pragma unroll
-                for (int i = 0; i < AT_D; ++i) o[i] = 0.f;
+                if (lane == 0) mbar_arrive(oempty);
             }
-            if (item.nblk > 0) ++qi;
-            const float inv = (have && l > 0.f) ? 1.f / l : 0.f;
-            const float lse = (have && l > 0.f) ? m * kLn2 + logf(l) : -INFINITY;
-            const int64_t hh = (int64_t)item.hg * AT_HEADS + h;
             if (a.splits == 1) {
-                uint16_t *orow = a.out + (item.row * a.H + hh) * AT_D;
-#pragma unroll
-                for (int c = 0; c < AT_D / 8; ++c) {
-                    uint4 w = make_uint4(pack_bf16(o[c * 8] * inv, o[c * 8 + 1] * inv),
-                                         pack_bf16(o[c * 8 + 2] * inv, o[c * 8 + 3] * inv),
-                                         pack_bf16(o[c * 8 + 4] * inv, o[c * 8 + 5] * inv),
-                                         pack_bf16(o[c * 8 + 6] * inv, o[c * 8 + 7] * inv));
-                    *reinterpret_cast<uint4 *>(orow + c * 8) = w;
-                }
                 if (a.lse) a.lse[item.row * a.H + hh] = lse;
             } else {
-                float *po = a.part + ((item.row * a.splits + item.split) * a.H + hh) * (int64_t)AT_D;
-                float *pl = a.part + a.rows * a.splits * (int64_t)a.H * AT_D +
-                            (item.row * a.splits + item.split) * a.H + hh;
-#pragma unroll
-                for (int c = 0; c < AT_D / 4; ++c)
-                    *reinterpret_cast<float4 *>(po + c * 4) =
-                        make_float4(o[c * 4] * inv, o[c * 4 + 1] * inv, o[c * 4 + 2] * inv, o[c * 4 + 3] * inv);
-                *pl = lse;
+                a.part[a.rows * a.splits * (int64_t)a.H * AT_D + (item.row * a.splits + item.split) * a.H + hh] = lse;
             }
+            if (item.nblk > 0) ++qi;
         }
     }
 
@@ -475,7 +592,8 @@ sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_con
         // let copies and MMAs in flight land before shared and tensor memory go
         for (int j = kv_consumed; j < kv_issued; ++j) mbar_wait(&kvfull[j % AT_STAGES], (j / AT_STAGES) & 1);
         for (int j = q_consumed; j < q_issued; ++j) mbar_wait(&qfull[j & 1], (j >> 1) & 1);
-        if (mma_blocks > 0) mbar_wait(&pempty[(mma_blocks - 1) & 1], ((mma_blocks - 1) >> 1) & 1);
+        if (pv_last & 4) mbar_wait(&pempty[pv_last & 1], (pv_last >> 1) & 1);
+        if (s_last & 4) mbar_wait(&sfull[s_last & 1], (s_last >> 1) & 1);
     }
     __syncthreads();
     tc_fence_after();
@@ -517,8 +635,11 @@ cudaError_t launch_sparse_attn_tc(const uint16_t *q, const uint16_t *k, const ui
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     const size_t smem = AtSmem::total;
-    cudaError_t e = cudaFuncSetAttribute(sparse_attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)smem);
+    cudaFuncAttributes fa;
+    cudaError_t e = cudaFuncGetAttributes(&fa, sparse_attn_tc_kernel);
+    if (e != cudaSuccess) return e;
+    if (fa.numRegs != AT_LAUNCH_REGS) return cudaErrorNotSupported;
+    e = cudaFuncSetAttribute(sparse_attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     const unsigned grid = (unsigned)std::min<int64_t>(a.items, sms);
     sparse_attn_tc_kernel<<<grid, AT_THREADS, smem, st>>>(qmap, kmap, vmap, a);
