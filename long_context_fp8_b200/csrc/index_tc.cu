@@ -34,13 +34,13 @@ constexpr int IT_BN = 256;                    // keys per work tile (UMMA N)
 constexpr int IT_QSTAGES = 4;
 constexpr int IT_KSTAGES = 2;
 constexpr int IT_EPI_WARPS = 8;
-constexpr int IT_THREADS = 32 * (4 + IT_EPI_WARPS);   // warpgroup 0: producer, MMA, 2 idle
+constexpr int IT_THREADS = 32 * (4 + IT_EPI_WARPS);   // warpgroup 0: producer, MMA, 2 coefficient warps
 // Register split (setmaxnreg): the kernel is built for 168 registers x 384
-// threads = 64512; warpgroup 0 gives up to 40 and the two epilogue warpgroups
-// take 232: 128 x 40 + 256 x 232 = 64512, the launch's own total.
+// threads = 64512; warpgroup 0 gives up to 56 and the two epilogue warpgroups
+// take 224: 128 x 56 + 256 x 224 = 64512, the launch's own total.
 constexpr int IT_LAUNCH_REGS = 168;
-constexpr int IT_REGS_LOW = 40;
-constexpr int IT_REGS_HIGH = 232;
+constexpr int IT_REGS_LOW = 56;
+constexpr int IT_REGS_HIGH = 224;
 static_assert(128 * IT_REGS_LOW + 256 * IT_REGS_HIGH <= IT_LAUNCH_REGS * IT_THREADS, "register split");
 constexpr int IT_QBYTES = IT_BM * 128;        // 16 KB
 constexpr int IT_KBYTES = IT_BN * 128;        // 32 KB
@@ -64,10 +64,10 @@ struct IdxTcArgs {
 struct SmemLayout {
     static constexpr size_t k_off = 0;
     static constexpr size_t q_off = k_off + (size_t)IT_KSTAGES * IT_KBYTES;
-    static constexpr size_t c_off = q_off + (size_t)IT_QSTAGES * IT_QBYTES;
-    static constexpr size_t sk_off = c_off + sizeof(float) * IT_MAX_H * IT_CS_STRIDE;
-    static constexpr size_t bar_off = sk_off + sizeof(float) * IT_BN;
-    static constexpr int n_bars = 2 * IT_KSTAGES + 2 * IT_QSTAGES + 4;
+    static constexpr size_t c_off = q_off + (size_t)IT_QSTAGES * IT_QBYTES;      // [2] c tables
+    static constexpr size_t sk_off = c_off + 2 * sizeof(float) * IT_MAX_H * IT_CS_STRIDE;   // [2] key scales
+    static constexpr size_t bar_off = sk_off + 2 * sizeof(float) * IT_BN;
+    static constexpr int n_bars = 2 * IT_KSTAGES + 2 * IT_QSTAGES + 4 + 4;
     static constexpr size_t slot_off = bar_off + 8 * n_bars;
     static constexpr size_t total = slot_off + 16 + 1024;   // + alignment slack
 };
@@ -109,8 +109,6 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t *bar, uint32_t parity, vo
     }
 }
 
-__device__ __forceinline__ void epi_bar_sync() { asm volatile("bar.sync 1, %0;" :: "n"(32 * IT_EPI_WARPS) : "memory"); }
-
 __global__ void __launch_bounds__(IT_THREADS, 1)
 index_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap kmap,
                 const IdxTcArgs a)
@@ -125,6 +123,7 @@ index_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant_
     uint64_t *kfull = bars, *kempty = bars + IT_KSTAGES;
     uint64_t *qfull = bars + 2 * IT_KSTAGES, *qempty = qfull + IT_QSTAGES;
     uint64_t *tfull = qempty + IT_QSTAGES, *tempty = tfull + 2;
+    uint64_t *cfull = tempty + 2, *cempty = cfull + 2;     // per work tile: c table and key scales
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + SmemLayout::slot_off);
     __shared__ volatile int abort_flag;
     // progress of the producer and the MMA issuer, for the wind-down after an abort
@@ -142,6 +141,7 @@ index_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant_
         for (int i = 0; i < IT_KSTAGES; ++i) { mbar_init(&kfull[i], 1); mbar_init(&kempty[i], 1); }
         for (int i = 0; i < IT_QSTAGES; ++i) { mbar_init(&qfull[i], 1); mbar_init(&qempty[i], 1); }
         for (int i = 0; i < 2; ++i) { mbar_init(&tfull[i], 1); mbar_init(&tempty[i], IT_EPI_WARPS); }
+        for (int i = 0; i < 2; ++i) { mbar_init(&cfull[i], 2); mbar_init(&cempty[i], IT_EPI_WARPS); }
         abort_flag = 0;
         q_issued = k_issued = q_consumed = k_consumed = mma_heads = 0;
         fence_mbar_init();
@@ -151,7 +151,7 @@ index_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant_
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
     if (warp < 4) {
-        // warpgroup 0 (warps 0-3): producer, MMA issuer, two idle warps
+        // warpgroup 0 (warps 0-3): producer, MMA issuer, two coefficient warps
         regs_dec<IT_REGS_LOW>();
         if (warp == 0) {
             // ------------------------------------------------ TMA producer
@@ -208,6 +208,56 @@ index_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant_
                     umma_commit(&kempty[kb]);
                 }
             }
+        } else {
+            // ------------------------------------------------ coefficient warps (2, 3)
+            // One work tile ahead of the epilogue: the c table c[t,h] = w[t,h] * sq[t]
+            // of the tile's query rows and its 256 key scales, into one of two buffers.
+            const int ct = tid - 64;                       // 0..63
+            const bool wvec = (H % 8) == 0 && (reinterpret_cast<uintptr_t>(a.w) & 15u) == 0;
+            TileWalk tw;
+            int lt = 0;
+            for (bool ok = tw.start(a, blockIdx.x); ok; ok = tw.next(a, gridDim.x), ++lt) {
+                const int cb = lt & 1;
+                if (!__all_sync(0xffffffffu, wait_or_abort(&cempty[cb], ((lt >> 1) & 1) ^ 1, &abort_flag))) break;
+                const int64_t t0 = a.row_begin + tw.rb * IT_BM;
+                const int64_t s0 = tw.kt * IT_BN;
+                float *cs = Cs + cb * IT_MAX_H * IT_CS_STRIDE;
+                if (wvec) {
+                    // thread = query row (two per thread): its H weights in 16-byte loads, four
+                    // in flight at a time, so a table costs a few memory latencies
+                    for (int r = ct; r < IT_BM; r += 64) {
+                        const int64_t t = t0 + r;
+                        const bool in = t < row_end;
+                        const float sqv = in ? a.sq[t] : 0.f;
+                        const uint4 *wr = reinterpret_cast<const uint4 *>(a.w + (in ? t : 0) * H);
+                        for (int j0 = 0; j0 < H / 8; j0 += 4) {
+                            uint4 u[4];
+#pragma unroll
+                            for (int j = 0; j < 4; ++j) u[j] = j0 + j < H / 8 && in ? __ldg(wr + j0 + j) : make_uint4(0, 0, 0, 0);
+#pragma unroll
+                            for (int j = 0; j < 4; ++j) {
+                                if (j0 + j >= H / 8) break;
+                                const uint32_t wv[4] = {u[j].x, u[j].y, u[j].z, u[j].w};
+#pragma unroll
+                                for (int e = 0; e < 4; ++e) {
+                                    const int h = (j0 + j) * 8 + 2 * e;
+                                    cs[h * IT_CS_STRIDE + r] = __uint_as_float(wv[e] << 16) * sqv;
+                                    cs[(h + 1) * IT_CS_STRIDE + r] = __uint_as_float(wv[e] & 0xffff0000u) * sqv;
+                                }
+                            }
+                        }
+                    }
+                } else {
+                    for (int i = ct; i < IT_BM * H; i += 64) {
+                        const int r = i / H, h = i % H;
+                        const int64_t t = t0 + r;
+                        cs[h * IT_CS_STRIDE + r] = t < row_end ? bf16_to_f32(a.w[t * H + h]) * a.sq[t] : 0.f;
+                    }
+                }
+                for (int i = ct; i < IT_BN; i += 64) Sk[cb * IT_BN + i] = s0 + i < a.T ? a.sk[s0 + i] : 0.f;
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&cfull[cb]);    // releases the tables to the epilogue
+            }
         }
     } else {
         regs_inc<IT_REGS_HIGH>();
@@ -219,24 +269,13 @@ index_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant_
         const uint32_t tlane = tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(half * 128);
         TileWalk tw;
         int lt = 0;
-        bool dead = false;   // after an abort: keep walking the tiles (so every epilogue warp
-                             // meets every named barrier) but do no work
-        for (bool ok = tw.start(a, blockIdx.x); ok; ok = tw.next(a, gridDim.x), ++lt) {
+        bool dead = false;   // after an abort: stop (every wait below is bounded)
+        for (bool ok = tw.start(a, blockIdx.x); ok && !dead; ok = tw.next(a, gridDim.x), ++lt) {
             const int64_t t0 = a.row_begin + tw.rb * IT_BM;
             const int64_t s0 = tw.kt * IT_BN;
-            epi_bar_sync();                          // the previous tile is done with Cs / Sk
-            dead = __any_sync(0xffffffffu, dead || abort_flag);
-            if (!dead) {
-                for (int i = et; i < IT_BM * H; i += 32 * IT_EPI_WARPS) {
-                    const int r = i / H, h = i % H;
-                    const int64_t t = t0 + r;
-                    Cs[h * IT_CS_STRIDE + r] = t < row_end ? bf16_to_f32(a.w[t * H + h]) * a.sq[t] : 0.f;
-                }
-                for (int i = et; i < IT_BN; i += 32 * IT_EPI_WARPS)
-                    Sk[i] = s0 + i < a.T ? a.sk[s0 + i] : 0.f;
-            }
-            epi_bar_sync();
-            if (dead) continue;
+            const int cb = lt & 1;
+            if (!__all_sync(0xffffffffu, wait_or_abort(&cfull[cb], (lt >> 1) & 1, &abort_flag))) { dead = true; break; }
+            const float *cs = Cs + cb * IT_MAX_H * IT_CS_STRIDE;
 
             uint64_t sc[64];                         // running scores, column pairs (2i, 2i+1)
 #pragma unroll
@@ -247,7 +286,7 @@ index_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant_
                 const bool ok = wait_or_abort(&tfull[acc], (g >> 1) & 1, &abort_flag);
                 if (!__all_sync(0xffffffffu, ok)) { dead = true; break; }
                 tc_fence_after();
-                const float c = Cs[h * IT_CS_STRIDE + row];
+                const float c = cs[h * IT_CS_STRIDE + row];
                 const uint64_t cc = f2_pack(c, c);
                 const uint32_t base = tlane + (uint32_t)(acc * IT_BN);
                 // 8 chunks of 16 columns; the load of chunk i+1 overlaps the math of chunk i
@@ -275,13 +314,13 @@ index_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant_
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&tempty[acc]);
             }
-            if (dead) continue;
+            if (dead) break;
             // key scales, causal mask, store
             const int64_t t = t0 + row;
             if (t < row_end) {
                 float *orow = a.out + (t - a.row_begin) * a.ld;
                 const int64_t sb = s0 + half * 128;
-                const float *skh = Sk + half * 128;
+                const float *skh = Sk + cb * IT_BN + half * 128;
 #pragma unroll
                 for (int j4 = 0; j4 < 32; ++j4) {
                     const int64_t s = sb + j4 * 4;
@@ -299,6 +338,8 @@ index_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant_
                     }
                 }
             }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&cempty[cb]);        // done with this tile's c table and key scales
         }
     }
 
