@@ -20,6 +20,7 @@
 // Every mbarrier wait is bounded; a timeout records DSA_ERR_TIMEOUT, makes
 // every role stop at its next wait, and the CTA still frees its tensor memory.
 #include <algorithm>
+#include <cstring>
 
 #include "kernels.h"
 #include "sm100.cuh"
@@ -31,7 +32,7 @@ using namespace sm100;
 
 constexpr int IT_BM = 128;                    // query rows per work tile (UMMA M)
 constexpr int IT_BN = 256;                    // keys per work tile (UMMA N)
-constexpr int IT_QSTAGES = 4;
+constexpr int IT_QSTAGES = 3;
 constexpr int IT_KSTAGES = 2;
 constexpr int IT_EPI_WARPS = 8;
 constexpr int IT_THREADS = 32 * (4 + IT_EPI_WARPS);   // warpgroup 0: producer, MMA, 2 coefficient warps
@@ -58,13 +59,15 @@ struct IdxTcArgs {
     float *out;
     int64_t ld;
     int vec_store;               // ld % 4 == 0 and out 16-byte aligned
+    int tma_store;               // tiles wholly below the diagonal leave through TMA stores (omap)
     WsHeader *hdr;
 };
 
 struct SmemLayout {
     static constexpr size_t k_off = 0;
     static constexpr size_t q_off = k_off + (size_t)IT_KSTAGES * IT_KBYTES;
-    static constexpr size_t c_off = q_off + (size_t)IT_QSTAGES * IT_QBYTES;      // [2] c tables
+    static constexpr size_t stg_off = q_off + (size_t)IT_QSTAGES * IT_QBYTES;    // [8 warps] 32 x 32 fp32 store staging
+    static constexpr size_t c_off = stg_off + (size_t)IT_EPI_WARPS * 4096;       // [2] c tables
     static constexpr size_t sk_off = c_off + 2 * sizeof(float) * IT_MAX_H * IT_CS_STRIDE;   // [2] key scales
     static constexpr size_t bar_off = sk_off + 2 * sizeof(float) * IT_BN;
     static constexpr int n_bars = 2 * IT_KSTAGES + 2 * IT_QSTAGES + 4 + 4;
@@ -111,13 +114,14 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t *bar, uint32_t parity, vo
 
 __global__ void __launch_bounds__(IT_THREADS, 1)
 index_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap kmap,
-                const IdxTcArgs a)
+                const __grid_constant__ CUtensorMap omap, const IdxTcArgs a)
 {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *Ks = smem + SmemLayout::k_off;
     uint8_t *Qs = smem + SmemLayout::q_off;
     float *Cs = reinterpret_cast<float *>(smem + SmemLayout::c_off);
+    uint8_t *Stg = smem + SmemLayout::stg_off;
     float *Sk = reinterpret_cast<float *>(smem + SmemLayout::sk_off);
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + SmemLayout::bar_off);
     uint64_t *kfull = bars, *kempty = bars + IT_KSTAGES;
@@ -317,7 +321,34 @@ index_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant_
             if (dead) break;
             // key scales, causal mask, store
             const int64_t t = t0 + row;
-            if (t < row_end) {
+            if (a.tma_store && s0 + IT_BN - 1 <= t0) {
+                // every key of the tile is at or below every row: the warp's 32 rows x 128
+                // keys leave as four 32 x 32 tiles through shared memory and TMA stores
+                // (coalesced, asynchronous; rows and keys past the ends are clipped)
+                uint8_t *stg = Stg + (warp - 4) * 4096;
+                const float *skh = Sk + cb * IT_BN + half * 128;
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    if (lane == 0) bulk_wait_group_read<0>();   // the last store has read the staging
+                    __syncwarp();
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) {          // row `lane`, 16-byte chunk j, 128-byte swizzle
+                        float v0, v1, v2, v3;
+                        f2_unpack(sc[c * 16 + 2 * j], v0, v1);
+                        f2_unpack(sc[c * 16 + 2 * j + 1], v2, v3);
+                        const float *kv = skh + c * 32 + j * 4;
+                        *reinterpret_cast<float4 *>(stg + lane * 128 + ((j ^ (lane & 7)) << 4)) =
+                            make_float4(v0 * kv[0], v1 * kv[1], v2 * kv[2], v3 * kv[3]);
+                    }
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) {
+                        tma_store_2d(&omap, stg, (int)(s0 + half * 128 + c * 32),
+                                     (int)(t0 - a.row_begin + quarter * 32));
+                        bulk_commit_group();
+                    }
+                }
+            } else if (t < row_end) {
                 float *orow = a.out + (t - a.row_begin) * a.ld;
                 const int64_t sb = s0 + half * 128;
                 const float *skh = Sk + cb * IT_BN + half * 128;
@@ -341,6 +372,7 @@ index_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant_
             __syncwarp();
             if (lane == 0) mbar_arrive(&cempty[cb]);        // done with this tile's c table and key scales
         }
+        if (lane == 0) bulk_wait_group<0>();               // stores complete before shared memory goes
     }
 
     tc_fence_before();
@@ -391,6 +423,10 @@ cudaError_t launch_index_tc(const uint8_t *q8, const float *sq, const uint8_t *k
     a.n_rb = ceil_div(row_count, IT_BM);
     a.out = out; a.ld = ld;
     a.vec_store = (ld % 4 == 0) && ((reinterpret_cast<uintptr_t>(out) & 15u) == 0);
+    CUtensorMap omap;
+    std::memset(&omap, 0, sizeof(omap));
+    a.tma_store = a.vec_store && row_count < ((int64_t)1 << 31) &&
+                  make_tmap_f32_2d(&omap, out, (uint64_t)T, (uint64_t)row_count, (uint64_t)ld * 4, 32, 32);
     a.hdr = hdr;
     // number of work tiles, to size the persistent grid
     int64_t tiles = 0;
@@ -417,7 +453,7 @@ cudaError_t launch_index_tc(const uint8_t *q8, const float *sq, const uint8_t *k
             fill_upper_kernel<<<dim3(8, (unsigned)n), 256, 0, st>>>(out + r0 * ld, ld, T, row_begin + r0);
         }
     }
-    index_tc_kernel<<<grid, IT_THREADS, smem, st>>>(qmap, kmap, a);
+    index_tc_kernel<<<grid, IT_THREADS, smem, st>>>(qmap, kmap, omap, a);
     return cudaGetLastError();
 }
 

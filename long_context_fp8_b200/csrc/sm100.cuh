@@ -118,6 +118,21 @@ __device__ __forceinline__ void tma_gather4(void *smem_dst, const CUtensorMap *m
         : "memory");
 }
 
+// TMA tile store shared -> global (clipped at the tensor's bounds), tracked by
+// this thread's bulk async-groups.
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap *map, const void *smem_src, int x, int y)
+{
+    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];"
+                 :: "l"(map), "r"(smem_u32(smem_src)), "r"(x), "r"(y) : "memory");
+}
+__device__ __forceinline__ void bulk_commit_group() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// Wait until at most N of this thread's bulk groups still read their shared-memory source.
+template <int N>
+__device__ __forceinline__ void bulk_wait_group_read() { asm volatile("cp.async.bulk.wait_group.read %0;" :: "n"(N) : "memory"); }
+// Wait until at most N of this thread's bulk groups are still in flight.
+template <int N>
+__device__ __forceinline__ void bulk_wait_group() { asm volatile("cp.async.bulk.wait_group %0;" :: "n"(N) : "memory"); }
+
 // Order this thread's generic-proxy shared-memory writes before later
 // async-proxy (tensor core, TMA) accesses.
 __device__ __forceinline__ void fence_proxy_async_smem()
@@ -337,5 +352,8 @@ bool make_tmap_u8(CUtensorMap *map, const void *base, int rank, const uint64_t *
 // Same for a 2-D bf16 tensor (dims/box in elements).
 bool make_tmap_bf16_2d(CUtensorMap *map, const void *base, uint64_t cols, uint64_t rows,
                        uint64_t row_stride_bytes, uint32_t box_cols, uint32_t box_rows);
+// 2-D fp32 tensor, 128-byte swizzle (box_cols * 4 must be 128 for the swizzle).
+bool make_tmap_f32_2d(CUtensorMap *map, const void *base, uint64_t cols, uint64_t rows,
+                      uint64_t row_stride_bytes, uint32_t box_cols, uint32_t box_rows);
 
 }  // namespace dsa

@@ -54,4 +54,17 @@ bool make_tmap_bf16_2d(CUtensorMap *map, const void *base, uint64_t cols, uint64
     return r == CUDA_SUCCESS;
 }
 
+bool make_tmap_f32_2d(CUtensorMap *map, const void *base, uint64_t cols, uint64_t rows,
+                      uint64_t row_stride_bytes, uint32_t box_cols, uint32_t box_rows)
+{
+    PFN_cuTensorMapEncodeTiled_v12000 fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t d[2] = {cols, rows}, s[1] = {row_stride_bytes};
+    cuuint32_t bx[2] = {box_cols, box_rows}, es[2] = {1, 1};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void *>(base), d, s, bx, es,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
 }  // namespace dsa
