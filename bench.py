@@ -422,7 +422,10 @@ def main():
     ap.add_argument("--steps", type=int, default=5)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="dsa", choices=["dsa", "reference"])
-    ap.add_argument("--workload", default="p128k", choices=["p128k", "p16k"])
+    ap.add_argument("--workload", default="p128k", choices=["p128k", "p16k", "p16k_hq128"])
+    ap.add_argument("--decode-workload", default="dec64x64k", choices=["dec64x64k", "dec_ragged"])
+    ap.add_argument("--decode-only", action="store_true",
+                    help="profiling aid: time only the decode step and print its own line")
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
@@ -432,7 +435,7 @@ def main():
 
     ws_n, rank, local = dist_setup()
     spec = dsa_synth.prefill_spec(args.workload)
-    dspec = dsa_synth.decode_spec("dec64x64k")
+    dspec = dsa_synth.decode_spec(args.decode_workload)
     metric = "DSA prefill tokens/s @128K; decode steps/s @64K ctx x64 seqs; % of roofline"
 
     if args.impl == "reference":
@@ -467,6 +470,24 @@ def main():
     dsa.load()
     peaks, peak_kind = load_peaks()
 
+    if args.decode_only:
+        dec = bench_decode(args, dsa, dspec, peaks, ws_n, rank)
+        us = dec["step_ms"] * 1e3
+        gbs = dec["bytes"] / (dec["step_ms"] * 1e-3) / 1e9
+        if rank == 0:
+            print(json.dumps({"metric": "DSA decode steps/s", "value": round(ws_n * 1e3 / dec["step_ms"], 1),
+                              "unit": "steps/s", "n_gpus": ws_n, "steps": args.steps, "warmup": args.warmup,
+                              "us_per_step": round(us, 2), "higher_is_better": True,
+                              "config": {"workload": workload_config(spec, dspec)["decode_workload"]},
+                              "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": peaks["hbm_gbs"],
+                                           "unit": "GB/s", "frac": round(gbs / peaks["hbm_gbs"], 4),
+                                           "algorithmic_bytes": dec["bytes"]},
+                              "gpu_launches_per_step": dec["per_kernel"], "device_status": dec["status"]}),
+                  flush=True)
+        if ws_n > 1:
+            torch.distributed.barrier()
+            torch.distributed.destroy_process_group()
+        return
     pre = bench_prefill(args, dsa, spec, peaks, peak_kind, ws_n, rank)
     dec = None if args.no_decode else bench_decode(args, dsa, dspec, peaks, ws_n, rank)
 

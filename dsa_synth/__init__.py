@@ -73,6 +73,10 @@ PRESETS: Dict[str, object] = {
     # 16K prefill: 1 % needles
     "p16k": PrefillSpec("p16k", L=16384, H_I=64, d_I=128, k=2048, H_q=16, d=128,
                         fp8=True, n_needles=164, seed=1),
+    # 16K prefill with the 128K workload's 128 query heads: a small case of the
+    # tensor-core attention path for profiling (inputs a few GB, still above L2)
+    "p16k_hq128": PrefillSpec("p16k_hq128", L=16384, H_I=64, d_I=128, k=2048, H_q=128, d=128,
+                              fp8=True, n_needles=164, seed=1),
     # 128K prefill: 0.5 % needles
     "p128k": PrefillSpec("p128k", L=131072, H_I=64, d_I=128, k=2048, H_q=128, d=128,
                          fp8=True, n_needles=655, seed=2),
