@@ -193,7 +193,7 @@ dsa_status dsa_decode(const void *q_idx, const float *q_scale, const void *w, co
  * (64 MiB) inside the library; every GPU that loads the library holds it
  * until the process exits.  A problem whose dsa_decode_workspace_size()
  * exceeds that size is rejected with DSA_ERR_WORKSPACE before any launch
- * (64 sequences x 64K context x k 2048 x 128 heads needs about 45 MiB).
+ * (64 sequences x 64K context x k 2048 x 128 heads needs about 33 MiB).
  * The first call on each device looks up the array's device address with
  * that device current; make that first call before any stream capture.
  * Every call on a device shares the one array and leaves its contents behind
