@@ -277,15 +277,9 @@ dsa_status dsa_decode(const void *q_idx, const float *q_scale, const void *w, co
                                     context_lens, num_pages, max_pages_per_seq, page_size, B,
                                     max_context, H_I, scores, max_context, hdr, st);
     }
-    if (e == cudaSuccess) {
-        // enough rows of moderate length: one CTA per row; few long rows: each
-        // row split over several CTAs
-        if (B >= 16 && max_context <= 262144)
-            e = launch_topk_rows(scores, max_context, 0, context_lens, max_context, B, k_sel, idx, hdr, st);
-        else
-            e = launch_topk_split(scores, max_context, context_lens, max_context, B, k_sel, idx, topk_ws,
-                                  hdr, st);
-    }
+    if (e == cudaSuccess)   // each row split over 16K-position chunks (CTAs), then one CTA per row
+        e = launch_topk_split(scores, max_context, context_lens, max_context, B, k_sel, idx, topk_ws,
+                              hdr, st);
     if (e == cudaSuccess) {
         bool done = false;
         if (sparse_attn_tc_supported(H_q, d) && (int64_t)num_pages * page_size < ((int64_t)1 << 31)) {

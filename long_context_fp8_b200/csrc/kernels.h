@@ -34,8 +34,10 @@ cudaError_t launch_topk_rows(const float *scores, int64_t ld, int64_t row_begin,
                              const int32_t *lens, int64_t max_len, int64_t row_count, int k,
                              int32_t *idx, WsHeader *hdr, cudaStream_t st);
 
-// Rows of lengths lens[r] split over CTAs of TL_CHUNK positions (few, long
-// rows: decode).  Scratch of topk_split_ws_bytes(rows, max_len) at ws_base.
+// Rows of lengths lens[r] (decode): each row split over CTAs of 16384
+// positions that share a sampled threshold and collect their candidates, then
+// one CTA per row finishes the exact select.  Scratch of
+// topk_split_ws_bytes(rows, max_len) at ws_base.
 size_t topk_split_ws_bytes(int64_t rows, int64_t max_len);
 cudaError_t launch_topk_split(const float *scores, int64_t ld, const int32_t *lens, int64_t max_len,
                               int64_t rows, int k, int32_t *idx, void *ws_base, WsHeader *hdr,

@@ -472,6 +472,52 @@ __device__ __forceinline__ void hist_top11(uint32_t *hist, const uint32_t (&keys
     }
 }
 
+// Threshold guess for a long row: the key of rank ~1.5 k (scaled to the
+// sample, at least 8) among 2048 evenly spaced samples, resolved to its top 22 bits (a
+// threshold at or below it).  Every thread calls it; every CTA working on the
+// same row computes the same value.
+__device__ uint32_t sampled_threshold(TopkSmem &sm, const float *row, int64_t n, int k)
+{
+    const int tid = threadIdx.x;
+    float sv[TK_SAMPLE / TK_THREADS];                     // all loads issued before any is used
+#pragma unroll
+    for (int q = 0; q < TK_SAMPLE / TK_THREADS; ++q)
+        sv[q] = __ldg(row + (int64_t)(tid + q * TK_THREADS) * n / TK_SAMPLE);
+#pragma unroll
+    for (int q = 0; q < TK_SAMPLE / TK_THREADS; ++q) sm.sample[tid + q * TK_THREADS] = float_key(sv[q]);
+    __syncthreads();
+    // at least 8 samples above the threshold: a rank of 1 or 2 (long rows, small k)
+    // estimates the count so loosely that it often lands below k
+    const double want = 1.5 * (double)k * TK_SAMPLE / (double)n;
+    const uint32_t rank = (uint32_t)min((double)TK_SAMPLE, max(8.0, ceil(want)));
+    uint32_t tau, unused;
+    radix_select_smem(sm, sm.sample, TK_SAMPLE, rank, &tau, &unused, 2);
+    return tau;
+}
+
+// Exact top-k of a row without a threshold guess: a histogram of the top 11
+// key bits fixes the bin of the k-th largest key; the keys in or above it go
+// on chip (or, if too many, a radix select runs over the row in global memory).
+__device__ __noinline__ void topk_row_histogram(TopkSmem &sm, const float *row, int64_t n, bool vec, int k,
+                                                int32_t *out)
+{
+    const int tid = threadIdx.x;
+    for (int i = tid; i < 2048; i += TK_THREADS) sm.hist[i] = 0u;
+    __syncthreads();
+    for (int64_t c0 = 0; c0 < n; c0 += TK_STEP) {
+        uint32_t keys[TK_ITEMS], valid;
+        load8(row, n, c0 + (int64_t)tid * TK_ITEMS, vec, keys, valid);
+        hist_top11(sm.hist, keys, valid);
+    }
+    __syncthreads();
+    find_bin(sm, 2048, (uint32_t)k);
+    const uint32_t b1 = sm.sh_bin;
+    const uint32_t remaining = (uint32_t)k - sm.sh_above;
+    const uint32_t ncand = collect_candidates(sm, row, n, vec, [b1](uint32_t key) { return (key >> 21) >= b1; });
+    if (ncand <= TK_CAP) select_on_chip(sm, ncand, b1, remaining, k, out);
+    else select_global(sm, row, n, vec, k, out);
+}
+
 __global__ void __launch_bounds__(TK_THREADS, 2)
 topk_rows_kernel(const float *__restrict__ scores, int64_t ld, int64_t row_begin,
                  const int32_t *__restrict__ lens, int64_t max_len, int k,
@@ -512,55 +558,34 @@ topk_rows_kernel(const float *__restrict__ scores, int64_t ld, int64_t row_begin
     // ---- guess a threshold from evenly spaced samples: about 1.5 k keys of the
     // row should lie at or above it; then one ordered pass collects them ----
     {
-        float sv[TK_SAMPLE / TK_THREADS];                 // all loads issued before any is used
-#pragma unroll
-        for (int q = 0; q < TK_SAMPLE / TK_THREADS; ++q)
-            sv[q] = __ldg(row + (int64_t)(tid + q * TK_THREADS) * n / TK_SAMPLE);
-#pragma unroll
-        for (int q = 0; q < TK_SAMPLE / TK_THREADS; ++q) sm.sample[tid + q * TK_THREADS] = float_key(sv[q]);
-        __syncthreads();
-        const double want = 1.5 * (double)k * TK_SAMPLE / (double)n;
-        const uint32_t rank = (uint32_t)min((double)TK_SAMPLE, max(1.0, ceil(want)));
-        uint32_t tau, unused;
-        radix_select_smem(sm, sm.sample, TK_SAMPLE, rank, &tau, &unused, 2);
+        const uint32_t tau = sampled_threshold(sm, row, n, k);
         const uint32_t c = collect_above_warp(sm, row, n, vec, key_float(tau));
         if (c >= (uint32_t)k && c <= TK_CAP) {        // the selection lies among the candidates
             select_candidates(sm, c, k, out);
             return;
         }
     }
-
-    // ---- fallback: histogram of the top 11 bits, then the keys in or above the
-    // threshold bin on chip (or, if too many, the radix select in global memory) ----
-    for (int i = tid; i < 2048; i += TK_THREADS) sm.hist[i] = 0u;
-    __syncthreads();
-    for (int64_t c0 = 0; c0 < n; c0 += TK_STEP) {
-        uint32_t keys[TK_ITEMS], valid;
-        load8(row, n, c0 + (int64_t)tid * TK_ITEMS, vec, keys, valid);
-        hist_top11(sm.hist, keys, valid);
-    }
-    __syncthreads();
-    find_bin(sm, 2048, (uint32_t)k);
-    const uint32_t b1 = sm.sh_bin;
-    const uint32_t remaining = (uint32_t)k - sm.sh_above;
-    const uint32_t ncand = collect_candidates(sm, row, n, vec, [b1](uint32_t key) { return (key >> 21) >= b1; });
-    if (ncand <= TK_CAP) select_on_chip(sm, ncand, b1, remaining, k, out);
-    else select_global(sm, row, n, vec, k, out);
+    // ---- fallback: the exact histogram path ----
+    topk_row_histogram(sm, row, n, vec, k, out);
 }
 
 
 // ---------------------------------------------------------------- long rows, split over CTAs
-// Workspace per row: hist[2048] (zeroed by the launcher), cnt[chunks], then
-// per chunk a fixed slot of TL_SLOT (key, position) candidates.
+// For few long rows (decode): every CTA of a row computes the same sampled
+// threshold, collects the candidates of its chunk of the row into a fixed
+// slot in global memory; one CTA per row then joins the slots in chunk order
+// (so in position order) and finishes the exact select on chip.  Rows whose
+// candidates do not fit (or fall short of k) take the exact histogram path.
+// Workspace per row: cnt[chunks], then per chunk a slot of TS_SLOT
+// (key, position) candidates.
 
-constexpr int TL_CHUNK = 32768;            // positions per CTA
-constexpr int TL_SLOT = 8192;              // candidate slot per chunk (more: the row falls back)
+constexpr int TS_CHUNK = 16384;            // positions per CTA
+constexpr int TS_SLOT = 2048;              // candidate slot per chunk (more: the row falls back)
 
 struct SplitWs {
-    uint32_t *hist;      // [rows][2048]
-    uint32_t *cnt;       // [rows][chunks]
-    uint32_t *ckey;      // [rows][chunks][TL_SLOT]
-    int32_t *cpos;       // [rows][chunks][TL_SLOT]
+    uint32_t *cnt;       // [rows][chunks]: candidates of the chunk, 0xffffffff: a warp overflowed
+    uint32_t *ckey;      // [rows][chunks][TS_SLOT]
+    int32_t *cpos;       // [rows][chunks][TS_SLOT]
     int chunks;
 };
 
@@ -570,34 +595,7 @@ __device__ __forceinline__ int64_t split_len(const int32_t *lens, int64_t max_le
     return (n < 1 || n > max_len) ? -1 : n;
 }
 
-// Pass 1: histogram of the top 11 bits of one chunk, added into the row's.
-__global__ void __launch_bounds__(TK_THREADS)
-topk_split_hist_kernel(const float *__restrict__ scores, int64_t ld, const int32_t *__restrict__ lens,
-                       int64_t max_len, int k, SplitWs ws, int vec_ok)
-{
-    __shared__ uint32_t hist[2048];
-    const int64_t r = blockIdx.y;
-    const int64_t n = split_len(lens, max_len, r);
-    const int64_t c0 = (int64_t)blockIdx.x * TL_CHUNK;
-    if (n <= k || c0 >= n) return;                  // short or invalid rows: the final kernel handles them
-    const int64_t c1 = min(n, c0 + TL_CHUNK);
-    const float *row = scores + r * ld;
-    for (int i = threadIdx.x; i < 2048; i += TK_THREADS) hist[i] = 0u;
-    __syncthreads();
-    for (int64_t s0 = c0; s0 < c1; s0 += TK_STEP) {
-        uint32_t keys[TK_ITEMS], valid;
-        load8(row, c1, s0 + (int64_t)threadIdx.x * TK_ITEMS, vec_ok != 0, keys, valid);
-        hist_top11(hist, keys, valid);
-    }
-    __syncthreads();
-    uint32_t *gh = ws.hist + r * 2048;
-    for (int i = threadIdx.x; i < 2048; i += TK_THREADS)
-        if (hist[i]) atomicAdd(&gh[i], hist[i]);
-}
-
-// Pass 2: ordered copy of the chunk's keys whose top 11 bits are >= the row's
-// threshold bin into the chunk's candidate slot.
-__global__ void __launch_bounds__(TK_THREADS)
+__global__ void __launch_bounds__(TK_THREADS, 2)
 topk_split_collect_kernel(const float *__restrict__ scores, int64_t ld, const int32_t *__restrict__ lens,
                           int64_t max_len, int k, SplitWs ws, int vec_ok)
 {
@@ -605,42 +603,21 @@ topk_split_collect_kernel(const float *__restrict__ scores, int64_t ld, const in
     TopkSmem &sm = *reinterpret_cast<TopkSmem *>(smem_raw);
     const int64_t r = blockIdx.y;
     const int64_t n = split_len(lens, max_len, r);
-    const int64_t c0 = (int64_t)blockIdx.x * TL_CHUNK;
-    if (n <= k || c0 >= n) return;
-    const int64_t c1 = min(n, c0 + TL_CHUNK);
+    const int64_t c0 = (int64_t)blockIdx.x * TS_CHUNK;
+    if (n <= TK_CAP || c0 >= n) return;              // short or invalid rows: the final kernel alone
+    const int64_t c1 = min(n, c0 + TS_CHUNK);
     const float *row = scores + r * ld;
-    for (int i = threadIdx.x; i < 2048; i += TK_THREADS) sm.hist[i] = ws.hist[r * 2048 + i];
-    __syncthreads();
-    find_bin(sm, 2048, (uint32_t)k);
-    const uint32_t b1 = sm.sh_bin;
-    const int64_t slot = (r * ws.chunks + blockIdx.x) * (int64_t)TL_SLOT;
-    uint32_t base = 0;
-    for (int64_t s0 = c0; s0 < c1; s0 += TK_STEP) {
-        const int64_t s = s0 + (int64_t)threadIdx.x * TK_ITEMS;
-        uint32_t keys[TK_ITEMS], valid, flags = 0, cnt = 0;
-        load8(row, c1, s, vec_ok != 0, keys, valid);
-#pragma unroll
-        for (int i = 0; i < TK_ITEMS; ++i)
-            if (((valid >> i) & 1u) && (keys[i] >> 21) >= b1) { flags |= 1u << i; ++cnt; }
-        uint32_t tot;
-        uint32_t off = base + block_excl_scan(cnt, sm.warp_buf, &tot);
-#pragma unroll
-        for (int i = 0; i < TK_ITEMS; ++i) {
-            if ((flags >> i) & 1u) {
-                if (off < TL_SLOT) {
-                    ws.ckey[slot + off] = keys[i];
-                    ws.cpos[slot + off] = (int32_t)(s + i);
-                }
-                ++off;
-            }
+    const uint32_t tau = sampled_threshold(sm, row, n, k);
+    const uint32_t c = collect_above_warp(sm, row + c0, c1 - c0, vec_ok != 0, key_float(tau));
+    const int64_t slot = (r * ws.chunks + blockIdx.x) * (int64_t)TS_SLOT;
+    if (c != 0xffffffffu)
+        for (uint32_t i = threadIdx.x; i < min(c, (uint32_t)TS_SLOT); i += TK_THREADS) {
+            ws.ckey[slot + i] = sm.ckey[i];
+            ws.cpos[slot + i] = (int32_t)(sm.cpos[i] + c0);
         }
-        base += tot;
-    }
-    if (threadIdx.x == 0) ws.cnt[r * ws.chunks + blockIdx.x] = base;
+    if (threadIdx.x == 0) ws.cnt[r * ws.chunks + blockIdx.x] = c;
 }
 
-// Pass 3: one CTA per row joins the chunks' candidates in chunk order (so in
-// position order), finishes the select on chip, or falls back to the row.
 __global__ void __launch_bounds__(TK_THREADS)
 topk_split_final_kernel(const float *__restrict__ scores, int64_t ld, const int32_t *__restrict__ lens,
                         int64_t max_len, int k, SplitWs ws, int32_t *__restrict__ idx, WsHeader *hdr,
@@ -662,34 +639,54 @@ topk_split_final_kernel(const float *__restrict__ scores, int64_t ld, const int3
         return;
     }
     const float *row = scores + r * ld;
-    for (int i = tid; i < 2048; i += TK_THREADS) sm.hist[i] = ws.hist[r * 2048 + i];
-    __syncthreads();
-    find_bin(sm, 2048, (uint32_t)k);
-    const uint32_t b1 = sm.sh_bin;
-    const uint32_t remaining = (uint32_t)k - sm.sh_above;
-    const int nch = (int)((n + TL_CHUNK - 1) / TL_CHUNK);
-    uint32_t total = 0;
-    bool fits = true;
-    for (int c = 0; c < nch; ++c) {
-        const uint32_t m = ws.cnt[r * ws.chunks + c];
-        total += m;
-        fits = fits && m <= TL_SLOT;
+    const bool vec = vec_ok != 0;
+    if (n <= TK_CAP) {                               // short rows: every key is a candidate
+        const uint32_t c = collect_candidates(sm, row, n, vec, [](uint32_t) { return true; });
+        select_candidates(sm, c, k, out);
+        return;
     }
-    if (fits && total <= TK_CAP) {
-        uint32_t off = 0;
-        for (int c = 0; c < nch; ++c) {
-            const uint32_t m = ws.cnt[r * ws.chunks + c];
-            const int64_t slot = (r * ws.chunks + c) * (int64_t)TL_SLOT;
-            for (uint32_t i = tid; i < m; i += TK_THREADS) {
-                sm.ckey[off + i] = ws.ckey[slot + i];
-                sm.cpos[off + i] = ws.cpos[slot + i];
+    const int nch = (int)((n + TS_CHUNK - 1) / TS_CHUNK);
+    bool use = nch <= TK_SAMPLE;                     // counts and offsets fit the scratch arrays
+    if (use) {
+        // chunk counts (sm.sample) and their exclusive prefix (sm.hist), in parallel
+        const int cpt = (nch + TK_THREADS - 1) / TK_THREADS;
+        uint32_t msum = 0;
+        bool fit = true;
+        for (int u = 0; u < cpt; ++u) {
+            const int c = tid * cpt + u;
+            if (c < nch) {
+                const uint32_t m = ws.cnt[r * ws.chunks + c];
+                fit = fit && m <= TS_SLOT;
+                sm.sample[c] = m <= TS_SLOT ? m : 0u;
+                msum += m <= TS_SLOT ? m : 0u;
             }
-            off += m;
+        }
+        use = __syncthreads_and(fit) != 0;
+        uint32_t total;
+        uint32_t run = block_excl_scan(msum, sm.warp_buf, &total);
+        for (int u = 0; u < cpt; ++u) {
+            const int c = tid * cpt + u;
+            if (c < nch) { sm.hist[c] = run; run += sm.sample[c]; }
         }
         __syncthreads();
-        select_on_chip(sm, total, b1, remaining, k, out);
-    } else {
-        select_global(sm, row, n, vec_ok != 0, k, out);
+        use = use && total >= (uint32_t)k && total <= TK_CAP;
+        if (use) {
+            // warp w copies chunks w, w + 16, ...: one memory latency per 16 chunks
+            const int lane = tid & 31, warp = tid >> 5;
+            for (int c = warp; c < nch; c += TK_WARPS) {
+                const uint32_t m = sm.sample[c], off = sm.hist[c];
+                const int64_t slot = (r * ws.chunks + c) * (int64_t)TS_SLOT;
+                for (uint32_t i = lane; i < m; i += 32) {
+                    sm.ckey[off + i] = ws.ckey[slot + i];
+                    sm.cpos[off + i] = ws.cpos[slot + i];
+                }
+            }
+            __syncthreads();
+            select_candidates(sm, total, k, out);
+        }
+    }
+    if (!use) {
+        topk_row_histogram(sm, row, n, vec, k, out);
     }
 }
 
@@ -712,10 +709,9 @@ cudaError_t launch_topk_rows(const float *scores, int64_t ld, int64_t row_begin,
 
 size_t topk_split_ws_bytes(int64_t rows, int64_t max_len)
 {
-    const int64_t chunks = ceil_div(max_len, TL_CHUNK);
-    return align_up(sizeof(uint32_t) * (size_t)rows * 2048, 256) +
-           align_up(sizeof(uint32_t) * (size_t)rows * chunks, 256) +
-           2 * align_up(sizeof(uint32_t) * (size_t)rows * chunks * TL_SLOT, 256);
+    const int64_t chunks = ceil_div(max_len, TS_CHUNK);
+    return align_up(sizeof(uint32_t) * (size_t)rows * chunks, 256) +
+           2 * align_up(sizeof(uint32_t) * (size_t)rows * chunks * TS_SLOT, 256);
 }
 
 cudaError_t launch_topk_split(const float *scores, int64_t ld, const int32_t *lens, int64_t max_len,
@@ -723,27 +719,22 @@ cudaError_t launch_topk_split(const float *scores, int64_t ld, const int32_t *le
                               cudaStream_t st)
 {
     if (rows <= 0) return cudaSuccess;
-    const int64_t chunks = ceil_div(max_len, TL_CHUNK);
+    const int64_t chunks = ceil_div(max_len, TS_CHUNK);
     uint8_t *p = static_cast<uint8_t *>(ws_base);
     SplitWs ws;
     ws.chunks = (int)chunks;
-    ws.hist = reinterpret_cast<uint32_t *>(p);
-    p += align_up(sizeof(uint32_t) * (size_t)rows * 2048, 256);
     ws.cnt = reinterpret_cast<uint32_t *>(p);
     p += align_up(sizeof(uint32_t) * (size_t)rows * chunks, 256);
     ws.ckey = reinterpret_cast<uint32_t *>(p);
-    p += align_up(sizeof(uint32_t) * (size_t)rows * chunks * TL_SLOT, 256);
+    p += align_up(sizeof(uint32_t) * (size_t)rows * chunks * TS_SLOT, 256);
     ws.cpos = reinterpret_cast<int32_t *>(p);
     const int vec_ok = (ld % 4 == 0) && ((reinterpret_cast<uintptr_t>(scores) & 15u) == 0);
     const size_t smem = sizeof(TopkSmem);
-    cudaError_t e = cudaMemsetAsync(ws.hist, 0, sizeof(uint32_t) * (size_t)rows * 2048, st);
-    if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(topk_split_collect_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaError_t e = cudaFuncSetAttribute(topk_split_collect_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     e = cudaFuncSetAttribute(topk_split_final_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     dim3 grid((unsigned)chunks, (unsigned)rows);
-    topk_split_hist_kernel<<<grid, TK_THREADS, 0, st>>>(scores, ld, lens, max_len, k, ws, vec_ok);
     topk_split_collect_kernel<<<grid, TK_THREADS, smem, st>>>(scores, ld, lens, max_len, k, ws, vec_ok);
     topk_split_final_kernel<<<(unsigned)rows, TK_THREADS, smem, st>>>(scores, ld, lens, max_len, k, ws, idx,
                                                                       hdr, vec_ok);

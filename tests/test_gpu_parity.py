@@ -235,7 +235,8 @@ def decode_reference_attention(inp, idx, sm):
                                            ((1500, 129, 640), 100, 16, 128),
                                            ((700, 300), 64, 16, 256),
                                            ((900, 17), 64, 16, 48),       # 48: mma.sync indexer
-                                           ((3000, 1000, 5000) * 6, 256, 16, 64)])   # 18 rows: one CTA per row
+                                           ((3000, 1000, 5000) * 6, 256, 16, 64),    # 18 short rows: whole rows on chip
+                                           ((40000, 20000, 9000), 512, 16, 64)])    # chunked sampled threshold
 def test_decode_end_to_end(lens, k, H_q, ps):
     spec = small_decode_spec(lens, k, H_q, seed=len(lens) + k, ps=ps)
     inp = dsa_synth.make_decode(spec)
