@@ -146,6 +146,33 @@ dsa_status dsa_prefill(const void *q_idx, const float *q_scale, const void *k_id
                        dsa_dtype dtype, void *workspace, size_t ws_bytes, void *stream);
 
 /*
+ * dsa_prefill_host -- dsa_prefill for inputs and outputs in HOST memory
+ * (dtype DSA_E4M3 only; layouts as in dsa_prefill).  The pages define the
+ * computation; moving it from and to the host is this library's.
+ *   q_idx, q_scale, k_idx, k_scale, w, q, k, v: host inputs (page-locked memory
+ *     lets the copies overlap the computation; pageable memory still works,
+ *     with the copies serialised by the driver);
+ *   out, lse_out (nullable), idx_out (nullable): host outputs.
+ * The query rows move to the device, and their outputs back, pass by pass on
+ * two copy streams of the library's own (created once per device), while the
+ * indexer, top-k and attention of the previous pass run on `stream`; the keys
+ * and values move first.  The call is asynchronous: the outputs are complete
+ * once `stream` reaches the point after the call (e.g. cudaStreamSynchronize).
+ * Host buffers must stay valid until then.
+ * workspace: device memory of at least dsa_prefill_host_workspace_size(...)
+ * bytes (device copies of every input and output plus the prefill scratch),
+ * 256-byte aligned.  Errors: DSA_ERR_INVALID_ARG (null pointer, bad size),
+ * DSA_ERR_UNSUPPORTED (dtype or shape), DSA_ERR_WORKSPACE, DSA_ERR_CUDA.
+ */
+size_t dsa_prefill_host_workspace_size(int64_t T, int H_I, int d_I, int H_q, int d, int k_sel,
+                                       dsa_dtype dtype);
+dsa_status dsa_prefill_host(const void *q_idx, const float *q_scale, const void *k_idx,
+                            const float *k_scale, const void *w, const void *q, const void *k,
+                            const void *v, int64_t T, int H_I, int d_I, int H_q, int d, int k_sel,
+                            float sm_scale, void *out, float *lse_out, int32_t *idx_out,
+                            dsa_dtype dtype, void *workspace, size_t ws_bytes, void *stream);
+
+/*
  * dsa_decode -- one decode step of B sequences against paged caches (the
  * current token is already appended; DSA on the decode path, plus the FP8
  * index-key cache).

@@ -1,6 +1,7 @@
 // C entry points: argument validation, workspace carving, stage sequencing.
 // Everything numeric happens in the kernels; this file only checks and launches.
 #include <cmath>
+#include <mutex>
 
 #include "kernels.h"
 
@@ -83,6 +84,22 @@ cudaError_t run_attn(const void *q, const void *k, const void *v, const int32_t 
                                    idx, T, T, H_q, d, k_sel, sm_scale, (uint16_t *)out, lse, st);
 }
 
+// Attention of `rows` query rows (q, idx, out, lse already offset to the first
+// row) against the whole contiguous K/V of T rows; bf16, for dsa_prefill_host.
+cudaError_t run_attn_rows(const void *q, const void *k, const void *v, const int32_t *idx, int64_t T,
+                          int64_t rows, int H_q, int d, int k_sel, float sm_scale, void *out, float *lse,
+                          cudaStream_t st)
+{
+    if (sparse_attn_tc_supported(H_q, d)) {
+        cudaError_t e = launch_sparse_attn_tc((const uint16_t *)q, (const uint16_t *)k, (const uint16_t *)v,
+                                              T, T, nullptr, nullptr, 0, 0, 0, idx, rows, H_q, d, k_sel,
+                                              sm_scale, (uint16_t *)out, lse, nullptr, 1, nullptr, st);
+        if (e != cudaErrorNotSupported) return e;
+    }
+    return launch_sparse_attn_bf16((const uint16_t *)q, (const uint16_t *)k, (const uint16_t *)v, idx, rows, T,
+                                   H_q, d, k_sel, sm_scale, (uint16_t *)out, lse, st);
+}
+
 cudaError_t run_index(const void *q_idx, const float *q_scale, const void *k_idx,
                       const float *k_scale, const void *w, int64_t T, int H_I, int d_I,
                       int64_t row_begin, int64_t row_count, float *out, int64_t ld,
@@ -102,6 +119,58 @@ cudaError_t run_index(const void *q_idx, const float *q_scale, const void *k_idx
     }
     return launch_index_f32((const float *)q_idx, (const float *)k_idx, (const float *)w, T, H_I,
                             d_I, row_begin, row_count, out, ld, write_upper, st);
+}
+
+// Device mirrors of a prefill's inputs and outputs plus the prefill scratch,
+// carved from one workspace (E4M3 layouts), for dsa_prefill_host.
+struct HostPrefillLayout {
+    size_t q_idx, q_scale, w, q, k_idx, k_scale, k, v, out, lse, idx, scores, total;
+    int64_t R;
+    HostPrefillLayout(int64_t T, int H_I, int d_I, int H_q, int d, int k_sel)
+    {
+        R = prefill_rows_default(T);
+        size_t off = kWsHeader;
+        auto take = [&](size_t bytes) { size_t o = off; off += align_up(bytes, 256); return o; };
+        q_idx = take((size_t)T * H_I * d_I);
+        q_scale = take(sizeof(float) * (size_t)T);
+        w = take(2 * (size_t)T * H_I);
+        q = take(2 * (size_t)T * H_q * d);
+        k_idx = take((size_t)T * d_I);
+        k_scale = take(sizeof(float) * (size_t)T);
+        k = take(2 * (size_t)T * d);
+        v = take(2 * (size_t)T * d);
+        out = take(2 * (size_t)T * H_q * d);
+        lse = take(sizeof(float) * (size_t)T * H_q);
+        idx = take(sizeof(int32_t) * (size_t)T * k_sel);
+        scores = take(sizeof(float) * (size_t)R * T);
+        total = off;
+    }
+};
+
+// Per-device copy streams and events for dsa_prefill_host, created on first
+// use and kept for the life of the process.
+struct CopyEngine {
+    cudaStream_t h2d = nullptr, d2h = nullptr;
+    cudaEvent_t start = nullptr, in = nullptr, out = nullptr, done = nullptr;
+    bool ok = false;
+};
+
+CopyEngine *copy_engine()
+{
+    static CopyEngine engines[64];
+    static std::once_flag once[64];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+    std::call_once(once[dev], [dev] {
+        CopyEngine &c = engines[dev];
+        c.ok = cudaStreamCreateWithFlags(&c.h2d, cudaStreamNonBlocking) == cudaSuccess &&
+               cudaStreamCreateWithFlags(&c.d2h, cudaStreamNonBlocking) == cudaSuccess &&
+               cudaEventCreateWithFlags(&c.start, cudaEventDisableTiming) == cudaSuccess &&
+               cudaEventCreateWithFlags(&c.in, cudaEventDisableTiming) == cudaSuccess &&
+               cudaEventCreateWithFlags(&c.out, cudaEventDisableTiming) == cudaSuccess &&
+               cudaEventCreateWithFlags(&c.done, cudaEventDisableTiming) == cudaSuccess;
+    });
+    return engines[dev].ok ? &engines[dev] : nullptr;
 }
 
 }  // namespace
@@ -212,6 +281,94 @@ dsa_status dsa_prefill(const void *q_idx, const float *q_scale, const void *k_id
     }
     if (e == cudaSuccess)
         e = run_attn(q, k, v, idx, T, H_q, d, k_sel, sm_scale, out, lse_out, dtype, st);
+    return cuda_status(e);
+}
+
+size_t dsa_prefill_host_workspace_size(int64_t T, int H_I, int d_I, int H_q, int d, int k_sel,
+                                       dsa_dtype dtype)
+{
+    if (dtype != DSA_E4M3 || T <= 0 || H_I <= 0 || d_I <= 0 || H_q <= 0 || d <= 0 || k_sel <= 0) return 0;
+    return HostPrefillLayout(T, H_I, d_I, H_q, d, k_sel).total;
+}
+
+dsa_status dsa_prefill_host(const void *q_idx, const float *q_scale, const void *k_idx,
+                            const float *k_scale, const void *w, const void *q, const void *k,
+                            const void *v, int64_t T, int H_I, int d_I, int H_q, int d, int k_sel,
+                            float sm_scale, void *out, float *lse_out, int32_t *idx_out,
+                            dsa_dtype dtype, void *workspace, size_t ws_bytes, void *stream)
+{
+    if (dtype != DSA_E4M3) return DSA_ERR_UNSUPPORTED;
+    if (!q_idx || !q_scale || !k_idx || !k_scale || !w || !q || !k || !v || !out) return DSA_ERR_INVALID_ARG;
+    if (T <= 0 || H_I <= 0 || d_I <= 0 || H_q <= 0 || d <= 0 || k_sel <= 0 || k_sel > 65536 ||
+        !std::isfinite(sm_scale))
+        return DSA_ERR_INVALID_ARG;
+    if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u)) return DSA_ERR_WORKSPACE;
+    const HostPrefillLayout L(T, H_I, d_I, H_q, d, k_sel);
+    if (ws_bytes < L.total) return DSA_ERR_WORKSPACE;
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    // the device mirrors must pass the same checks as dsa_prefill's arguments
+    dsa_status s = check_index_args(ws + L.q_idx, (const float *)(ws + L.q_scale), ws + L.k_idx,
+                                    (const float *)(ws + L.k_scale), ws + L.w, T, H_I, d_I, dtype);
+    if (s != DSA_OK) return s;
+    s = check_attn_args(ws + L.q, ws + L.k, ws + L.v, (const int32_t *)(ws + L.idx), T, H_q, d, k_sel,
+                        ws + L.out, dtype);
+    if (s != DSA_OK) return s;
+    CopyEngine *ce = copy_engine();
+    if (!ce) return DSA_ERR_CUDA;
+    cudaStream_t st = as_stream(stream);
+    WsHeader *hdr = reinterpret_cast<WsHeader *>(ws);
+    float *scores = reinterpret_cast<float *>(ws + L.scores);
+    int32_t *idx = reinterpret_cast<int32_t *>(ws + L.idx);
+    const int64_t R = L.R;
+    const size_t qi_row = (size_t)H_I * d_I, q_row = 2 * (size_t)H_q * d;
+    auto h2d = [&](size_t off, const void *src, size_t bytes) {
+        return cudaMemcpyAsync(ws + off, src, bytes, cudaMemcpyHostToDevice, ce->h2d);
+    };
+    auto d2h = [&](void *dst, size_t off, size_t bytes) {
+        return cudaMemcpyAsync(dst, ws + off, bytes, cudaMemcpyDeviceToHost, ce->d2h);
+    };
+    // The copy streams start behind the caller's stream's earlier work; inputs move
+    // pass by pass ahead of the compute, and each pass's outputs leave while the next
+    // pass computes.
+    cudaError_t e = cudaMemsetAsync(hdr, 0, sizeof(WsHeader), st);
+    if (e == cudaSuccess) e = cudaEventRecord(ce->start, st);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(ce->h2d, ce->start, 0);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(ce->d2h, ce->start, 0);
+    if (e == cudaSuccess) e = h2d(L.k_idx, k_idx, (size_t)T * d_I);
+    if (e == cudaSuccess) e = h2d(L.k_scale, k_scale, sizeof(float) * (size_t)T);
+    if (e == cudaSuccess) e = h2d(L.k, k, 2 * (size_t)T * d);
+    if (e == cudaSuccess) e = h2d(L.v, v, 2 * (size_t)T * d);
+    if (e == cudaSuccess) e = h2d(L.q_scale, q_scale, sizeof(float) * (size_t)T);
+    if (e == cudaSuccess) e = h2d(L.w, w, 2 * (size_t)T * H_I);
+    for (int64_t r0 = 0; e == cudaSuccess && r0 < T; r0 += R) {
+        const int64_t n = T - r0 < R ? T - r0 : R;
+        e = h2d(L.q_idx + r0 * qi_row, static_cast<const uint8_t *>(q_idx) + r0 * qi_row, n * qi_row);
+        if (e == cudaSuccess) e = h2d(L.q + r0 * q_row, static_cast<const uint8_t *>(q) + r0 * q_row, n * q_row);
+        if (e == cudaSuccess) e = cudaEventRecord(ce->in, ce->h2d);
+        if (e == cudaSuccess) e = cudaStreamWaitEvent(st, ce->in, 0);
+        if (e == cudaSuccess)
+            e = run_index(ws + L.q_idx, (const float *)(ws + L.q_scale), ws + L.k_idx,
+                          (const float *)(ws + L.k_scale), ws + L.w, T, H_I, d_I, r0, n, scores, T, false,
+                          dtype, st);
+        if (e == cudaSuccess)
+            e = launch_topk_rows(scores, T, r0, nullptr, T, n, k_sel, idx + r0 * (int64_t)k_sel, hdr, st);
+        if (e == cudaSuccess)
+            e = run_attn_rows(ws + L.q + r0 * q_row, ws + L.k, ws + L.v, idx + r0 * (int64_t)k_sel, T, n, H_q,
+                              d, k_sel, sm_scale, ws + L.out + r0 * q_row,
+                              reinterpret_cast<float *>(ws + L.lse) + r0 * H_q, st);
+        if (e == cudaSuccess) e = cudaEventRecord(ce->out, st);
+        if (e == cudaSuccess) e = cudaStreamWaitEvent(ce->d2h, ce->out, 0);
+        if (e == cudaSuccess)
+            e = d2h(static_cast<uint8_t *>(out) + r0 * q_row, L.out + r0 * q_row, n * q_row);
+        if (e == cudaSuccess && lse_out)
+            e = d2h(lse_out + r0 * H_q, L.lse + sizeof(float) * r0 * H_q, sizeof(float) * n * H_q);
+        if (e == cudaSuccess && idx_out)
+            e = d2h(idx_out + r0 * (int64_t)k_sel, L.idx + sizeof(int32_t) * r0 * k_sel,
+                    sizeof(int32_t) * n * k_sel);
+    }
+    // the caller's stream completes only once the last outputs are on the host
+    if (e == cudaSuccess) e = cudaEventRecord(ce->done, ce->d2h);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(st, ce->done, 0);
     return cuda_status(e);
 }
 

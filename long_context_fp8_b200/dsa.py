@@ -25,6 +25,7 @@ STATUS = {0: "DSA_OK", 1: "DSA_ERR_INVALID_ARG", 2: "DSA_ERR_UNSUPPORTED", 3: "D
 # Every symbol include/dsa.h declares.
 EXPORTS = ("dsa_status_string", "dsa_version", "dsa_index_scores", "dsa_topk_workspace_size",
            "dsa_topk", "dsa_sparse_attn", "dsa_prefill_workspace_size", "dsa_prefill",
+           "dsa_prefill_host_workspace_size", "dsa_prefill_host",
            "dsa_decode_workspace_size", "dsa_decode", "dsa_decode_noalloc", "dsa_stream_status")
 
 
@@ -58,6 +59,9 @@ def load(path: str = LIB_PATH):
         "dsa_prefill_workspace_size": ([I64, I32, I32, I32, I32, I32, I32], SZ),
         "dsa_prefill": ([P, P, P, P, P, P, P, P, I64, I32, I32, I32, I32, I32, F, P, P, P, I32, P,
                          SZ, P], I32),
+        "dsa_prefill_host_workspace_size": ([I64, I32, I32, I32, I32, I32, I32], SZ),
+        "dsa_prefill_host": ([P, P, P, P, P, P, P, P, I64, I32, I32, I32, I32, I32, F, P, P, P, I32, P,
+                              SZ, P], I32),
         "dsa_decode_workspace_size": ([I32, I64, I32, I32, I32], SZ),
         "dsa_decode": ([P, P, P, P, P, P, P, P, P, P, I64, I32, I32, I32, I64, I32, I32, I32, I32,
                         I32, F, P, P, P, P, SZ, P], I32),
@@ -191,6 +195,43 @@ def dsa_prefill(inp: dict, k_sel: int, sm_scale=None, out=None, lse=None, idx_ou
                          k_sel, sm_scale, _p(out), _p(lse), _p(idx_out), dt, _p(ws), ws.numel(),
                          _stream(stream))
     _check("dsa_prefill", st)
+    return out, lse, idx_out
+
+
+def _h(t: Optional[torch.Tensor]):
+    """Host tensor pointer (contiguous, CPU; page-locked for overlapped copies)."""
+    if t is None:
+        return None
+    if t.is_cuda:
+        raise ValueError("dsa_prefill_host takes host (CPU) tensors")
+    if not t.is_contiguous():
+        raise ValueError("DSA entry points take contiguous tensors")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def prefill_host_workspace_size(T, H_I, d_I, H_q, d, k_sel) -> int:
+    return load().dsa_prefill_host_workspace_size(T, H_I, d_I, H_q, d, k_sel, DSA_E4M3)
+
+
+def dsa_prefill_host(inp: dict, k_sel: int, out, sm_scale=None, lse=None, idx_out=None, ws=None,
+                     stream=None):
+    """dsa_prefill with host (CPU) inputs and outputs: the library moves the query
+    rows in and the outputs back pass by pass, overlapped with the computation.
+    Asynchronous on `stream`; `out` (and lse / idx_out) hold the results once the
+    stream has reached this point."""
+    q_idx, q = inp["q_idx"], inp["q"]
+    T, H_I, d_I = q_idx.shape
+    _, H_q, d = q.shape
+    sm_scale = 1.0 / math.sqrt(d) if sm_scale is None else sm_scale
+    lib = load()
+    if ws is None:
+        ws = workspace(lib.dsa_prefill_host_workspace_size(T, H_I, d_I, H_q, d, k_sel, _idx_dtype(q_idx)),
+                       torch.device("cuda"))
+    st = lib.dsa_prefill_host(_h(q_idx), _h(inp["q_scale"]), _h(inp["k_idx"]), _h(inp["k_scale"]),
+                              _h(inp["w"]), _h(q), _h(inp["k"]), _h(inp["v"]), T, H_I, d_I, H_q, d, k_sel,
+                              sm_scale, _h(out), _h(lse), _h(idx_out), _idx_dtype(q_idx), _p(ws), ws.numel(),
+                              _stream(stream))
+    _check("dsa_prefill_host", st)
     return out, lse, idx_out
 
 

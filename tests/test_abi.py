@@ -90,6 +90,16 @@ def test_host_argument_errors(lib):
     assert lib.dsa_prefill(*args, None, 0, None) == WS
     assert lib.dsa_prefill(*args, fake, 1024, None) == WS
     assert lib.dsa_prefill(*args, P(0x1080), 1 << 30, None) == WS
+    # host-memory prefill: E4M3 only, null host pointer, missing / short workspace
+    hws = lib.dsa_prefill_host_workspace_size(1000, 64, 128, 16, 128, 64, 2)
+    assert hws > 1000 * (64 * 128 + 2 * 16 * 128 * 2)          # at least q_idx, q and out mirrors
+    assert lib.dsa_prefill_host_workspace_size(1000, 64, 128, 16, 128, 64, 0) == 0
+    assert lib.dsa_prefill_host(*args[:-1], 0, fake, hws, None) == UNSUP
+    bad = list(args)
+    bad[5] = None                                                # q
+    assert lib.dsa_prefill_host(*bad, fake, hws, None) == INVALID
+    assert lib.dsa_prefill_host(*args, None, hws, None) == WS
+    assert lib.dsa_prefill_host(*args, fake, hws - 256, None) == WS
     # decode: unsupported page size, short workspace
     dargs = [fake] * 10 + [100, 4, 64, 2, 256, 64, 128, 128, 128, 64, 0.1, fake, None, None]
     assert lib.dsa_decode(*dargs, fake, 10, None) == WS

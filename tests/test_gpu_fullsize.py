@@ -102,3 +102,24 @@ def test_decode_fullsize_sampled(name, seqs):
         hits_g += len(pos & set(idx_s[i].tolist()))
         hits_o += len(pos & set(ref["idx"][i].tolist()))
     assert abs(hits_g - hits_o) <= max(2, hits_o // 100), (hits_g, hits_o)
+
+
+@pytest.mark.parametrize("name", ["p16k_hq128"])
+def test_prefill_host_matches_device(name):
+    """dsa_prefill_host (inputs and outputs in page-locked host memory, moved
+    pass by pass alongside the computation) returns exactly what dsa_prefill
+    returns on device-resident inputs: same kernels, same passes."""
+    spec = dsa_synth.prefill_spec(name)
+    inp = dsa_synth.make_prefill(spec, device="cuda")
+    out_d, lse_d, idx_d = dsa.dsa_prefill(inp, spec.k, sm_of(spec.d))
+    torch.cuda.synchronize()
+    keys = ("q_idx", "q_scale", "k_idx", "k_scale", "w", "q", "k", "v")
+    host = {key: inp[key].cpu().pin_memory() for key in keys}
+    out_h = torch.empty(out_d.shape, dtype=out_d.dtype).pin_memory()
+    lse_h = torch.empty(lse_d.shape, dtype=lse_d.dtype).pin_memory()
+    idx_h = torch.empty(idx_d.shape, dtype=idx_d.dtype).pin_memory()
+    dsa.dsa_prefill_host(host, spec.k, out_h, sm_of(spec.d), lse=lse_h, idx_out=idx_h)
+    torch.cuda.synchronize()
+    assert torch.equal(idx_h, idx_d.cpu())
+    assert torch.equal(out_h, out_d.cpu())
+    assert torch.equal(lse_h, lse_d.cpu())
