@@ -340,7 +340,12 @@ dsa_status dsa_prefill_host(const void *q_idx, const float *q_scale, const void 
     if (e == cudaSuccess) e = h2d(L.v, v, 2 * (size_t)T * d);
     if (e == cudaSuccess) e = h2d(L.q_scale, q_scale, sizeof(float) * (size_t)T);
     if (e == cudaSuccess) e = h2d(L.w, w, 2 * (size_t)T * H_I);
-    for (int64_t r0 = 0; e == cudaSuccess && r0 < T; r0 += R) {
+    // Passes run from the last rows to the first: late rows carry the most work per
+    // copied byte (their causal rows are longest), so the copies stay ahead of the
+    // computation from the start, and the last pass's outputs are the cheapest.
+    const int64_t npass = ceil_div(T, R);
+    for (int64_t pi = npass - 1; e == cudaSuccess && pi >= 0; --pi) {
+        const int64_t r0 = pi * R;
         const int64_t n = T - r0 < R ? T - r0 : R;
         e = h2d(L.q_idx + r0 * qi_row, static_cast<const uint8_t *>(q_idx) + r0 * qi_row, n * qi_row);
         if (e == cudaSuccess) e = h2d(L.q + r0 * q_row, static_cast<const uint8_t *>(q) + r0 * q_row, n * q_row);
