@@ -294,6 +294,40 @@ __global__ void merge_splits_kernel(const float *__restrict__ part, int rows, in
     if (lse && d == 0) lse[row * H + h] = den > 0.f ? mx + logf(den) : -INFINITY;
 }
 
+// The same merge for D = 128 with one warp per (row, head): lane l owns
+// dimensions 4l .. 4l+3 (16-byte loads of each split's partial), eight heads
+// per 256-thread block, so a decode step's merge is a few waves of blocks.
+__global__ void __launch_bounds__(256)
+merge_splits_warp_kernel(const float *__restrict__ part, int rows, int splits, int H,
+                         uint16_t *__restrict__ out, float *__restrict__ lse)
+{
+    constexpr int D = 128;
+    const int64_t row = blockIdx.x;
+    const int h = blockIdx.y * 8 + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    if (h >= H) return;
+    const float *pl = part + (int64_t)rows * splits * H * D;
+    float mx = -INFINITY;
+    for (int i = 0; i < splits; ++i) mx = fmaxf(mx, __ldg(pl + (row * splits + i) * H + h));
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    float den = 0.f;
+    if (mx != -INFINITY) {
+        for (int i = 0; i < splits; ++i) {
+            const float li = __ldg(pl + (row * splits + i) * H + h);
+            const float wgt = li == -INFINITY ? 0.f : __expf(li - mx);
+            den += wgt;
+            const float4 o = __ldg(reinterpret_cast<const float4 *>(part + ((row * splits + i) * H + h) * (int64_t)D) + lane);
+            acc.x += wgt * o.x; acc.y += wgt * o.y; acc.z += wgt * o.z; acc.w += wgt * o.w;
+        }
+    }
+    const float inv = den > 0.f ? 1.f / den : 0.f;
+    uint2 packed;
+    packed.x = pack_bf16x2(acc.x * inv, acc.y * inv);
+    packed.y = pack_bf16x2(acc.z * inv, acc.w * inv);
+    *reinterpret_cast<uint2 *>(out + (row * H + h) * (int64_t)D + lane * 4) = packed;
+    if (lse && lane == 0) lse[row * H + h] = den > 0.f ? mx + logf(den) : -INFINITY;
+}
+
 // fp32 attention for small shapes: one warp per (query row, head).
 __global__ void sparse_attn_f32_kernel(const float *__restrict__ q, const float *__restrict__ k,
                                        const float *__restrict__ v, const int32_t *__restrict__ idx,
@@ -417,8 +451,8 @@ cudaError_t launch_merge_splits(const float *part, int rows, int splits, int H, 
 {
     if (rows <= 0 || splits <= 1) return cudaSuccess;
     if (d != 128) return cudaErrorNotSupported;
-    dim3 mg((unsigned)rows, (unsigned)H);
-    merge_splits_kernel<128><<<mg, 128, 0, st>>>(part, rows, splits, H, out, lse);
+    dim3 mg((unsigned)rows, (unsigned)((H + 7) / 8));
+    merge_splits_warp_kernel<<<mg, 256, 0, st>>>(part, rows, splits, H, out, lse);
     return cudaGetLastError();
 }
 
