@@ -247,10 +247,38 @@ __device__ void radix_select_smem(TopkSmem &sm, const uint32_t *keys, uint32_t n
         __syncthreads();
         find_bin(sm, nb, remaining);
         remaining -= sm.sh_above;
+        const uint32_t in_bin = sm.hist[sm.sh_bin];
         prefix |= sm.sh_bin << shift;
         pmask |= bmask << shift;
         lo = shift;
         __syncthreads();
+        if (lo > 0 && in_bin <= 64) {
+            // Few keys share the bin of the rank-th key: gather them (their order does
+            // not matter) and find it among them directly, instead of more passes:
+            // it is the x with  #{y > x} < remaining <= #{y >= x}.
+            uint32_t *bk = sm.hist;
+            if (tid == 0) sm.sh_count = 0u;
+            __syncthreads();
+            for (uint32_t j = tid; j < n; j += TK_THREADS) {
+                const uint32_t key = keys[j];
+                if ((key & pmask) == prefix) bk[atomicAdd(&sm.sh_count, 1u)] = key;
+            }
+            __syncthreads();
+            if (tid < 32) {
+                const uint32_t m = sm.sh_count;
+                for (uint32_t i = tid; i < m; i += 32) {
+                    const uint32_t x = bk[i];
+                    uint32_t gt = 0, ge = 0;
+                    for (uint32_t u = 0; u < m; ++u) { gt += bk[u] > x; ge += bk[u] >= x; }
+                    if (gt < remaining && remaining <= ge) { sm.sh_bin = x; sm.sh_above = remaining - gt; }
+                }
+            }
+            __syncthreads();
+            *thr = sm.sh_bin;
+            *need = sm.sh_above;
+            __syncthreads();
+            return;
+        }
     }
     *thr = prefix;
     *need = remaining;
@@ -473,7 +501,7 @@ __device__ __forceinline__ void hist_top11(uint32_t *hist, const uint32_t (&keys
 }
 
 // Threshold guess for a long row: the key of rank ~1.5 k (scaled to the
-// sample, at least 8) among 2048 evenly spaced samples, resolved to its top 22 bits (a
+// sample, at least 8) among 2048 evenly spaced samples, resolved by one radix pass (a
 // threshold at or below it).  Every thread calls it; every CTA working on the
 // same row computes the same value.
 __device__ uint32_t sampled_threshold(TopkSmem &sm, const float *row, int64_t n, int k)
@@ -491,7 +519,7 @@ __device__ uint32_t sampled_threshold(TopkSmem &sm, const float *row, int64_t n,
     const double want = 1.5 * (double)k * TK_SAMPLE / (double)n;
     const uint32_t rank = (uint32_t)min((double)TK_SAMPLE, max(8.0, ceil(want)));
     uint32_t tau, unused;
-    radix_select_smem(sm, sm.sample, TK_SAMPLE, rank, &tau, &unused, 2);
+    radix_select_smem(sm, sm.sample, TK_SAMPLE, rank, &tau, &unused, 1);
     return tau;
 }
 
