@@ -18,13 +18,15 @@
 //   warp 6    S issuer: S = Q K^T (kind::f16, M 128 heads, N 64 rows,
 //             K = 128 = 8 x 16) into one of two TMEM buffers, as soon as the
 //             K tile is in and the softmax has read that buffer's last S;
-//   warp 7    PV issuer: O += P V (V read MN-major straight from the gathered
-//             rows) into one of two TMEM O buffers (per item), as soon as P
-//             is written.  Two issuing threads keep the S MMAs from queueing
-//             behind the PV MMAs, which wait for the softmax;
+//   warp 7    PV issuer: O += P V (P from tensor memory, V read MN-major
+//             straight from the gathered rows) into one of two TMEM O buffers
+//             (per item), as soon as P is written.  Two issuing threads keep
+//             the S MMAs from queueing behind the PV MMAs, which wait for the
+//             softmax;
 //   warps 0-3 softmax: thread = head row.  Reads its S row from TMEM, masks
 //             unused slots, keeps the running max m and sum l in registers,
-//             writes P (bf16) to one of two shared buffers for the PV MMA.  O is rescaled
+//             writes P (bf16 pairs) to tensor memory, the A operand of the PV
+//             MMA (no shared-memory round trip, no proxy fence).  O is rescaled
 //             (a TMEM round trip) only when the block max exceeds m by more
 //             than 2^8 -- otherwise P <= 256 and m stays -- which is exact up
 //             to rounding.  At the end O / l and the log-sum-exp are written.
@@ -59,7 +61,6 @@ constexpr int AT_QTILE = 2 * AT_QHALF;       // Q of one item (32 KB)
 constexpr int AT_KHALF = AT_BLK * 128;       // one 64-column half of a 64-row K or V tile (8 KB)
 constexpr int AT_KTILE = 2 * AT_KHALF;       // a 64 x 128 bf16 tile (16 KB)
 constexpr int AT_STAGE = 2 * AT_KTILE;       // K + V of one block (32 KB)
-constexpr int AT_PTILE = AT_HEADS * 128;     // P of one block: 128 rows x 64 bf16 (16 KB)
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescaleThreshold = 8.f;     // log2 units
@@ -90,8 +91,7 @@ struct AttnTcArgs {
 struct AtSmem {
     static constexpr size_t q_off = 0;                                   // [2] Q tiles
     static constexpr size_t kv_off = q_off + 2 * AT_QTILE;                // [stages] K, V tiles
-    static constexpr size_t p_off = kv_off + (size_t)AT_STAGES * AT_STAGE; // [2] P tiles
-    static constexpr size_t valid_off = p_off + 2 * AT_PTILE;            // [stages][2] validity bits
+    static constexpr size_t valid_off = kv_off + (size_t)AT_STAGES * AT_STAGE; // [stages][2] validity bits
     static constexpr size_t ml_off = valid_off + AT_STAGES * 2 * 4;      // set 1's (m, l) per head
     static constexpr size_t bar_off = ml_off + 2 * AT_HEADS * 4;
     // qfull[2] qempty[2] kvfull[S] kvempty[S] sfull[2] sempty[2] pfull[2] pempty[2] ofull oempty mlfull mlempty
@@ -154,7 +154,6 @@ sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_con
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *Qs = smem + AtSmem::q_off;
     uint8_t *KVs = smem + AtSmem::kv_off;
-    uint8_t *Ps = smem + AtSmem::p_off;
     uint32_t *valid = reinterpret_cast<uint32_t *>(smem + AtSmem::valid_off);
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + AtSmem::bar_off);
     uint64_t *qfull = bars, *qempty = bars + 2, *kvfull = bars + 4, *kvempty = kvfull + AT_STAGES;
@@ -196,6 +195,7 @@ sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_con
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
     const uint32_t tS = tmem, tO = tmem + 2 * AT_BLK;    // S [0,128), O [128,384)
+    const uint32_t tP = tmem + 6 * AT_BLK;               // P [384,448): 32 columns of bf16 pairs per set
 
     if (warp >= 4 && warp < 8) {
         regs_dec<AT_REGS_LOW>();
@@ -355,13 +355,11 @@ sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_con
                         }
                         fence_proxy_async_smem();
                         tc_fence_after();
-                        const uint32_t pa = smem_u32(Ps + x * AT_PTILE);
                         const uint32_t va = smem_u32(KVs + st * AT_STAGE + AT_KTILE);
 #pragma unroll
                         for (int kk = 0; kk < AT_BLK / 16; ++kk) {
-                            const uint64_t ad = umma_desc_k_sw128_sbo(pa + kk * 32, 1024);
                             const uint64_t bd = umma_desc_mn_sw128(va + kk * 2048, AT_KHALF, 1024);
-                            umma_f16(tO + x * AT_D, ad, bd, idesc_o, (b > 1 || kk > 0) ? 1u : 0u);
+                            umma_f16_ts(tO + x * AT_D, tP + x * 32 + kk * 8, bd, idesc_o, (b > 1 || kk > 0) ? 1u : 0u);
                         }
                         umma_commit(&kvempty[st]);        // S(b) completed before P(b) existed
                         umma_commit(&pempty[x]);
@@ -386,7 +384,6 @@ sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_con
         const int h = q4 * 32 + lane;
         const uint32_t trow = (uint32_t)(q4 * 32) << 16;
         const uint32_t tSx = tS + x * AT_BLK, tOx = tO + x * AT_D;
-        uint8_t *Px = Ps + x * AT_PTILE;
         int qi = 0, g = 0, k = 0, mi = 0;   // items, blocks before this item, this set's blocks, merged items
         bool dead = false;
         for (int64_t it = it_begin; it < it_end; ++it) {
@@ -478,13 +475,9 @@ sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_con
                     }
                     tmem_wait_st();
                 }
-                // P row h: 64 keys = 128 bytes, 16-byte chunks swizzled by h % 8
-                uint8_t *prow = Px + h * 128;
-#pragma unroll
-                for (int c = 0; c < 8; ++c)
-                    *reinterpret_cast<uint4 *>(prow + ((c ^ (h & 7)) << 4)) =
-                        make_uint4(pk[c * 4], pk[c * 4 + 1], pk[c * 4 + 2], pk[c * 4 + 3]);
-                fence_proxy_async_smem();
+                // P row h into tensor memory: 64 keys as 32 columns of bf16 pairs
+                tmem_st32(tP + x * 32 + trow, pk);
+                tmem_wait_st();
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&pfull[x]);
