@@ -111,15 +111,22 @@ class ClockSampler:
 
 # ----------------------------------------------------------------------------- helpers
 
-def dist_setup():
+def dist_setup(backend=None):
+    """Process group from the torchrun environment.  `backend` defaults to
+    NCCL when a GPU is present, else gloo (the CPU tests of the multi-rank
+    bookkeeping)."""
     ws = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
+    if backend is None:
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
     if ws > 1:
         import datetime
-        torch.cuda.set_device(local)
-        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
-                                             device_id=torch.device("cuda", local))
+        kw = {}
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+            kw["device_id"] = torch.device("cuda", local)
+        torch.distributed.init_process_group(backend, timeout=datetime.timedelta(seconds=300), **kw)
     elif torch.cuda.is_available():
         torch.cuda.set_device(local)
     return ws, rank, local
@@ -131,11 +138,21 @@ def barrier(ws):
 
 
 def max_over_ranks(x: float, ws: int) -> float:
+    """Max of a per-rank step time over all ranks (one all-reduce of one
+    float; on the GPU under NCCL, on the host under gloo)."""
     if ws == 1:
         return x
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    on_gpu = torch.distributed.get_backend() == "nccl"
+    t = torch.tensor([x], dtype=torch.float64, device="cuda" if on_gpu else "cpu")
     torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
     return float(t.item())
+
+
+def whole_job_rate(ws: int, units_per_rank: float, step_ms_max: float) -> float:
+    """Units per second of the whole job: every rank processes its own
+    `units_per_rank` per step (weak scaling) and the job's step takes the
+    slowest rank's time."""
+    return ws * units_per_rank / (step_ms_max * 1e-3)
 
 
 def timed_steps(fn, steps, warmup, flush):
@@ -232,7 +249,7 @@ def sum_pairs(r0, n):
 
 def bench_prefill(args, dsa, spec, peaks, peak_kind, ws_n, rank):
     dev = torch.device("cuda")
-    inp = dsa_synth.make_prefill(dataclass_replace_seed(spec, rank), device=dev)
+    inp = dsa_synth.make_prefill(replica_spec(spec, rank), device=dev)
     torch.cuda.synchronize()
     T, k, H_q, d = spec.L, spec.k, spec.H_q, spec.d
     sm = 1.0 / math.sqrt(d)
@@ -287,7 +304,8 @@ def rows_per_pass_of(wsb, T, k):
     return min(R, ((T + 63) // 64) * 64)
 
 
-def dataclass_replace_seed(spec, rank):
+def replica_spec(spec, rank):
+    """Rank r's own independent problem: the same shapes, seed + 1000 r."""
     from dataclasses import replace
     return replace(spec, seed=spec.seed + 1000 * rank) if rank else spec
 
@@ -332,9 +350,7 @@ def decode_hbm_bytes(spec):
 
 def bench_decode(args, dsa, spec, peaks, ws_n, rank):
     dev = torch.device("cuda")
-    from dataclasses import replace
-    inp = dsa_synth.make_decode(replace(spec, seed=spec.seed + 1000 * rank) if rank else spec,
-                                device=dev)
+    inp = dsa_synth.make_decode(replica_spec(spec, rank), device=dev)
     inp.pop("needle_pos")
     torch.cuda.synchronize()
     maxc = max(spec.context_lens)
@@ -477,7 +493,7 @@ def main():
         us = dec["step_ms"] * 1e3
         gbs = dec["bytes"] / (dec["step_ms"] * 1e-3) / 1e9
         if rank == 0:
-            print(json.dumps({"metric": "DSA decode steps/s", "value": round(ws_n * 1e3 / dec["step_ms"], 1),
+            print(json.dumps({"metric": "DSA decode steps/s", "value": round(whole_job_rate(ws_n, 1, dec["step_ms"]), 1),
                               "unit": "steps/s", "n_gpus": ws_n, "steps": args.steps, "warmup": args.warmup,
                               "us_per_step": round(us, 2), "higher_is_better": True,
                               "config": {"workload": workload_config(spec, dspec)["decode_workload"]},
@@ -494,7 +510,7 @@ def main():
     dec = None if args.no_decode else bench_decode(args, dsa, dspec, peaks, ws_n, rank)
 
     T = spec.L
-    value = ws_n * T / (pre["step_ms"] * 1e-3)
+    value = whole_job_rate(ws_n, T, pre["step_ms"])
     br = pre["breakdown"]
     idx_peak = pre["fp8_peak"]
     roofline = {"bound": "tensor", "kernel": "indexer (FP8 e4m3 x e4m3 -> fp32)",
@@ -520,13 +536,13 @@ def main():
             "gpu_launches_per_step": pre["per_kernel"]}
     if pre["e2e"]:
         e = pre["e2e"]
-        line["e2e"] = {"value": round(ws_n * T / (e["step_ms"] * 1e-3), 1), "unit": "tokens/s",
+        line["e2e"] = {"value": round(whole_job_rate(ws_n, T, e["step_ms"]), 1), "unit": "tokens/s",
                        "h2d_bytes_per_step": e["h2d"], "d2h_bytes_per_step": e["d2h"],
                        "ms_per_step": round(e["step_ms"], 3)}
     if dec:
         us = dec["step_ms"] * 1e3
         gbs = dec["bytes"] / (dec["step_ms"] * 1e-3) / 1e9
-        line["decode"] = {"value": round(ws_n * 1e3 / dec["step_ms"], 1), "unit": "steps/s",
+        line["decode"] = {"value": round(whole_job_rate(ws_n, 1, dec["step_ms"]), 1), "unit": "steps/s",
                           "us_per_step": round(us, 2),
                           "roofline": {"bound": "hbm", "achieved": round(gbs, 1),
                                        "peak": peaks["hbm_gbs"], "unit": "GB/s",
