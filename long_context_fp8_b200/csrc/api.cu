@@ -452,7 +452,7 @@ dsa_status dsa_decode(const void *q_idx, const float *q_scale, const void *w, co
                                       (const uint16_t *)v_cache, num_pages * page_size, 0,
                                       block_table, context_lens, num_pages, max_pages_per_seq,
                                       page_size, idx, B, H_q, d, k_sel, sm_scale, (uint16_t *)out,
-                                      lse_out, part, tc_splits, hdr, st);
+                                      lse_out, part, tc_splits, hdr, st, /*chained=*/true);
             if (e == cudaSuccess) e = launch_merge_splits(part, B, tc_splits, H_q, d, (uint16_t *)out, lse_out, st);
             done = e != cudaErrorNotSupported;
         }

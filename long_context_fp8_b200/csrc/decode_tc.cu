@@ -168,6 +168,7 @@ decode_index_tc_kernel(const __grid_constant__ CUtensorMap kmap,
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int ps = a.page_size;
+    grid_dep_trigger();                              // the top-k may be scheduled (it waits for the scores)
 
     // per-sequence lengths and tile prefix sums (warp 0: lane l scans a block of sequences)
     if (warp == 0) {

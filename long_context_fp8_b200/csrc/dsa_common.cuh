@@ -30,6 +30,35 @@ __device__ __forceinline__ void record_error(WsHeader *h, dsa_status s, unsigned
     }
 }
 
+// Programmatic dependent launch.  A kernel launched with launch_chained() may
+// be scheduled while the kernel before it on the stream is still running; it
+// calls grid_dep_wait() before it reads what that kernel wrote or writes
+// anything that kernel might still read (the wait returns once the earlier
+// grid has completed and its writes are visible; without the launch
+// attribute it returns at once).  grid_dep_trigger() lets the next chained
+// kernel be scheduled before this one ends.
+__device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;\n" ::: "memory"); }
+__device__ __forceinline__ void grid_dep_trigger() { asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory"); }
+
+// Launches kernel<<<grid, block, smem, st>>>(args...) so that it may start
+// while the previous kernel on `st` finishes (see grid_dep_wait).
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_chained(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                                  cudaStream_t st, Args &&...args)
+{
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+
 __device__ __forceinline__ float bf16_to_f32(uint16_t b)
 {
     return __uint_as_float(((uint32_t)b) << 16);

@@ -75,13 +75,15 @@ cudaError_t launch_sparse_attn_f32(const float *q, const float *k, const float *
 
 // tcgen05 attention (sparse_attn_tc.cu): H a multiple of 128, d == 128.
 // Contiguous K/V when block_table is null (positions < T), else paged.
+// chained: launched so that it may start while the kernel before it on the
+// stream finishes (it waits for that kernel before reading idx).
 bool sparse_attn_tc_supported(int H, int d);
 cudaError_t launch_sparse_attn_tc(const uint16_t *q, const uint16_t *k, const uint16_t *v,
                                   int64_t kv_rows, int64_t T, const int32_t *block_table,
                                   const int32_t *context_lens, int64_t num_pages, int max_pages,
                                   int page_size, const int32_t *idx, int64_t rows, int H, int d,
                                   int ksel, float sm_scale, uint16_t *out, float *lse, float *part,
-                                  int splits, WsHeader *hdr, cudaStream_t st);
+                                  int splits, WsHeader *hdr, cudaStream_t st, bool chained = false);
 
 // ---- decode indexer (decode_tc.cu: tcgen05 + TMA; decode.cu: mma.sync) ----
 bool decode_index_tc_supported(int H, int page_size);

@@ -302,6 +302,7 @@ merge_splits_warp_kernel(const float *__restrict__ part, int rows, int splits, i
                          uint16_t *__restrict__ out, float *__restrict__ lse)
 {
     constexpr int D = 128;
+    grid_dep_wait();                                 // the attention's partials
     const int64_t row = blockIdx.x;
     const int h = blockIdx.y * 8 + (threadIdx.x >> 5);
     const int lane = threadIdx.x & 31;
@@ -452,7 +453,9 @@ cudaError_t launch_merge_splits(const float *part, int rows, int splits, int H, 
     if (rows <= 0 || splits <= 1) return cudaSuccess;
     if (d != 128) return cudaErrorNotSupported;
     dim3 mg((unsigned)rows, (unsigned)((H + 7) / 8));
-    merge_splits_warp_kernel<<<mg, 256, 0, st>>>(part, rows, splits, H, out, lse);
+    cudaError_t e = launch_chained(merge_splits_warp_kernel, mg, dim3(256), 0, st, part, rows, splits, H,
+                                   out, lse);
+    if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
 

@@ -193,6 +193,8 @@ sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_con
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
+    grid_dep_wait();                                 // chained launch: the index lists of the kernel before
+    grid_dep_trigger();
     const uint32_t tmem = *tmem_slot;
     const uint32_t tS = tmem, tO = tmem + 2 * AT_BLK;    // S [0,128), O [128,384)
     const uint32_t tP = tmem + 6 * AT_BLK;               // P [384,448): 32 columns of bf16 pairs per set
@@ -602,7 +604,7 @@ cudaError_t launch_sparse_attn_tc(const uint16_t *q, const uint16_t *k, const ui
                                   const int32_t *context_lens, int64_t num_pages, int max_pages,
                                   int page_size, const int32_t *idx, int64_t rows, int H, int d,
                                   int ksel, float sm_scale, uint16_t *out, float *lse, float *part,
-                                  int splits, WsHeader *hdr, cudaStream_t st)
+                                  int splits, WsHeader *hdr, cudaStream_t st, bool chained)
 {
     if (rows <= 0) return cudaSuccess;
     if (!sparse_attn_tc_supported(H, d) || kv_rows >= ((int64_t)1 << 31) ||
@@ -635,7 +637,12 @@ cudaError_t launch_sparse_attn_tc(const uint16_t *q, const uint16_t *k, const ui
     e = cudaFuncSetAttribute(sparse_attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     const unsigned grid = (unsigned)std::min<int64_t>(a.items, sms);
-    sparse_attn_tc_kernel<<<grid, AT_THREADS, smem, st>>>(qmap, kmap, vmap, a);
+    if (chained) {
+        e = launch_chained(sparse_attn_tc_kernel, dim3(grid), dim3(AT_THREADS), smem, st, qmap, kmap, vmap, a);
+        if (e != cudaSuccess) return e;
+    } else {
+        sparse_attn_tc_kernel<<<grid, AT_THREADS, smem, st>>>(qmap, kmap, vmap, a);
+    }
     return cudaGetLastError();
 }
 

@@ -629,6 +629,8 @@ topk_split_collect_kernel(const float *__restrict__ scores, int64_t ld, const in
 {
     extern __shared__ __align__(16) uint8_t smem_raw[];
     TopkSmem &sm = *reinterpret_cast<TopkSmem *>(smem_raw);
+    grid_dep_wait();                                 // the scores of the kernel before
+    grid_dep_trigger();
     const int64_t r = blockIdx.y;
     const int64_t n = split_len(lens, max_len, r);
     const int64_t c0 = (int64_t)blockIdx.x * TS_CHUNK;
@@ -653,6 +655,8 @@ topk_split_final_kernel(const float *__restrict__ scores, int64_t ld, const int3
 {
     extern __shared__ __align__(16) uint8_t smem_raw[];
     TopkSmem &sm = *reinterpret_cast<TopkSmem *>(smem_raw);
+    grid_dep_wait();                                 // the collect kernel's slots
+    grid_dep_trigger();
     const int64_t r = blockIdx.x;
     const int tid = threadIdx.x;
     int32_t *out = idx + r * (int64_t)k;
@@ -763,9 +767,12 @@ cudaError_t launch_topk_split(const float *scores, int64_t ld, const int32_t *le
     e = cudaFuncSetAttribute(topk_split_final_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     dim3 grid((unsigned)chunks, (unsigned)rows);
-    topk_split_collect_kernel<<<grid, TK_THREADS, smem, st>>>(scores, ld, lens, max_len, k, ws, vec_ok);
-    topk_split_final_kernel<<<(unsigned)rows, TK_THREADS, smem, st>>>(scores, ld, lens, max_len, k, ws, idx,
-                                                                      hdr, vec_ok);
+    e = launch_chained(topk_split_collect_kernel, grid, dim3(TK_THREADS), smem, st, scores, ld, lens,
+                       max_len, k, ws, vec_ok);
+    if (e != cudaSuccess) return e;
+    e = launch_chained(topk_split_final_kernel, dim3((unsigned)rows), dim3(TK_THREADS), smem, st, scores,
+                       ld, lens, max_len, k, ws, idx, hdr, vec_ok);
+    if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
 

@@ -346,3 +346,37 @@ def test_topk_long_rows_sampled_threshold(k):
     sc[1, 40000:] += 3.0                      # the best keys all at the end
     sc[2, :100] += 3.0                        # ... or all at the start
     _topk_check(sc, k, row_begin=T - 6)
+
+
+def test_decode_cuda_graph_replay_matches_eager():
+    """The decode step captured in a CUDA graph (the kernels after the indexer
+    are launched so that each may start while the one before it finishes)
+    replays to exactly the eager step's outputs, replay after replay."""
+    spec = small_decode_spec((40000, 20000, 9000, 3000), k=512, H_q=128, seed=5)
+    inp = dsa_synth.make_decode(spec)
+    dev = to_dev(inp)
+    maxc, sm = 40000, sm_of(128)
+    lib = dsa.load()
+    ws = dsa.workspace(lib.dsa_decode_workspace_size(len(spec.context_lens), maxc, 128, 128, spec.k), "cuda")
+    out0, lse0, idx0 = dsa.dsa_decode(dev, spec.k, maxc, sm, ws=ws)
+    assert dsa.dsa_stream_status(ws) == 0
+    out, lse, idx = torch.empty_like(out0), torch.empty_like(lse0), torch.empty_like(idx0)
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        dsa.dsa_decode(dev, spec.k, maxc, sm, out=out, lse=lse, idx_out=idx, ws=ws)
+    torch.cuda.current_stream().wait_stream(side)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        dsa.dsa_decode(dev, spec.k, maxc, sm, out=out, lse=lse, idx_out=idx, ws=ws)
+    for _ in range(3):
+        out.zero_()
+        lse.zero_()
+        idx.fill_(-7)
+        g.replay()
+        torch.cuda.synchronize()
+        assert torch.equal(idx, idx0)
+        assert torch.equal(out, out0)
+        assert torch.equal(lse, lse0)
+    assert dsa.dsa_stream_status(ws) == 0
+    del g
