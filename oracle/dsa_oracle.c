@@ -23,6 +23,21 @@
  *     lse = max z + log sum exp(z - max z), natural log.
  *  4. Decode: stages 1-3 for one query per sequence whose context (already
  *     holding the current token) lives in paged caches.
+ *  5. Sliding window with top-k ("DeepSeek-V4 百万 token 上下文的工程实现",
+ *     section on the sliding-window KV cache and the hybrid strategy: the most
+ *     recent 4K-16K tokens keep their full KV, older tokens are kept only as
+ *     far as an importance score retains them): the W most recent positions
+ *     of a query are always attended, and stage 2 selects min(k, t+1-W) of
+ *     the older positions 0..t-W by indexer score.  Output: the top-k part in
+ *     ascending position, then the window positions, then -1 up to k + W.
+ *  6. FP8 quantisation of the indexer's query and key ("DeepSeek-V3.2-Exp
+ *     DSA 技术深度解析", section 1: FP8 indexer; the hotdry page's section on
+ *     FP8 decoding) and the append of a new token to the paged caches: one
+ *     fp32 scale per token, scale = amax / 448 (1 when that is 0), code =
+ *     the E4M3 value nearest to x / scale, ties to an even code, magnitudes
+ *     past 448 saturating to 448.  The scale and the quotient are fp32
+ *     operations (the precision the library computes them in), so that the
+ *     integer codes are decided the same way on both sides.
  *
  * Number formats are decoded from their published definitions:
  *   E4M3 (OCP 8-bit floating point, "E4M3FN"): 1 sign, 4 exponent (bias 7),
@@ -33,12 +48,18 @@
  * Build: gcc -O2 -fopenmp -shared -fPIC (no fast-math: every sum is taken in
  * the order written here, in double precision).
  */
+#include <float.h>
 #include <math.h>
 #include <stdint.h>
 #include <stdlib.h>
 #include <string.h>
 
 enum { OR_F32 = 0, OR_BF16 = 1, OR_E4M3 = 2 };
+
+/* Stage 6's fp32 operations must round once, in single precision. */
+#if FLT_EVAL_METHOD != 0
+#error "the quantiser needs FLT_EVAL_METHOD == 0 (single-precision float arithmetic)"
+#endif
 
 /* ---------------- number formats ---------------- */
 
@@ -209,6 +230,48 @@ int dsa_or_topk(const double *scores, int64_t ld, const int64_t *rows, int64_t n
     return err;
 }
 
+/* Stage 5 for one row of n = t+1 candidates: positions before the window
+ * (0..n-1-window) compete by score for k slots, the last `window` positions
+ * are taken as they are.  out[k + window]: the selected older positions
+ * ascending, the window positions ascending, then -1. */
+static void select_row_window(const double *scores, int64_t n, int k, int window, int32_t *out,
+                              cand_t *buf)
+{
+    int64_t older = n > window ? n - window : 0;
+    int64_t m = older < k ? older : k;
+    if (older > 0) select_row(scores, older, k, out, buf);
+    int64_t i = m;
+    for (int64_t s = older; s < n; ++s) out[i++] = (int32_t)s;
+    for (; i < (int64_t)k + window; ++i) out[i] = -1;
+}
+
+/*
+ * Window-plus-top-k selection of each score row (stage 5): row r belongs to
+ * query position rows[r]; idx_out[r*(k+window) + i] as select_row_window.
+ */
+int dsa_or_topk_window(const double *scores, int64_t ld, const int64_t *rows, int64_t nrows, int k,
+                       int window, int32_t *idx_out)
+{
+    int err = 0;
+    const int64_t width = (int64_t)k + window;
+#pragma omp parallel
+    {
+        int64_t maxn = 0;
+        for (int64_t r = 0; r < nrows; ++r) if (rows[r] + 1 > maxn) maxn = rows[r] + 1;
+        cand_t *buf = (cand_t *)malloc(sizeof(cand_t) * (size_t)(maxn > 0 ? maxn : 1));
+        if (!buf) {
+#pragma omp atomic write
+            err = -1;
+        } else {
+#pragma omp for schedule(dynamic, 4)
+            for (int64_t r = 0; r < nrows; ++r)
+                select_row_window(scores + r * ld, rows[r] + 1, k, window, idx_out + r * width, buf);
+        }
+        free(buf);
+    }
+    return err;
+}
+
 /* ---------------- stage 3: attention over the selected set ---------------- */
 
 /* Attention of one query token (H heads of dimension D) over the rows listed
@@ -283,14 +346,17 @@ int dsa_or_sparse_attn(const void *q, const void *K, const void *V, int dtype, c
  * physical page bt[b*max_pages + s/ps], slot s%ps.
  *   q_idx  e4m3 [B,H_I,D_I], q_scale [B], w bf16 [B,H_I], q bf16 [B,H_q,D]
  *   kidx   e4m3 [P,ps,D_I], kscale f32 [P,ps], kc/vc bf16 [P,ps,D]
- * Outputs: scores_out [B, ld] (nullable; entries s < n), idx_out [B,k]
- * (positions, ascending, -1 padded), out [B,H_q,D], lse [B,H_q] (nullable).
+ * window > 0 applies stage 5: the last `window` positions are always
+ * attended and the top-k runs over the positions before them.
+ * Outputs: scores_out [B, ld] (nullable; entries s < n), idx_out
+ * [B, k+window] (positions, ascending, -1 padded), out [B,H_q,D], lse [B,H_q]
+ * (nullable).
  */
 int dsa_or_decode(const uint8_t *q_idx, const float *q_scale, const uint16_t *w,
                   const uint16_t *q, const uint8_t *kidx, const float *kscale,
                   const uint16_t *kc, const uint16_t *vc, const int32_t *bt,
                   const int32_t *ctx, int B, int max_pages, int ps, int H_I, int D_I,
-                  int H_q, int D, int k, double sm, double *scores_out, int64_t ld,
+                  int H_q, int D, int k, int window, double sm, double *scores_out, int64_t ld,
                   int32_t *idx_out, double *out, double *lse)
 {
     int err = 0;
@@ -300,8 +366,9 @@ int dsa_or_decode(const uint8_t *q_idx, const float *q_scale, const uint16_t *w,
         double *q_row = (double *)malloc(sizeof(double) * (size_t)H_I * D_I);
         double *w_row = (double *)malloc(sizeof(double) * (size_t)H_I);
         cand_t *buf = (cand_t *)malloc(sizeof(cand_t) * (size_t)(n > 0 ? n : 1));
-        int64_t *koff = (int64_t *)malloc(sizeof(int64_t) * (size_t)k);
-        double *z = (double *)malloc(sizeof(double) * (size_t)k);
+        const int width = k + window;
+        int64_t *koff = (int64_t *)malloc(sizeof(int64_t) * (size_t)width);
+        double *z = (double *)malloc(sizeof(double) * (size_t)width);
         if (!sc || !q_row || !w_row || !buf || !koff || !z) err = -1;
         if (!err) {
             double sq = q_scale[b];
@@ -321,10 +388,11 @@ int dsa_or_decode(const uint8_t *q_idx, const float *q_scale, const uint16_t *w,
                 }
             }
             if (scores_out) for (int64_t s = 0; s < n; ++s) scores_out[(int64_t)b * ld + s] = sc[s];
-            int32_t *sel = idx_out + (int64_t)b * k;
-            select_row(sc, n, k, sel, buf);
+            int32_t *sel = idx_out + (int64_t)b * width;
+            if (window > 0) select_row_window(sc, n, k, window, sel, buf);
+            else select_row(sc, n, k, sel, buf);
             int64_t m = 0;
-            for (int i = 0; i < k; ++i) {
+            for (int i = 0; i < width; ++i) {
                 if (sel[i] < 0) continue;
                 int64_t page = bt[(int64_t)b * max_pages + sel[i] / ps];
                 koff[m++] = (page * ps + sel[i] % ps) * D;
@@ -337,4 +405,92 @@ int dsa_or_decode(const uint8_t *q_idx, const float *q_scale, const uint16_t *w,
         free(sc); free(q_row); free(w_row); free(buf); free(koff); free(z);
     }
     return err;
+}
+
+/* ---------------- stage 6: FP8 quantisation and cache append ---------------- */
+
+/* The E4M3 code nearest to y: codes 0x00..0x7E are the non-negative finite
+ * values in increasing order, so the two neighbours of |y| are found by a
+ * scan; a tie goes to the even code (last mantissa bit 0); magnitudes past
+ * the largest finite value (448) saturate to it.  The sign bit follows y's
+ * sign (so -0 and negatives that round to zero give 0x80).  y must not be
+ * NaN. */
+uint8_t dsa_or_e4m3_encode(float y)
+{
+    double a = fabs((double)y);
+    int lo = 0;
+    for (int c = 0; c <= 0x7E; ++c)
+        if (dsa_or_e4m3((uint8_t)c) <= a) lo = c;
+    int mag;
+    if (lo == 0x7E || dsa_or_e4m3((uint8_t)lo) == a) {
+        mag = lo;
+    } else {
+        double below = a - dsa_or_e4m3((uint8_t)lo), above = dsa_or_e4m3((uint8_t)(lo + 1)) - a;
+        if (below < above) mag = lo;
+        else if (above < below) mag = lo + 1;
+        else mag = (lo % 2 == 0) ? lo : lo + 1;
+    }
+    return (uint8_t)((signbit(y) ? 0x80 : 0x00) | mag);
+}
+
+/* Per-token scale and codes of one row of `cols` values. */
+static void quantize_row(const void *x, int dtype, int64_t off, int64_t cols, uint8_t *codes,
+                         float *scale)
+{
+    float amax = 0.0f;
+    for (int64_t j = 0; j < cols; ++j) {
+        float m = fabsf((float)load_elem(x, dtype, off + j));
+        if (m > amax) amax = m;
+    }
+    float s = amax / 448.0f;
+    if (!(s > 0.0f)) s = 1.0f;
+    *scale = s;
+    for (int64_t j = 0; j < cols; ++j) {
+        float v = (float)load_elem(x, dtype, off + j);
+        float y = v / s;
+        codes[j] = dsa_or_e4m3_encode(y);
+    }
+}
+
+/*
+ * FP8 E4M3 quantisation with one scale per row: x [rows, cols] of dtype
+ * OR_F32 or OR_BF16 (finite values) -> codes uint8 [rows, cols], scale f32
+ * [rows].  Returns 0.
+ */
+int dsa_or_quantize_e4m3(const void *x, int dtype, int64_t rows, int64_t cols, uint8_t *codes,
+                         float *scale)
+{
+#pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < rows; ++r) quantize_row(x, dtype, r * cols, cols, codes + r * cols, scale + r);
+    return 0;
+}
+
+/*
+ * Append N new tokens to the paged caches.  Token i goes to sequence seq[i]
+ * at position pos[i], i.e. physical page bt[seq[i]*max_pages + pos[i]/ps],
+ * slot pos[i]%ps: its index key kidx_new[i, 0..D_I) (OR_F32 or OR_BF16) is
+ * quantised into kidx_cache/kscale_cache (stage 6), and its bf16 K and V rows
+ * are copied into k_cache/v_cache.  bt is [B, max_pages].  Returns 0, or -2
+ * (and stops) at the first token whose sequence, position or page id is out
+ * of range.
+ */
+int dsa_or_cache_append(const void *kidx_new, int kdt, const uint16_t *k_new, const uint16_t *v_new,
+                        const int32_t *seq, const int32_t *pos, int64_t N, int B, const int32_t *bt,
+                        int max_pages, int64_t num_pages, int ps, int D_I, int D,
+                        uint8_t *kidx_cache, float *kscale_cache, uint16_t *k_cache,
+                        uint16_t *v_cache)
+{
+    for (int64_t i = 0; i < N; ++i) {
+        int64_t p = pos[i];
+        if (seq[i] < 0 || seq[i] >= B || p < 0 || p >= (int64_t)max_pages * ps) return -2;
+        int64_t page = bt[(int64_t)seq[i] * max_pages + p / ps];
+        if (page < 0 || page >= num_pages) return -2;
+        int64_t slot = page * ps + p % ps;
+        quantize_row(kidx_new, kdt, i * D_I, D_I, kidx_cache + slot * D_I, kscale_cache + slot);
+        for (int c = 0; c < D; ++c) {
+            k_cache[slot * D + c] = k_new[i * D + c];
+            v_cache[slot * D + c] = v_new[i * D + c];
+        }
+    }
+    return 0;
 }

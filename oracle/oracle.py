@@ -55,8 +55,17 @@ def load(path: Optional[str] = None):
     lib.dsa_or_sparse_attn.argtypes = [P, P, P, I32, P, I64, I32, I32, I32, D, P, P]
     lib.dsa_or_sparse_attn.restype = I32
     lib.dsa_or_decode.argtypes = [P, P, P, P, P, P, P, P, P, P, I32, I32, I32, I32, I32,
-                                  I32, I32, I32, D, P, I64, P, P, P]
+                                  I32, I32, I32, I32, D, P, I64, P, P, P]
     lib.dsa_or_decode.restype = I32
+    lib.dsa_or_topk_window.argtypes = [P, I64, P, I64, I32, I32, P]
+    lib.dsa_or_topk_window.restype = I32
+    lib.dsa_or_e4m3_encode.argtypes = [ctypes.c_float]
+    lib.dsa_or_e4m3_encode.restype = ctypes.c_uint8
+    lib.dsa_or_quantize_e4m3.argtypes = [P, I32, I64, I64, P, P]
+    lib.dsa_or_quantize_e4m3.restype = I32
+    lib.dsa_or_cache_append.argtypes = [P, I32, P, P, P, P, I64, I32, P, I32, I64, I32, I32, I32,
+                                        P, P, P, P]
+    lib.dsa_or_cache_append.restype = I32
     if path == _LIB:
         _lib = lib
     return lib
@@ -161,6 +170,64 @@ def topk(scores, rows, k, lib=None) -> np.ndarray:
     return out
 
 
+def topk_window(scores, rows, k, window, lib=None) -> np.ndarray:
+    """Sliding window plus top-k of each row (stage 5 of the oracle header);
+    int32 [nrows, k + window]: the top-k of positions 0..rows[r]-window
+    ascending, then the window positions, then -1."""
+    lib = lib or load()
+    s = np.ascontiguousarray(np.asarray(scores, dtype=np.float64))
+    rows = np.ascontiguousarray(np.asarray(rows, dtype=np.int64))
+    out = np.empty((rows.size, k + window), dtype=np.int32)
+    rc = lib.dsa_or_topk_window(_ptr(s), s.shape[1], _ptr(rows), rows.size, k, window, _ptr(out))
+    assert rc == 0
+    return out
+
+
+def e4m3_encode(y: float) -> int:
+    """E4M3 code nearest to the fp32 value y (stage 6: ties to even, saturating)."""
+    return int(load().dsa_or_e4m3_encode(float(y)))
+
+
+def quantize_e4m3(x, lib=None):
+    """Per-row FP8 quantisation (stage 6) of fp32 or bf16 ``x[rows, ...]``:
+    (uint8 codes of x's shape, fp32 scale[rows])."""
+    lib = lib or load()
+    dt = _val_dtype(x)
+    a = _np(x)
+    if dt == OR_F32:
+        a = np.ascontiguousarray(a.astype(np.float32))
+    rows = a.shape[0]
+    cols = int(np.prod(a.shape[1:])) if a.ndim > 1 else 1
+    codes = np.empty(a.shape, dtype=np.uint8)
+    scale = np.empty(rows, dtype=np.float32)
+    rc = lib.dsa_or_quantize_e4m3(_ptr(a), dt, rows, cols, _ptr(codes), _ptr(scale))
+    assert rc == 0
+    return codes, scale
+
+
+def cache_append(caches: dict, kidx_new, k_new, v_new, seq, pos, block_table, lib=None) -> int:
+    """Append tokens to copies of the paged caches (stage 6).  ``caches`` holds
+    numpy arrays kidx_cache/kscale_cache/k_cache/v_cache (bf16 as uint16
+    bits), updated in place.  Returns the oracle's status (0, or -2 for an
+    out-of-range sequence, position or page)."""
+    lib = lib or load()
+    dt = _val_dtype(kidx_new)
+    kn = _np(kidx_new)
+    if dt == OR_F32:
+        kn = np.ascontiguousarray(kn.astype(np.float32))
+    kk, vv = _np(k_new), _np(v_new)
+    sq, ps_ = _np(seq, np.int32), _np(pos, np.int32)
+    bt = _np(block_table, np.int32)
+    kic, ksc, kc, vc = (caches[n] for n in ("kidx_cache", "kscale_cache", "k_cache", "v_cache"))
+    for a in (kic, ksc, kc, vc):
+        assert a.flags.c_contiguous
+    P, ps, D_I = kic.shape
+    D = kc.shape[2]
+    return lib.dsa_or_cache_append(_ptr(kn), dt, _ptr(kk), _ptr(vv), _ptr(sq), _ptr(ps_), sq.size,
+                                   bt.shape[0], _ptr(bt), bt.shape[1], P, ps, D_I, D, _ptr(kic),
+                                   _ptr(ksc), _ptr(kc), _ptr(vc))
+
+
 def sparse_attn(q, K, V, idx, rows, sm_scale, lib=None, compact=False):
     """Attention of query rows over their selected K/V rows (stage 3); (out, lse) fp64.
 
@@ -187,8 +254,9 @@ def sparse_attn(q, K, V, idx, rows, sm_scale, lib=None, compact=False):
     return out, lse
 
 
-def decode(inp: dict, k: int, sm_scale: float, want_scores: bool = False, lib=None):
-    """One decode step over paged caches (stage 4); returns dict idx/out/lse[/scores]."""
+def decode(inp: dict, k: int, sm_scale: float, want_scores: bool = False, lib=None, window: int = 0):
+    """One decode step over paged caches (stage 4; with window > 0, stage 5's
+    selection); returns dict idx [B, k+window]/out/lse[/scores]."""
     lib = lib or load()
     q_idx, q_scale, w, q = _np(inp["q_idx"]), _np(inp["q_scale"], np.float32), _np(inp["w"]), _np(inp["q"])
     kidx, ksc = _np(inp["kidx_cache"]), _np(inp["kscale_cache"], np.float32)
@@ -199,12 +267,12 @@ def decode(inp: dict, k: int, sm_scale: float, want_scores: bool = False, lib=No
     ps = kidx.shape[1]
     ld = int(ctx.max()) if want_scores else 0
     scores = np.full((B, ld), np.nan) if want_scores else None
-    idx = np.empty((B, k), dtype=np.int32)
+    idx = np.empty((B, k + window), dtype=np.int32)
     out = np.empty((B, H_q, D), dtype=np.float64)
     lse = np.empty((B, H_q), dtype=np.float64)
     rc = lib.dsa_or_decode(_ptr(q_idx), _ptr(q_scale), _ptr(w), _ptr(q), _ptr(kidx), _ptr(ksc),
                            _ptr(kc), _ptr(vc), _ptr(bt), _ptr(ctx), B, bt.shape[1], ps, H_I,
-                           D_I, H_q, D, k, float(sm_scale), _ptr(scores), ld, _ptr(idx),
+                           D_I, H_q, D, k, window, float(sm_scale), _ptr(scores), ld, _ptr(idx),
                            _ptr(out), _ptr(lse))
     assert rc == 0
     res = dict(idx=idx, out=out, lse=lse)
@@ -213,10 +281,11 @@ def decode(inp: dict, k: int, sm_scale: float, want_scores: bool = False, lib=No
     return res
 
 
-def prefill(inp: dict, k: int, sm_scale: float, rows, lib=None):
-    """Stages 1-3 for the listed query rows: dict scores/idx/out/lse."""
+def prefill(inp: dict, k: int, sm_scale: float, rows, lib=None, window: int = 0):
+    """Stages 1-3 (with window > 0, stage 5's selection) for the listed query
+    rows: dict scores/idx/out/lse."""
     rows = np.asarray(rows, dtype=np.int64)
     sc = index_scores(inp["q_idx"], inp["q_scale"], inp["k_idx"], inp["k_scale"], inp["w"], rows, lib)
-    idx = topk(sc, rows, k, lib)
+    idx = topk_window(sc, rows, k, window, lib) if window > 0 else topk(sc, rows, k, lib)
     out, lse = sparse_attn(inp["q"], inp["k"], inp["v"], idx, rows, sm_scale, lib)
     return dict(scores=sc, idx=idx, out=out, lse=lse)

@@ -311,3 +311,214 @@ def test_needles_are_selected():
     res = oracle.prefill(inp, 16, 0.25, src)
     hits = [p in set(res["idx"][i].tolist()) for i, p in enumerate(pos)]
     assert np.mean(hits) >= 0.5
+
+
+# ---------------------------------------------------------------- FP8 quantisation (stage 6)
+
+def _finite_codes():
+    return [c for c in range(256) if c not in (0x7F, 0xFF)]
+
+
+def test_e4m3_encode_round_trips_every_code():
+    """Every finite code's own value encodes back to that code (-0 to 0x80)."""
+    for c in _finite_codes():
+        v = oracle.e4m3(c)
+        assert oracle.e4m3_encode(v) == c, hex(c)
+
+
+def test_e4m3_encode_golden_points():
+    g = _golden("e4m3_rounding_points.json")
+    for val, code, why in g["encode"]:
+        assert oracle.e4m3_encode(val) == int(code, 16), why
+
+
+def test_e4m3_encode_matches_torch_conversion():
+    """The library's float -> float8_e4m3fn conversion (round to nearest even) on
+    values inside the finite range: random magnitudes over every binade, the
+    exact midpoints between neighbouring codes, and values just beside them."""
+    rng = np.random.default_rng(8)
+    vals = [rng.standard_normal(20000).astype(np.float32) * np.float32(2.0) ** rng.integers(-14, 9, 20000)]
+    pos = np.array([oracle.e4m3(c) for c in range(0x7F)])
+    mid = ((pos[1:] + pos[:-1]) / 2).astype(np.float32)
+    vals += [mid, -mid, np.nextafter(mid, np.float32(0)), np.nextafter(mid, np.float32(1e9))]
+    x = np.concatenate(vals).astype(np.float32)
+    x = np.clip(x, -448.0, 448.0).astype(np.float32)
+    ref = torch.from_numpy(x).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    got = np.array([oracle.e4m3_encode(v) for v in x], np.uint8)
+    bad = np.nonzero(got != ref)[0]
+    assert bad.size == 0, [(float(x[i]), hex(got[i]), hex(ref[i])) for i in bad[:5]]
+
+
+def test_quantize_golden_rows():
+    g = _golden("e4m3_rounding_points.json")["quantize"]
+    for ex in g:
+        x = np.array([ex["x"]], np.float32)
+        codes, scale = oracle.quantize_e4m3(x)
+        want = np.float32(3.0) / np.float32(448.0) if "scale_expr" in ex else np.float32(ex["scale"])
+        assert scale[0] == want, ex["why"]
+        assert [hex(c) for c in codes[0]] == [hex(int(c, 16)) for c in ex["codes"]], ex["why"]
+
+
+def test_quantize_matches_torch_per_token():
+    """amax/448 in fp32 and torch's float8 conversion of x / scale, bf16 and fp32 rows."""
+    rng = np.random.default_rng(12)
+    x32 = (rng.standard_normal((64, 300)) * 10.0 ** rng.uniform(-6, 6, (64, 1))).astype(np.float32)
+    for x in (torch.from_numpy(x32), torch.from_numpy(x32).to(torch.bfloat16)):
+        codes, scale = oracle.quantize_e4m3(x)
+        xf = x.float()
+        amax = xf.abs().amax(dim=1)
+        ref_scale = amax / 448.0
+        ref = (xf / ref_scale[:, None]).clamp(-448.0, 448.0).to(torch.float8_e4m3fn).view(torch.uint8)
+        np.testing.assert_array_equal(scale, ref_scale.numpy())
+        np.testing.assert_array_equal(codes, ref.numpy())
+
+
+def test_quantize_invariants():
+    rng = np.random.default_rng(13)
+    x = rng.standard_normal((32, 128)).astype(np.float32) * rng.uniform(0.01, 100, (32, 1)).astype(np.float32)
+    codes, scale = oracle.quantize_e4m3(x)
+    am = np.argmax(np.abs(x), axis=1)
+    # the row's largest magnitude maps to the largest finite code, with its sign
+    for r in range(32):
+        assert codes[r, am[r]] & 0x7F == 0x7E
+        assert (codes[r, am[r]] >> 7) == (x[r, am[r]] < 0)
+    # dequantised error: at most half a step (2^-4 relative in the normal range,
+    # 2^-10 * scale below the smallest normal 2^-6 * scale)
+    deq = np.vectorize(oracle.e4m3)(codes) * scale[:, None].astype(np.float64)
+    bound = np.maximum(np.abs(x) * 2.0 ** -4, scale[:, None] * 2.0 ** -10) * (1 + 1e-6)
+    assert np.all(np.abs(deq - x) <= bound)
+    # rows quantise independently; scaling a row by a power of two scales only its scale
+    x2 = x.copy(); x2[5] *= 8.0
+    c2, s2 = oracle.quantize_e4m3(x2)
+    np.testing.assert_array_equal(c2, codes)
+    assert s2[5] == scale[5] * 8 and np.array_equal(np.delete(s2, 5), np.delete(scale, 5))
+
+
+def test_quantize_degenerate_rows():
+    x = np.zeros((3, 16), np.float32)
+    x[1, 3] = 1e-44                                   # amax/448 underflows to 0: scale 1
+    x[2, :] = -0.0
+    codes, scale = oracle.quantize_e4m3(x)
+    assert scale.tolist() == [1.0, 1.0, 1.0]
+    assert np.all(codes[0] == 0) and np.all(codes[1] == 0) and np.all(codes[2] == 0x80)
+
+
+def _paged_caches(rng, P, ps, D_I, D):
+    return dict(kidx_cache=rng.integers(0, 0x7E, (P, ps, D_I)).astype(np.uint8),
+                kscale_cache=rng.uniform(0.5, 2, (P, ps)).astype(np.float32),
+                k_cache=rng.integers(0, 1 << 15, (P, ps, D)).astype(np.uint16),
+                v_cache=rng.integers(0, 1 << 15, (P, ps, D)).astype(np.uint16))
+
+
+def test_cache_append_writes_exactly_the_addressed_slots():
+    rng = np.random.default_rng(14)
+    B, P, ps, D_I, D, maxp = 5, 40, 16, 32, 24, 6
+    bt = np.stack([rng.permutation(P)[:maxp] for _ in range(B)]).astype(np.int32)
+    caches = _paged_caches(rng, P, ps, D_I, D)
+    before = {k: v.copy() for k, v in caches.items()}
+    N = 9
+    seq = np.array([0, 1, 2, 3, 4, 0, 0, 3, 2], np.int32)
+    pos = np.array([0, 15, 16, 95, 40, 1, 2, 17, 33], np.int32)
+    kin = torch.from_numpy(rng.standard_normal((N, D_I)).astype(np.float32)).to(torch.bfloat16)
+    kn = rng.integers(0, 1 << 15, (N, D)).astype(np.uint16)
+    vn = rng.integers(0, 1 << 15, (N, D)).astype(np.uint16)
+    assert oracle.cache_append(caches, kin, kn, vn, seq, pos, bt) == 0
+    codes, scale = oracle.quantize_e4m3(kin)
+    touched = np.zeros((P, ps), bool)
+    for i in range(N):
+        page, slot = bt[seq[i], pos[i] // ps], pos[i] % ps
+        touched[page, slot] = True
+        np.testing.assert_array_equal(caches["kidx_cache"][page, slot], codes[i])
+        assert caches["kscale_cache"][page, slot] == scale[i]
+        np.testing.assert_array_equal(caches["k_cache"][page, slot], kn[i])
+        np.testing.assert_array_equal(caches["v_cache"][page, slot], vn[i])
+    for name in caches:
+        np.testing.assert_array_equal(caches[name][~touched], before[name][~touched])
+
+
+def test_cache_append_rejects_out_of_range():
+    rng = np.random.default_rng(15)
+    B, P, ps, maxp = 2, 8, 16, 2
+    bt = np.array([[0, 1], [2, 99]], np.int32)                    # page 99 does not exist
+    caches = _paged_caches(rng, P, ps, 16, 8)
+    kin = np.ones((1, 16), np.float32)
+    kv = np.zeros((1, 8), np.uint16)
+    for seq, pos in ((0, 32), (0, -1), (1, 20), (2, 0)):
+        assert oracle.cache_append(caches, kin, kv, kv, [seq], [pos], bt) == -2, (seq, pos)
+    assert oracle.cache_append(caches, kin, kv, kv, [1], [3], bt) == 0
+
+
+# ---------------------------------------------------------------- sliding window + top-k (stage 5)
+
+def _brute_window_rows(scores, rows, k, W):
+    out = np.full((len(rows), k + W), -1, np.int32)
+    for r, t in enumerate(rows):
+        n = t + 1
+        older = max(0, n - W)
+        order = sorted(range(older), key=lambda s: (-scores[r, s], s))
+        sel = sorted(order[: min(k, older)]) + list(range(older, n))
+        out[r, : len(sel)] = sel
+    return out
+
+
+def test_topk_window_vs_sort():
+    rng = np.random.default_rng(16)
+    T = 260
+    scores = np.round(rng.standard_normal((50, T)) * 4) / 4
+    rows = rng.integers(0, T, 50)
+    rows[:4] = [0, T - 1, 9, 10]
+    for k, W in ((1, 1), (8, 10), (16, 3), (64, 100), (300, 5), (5, 400)):
+        got = oracle.topk_window(scores, rows, k, W)
+        np.testing.assert_array_equal(got, _brute_window_rows(scores, rows, k, W), err_msg=f"k={k} W={W}")
+
+
+def test_topk_window_special_cases():
+    rng = np.random.default_rng(17)
+    T, k = 200, 12
+    scores = rng.standard_normal((30, T))
+    rows = rng.integers(0, T, 30)
+    # W = 0 is the plain selector
+    np.testing.assert_array_equal(oracle.topk_window(scores, rows, k, 0), oracle.topk(scores, rows, k))
+    # the window positions are taken whatever their scores
+    low = scores.copy(); low[:, :] = 5.0
+    for r, t in enumerate(rows):
+        low[r, max(0, t - 7): t + 1] = -1e300
+    got = oracle.topk_window(low, rows, k, 8)
+    for r, t in enumerate(rows):
+        n = t + 1
+        sel = got[r][got[r] >= 0]
+        assert sel.size == min(k, max(0, n - 8)) + min(8, n)
+        assert set(range(max(0, n - 8), n)) <= set(sel.tolist())
+        assert np.all(np.diff(sel) > 0) and np.all(got[r][sel.size:] == -1)
+    # k + W >= t + 1: every causal position
+    got = oracle.topk_window(scores, [50], 20, 31)
+    assert got[0].tolist() == list(range(51))
+
+
+def test_decode_window_matches_dense_mask():
+    """Decode with a window: dense masked attention over window U top-k(older)."""
+    spec = dsa_synth.DecodeSpec("dw", context_lens=(130, 9, 1, 257), H_I=4, d_I=32, k=12,
+                                H_q=3, d=16, page_size=16, needle_frac=0.05,
+                                needle_min_age=4, seed=19)
+    inp = dsa_synth.make_decode(spec)
+    sm, W = 0.25, 20
+    res = oracle.decode(inp, spec.k, sm, want_scores=True, window=W)
+    bt = inp["block_table"].numpy()
+    for b, n in enumerate(spec.context_lens):
+        pos = np.arange(n)
+        slot = bt[b, pos // 16].astype(np.int64) * 16 + pos % 16
+        sc = res["scores"][b, :n]
+        older = max(0, n - W)
+        order = np.argsort(-sc[:older], kind="stable")[: min(spec.k, older)]
+        mask = np.zeros(n, bool); mask[order] = True; mask[older:] = True
+        sel = np.nonzero(mask)[0]
+        assert res["idx"][b][: sel.size].tolist() == sel.tolist()
+        assert np.all(res["idx"][b][sel.size:] == -1)
+        kc = inp["k_cache"].reshape(-1, 16)[slot]
+        vc = inp["v_cache"].reshape(-1, 16)[slot]
+        qq = torch.zeros((n, 3, 16), dtype=torch.bfloat16); qq[n - 1] = inp["q"][b]
+        m = np.zeros((n, n), bool); m[n - 1] = mask
+        m[: n - 1, 0] = True
+        out, lse = brute.dense_masked_attention(qq, kc, vc, m, sm)
+        np.testing.assert_allclose(res["out"][b], out[n - 1], rtol=1e-10, atol=1e-12)
+        np.testing.assert_allclose(res["lse"][b], lse[n - 1], rtol=1e-12, atol=1e-12)
