@@ -339,31 +339,40 @@ def prefill_e2e(dsa, inp, spec, out, lse, idx, ws, flush, args, ws_n):
 
 # ----------------------------------------------------------------------------- decode
 
-def decode_hbm_bytes(spec):
-    """Algorithmic HBM bytes of one decode step (what the method must move)."""
+def decode_hbm_bytes(spec, window=0):
+    """Algorithmic HBM bytes of one decode step (what the method must move);
+    with a window, the window's K/V rows are gathered besides the top-k's."""
     B, n = spec.B, sum(spec.context_lens)
-    sel = sum(min(spec.k, c) for c in spec.context_lens)
+    sel = sum(min(spec.k, max(0, c - window)) + min(window, c) for c in spec.context_lens)
     return dict(index_keys=n * spec.d_I, key_scales=n * 4, kv_gather=sel * spec.d * 2 * 2,
                 q=B * spec.H_q * spec.d * 2, out=B * spec.H_q * spec.d * 2,
-                q_idx=B * spec.H_I * spec.d_I + B * 4 + B * spec.H_I * 2, idx=B * spec.k * 4)
+                q_idx=B * spec.H_I * spec.d_I + B * 4 + B * spec.H_I * 2, idx=B * (spec.k + window) * 4)
 
 
-def bench_decode(args, dsa, spec, peaks, ws_n, rank):
+def bench_decode(args, dsa, spec, peaks, ws_n, rank, window=0, with_append=False):
+    """The decode step through dsa_decode (window 0) or dsa_decode_window;
+    with_append also times the step's quantise-and-append of the B new
+    tokens (dsa_quantize_e4m3 of the index queries, dsa_cache_append)."""
     dev = torch.device("cuda")
     inp = dsa_synth.make_decode(replica_spec(spec, rank), device=dev)
     inp.pop("needle_pos")
     torch.cuda.synchronize()
     maxc = max(spec.context_lens)
     lib = dsa.load()
-    ws = dsa.workspace(lib.dsa_decode_workspace_size(spec.B, maxc, spec.H_q, spec.d, spec.k), dev)
+    kw = spec.k + window
+    ws = dsa.workspace(lib.dsa_decode_workspace_size(spec.B, maxc, spec.H_q, spec.d, kw), dev)
     out = torch.empty_like(inp["q"])
     lse = torch.empty((spec.B, spec.H_q), dtype=torch.float32, device=dev)
-    idx = torch.empty((spec.B, spec.k), dtype=torch.int32, device=dev)
+    idx = torch.empty((spec.B, kw), dtype=torch.int32, device=dev)
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
     sm = 1.0 / math.sqrt(spec.d)
 
-    def step():
-        dsa.dsa_decode(inp, spec.k, maxc, sm, out=out, lse=lse, idx_out=idx, ws=ws)
+    if window:
+        def step():
+            dsa.dsa_decode_window(inp, spec.k, window, maxc, sm, out=out, lse=lse, idx_out=idx, ws=ws)
+    else:
+        def step():
+            dsa.dsa_decode(inp, spec.k, maxc, sm, out=out, lse=lse, idx_out=idx, ws=ws)
 
     step()
     torch.cuda.synchronize()
@@ -372,12 +381,84 @@ def bench_decode(args, dsa, spec, peaks, ws_n, rank):
     ms = timed_steps(step, max(args.steps, 20), args.warmup, flush)
     step_ms = max_over_ranks(sum(ms) / len(ms), ws_n)
     status = dsa.dsa_stream_status(ws)
-    by = decode_hbm_bytes(spec)
+    by = decode_hbm_bytes(spec, window)
     total = sum(by.values())
+    app = None
+    if with_append:
+        app = bench_append(dsa, spec, inp, args, flush)
     del inp, ws
     torch.cuda.empty_cache()
     return dict(step_ms=step_ms, launches=n_launch, per_kernel=per_kernel, bytes=total,
-                bytes_detail=by, status=status)
+                bytes_detail=by, status=status, append=app)
+
+
+def bench_append(dsa, spec, inp, args, flush):
+    """One decode step's new tokens: the B index queries quantised
+    (dsa_quantize_e4m3) and the B index keys, K and V rows appended to the
+    paged caches (dsa_cache_append), at each sequence's last position."""
+    dev = inp["q"].device
+    g = torch.Generator(device=dev).manual_seed(99)
+    B = spec.B
+    q_src = torch.randn((B, spec.H_I, spec.d_I), generator=g, device=dev).to(torch.bfloat16)
+    k_src = torch.randn((B, spec.d_I), generator=g, device=dev).to(torch.bfloat16)
+    kn = torch.randn((B, spec.d), generator=g, device=dev).to(torch.bfloat16)
+    vn = torch.randn((B, spec.d), generator=g, device=dev).to(torch.bfloat16)
+    seq = torch.arange(B, dtype=torch.int32, device=dev)
+    pos = (inp["context_lens"] - 1).to(torch.int32)
+    codes = torch.empty((B, spec.H_I, spec.d_I), dtype=torch.uint8, device=dev)
+    scale = torch.empty((B,), dtype=torch.float32, device=dev)
+
+    def step():
+        dsa.dsa_quantize_e4m3(q_src, codes=codes, scale=scale)
+        dsa.dsa_cache_append(inp, k_src, kn, vn, seq, pos, inp["block_table"])
+
+    ms = timed_steps(step, max(args.steps, 20), args.warmup, flush)
+    return dict(us=1e3 * sum(ms) / len(ms), launches=2)
+
+
+def bench_quantize(args, dsa, spec, peaks):
+    """FP8 quantisation of the prefill's index query [T, H_I * d_I] and key
+    [T, d_I] from bf16 (dsa_quantize_e4m3, one scale per token): HBM-bound,
+    algorithmic bytes = 2 B read + 1 B written per value + 4 B per scale."""
+    dev = torch.device("cuda")
+    T, H, D = spec.L, spec.H_I, spec.d_I
+    g = torch.Generator(device=dev).manual_seed(7)
+    xq = torch.randn((T, H, D), generator=g, device=dev, dtype=torch.float32).to(torch.bfloat16)
+    xk = torch.randn((T, D), generator=g, device=dev, dtype=torch.float32).to(torch.bfloat16)
+    cq = torch.empty((T, H, D), dtype=torch.uint8, device=dev)
+    ck = torch.empty((T, D), dtype=torch.uint8, device=dev)
+    sq = torch.empty((T,), dtype=torch.float32, device=dev)
+    sk = torch.empty((T,), dtype=torch.float32, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream()
+    for _ in range(args.warmup):
+        dsa.dsa_quantize_e4m3(xq, codes=cq, scale=sq)
+        dsa.dsa_quantize_e4m3(xk, codes=ck, scale=sk)
+    torch.cuda.synchronize()
+    reps = max(args.steps, 10)
+    evs = []
+    for _ in range(reps):
+        flush.zero_()
+        e = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+        e[0].record(stream)
+        dsa.dsa_quantize_e4m3(xq, codes=cq, scale=sq)
+        e[1].record(stream)
+        dsa.dsa_quantize_e4m3(xk, codes=ck, scale=sk)
+        e[2].record(stream)
+        evs.append(e)
+    torch.cuda.synchronize()
+    q_ms = sum(e[0].elapsed_time(e[1]) for e in evs) / reps
+    k_ms = sum(e[1].elapsed_time(e[2]) for e in evs) / reps
+    q_bytes = T * H * D * 3 + T * 4
+    k_bytes = T * D * 3 + T * 4
+    q_gbs = q_bytes / (q_ms * 1e-3) / 1e9
+    del xq, xk, cq, ck
+    torch.cuda.empty_cache()
+    return {"kernel": "quantize_rows_kernel (bf16 -> e4m3 + per-token scale)",
+            "query_us": round(q_ms * 1e3, 2), "key_us": round(k_ms * 1e3, 2),
+            "roofline": {"bound": "hbm", "achieved": round(q_gbs, 1), "peak": peaks["hbm_gbs"],
+                         "unit": "GB/s", "frac": round(q_gbs / peaks["hbm_gbs"], 4),
+                         "algorithmic_bytes": q_bytes, "of": "the query pass"}}
 
 
 # ----------------------------------------------------------------------------- CPU oracle
@@ -448,6 +529,12 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
+    ap.add_argument("--quantize-only", action="store_true",
+                    help="profiling aid: time only the FP8 quantiser on the workload's index query/key")
+    ap.add_argument("--no-extras", action="store_true",
+                    help="skip the quantiser, cache-append and sliding-window decode lines")
+    ap.add_argument("--window", type=int, default=8192,
+                    help="sliding window of the extra decode line (the pages' 8K example)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3) if args.impl == "dsa" else args.warmup
 
@@ -488,6 +575,18 @@ def main():
     dsa.load()
     peaks, peak_kind = load_peaks()
 
+    if args.quantize_only:
+        q = bench_quantize(args, dsa, spec, peaks)
+        if rank == 0:
+            print(json.dumps({"metric": "FP8 quantisation of the index query (HBM GB/s)",
+                              "value": q["roofline"]["achieved"], "unit": "GB/s", "n_gpus": ws_n,
+                              "steps": args.steps, "warmup": args.warmup, "higher_is_better": True,
+                              "config": {"workload": f"quantize_T{spec.L}_HI{spec.H_I}_dI{spec.d_I}_bf16"},
+                              "quantize": q}), flush=True)
+        if ws_n > 1:
+            torch.distributed.barrier()
+            torch.distributed.destroy_process_group()
+        return
     if args.decode_only:
         dec = bench_decode(args, dsa, dspec, peaks, ws_n, rank)
         us = dec["step_ms"] * 1e3
@@ -507,7 +606,13 @@ def main():
             torch.distributed.destroy_process_group()
         return
     pre = bench_prefill(args, dsa, spec, peaks, peak_kind, ws_n, rank)
-    dec = None if args.no_decode else bench_decode(args, dsa, dspec, peaks, ws_n, rank)
+    extras = not args.no_extras
+    dec = None if args.no_decode else bench_decode(args, dsa, dspec, peaks, ws_n, rank,
+                                                   with_append=extras)
+    decw = None
+    if extras and not args.no_decode:
+        decw = bench_decode(args, dsa, dspec, peaks, ws_n, rank, window=args.window)
+    quant = bench_quantize(args, dsa, spec, peaks) if extras else None
 
     T = spec.L
     value = whole_job_rate(ws_n, T, pre["step_ms"])
@@ -549,6 +654,20 @@ def main():
                                        "frac": round(gbs / peaks["hbm_gbs"], 4),
                                        "algorithmic_bytes": dec["bytes"]},
                           "gpu_launches_per_step": dec["per_kernel"], "device_status": dec["status"]}
+        if dec["append"]:
+            line["decode"]["append_us"] = round(dec["append"]["us"], 2)
+    if decw:
+        gbs = decw["bytes"] / (decw["step_ms"] * 1e-3) / 1e9
+        line["decode_window"] = {"window": args.window, "top_k": dspec.k,
+                                 "value": round(whole_job_rate(ws_n, 1, decw["step_ms"]), 1),
+                                 "unit": "steps/s", "us_per_step": round(decw["step_ms"] * 1e3, 2),
+                                 "roofline": {"bound": "hbm", "achieved": round(gbs, 1),
+                                              "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                                              "frac": round(gbs / peaks["hbm_gbs"], 4),
+                                              "algorithmic_bytes": decw["bytes"]},
+                                 "device_status": decw["status"]}
+    if quant:
+        line["quantize"] = quant
     if rank == 0 and ws_n == 1 and not args.no_cpu:
         os.environ.setdefault("OMP_NUM_THREADS", str(oracle_threads()))
         inp_cpu = cpu_inputs_for(spec)

@@ -112,6 +112,24 @@ dsa_status dsa_topk(const float *scores, int64_t ld_scores, int64_t row_begin,
                     size_t ws_bytes, void *stream);
 
 /*
+ * dsa_topk_window -- the selector with a sliding window ("DeepSeek-V4 百万
+ * token 上下文的工程实现", section on the sliding-window KV cache and the
+ * hybrid strategy: the most recent 4K-16K tokens keep their full KV, older
+ * tokens are kept only as far as an importance score retains them).  For row
+ * r (query position t = row_begin + r, n = t + 1 causal positions) the last
+ * `window` positions max(0, n - window) .. t are always selected, and
+ * min(k, n - window) of the older positions 0 .. t - window are selected as
+ * dsa_topk does (largest score, ties to the lower s, +0 equals -0).
+ *   idx_out int32 [row_count, k + window]: the selected older positions
+ *   ascending, then the window positions ascending, then -1 padding.
+ * window == 0 gives dsa_topk's result.  Requires 0 <= window <= 2^24 and the
+ * other constraints of dsa_topk; workspace as dsa_topk.
+ */
+dsa_status dsa_topk_window(const float *scores, int64_t ld_scores, int64_t row_begin,
+                           int64_t row_count, int64_t T, int k, int window, int32_t *idx_out,
+                           void *workspace, size_t ws_bytes, void *stream);
+
+/*
  * dsa_sparse_attn -- main attention restricted to the selected KV rows
  * (DSA section 1: the main attention only looks at the selected subset).
  *   q   [T, H_q, d], k and v [T, d] (one shared KV head), out [T, H_q, d]:
@@ -144,6 +162,20 @@ dsa_status dsa_prefill(const void *q_idx, const float *q_scale, const void *k_id
                        const void *v, int64_t T, int H_I, int d_I, int H_q, int d, int k_sel,
                        float sm_scale, void *out, float *lse_out, int32_t *idx_out,
                        dsa_dtype dtype, void *workspace, size_t ws_bytes, void *stream);
+
+/*
+ * dsa_prefill_window -- dsa_prefill with dsa_topk_window's selection: the last
+ * `window` positions of every query are always attended, and the indexer's
+ * top-k picks k_sel of the older ones.  idx_out is [T, k_sel + window]; the
+ * workspace must hold dsa_prefill_workspace_size(T, H_I, d_I, H_q, d,
+ * k_sel + window, dtype) bytes.  window == 0 is dsa_prefill.
+ */
+dsa_status dsa_prefill_window(const void *q_idx, const float *q_scale, const void *k_idx,
+                              const float *k_scale, const void *w, const void *q, const void *k,
+                              const void *v, int64_t T, int H_I, int d_I, int H_q, int d, int k_sel,
+                              int window, float sm_scale, void *out, float *lse_out,
+                              int32_t *idx_out, dsa_dtype dtype, void *workspace, size_t ws_bytes,
+                              void *stream);
 
 /*
  * dsa_prefill_host -- dsa_prefill for inputs and outputs in HOST memory
@@ -202,6 +234,68 @@ dsa_status dsa_decode(const void *q_idx, const float *q_scale, const void *w, co
                       int page_size, int B, int64_t max_context, int H_I, int d_I, int H_q,
                       int d, int k_sel, float sm_scale, void *out, float *lse_out,
                       int32_t *idx_out, void *workspace, size_t ws_bytes, void *stream);
+
+/*
+ * dsa_decode_window -- dsa_decode with dsa_topk_window's selection (the last
+ * `window` cached positions of each sequence are always attended; the top-k
+ * picks k_sel of the older ones).  idx_out is [B, k_sel + window]; the
+ * workspace must hold dsa_decode_workspace_size(B, max_context, H_q, d,
+ * k_sel + window) bytes.  window == 0 is dsa_decode.
+ */
+dsa_status dsa_decode_window(const void *q_idx, const float *q_scale, const void *w, const void *q,
+                             const void *kidx_cache, const float *kscale_cache, const void *k_cache,
+                             const void *v_cache, const int32_t *block_table,
+                             const int32_t *context_lens, int64_t num_pages, int max_pages_per_seq,
+                             int page_size, int B, int64_t max_context, int H_I, int d_I, int H_q,
+                             int d, int k_sel, int window, float sm_scale, void *out, float *lse_out,
+                             int32_t *idx_out, void *workspace, size_t ws_bytes, void *stream);
+
+/*
+ * dsa_quantize_e4m3 -- FP8 E4M3 quantisation with one fp32 scale per row, the
+ * storage of the indexer's query and key ("DeepSeek-V3.2-Exp DSA 技术深度解析",
+ * section 1: FP8 indexer; the DeepSeek-V4 engineering page's FP8 decoding
+ * section).  For each row r of x [rows, cols] (bf16 or fp32, x_dtype DSA_BF16
+ * or DSA_F32):
+ *   scale_out[r] = amax_r / 448 (fp32 division; 1 when that is 0), where
+ *                  amax_r = max_j |x[r, j]|;
+ *   codes_out[r, j] = the E4M3 value nearest to x[r, j] / scale_out[r] (fp32
+ *                  division), ties to the even code, magnitudes past 448
+ *                  saturating to +-448 (OCP E4M3FN bytes).
+ * For the indexer query pass x = q_I viewed as [T, H_I * d_I] (one scale per
+ * token over all heads); for the key x = k_I [T, d_I].
+ * x: device, 16-byte aligned; codes_out uint8 [rows, cols], 8-byte aligned;
+ * scale_out f32 [rows].  cols a multiple of 8, at most 16384 (else
+ * DSA_ERR_UNSUPPORTED).  x must be finite (a NaN or infinity makes its row's
+ * scale and codes meaningless).  rows == 0 is a no-op.
+ */
+dsa_status dsa_quantize_e4m3(const void *x, dsa_dtype x_dtype, int64_t rows, int64_t cols,
+                             uint8_t *codes_out, float *scale_out, void *stream);
+
+/*
+ * dsa_cache_append -- writes N new tokens into the paged decode caches (the
+ * step before dsa_decode in every decode step: the current token is appended,
+ * then attended).  Token i belongs to sequence seq_ids[i] at position
+ * positions[i], i.e. physical page block_table[seq_ids[i], positions[i] /
+ * page_size], slot positions[i] % page_size.  Its index key kidx_new[i, :]
+ * (bf16 or fp32 [N, d_I], kidx_dtype DSA_BF16 or DSA_F32) is quantised as by
+ * dsa_quantize_e4m3 into kidx_cache [num_pages, page_size, d_I] (uint8) and
+ * kscale_cache [num_pages, page_size] (f32); its K and V rows k_new, v_new
+ * (bf16 [N, d]) are copied into k_cache, v_cache (bf16 [num_pages,
+ * page_size, d]).  Tokens must address distinct slots.
+ * A token whose sequence is outside [0, B), whose position is outside
+ * [0, max_pages_per_seq * page_size) or whose page id is outside
+ * [0, num_pages) is skipped, and DSA_ERR_INVALID_ARG is written to *status
+ * (a device uint32_t the caller zeroes beforehand; nullable) unless it
+ * already holds an error.  Supported: d_I a multiple of 8 up to 256, d a
+ * multiple of 8.  kidx_new, k_new, v_new, k_cache, v_cache 16-byte aligned,
+ * kidx_cache 8-byte aligned.  N == 0 is a no-op.
+ */
+dsa_status dsa_cache_append(const void *kidx_new, dsa_dtype kidx_dtype, const void *k_new,
+                            const void *v_new, const int32_t *seq_ids, const int32_t *positions,
+                            int64_t N, int B, const int32_t *block_table, int max_pages_per_seq,
+                            int64_t num_pages, int page_size, int d_I, int d, void *kidx_cache,
+                            float *kscale_cache, void *k_cache, void *v_cache, uint32_t *status,
+                            void *stream);
 
 /*
  * dsa_decode_noalloc -- dsa_decode without a caller workspace.  The paper has

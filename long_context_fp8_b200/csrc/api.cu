@@ -29,6 +29,9 @@ inline int64_t prefill_rows_default(int64_t T)
 
 inline size_t idx_bytes(int64_t rows, int k) { return align_up(sizeof(int32_t) * (size_t)rows * k, 256); }
 
+// Largest sliding window (positions) the window entry points accept.
+constexpr int kMaxWindow = 1 << 24;
+
 dsa_status check_index_args(const void *q_idx, const float *q_scale, const void *k_idx,
                             const float *k_scale, const void *w, int64_t T, int H_I, int d_I,
                             dsa_dtype dtype)
@@ -226,6 +229,20 @@ dsa_status dsa_topk(const float *scores, int64_t ld_scores, int64_t row_begin,
                                         idx_out, nullptr, as_stream(stream)));
 }
 
+dsa_status dsa_topk_window(const float *scores, int64_t ld_scores, int64_t row_begin,
+                           int64_t row_count, int64_t T, int k, int window, int32_t *idx_out,
+                           void *workspace, size_t ws_bytes, void *stream)
+{
+    (void)workspace; (void)ws_bytes;
+    if (!scores || !idx_out || T <= 0 || k < 1 || k > 65536 || window < 0 || window > kMaxWindow)
+        return DSA_ERR_INVALID_ARG;
+    if (row_begin < 0 || row_count < 0 || row_begin + row_count > T || ld_scores < T)
+        return DSA_ERR_INVALID_ARG;
+    if (row_count == 0) return DSA_OK;
+    return cuda_status(launch_topk_rows(scores, ld_scores, row_begin, nullptr, T, row_count, k,
+                                        idx_out, nullptr, as_stream(stream), window));
+}
+
 dsa_status dsa_sparse_attn(const void *q, const void *k, const void *v, const int32_t *idx,
                            int64_t T, int H_q, int d, int k_sel, float sm_scale, void *out,
                            float *lse_out, dsa_dtype dtype, void *stream)
@@ -246,11 +263,17 @@ size_t dsa_prefill_workspace_size(int64_t T, int H_I, int d_I, int H_q, int d, i
     return kWsHeader + idx_bytes(T, k_sel) + align_up(sizeof(float) * (size_t)R * T, 256);
 }
 
-dsa_status dsa_prefill(const void *q_idx, const float *q_scale, const void *k_idx,
-                       const float *k_scale, const void *w, const void *q, const void *k,
-                       const void *v, int64_t T, int H_I, int d_I, int H_q, int d, int k_sel,
-                       float sm_scale, void *out, float *lse_out, int32_t *idx_out,
-                       dsa_dtype dtype, void *workspace, size_t ws_bytes, void *stream)
+}  // extern "C"
+
+namespace {
+
+// dsa_prefill with a sliding window of `window` positions (0: none); the
+// selection rows are k_sel + window wide.
+dsa_status prefill_impl(const void *q_idx, const float *q_scale, const void *k_idx,
+                        const float *k_scale, const void *w, const void *q, const void *k,
+                        const void *v, int64_t T, int H_I, int d_I, int H_q, int d, int k_sel,
+                        int window, float sm_scale, void *out, float *lse_out, int32_t *idx_out,
+                        dsa_dtype dtype, void *workspace, size_t ws_bytes, void *stream)
 {
     if (dtype != DSA_E4M3 && dtype != DSA_F32) return DSA_ERR_UNSUPPORTED;
     dsa_status s = check_index_args(q_idx, q_scale, k_idx, k_scale, w, T, H_I, d_I, dtype);
@@ -258,9 +281,11 @@ dsa_status dsa_prefill(const void *q_idx, const float *q_scale, const void *k_id
     // any non-null placeholder for idx: only the other attention arguments are checked here
     s = check_attn_args(q, k, v, reinterpret_cast<const int32_t *>(q), T, H_q, d, k_sel, out, dtype);
     if (s != DSA_OK) return s;
-    if (k_sel > 65536 || !std::isfinite(sm_scale)) return DSA_ERR_INVALID_ARG;
+    if (k_sel > 65536 || window < 0 || window > kMaxWindow || !std::isfinite(sm_scale))
+        return DSA_ERR_INVALID_ARG;
     if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u)) return DSA_ERR_WORKSPACE;
-    size_t fixed = kWsHeader + (idx_out ? 0 : idx_bytes(T, k_sel));
+    const int kw = k_sel + window;                    // selection row width
+    size_t fixed = kWsHeader + (idx_out ? 0 : idx_bytes(T, kw));
     if (ws_bytes < fixed + sizeof(float) * 64 * (size_t)T) return DSA_ERR_WORKSPACE;
     int64_t R = (int64_t)((ws_bytes - fixed) / (sizeof(float) * (size_t)T)) / 64 * 64;
     R = R < T ? R : ceil_div(T, 64) * 64;
@@ -276,12 +301,37 @@ dsa_status dsa_prefill(const void *q_idx, const float *q_scale, const void *k_id
         e = run_index(q_idx, q_scale, k_idx, k_scale, w, T, H_I, d_I, r0, n, scores, T, false,
                       dtype, st);
         if (e == cudaSuccess)
-            e = launch_topk_rows(scores, T, r0, nullptr, T, n, k_sel, idx + r0 * (int64_t)k_sel,
-                                 hdr, st);
+            e = launch_topk_rows(scores, T, r0, nullptr, T, n, k_sel, idx + r0 * (int64_t)kw,
+                                 hdr, st, window);
     }
     if (e == cudaSuccess)
-        e = run_attn(q, k, v, idx, T, H_q, d, k_sel, sm_scale, out, lse_out, dtype, st);
+        e = run_attn(q, k, v, idx, T, H_q, d, kw, sm_scale, out, lse_out, dtype, st);
     return cuda_status(e);
+}
+
+}  // namespace
+
+extern "C" {
+
+dsa_status dsa_prefill(const void *q_idx, const float *q_scale, const void *k_idx,
+                       const float *k_scale, const void *w, const void *q, const void *k,
+                       const void *v, int64_t T, int H_I, int d_I, int H_q, int d, int k_sel,
+                       float sm_scale, void *out, float *lse_out, int32_t *idx_out,
+                       dsa_dtype dtype, void *workspace, size_t ws_bytes, void *stream)
+{
+    return prefill_impl(q_idx, q_scale, k_idx, k_scale, w, q, k, v, T, H_I, d_I, H_q, d, k_sel, 0,
+                        sm_scale, out, lse_out, idx_out, dtype, workspace, ws_bytes, stream);
+}
+
+dsa_status dsa_prefill_window(const void *q_idx, const float *q_scale, const void *k_idx,
+                              const float *k_scale, const void *w, const void *q, const void *k,
+                              const void *v, int64_t T, int H_I, int d_I, int H_q, int d, int k_sel,
+                              int window, float sm_scale, void *out, float *lse_out,
+                              int32_t *idx_out, dsa_dtype dtype, void *workspace, size_t ws_bytes,
+                              void *stream)
+{
+    return prefill_impl(q_idx, q_scale, k_idx, k_scale, w, q, k, v, T, H_I, d_I, H_q, d, k_sel,
+                        window, sm_scale, out, lse_out, idx_out, dtype, workspace, ws_bytes, stream);
 }
 
 size_t dsa_prefill_host_workspace_size(int64_t T, int H_I, int d_I, int H_q, int d, int k_sel,
@@ -386,14 +436,22 @@ size_t dsa_decode_workspace_size(int B, int64_t max_context, int H_q, int d, int
            align_up(topk_split_ws_bytes(B, max_context), 256);
 }
 
-dsa_status dsa_decode(const void *q_idx, const float *q_scale, const void *w, const void *q,
-                      const void *kidx_cache, const float *kscale_cache, const void *k_cache,
-                      const void *v_cache, const int32_t *block_table,
-                      const int32_t *context_lens, int64_t num_pages, int max_pages_per_seq,
-                      int page_size, int B, int64_t max_context, int H_I, int d_I, int H_q,
-                      int d, int k_sel, float sm_scale, void *out, float *lse_out,
-                      int32_t *idx_out, void *workspace, size_t ws_bytes, void *stream)
+}  // extern "C"
+
+namespace {
+
+// dsa_decode with a sliding window of `window` positions (0: none); the
+// selection rows (and the attention's index lists) are k_sel + window wide.
+dsa_status decode_impl(const void *q_idx, const float *q_scale, const void *w, const void *q,
+                       const void *kidx_cache, const float *kscale_cache, const void *k_cache,
+                       const void *v_cache, const int32_t *block_table,
+                       const int32_t *context_lens, int64_t num_pages, int max_pages_per_seq,
+                       int page_size, int B, int64_t max_context, int H_I, int d_I, int H_q,
+                       int d, int k_sel, int window, float sm_scale, void *out, float *lse_out,
+                       int32_t *idx_out, void *workspace, size_t ws_bytes, void *stream)
 {
+    if (window < 0 || window > kMaxWindow || k_sel > 65536) return DSA_ERR_INVALID_ARG;
+    const int kw = k_sel + window;                    // selection row width
     if (!q_idx || !q_scale || !w || !q || !kidx_cache || !kscale_cache || !k_cache || !v_cache ||
         !block_table || !context_lens || !out)
         return DSA_ERR_INVALID_ARG;
@@ -408,7 +466,7 @@ dsa_status dsa_decode(const void *q_idx, const float *q_scale, const void *w, co
     if (H_q > 128 && H_q % 128 != 0) return DSA_ERR_UNSUPPORTED;
     if (B > 65535) return DSA_ERR_UNSUPPORTED;
     if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u)) return DSA_ERR_WORKSPACE;
-    if (ws_bytes < dsa_decode_workspace_size(B, max_context, H_q, d, k_sel)) return DSA_ERR_WORKSPACE;
+    if (ws_bytes < dsa_decode_workspace_size(B, max_context, H_q, d, kw)) return DSA_ERR_WORKSPACE;
 
     cudaStream_t st = as_stream(stream);
     uint8_t *ws = static_cast<uint8_t *>(workspace);
@@ -417,12 +475,12 @@ dsa_status dsa_decode(const void *q_idx, const float *q_scale, const void *w, co
     float *scores = reinterpret_cast<float *>(ws + off);
     off += align_up(sizeof(float) * (size_t)B * max_context, 256);
     int32_t *idx = reinterpret_cast<int32_t *>(ws + off);
-    off += idx_bytes(B, k_sel);
+    off += idx_bytes(B, kw);
     float *part = reinterpret_cast<float *>(ws + off);
-    off += align_up(sparse_attn_paged_part_bytes(B, H_q, d, sparse_attn_paged_splits(B, k_sel)), 256);
+    off += align_up(sparse_attn_paged_part_bytes(B, H_q, d, sparse_attn_paged_splits(B, kw)), 256);
     void *topk_ws = ws + off;
     if (idx_out) idx = idx_out;
-    const int splits = sparse_attn_paged_splits(B, k_sel);
+    const int splits = sparse_attn_paged_splits(B, kw);
 
     cudaError_t e = cudaMemsetAsync(hdr, 0, sizeof(WsHeader), st);
     if (e == cudaSuccess) {
@@ -441,17 +499,17 @@ dsa_status dsa_decode(const void *q_idx, const float *q_scale, const void *w, co
     }
     if (e == cudaSuccess)   // each row split over 16K-position chunks (CTAs), then one CTA per row
         e = launch_topk_split(scores, max_context, context_lens, max_context, B, k_sel, idx, topk_ws,
-                              hdr, st);
+                              hdr, st, window);
     if (e == cudaSuccess) {
         bool done = false;
         if (sparse_attn_tc_supported(H_q, d) && (int64_t)num_pages * page_size < ((int64_t)1 << 31)) {
             // tcgen05 kernel over the paged caches, the index list split in 128-row blocks
-            const int chunk = (int)(ceil_div(ceil_div(k_sel, splits), 128) * 128);
-            const int tc_splits = (int)ceil_div(k_sel, chunk);
+            const int chunk = (int)(ceil_div(ceil_div(kw, splits), 128) * 128);
+            const int tc_splits = (int)ceil_div(kw, chunk);
             e = launch_sparse_attn_tc((const uint16_t *)q, (const uint16_t *)k_cache,
                                       (const uint16_t *)v_cache, num_pages * page_size, 0,
                                       block_table, context_lens, num_pages, max_pages_per_seq,
-                                      page_size, idx, B, H_q, d, k_sel, sm_scale, (uint16_t *)out,
+                                      page_size, idx, B, H_q, d, kw, sm_scale, (uint16_t *)out,
                                       lse_out, part, tc_splits, hdr, st, /*chained=*/true);
             if (e == cudaSuccess) e = launch_merge_splits(part, B, tc_splits, H_q, d, (uint16_t *)out, lse_out, st);
             done = e != cudaErrorNotSupported;
@@ -459,11 +517,82 @@ dsa_status dsa_decode(const void *q_idx, const float *q_scale, const void *w, co
         if (!done) {
             PagedKV kv{(const uint16_t *)k_cache, (const uint16_t *)v_cache, block_table, context_lens,
                        num_pages, max_pages_per_seq, page_size};
-            e = launch_sparse_attn_paged_bf16((const uint16_t *)q, kv, idx, B, H_q, d, k_sel, sm_scale,
+            e = launch_sparse_attn_paged_bf16((const uint16_t *)q, kv, idx, B, H_q, d, kw, sm_scale,
                                               (uint16_t *)out, lse_out, part, splits, hdr, st);
         }
     }
     return cuda_status(e);
+}
+
+}  // namespace
+
+extern "C" {
+
+dsa_status dsa_decode(const void *q_idx, const float *q_scale, const void *w, const void *q,
+                      const void *kidx_cache, const float *kscale_cache, const void *k_cache,
+                      const void *v_cache, const int32_t *block_table,
+                      const int32_t *context_lens, int64_t num_pages, int max_pages_per_seq,
+                      int page_size, int B, int64_t max_context, int H_I, int d_I, int H_q,
+                      int d, int k_sel, float sm_scale, void *out, float *lse_out,
+                      int32_t *idx_out, void *workspace, size_t ws_bytes, void *stream)
+{
+    return decode_impl(q_idx, q_scale, w, q, kidx_cache, kscale_cache, k_cache, v_cache, block_table,
+                       context_lens, num_pages, max_pages_per_seq, page_size, B, max_context, H_I, d_I,
+                       H_q, d, k_sel, 0, sm_scale, out, lse_out, idx_out, workspace, ws_bytes, stream);
+}
+
+dsa_status dsa_decode_window(const void *q_idx, const float *q_scale, const void *w, const void *q,
+                             const void *kidx_cache, const float *kscale_cache, const void *k_cache,
+                             const void *v_cache, const int32_t *block_table,
+                             const int32_t *context_lens, int64_t num_pages, int max_pages_per_seq,
+                             int page_size, int B, int64_t max_context, int H_I, int d_I, int H_q,
+                             int d, int k_sel, int window, float sm_scale, void *out, float *lse_out,
+                             int32_t *idx_out, void *workspace, size_t ws_bytes, void *stream)
+{
+    return decode_impl(q_idx, q_scale, w, q, kidx_cache, kscale_cache, k_cache, v_cache, block_table,
+                       context_lens, num_pages, max_pages_per_seq, page_size, B, max_context, H_I, d_I,
+                       H_q, d, k_sel, window, sm_scale, out, lse_out, idx_out, workspace, ws_bytes,
+                       stream);
+}
+
+dsa_status dsa_quantize_e4m3(const void *x, dsa_dtype x_dtype, int64_t rows, int64_t cols,
+                             uint8_t *codes_out, float *scale_out, void *stream)
+{
+    if (x_dtype != DSA_BF16 && x_dtype != DSA_F32) return DSA_ERR_UNSUPPORTED;
+    if (rows < 0 || cols <= 0) return DSA_ERR_INVALID_ARG;
+    if (rows == 0) return DSA_OK;
+    if (!x || !codes_out || !scale_out || !aligned16(x) || (reinterpret_cast<uintptr_t>(codes_out) & 7u))
+        return DSA_ERR_INVALID_ARG;
+    if (cols % 8 != 0 || cols > 16384) return DSA_ERR_UNSUPPORTED;
+    return cuda_status(launch_quantize_e4m3(x, x_dtype == DSA_BF16, rows, (int)cols, codes_out, scale_out,
+                                            as_stream(stream)));
+}
+
+dsa_status dsa_cache_append(const void *kidx_new, dsa_dtype kidx_dtype, const void *k_new,
+                            const void *v_new, const int32_t *seq_ids, const int32_t *positions,
+                            int64_t N, int B, const int32_t *block_table, int max_pages_per_seq,
+                            int64_t num_pages, int page_size, int d_I, int d, void *kidx_cache,
+                            float *kscale_cache, void *k_cache, void *v_cache, uint32_t *status,
+                            void *stream)
+{
+    if (kidx_dtype != DSA_BF16 && kidx_dtype != DSA_F32) return DSA_ERR_UNSUPPORTED;
+    if (N < 0) return DSA_ERR_INVALID_ARG;
+    if (N == 0) return DSA_OK;
+    if (!kidx_new || !k_new || !v_new || !seq_ids || !positions || !block_table || !kidx_cache ||
+        !kscale_cache || !k_cache || !v_cache)
+        return DSA_ERR_INVALID_ARG;
+    if (B <= 0 || max_pages_per_seq <= 0 || num_pages <= 0 || page_size <= 0 || d_I <= 0 || d <= 0)
+        return DSA_ERR_INVALID_ARG;
+    if (!aligned16(kidx_new) || !aligned16(k_new) || !aligned16(v_new) || !aligned16(k_cache) ||
+        !aligned16(v_cache) || (reinterpret_cast<uintptr_t>(kidx_cache) & 7u) ||
+        (reinterpret_cast<uintptr_t>(status) & 3u))
+        return DSA_ERR_INVALID_ARG;
+    if (d_I % 8 != 0 || d_I > 256 || d % 8 != 0) return DSA_ERR_UNSUPPORTED;
+    return cuda_status(launch_cache_append(kidx_new, kidx_dtype == DSA_BF16, (const uint16_t *)k_new,
+                                           (const uint16_t *)v_new, seq_ids, positions, N, B, block_table,
+                                           max_pages_per_seq, num_pages, page_size, d_I, d,
+                                           (uint8_t *)kidx_cache, kscale_cache, (uint16_t *)k_cache,
+                                           (uint16_t *)v_cache, status, as_stream(stream)));
 }
 
 dsa_status dsa_stream_status(void *workspace, void *stream)

@@ -27,12 +27,13 @@ cudaError_t launch_index_f32(const float *q, const float *k, const float *w, int
 
 // ---- top-k (topk.cu) ----
 // Row r: candidates scores[r*ld + s] for s < n_r, where n_r = lens[r] if
-// lens != nullptr, else row_begin + r + 1.  Output idx[r*k ...] ascending,
-// -1 padded.  Rows with lens[r] outside [1, max_len] are skipped (set to -1)
-// and reported in hdr.
+// lens != nullptr, else row_begin + r + 1.  Output idx[r*(k+window) ...]
+// ascending, -1 padded.  With window > 0 only s < n_r - window compete and
+// the window positions follow the selected ones.  Rows with lens[r] outside
+// [1, max_len] are skipped (set to -1) and reported in hdr.
 cudaError_t launch_topk_rows(const float *scores, int64_t ld, int64_t row_begin,
                              const int32_t *lens, int64_t max_len, int64_t row_count, int k,
-                             int32_t *idx, WsHeader *hdr, cudaStream_t st);
+                             int32_t *idx, WsHeader *hdr, cudaStream_t st, int window = 0);
 
 // Rows of lengths lens[r] (decode): each row split over CTAs of 16384
 // positions that share a sampled threshold and collect their candidates, then
@@ -41,7 +42,22 @@ cudaError_t launch_topk_rows(const float *scores, int64_t ld, int64_t row_begin,
 size_t topk_split_ws_bytes(int64_t rows, int64_t max_len);
 cudaError_t launch_topk_split(const float *scores, int64_t ld, const int32_t *lens, int64_t max_len,
                               int64_t rows, int k, int32_t *idx, void *ws_base, WsHeader *hdr,
-                              cudaStream_t st);
+                              cudaStream_t st, int window = 0);
+
+// ---- FP8 quantisation and cache append (quant.cu) ----
+// codes[r, :] / scale[r] of x[r, 0..cols) (bf16 or fp32), one scale per row;
+// cols a multiple of 8 and at most 16384, x 16-byte and codes 8-byte aligned.
+cudaError_t launch_quantize_e4m3(const void *x, bool bf16_in, int64_t rows, int cols, uint8_t *codes,
+                                 float *scale, cudaStream_t st);
+// Token i -> sequence seq[i], position pos[i] of the paged caches: quantised
+// index key (d_I <= 256, a multiple of 8), bf16 K and V rows (d a multiple
+// of 8).  Out-of-range tokens are skipped and DSA_ERR_INVALID_ARG is
+// recorded in *status (nullable).
+cudaError_t launch_cache_append(const void *kidx_new, bool bf16_in, const uint16_t *k_new,
+                                const uint16_t *v_new, const int32_t *seq, const int32_t *pos, int64_t N,
+                                int B, const int32_t *bt, int max_pages, int64_t num_pages, int ps,
+                                int d_I, int d, uint8_t *kidx_cache, float *kscale_cache,
+                                uint16_t *k_cache, uint16_t *v_cache, uint32_t *status, cudaStream_t st);
 
 // ---- sparse attention (sparse_attn.cu) ----
 struct PagedKV {

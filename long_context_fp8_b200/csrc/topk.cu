@@ -16,6 +16,11 @@
 // the bin holding the k-th largest key, the keys in or above it go on chip;
 // and if even those do not fit, a radix select runs over the row in global
 // memory.  Every path is exact; the guess only decides which one is taken.
+//
+// With a sliding window of W positions ("DeepSeek-V4 百万 token 上下文的工程实现",
+// section on the sliding-window KV cache: the most recent tokens keep their
+// full KV) only the positions before the window compete, and the W window
+// positions follow the selected ones in the output row of k + W entries.
 #include "kernels.h"
 
 namespace dsa {
@@ -546,9 +551,25 @@ __device__ __noinline__ void topk_row_histogram(TopkSmem &sm, const float *row, 
     else select_global(sm, row, n, vec, k, out);
 }
 
+// Row of n_all causal positions with a window of W: positions [0, n) compete
+// (n = n_all - W, or 0), [n, n_all) are always taken.  When n <= k the whole
+// row is selected, so out[i] = i for i < n_all, then -1 up to k + W.
+// Otherwise the top-k part fills out[0, k) and the window out[k, k + W).
+__device__ __forceinline__ void emit_window(int32_t *out, int k, int window, int64_t n)
+{
+    for (int i = threadIdx.x; i < window; i += TK_THREADS) out[k + i] = (int32_t)(n + i);
+}
+
+__device__ __forceinline__ bool emit_whole_row(int32_t *out, int k, int window, int64_t n, int64_t n_all)
+{
+    if (n > k) return false;
+    for (int i = threadIdx.x; i < k + window; i += TK_THREADS) out[i] = i < n_all ? i : -1;
+    return true;
+}
+
 __global__ void __launch_bounds__(TK_THREADS, 2)
 topk_rows_kernel(const float *__restrict__ scores, int64_t ld, int64_t row_begin,
-                 const int32_t *__restrict__ lens, int64_t max_len, int k,
+                 const int32_t *__restrict__ lens, int64_t max_len, int k, int window,
                  int32_t *__restrict__ idx, WsHeader *hdr, int vec_ok)
 {
     extern __shared__ __align__(16) uint8_t smem_raw[];
@@ -557,22 +578,21 @@ topk_rows_kernel(const float *__restrict__ scores, int64_t ld, int64_t row_begin
     const int64_t r = blockIdx.x;
     const int tid = threadIdx.x;
     const float *row = scores + r * ld;
-    int32_t *out = idx + r * (int64_t)k;
-    int64_t n;
+    int32_t *out = idx + r * (int64_t)(k + window);
+    int64_t n_all;
     if (lens) {
-        n = lens[r];
-        if (n < 1 || n > max_len) {
+        n_all = lens[r];
+        if (n_all < 1 || n_all > max_len) {
             if (tid == 0) record_error(hdr, DSA_ERR_INVALID_ARG, (unsigned)r);
-            for (int i = tid; i < k; i += TK_THREADS) out[i] = -1;
+            for (int i = tid; i < k + window; i += TK_THREADS) out[i] = -1;
             return;
         }
     } else {
-        n = row_begin + r + 1;
+        n_all = row_begin + r + 1;
     }
-    if (n <= k) {
-        for (int i = tid; i < k; i += TK_THREADS) out[i] = i < n ? i : -1;
-        return;
-    }
+    const int64_t n = n_all > window ? n_all - window : 0;     // positions before the window
+    if (emit_whole_row(out, k, window, n, n_all)) return;
+    emit_window(out, k, window, n);
     const bool vec = vec_ok != 0;
     if (tid == 0) { sm.sh_count = 0; sm.sh_overflow = 0; }
 
@@ -623,16 +643,23 @@ __device__ __forceinline__ int64_t split_len(const int32_t *lens, int64_t max_le
     return (n < 1 || n > max_len) ? -1 : n;
 }
 
+// Positions of a row of n_all (>= 0) that compete for the k slots.
+__device__ __forceinline__ int64_t before_window(int64_t n_all, int window)
+{
+    return n_all > window ? n_all - window : 0;
+}
+
 __global__ void __launch_bounds__(TK_THREADS, 2)
 topk_split_collect_kernel(const float *__restrict__ scores, int64_t ld, const int32_t *__restrict__ lens,
-                          int64_t max_len, int k, SplitWs ws, int vec_ok)
+                          int64_t max_len, int k, int window, SplitWs ws, int vec_ok)
 {
     extern __shared__ __align__(16) uint8_t smem_raw[];
     TopkSmem &sm = *reinterpret_cast<TopkSmem *>(smem_raw);
     grid_dep_wait();                                 // the scores of the kernel before
     grid_dep_trigger();
     const int64_t r = blockIdx.y;
-    const int64_t n = split_len(lens, max_len, r);
+    const int64_t n_all = split_len(lens, max_len, r);
+    const int64_t n = n_all < 0 ? -1 : before_window(n_all, window);
     const int64_t c0 = (int64_t)blockIdx.x * TS_CHUNK;
     if (n <= TK_CAP || c0 >= n) return;              // short or invalid rows: the final kernel alone
     const int64_t c1 = min(n, c0 + TS_CHUNK);
@@ -650,8 +677,8 @@ topk_split_collect_kernel(const float *__restrict__ scores, int64_t ld, const in
 
 __global__ void __launch_bounds__(TK_THREADS)
 topk_split_final_kernel(const float *__restrict__ scores, int64_t ld, const int32_t *__restrict__ lens,
-                        int64_t max_len, int k, SplitWs ws, int32_t *__restrict__ idx, WsHeader *hdr,
-                        int vec_ok)
+                        int64_t max_len, int k, int window, SplitWs ws, int32_t *__restrict__ idx,
+                        WsHeader *hdr, int vec_ok)
 {
     extern __shared__ __align__(16) uint8_t smem_raw[];
     TopkSmem &sm = *reinterpret_cast<TopkSmem *>(smem_raw);
@@ -659,17 +686,16 @@ topk_split_final_kernel(const float *__restrict__ scores, int64_t ld, const int3
     grid_dep_trigger();
     const int64_t r = blockIdx.x;
     const int tid = threadIdx.x;
-    int32_t *out = idx + r * (int64_t)k;
-    const int64_t n = split_len(lens, max_len, r);
-    if (n < 0) {
+    int32_t *out = idx + r * (int64_t)(k + window);
+    const int64_t n_all = split_len(lens, max_len, r);
+    if (n_all < 0) {
         if (tid == 0) record_error(hdr, DSA_ERR_INVALID_ARG, (unsigned)r);
-        for (int i = tid; i < k; i += TK_THREADS) out[i] = -1;
+        for (int i = tid; i < k + window; i += TK_THREADS) out[i] = -1;
         return;
     }
-    if (n <= k) {
-        for (int i = tid; i < k; i += TK_THREADS) out[i] = i < n ? i : -1;
-        return;
-    }
+    const int64_t n = before_window(n_all, window);
+    if (emit_whole_row(out, k, window, n, n_all)) return;
+    emit_window(out, k, window, n);
     const float *row = scores + r * ld;
     const bool vec = vec_ok != 0;
     if (n <= TK_CAP) {                               // short rows: every key is a candidate
@@ -703,14 +729,30 @@ topk_split_final_kernel(const float *__restrict__ scores, int64_t ld, const int3
         __syncthreads();
         use = use && total >= (uint32_t)k && total <= TK_CAP;
         if (use) {
-            // warp w copies chunks w, w + 16, ...: one memory latency per 16 chunks
-            const int lane = tid & 31, warp = tid >> 5;
-            for (int c = warp; c < nch; c += TK_WARPS) {
-                const uint32_t m = sm.sample[c], off = sm.hist[c];
-                const int64_t slot = (r * ws.chunks + c) * (int64_t)TS_SLOT;
-                for (uint32_t i = lane; i < m; i += 32) {
-                    sm.ckey[off + i] = ws.ckey[slot + i];
-                    sm.cpos[off + i] = ws.cpos[slot + i];
+            // Every thread copies joined entries tid, tid + 512, ... with four
+            // entries' loads in flight: entry i comes from the last chunk c whose
+            // offset hist[c] <= i (that chunk is never empty), at i - hist[c].
+            for (uint32_t base = 0; base < total; base += TK_THREADS * 4) {
+                uint32_t kk[4];
+                int32_t pp[4];
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const uint32_t i = base + (uint32_t)(q * TK_THREADS + tid);
+                    if (i < total) {
+                        int lo = 0, hi = nch - 1;
+                        while (lo < hi) {
+                            const int mid = (lo + hi + 1) >> 1;
+                            if (sm.hist[mid] <= i) lo = mid; else hi = mid - 1;
+                        }
+                        const int64_t src = (r * ws.chunks + lo) * (int64_t)TS_SLOT + (i - sm.hist[lo]);
+                        kk[q] = ws.ckey[src];
+                        pp[q] = ws.cpos[src];
+                    }
+                }
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const uint32_t i = base + (uint32_t)(q * TK_THREADS + tid);
+                    if (i < total) { sm.ckey[i] = kk[q]; sm.cpos[i] = pp[q]; }
                 }
             }
             __syncthreads();
@@ -726,7 +768,7 @@ topk_split_final_kernel(const float *__restrict__ scores, int64_t ld, const int3
 
 cudaError_t launch_topk_rows(const float *scores, int64_t ld, int64_t row_begin,
                              const int32_t *lens, int64_t max_len, int64_t row_count, int k,
-                             int32_t *idx, WsHeader *hdr, cudaStream_t st)
+                             int32_t *idx, WsHeader *hdr, cudaStream_t st, int window)
 {
     if (row_count <= 0) return cudaSuccess;
     const size_t smem = sizeof(TopkSmem);
@@ -735,7 +777,7 @@ cudaError_t launch_topk_rows(const float *scores, int64_t ld, int64_t row_begin,
     if (e != cudaSuccess) return e;
     const int vec_ok = (ld % 4 == 0) && ((reinterpret_cast<uintptr_t>(scores) & 15u) == 0);
     topk_rows_kernel<<<(unsigned)row_count, TK_THREADS, smem, st>>>(scores, ld, row_begin, lens,
-                                                                     max_len, k, idx, hdr, vec_ok);
+                                                                     max_len, k, window, idx, hdr, vec_ok);
     return cudaGetLastError();
 }
 
@@ -748,7 +790,7 @@ size_t topk_split_ws_bytes(int64_t rows, int64_t max_len)
 
 cudaError_t launch_topk_split(const float *scores, int64_t ld, const int32_t *lens, int64_t max_len,
                               int64_t rows, int k, int32_t *idx, void *ws_base, WsHeader *hdr,
-                              cudaStream_t st)
+                              cudaStream_t st, int window)
 {
     if (rows <= 0) return cudaSuccess;
     const int64_t chunks = ceil_div(max_len, TS_CHUNK);
@@ -768,10 +810,10 @@ cudaError_t launch_topk_split(const float *scores, int64_t ld, const int32_t *le
     if (e != cudaSuccess) return e;
     dim3 grid((unsigned)chunks, (unsigned)rows);
     e = launch_chained(topk_split_collect_kernel, grid, dim3(TK_THREADS), smem, st, scores, ld, lens,
-                       max_len, k, ws, vec_ok);
+                       max_len, k, window, ws, vec_ok);
     if (e != cudaSuccess) return e;
     e = launch_chained(topk_split_final_kernel, dim3((unsigned)rows), dim3(TK_THREADS), smem, st, scores,
-                       ld, lens, max_len, k, ws, idx, hdr, vec_ok);
+                       ld, lens, max_len, k, window, ws, idx, hdr, vec_ok);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }

@@ -24,9 +24,10 @@ STATUS = {0: "DSA_OK", 1: "DSA_ERR_INVALID_ARG", 2: "DSA_ERR_UNSUPPORTED", 3: "D
 
 # Every symbol include/dsa.h declares.
 EXPORTS = ("dsa_status_string", "dsa_version", "dsa_index_scores", "dsa_topk_workspace_size",
-           "dsa_topk", "dsa_sparse_attn", "dsa_prefill_workspace_size", "dsa_prefill",
-           "dsa_prefill_host_workspace_size", "dsa_prefill_host",
-           "dsa_decode_workspace_size", "dsa_decode", "dsa_decode_noalloc", "dsa_stream_status")
+           "dsa_topk", "dsa_topk_window", "dsa_sparse_attn", "dsa_prefill_workspace_size",
+           "dsa_prefill", "dsa_prefill_window", "dsa_prefill_host_workspace_size", "dsa_prefill_host",
+           "dsa_decode_workspace_size", "dsa_decode", "dsa_decode_window", "dsa_quantize_e4m3",
+           "dsa_cache_append", "dsa_decode_noalloc", "dsa_stream_status")
 
 
 class DSAError(RuntimeError):
@@ -67,6 +68,14 @@ def load(path: str = LIB_PATH):
                         I32, F, P, P, P, P, SZ, P], I32),
         "dsa_decode_noalloc": ([P, P, P, P, P, P, P, P, P, P, I64, I32, I32, I32, I64, I32, I32, I32,
                                 I32, I32, F, P, P, P, P, P], I32),
+        "dsa_topk_window": ([P, I64, I64, I64, I64, I32, I32, P, P, SZ, P], I32),
+        "dsa_prefill_window": ([P, P, P, P, P, P, P, P, I64, I32, I32, I32, I32, I32, I32, F, P, P, P,
+                                I32, P, SZ, P], I32),
+        "dsa_decode_window": ([P, P, P, P, P, P, P, P, P, P, I64, I32, I32, I32, I64, I32, I32, I32, I32,
+                               I32, I32, F, P, P, P, P, SZ, P], I32),
+        "dsa_quantize_e4m3": ([P, I32, I64, I64, P, P, P], I32),
+        "dsa_cache_append": ([P, I32, P, P, P, P, I64, I32, P, I32, I64, I32, I32, I32, P, P, P, P, P, P],
+                             I32),
         "dsa_stream_status": ([P, P], I32),
     }
     for name, (args, res) in sig.items():
@@ -154,6 +163,49 @@ def dsa_topk(scores, k, row_begin=0, T=None, out=None, stream=None):
     return out
 
 
+def dsa_topk_window(scores, k, window, row_begin=0, T=None, out=None, stream=None):
+    """Sliding window plus top-k of score rows -> int32 [rows, k + window]."""
+    rows, ld = scores.shape
+    T = ld if T is None else T
+    if out is None:
+        out = torch.empty((rows, k + window), dtype=torch.int32, device=scores.device)
+    st = load().dsa_topk_window(_p(scores), ld, row_begin, rows, T, k, window, _p(out), None, 0,
+                                _stream(stream))
+    _check("dsa_topk_window", st)
+    return out
+
+
+def dsa_quantize_e4m3(x, codes=None, scale=None, stream=None):
+    """Per-row FP8 E4M3 quantisation of bf16/fp32 ``x[rows, ...]`` ->
+    (uint8 codes of x's shape, fp32 scale[rows])."""
+    rows = x.shape[0]
+    cols = x.numel() // max(rows, 1) if rows else (x[0].numel() if x.dim() > 1 else 1)
+    if codes is None:
+        codes = torch.empty(x.shape, dtype=torch.uint8, device=x.device)
+    if scale is None:
+        scale = torch.empty((rows,), dtype=torch.float32, device=x.device)
+    st = load().dsa_quantize_e4m3(_p(x), _val_dtype(x), rows, cols, _p(codes), _p(scale), _stream(stream))
+    _check("dsa_quantize_e4m3", st)
+    return codes, scale
+
+
+def dsa_cache_append(caches: dict, kidx_new, k_new, v_new, seq_ids, positions, block_table,
+                     status=None, stream=None):
+    """Quantise and write N new tokens' index keys and copy their K/V rows into
+    the paged caches (``caches``: kidx_cache, kscale_cache, k_cache, v_cache,
+    updated in place).  ``status``: optional int32 [1] device tensor that
+    receives DSA_ERR_INVALID_ARG for an out-of-range token."""
+    N, d_I = kidx_new.shape
+    d = k_new.shape[1]
+    P, ps, _ = caches["kidx_cache"].shape
+    B, max_pages = block_table.shape
+    st = load().dsa_cache_append(_p(kidx_new), _val_dtype(kidx_new), _p(k_new), _p(v_new), _p(seq_ids),
+                                 _p(positions), N, B, _p(block_table), max_pages, P, ps, d_I, d,
+                                 _p(caches["kidx_cache"]), _p(caches["kscale_cache"]), _p(caches["k_cache"]),
+                                 _p(caches["v_cache"]), _p(status), _stream(stream))
+    _check("dsa_cache_append", st)
+
+
 def dsa_sparse_attn(q, k, v, idx, sm_scale=None, out=None, lse=None, stream=None):
     """Attention of each query row over its selected K/V rows -> (out, lse)."""
     T, H, D = q.shape
@@ -195,6 +247,32 @@ def dsa_prefill(inp: dict, k_sel: int, sm_scale=None, out=None, lse=None, idx_ou
                          k_sel, sm_scale, _p(out), _p(lse), _p(idx_out), dt, _p(ws), ws.numel(),
                          _stream(stream))
     _check("dsa_prefill", st)
+    return out, lse, idx_out
+
+
+def dsa_prefill_window(inp: dict, k_sel: int, window: int, sm_scale=None, out=None, lse=None,
+                       idx_out=None, ws=None, want_idx=True, stream=None):
+    """dsa_prefill with a sliding window: the last `window` positions of every
+    query are always attended, top-k over the older ones; idx [T, k_sel + window]."""
+    q_idx, q = inp["q_idx"], inp["q"]
+    T, H_I, d_I = q_idx.shape
+    _, H_q, d = q.shape
+    dt = _idx_dtype(q_idx)
+    sm_scale = 1.0 / math.sqrt(d) if sm_scale is None else sm_scale
+    lib = load()
+    if ws is None:
+        ws = workspace(lib.dsa_prefill_workspace_size(T, H_I, d_I, H_q, d, k_sel + window, dt), q.device)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((T, H_q), dtype=torch.float32, device=q.device)
+    if idx_out is None and want_idx:
+        idx_out = torch.empty((T, k_sel + window), dtype=torch.int32, device=q.device)
+    st = lib.dsa_prefill_window(_p(q_idx), _p(inp["q_scale"]), _p(inp["k_idx"]), _p(inp["k_scale"]),
+                                _p(inp["w"]), _p(q), _p(inp["k"]), _p(inp["v"]), T, H_I, d_I, H_q, d,
+                                k_sel, window, sm_scale, _p(out), _p(lse), _p(idx_out), dt, _p(ws),
+                                ws.numel(), _stream(stream))
+    _check("dsa_prefill_window", st)
     return out, lse, idx_out
 
 
@@ -262,6 +340,35 @@ def dsa_decode(inp: dict, k_sel: int, max_context: int, sm_scale=None, out=None,
                         P, max_pages, ps, B, max_context, H_I, d_I, H_q, d, k_sel, sm_scale,
                         _p(out), _p(lse), _p(idx_out), _p(ws), ws.numel(), _stream(stream))
     _check("dsa_decode", st)
+    return out, lse, idx_out
+
+
+def dsa_decode_window(inp: dict, k_sel: int, window: int, max_context: int, sm_scale=None, out=None,
+                      lse=None, idx_out=None, ws=None, want_idx=True, stream=None):
+    """dsa_decode with a sliding window (the last `window` cached positions of
+    each sequence always attended) -> (out, lse, idx [B, k_sel + window])."""
+    B, H_I, d_I = inp["q_idx"].shape
+    _, H_q, d = inp["q"].shape
+    P, ps, _ = inp["kidx_cache"].shape
+    max_pages = inp["block_table"].shape[1]
+    sm_scale = 1.0 / math.sqrt(d) if sm_scale is None else sm_scale
+    lib = load()
+    kw = k_sel + window
+    if ws is None:
+        ws = workspace(lib.dsa_decode_workspace_size(B, max_context, H_q, d, kw), inp["q"].device)
+    if out is None:
+        out = torch.empty_like(inp["q"])
+    if lse is None:
+        lse = torch.empty((B, H_q), dtype=torch.float32, device=inp["q"].device)
+    if idx_out is None and want_idx:
+        idx_out = torch.empty((B, kw), dtype=torch.int32, device=inp["q"].device)
+    st = lib.dsa_decode_window(_p(inp["q_idx"]), _p(inp["q_scale"]), _p(inp["w"]), _p(inp["q"]),
+                               _p(inp["kidx_cache"]), _p(inp["kscale_cache"]), _p(inp["k_cache"]),
+                               _p(inp["v_cache"]), _p(inp["block_table"]), _p(inp["context_lens"]),
+                               P, max_pages, ps, B, max_context, H_I, d_I, H_q, d, k_sel, window,
+                               sm_scale, _p(out), _p(lse), _p(idx_out), _p(ws), ws.numel(),
+                               _stream(stream))
+    _check("dsa_decode_window", st)
     return out, lse, idx_out
 
 
