@@ -55,8 +55,28 @@ __device__ __forceinline__ float e4m3_scale_of(float amax)
     return s > 0.0f ? s : 1.0f;
 }
 
-// Eight codes of v / s, packed little-endian (value i in byte i).
-__device__ __forceinline__ uint2 e4m3_codes8(const float (&v)[QZ_VEC], float s)
+// The quotient v / s that decides a code, taken cheaply where that is exact.
+// With r = RN(1 / s), the product q' = RN(v * r) equals (v / s)(1 + d1)(1 + d2)
+// with |d1|, |d2| <= 2^-24, so it lies within 2 ulps of v / s, and the IEEE
+// quotient q = RN(v / s) within half an ulp of it: q and q' are at most 3 ulps
+// apart.  The E4M3 rounding of a value only changes at the midpoints between
+// neighbouring codes; for |q'| >= 2^-6 (the normal E4M3 range) those are the
+// fp32 values whose low 20 mantissa bits are 0x80000 (code spacing 2^20 fp32
+// ulps, midpoint half-way), so if q' is more than 4 ulps from such a pattern,
+// q and q' round to the same code.  Otherwise -- near a midpoint, below 2^-6
+// (the E4M3 subnormal range), or when r is not finite (s below 2^-126) -- the
+// IEEE division decides.
+__device__ __forceinline__ float e4m3_quotient(float v, float s, float r, bool r_ok)
+{
+    const float q = v * r;
+    const uint32_t b = __float_as_uint(q);
+    const int d = (int)(b & 0xFFFFFu) - 0x80000;
+    const bool safe = r_ok && fabsf(q) >= 0.015625f && (d > 4 || d < -4);
+    return safe ? q : __fdiv_rn(v, s);
+}
+
+// Eight codes of v / s, packed little-endian (value i in byte i); r = RN(1 / s).
+__device__ __forceinline__ uint2 e4m3_codes8(const float (&v)[QZ_VEC], float s, float r, bool r_ok)
 {
     uint32_t w[2];
 #pragma unroll
@@ -65,14 +85,22 @@ __device__ __forceinline__ uint2 e4m3_codes8(const float (&v)[QZ_VEC], float s)
 #pragma unroll
         for (int i = 0; i < 2; ++i) {
             float2 pr;
-            pr.x = __fdiv_rn(v[4 * h + 2 * i], s);
-            pr.y = __fdiv_rn(v[4 * h + 2 * i + 1], s);
+            pr.x = e4m3_quotient(v[4 * h + 2 * i], s, r, r_ok);
+            pr.y = e4m3_quotient(v[4 * h + 2 * i + 1], s, r, r_ok);
             const __nv_fp8x2_storage_t c = __nv_cvt_float2_to_fp8x2(pr, __NV_SATFINITE, __NV_E4M3);
             word |= (uint32_t)c << (16 * i);
         }
         w[h] = word;
     }
     return make_uint2(w[0], w[1]);
+}
+
+// RN(1 / s) and whether it is finite (it is not for s below 2^-126 or so).
+__device__ __forceinline__ float e4m3_recip(float s, bool &ok)
+{
+    const float r = __frcp_rn(s);
+    ok = isfinite(r);
+    return r;
 }
 
 // Rows of `cols` values (cols a multiple of 8, at most TPR * 8 * NCH), TPR
@@ -112,13 +140,15 @@ quantize_rows_kernel(const In *__restrict__ x, int64_t rows, int cols, uint8_t *
             __syncthreads();                         // red is reused by the next row
         }
         const float s = e4m3_scale_of(amax);
+        bool r_ok;
+        const float rs = e4m3_recip(s, r_ok);
         if (!live) continue;
         if (sub == 0) scale[r] = s;
 #pragma unroll
         for (int c = 0; c < NCH; ++c) {
             const int ch = sub + c * TPR;
             if (ch < nch)
-                *reinterpret_cast<uint2 *>(codes + r * cols + (int64_t)ch * QZ_VEC) = e4m3_codes8(v[c], s);
+                *reinterpret_cast<uint2 *>(codes + r * cols + (int64_t)ch * QZ_VEC) = e4m3_codes8(v[c], s, rs, r_ok);
         }
     }
 }
@@ -186,8 +216,10 @@ cache_append_kernel(const In *__restrict__ kidx_new, const uint16_t *__restrict_
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
         const float s = e4m3_scale_of(amax);
+        bool r_ok;
+        const float rs = e4m3_recip(s, r_ok);
         if (lane < nch)
-            *reinterpret_cast<uint2 *>(kidx_cache + slot * d_I + lane * QZ_VEC) = e4m3_codes8(v, s);
+            *reinterpret_cast<uint2 *>(kidx_cache + slot * d_I + lane * QZ_VEC) = e4m3_codes8(v, s, rs, r_ok);
         if (lane == 0) kscale_cache[slot] = s;
         // K and V rows: 16-byte chunks
         const int vch = d / 8;

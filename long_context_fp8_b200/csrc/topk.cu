@@ -26,25 +26,44 @@
 namespace dsa {
 namespace {
 
-constexpr int TK_THREADS = 512;
-constexpr int TK_WARPS = TK_THREADS / 32;
 constexpr int TK_ITEMS = 8;                          // consecutive positions per thread per step
-constexpr int TK_STEP = TK_THREADS * TK_ITEMS;       // positions per block-wide step
-constexpr int TK_CAP = 8192;                         // shared-memory candidate capacity (two CTAs fit an SM)
 
-constexpr int TK_SAMPLE = 2048;                     // evenly spaced samples for the threshold guess
+// Launch shape of a top-k kernel: NT threads per CTA, a shared-memory
+// candidate buffer of CAP entries, NSAMP samples for the threshold guess,
+// taken one by one at evenly spaced positions or (RUNS) as runs of 8
+// consecutive positions (one 32-byte sector each, instead of a sector per
+// sample), kept in the candidate buffer, which is free until the guess is made.
+template <int NT_, int CAP_, int NSAMP_, bool RUNS_>
+struct TopkCfg {
+    static constexpr int NT = NT_;
+    static constexpr int WARPS = NT_ / 32;
+    static constexpr int STEP = NT_ * TK_ITEMS;      // positions per block-wide step
+    static constexpr int CAP = CAP_;
+    static constexpr int WCAP = CAP_ / WARPS;        // candidate slots per warp
+    static constexpr int NSAMP = NSAMP_;
+    static constexpr bool RUNS = RUNS_;
+    static_assert(!RUNS_ || (NSAMP_ <= CAP_ && NSAMP_ % (8 * NT_) == 0), "sample runs must fit the buffer");
+};
+// Causal prefill rows: two 512-thread CTAs per SM; 4096 threshold samples in
+// runs of 8 (a sector each) kept in the candidate buffer.
+using RowsCfg = TopkCfg<512, 8192, 4096, true>;
+// Decode rows split over CTAs (and the final join of their candidates).
+using SplitCfg = TopkCfg<512, 8192, 2048, false>;
 
+template <class C>
 struct TopkSmem {
     uint32_t hist[2048];
     uint32_t warp_buf[32];
     uint32_t sh_bin, sh_above, sh_count, sh_overflow, sh_diff;
-    uint32_t wcnt[TK_WARPS], wbefore[TK_WARPS + 1];
-    uint32_t sample[TK_SAMPLE];
-    uint32_t ckey[TK_CAP];
-    int32_t cpos[TK_CAP];
+    uint32_t wcnt[C::WARPS], wbefore[C::WARPS + 1];
+    uint32_t sample_store[C::RUNS ? 1 : C::NSAMP];
+    uint32_t ckey[C::CAP];
+    int32_t cpos[C::CAP];
+    __device__ __forceinline__ uint32_t *sample() { return C::RUNS ? ckey : sample_store; }
 };
 
 // Exclusive block-wide prefix sum of `v`; the block total goes to *total.
+template <class C>
 __device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t *warp_buf, uint32_t *total)
 {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -57,17 +76,17 @@ __device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t *warp_b
     if (lane == 31) warp_buf[warp] = x;
     __syncthreads();
     if (warp == 0) {
-        uint32_t s = lane < TK_WARPS ? warp_buf[lane] : 0u;
+        uint32_t s = lane < C::WARPS ? warp_buf[lane] : 0u;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
             uint32_t y = __shfl_up_sync(0xffffffffu, s, o);
             if (lane >= o) s += y;
         }
-        if (lane < TK_WARPS) warp_buf[lane] = s;
+        if (lane < C::WARPS) warp_buf[lane] = s;
     }
     __syncthreads();
     uint32_t before = (warp > 0 ? warp_buf[warp - 1] : 0u) + x - v;
-    *total = warp_buf[TK_WARPS - 1];
+    *total = warp_buf[C::WARPS - 1];
     __syncthreads();
     return before;
 }
@@ -110,17 +129,18 @@ __device__ __forceinline__ void load8(const float *row, int64_t n, int64_t s, bo
 
 // Bin holding the `remaining`-th largest count (from the top), and how many
 // counts lie strictly above it.  All threads call it; results in smem.
-__device__ __forceinline__ void find_bin(TopkSmem &sm, int nb, uint32_t remaining)
+template <class C>
+__device__ __forceinline__ void find_bin(TopkSmem<C> &sm, int nb, uint32_t remaining)
 {
     const int tid = threadIdx.x;
-    const int bpt = nb > TK_THREADS ? nb / TK_THREADS : 1;     // nb: a power of two
+    const int bpt = nb > C::NT ? nb / C::NT : 1;     // nb: a power of two
     uint32_t local = 0;
     for (int j = 0; j < bpt; ++j) {
         const int b = nb - 1 - (tid * bpt + j);
         if (b >= 0) local += sm.hist[b];
     }
     uint32_t tot;
-    uint32_t cum = block_excl_scan(local, sm.warp_buf, &tot);
+    uint32_t cum = block_excl_scan<C>(local, sm.warp_buf, &tot);
     for (int j = 0; j < bpt; ++j) {
         const int b = nb - 1 - (tid * bpt + j);
         if (b < 0) break;
@@ -133,13 +153,13 @@ __device__ __forceinline__ void find_bin(TopkSmem &sm, int nb, uint32_t remainin
 
 // Ordered compaction of a key sequence given by get(i) for i in [0, n):
 // emits pos(i) for keys above thr and for the first `need` keys equal to thr.
-template <class GetKey, class GetPos>
-__device__ __forceinline__ void emit_selected(TopkSmem &sm, int64_t n, uint32_t thr, uint32_t need,
+template <class C, class GetKey, class GetPos>
+__device__ __forceinline__ void emit_selected(TopkSmem<C> &sm, int64_t n, uint32_t thr, uint32_t need,
                                               int k, int32_t *out, GetKey get, GetPos pos_of)
 {
     const int tid = threadIdx.x;
     uint32_t base_gt = 0, base_eq = 0;
-    for (int64_t c0 = 0; c0 < n; c0 += TK_STEP) {
+    for (int64_t c0 = 0; c0 < n; c0 += C::STEP) {
         const int64_t i0 = c0 + (int64_t)tid * TK_ITEMS;
         uint32_t flags_gt = 0, flags_eq = 0, n_gt = 0, n_eq = 0;
         uint32_t keys[TK_ITEMS], valid;
@@ -152,7 +172,7 @@ __device__ __forceinline__ void emit_selected(TopkSmem &sm, int64_t n, uint32_t 
             }
         }
         uint32_t tot;
-        uint32_t ex = block_excl_scan((n_gt << 16) | n_eq, sm.warp_buf, &tot);
+        uint32_t ex = block_excl_scan<C>((n_gt << 16) | n_eq, sm.warp_buf, &tot);
         uint32_t gt_before = base_gt + (ex >> 16), eq_before = base_eq + (ex & 0xffffu);
 #pragma unroll
         for (int i = 0; i < TK_ITEMS; ++i) {
@@ -172,7 +192,8 @@ __device__ __forceinline__ void emit_selected(TopkSmem &sm, int64_t n, uint32_t 
 // Given the candidates (every key whose top 11 bits are >= b1, in ascending
 // position order) in shared memory, resolve the remaining 21 bits of the
 // threshold on chip and emit the selection in position order.
-__device__ __noinline__ void select_on_chip(TopkSmem &sm, uint32_t ncand, uint32_t b1, uint32_t remaining, int k,
+template <class C>
+__device__ __noinline__ void select_on_chip(TopkSmem<C> &sm, uint32_t ncand, uint32_t b1, uint32_t remaining, int k,
                                int32_t *out)
 {
     const int tid = threadIdx.x;
@@ -182,9 +203,9 @@ __device__ __noinline__ void select_on_chip(TopkSmem &sm, uint32_t ncand, uint32
         const int shift = pass == 0 ? 10 : 0;
         const int nb = pass == 0 ? 2048 : 1024;
         const uint32_t bmask = (uint32_t)nb - 1u;
-        for (int i = tid; i < nb; i += TK_THREADS) sm.hist[i] = 0u;
+        for (int i = tid; i < nb; i += C::NT) sm.hist[i] = 0u;
         __syncthreads();
-        for (uint32_t j = tid; j < ncand; j += TK_THREADS) {
+        for (uint32_t j = tid; j < ncand; j += C::NT) {
             uint32_t key = sm.ckey[j];
             if ((key & pmask) == prefix) atomicAdd(&sm.hist[(key >> shift) & bmask], 1u);
         }
@@ -215,7 +236,8 @@ __device__ __noinline__ void select_on_chip(TopkSmem &sm, uint32_t ncand, uint32
 // over the keys' actual range instead of piling onto one bin of the top bits.
 // With passes = 3 the result is exact; with fewer, the bits not yet resolved
 // are zero in *thr (a threshold at or below the exact key).
-__device__ void radix_select_smem(TopkSmem &sm, const uint32_t *keys, uint32_t n, uint32_t rank,
+template <class C>
+__device__ void radix_select_smem(TopkSmem<C> &sm, const uint32_t *keys, uint32_t n, uint32_t rank,
                                   uint32_t *thr, uint32_t *need, int passes = 3)
 {
     const int tid = threadIdx.x;
@@ -223,7 +245,7 @@ __device__ void radix_select_smem(TopkSmem &sm, const uint32_t *keys, uint32_t n
     if (tid == 0) sm.sh_diff = 0u;
     __syncthreads();
     uint32_t diff = 0;
-    for (uint32_t j = tid; j < n; j += TK_THREADS) diff |= keys[j] ^ first;
+    for (uint32_t j = tid; j < n; j += C::NT) diff |= keys[j] ^ first;
     diff = __reduce_or_sync(0xffffffffu, diff);
     if ((tid & 31) == 0 && diff) atomicOr(&sm.sh_diff, diff);
     __syncthreads();
@@ -243,9 +265,9 @@ __device__ void radix_select_smem(TopkSmem &sm, const uint32_t *keys, uint32_t n
         const int shift = lo - width;
         const int nb = 1 << width;
         const uint32_t bmask = (uint32_t)nb - 1u;
-        for (int i = tid; i < nb; i += TK_THREADS) sm.hist[i] = 0u;
+        for (int i = tid; i < nb; i += C::NT) sm.hist[i] = 0u;
         __syncthreads();
-        for (uint32_t j = tid; j < n; j += TK_THREADS) {
+        for (uint32_t j = tid; j < n; j += C::NT) {
             const uint32_t key = keys[j];
             if ((key & pmask) == prefix) atomicAdd(&sm.hist[(key >> shift) & bmask], 1u);
         }
@@ -264,7 +286,7 @@ __device__ void radix_select_smem(TopkSmem &sm, const uint32_t *keys, uint32_t n
             uint32_t *bk = sm.hist;
             if (tid == 0) sm.sh_count = 0u;
             __syncthreads();
-            for (uint32_t j = tid; j < n; j += TK_THREADS) {
+            for (uint32_t j = tid; j < n; j += C::NT) {
                 const uint32_t key = keys[j];
                 if ((key & pmask) == prefix) bk[atomicAdd(&sm.sh_count, 1u)] = key;
             }
@@ -291,7 +313,8 @@ __device__ void radix_select_smem(TopkSmem &sm, const uint32_t *keys, uint32_t n
 
 // Exact select among the candidates in shared memory (every key that could
 // be selected, in ascending position order), emitted in position order.
-__device__ void select_candidates(TopkSmem &sm, uint32_t ncand, int k, int32_t *out)
+template <class C>
+__device__ void select_candidates(TopkSmem<C> &sm, uint32_t ncand, int k, int32_t *out)
 {
     uint32_t thr, need;
     radix_select_smem(sm, sm.ckey, ncand, (uint32_t)k, &thr, &need);
@@ -309,11 +332,11 @@ __device__ void select_candidates(TopkSmem &sm, uint32_t ncand, int k, int32_t *
 }
 
 // Ordered copy of every key of the row that passes `keep` into the candidate
-// buffer; returns the total count (entries past TK_CAP are counted, not
+// buffer; returns the total count (entries past C::CAP are counted, not
 // stored).  Each thread takes 8 consecutive positions per step (two 16-byte
 // loads), one block scan per 4K positions.
-template <class Keep>
-__device__ uint32_t collect_candidates(TopkSmem &sm, const float *row, int64_t n, bool vec, Keep keep)
+template <class C, class Keep>
+__device__ uint32_t collect_candidates(TopkSmem<C> &sm, const float *row, int64_t n, bool vec, Keep keep)
 {
     constexpr int D = 2;                                   // steps of loads in flight
     const int tid = threadIdx.x;
@@ -321,26 +344,26 @@ __device__ uint32_t collect_candidates(TopkSmem &sm, const float *row, int64_t n
     float ring[D][TK_ITEMS];
 #pragma unroll
     for (int q = 0; q < D; ++q)
-        if ((int64_t)q * TK_STEP < n) load_raw8(row, n, (int64_t)q * TK_STEP + (int64_t)tid * TK_ITEMS, vec, ring[q]);
-    for (int64_t c0 = 0; c0 < n; c0 += (int64_t)D * TK_STEP) {
+        if ((int64_t)q * C::STEP < n) load_raw8(row, n, (int64_t)q * C::STEP + (int64_t)tid * TK_ITEMS, vec, ring[q]);
+    for (int64_t c0 = 0; c0 < n; c0 += (int64_t)D * C::STEP) {
 #pragma unroll
         for (int q = 0; q < D; ++q) {
-            const int64_t cq = c0 + (int64_t)q * TK_STEP;
+            const int64_t cq = c0 + (int64_t)q * C::STEP;
             if (cq >= n) break;                            // block-uniform
             const int64_t s0 = cq + (int64_t)tid * TK_ITEMS;
             uint32_t keys[TK_ITEMS], valid;
             keys_of(ring[q], n, s0, keys, valid);
-            if (cq + (int64_t)D * TK_STEP < n) load_raw8(row, n, s0 + (int64_t)D * TK_STEP, vec, ring[q]);
+            if (cq + (int64_t)D * C::STEP < n) load_raw8(row, n, s0 + (int64_t)D * C::STEP, vec, ring[q]);
             uint32_t flags = 0, cnt = 0;
 #pragma unroll
             for (int i = 0; i < TK_ITEMS; ++i)
                 if (((valid >> i) & 1u) && keep(keys[i])) { flags |= 1u << i; ++cnt; }
             uint32_t tot;
-            uint32_t off = base + block_excl_scan(cnt, sm.warp_buf, &tot);
+            uint32_t off = base + block_excl_scan<C>(cnt, sm.warp_buf, &tot);
 #pragma unroll
             for (int i = 0; i < TK_ITEMS; ++i) {
                 if ((flags >> i) & 1u) {
-                    if (off < TK_CAP) { sm.ckey[off] = keys[i]; sm.cpos[off] = (int32_t)(s0 + i); }
+                    if (off < C::CAP) { sm.ckey[off] = keys[i]; sm.cpos[off] = (int32_t)(s0 + i); }
                     ++off;
                 }
             }
@@ -357,42 +380,68 @@ __device__ __forceinline__ float key_float(uint32_t key)
     return __uint_as_float((key & 0x80000000u) ? (key & 0x7fffffffu) : ~key);
 }
 
-constexpr int TK_WCAP = TK_CAP / TK_WARPS;          // candidate slots per warp
 
 // Candidates x >= tau_f of the row, in ascending position order, into
 // sm.ckey / sm.cpos[0, count).  Each warp scans its own contiguous chunk of
-// the row (four steps of 256 scores in flight, warp-level ordered
-// compaction, no block barrier) into its own TK_WCAP slots; one barrier, then
-// the warps' lists are packed in warp order.  Returns the count, or
-// 0xffffffff if a warp's chunk held more than TK_WCAP candidates (the caller
-// falls back).
-__device__ uint32_t collect_above_warp(TopkSmem &sm, const float *row, int64_t n, bool vec, float tau_f)
+// the row (two steps of 512 scores in flight, warp-level ordered
+// compaction, no block barrier) into its own WCAP slots; one barrier, then
+// the warps' lists are packed in warp order.  The scan is issue-bound, so it
+// keeps per-score work minimal: full steps skip the bounds test, positions
+// are 32-bit (rows are shorter than 2^31), and the slots hold the raw score
+// bits, turned into keys by the pack pass, which touches every candidate
+// anyway.  Returns the count, or 0xffffffff if a warp's chunk held more than
+// WCAP candidates (the caller falls back).
+// Raw scores of positions [s, s + 16) of a row (0 past n): four 16-byte loads.
+__device__ __forceinline__ void load_raw16(const float *row, int n, int s, bool vec, float (&v)[16])
 {
-    constexpr int D = 4;
+    if (vec && s + 16 <= n) {
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const float4 a = __ldg(reinterpret_cast<const float4 *>(row + s + 4 * j));
+            v[4 * j] = a.x; v[4 * j + 1] = a.y; v[4 * j + 2] = a.z; v[4 * j + 3] = a.w;
+        }
+    } else {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) v[i] = s + i < n ? row[s + i] : 0.f;
+    }
+}
+
+template <class C>
+__device__ uint32_t collect_above_warp(TopkSmem<C> &sm, const float *row, int64_t n_, bool vec, float tau_f)
+{
+    // Steps of 512 scores per warp (16 per lane), two in flight: the per-step
+    // cost (ordered prefix over the lanes, candidate writes) is paid once per
+    // 2 KB, which measured markedly faster than 1 KB steps four deep.
+    constexpr int D = 2, IT = 16, SW = 32 * IT;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int64_t per = ((n + TK_WARPS - 1) / TK_WARPS + 255) / 256 * 256;
-    const int64_t w0 = (int64_t)warp * per, w1 = min(n, w0 + per);
-    uint32_t *wk = sm.ckey + warp * TK_WCAP;
-    int32_t *wp = sm.cpos + warp * TK_WCAP;
+    const int n = (int)n_;
+    const int per = ((n + C::WARPS - 1) / C::WARPS + SW - 1) / SW * SW;
+    const int w0 = warp * per, w1 = min(n, w0 + per);
+    uint32_t *wk = sm.ckey + warp * C::WCAP;
+    int32_t *wp = sm.cpos + warp * C::WCAP;
     uint32_t cnt = 0;                                      // warp-uniform
-    float ring[D][TK_ITEMS];
+    float ring[D][IT];
 #pragma unroll
     for (int q = 0; q < D; ++q)
-        if (w0 + q * 256 < w1) load_raw8(row, w1, w0 + q * 256 + lane * TK_ITEMS, vec, ring[q]);
-    for (int64_t c0 = w0; c0 < w1; c0 += D * 256) {
+        if (w0 + q * SW < w1) load_raw16(row, w1, w0 + q * SW + lane * IT, vec, ring[q]);
+    for (int c0 = w0; c0 < w1; c0 += D * SW) {
 #pragma unroll
         for (int q = 0; q < D; ++q) {
-            const int64_t cq = c0 + q * 256;
+            const int cq = c0 + q * SW;
             if (cq >= w1) break;                           // warp-uniform
-            const int64_t s0 = cq + lane * TK_ITEMS;
-            float v[TK_ITEMS];
+            const int s0 = cq + lane * IT;
+            float v[IT];
 #pragma unroll
-            for (int i = 0; i < TK_ITEMS; ++i) v[i] = ring[q][i];
-            if (cq + D * 256 < w1) load_raw8(row, w1, s0 + D * 256, vec, ring[q]);
+            for (int i = 0; i < IT; ++i) v[i] = ring[q][i];
+            if (cq + D * SW < w1) load_raw16(row, w1, s0 + D * SW, vec, ring[q]);
             uint32_t flags = 0;
+            if (cq + SW <= w1) {                           // warp-uniform: a full step
 #pragma unroll
-            for (int i = 0; i < TK_ITEMS; ++i)
-                if (s0 + i < w1 && v[i] >= tau_f) flags |= 1u << i;
+                for (int i = 0; i < IT; ++i) flags |= (uint32_t)(v[i] >= tau_f) << i;
+            } else {
+#pragma unroll
+                for (int i = 0; i < IT; ++i) flags |= (uint32_t)(s0 + i < w1 && v[i] >= tau_f) << i;
+            }
             const uint32_t c = (uint32_t)__popc(flags);
             uint32_t x = c;
 #pragma unroll
@@ -404,7 +453,7 @@ __device__ uint32_t collect_above_warp(TopkSmem &sm, const float *row, int64_t n
             while (flags) {
                 const int i = __ffs(flags) - 1;
                 flags &= flags - 1;
-                if (off < TK_WCAP) { wk[off] = float_key(v[i]); wp[off] = (int32_t)(s0 + i); }
+                if (off < C::WCAP) { wk[off] = __float_as_uint(v[i]); wp[off] = s0 + i; }
                 ++off;
             }
             cnt += __shfl_sync(0xffffffffu, x, 31);
@@ -413,42 +462,42 @@ __device__ uint32_t collect_above_warp(TopkSmem &sm, const float *row, int64_t n
     if (lane == 0) sm.wcnt[warp] = cnt;
     __syncthreads();
     if (warp == 0) {                                       // exclusive prefix of the warps' counts
-        const uint32_t c = lane < TK_WARPS ? sm.wcnt[lane] : 0u;
+        const uint32_t c = lane < C::WARPS ? sm.wcnt[lane] : 0u;
         uint32_t x = c;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
             const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
             if (lane >= o) x += y;
         }
-        const bool over = __any_sync(0xffffffffu, c > TK_WCAP);
-        if (lane <= TK_WARPS) sm.wbefore[lane] = over ? 0xffffffffu : x - c;
+        const bool over = __any_sync(0xffffffffu, c > C::WCAP);
+        if (lane <= C::WARPS) sm.wbefore[lane] = over ? 0xffffffffu : x - c;
     }
     __syncthreads();
-    const uint32_t total = sm.wbefore[TK_WARPS];
+    const uint32_t total = sm.wbefore[C::WARPS];
     if (total == 0xffffffffu) return total;                // a warp overflowed (block-uniform)
-    // Pack in rounds of TK_THREADS * 4 entries in increasing order: an entry only
-    // moves down, so a round's targets never hold a later round's sources; each
-    // round reads all its sources before it writes.
-    for (uint32_t r0 = 0; r0 < total; r0 += TK_THREADS * 4) {
+    // Pack in rounds of NT * 4 entries in increasing order: an entry only moves
+    // down, so a round's targets never hold a later round's sources; each round
+    // reads all its sources before it writes.  Raw score bits become keys here.
+    for (uint32_t r0 = 0; r0 < total; r0 += C::NT * 4) {
         uint32_t kk[4];
         int32_t pp[4];
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
-            const uint32_t i = r0 + tid + q * TK_THREADS;
+            const uint32_t i = r0 + tid + q * C::NT;
             if (i < total) {
                 int w = 0;                                 // last warp with wbefore[w] <= i
 #pragma unroll
-                for (int step = TK_WARPS / 2; step > 0; step >>= 1)
+                for (int step = C::WARPS / 2; step > 0; step >>= 1)
                     if (sm.wbefore[w + step] <= i) w += step;
-                const uint32_t src = w * TK_WCAP + (i - sm.wbefore[w]);
-                kk[q] = sm.ckey[src];
+                const uint32_t src = w * C::WCAP + (i - sm.wbefore[w]);
+                kk[q] = float_key(__uint_as_float(sm.ckey[src]));
                 pp[q] = sm.cpos[src];
             }
         }
         __syncthreads();
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
-            const uint32_t i = r0 + tid + q * TK_THREADS;
+            const uint32_t i = r0 + tid + q * C::NT;
             if (i < total) { sm.ckey[i] = kk[q]; sm.cpos[i] = pp[q]; }
         }
         __syncthreads();
@@ -457,7 +506,8 @@ __device__ uint32_t collect_above_warp(TopkSmem &sm, const float *row, int64_t n
 }
 
 // Radix select run over the whole row in global memory (candidates did not fit).
-__device__ __noinline__ void select_global(TopkSmem &sm, const float *row, int64_t n, bool vec, int k, int32_t *out)
+template <class C>
+__device__ __noinline__ void select_global(TopkSmem<C> &sm, const float *row, int64_t n, bool vec, int k, int32_t *out)
 {
     const int tid = threadIdx.x;
     auto row_keys = [&](int64_t s, uint32_t (&keys)[TK_ITEMS], uint32_t &valid) {
@@ -469,9 +519,9 @@ __device__ __noinline__ void select_global(TopkSmem &sm, const float *row, int64
         const int shift = pass == 0 ? 21 : (pass == 1 ? 10 : 0);
         const int nb = pass == 2 ? 1024 : 2048;
         const uint32_t bmask = (uint32_t)nb - 1u;
-        for (int i = tid; i < nb; i += TK_THREADS) sm.hist[i] = 0u;
+        for (int i = tid; i < nb; i += C::NT) sm.hist[i] = 0u;
         __syncthreads();
-        for (int64_t c0 = 0; c0 < n; c0 += TK_STEP) {
+        for (int64_t c0 = 0; c0 < n; c0 += C::STEP) {
             uint32_t keys[TK_ITEMS], valid;
             row_keys(c0 + (int64_t)tid * TK_ITEMS, keys, valid);
 #pragma unroll
@@ -506,38 +556,57 @@ __device__ __forceinline__ void hist_top11(uint32_t *hist, const uint32_t (&keys
 }
 
 // Threshold guess for a long row: the key of rank ~1.5 k (scaled to the
-// sample, at least 8) among 2048 evenly spaced samples, resolved by one radix pass (a
-// threshold at or below it).  Every thread calls it; every CTA working on the
-// same row computes the same value.
-__device__ uint32_t sampled_threshold(TopkSmem &sm, const float *row, int64_t n, int k)
+// sample, at least 8) among NSAMP samples spread evenly over the row, resolved
+// by one radix pass (a threshold at or below it).  Every thread calls it;
+// every CTA working on the same row computes the same value.  With RUNS the
+// samples are runs of 8 consecutive positions starting at multiples of 8
+// (n > CAP >= NSAMP, so the runs do not overlap and stay inside the row).
+template <class C>
+__device__ uint32_t sampled_threshold(TopkSmem<C> &sm, const float *row, int64_t n, int k, bool vec)
 {
     const int tid = threadIdx.x;
-    float sv[TK_SAMPLE / TK_THREADS];                     // all loads issued before any is used
+    uint32_t *smp = sm.sample();
+    if constexpr (C::RUNS) {
+        constexpr int NRUN = C::NSAMP / 8, RPT = NRUN / C::NT;
+        float sv[RPT][TK_ITEMS];                          // all loads issued before any is used
 #pragma unroll
-    for (int q = 0; q < TK_SAMPLE / TK_THREADS; ++q)
-        sv[q] = __ldg(row + (int64_t)(tid + q * TK_THREADS) * n / TK_SAMPLE);
+        for (int q = 0; q < RPT; ++q) {
+            const int64_t j = tid + q * C::NT;
+            load_raw8(row, n, (j * n / NRUN) & ~(int64_t)7, vec, sv[q]);
+        }
 #pragma unroll
-    for (int q = 0; q < TK_SAMPLE / TK_THREADS; ++q) sm.sample[tid + q * TK_THREADS] = float_key(sv[q]);
+        for (int q = 0; q < RPT; ++q)
+#pragma unroll
+            for (int i = 0; i < TK_ITEMS; ++i) smp[(tid + q * C::NT) * TK_ITEMS + i] = float_key(sv[q][i]);
+    } else {
+        float sv[C::NSAMP / C::NT];
+#pragma unroll
+        for (int q = 0; q < C::NSAMP / C::NT; ++q)
+            sv[q] = __ldg(row + (int64_t)(tid + q * C::NT) * n / C::NSAMP);
+#pragma unroll
+        for (int q = 0; q < C::NSAMP / C::NT; ++q) smp[tid + q * C::NT] = float_key(sv[q]);
+    }
     __syncthreads();
     // at least 8 samples above the threshold: a rank of 1 or 2 (long rows, small k)
     // estimates the count so loosely that it often lands below k
-    const double want = 1.5 * (double)k * TK_SAMPLE / (double)n;
-    const uint32_t rank = (uint32_t)min((double)TK_SAMPLE, max(8.0, ceil(want)));
+    const double want = 1.5 * (double)k * C::NSAMP / (double)n;
+    const uint32_t rank = (uint32_t)min((double)C::NSAMP, max(8.0, ceil(want)));
     uint32_t tau, unused;
-    radix_select_smem(sm, sm.sample, TK_SAMPLE, rank, &tau, &unused, 1);
+    radix_select_smem(sm, smp, C::NSAMP, rank, &tau, &unused, 1);
     return tau;
 }
 
 // Exact top-k of a row without a threshold guess: a histogram of the top 11
 // key bits fixes the bin of the k-th largest key; the keys in or above it go
 // on chip (or, if too many, a radix select runs over the row in global memory).
-__device__ __noinline__ void topk_row_histogram(TopkSmem &sm, const float *row, int64_t n, bool vec, int k,
+template <class C>
+__device__ __noinline__ void topk_row_histogram(TopkSmem<C> &sm, const float *row, int64_t n, bool vec, int k,
                                                 int32_t *out)
 {
     const int tid = threadIdx.x;
-    for (int i = tid; i < 2048; i += TK_THREADS) sm.hist[i] = 0u;
+    for (int i = tid; i < 2048; i += C::NT) sm.hist[i] = 0u;
     __syncthreads();
-    for (int64_t c0 = 0; c0 < n; c0 += TK_STEP) {
+    for (int64_t c0 = 0; c0 < n; c0 += C::STEP) {
         uint32_t keys[TK_ITEMS], valid;
         load8(row, n, c0 + (int64_t)tid * TK_ITEMS, vec, keys, valid);
         hist_top11(sm.hist, keys, valid);
@@ -547,7 +616,7 @@ __device__ __noinline__ void topk_row_histogram(TopkSmem &sm, const float *row, 
     const uint32_t b1 = sm.sh_bin;
     const uint32_t remaining = (uint32_t)k - sm.sh_above;
     const uint32_t ncand = collect_candidates(sm, row, n, vec, [b1](uint32_t key) { return (key >> 21) >= b1; });
-    if (ncand <= TK_CAP) select_on_chip(sm, ncand, b1, remaining, k, out);
+    if (ncand <= C::CAP) select_on_chip(sm, ncand, b1, remaining, k, out);
     else select_global(sm, row, n, vec, k, out);
 }
 
@@ -555,25 +624,28 @@ __device__ __noinline__ void topk_row_histogram(TopkSmem &sm, const float *row, 
 // (n = n_all - W, or 0), [n, n_all) are always taken.  When n <= k the whole
 // row is selected, so out[i] = i for i < n_all, then -1 up to k + W.
 // Otherwise the top-k part fills out[0, k) and the window out[k, k + W).
+template <class C>
 __device__ __forceinline__ void emit_window(int32_t *out, int k, int window, int64_t n)
 {
-    for (int i = threadIdx.x; i < window; i += TK_THREADS) out[k + i] = (int32_t)(n + i);
+    for (int i = threadIdx.x; i < window; i += C::NT) out[k + i] = (int32_t)(n + i);
 }
 
+template <class C>
 __device__ __forceinline__ bool emit_whole_row(int32_t *out, int k, int window, int64_t n, int64_t n_all)
 {
     if (n > k) return false;
-    for (int i = threadIdx.x; i < k + window; i += TK_THREADS) out[i] = i < n_all ? i : -1;
+    for (int i = threadIdx.x; i < k + window; i += C::NT) out[i] = i < n_all ? i : -1;
     return true;
 }
 
-__global__ void __launch_bounds__(TK_THREADS, 2)
+__global__ void __launch_bounds__(RowsCfg::NT, 2)
 topk_rows_kernel(const float *__restrict__ scores, int64_t ld, int64_t row_begin,
                  const int32_t *__restrict__ lens, int64_t max_len, int k, int window,
                  int32_t *__restrict__ idx, WsHeader *hdr, int vec_ok)
 {
+    using C = RowsCfg;
     extern __shared__ __align__(16) uint8_t smem_raw[];
-    TopkSmem &sm = *reinterpret_cast<TopkSmem *>(smem_raw);
+    TopkSmem<C> &sm = *reinterpret_cast<TopkSmem<C> *>(smem_raw);
 
     const int64_t r = blockIdx.x;
     const int tid = threadIdx.x;
@@ -584,20 +656,20 @@ topk_rows_kernel(const float *__restrict__ scores, int64_t ld, int64_t row_begin
         n_all = lens[r];
         if (n_all < 1 || n_all > max_len) {
             if (tid == 0) record_error(hdr, DSA_ERR_INVALID_ARG, (unsigned)r);
-            for (int i = tid; i < k + window; i += TK_THREADS) out[i] = -1;
+            for (int i = tid; i < k + window; i += C::NT) out[i] = -1;
             return;
         }
     } else {
         n_all = row_begin + r + 1;
     }
     const int64_t n = n_all > window ? n_all - window : 0;     // positions before the window
-    if (emit_whole_row(out, k, window, n, n_all)) return;
-    emit_window(out, k, window, n);
+    if (emit_whole_row<C>(out, k, window, n, n_all)) return;
+    emit_window<C>(out, k, window, n);
     const bool vec = vec_ok != 0;
     if (tid == 0) { sm.sh_count = 0; sm.sh_overflow = 0; }
 
     // ---- short rows: every key is a candidate ----
-    if (n <= TK_CAP) {
+    if (n <= C::CAP) {
         const uint32_t c = collect_candidates(sm, row, n, vec, [](uint32_t) { return true; });
         select_candidates(sm, c, k, out);
         return;
@@ -606,9 +678,9 @@ topk_rows_kernel(const float *__restrict__ scores, int64_t ld, int64_t row_begin
     // ---- guess a threshold from evenly spaced samples: about 1.5 k keys of the
     // row should lie at or above it; then one ordered pass collects them ----
     {
-        const uint32_t tau = sampled_threshold(sm, row, n, k);
+        const uint32_t tau = sampled_threshold(sm, row, n, k, vec);
         const uint32_t c = collect_above_warp(sm, row, n, vec, key_float(tau));
-        if (c >= (uint32_t)k && c <= TK_CAP) {        // the selection lies among the candidates
+        if (c >= (uint32_t)k && c <= C::CAP) {        // the selection lies among the candidates
             select_candidates(sm, c, k, out);
             return;
         }
@@ -649,39 +721,41 @@ __device__ __forceinline__ int64_t before_window(int64_t n_all, int window)
     return n_all > window ? n_all - window : 0;
 }
 
-__global__ void __launch_bounds__(TK_THREADS, 2)
+__global__ void __launch_bounds__(SplitCfg::NT, 2)
 topk_split_collect_kernel(const float *__restrict__ scores, int64_t ld, const int32_t *__restrict__ lens,
                           int64_t max_len, int k, int window, SplitWs ws, int vec_ok)
 {
+    using C = SplitCfg;
     extern __shared__ __align__(16) uint8_t smem_raw[];
-    TopkSmem &sm = *reinterpret_cast<TopkSmem *>(smem_raw);
+    TopkSmem<C> &sm = *reinterpret_cast<TopkSmem<C> *>(smem_raw);
     grid_dep_wait();                                 // the scores of the kernel before
     grid_dep_trigger();
     const int64_t r = blockIdx.y;
     const int64_t n_all = split_len(lens, max_len, r);
     const int64_t n = n_all < 0 ? -1 : before_window(n_all, window);
     const int64_t c0 = (int64_t)blockIdx.x * TS_CHUNK;
-    if (n <= TK_CAP || c0 >= n) return;              // short or invalid rows: the final kernel alone
+    if (n <= C::CAP || c0 >= n) return;              // short or invalid rows: the final kernel alone
     const int64_t c1 = min(n, c0 + TS_CHUNK);
     const float *row = scores + r * ld;
-    const uint32_t tau = sampled_threshold(sm, row, n, k);
+    const uint32_t tau = sampled_threshold(sm, row, n, k, vec_ok != 0);
     const uint32_t c = collect_above_warp(sm, row + c0, c1 - c0, vec_ok != 0, key_float(tau));
     const int64_t slot = (r * ws.chunks + blockIdx.x) * (int64_t)TS_SLOT;
     if (c != 0xffffffffu)
-        for (uint32_t i = threadIdx.x; i < min(c, (uint32_t)TS_SLOT); i += TK_THREADS) {
+        for (uint32_t i = threadIdx.x; i < min(c, (uint32_t)TS_SLOT); i += C::NT) {
             ws.ckey[slot + i] = sm.ckey[i];
             ws.cpos[slot + i] = (int32_t)(sm.cpos[i] + c0);
         }
     if (threadIdx.x == 0) ws.cnt[r * ws.chunks + blockIdx.x] = c;
 }
 
-__global__ void __launch_bounds__(TK_THREADS)
+__global__ void __launch_bounds__(SplitCfg::NT)
 topk_split_final_kernel(const float *__restrict__ scores, int64_t ld, const int32_t *__restrict__ lens,
                         int64_t max_len, int k, int window, SplitWs ws, int32_t *__restrict__ idx,
                         WsHeader *hdr, int vec_ok)
 {
+    using C = SplitCfg;
     extern __shared__ __align__(16) uint8_t smem_raw[];
-    TopkSmem &sm = *reinterpret_cast<TopkSmem *>(smem_raw);
+    TopkSmem<C> &sm = *reinterpret_cast<TopkSmem<C> *>(smem_raw);
     grid_dep_wait();                                 // the collect kernel's slots
     grid_dep_trigger();
     const int64_t r = blockIdx.x;
@@ -690,24 +764,24 @@ topk_split_final_kernel(const float *__restrict__ scores, int64_t ld, const int3
     const int64_t n_all = split_len(lens, max_len, r);
     if (n_all < 0) {
         if (tid == 0) record_error(hdr, DSA_ERR_INVALID_ARG, (unsigned)r);
-        for (int i = tid; i < k + window; i += TK_THREADS) out[i] = -1;
+        for (int i = tid; i < k + window; i += C::NT) out[i] = -1;
         return;
     }
     const int64_t n = before_window(n_all, window);
-    if (emit_whole_row(out, k, window, n, n_all)) return;
-    emit_window(out, k, window, n);
+    if (emit_whole_row<C>(out, k, window, n, n_all)) return;
+    emit_window<C>(out, k, window, n);
     const float *row = scores + r * ld;
     const bool vec = vec_ok != 0;
-    if (n <= TK_CAP) {                               // short rows: every key is a candidate
+    if (n <= C::CAP) {                               // short rows: every key is a candidate
         const uint32_t c = collect_candidates(sm, row, n, vec, [](uint32_t) { return true; });
         select_candidates(sm, c, k, out);
         return;
     }
     const int nch = (int)((n + TS_CHUNK - 1) / TS_CHUNK);
-    bool use = nch <= TK_SAMPLE;                     // counts and offsets fit the scratch arrays
+    bool use = nch <= C::NSAMP;                     // counts and offsets fit the scratch arrays
     if (use) {
         // chunk counts (sm.sample) and their exclusive prefix (sm.hist), in parallel
-        const int cpt = (nch + TK_THREADS - 1) / TK_THREADS;
+        const int cpt = (nch + C::NT - 1) / C::NT;
         uint32_t msum = 0;
         bool fit = true;
         for (int u = 0; u < cpt; ++u) {
@@ -715,29 +789,29 @@ topk_split_final_kernel(const float *__restrict__ scores, int64_t ld, const int3
             if (c < nch) {
                 const uint32_t m = ws.cnt[r * ws.chunks + c];
                 fit = fit && m <= TS_SLOT;
-                sm.sample[c] = m <= TS_SLOT ? m : 0u;
+                sm.sample()[c] = m <= TS_SLOT ? m : 0u;
                 msum += m <= TS_SLOT ? m : 0u;
             }
         }
         use = __syncthreads_and(fit) != 0;
         uint32_t total;
-        uint32_t run = block_excl_scan(msum, sm.warp_buf, &total);
+        uint32_t run = block_excl_scan<C>(msum, sm.warp_buf, &total);
         for (int u = 0; u < cpt; ++u) {
             const int c = tid * cpt + u;
-            if (c < nch) { sm.hist[c] = run; run += sm.sample[c]; }
+            if (c < nch) { sm.hist[c] = run; run += sm.sample()[c]; }
         }
         __syncthreads();
-        use = use && total >= (uint32_t)k && total <= TK_CAP;
+        use = use && total >= (uint32_t)k && total <= C::CAP;
         if (use) {
             // Every thread copies joined entries tid, tid + 512, ... with four
             // entries' loads in flight: entry i comes from the last chunk c whose
             // offset hist[c] <= i (that chunk is never empty), at i - hist[c].
-            for (uint32_t base = 0; base < total; base += TK_THREADS * 4) {
+            for (uint32_t base = 0; base < total; base += C::NT * 4) {
                 uint32_t kk[4];
                 int32_t pp[4];
 #pragma unroll
                 for (int q = 0; q < 4; ++q) {
-                    const uint32_t i = base + (uint32_t)(q * TK_THREADS + tid);
+                    const uint32_t i = base + (uint32_t)(q * C::NT + tid);
                     if (i < total) {
                         int lo = 0, hi = nch - 1;
                         while (lo < hi) {
@@ -751,7 +825,7 @@ topk_split_final_kernel(const float *__restrict__ scores, int64_t ld, const int3
                 }
 #pragma unroll
                 for (int q = 0; q < 4; ++q) {
-                    const uint32_t i = base + (uint32_t)(q * TK_THREADS + tid);
+                    const uint32_t i = base + (uint32_t)(q * C::NT + tid);
                     if (i < total) { sm.ckey[i] = kk[q]; sm.cpos[i] = pp[q]; }
                 }
             }
@@ -771,12 +845,12 @@ cudaError_t launch_topk_rows(const float *scores, int64_t ld, int64_t row_begin,
                              int32_t *idx, WsHeader *hdr, cudaStream_t st, int window)
 {
     if (row_count <= 0) return cudaSuccess;
-    const size_t smem = sizeof(TopkSmem);
+    const size_t smem = sizeof(TopkSmem<RowsCfg>);
     cudaError_t e = cudaFuncSetAttribute(topk_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)smem);
     if (e != cudaSuccess) return e;
     const int vec_ok = (ld % 4 == 0) && ((reinterpret_cast<uintptr_t>(scores) & 15u) == 0);
-    topk_rows_kernel<<<(unsigned)row_count, TK_THREADS, smem, st>>>(scores, ld, row_begin, lens,
+    topk_rows_kernel<<<(unsigned)row_count, RowsCfg::NT, smem, st>>>(scores, ld, row_begin, lens,
                                                                      max_len, k, window, idx, hdr, vec_ok);
     return cudaGetLastError();
 }
@@ -803,16 +877,16 @@ cudaError_t launch_topk_split(const float *scores, int64_t ld, const int32_t *le
     p += align_up(sizeof(uint32_t) * (size_t)rows * chunks * TS_SLOT, 256);
     ws.cpos = reinterpret_cast<int32_t *>(p);
     const int vec_ok = (ld % 4 == 0) && ((reinterpret_cast<uintptr_t>(scores) & 15u) == 0);
-    const size_t smem = sizeof(TopkSmem);
+    const size_t smem = sizeof(TopkSmem<SplitCfg>);
     cudaError_t e = cudaFuncSetAttribute(topk_split_collect_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     e = cudaFuncSetAttribute(topk_split_final_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     dim3 grid((unsigned)chunks, (unsigned)rows);
-    e = launch_chained(topk_split_collect_kernel, grid, dim3(TK_THREADS), smem, st, scores, ld, lens,
+    e = launch_chained(topk_split_collect_kernel, grid, dim3(SplitCfg::NT), smem, st, scores, ld, lens,
                        max_len, k, window, ws, vec_ok);
     if (e != cudaSuccess) return e;
-    e = launch_chained(topk_split_final_kernel, dim3((unsigned)rows), dim3(TK_THREADS), smem, st, scores,
+    e = launch_chained(topk_split_final_kernel, dim3((unsigned)rows), dim3(SplitCfg::NT), smem, st, scores,
                        ld, lens, max_len, k, window, ws, idx, hdr, vec_ok);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();

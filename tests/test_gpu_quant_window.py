@@ -47,6 +47,36 @@ def test_quantize_bit_exact(rows, cols, dtype):
     assert bad.size == 0, f"{len(bad)} codes differ, first at {bad[:3].tolist()}"
 
 
+def test_quantize_values_beside_every_rounding_midpoint():
+    """Rows whose quotients x / scale land on, and a few ulps beside, every
+    midpoint between neighbouring E4M3 values (where the rounding of the fp32
+    quotient decides the code), with scales whose reciprocals are inexact."""
+    codes_pos = np.array([oracle.e4m3(c) for c in range(0x7F)])
+    mids = (codes_pos[1:] + codes_pos[:-1]) / 2
+    rows = []
+    for amax in (3.0, 7.0, 0.1, 1e-20, 5e4):
+        s = np.float32(amax) / np.float32(448.0)
+        base = (mids * np.float64(s)).astype(np.float32)
+        vals = [np.float32(amax)]
+        for k in range(-6, 7):
+            v = base.copy()
+            for _ in range(abs(k)):
+                v = np.nextafter(v, np.float32(np.inf if k > 0 else 0)).astype(np.float32)
+            vals.append(v)
+            vals.append(-v)
+        row = np.concatenate([np.atleast_1d(np.asarray(a, np.float32)) for a in vals])
+        row = row[np.abs(row) <= np.float32(amax)]
+        rows.append(row[: (row.size // 8) * 8])
+    width = max(r.size for r in rows)
+    x = np.zeros((len(rows), width), np.float32)
+    for i, r in enumerate(rows):
+        x[i, : r.size] = r
+    codes, scale = dsa.dsa_quantize_e4m3(torch.from_numpy(x).cuda())
+    ref_codes, ref_scale = oracle.quantize_e4m3(x)
+    np.testing.assert_array_equal(scale.cpu().numpy(), ref_scale)
+    np.testing.assert_array_equal(codes.cpu().numpy(), ref_codes)
+
+
 def test_quantize_matches_the_input_generator():
     """The generator packs its sources with torch (amax / 448, float8 cast);
     the kernel reproduces those bytes from the same sources."""
