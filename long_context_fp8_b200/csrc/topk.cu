@@ -235,10 +235,12 @@ __device__ __noinline__ void select_on_chip(TopkSmem<C> &sm, uint32_t ncand, uin
 // by an OR-reduction of key ^ keys[0]), so that the first histogram spreads
 // over the keys' actual range instead of piling onto one bin of the top bits.
 // With passes = 3 the result is exact; with fewer, the bits not yet resolved
-// are zero in *thr (a threshold at or below the exact key).
+// are zero in *thr (a threshold at or below the exact key).  refine = false
+// skips the direct search among a small last bin (for a threshold guess, the
+// bin's lower bound serves as well and saves its barriers).
 template <class C>
 __device__ void radix_select_smem(TopkSmem<C> &sm, const uint32_t *keys, uint32_t n, uint32_t rank,
-                                  uint32_t *thr, uint32_t *need, int passes = 3)
+                                  uint32_t *thr, uint32_t *need, int passes = 3, bool refine = true)
 {
     const int tid = threadIdx.x;
     const uint32_t first = keys[0];
@@ -279,7 +281,7 @@ __device__ void radix_select_smem(TopkSmem<C> &sm, const uint32_t *keys, uint32_
         pmask |= bmask << shift;
         lo = shift;
         __syncthreads();
-        if (lo > 0 && in_bin <= 64) {
+        if (refine && lo > 0 && in_bin <= 64) {
             // Few keys share the bin of the rank-th key: gather them (their order does
             // not matter) and find it among them directly, instead of more passes:
             // it is the x with  #{y > x} < remaining <= #{y >= x}.
@@ -592,7 +594,7 @@ __device__ uint32_t sampled_threshold(TopkSmem<C> &sm, const float *row, int64_t
     const double want = 1.5 * (double)k * C::NSAMP / (double)n;
     const uint32_t rank = (uint32_t)min((double)C::NSAMP, max(8.0, ceil(want)));
     uint32_t tau, unused;
-    radix_select_smem(sm, smp, C::NSAMP, rank, &tau, &unused, 1);
+    radix_select_smem(sm, smp, C::NSAMP, rank, &tau, &unused, 1, false);
     return tau;
 }
 
