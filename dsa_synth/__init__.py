@@ -280,3 +280,18 @@ def prefill_flops(spec: PrefillSpec) -> Dict[str, float]:
     return dict(pairs=pairs, selected=sel,
                 indexer_flop=2.0 * spec.H_I * spec.d_I * pairs,
                 attn_flop=4.0 * spec.H_q * spec.d * sel)
+
+
+def decode_kv_to_fp8(inp: Dict[str, torch.Tensor]) -> Dict[str, torch.Tensor]:
+    """Copy of a decode input whose K/V caches are stored as FP8 E4M3 codes with
+    one fp32 scale per cached token (storage packing only: the bf16 cache rows
+    are packed by quantize_e4m3_per_token).  k_cache/v_cache become uint8
+    [P, ps, d]; k_cache_scale/v_cache_scale are added as f32 [P, ps]."""
+    out = dict(inp)
+    for name in ("k", "v"):
+        c = inp[name + "_cache"]
+        P, ps, d = c.shape
+        codes, scale = quantize_e4m3_per_token(c.reshape(P * ps, d).float())
+        out[name + "_cache"] = codes.reshape(P, ps, d).contiguous()
+        out[name + "_cache_scale"] = scale.reshape(P, ps).contiguous()
+    return out

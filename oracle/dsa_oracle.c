@@ -30,6 +30,11 @@
  *     of a query are always attended, and stage 2 selects min(k, t+1-W) of
  *     the older positions 0..t-W by indexer score.  Output: the top-k part in
  *     ascending position, then the window positions, then -1 up to k + W.
+ *  7. FP8 K/V for the main attention (the hotdry page's FP8 decoding
+ *     section: the KV cache moves from 16-bit to FP8): the decode caches hold
+ *     E4M3 codes with one fp32 scale per cached token for K and for V, and the
+ *     attention of stage 3 uses Khat[j] = e4m3(k8[j]) * ks[j],
+ *     Vhat[j] = e4m3(v8[j]) * vs[j].
  *  6. FP8 quantisation of the indexer's query and key ("DeepSeek-V3.2-Exp
  *     DSA 技术深度解析", section 1: FP8 indexer; the hotdry page's section on
  *     FP8 decoding) and the append of a new token to the paged caches: one
@@ -278,16 +283,17 @@ int dsa_or_topk_window(const double *scores, int64_t ld, const int64_t *rows, in
  * in sel[0..k) (-1 = unused).  krow(j)/vrow(j) give the key / value element
  * offsets of cache row j.  Writes o[H*D] and lse[H] (lse = -inf, o = 0 when
  * nothing is selected). */
-static void attend_one(const void *q, int64_t q_off, const void *K, const void *V, int dtype,
-                       const int64_t *koff, int64_t nsel, int H, int D, double sm,
-                       double *o, double *lse, double *z)
+static void attend_one_kv(const void *q, int64_t q_off, int qdt, const void *K, const void *V, int kvdt,
+                          const float *ks, const float *vs, const int64_t *koff, int64_t nsel, int H,
+                          int D, double sm, double *o, double *lse, double *z)
 {
     for (int h = 0; h < H; ++h) {
         double zmax = -INFINITY;
         for (int64_t j = 0; j < nsel; ++j) {
+            double kscale = ks ? (double)ks[koff[j] / D] : 1.0;
             double dot = 0.0;
             for (int c = 0; c < D; ++c)
-                dot += load_elem(q, dtype, q_off + (int64_t)h * D + c) * load_elem(K, dtype, koff[j] + c);
+                dot += load_elem(q, qdt, q_off + (int64_t)h * D + c) * (load_elem(K, kvdt, koff[j] + c) * kscale);
             z[j] = sm * dot;
             if (z[j] > zmax) zmax = z[j];
         }
@@ -295,11 +301,22 @@ static void attend_one(const void *q, int64_t q_off, const void *K, const void *
         for (int64_t j = 0; j < nsel; ++j) { z[j] = exp(z[j] - zmax); l += z[j]; }
         for (int c = 0; c < D; ++c) {
             double acc = 0.0;
-            for (int64_t j = 0; j < nsel; ++j) acc += z[j] * load_elem(V, dtype, koff[j] + c);
+            for (int64_t j = 0; j < nsel; ++j) {
+                double vscale = vs ? (double)vs[koff[j] / D] : 1.0;
+                acc += z[j] * (load_elem(V, kvdt, koff[j] + c) * vscale);
+            }
             o[(int64_t)h * D + c] = nsel > 0 ? acc / l : 0.0;
         }
         lse[h] = nsel > 0 ? zmax + log(l) : -INFINITY;
     }
+}
+
+/* Stage 3 with Q, K and V of one dtype and no scales. */
+static void attend_one(const void *q, int64_t q_off, const void *K, const void *V, int dtype,
+                       const int64_t *koff, int64_t nsel, int H, int D, double sm,
+                       double *o, double *lse, double *z)
+{
+    attend_one_kv(q, q_off, dtype, K, V, dtype, NULL, NULL, koff, nsel, H, D, sm, o, lse, z);
 }
 
 /*
@@ -345,7 +362,8 @@ int dsa_or_sparse_attn(const void *q, const void *K, const void *V, int dtype, c
  * (the current token included) at positions 0..n-1; position s lives in
  * physical page bt[b*max_pages + s/ps], slot s%ps.
  *   q_idx  e4m3 [B,H_I,D_I], q_scale [B], w bf16 [B,H_I], q bf16 [B,H_q,D]
- *   kidx   e4m3 [P,ps,D_I], kscale f32 [P,ps], kc/vc bf16 [P,ps,D]
+ *   kidx   e4m3 [P,ps,D_I], kscale f32 [P,ps], kc/vc bf16 [P,ps,D], or (stage
+ *   7, when kcs and vcs are given) e4m3 [P,ps,D] with scales kcs/vcs f32 [P,ps]
  * window > 0 applies stage 5: the last `window` positions are always
  * attended and the top-k runs over the positions before them.
  * Outputs: scores_out [B, ld] (nullable; entries s < n), idx_out
@@ -354,10 +372,10 @@ int dsa_or_sparse_attn(const void *q, const void *K, const void *V, int dtype, c
  */
 int dsa_or_decode(const uint8_t *q_idx, const float *q_scale, const uint16_t *w,
                   const uint16_t *q, const uint8_t *kidx, const float *kscale,
-                  const uint16_t *kc, const uint16_t *vc, const int32_t *bt,
-                  const int32_t *ctx, int B, int max_pages, int ps, int H_I, int D_I,
-                  int H_q, int D, int k, int window, double sm, double *scores_out, int64_t ld,
-                  int32_t *idx_out, double *out, double *lse)
+                  const void *kc, const void *vc, const float *kcs, const float *vcs,
+                  const int32_t *bt, const int32_t *ctx, int B, int max_pages, int ps, int H_I,
+                  int D_I, int H_q, int D, int k, int window, double sm, double *scores_out,
+                  int64_t ld, int32_t *idx_out, double *out, double *lse)
 {
     int err = 0;
     for (int b = 0; b < B && !err; ++b) {
@@ -398,8 +416,8 @@ int dsa_or_decode(const uint8_t *q_idx, const float *q_scale, const uint16_t *w,
                 koff[m++] = (page * ps + sel[i] % ps) * D;
             }
             double l[1024];
-            attend_one(q, (int64_t)b * H_q * D, kc, vc, OR_BF16, koff, m, H_q, D, sm,
-                       out + (int64_t)b * H_q * D, l, z);
+            attend_one_kv(q, (int64_t)b * H_q * D, OR_BF16, kc, vc, kcs ? OR_E4M3 : OR_BF16, kcs, vcs,
+                          koff, m, H_q, D, sm, out + (int64_t)b * H_q * D, l, z);
             if (lse) for (int h = 0; h < H_q; ++h) lse[(int64_t)b * H_q + h] = l[h];
         }
         free(sc); free(q_row); free(w_row); free(buf); free(koff); free(z);

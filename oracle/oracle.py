@@ -54,7 +54,7 @@ def load(path: Optional[str] = None):
     lib.dsa_or_topk.restype = I32
     lib.dsa_or_sparse_attn.argtypes = [P, P, P, I32, P, I64, I32, I32, I32, D, P, P]
     lib.dsa_or_sparse_attn.restype = I32
-    lib.dsa_or_decode.argtypes = [P, P, P, P, P, P, P, P, P, P, I32, I32, I32, I32, I32,
+    lib.dsa_or_decode.argtypes = [P, P, P, P, P, P, P, P, P, P, P, P, I32, I32, I32, I32, I32,
                                   I32, I32, I32, I32, D, P, I64, P, P, P]
     lib.dsa_or_decode.restype = I32
     lib.dsa_or_topk_window.argtypes = [P, I64, P, I64, I32, I32, P]
@@ -256,11 +256,16 @@ def sparse_attn(q, K, V, idx, rows, sm_scale, lib=None, compact=False):
 
 def decode(inp: dict, k: int, sm_scale: float, want_scores: bool = False, lib=None, window: int = 0):
     """One decode step over paged caches (stage 4; with window > 0, stage 5's
-    selection); returns dict idx [B, k+window]/out/lse[/scores]."""
+    selection; with FP8 K/V caches -- uint8 k_cache/v_cache plus
+    k_cache_scale/v_cache_scale -- stage 7's attention); returns dict
+    idx [B, k+window]/out/lse[/scores]."""
     lib = lib or load()
     q_idx, q_scale, w, q = _np(inp["q_idx"]), _np(inp["q_scale"], np.float32), _np(inp["w"]), _np(inp["q"])
     kidx, ksc = _np(inp["kidx_cache"]), _np(inp["kscale_cache"], np.float32)
     kc, vc = _np(inp["k_cache"]), _np(inp["v_cache"])
+    kv8 = kc.dtype == np.uint8
+    kcs = _np(inp["k_cache_scale"], np.float32) if kv8 else None
+    vcs = _np(inp["v_cache_scale"], np.float32) if kv8 else None
     bt, ctx = _np(inp["block_table"], np.int32), _np(inp["context_lens"], np.int32)
     B, H_I, D_I = q_idx.shape
     H_q, D = q.shape[1], q.shape[2]
@@ -271,7 +276,7 @@ def decode(inp: dict, k: int, sm_scale: float, want_scores: bool = False, lib=No
     out = np.empty((B, H_q, D), dtype=np.float64)
     lse = np.empty((B, H_q), dtype=np.float64)
     rc = lib.dsa_or_decode(_ptr(q_idx), _ptr(q_scale), _ptr(w), _ptr(q), _ptr(kidx), _ptr(ksc),
-                           _ptr(kc), _ptr(vc), _ptr(bt), _ptr(ctx), B, bt.shape[1], ps, H_I,
+                           _ptr(kc), _ptr(vc), _ptr(kcs), _ptr(vcs), _ptr(bt), _ptr(ctx), B, bt.shape[1], ps, H_I,
                            D_I, H_q, D, k, window, float(sm_scale), _ptr(scores), ld, _ptr(idx),
                            _ptr(out), _ptr(lse))
     assert rc == 0

@@ -522,3 +522,57 @@ def test_decode_window_matches_dense_mask():
         out, lse = brute.dense_masked_attention(qq, kc, vc, m, sm)
         np.testing.assert_allclose(res["out"][b], out[n - 1], rtol=1e-10, atol=1e-12)
         np.testing.assert_allclose(res["lse"][b], lse[n - 1], rtol=1e-12, atol=1e-12)
+
+
+# ---------------------------------------------------------------- FP8 K/V (stage 7)
+
+def test_decode_fp8_kv_matches_dense_mask():
+    """Decode over E4M3 K/V caches with per-token scales: dense masked attention
+    over the dequantised rows (torch's float8 decode times the scale)."""
+    spec = dsa_synth.DecodeSpec("dk", context_lens=(130, 64, 1, 257), H_I=4, d_I=32, k=16,
+                                H_q=3, d=16, page_size=16, needle_frac=0.05,
+                                needle_min_age=4, seed=29)
+    inp = dsa_synth.decode_kv_to_fp8(dsa_synth.make_decode(spec))
+    sm = 0.25
+    res = oracle.decode(inp, spec.k, sm)
+    bt = inp["block_table"].numpy()
+    for b, n in enumerate(spec.context_lens):
+        pos = np.arange(n)
+        slot = bt[b, pos // 16].astype(np.int64) * 16 + pos % 16
+        kd = brute.decode_storage(inp["k_cache"].reshape(-1, 16)[slot]) * inp["k_cache_scale"].reshape(-1)[slot].double().numpy()[:, None]
+        vd = brute.decode_storage(inp["v_cache"].reshape(-1, 16)[slot]) * inp["v_cache_scale"].reshape(-1)[slot].double().numpy()[:, None]
+        sel = res["idx"][b][res["idx"][b] >= 0]
+        mask = np.zeros((n, n), bool); mask[n - 1, sel] = True
+        mask[: n - 1, 0] = True
+        qq = torch.zeros((n, 3, 16), dtype=torch.bfloat16); qq[n - 1] = inp["q"][b]
+        out, lse = brute.dense_masked_attention(qq, kd, vd, mask, sm)
+        np.testing.assert_allclose(res["out"][b], out[n - 1], rtol=1e-10, atol=1e-12)
+        np.testing.assert_allclose(res["lse"][b], lse[n - 1], rtol=1e-12, atol=1e-12)
+
+
+def test_decode_fp8_kv_power_of_two_scales_equal_bf16_path():
+    """With power-of-two scales every dequantised value is exact in bf16, so the
+    FP8 K/V decode equals the bf16 decode over those values (a dropped or
+    misplaced scale fails this)."""
+    spec = dsa_synth.DecodeSpec("dp", context_lens=(90, 33), H_I=4, d_I=32, k=8, H_q=2, d=16,
+                                page_size=16, needle_frac=0.0, needle_min_age=0, seed=31)
+    inp = dsa_synth.make_decode(spec)
+    rng = np.random.default_rng(3)
+    P, ps = inp["kidx_cache"].shape[:2]
+    kv8 = dict(inp)
+    bf = dict(inp)
+    for name in ("k", "v"):
+        codes = torch.from_numpy(rng.integers(0, 0x7F, (P, ps, 16)).astype(np.uint8))
+        codes[codes == 0x7F] = 0
+        codes |= torch.from_numpy((rng.integers(0, 2, (P, ps, 16)) << 7).astype(np.uint8))
+        codes[(codes & 0x7F) == 0x7F] = 0
+        scale = torch.from_numpy((2.0 ** rng.integers(-6, 6, (P, ps))).astype(np.float32))
+        kv8[name + "_cache"], kv8[name + "_cache_scale"] = codes, scale
+        vals = codes.view(torch.float8_e4m3fn).float() * scale[..., None]
+        bf[name + "_cache"] = vals.to(torch.bfloat16)
+        assert torch.equal(bf[name + "_cache"].float(), vals)        # exact in bf16
+    a = oracle.decode(kv8, spec.k, 0.3)
+    b = oracle.decode(bf, spec.k, 0.3)
+    np.testing.assert_array_equal(a["idx"], b["idx"])
+    np.testing.assert_allclose(a["out"], b["out"], rtol=1e-15, atol=1e-15)
+    np.testing.assert_allclose(a["lse"], b["lse"], rtol=1e-15, atol=1e-15)
