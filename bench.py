@@ -339,23 +339,28 @@ def prefill_e2e(dsa, inp, spec, out, lse, idx, ws, flush, args, ws_n):
 
 # ----------------------------------------------------------------------------- decode
 
-def decode_hbm_bytes(spec, window=0):
+def decode_hbm_bytes(spec, window=0, kv8=False):
     """Algorithmic HBM bytes of one decode step (what the method must move);
-    with a window, the window's K/V rows are gathered besides the top-k's."""
+    with a window, the window's K/V rows are gathered besides the top-k's;
+    with FP8 K/V each gathered row is d bytes plus a 4-byte scale, for K and V."""
     B, n = spec.B, sum(spec.context_lens)
     sel = sum(min(spec.k, max(0, c - window)) + min(window, c) for c in spec.context_lens)
-    return dict(index_keys=n * spec.d_I, key_scales=n * 4, kv_gather=sel * spec.d * 2 * 2,
+    row = (spec.d + 4) if kv8 else spec.d * 2
+    return dict(index_keys=n * spec.d_I, key_scales=n * 4, kv_gather=sel * row * 2,
                 q=B * spec.H_q * spec.d * 2, out=B * spec.H_q * spec.d * 2,
                 q_idx=B * spec.H_I * spec.d_I + B * 4 + B * spec.H_I * 2, idx=B * (spec.k + window) * 4)
 
 
-def bench_decode(args, dsa, spec, peaks, ws_n, rank, window=0, with_append=False):
-    """The decode step through dsa_decode (window 0) or dsa_decode_window;
-    with_append also times the step's quantise-and-append of the B new
-    tokens (dsa_quantize_e4m3 of the index queries, dsa_cache_append)."""
+def bench_decode(args, dsa, spec, peaks, ws_n, rank, window=0, with_append=False, kv8=False):
+    """The decode step through dsa_decode (window 0), dsa_decode_window, or
+    (kv8) dsa_decode_kv8 over FP8 K/V caches; with_append also times the
+    step's quantise-and-append of the B new tokens (dsa_quantize_e4m3 of the
+    index queries, dsa_cache_append)."""
     dev = torch.device("cuda")
     inp = dsa_synth.make_decode(replica_spec(spec, rank), device=dev)
     inp.pop("needle_pos")
+    if kv8:
+        inp = dsa_synth.decode_kv_to_fp8(inp)
     torch.cuda.synchronize()
     maxc = max(spec.context_lens)
     lib = dsa.load()
@@ -367,7 +372,11 @@ def bench_decode(args, dsa, spec, peaks, ws_n, rank, window=0, with_append=False
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
     sm = 1.0 / math.sqrt(spec.d)
 
-    if window:
+    if kv8:
+        def step():
+            dsa.dsa_decode_kv8(inp, spec.k, maxc, window=window, sm_scale=sm, out=out, lse=lse, idx_out=idx,
+                               ws=ws)
+    elif window:
         def step():
             dsa.dsa_decode_window(inp, spec.k, window, maxc, sm, out=out, lse=lse, idx_out=idx, ws=ws)
     else:
@@ -381,7 +390,7 @@ def bench_decode(args, dsa, spec, peaks, ws_n, rank, window=0, with_append=False
     ms = timed_steps(step, max(args.steps, 20), args.warmup, flush)
     step_ms = max_over_ranks(sum(ms) / len(ms), ws_n)
     status = dsa.dsa_stream_status(ws)
-    by = decode_hbm_bytes(spec, window)
+    by = decode_hbm_bytes(spec, window, kv8)
     total = sum(by.values())
     app = None
     if with_append:
@@ -523,6 +532,7 @@ def main():
     ap.add_argument("--impl", default="dsa", choices=["dsa", "reference"])
     ap.add_argument("--workload", default="p128k", choices=["p128k", "p16k", "p16k_hq128"])
     ap.add_argument("--decode-workload", default="dec64x64k", choices=["dec64x64k", "dec_ragged"])
+    ap.add_argument("--kv8", action="store_true", help="with --decode-only: the FP8 K/V decode")
     ap.add_argument("--decode-only", action="store_true",
                     help="profiling aid: time only the decode step and print its own line")
     ap.add_argument("--no-decode", action="store_true")
@@ -588,7 +598,7 @@ def main():
             torch.distributed.destroy_process_group()
         return
     if args.decode_only:
-        dec = bench_decode(args, dsa, dspec, peaks, ws_n, rank)
+        dec = bench_decode(args, dsa, dspec, peaks, ws_n, rank, kv8=args.kv8)
         us = dec["step_ms"] * 1e3
         gbs = dec["bytes"] / (dec["step_ms"] * 1e-3) / 1e9
         if rank == 0:
@@ -612,6 +622,9 @@ def main():
     decw = None
     if extras and not args.no_decode:
         decw = bench_decode(args, dsa, dspec, peaks, ws_n, rank, window=args.window)
+    deck = None
+    if extras and not args.no_decode:
+        deck = bench_decode(args, dsa, dspec, peaks, ws_n, rank, kv8=True)
     quant = bench_quantize(args, dsa, spec, peaks) if extras else None
 
     T = spec.L
@@ -673,6 +686,15 @@ def main():
                                               "frac": round(gbs / peaks["hbm_gbs"], 4),
                                               "algorithmic_bytes": decw["bytes"]},
                                  "device_status": decw["status"]}
+    if deck:
+        gbs = deck["bytes"] / (deck["step_ms"] * 1e-3) / 1e9
+        line["decode_kv8"] = {"kv_cache": "e4m3 + fp32 scale per token", "top_k": dspec.k,
+                              "value": round(whole_job_rate(ws_n, 1, deck["step_ms"]), 1), "unit": "steps/s",
+                              "us_per_step": round(deck["step_ms"] * 1e3, 2),
+                              "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": peaks["hbm_gbs"],
+                                           "unit": "GB/s", "frac": round(gbs / peaks["hbm_gbs"], 4),
+                                           "algorithmic_bytes": deck["bytes"]},
+                              "device_status": deck["status"]}
     if quant:
         line["quantize"] = quant
     if rank == 0 and ws_n == 1 and not args.no_cpu:

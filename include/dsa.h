@@ -251,6 +251,28 @@ dsa_status dsa_decode_window(const void *q_idx, const float *q_scale, const void
                              int32_t *idx_out, void *workspace, size_t ws_bytes, void *stream);
 
 /*
+ * dsa_decode_kv8 -- dsa_decode_window over FP8 K/V caches (the DeepSeek-V4
+ * engineering page's FP8 decoding section: the KV cache moves from 16-bit to
+ * FP8, halving its memory and the bytes each decode step gathers).
+ *   k_cache, v_cache uint8 E4M3 [num_pages, page_size, d] (16-byte aligned);
+ *   k_cache_scale, v_cache_scale f32 [num_pages, page_size]: the attention
+ *   uses Khat[s] = e4m3(k_cache[s]) * k_cache_scale[s] and likewise V
+ *   (dsa_cache_append_kv8 writes this layout).
+ * Every other argument, the result and the workspace are those of
+ * dsa_decode_window (window 0: no window).  Supported as dsa_decode, with
+ * H_q a multiple of 128 and d == 128 (else DSA_ERR_UNSUPPORTED).  The
+ * attention widens the gathered codes to bf16 times their scale (one
+ * rounding) before the tensor-core products.
+ */
+dsa_status dsa_decode_kv8(const void *q_idx, const float *q_scale, const void *w, const void *q,
+                          const void *kidx_cache, const float *kscale_cache, const void *k_cache,
+                          const float *k_cache_scale, const void *v_cache, const float *v_cache_scale,
+                          const int32_t *block_table, const int32_t *context_lens, int64_t num_pages,
+                          int max_pages_per_seq, int page_size, int B, int64_t max_context, int H_I,
+                          int d_I, int H_q, int d, int k_sel, int window, float sm_scale, void *out,
+                          float *lse_out, int32_t *idx_out, void *workspace, size_t ws_bytes, void *stream);
+
+/*
  * dsa_quantize_e4m3 -- FP8 E4M3 quantisation with one fp32 scale per row, the
  * storage of the indexer's query and key ("DeepSeek-V3.2-Exp DSA 技术深度解析",
  * section 1: FP8 indexer; the DeepSeek-V4 engineering page's FP8 decoding
@@ -296,6 +318,23 @@ dsa_status dsa_cache_append(const void *kidx_new, dsa_dtype kidx_dtype, const vo
                             int64_t num_pages, int page_size, int d_I, int d, void *kidx_cache,
                             float *kscale_cache, void *k_cache, void *v_cache, uint32_t *status,
                             void *stream);
+
+/*
+ * dsa_cache_append_kv8 -- dsa_cache_append for FP8 K/V caches: each new
+ * token's index key, K row and V row are each quantised as by
+ * dsa_quantize_e4m3 (one scale per row) into kidx_cache/kscale_cache,
+ * k_cache/k_cache_scale and v_cache/v_cache_scale (uint8 [num_pages,
+ * page_size, d] and f32 [num_pages, page_size]).  k_new, v_new bf16 [N, d].
+ * Supported: d_I and d multiples of 8 up to 256.  kidx_new, k_new, v_new
+ * 16-byte aligned; the code caches 8-byte aligned.  Errors and out-of-range
+ * tokens as dsa_cache_append.
+ */
+dsa_status dsa_cache_append_kv8(const void *kidx_new, dsa_dtype kidx_dtype, const void *k_new,
+                                const void *v_new, const int32_t *seq_ids, const int32_t *positions,
+                                int64_t N, int B, const int32_t *block_table, int max_pages_per_seq,
+                                int64_t num_pages, int page_size, int d_I, int d, void *kidx_cache,
+                                float *kscale_cache, void *k_cache, float *k_cache_scale, void *v_cache,
+                                float *v_cache_scale, uint32_t *status, void *stream);
 
 /*
  * dsa_decode_noalloc -- dsa_decode without a caller workspace.  The paper has

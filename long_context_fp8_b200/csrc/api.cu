@@ -442,14 +442,22 @@ namespace {
 
 // dsa_decode with a sliding window of `window` positions (0: none); the
 // selection rows (and the attention's index lists) are k_sel + window wide.
+// k_cache_scale / v_cache_scale non-null: the K/V caches hold E4M3 codes with
+// one fp32 scale per cached token (tcgen05 attention only).
 dsa_status decode_impl(const void *q_idx, const float *q_scale, const void *w, const void *q,
                        const void *kidx_cache, const float *kscale_cache, const void *k_cache,
                        const void *v_cache, const int32_t *block_table,
                        const int32_t *context_lens, int64_t num_pages, int max_pages_per_seq,
                        int page_size, int B, int64_t max_context, int H_I, int d_I, int H_q,
                        int d, int k_sel, int window, float sm_scale, void *out, float *lse_out,
-                       int32_t *idx_out, void *workspace, size_t ws_bytes, void *stream)
+                       int32_t *idx_out, void *workspace, size_t ws_bytes, void *stream,
+                       const float *k_cache_scale = nullptr, const float *v_cache_scale = nullptr)
 {
+    const bool kv8 = k_cache_scale != nullptr;
+    if (kv8 && (!v_cache_scale || (reinterpret_cast<uintptr_t>(k_cache_scale) & 3u) ||
+                (reinterpret_cast<uintptr_t>(v_cache_scale) & 3u)))
+        return DSA_ERR_INVALID_ARG;
+    if (kv8 && !sparse_attn_tc_supported(H_q, d)) return DSA_ERR_UNSUPPORTED;
     if (window < 0 || window > kMaxWindow || k_sel > 65536) return DSA_ERR_INVALID_ARG;
     const int kw = k_sel + window;                    // selection row width
     if (!q_idx || !q_scale || !w || !q || !kidx_cache || !kscale_cache || !k_cache || !v_cache ||
@@ -500,6 +508,20 @@ dsa_status decode_impl(const void *q_idx, const float *q_scale, const void *w, c
     if (e == cudaSuccess)   // each row split over 16K-position chunks (CTAs), then one CTA per row
         e = launch_topk_split(scores, max_context, context_lens, max_context, B, k_sel, idx, topk_ws,
                               hdr, st, window);
+    if (e == cudaSuccess && kv8) {
+        // tcgen05 kernel over the FP8 caches, the index list split in 128-row blocks
+        if ((int64_t)num_pages * page_size >= ((int64_t)1 << 31)) return DSA_ERR_UNSUPPORTED;
+        const int chunk = (int)(ceil_div(ceil_div(kw, splits), 128) * 128);
+        const int tc_splits = (int)ceil_div(kw, chunk);
+        e = launch_sparse_attn_tc_kv8((const uint16_t *)q, (const uint8_t *)k_cache, k_cache_scale,
+                                      (const uint8_t *)v_cache, v_cache_scale, num_pages * page_size,
+                                      block_table, context_lens, num_pages, max_pages_per_seq, page_size, idx,
+                                      B, H_q, d, kw, sm_scale, (uint16_t *)out, lse_out, part, tc_splits, hdr,
+                                      st, /*chained=*/true);
+        if (e == cudaErrorNotSupported) return DSA_ERR_UNSUPPORTED;
+        if (e == cudaSuccess) e = launch_merge_splits(part, B, tc_splits, H_q, d, (uint16_t *)out, lse_out, st);
+        return cuda_status(e);
+    }
     if (e == cudaSuccess) {
         bool done = false;
         if (sparse_attn_tc_supported(H_q, d) && (int64_t)num_pages * page_size < ((int64_t)1 << 31)) {
@@ -555,6 +577,21 @@ dsa_status dsa_decode_window(const void *q_idx, const float *q_scale, const void
                        stream);
 }
 
+dsa_status dsa_decode_kv8(const void *q_idx, const float *q_scale, const void *w, const void *q,
+                          const void *kidx_cache, const float *kscale_cache, const void *k_cache,
+                          const float *k_cache_scale, const void *v_cache, const float *v_cache_scale,
+                          const int32_t *block_table, const int32_t *context_lens, int64_t num_pages,
+                          int max_pages_per_seq, int page_size, int B, int64_t max_context, int H_I,
+                          int d_I, int H_q, int d, int k_sel, int window, float sm_scale, void *out,
+                          float *lse_out, int32_t *idx_out, void *workspace, size_t ws_bytes, void *stream)
+{
+    if (!k_cache_scale || !v_cache_scale) return DSA_ERR_INVALID_ARG;
+    return decode_impl(q_idx, q_scale, w, q, kidx_cache, kscale_cache, k_cache, v_cache, block_table,
+                       context_lens, num_pages, max_pages_per_seq, page_size, B, max_context, H_I, d_I,
+                       H_q, d, k_sel, window, sm_scale, out, lse_out, idx_out, workspace, ws_bytes,
+                       stream, k_cache_scale, v_cache_scale);
+}
+
 dsa_status dsa_quantize_e4m3(const void *x, dsa_dtype x_dtype, int64_t rows, int64_t cols,
                              uint8_t *codes_out, float *scale_out, void *stream)
 {
@@ -591,8 +628,35 @@ dsa_status dsa_cache_append(const void *kidx_new, dsa_dtype kidx_dtype, const vo
     return cuda_status(launch_cache_append(kidx_new, kidx_dtype == DSA_BF16, (const uint16_t *)k_new,
                                            (const uint16_t *)v_new, seq_ids, positions, N, B, block_table,
                                            max_pages_per_seq, num_pages, page_size, d_I, d,
-                                           (uint8_t *)kidx_cache, kscale_cache, (uint16_t *)k_cache,
-                                           (uint16_t *)v_cache, status, as_stream(stream)));
+                                           (uint8_t *)kidx_cache, kscale_cache, k_cache, v_cache, nullptr,
+                                           nullptr, status, as_stream(stream)));
+}
+
+dsa_status dsa_cache_append_kv8(const void *kidx_new, dsa_dtype kidx_dtype, const void *k_new,
+                                const void *v_new, const int32_t *seq_ids, const int32_t *positions,
+                                int64_t N, int B, const int32_t *block_table, int max_pages_per_seq,
+                                int64_t num_pages, int page_size, int d_I, int d, void *kidx_cache,
+                                float *kscale_cache, void *k_cache, float *k_cache_scale, void *v_cache,
+                                float *v_cache_scale, uint32_t *status, void *stream)
+{
+    if (kidx_dtype != DSA_BF16 && kidx_dtype != DSA_F32) return DSA_ERR_UNSUPPORTED;
+    if (N < 0) return DSA_ERR_INVALID_ARG;
+    if (N == 0) return DSA_OK;
+    if (!kidx_new || !k_new || !v_new || !seq_ids || !positions || !block_table || !kidx_cache ||
+        !kscale_cache || !k_cache || !k_cache_scale || !v_cache || !v_cache_scale)
+        return DSA_ERR_INVALID_ARG;
+    if (B <= 0 || max_pages_per_seq <= 0 || num_pages <= 0 || page_size <= 0 || d_I <= 0 || d <= 0)
+        return DSA_ERR_INVALID_ARG;
+    if (!aligned16(kidx_new) || !aligned16(k_new) || !aligned16(v_new) ||
+        (reinterpret_cast<uintptr_t>(kidx_cache) & 7u) || (reinterpret_cast<uintptr_t>(k_cache) & 7u) ||
+        (reinterpret_cast<uintptr_t>(v_cache) & 7u) || (reinterpret_cast<uintptr_t>(status) & 3u))
+        return DSA_ERR_INVALID_ARG;
+    if (d_I % 8 != 0 || d_I > 256 || d % 8 != 0 || d > 256) return DSA_ERR_UNSUPPORTED;
+    return cuda_status(launch_cache_append(kidx_new, kidx_dtype == DSA_BF16, (const uint16_t *)k_new,
+                                           (const uint16_t *)v_new, seq_ids, positions, N, B, block_table,
+                                           max_pages_per_seq, num_pages, page_size, d_I, d,
+                                           (uint8_t *)kidx_cache, kscale_cache, k_cache, v_cache, k_cache_scale,
+                                           v_cache_scale, status, as_stream(stream)));
 }
 
 dsa_status dsa_stream_status(void *workspace, void *stream)

@@ -51,13 +51,15 @@ cudaError_t launch_quantize_e4m3(const void *x, bool bf16_in, int64_t rows, int 
                                  float *scale, cudaStream_t st);
 // Token i -> sequence seq[i], position pos[i] of the paged caches: quantised
 // index key (d_I <= 256, a multiple of 8), bf16 K and V rows (d a multiple
-// of 8).  Out-of-range tokens are skipped and DSA_ERR_INVALID_ARG is
-// recorded in *status (nullable).
+// of 8) -- or, when k_cache_scale is given, K and V rows quantised to E4M3
+// with one scale each (d <= 256).  Out-of-range tokens are skipped and
+// DSA_ERR_INVALID_ARG is recorded in *status (nullable).
 cudaError_t launch_cache_append(const void *kidx_new, bool bf16_in, const uint16_t *k_new,
                                 const uint16_t *v_new, const int32_t *seq, const int32_t *pos, int64_t N,
                                 int B, const int32_t *bt, int max_pages, int64_t num_pages, int ps,
                                 int d_I, int d, uint8_t *kidx_cache, float *kscale_cache,
-                                uint16_t *k_cache, uint16_t *v_cache, uint32_t *status, cudaStream_t st);
+                                void *k_cache, void *v_cache, float *k_cache_scale, float *v_cache_scale,
+                                uint32_t *status, cudaStream_t st);
 
 // ---- sparse attention (sparse_attn.cu) ----
 struct PagedKV {
@@ -100,6 +102,15 @@ cudaError_t launch_sparse_attn_tc(const uint16_t *q, const uint16_t *k, const ui
                                   int page_size, const int32_t *idx, int64_t rows, int H, int d,
                                   int ksel, float sm_scale, uint16_t *out, float *lse, float *part,
                                   int splits, WsHeader *hdr, cudaStream_t st, bool chained = false);
+
+// The same over paged FP8 E4M3 K/V caches with one fp32 scale per cached row
+// (k8/v8 [num_pages * page_size, d], ks/vs [num_pages * page_size]).
+cudaError_t launch_sparse_attn_tc_kv8(const uint16_t *q, const uint8_t *k8, const float *ks, const uint8_t *v8,
+                                      const float *vs, int64_t kv_rows, const int32_t *block_table,
+                                      const int32_t *context_lens, int64_t num_pages, int max_pages,
+                                      int page_size, const int32_t *idx, int64_t rows, int H, int d, int ksel,
+                                      float sm_scale, uint16_t *out, float *lse, float *part, int splits,
+                                      WsHeader *hdr, cudaStream_t st, bool chained = false);
 
 // ---- decode indexer (decode_tc.cu: tcgen05 + TMA; decode.cu: mma.sync) ----
 bool decode_index_tc_supported(int H, int page_size);

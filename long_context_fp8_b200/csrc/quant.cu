@@ -182,15 +182,39 @@ cudaError_t launch_quantize_in(const In *x, int64_t rows, int cols, uint8_t *cod
     return launch_quantize_t<In, QZ_THREADS, 8>(x, rows, cols, codes, scale, st);
 }
 
-// One warp per new token: quantise its index key (d_I values, at most 256)
-// into the FP8 cache slot and copy its bf16 K and V rows (d values each).
+// A warp quantises one row of `cols` values (cols a multiple of 8, at most
+// 256; lane l holds chunk l) into dst[0, cols) and *dst_scale.
 template <typename In>
+__device__ __forceinline__ void warp_quantize_row(const In *src, int cols, uint8_t *dst, float *dst_scale, int lane)
+{
+    const int nch = cols / QZ_VEC;
+    float v[QZ_VEC];
+    float amax = 0.0f;
+    if (lane < nch) {
+        Chunk8<In>::load(src + lane * QZ_VEC, v);
+#pragma unroll
+        for (int j = 0; j < QZ_VEC; ++j) amax = fmaxf(amax, fabsf(v[j]));
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+    const float s = e4m3_scale_of(amax);
+    bool r_ok;
+    const float rs = e4m3_recip(s, r_ok);
+    if (lane < nch) *reinterpret_cast<uint2 *>(dst + lane * QZ_VEC) = e4m3_codes8(v, s, rs, r_ok);
+    if (lane == 0) *dst_scale = s;
+}
+
+// One warp per new token: quantise its index key (d_I values, at most 256)
+// into the FP8 cache slot, and copy its bf16 K and V rows (d values each), or
+// with KV8 quantise them too (d at most 256) into FP8 K/V caches with scales.
+template <typename In, bool KV8>
 __global__ void __launch_bounds__(QZ_THREADS)
 cache_append_kernel(const In *__restrict__ kidx_new, const uint16_t *__restrict__ k_new,
                     const uint16_t *__restrict__ v_new, const int32_t *__restrict__ seq,
                     const int32_t *__restrict__ pos, int64_t N, int B, const int32_t *__restrict__ bt,
                     int max_pages, int64_t num_pages, int ps, int d_I, int d, uint8_t *kidx_cache,
-                    float *kscale_cache, uint16_t *k_cache, uint16_t *v_cache, uint32_t *status)
+                    float *kscale_cache, void *k_cache, void *v_cache, float *k_cache_scale,
+                    float *v_cache_scale, uint32_t *status)
 {
     const int lane = threadIdx.x & 31;
     const int64_t warps = (int64_t)gridDim.x * (QZ_THREADS / 32);
@@ -204,30 +228,19 @@ cache_append_kernel(const In *__restrict__ kidx_new, const uint16_t *__restrict_
             continue;
         }
         const int64_t slot = page * ps + p % ps;
-        // index key: lane l holds chunk l of 8 values (d_I <= 256)
-        const int nch = d_I / QZ_VEC;
-        float v[QZ_VEC];
-        float amax = 0.0f;
-        if (lane < nch) {
-            Chunk8<In>::load(kidx_new + i * d_I + lane * QZ_VEC, v);
-#pragma unroll
-            for (int j = 0; j < QZ_VEC; ++j) amax = fmaxf(amax, fabsf(v[j]));
-        }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-        const float s = e4m3_scale_of(amax);
-        bool r_ok;
-        const float rs = e4m3_recip(s, r_ok);
-        if (lane < nch)
-            *reinterpret_cast<uint2 *>(kidx_cache + slot * d_I + lane * QZ_VEC) = e4m3_codes8(v, s, rs, r_ok);
-        if (lane == 0) kscale_cache[slot] = s;
-        // K and V rows: 16-byte chunks
-        const int vch = d / 8;
-        for (int c = lane; c < 2 * vch; c += 32) {
-            const bool is_v = c >= vch;
-            const int cc = is_v ? c - vch : c;
-            const uint4 val = __ldg(reinterpret_cast<const uint4 *>((is_v ? v_new : k_new) + i * d) + cc);
-            reinterpret_cast<uint4 *>((is_v ? v_cache : k_cache) + slot * d)[cc] = val;
+        warp_quantize_row(kidx_new + i * d_I, d_I, kidx_cache + slot * d_I, kscale_cache + slot, lane);
+        if constexpr (KV8) {
+            warp_quantize_row(k_new + i * d, d, static_cast<uint8_t *>(k_cache) + slot * d, k_cache_scale + slot, lane);
+            warp_quantize_row(v_new + i * d, d, static_cast<uint8_t *>(v_cache) + slot * d, v_cache_scale + slot, lane);
+        } else {
+            // K and V rows: 16-byte chunks
+            const int vch = d / 8;
+            for (int c = lane; c < 2 * vch; c += 32) {
+                const bool is_v = c >= vch;
+                const int cc = is_v ? c - vch : c;
+                const uint4 val = __ldg(reinterpret_cast<const uint4 *>((is_v ? v_new : k_new) + i * d) + cc);
+                reinterpret_cast<uint4 *>(static_cast<uint16_t *>(is_v ? v_cache : k_cache) + slot * d)[cc] = val;
+            }
         }
     }
 }
@@ -246,19 +259,23 @@ cudaError_t launch_cache_append(const void *kidx_new, bool bf16_in, const uint16
                                 const uint16_t *v_new, const int32_t *seq, const int32_t *pos, int64_t N,
                                 int B, const int32_t *bt, int max_pages, int64_t num_pages, int ps,
                                 int d_I, int d, uint8_t *kidx_cache, float *kscale_cache,
-                                uint16_t *k_cache, uint16_t *v_cache, uint32_t *status, cudaStream_t st)
+                                void *k_cache, void *v_cache, float *k_cache_scale, float *v_cache_scale,
+                                uint32_t *status, cudaStream_t st)
 {
     if (N <= 0) return cudaSuccess;
     const int64_t need = ceil_div(N, QZ_THREADS / 32);
     const unsigned grid = (unsigned)(need < 148 * 8 ? need : 148 * 8);
-    if (bf16_in)
-        cache_append_kernel<uint16_t><<<grid, QZ_THREADS, 0, st>>>(
-            static_cast<const uint16_t *>(kidx_new), k_new, v_new, seq, pos, N, B, bt, max_pages, num_pages,
-            ps, d_I, d, kidx_cache, kscale_cache, k_cache, v_cache, status);
-    else
-        cache_append_kernel<float><<<grid, QZ_THREADS, 0, st>>>(
-            static_cast<const float *>(kidx_new), k_new, v_new, seq, pos, N, B, bt, max_pages, num_pages, ps,
-            d_I, d, kidx_cache, kscale_cache, k_cache, v_cache, status);
+    const bool kv8 = k_cache_scale != nullptr;
+#define DSA_APPEND(IN, KV)                                                                                     \
+    cache_append_kernel<IN, KV><<<grid, QZ_THREADS, 0, st>>>(                                                  \
+        static_cast<const IN *>(kidx_new), k_new, v_new, seq, pos, N, B, bt, max_pages, num_pages, ps, d_I, d, \
+        kidx_cache, kscale_cache, k_cache, v_cache, k_cache_scale, v_cache_scale, status)
+    if (bf16_in) {
+        if (kv8) DSA_APPEND(uint16_t, true); else DSA_APPEND(uint16_t, false);
+    } else {
+        if (kv8) DSA_APPEND(float, true); else DSA_APPEND(float, false);
+    }
+#undef DSA_APPEND
     return cudaGetLastError();
 }
 

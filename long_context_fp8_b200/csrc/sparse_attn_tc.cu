@@ -33,6 +33,8 @@
 // Every mbarrier wait is bounded (DSA_ERR_TIMEOUT on expiry).
 #include <algorithm>
 
+#include <cuda_fp8.h>
+
 #include "kernels.h"
 #include "sm100.cuh"
 
@@ -68,6 +70,9 @@ constexpr float kRescaleThreshold = 8.f;     // log2 units
 struct AttnTcArgs {
     const uint16_t *k;       // K rows [kv_rows, D] (contiguous or paged cache)
     const uint16_t *v;
+    // FP8 K/V (the KV8 kernel): E4M3 rows [kv_rows, D] and one fp32 scale per row
+    const uint8_t *k8, *v8;
+    const float *ks, *vs;
     const int32_t *idx;      // [rows, ksel]
     int ksel;
     int H;                   // query heads (multiple of 128)
@@ -98,7 +103,31 @@ struct AtSmem {
     static constexpr int n_bars = 2 * AT_STAGES + 16;
     static constexpr size_t slot_off = bar_off + 8 * n_bars;
     static constexpr size_t total = slot_off + 16 + 1024;
+    // KV8: two staging buffers of one block's E4M3 K and V rows (64 x 256 bytes)
+    static constexpr size_t stg_bytes = (size_t)AT_BLK * 2 * AT_D;
+    static constexpr size_t stg_off = (slot_off + 16 + 127) / 128 * 128;
+    static constexpr size_t total_kv8 = stg_off + 2 * stg_bytes + 1024;
 };
+static_assert(AtSmem::total_kv8 + 64 <= 232448, "KV8 staging fits the shared memory of a CTA");
+
+// Eight bf16 pairs of 16 E4M3 codes times a scale (code j in byte j of the 16).
+__device__ __forceinline__ void e4m3x16_to_bf16_scaled(const uint4 &raw, float sc, uint32_t (&out)[8])
+{
+    const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const __nv_fp8x2_storage_t two = (__nv_fp8x2_storage_t)((w[i >> 1] >> (16 * (i & 1))) & 0xffffu);
+        const __half2_raw hr = __nv_cvt_fp8x2_to_halfraw2(two, __NV_E4M3);
+        const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&hr));
+        out[i] = pack_bf16x2(f.x * sc, f.y * sc);
+    }
+}
+
+__device__ __forceinline__ void st_shared_v4(void *p, uint32_t a, uint32_t b, uint32_t c, uint32_t d)
+{
+    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" :: "r"(smem_u32(p)), "r"(a), "r"(b), "r"(c), "r"(d)
+                 : "memory");
+}
 
 __device__ __forceinline__ bool wait_or_abort(uint64_t *bar, uint32_t parity, volatile int *abort)
 {
@@ -146,6 +175,11 @@ struct Item {
     }
 };
 
+// KV8: the K/V rows are FP8 E4M3 with a per-row scale (the paged decode
+// caches); the producers stage a block's codes one block ahead with cp.async
+// and widen them to bf16 (times the scale) into the same swizzled tiles, so
+// the MMA and softmax roles are those of the bf16 kernel.
+template <bool KV8>
 __global__ void __launch_bounds__(AT_THREADS, 1)
 sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap kmap,
                       const __grid_constant__ CUtensorMap vmap, const AttnTcArgs a)
@@ -254,19 +288,11 @@ sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_con
                 int p2 = (1 < item.nblk && e < item.e1) ? __ldg(irow + e) : -1;
                 const int chunk = lane & 15;
                 const bool is_v = lane >= 16;
-                for (int b = 0; b < item.nblk && !stop; ++b, ++g) {
-                    const int st = g % AT_STAGES;
-                    const int p = p1, pg = pg1;
-                    p1 = p2;
-                    pg1 = paged && p1 >= 0 && p1 < ctx ? __ldg(brow + p1 / a.page_size) : -1;
-                    e += AT_BLK;
-                    p2 = (b + 2 < item.nblk && e < item.e1) ? __ldg(irow + e) : -1;
-                    // warp-uniform outcome: the ballot and shuffles below need every lane
-                    const bool ok = __all_sync(0xffffffffu,
-                                               wait_or_abort(&kvempty[st], ((g / AT_STAGES) & 1) ^ 1, &abort_flag));
-                    if (!ok) { stop = true; break; }
-                    int r = 0;                            // K/V row (kv_rows < 2^31)
-                    bool v = false;
+                // K/V row of selected position p (page pg): lane l resolves row
+                // rbase + l of a block; out-of-range page ids are reported, not read.
+                auto resolve = [&](int p, int pg, int &r, bool &v) {
+                    r = 0;                                // K/V row (kv_rows < 2^31)
+                    v = false;
                     if (paged) {
                         if (p >= 0 && p < ctx) {
                             if (pg >= 0 && pg < a.num_pages) {
@@ -280,19 +306,98 @@ sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_con
                         r = p;
                         v = true;
                     }
-                    const unsigned vw = __ballot_sync(0xffffffffu, v);
-                    if (lane == 0) {
-                        valid[st * 2 + (warp - 4)] = vw;
-                        mbar_arrive(&kvfull[st]);          // releases the validity bits
-                    }
-                    uint8_t *tile = KVs + st * AT_STAGE + (is_v ? AT_KTILE : 0) + (chunk >> 3) * AT_KHALF + rbase * 128;
-                    const uint16_t *base = (is_v ? a.v : a.k) + chunk * 8;
+                };
+                // KV8: lane l copies (and later widens) 16-byte code chunk l % 16 -- K
+                // for l % 16 < 8, V otherwise -- of rows l / 16, l / 16 + 2, ... of
+                // the warp's 32, into staging buffer g % 2; the rows' scales ride one
+                // block ahead in registers (lane i: row rbase + i).
+                uint8_t *stg = smem + AtSmem::stg_off;
+                int r_cur = 0, r_nx = 0;
+                bool v_cur = false, v_nx = false;
+                float ks_cur = 0.f, vs_cur = 0.f, ks_nx = 0.f, vs_nx = 0.f;
+                auto stage = [&](int gb, int r, bool v) {
+                    const unsigned vb = __ballot_sync(0xffffffffu, v);
+                    uint8_t *sb = stg + (gb & 1) * AtSmem::stg_bytes + rbase * 2 * AT_D + chunk * 16;
+                    const uint8_t *src = (chunk < 8 ? a.k8 : a.v8) + (chunk & 7) * 16;
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) {        // row rbase + i of the block (rbase % 8 == 0)
+                    for (int j = 0; j < 16; ++j) {
+                        const int i = 2 * j + (lane >> 4);
                         const int ri = __shfl_sync(0xffffffffu, r, i);
-                        cp_async_16(tile + i * 128 + (((chunk ^ i) & 7) << 4), base + (int64_t)ri * AT_D, (vw >> i) & 1u);
+                        cp_async_16(sb + i * 2 * AT_D, src + (int64_t)ri * AT_D, (vb >> i) & 1u);
                     }
-                    cp_async_arrive_noinc(&kvfull[st]);   // fires when this thread's copies land
+                };
+                if constexpr (KV8) {
+                    if (item.nblk > 0 && !stop) {
+                        resolve(p1, pg1, r_cur, v_cur);
+                        stage(g, r_cur, v_cur);
+                        ks_cur = v_cur ? __ldg(a.ks + r_cur) : 0.f;
+                        vs_cur = v_cur ? __ldg(a.vs + r_cur) : 0.f;
+                    }
+                    cp_async_commit();
+                }
+                for (int b = 0; b < item.nblk && !stop; ++b, ++g) {
+                    const int st = g % AT_STAGES;
+                    const int p = p1, pg = pg1;
+                    p1 = p2;
+                    pg1 = paged && p1 >= 0 && p1 < ctx ? __ldg(brow + p1 / a.page_size) : -1;
+                    e += AT_BLK;
+                    p2 = (b + 2 < item.nblk && e < item.e1) ? __ldg(irow + e) : -1;
+                    // warp-uniform outcome: the ballot and shuffles below need every lane
+                    const bool ok = __all_sync(0xffffffffu,
+                                               wait_or_abort(&kvempty[st], ((g / AT_STAGES) & 1) ^ 1, &abort_flag));
+                    if (!ok) { stop = true; break; }
+                    if constexpr (!KV8) {
+                        int r;
+                        bool v;
+                        resolve(p, pg, r, v);
+                        const unsigned vw = __ballot_sync(0xffffffffu, v);
+                        if (lane == 0) {
+                            valid[st * 2 + (warp - 4)] = vw;
+                            mbar_arrive(&kvfull[st]);      // releases the validity bits
+                        }
+                        uint8_t *tile = KVs + st * AT_STAGE + (is_v ? AT_KTILE : 0) + (chunk >> 3) * AT_KHALF + rbase * 128;
+                        const uint16_t *base = (is_v ? a.v : a.k) + chunk * 8;
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) {    // row rbase + i of the block (rbase % 8 == 0)
+                            const int ri = __shfl_sync(0xffffffffu, r, i);
+                            cp_async_16(tile + i * 128 + (((chunk ^ i) & 7) << 4), base + (int64_t)ri * AT_D, (vw >> i) & 1u);
+                        }
+                        cp_async_arrive_noinc(&kvfull[st]);   // fires when this thread's copies land
+                    } else {
+                        const unsigned vw = __ballot_sync(0xffffffffu, v_cur);
+                        if (lane == 0) {
+                            valid[st * 2 + (warp - 4)] = vw;
+                            mbar_arrive(&kvfull[st]);      // releases the validity bits
+                        }
+                        // the next block's codes and scales go out before this block is widened
+                        if (b + 1 < item.nblk) {
+                            resolve(p1, pg1, r_nx, v_nx);
+                            stage(g + 1, r_nx, v_nx);
+                            ks_nx = v_nx ? __ldg(a.ks + r_nx) : 0.f;
+                            vs_nx = v_nx ? __ldg(a.vs + r_nx) : 0.f;
+                        }
+                        cp_async_commit();
+                        cp_async_wait<1>();               // this lane's copies of block g have landed
+                        const uint8_t *sb = stg + (g & 1) * AtSmem::stg_bytes + rbase * 2 * AT_D + chunk * 16;
+                        uint8_t *tile = KVs + st * AT_STAGE + (chunk < 8 ? 0 : AT_KTILE) + ((chunk & 7) >> 2) * AT_KHALF +
+                                        rbase * 128;
+                        const int c0 = 2 * (chunk & 7);   // bf16 chunks c0, c0 + 1 of the row
+#pragma unroll 4
+                        for (int j = 0; j < 16; ++j) {
+                            const int i = 2 * j + (lane >> 4);
+                            const float sk = __shfl_sync(0xffffffffu, ks_cur, i);
+                            const float sv = __shfl_sync(0xffffffffu, vs_cur, i);
+                            const uint4 raw = *reinterpret_cast<const uint4 *>(sb + i * 2 * AT_D);
+                            uint32_t o[8];
+                            e4m3x16_to_bf16_scaled(raw, chunk < 8 ? sk : sv, o);
+                            uint8_t *row = tile + i * 128;
+                            st_shared_v4(row + ((((c0) ^ i) & 7) << 4), o[0], o[1], o[2], o[3]);
+                            st_shared_v4(row + ((((c0 + 1) ^ i) & 7) << 4), o[4], o[5], o[6], o[7]);
+                        }
+                        fence_proxy_async_smem();         // generic writes, read by the tensor cores
+                        mbar_arrive(&kvfull[st]);
+                        r_cur = r_nx; v_cur = v_nx; ks_cur = ks_nx; vs_cur = vs_nx;
+                    }
                     if (pt == 0) kv_issued = g + 1;
                 }
             }
@@ -599,6 +704,49 @@ sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_con
 
 bool sparse_attn_tc_supported(int H, int d) { return d == AT_D && H % AT_HEADS == 0 && H / AT_HEADS <= 65535; }
 
+namespace {
+
+template <bool KV8>
+cudaError_t launch_attn_tc_impl(const CUtensorMap &qmap, const CUtensorMap &kmap, const CUtensorMap &vmap,
+                                const AttnTcArgs &a, cudaStream_t st, bool chained)
+{
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const size_t smem = KV8 ? AtSmem::total_kv8 : AtSmem::total;
+    cudaFuncAttributes fa;
+    cudaError_t e = cudaFuncGetAttributes(&fa, sparse_attn_tc_kernel<KV8>);
+    if (e != cudaSuccess) return e;
+    if (fa.numRegs != AT_LAUNCH_REGS) return cudaErrorNotSupported;   // the register split assumes it
+    e = cudaFuncSetAttribute(sparse_attn_tc_kernel<KV8>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    const unsigned grid = (unsigned)std::min<int64_t>(a.items, sms);
+    if (chained) {
+        e = launch_chained(sparse_attn_tc_kernel<KV8>, dim3(grid), dim3(AT_THREADS), smem, st, qmap, kmap, vmap, a);
+        if (e != cudaSuccess) return e;
+    } else {
+        sparse_attn_tc_kernel<KV8><<<grid, AT_THREADS, smem, st>>>(qmap, kmap, vmap, a);
+    }
+    return cudaGetLastError();
+}
+
+void fill_common(AttnTcArgs &a, const int32_t *idx, int64_t rows, int H, int ksel, int64_t kv_rows, int64_t T,
+                 const int32_t *block_table, const int32_t *context_lens, int64_t num_pages, int max_pages,
+                 int page_size, float sm_scale, uint16_t *out, float *lse, float *part, int splits, WsHeader *hdr)
+{
+    a.idx = idx; a.ksel = ksel; a.H = H; a.kv_rows = kv_rows; a.T = T;
+    a.block_table = block_table; a.context_lens = context_lens; a.num_pages = num_pages;
+    a.max_pages = max_pages; a.page_size = page_size;
+    a.scale_log2 = sm_scale * kLog2e;
+    a.out = out; a.lse = lse; a.part = part; a.rows = rows;
+    a.splits = splits;
+    a.chunk = (int)(ceil_div(ceil_div(ksel, splits), AT_BLK) * AT_BLK);
+    a.items = rows * (H / AT_HEADS) * splits;
+    a.hdr = hdr;
+}
+
+}  // namespace
+
 cudaError_t launch_sparse_attn_tc(const uint16_t *q, const uint16_t *k, const uint16_t *v,
                                   int64_t kv_rows, int64_t T, const int32_t *block_table,
                                   const int32_t *context_lens, int64_t num_pages, int max_pages,
@@ -617,33 +765,31 @@ cudaError_t launch_sparse_attn_tc(const uint16_t *q, const uint16_t *k, const ui
         return cudaErrorNotSupported;
     AttnTcArgs a{};
     a.k = k; a.v = v;
-    a.idx = idx; a.ksel = ksel; a.H = H; a.kv_rows = kv_rows; a.T = T;
-    a.block_table = block_table; a.context_lens = context_lens; a.num_pages = num_pages;
-    a.max_pages = max_pages; a.page_size = page_size;
-    a.scale_log2 = sm_scale * kLog2e;
-    a.out = out; a.lse = lse; a.part = part; a.rows = rows;
-    a.splits = splits;
-    a.chunk = (int)(ceil_div(ceil_div(ksel, splits), AT_BLK) * AT_BLK);
-    a.items = rows * (H / AT_HEADS) * splits;
-    a.hdr = hdr;
-    int dev = 0, sms = 148;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    const size_t smem = AtSmem::total;
-    cudaFuncAttributes fa;
-    cudaError_t e = cudaFuncGetAttributes(&fa, sparse_attn_tc_kernel);
-    if (e != cudaSuccess) return e;
-    if (fa.numRegs != AT_LAUNCH_REGS) return cudaErrorNotSupported;
-    e = cudaFuncSetAttribute(sparse_attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    const unsigned grid = (unsigned)std::min<int64_t>(a.items, sms);
-    if (chained) {
-        e = launch_chained(sparse_attn_tc_kernel, dim3(grid), dim3(AT_THREADS), smem, st, qmap, kmap, vmap, a);
-        if (e != cudaSuccess) return e;
-    } else {
-        sparse_attn_tc_kernel<<<grid, AT_THREADS, smem, st>>>(qmap, kmap, vmap, a);
-    }
-    return cudaGetLastError();
+    fill_common(a, idx, rows, H, ksel, kv_rows, T, block_table, context_lens, num_pages, max_pages, page_size,
+                sm_scale, out, lse, part, splits, hdr);
+    return launch_attn_tc_impl<false>(qmap, kmap, vmap, a, st, chained);
+}
+
+cudaError_t launch_sparse_attn_tc_kv8(const uint16_t *q, const uint8_t *k8, const float *ks, const uint8_t *v8,
+                                      const float *vs, int64_t kv_rows, const int32_t *block_table,
+                                      const int32_t *context_lens, int64_t num_pages, int max_pages,
+                                      int page_size, const int32_t *idx, int64_t rows, int H, int d, int ksel,
+                                      float sm_scale, uint16_t *out, float *lse, float *part, int splits,
+                                      WsHeader *hdr, cudaStream_t st, bool chained)
+{
+    if (rows <= 0) return cudaSuccess;
+    if (!sparse_attn_tc_supported(H, d) || kv_rows >= ((int64_t)1 << 31) ||
+        rows * H >= ((int64_t)1 << 31))
+        return cudaErrorNotSupported;
+    CUtensorMap qmap;
+    if (!make_tmap_bf16_2d(&qmap, q, AT_D, (uint64_t)rows * H, AT_D * 2, 64, AT_HEADS)) return cudaErrorNotSupported;
+    AttnTcArgs a{};
+    a.k8 = k8; a.v8 = v8; a.ks = ks; a.vs = vs;
+    fill_common(a, idx, rows, H, ksel, kv_rows, 0, block_table, context_lens, num_pages, max_pages, page_size,
+                sm_scale, out, lse, part, splits, hdr);
+    // the K/V maps are parameters of the bf16 kernel's signature only; the KV8
+    // producers copy with cp.async, so the query map stands in for them
+    return launch_attn_tc_impl<true>(qmap, qmap, qmap, a, st, chained);
 }
 
 }  // namespace dsa

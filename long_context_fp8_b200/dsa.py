@@ -26,8 +26,9 @@ STATUS = {0: "DSA_OK", 1: "DSA_ERR_INVALID_ARG", 2: "DSA_ERR_UNSUPPORTED", 3: "D
 EXPORTS = ("dsa_status_string", "dsa_version", "dsa_index_scores", "dsa_topk_workspace_size",
            "dsa_topk", "dsa_topk_window", "dsa_sparse_attn", "dsa_prefill_workspace_size",
            "dsa_prefill", "dsa_prefill_window", "dsa_prefill_host_workspace_size", "dsa_prefill_host",
-           "dsa_decode_workspace_size", "dsa_decode", "dsa_decode_window", "dsa_quantize_e4m3",
-           "dsa_cache_append", "dsa_decode_noalloc", "dsa_stream_status")
+           "dsa_decode_workspace_size", "dsa_decode", "dsa_decode_window", "dsa_decode_kv8",
+           "dsa_quantize_e4m3", "dsa_cache_append", "dsa_cache_append_kv8", "dsa_decode_noalloc",
+           "dsa_stream_status")
 
 
 class DSAError(RuntimeError):
@@ -74,6 +75,10 @@ def load(path: str = LIB_PATH):
         "dsa_decode_window": ([P, P, P, P, P, P, P, P, P, P, I64, I32, I32, I32, I64, I32, I32, I32, I32,
                                I32, I32, F, P, P, P, P, SZ, P], I32),
         "dsa_quantize_e4m3": ([P, I32, I64, I64, P, P, P], I32),
+        "dsa_decode_kv8": ([P, P, P, P, P, P, P, P, P, P, P, P, I64, I32, I32, I32, I64, I32, I32, I32, I32,
+                            I32, I32, F, P, P, P, P, SZ, P], I32),
+        "dsa_cache_append_kv8": ([P, I32, P, P, P, P, I64, I32, P, I32, I64, I32, I32, I32, P, P, P, P, P, P,
+                                  P, P], I32),
         "dsa_cache_append": ([P, I32, P, P, P, P, I64, I32, P, I32, I64, I32, I32, I32, P, P, P, P, P, P],
                              I32),
         "dsa_stream_status": ([P, P], I32),
@@ -370,6 +375,51 @@ def dsa_decode_window(inp: dict, k_sel: int, window: int, max_context: int, sm_s
                                _stream(stream))
     _check("dsa_decode_window", st)
     return out, lse, idx_out
+
+
+def dsa_decode_kv8(inp: dict, k_sel: int, max_context: int, window: int = 0, sm_scale=None, out=None,
+                   lse=None, idx_out=None, ws=None, want_idx=True, stream=None):
+    """Decode over FP8 K/V caches (``inp`` holds uint8 k_cache/v_cache and f32
+    k_cache_scale/v_cache_scale) -> (out, lse, idx [B, k_sel + window])."""
+    B, H_I, d_I = inp["q_idx"].shape
+    _, H_q, d = inp["q"].shape
+    P, ps, _ = inp["kidx_cache"].shape
+    max_pages = inp["block_table"].shape[1]
+    sm_scale = 1.0 / math.sqrt(d) if sm_scale is None else sm_scale
+    lib = load()
+    kw = k_sel + window
+    if ws is None:
+        ws = workspace(lib.dsa_decode_workspace_size(B, max_context, H_q, d, kw), inp["q"].device)
+    if out is None:
+        out = torch.empty_like(inp["q"])
+    if lse is None:
+        lse = torch.empty((B, H_q), dtype=torch.float32, device=inp["q"].device)
+    if idx_out is None and want_idx:
+        idx_out = torch.empty((B, kw), dtype=torch.int32, device=inp["q"].device)
+    st = lib.dsa_decode_kv8(_p(inp["q_idx"]), _p(inp["q_scale"]), _p(inp["w"]), _p(inp["q"]),
+                            _p(inp["kidx_cache"]), _p(inp["kscale_cache"]), _p(inp["k_cache"]),
+                            _p(inp["k_cache_scale"]), _p(inp["v_cache"]), _p(inp["v_cache_scale"]),
+                            _p(inp["block_table"]), _p(inp["context_lens"]), P, max_pages, ps, B, max_context,
+                            H_I, d_I, H_q, d, k_sel, window, sm_scale, _p(out), _p(lse), _p(idx_out), _p(ws),
+                            ws.numel(), _stream(stream))
+    _check("dsa_decode_kv8", st)
+    return out, lse, idx_out
+
+
+def dsa_cache_append_kv8(caches: dict, kidx_new, k_new, v_new, seq_ids, positions, block_table,
+                         status=None, stream=None):
+    """dsa_cache_append for FP8 K/V caches (``caches`` also holds
+    k_cache_scale/v_cache_scale): index key, K and V rows all quantised."""
+    N, d_I = kidx_new.shape
+    d = k_new.shape[1]
+    P, ps, _ = caches["kidx_cache"].shape
+    B, max_pages = block_table.shape
+    st = load().dsa_cache_append_kv8(_p(kidx_new), _val_dtype(kidx_new), _p(k_new), _p(v_new), _p(seq_ids),
+                                     _p(positions), N, B, _p(block_table), max_pages, P, ps, d_I, d,
+                                     _p(caches["kidx_cache"]), _p(caches["kscale_cache"]), _p(caches["k_cache"]),
+                                     _p(caches["k_cache_scale"]), _p(caches["v_cache"]),
+                                     _p(caches["v_cache_scale"]), _p(status), _stream(stream))
+    _check("dsa_cache_append_kv8", st)
 
 
 NOALLOC_SCRATCH_BYTES = 64 << 20

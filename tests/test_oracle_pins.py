@@ -576,3 +576,32 @@ def test_decode_fp8_kv_power_of_two_scales_equal_bf16_path():
     np.testing.assert_array_equal(a["idx"], b["idx"])
     np.testing.assert_allclose(a["out"], b["out"], rtol=1e-15, atol=1e-15)
     np.testing.assert_allclose(a["lse"], b["lse"], rtol=1e-15, atol=1e-15)
+
+
+def test_cache_append_fp8_kv_quantises_k_and_v():
+    rng = np.random.default_rng(33)
+    B, P, ps, D_I, D, maxp = 3, 20, 16, 32, 24, 4
+    bt = np.stack([rng.permutation(P)[:maxp] for _ in range(B)]).astype(np.int32)
+    caches = dict(kidx_cache=rng.integers(0, 0x7E, (P, ps, D_I)).astype(np.uint8),
+                  kscale_cache=np.ones((P, ps), np.float32),
+                  k_cache=rng.integers(0, 0x7E, (P, ps, D)).astype(np.uint8),
+                  v_cache=rng.integers(0, 0x7E, (P, ps, D)).astype(np.uint8),
+                  k_cache_scale=np.ones((P, ps), np.float32), v_cache_scale=np.ones((P, ps), np.float32))
+    before = {k: v.copy() for k, v in caches.items()}
+    seq = np.array([0, 1, 2, 2], np.int32)
+    pos = np.array([5, 63, 0, 17], np.int32)
+    kin = torch.from_numpy(rng.standard_normal((4, D_I)).astype(np.float32)).to(torch.bfloat16)
+    kn = torch.from_numpy(rng.standard_normal((4, D)).astype(np.float32) * 5).to(torch.bfloat16)
+    vn = torch.from_numpy(rng.standard_normal((4, D)).astype(np.float32) / 5).to(torch.bfloat16)
+    assert oracle.cache_append(caches, kin, kn, vn, seq, pos, bt) == 0
+    kc, ksc = oracle.quantize_e4m3(kn)
+    vc, vsc = oracle.quantize_e4m3(vn)
+    touched = np.zeros((P, ps), bool)
+    for i in range(4):
+        page, slot = bt[seq[i], pos[i] // ps], pos[i] % ps
+        touched[page, slot] = True
+        np.testing.assert_array_equal(caches["k_cache"][page, slot], kc[i])
+        np.testing.assert_array_equal(caches["v_cache"][page, slot], vc[i])
+        assert caches["k_cache_scale"][page, slot] == ksc[i] and caches["v_cache_scale"][page, slot] == vsc[i]
+    for name in caches:
+        np.testing.assert_array_equal(caches[name][~touched], before[name][~touched])
