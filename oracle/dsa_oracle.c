@@ -488,15 +488,16 @@ int dsa_or_quantize_e4m3(const void *x, int dtype, int64_t rows, int64_t cols, u
  * at position pos[i], i.e. physical page bt[seq[i]*max_pages + pos[i]/ps],
  * slot pos[i]%ps: its index key kidx_new[i, 0..D_I) (OR_F32 or OR_BF16) is
  * quantised into kidx_cache/kscale_cache (stage 6), and its bf16 K and V rows
- * are copied into k_cache/v_cache.  bt is [B, max_pages].  Returns 0, or -2
+ * are copied into k_cache/v_cache -- or, when kcs/vcs are given (stage 7),
+ * quantised into E4M3 k_cache/v_cache with scales kcs/vcs [P,ps].  bt is [B, max_pages].  Returns 0, or -2
  * (and stops) at the first token whose sequence, position or page id is out
  * of range.
  */
 int dsa_or_cache_append(const void *kidx_new, int kdt, const uint16_t *k_new, const uint16_t *v_new,
                         const int32_t *seq, const int32_t *pos, int64_t N, int B, const int32_t *bt,
                         int max_pages, int64_t num_pages, int ps, int D_I, int D,
-                        uint8_t *kidx_cache, float *kscale_cache, uint16_t *k_cache,
-                        uint16_t *v_cache)
+                        uint8_t *kidx_cache, float *kscale_cache, void *k_cache,
+                        void *v_cache, float *kcs, float *vcs)
 {
     for (int64_t i = 0; i < N; ++i) {
         int64_t p = pos[i];
@@ -505,9 +506,14 @@ int dsa_or_cache_append(const void *kidx_new, int kdt, const uint16_t *k_new, co
         if (page < 0 || page >= num_pages) return -2;
         int64_t slot = page * ps + p % ps;
         quantize_row(kidx_new, kdt, i * D_I, D_I, kidx_cache + slot * D_I, kscale_cache + slot);
-        for (int c = 0; c < D; ++c) {
-            k_cache[slot * D + c] = k_new[i * D + c];
-            v_cache[slot * D + c] = v_new[i * D + c];
+        if (kcs) {                                  /* stage 7: FP8 K/V rows, one scale each */
+            quantize_row(k_new, OR_BF16, i * D, D, (uint8_t *)k_cache + slot * D, kcs + slot);
+            quantize_row(v_new, OR_BF16, i * D, D, (uint8_t *)v_cache + slot * D, vcs + slot);
+        } else {
+            for (int c = 0; c < D; ++c) {
+                ((uint16_t *)k_cache)[slot * D + c] = k_new[i * D + c];
+                ((uint16_t *)v_cache)[slot * D + c] = v_new[i * D + c];
+            }
         }
     }
     return 0;

@@ -64,7 +64,7 @@ def load(path: Optional[str] = None):
     lib.dsa_or_quantize_e4m3.argtypes = [P, I32, I64, I64, P, P]
     lib.dsa_or_quantize_e4m3.restype = I32
     lib.dsa_or_cache_append.argtypes = [P, I32, P, P, P, P, I64, I32, P, I32, I64, I32, I32, I32,
-                                        P, P, P, P]
+                                        P, P, P, P, P, P]
     lib.dsa_or_cache_append.restype = I32
     if path == _LIB:
         _lib = lib
@@ -219,13 +219,14 @@ def cache_append(caches: dict, kidx_new, k_new, v_new, seq, pos, block_table, li
     sq, ps_ = _np(seq, np.int32), _np(pos, np.int32)
     bt = _np(block_table, np.int32)
     kic, ksc, kc, vc = (caches[n] for n in ("kidx_cache", "kscale_cache", "k_cache", "v_cache"))
-    for a in (kic, ksc, kc, vc):
+    kcs, vcs = caches.get("k_cache_scale"), caches.get("v_cache_scale")   # FP8 K/V (stage 7)
+    for a in (kic, ksc, kc, vc) + ((kcs, vcs) if kcs is not None else ()):
         assert a.flags.c_contiguous
     P, ps, D_I = kic.shape
     D = kc.shape[2]
     return lib.dsa_or_cache_append(_ptr(kn), dt, _ptr(kk), _ptr(vv), _ptr(sq), _ptr(ps_), sq.size,
                                    bt.shape[0], _ptr(bt), bt.shape[1], P, ps, D_I, D, _ptr(kic),
-                                   _ptr(ksc), _ptr(kc), _ptr(vc))
+                                   _ptr(ksc), _ptr(kc), _ptr(vc), _ptr(kcs), _ptr(vcs))
 
 
 def sparse_attn(q, K, V, idx, rows, sm_scale, lib=None, compact=False):
