@@ -12,7 +12,7 @@
 //   warps 4-5 producers: thread p resolves selected position p of a 64-row
 //             block (through the page table for the paged caches) and copies
 //             its K and V rows with 16-byte cp.async into the 128-byte-swizzled
-//             tiles of a 4-stage ring (many small loads in flight per SM: the
+//             tiles of a 5-stage ring (many small loads in flight per SM: the
 //             rows are scattered); one thread also brings the next item's Q
 //             with TMA into a second Q buffer;
 //   warp 6    S issuer: S = Q K^T (kind::f16, M 128 heads, N 64 rows,
@@ -46,7 +46,11 @@ using namespace sm100;
 constexpr int AT_HEADS = 128;          // UMMA M: query heads per item
 constexpr int AT_D = 128;              // head dim
 constexpr int AT_BLK = 64;             // selected rows per block (UMMA N of S, K of PV)
-constexpr int AT_STAGES = 4;           // K/V gather ring depth
+// K/V gather ring depth: a block holds its stage from the gather to the end of
+// its PV product (about four block periods), so the ring bounds the block rate.
+// Five stages fill the shared memory of the bf16 kernel; the KV8 kernel keeps
+// four beside its staging buffers.
+template <bool KV8> constexpr int at_stages() { return KV8 ? 4 : 5; }
 constexpr int AT_THREADS = 384;        // 2 x 4 softmax warps, 2 producer warps, S and PV issuer warps
 constexpr int AT_PRODUCERS = 64;       // producer threads: one selected row each per block
 // Register split by warpgroup: producers and issuers (warps 4-7) give theirs to
@@ -93,14 +97,15 @@ struct AttnTcArgs {
     WsHeader *hdr;
 };
 
-struct AtSmem {
+template <int NST>
+struct AtSmemT {
     static constexpr size_t q_off = 0;                                   // [2] Q tiles
     static constexpr size_t kv_off = q_off + 2 * AT_QTILE;                // [stages] K, V tiles
-    static constexpr size_t valid_off = kv_off + (size_t)AT_STAGES * AT_STAGE; // [stages][2] validity bits
-    static constexpr size_t ml_off = valid_off + AT_STAGES * 2 * 4;      // set 1's (m, l) per head
+    static constexpr size_t valid_off = kv_off + (size_t)NST * AT_STAGE;  // [stages][2] validity bits
+    static constexpr size_t ml_off = valid_off + NST * 2 * 4;            // set 1's (m, l) per head
     static constexpr size_t bar_off = ml_off + 2 * AT_HEADS * 4;
     // qfull[2] qempty[2] kvfull[S] kvempty[S] sfull[2] sempty[2] pfull[2] pempty[2] ofull oempty mlfull mlempty
-    static constexpr int n_bars = 2 * AT_STAGES + 16;
+    static constexpr int n_bars = 2 * NST + 16;
     static constexpr size_t slot_off = bar_off + 8 * n_bars;
     static constexpr size_t total = slot_off + 16 + 1024;
     // KV8: two staging buffers of one block's E4M3 K and V rows (64 x 256 bytes)
@@ -108,7 +113,10 @@ struct AtSmem {
     static constexpr size_t stg_off = (slot_off + 16 + 127) / 128 * 128;
     static constexpr size_t total_kv8 = stg_off + 2 * stg_bytes + 1024;
 };
-static_assert(AtSmem::total_kv8 + 64 <= 232448, "KV8 staging fits the shared memory of a CTA");
+using AtSmemBf16 = AtSmemT<at_stages<false>()>;
+using AtSmemKv8 = AtSmemT<at_stages<true>()>;
+static_assert(AtSmemBf16::total + 64 <= 232448, "the bf16 kernel's ring fits the shared memory of a CTA");
+static_assert(AtSmemKv8::total_kv8 + 64 <= 232448, "KV8 staging fits the shared memory of a CTA");
 
 // Eight bf16 pairs of 16 E4M3 codes times a scale (code j in byte j of the 16).
 __device__ __forceinline__ void e4m3x16_to_bf16_scaled(const uint4 &raw, float sc, uint32_t (&out)[8])
@@ -184,6 +192,8 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
 sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap kmap,
                       const __grid_constant__ CUtensorMap vmap, const AttnTcArgs a)
 {
+    constexpr int AT_STAGES = at_stages<KV8>();
+    using AtSmem = AtSmemT<AT_STAGES>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *Qs = smem + AtSmem::q_off;
@@ -713,7 +723,7 @@ cudaError_t launch_attn_tc_impl(const CUtensorMap &qmap, const CUtensorMap &kmap
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    const size_t smem = KV8 ? AtSmem::total_kv8 : AtSmem::total;
+    const size_t smem = KV8 ? AtSmemKv8::total_kv8 : AtSmemBf16::total;
     cudaFuncAttributes fa;
     cudaError_t e = cudaFuncGetAttributes(&fa, sparse_attn_tc_kernel<KV8>);
     if (e != cudaSuccess) return e;
