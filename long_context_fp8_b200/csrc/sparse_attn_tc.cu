@@ -50,7 +50,8 @@ constexpr int AT_BLK = 64;             // selected rows per block (UMMA N of S, 
 // its PV product (about four block periods), so the ring bounds the block rate.
 // Five stages fill the shared memory of the bf16 kernel; the KV8 kernel keeps
 // four beside its staging buffers.
-template <bool KV8> constexpr int at_stages() { return KV8 ? 4 : 5; }
+template <bool KV8> constexpr int at_stages() { return KV8 ? 2 : 5; }
+constexpr int AT_NSTG = 4;             // KV8: staging buffers of E4M3 blocks (three blocks of lookahead)
 constexpr int AT_THREADS = 384;        // 2 x 4 softmax warps, 2 producer warps, S and PV issuer warps
 constexpr int AT_PRODUCERS = 64;       // producer threads: one selected row each per block
 // Register split by warpgroup: producers and issuers (warps 4-7) give theirs to
@@ -107,16 +108,19 @@ struct AtSmemT {
     // qfull[2] qempty[2] kvfull[S] kvempty[S] sfull[2] sempty[2] pfull[2] pempty[2] ofull oempty mlfull mlempty
     static constexpr int n_bars = 2 * NST + 16;
     static constexpr size_t slot_off = bar_off + 8 * n_bars;
-    static constexpr size_t total = slot_off + 16 + 1024;
-    // KV8: two staging buffers of one block's E4M3 K and V rows (64 x 256 bytes)
+    static constexpr size_t total() { return slot_off + 16 + 1024; }
+    // KV8: staging buffers of one block's E4M3 K and V rows (64 x 256 bytes), then
+    // their K and V scales ([buf][2][64] floats) and validity words ([buf][2])
     static constexpr size_t stg_bytes = (size_t)AT_BLK * 2 * AT_D;
     static constexpr size_t stg_off = (slot_off + 16 + 127) / 128 * 128;
-    static constexpr size_t total_kv8 = stg_off + 2 * stg_bytes + 1024;
+    static constexpr size_t stg_sc_off = stg_off + AT_NSTG * stg_bytes;
+    static constexpr size_t stg_vw_off = stg_sc_off + AT_NSTG * 2 * AT_BLK * 4;
+    static constexpr size_t total_kv8() { return stg_vw_off + AT_NSTG * 2 * 4 + 1024; }
 };
 using AtSmemBf16 = AtSmemT<at_stages<false>()>;
 using AtSmemKv8 = AtSmemT<at_stages<true>()>;
-static_assert(AtSmemBf16::total + 64 <= 232448, "the bf16 kernel's ring fits the shared memory of a CTA");
-static_assert(AtSmemKv8::total_kv8 + 64 <= 232448, "KV8 staging fits the shared memory of a CTA");
+static_assert(AtSmemBf16::total() + 64 <= 232448, "the bf16 kernel's ring fits the shared memory of a CTA");
+static_assert(AtSmemKv8::total_kv8() + 64 <= 232448, "KV8 staging fits the shared memory of a CTA");
 
 // Eight bf16 pairs of 16 E4M3 codes times a scale (code j in byte j of the 16).
 __device__ __forceinline__ void e4m3x16_to_bf16_scaled(const uint4 &raw, float sc, uint32_t (&out)[8])
@@ -129,6 +133,13 @@ __device__ __forceinline__ void e4m3x16_to_bf16_scaled(const uint4 &raw, float s
         const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&hr));
         out[i] = pack_bf16x2(f.x * sc, f.y * sc);
     }
+}
+
+// 4-byte cp.async (zero-filled when !valid).
+__device__ __forceinline__ void cp_async_4(void *smem, const void *gmem, bool valid)
+{
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;\n"
+                 :: "r"(smem_u32(smem)), "l"(gmem), "r"(valid ? 4u : 0u) : "memory");
 }
 
 __device__ __forceinline__ void st_shared_v4(void *p, uint32_t a, uint32_t b, uint32_t c, uint32_t d)
@@ -319,15 +330,27 @@ sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_con
                 };
                 // KV8: lane l copies (and later widens) 16-byte code chunk l % 16 -- K
                 // for l % 16 < 8, V otherwise -- of rows l / 16, l / 16 + 2, ... of
-                // the warp's 32, into staging buffer g % 2; the rows' scales ride one
-                // block ahead in registers (lane i: row rbase + i).
+                // the warp's 32, into staging buffer g % AT_NSTG, three blocks ahead;
+                // lane l also copies row rbase + l's two scales, and lane 0 records the
+                // block's validity word.  The positions run one block and the page ids
+                // one block ahead of the staging.
                 uint8_t *stg = smem + AtSmem::stg_off;
-                int r_cur = 0, r_nx = 0;
-                bool v_cur = false, v_nx = false;
-                float ks_cur = 0.f, vs_cur = 0.f, ks_nx = 0.f, vs_nx = 0.f;
-                auto stage = [&](int gb, int r, bool v) {
+                float *stg_sc = reinterpret_cast<float *>(smem + AtSmem::stg_sc_off);
+                uint32_t *stg_vw = reinterpret_cast<uint32_t *>(smem + AtSmem::stg_vw_off);
+                auto pos_of = [&](int bb) -> int {
+                    const int ee = item.e0 + bb * AT_BLK + rbase + lane;
+                    return (bb < item.nblk && ee < item.e1) ? __ldg(irow + ee) : -1;
+                };
+                auto page_of = [&](int pp) -> int {
+                    return paged && pp >= 0 && pp < ctx ? __ldg(brow + pp / a.page_size) : -1;
+                };
+                auto stage = [&](int gb, int pp, int pg) {
+                    int r;
+                    bool v;
+                    resolve(pp, pg, r, v);
                     const unsigned vb = __ballot_sync(0xffffffffu, v);
-                    uint8_t *sb = stg + (gb & 1) * AtSmem::stg_bytes + rbase * 2 * AT_D + chunk * 16;
+                    const int buf = gb % AT_NSTG;
+                    uint8_t *sb = stg + buf * AtSmem::stg_bytes + rbase * 2 * AT_D + chunk * 16;
                     const uint8_t *src = (chunk < 8 ? a.k8 : a.v8) + (chunk & 7) * 16;
 #pragma unroll
                     for (int j = 0; j < 16; ++j) {
@@ -335,23 +358,32 @@ sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_con
                         const int ri = __shfl_sync(0xffffffffu, r, i);
                         cp_async_16(sb + i * 2 * AT_D, src + (int64_t)ri * AT_D, (vb >> i) & 1u);
                     }
+                    cp_async_4(stg_sc + (buf * 2 + 0) * AT_BLK + rbase + lane, a.ks + r, v);
+                    cp_async_4(stg_sc + (buf * 2 + 1) * AT_BLK + rbase + lane, a.vs + r, v);
+                    if (lane == 0) stg_vw[buf * 2 + (warp - 4)] = vb;
                 };
+                int pnx = -1, pgnx = -1, pnx2 = -1;           // block b + 3's position and page, b + 4's position
                 if constexpr (KV8) {
-                    if (item.nblk > 0 && !stop) {
-                        resolve(p1, pg1, r_cur, v_cur);
-                        stage(g, r_cur, v_cur);
-                        ks_cur = v_cur ? __ldg(a.ks + r_cur) : 0.f;
-                        vs_cur = v_cur ? __ldg(a.vs + r_cur) : 0.f;
+                    for (int bb = 0; bb < AT_NSTG - 1; ++bb) {
+                        if (bb < item.nblk && !stop) {
+                            const int pp = pos_of(bb);
+                            stage(g + bb, pp, page_of(pp));
+                        }
+                        cp_async_commit();
                     }
-                    cp_async_commit();
+                    pnx = pos_of(AT_NSTG - 1);
+                    pgnx = page_of(pnx);
+                    pnx2 = pos_of(AT_NSTG);
                 }
                 for (int b = 0; b < item.nblk && !stop; ++b, ++g) {
                     const int st = g % AT_STAGES;
                     const int p = p1, pg = pg1;
-                    p1 = p2;
-                    pg1 = paged && p1 >= 0 && p1 < ctx ? __ldg(brow + p1 / a.page_size) : -1;
-                    e += AT_BLK;
-                    p2 = (b + 2 < item.nblk && e < item.e1) ? __ldg(irow + e) : -1;
+                    if constexpr (!KV8) {
+                        p1 = p2;
+                        pg1 = paged && p1 >= 0 && p1 < ctx ? __ldg(brow + p1 / a.page_size) : -1;
+                        e += AT_BLK;
+                        p2 = (b + 2 < item.nblk && e < item.e1) ? __ldg(irow + e) : -1;
+                    }
                     // warp-uniform outcome: the ballot and shuffles below need every lane
                     const bool ok = __all_sync(0xffffffffu,
                                                wait_or_abort(&kvempty[st], ((g / AT_STAGES) & 1) ^ 1, &abort_flag));
@@ -374,39 +406,38 @@ sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_con
                         }
                         cp_async_arrive_noinc(&kvfull[st]);   // fires when this thread's copies land
                     } else {
-                        const unsigned vw = __ballot_sync(0xffffffffu, v_cur);
+                        cp_async_wait<AT_NSTG - 2>();     // this lane's copies of block g have landed
+                        __syncwarp();                     // and every lane's (scales, validity word)
+                        const int buf = g % AT_NSTG;
+                        const unsigned vw = stg_vw[buf * 2 + (warp - 4)];
                         if (lane == 0) {
                             valid[st * 2 + (warp - 4)] = vw;
                             mbar_arrive(&kvfull[st]);      // releases the validity bits
                         }
-                        // the next block's codes and scales go out before this block is widened
-                        if (b + 1 < item.nblk) {
-                            resolve(p1, pg1, r_nx, v_nx);
-                            stage(g + 1, r_nx, v_nx);
-                            ks_nx = v_nx ? __ldg(a.ks + r_nx) : 0.f;
-                            vs_nx = v_nx ? __ldg(a.vs + r_nx) : 0.f;
-                        }
-                        cp_async_commit();
-                        cp_async_wait<1>();               // this lane's copies of block g have landed
-                        const uint8_t *sb = stg + (g & 1) * AtSmem::stg_bytes + rbase * 2 * AT_D + chunk * 16;
+                        const uint8_t *sb = stg + buf * AtSmem::stg_bytes + rbase * 2 * AT_D + chunk * 16;
+                        const float *scl = stg_sc + (buf * 2 + (chunk < 8 ? 0 : 1)) * AT_BLK + rbase;
                         uint8_t *tile = KVs + st * AT_STAGE + (chunk < 8 ? 0 : AT_KTILE) + ((chunk & 7) >> 2) * AT_KHALF +
                                         rbase * 128;
                         const int c0 = 2 * (chunk & 7);   // bf16 chunks c0, c0 + 1 of the row
 #pragma unroll 4
                         for (int j = 0; j < 16; ++j) {
                             const int i = 2 * j + (lane >> 4);
-                            const float sk = __shfl_sync(0xffffffffu, ks_cur, i);
-                            const float sv = __shfl_sync(0xffffffffu, vs_cur, i);
                             const uint4 raw = *reinterpret_cast<const uint4 *>(sb + i * 2 * AT_D);
                             uint32_t o[8];
-                            e4m3x16_to_bf16_scaled(raw, chunk < 8 ? sk : sv, o);
+                            e4m3x16_to_bf16_scaled(raw, scl[i], o);
                             uint8_t *row = tile + i * 128;
                             st_shared_v4(row + ((((c0) ^ i) & 7) << 4), o[0], o[1], o[2], o[3]);
                             st_shared_v4(row + ((((c0 + 1) ^ i) & 7) << 4), o[4], o[5], o[6], o[7]);
                         }
                         fence_proxy_async_smem();         // generic writes, read by the tensor cores
                         mbar_arrive(&kvfull[st]);
-                        r_cur = r_nx; v_cur = v_nx; ks_cur = ks_nx; vs_cur = vs_nx;
+                        // refill buffer (g + 3) % AT_NSTG -- block g - 1's, converted last
+                        // iteration -- with block b + 3, and run the lookahead on
+                        if (b + AT_NSTG - 1 < item.nblk) stage(g + AT_NSTG - 1, pnx, pgnx);
+                        cp_async_commit();
+                        pnx = pnx2;
+                        pgnx = page_of(pnx);
+                        pnx2 = pos_of(b + AT_NSTG + 1);
                     }
                     if (pt == 0) kv_issued = g + 1;
                 }
@@ -723,7 +754,7 @@ cudaError_t launch_attn_tc_impl(const CUtensorMap &qmap, const CUtensorMap &kmap
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    const size_t smem = KV8 ? AtSmemKv8::total_kv8 : AtSmemBf16::total;
+    const size_t smem = KV8 ? AtSmemKv8::total_kv8() : AtSmemBf16::total();
     cudaFuncAttributes fa;
     cudaError_t e = cudaFuncGetAttributes(&fa, sparse_attn_tc_kernel<KV8>);
     if (e != cudaSuccess) return e;
