@@ -69,9 +69,11 @@ __device__ __forceinline__ float e4m3_scale_of(float amax)
 __device__ __forceinline__ float e4m3_quotient(float v, float s, float r, bool r_ok)
 {
     const float q = v * r;
-    const uint32_t b = __float_as_uint(q);
-    const int d = (int)(b & 0xFFFFFu) - 0x80000;
-    const bool safe = r_ok && fabsf(q) >= 0.015625f && (d > 4 || d < -4);
+    // near a midpoint: the low 20 bits within 4 of 0x80000, i.e. (low 20 bits of
+    // b - 0x7FFFC) <= 8 (a wrap-around of the low bits only happens next to a
+    // binade boundary, which is no midpoint, and leaves the value large)
+    const bool near = ((__float_as_uint(q) - 0x7FFFCu) & 0xFFFFFu) < 9u;
+    const bool safe = r_ok && fabsf(q) >= 0.015625f && !near;
     return safe ? q : __fdiv_rn(v, s);
 }
 
@@ -153,6 +155,69 @@ quantize_rows_kernel(const In *__restrict__ x, int64_t rows, int cols, uint8_t *
     }
 }
 
+// bf16 rows: each chunk stays packed (four 32-bit words) between the two
+// passes, and the amax is taken on the packed pairs (sign bits cleared, a bf16x2
+// max: exact), which halves the registers a chunk holds and the instructions
+// the reduction costs.  The codes are those of the fp32 path.
+template <int TPR, int NCH>
+__global__ void __launch_bounds__(QZ_THREADS)
+quantize_rows_bf16_kernel(const uint16_t *__restrict__ x, int64_t rows, int cols, uint8_t *__restrict__ codes,
+                          float *__restrict__ scale)
+{
+    constexpr int RPB = QZ_THREADS / TPR;
+    __shared__ float red[QZ_THREADS / 32];
+    const int tid = threadIdx.x, lane = tid & 31;
+    const int sub = tid % TPR;
+    const int nch = cols / QZ_VEC;
+    for (int64_t r0 = (int64_t)blockIdx.x * RPB; r0 < rows; r0 += (int64_t)gridDim.x * RPB) {
+        const int64_t r = r0 + tid / TPR;
+        const bool live = r < rows;                  // uniform per row group
+        uint4 raw[NCH];
+        __nv_bfloat162 m2 = __float2bfloat162_rn(0.f);
+#pragma unroll
+        for (int c = 0; c < NCH; ++c) {
+            const int ch = sub + c * TPR;
+            raw[c] = make_uint4(0u, 0u, 0u, 0u);
+            if (live && ch < nch) raw[c] = __ldg(reinterpret_cast<const uint4 *>(x + r * cols + (int64_t)ch * QZ_VEC));
+            const uint32_t w[4] = {raw[c].x, raw[c].y, raw[c].z, raw[c].w};
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const uint32_t a = w[i] & 0x7fff7fffu;     // |x| of both halves
+                m2 = __hmax2(m2, *reinterpret_cast<const __nv_bfloat162 *>(&a));
+            }
+        }
+        float amax = fmaxf(__low2float(m2), __high2float(m2));
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+        if (TPR > 32) {
+            if (lane == 0) red[tid >> 5] = amax;
+            __syncthreads();
+#pragma unroll
+            for (int w = 0; w < TPR / 32; ++w) amax = fmaxf(amax, red[w]);
+            __syncthreads();                         // red is reused by the next row
+        }
+        const float s = e4m3_scale_of(amax);
+        bool r_ok;
+        const float rs = e4m3_recip(s, r_ok);
+        if (!live) continue;
+        if (sub == 0) scale[r] = s;
+#pragma unroll
+        for (int c = 0; c < NCH; ++c) {
+            const int ch = sub + c * TPR;
+            if (ch < nch) {
+                float v[QZ_VEC];
+                const uint32_t w[4] = {raw[c].x, raw[c].y, raw[c].z, raw[c].w};
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    v[2 * i] = __uint_as_float(w[i] << 16);
+                    v[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+                }
+                *reinterpret_cast<uint2 *>(codes + r * cols + (int64_t)ch * QZ_VEC) = e4m3_codes8(v, s, rs, r_ok);
+            }
+        }
+    }
+}
+
 template <typename In, int TPR, int NCH>
 cudaError_t launch_quantize_t(const In *x, int64_t rows, int cols, uint8_t *codes, float *scale,
                               cudaStream_t st)
@@ -161,12 +226,20 @@ cudaError_t launch_quantize_t(const In *x, int64_t rows, int cols, uint8_t *code
     int dev = 0, sms = 148, per_sm = 4;
     if (cudaGetDevice(&dev) == cudaSuccess)
         cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, quantize_rows_kernel<In, TPR, NCH>, QZ_THREADS, 0);
+    constexpr bool kBf16 = sizeof(In) == 2;
+    if constexpr (kBf16)
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, quantize_rows_bf16_kernel<TPR, NCH>, QZ_THREADS, 0);
+    else
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, quantize_rows_kernel<In, TPR, NCH>, QZ_THREADS, 0);
     if (per_sm < 1) per_sm = 1;
     const int64_t need = ceil_div(rows, RPB);
     const int64_t cap = (int64_t)sms * per_sm;        // persistent: every resident CTA loops over rows
     const unsigned grid = (unsigned)(need < cap ? need : cap);
-    quantize_rows_kernel<In, TPR, NCH><<<grid, QZ_THREADS, 0, st>>>(x, rows, cols, codes, scale);
+    if constexpr (kBf16)
+        quantize_rows_bf16_kernel<TPR, NCH><<<grid, QZ_THREADS, 0, st>>>(reinterpret_cast<const uint16_t *>(x), rows, cols,
+                                                                         codes, scale);
+    else
+        quantize_rows_kernel<In, TPR, NCH><<<grid, QZ_THREADS, 0, st>>>(x, rows, cols, codes, scale);
     return cudaGetLastError();
 }
 
