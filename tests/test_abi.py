@@ -107,3 +107,58 @@ def test_host_argument_errors(lib):
     dargs_bad[12] = 24          # page_size not a multiple of 16
     assert lib.dsa_decode(*dargs_bad, fake, 1 << 30, None) == UNSUP
     assert lib.dsa_stream_status(None, None) == INVALID
+
+
+def test_host_argument_errors_window_quantiser_kv8(lib):
+    """The sliding-window, quantiser, cache-append and FP8 K/V entry points
+    reject bad arguments on the host, before any launch (no GPU needed)."""
+    P = ctypes.c_void_p
+    fake = P(0x1000)            # never dereferenced: every call below fails validation first
+    OK, INVALID, UNSUP, WS = 0, 1, 2, 3
+    # window top-k: negative / too large window, bad k, rows out of range; no rows is a no-op
+    assert lib.dsa_topk_window(fake, 10, 0, 1, 10, 4, -1, fake, None, 0, None) == INVALID
+    assert lib.dsa_topk_window(fake, 10, 0, 1, 10, 4, (1 << 24) + 1, fake, None, 0, None) == INVALID
+    assert lib.dsa_topk_window(fake, 10, 0, 1, 10, 0, 8, fake, None, 0, None) == INVALID
+    assert lib.dsa_topk_window(fake, 10, 8, 3, 10, 4, 8, fake, None, 0, None) == INVALID
+    assert lib.dsa_topk_window(fake, 10, 0, 0, 10, 4, 8, fake, None, 0, None) == OK
+    # prefill / decode with a window: negative window
+    pargs = [fake] * 8 + [1000, 64, 128, 16, 128, 64, -1, 0.1, fake, None, None, 2, fake, 1 << 30, None]
+    assert lib.dsa_prefill_window(*pargs) == INVALID
+    dargs = [fake] * 10 + [100, 4, 64, 2, 256, 64, 128, 128, 128, 64, -1, 0.1, fake, None, None, fake, 1 << 30, None]
+    assert lib.dsa_decode_window(*dargs) == INVALID
+    # FP8 K/V decode: scales required; heads the tensor-core attention cannot take
+    kargs = [fake] * 6 + [fake, None, fake, fake] + [fake, fake, 100, 4, 64, 2, 256, 64, 128, 128, 128, 64, 0,
+                                                      0.1, fake, None, None, fake, 1 << 30, None]
+    assert lib.dsa_decode_kv8(*kargs) == INVALID
+    kargs[7] = fake
+    kargs[19] = 16                                               # H_q
+    assert lib.dsa_decode_kv8(*kargs) == UNSUP
+    kargs[19] = 128
+    kargs[18] = 64                                               # d_I
+    assert lib.dsa_decode_kv8(*kargs) == UNSUP
+    # quantiser: dtype, width, alignment; no rows is a no-op
+    assert lib.dsa_quantize_e4m3(fake, 2, 4, 128, fake, fake, None) == UNSUP         # E4M3 input
+    assert lib.dsa_quantize_e4m3(fake, 1, 4, 12, fake, fake, None) == UNSUP          # cols % 8
+    assert lib.dsa_quantize_e4m3(fake, 1, 4, 16392, fake, fake, None) == UNSUP       # cols > 16384
+    assert lib.dsa_quantize_e4m3(fake, 1, 4, 128, P(0x1004), fake, None) == INVALID  # codes not 8-aligned
+    assert lib.dsa_quantize_e4m3(P(0x1008), 1, 4, 128, fake, fake, None) == INVALID  # x not 16-aligned
+    assert lib.dsa_quantize_e4m3(None, 1, 4, 128, fake, fake, None) == INVALID
+    assert lib.dsa_quantize_e4m3(fake, 1, 0, 128, fake, fake, None) == OK
+    # cache append: nothing to do, null pointers, key width, status alignment, dtype
+    aargs = [fake, 1, fake, fake, fake, fake, 5, 2, fake, 4, 100, 64, 128, 128, fake, fake, fake, fake, None, None]
+    assert lib.dsa_cache_append(*aargs[:6], 0, *aargs[7:]) == OK
+    bad = list(aargs); bad[2] = None
+    assert lib.dsa_cache_append(*bad) == INVALID
+    bad = list(aargs); bad[12] = 264                             # d_I
+    assert lib.dsa_cache_append(*bad) == UNSUP
+    bad = list(aargs); bad[18] = P(0x1002)                       # status
+    assert lib.dsa_cache_append(*bad) == INVALID
+    bad = list(aargs); bad[1] = 2                                # E4M3 keys
+    assert lib.dsa_cache_append(*bad) == UNSUP
+    # FP8 K/V append: the K/V scale caches are required; d up to 256
+    kv = [fake, 1, fake, fake, fake, fake, 5, 2, fake, 4, 100, 64, 128, 128, fake, fake, fake, None, fake, fake,
+          None, None]
+    assert lib.dsa_cache_append_kv8(*kv) == INVALID
+    kv[17] = fake
+    kv[13] = 264                                                 # d
+    assert lib.dsa_cache_append_kv8(*kv) == UNSUP
