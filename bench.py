@@ -425,6 +425,69 @@ def bench_append(dsa, spec, inp, args, flush):
     return dict(us=1e3 * sum(ms) / len(ms), launches=2)
 
 
+def bench_split(args, dsa, spec, shards_n, flush):
+    """The decode of contexts split over `shards_n` devices (dsa_decode_select,
+    dsa_merge_selections, dsa_decode_attend, dsa_merge_partials), the shards
+    run one after another on this GPU: each entry point's device time per
+    shard, the per-rank step (the slowest shard's select and attend plus the
+    two merges; the two all-gathers, which need several GPUs, are not
+    included) and the whole-context dsa_decode of the same input beside it."""
+    from long_context_fp8_b200 import split_decode
+    dev = torch.device("cuda")
+    inp = dsa_synth.make_decode(spec, device=dev)
+    inp.pop("needle_pos")
+    shards = dsa_synth.split_decode_input(inp, shards_n)
+    B, H_q, d, k = spec.B, spec.H_q, spec.d, spec.k
+    sm = 1.0 / math.sqrt(d)
+    maxc = max(int(sh["context_lens"].max()) for sh, _ in shards)
+    ws = dsa.workspace(dsa.split_workspace_size(shards_n, B, maxc, H_q, d, k), dev)
+    _, recv = split_decode.candidate_message(B, k, shards_n, dev)
+    _, precv = split_decode.partial_message(B, H_q, d, shards_n, dev)
+    idx = torch.empty((B, k), dtype=torch.int32, device=dev)
+    out = torch.empty((B, H_q, d), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((B, H_q), dtype=torch.float32, device=dev)
+    steps = max(args.steps, 10)
+
+    def mean_ms(fn):
+        ms = timed_steps(fn, steps, args.warmup, flush)
+        return sum(ms) / len(ms)
+
+    sel_ms, att_ms = [], []
+    for g, (sh, base) in enumerate(shards):
+        pos, score = split_decode.candidate_views(recv[g])
+        sel_ms.append(mean_ms(lambda: dsa.dsa_decode_select(sh, base, k, maxc, cand_pos=pos, cand_score=score,
+                                                            ws=ws)))
+    cpos, cscore = split_decode.candidate_views(recv)
+    mrg_ms = mean_ms(lambda: dsa.dsa_merge_selections(cpos, cscore, idx_out=idx, ws=ws))
+    for g, (sh, base) in enumerate(shards):
+        o, l = split_decode.partial_views(precv[g], B, H_q, d)
+        att_ms.append(mean_ms(lambda: dsa.dsa_decode_attend(sh, base, idx, sm, out=o, lse=l, ws=ws)))
+    po, pl = split_decode.partial_views(precv, B, H_q, d)
+    mp_ms = mean_ms(lambda: dsa.dsa_merge_partials(po, pl, out=out, lse=lse))
+    status = dsa.dsa_stream_status(ws)
+    del shards, ws
+    torch.cuda.empty_cache()
+    wws = dsa.workspace(dsa.decode_workspace_size(B, max(spec.context_lens), H_q, d, k), dev)
+    w_idx = torch.empty_like(idx)
+    whole_ms = mean_ms(lambda: dsa.dsa_decode(inp, k, max(spec.context_lens), sm, idx_out=w_idx, ws=wws))
+    same = bool(torch.equal(w_idx, idx))
+    rank_ms = max(a + b for a, b in zip(sel_ms, att_ms)) + mrg_ms + mp_ms
+    del inp, wws
+    torch.cuda.empty_cache()
+    return {"shards": shards_n, "top_k": k,
+            "workload": f"{B} sequences of {'/'.join(str(c) for c in spec.context_lens)} cached positions, "
+                        f"each cut into {shards_n} contiguous shards",
+            "rank_step_us": round(rank_ms * 1e3, 2), "whole_context_decode_us": round(whole_ms * 1e3, 2),
+            "select_us": [round(x * 1e3, 2) for x in sel_ms],
+            "merge_selections_us": round(mrg_ms * 1e3, 2),
+            "attend_us": [round(x * 1e3, 2) for x in att_ms],
+            "merge_partials_us": round(mp_ms * 1e3, 2),
+            "message_bytes": {"candidates": shards_n * B * k * 8,
+                              "partials": shards_n * 4 * split_decode.partial_words(B, H_q, d)},
+            "selection_equals_whole_context": same, "device_status": status,
+            "note": "shards timed one after another on one GPU; the two all-gathers are not included"}
+
+
 def bench_quantize(args, dsa, spec, peaks):
     """FP8 quantisation of the prefill's index query [T, H_I * d_I] and key
     [T, d_I] from bf16 (dsa_quantize_e4m3, one scale per token): HBM-bound,
@@ -543,6 +606,11 @@ def main():
                     help="profiling aid: time only the FP8 quantiser on the workload's index query/key")
     ap.add_argument("--no-extras", action="store_true",
                     help="skip the quantiser, cache-append and sliding-window decode lines")
+    ap.add_argument("--split-shards", type=int, default=8,
+                    help="shards of the ragged long-context decode for the split-context measurement "
+                         "(0: skip it)")
+    ap.add_argument("--split-only", action="store_true",
+                    help="only the split-context decode measurement")
     ap.add_argument("--window", type=int, default=8192,
                     help="sliding window of the extra decode line (the pages' 8K example)")
     args = ap.parse_args()
@@ -597,6 +665,18 @@ def main():
             torch.distributed.barrier()
             torch.distributed.destroy_process_group()
         return
+    if args.split_only:
+        flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device="cuda")
+        r = bench_split(args, dsa, dsa_synth.decode_spec("dec_ragged"), max(args.split_shards, 1), flush)
+        if rank == 0:
+            print(json.dumps({"metric": "split-context decode, per-rank device time", "value": r["rank_step_us"],
+                              "unit": "us", "n_gpus": ws_n, "steps": args.steps, "warmup": args.warmup,
+                              "higher_is_better": False, "config": {"workload": "dec_ragged split"},
+                              "decode_split": r}), flush=True)
+        if ws_n > 1:
+            torch.distributed.barrier()
+            torch.distributed.destroy_process_group()
+        return
     if args.decode_only:
         dec = bench_decode(args, dsa, dspec, peaks, ws_n, rank, kv8=args.kv8)
         us = dec["step_ms"] * 1e3
@@ -626,6 +706,11 @@ def main():
     if extras and not args.no_decode:
         deck = bench_decode(args, dsa, dspec, peaks, ws_n, rank, kv8=True)
     quant = bench_quantize(args, dsa, spec, peaks) if extras else None
+    split = None
+    if extras and not args.no_decode and args.split_shards > 0:
+        flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device="cuda")
+        split = bench_split(args, dsa, dsa_synth.decode_spec("dec_ragged"), args.split_shards, flush)
+        del flush
 
     T = spec.L
     value = whole_job_rate(ws_n, T, pre["step_ms"])
@@ -697,6 +782,8 @@ def main():
                               "device_status": deck["status"]}
     if quant:
         line["quantize"] = quant
+    if split:
+        line["decode_split"] = split
     if rank == 0 and ws_n == 1 and not args.no_cpu:
         os.environ.setdefault("OMP_NUM_THREADS", str(oracle_threads()))
         inp_cpu = cpu_inputs_for(spec)

@@ -295,3 +295,49 @@ def decode_kv_to_fp8(inp: Dict[str, torch.Tensor]) -> Dict[str, torch.Tensor]:
         out[name + "_cache"] = codes.reshape(P, ps, d).contiguous()
         out[name + "_cache_scale"] = scale.reshape(P, ps).contiguous()
     return out
+
+
+def split_decode_input(inp: Dict[str, torch.Tensor], G: int):
+    """Cut a decode input's caches into G contiguous shards of every sequence's
+    positions (shard g of a context of n positions: [floor(g n / G),
+    floor((g + 1) n / G))), each shard in paged caches of its own, the pages
+    in reverse order so that paging is exercised.  Returns a list of
+    (shard dict, pos_base int32 [B]); queries are shared.  Only re-packs
+    cache rows."""
+    dev = inp["q"].device
+    ps = inp["kidx_cache"].shape[1]
+    lens = inp["context_lens"].cpu().long()
+    B = lens.numel()
+    bt = inp["block_table"].cpu().long()
+    g_ = torch.arange(G + 1, dtype=torch.int64)[:, None]
+    edges = (g_ * lens[None, :]) // G
+    cache_keys = [k for k in ("kidx_cache", "kscale_cache", "k_cache", "v_cache", "k_cache_scale",
+                              "v_cache_scale") if k in inp]
+    flat = {k: inp[k].reshape((-1,) + tuple(inp[k].shape[2:])) for k in cache_keys}
+    shards = []
+    for g in range(G):
+        base, n = edges[g], edges[g + 1] - edges[g]
+        pages = [(int(x) + ps - 1) // ps for x in n]
+        P = max(sum(pages), 1)
+        order = torch.arange(P - 1, -1, -1, dtype=torch.int64)
+        table = torch.full((B, max(max(pages), 1)), -1, dtype=torch.int32)
+        sh = {k: inp[k] for k in ("q_idx", "q_scale", "w", "q")}
+        for k in cache_keys:
+            fill = 1 if "scale" in k else 0
+            sh[k] = torch.full((P * ps,) + tuple(inp[k].shape[2:]), fill, dtype=inp[k].dtype, device=dev)
+        off = 0
+        for b in range(B):
+            table[b, :pages[b]] = order[off:off + pages[b]].int()
+            p = torch.arange(int(base[b]), int(base[b] + n[b]), dtype=torch.int64)
+            src = bt[b, p // ps] * ps + p % ps
+            local = torch.arange(int(n[b]), dtype=torch.int64)
+            dst = table[b].long()[local // ps] * ps + local % ps
+            for k in cache_keys:
+                sh[k][dst.to(dev)] = flat[k][src.to(dev)]
+            off += pages[b]
+        for k in cache_keys:
+            sh[k] = sh[k].view((P, ps) + tuple(inp[k].shape[2:]))
+        sh["block_table"] = table.to(dev)
+        sh["context_lens"] = n.to(torch.int32).to(dev)
+        shards.append((sh, base.to(torch.int32).to(dev)))
+    return shards

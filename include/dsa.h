@@ -273,6 +273,94 @@ dsa_status dsa_decode_kv8(const void *q_idx, const float *q_scale, const void *w
                           float *lse_out, int32_t *idx_out, void *workspace, size_t ws_bytes, void *stream);
 
 /*
+ * Decode of one context split over G devices.  The pages' decode step
+ * (indexer, top-k, attention over the selected rows; the 1M-context setting of
+ * "DeepSeek V4 ... 稀疏注意力" on hotdry) is computed exactly when the cached
+ * positions of every sequence are cut into G contiguous shards, shard g
+ * holding positions [pos_base_g[b], pos_base_g[b] + context_lens_g[b]) in its
+ * own paged caches at local positions 0.. context_lens_g[b]-1, shards in
+ * position order:
+ *   1. dsa_decode_select on every shard: its indexer scores and its own top-k
+ *      (k_sel) as GLOBAL positions with their scores.  Every member of the
+ *      global top-k is in its shard's top-k, so the union holds it.
+ *   2. the G candidate lists are gathered (an all-gather of G*B*k_sel*8 bytes)
+ *      into cand_pos [G, B, k_sel] / cand_score [G, B, k_sel], shard order.
+ *   3. dsa_merge_selections on every device: the exact top-k of the union,
+ *      ties toward the lower position -- the selection dsa_decode makes over
+ *      the whole context, bit for bit.
+ *   4. dsa_decode_attend on every shard: attention over the selected positions
+ *      that shard holds, giving a partial bf16 output and its log-sum-exp
+ *      (-inf and zeros when the shard holds none of them).
+ *   5. the G partials are gathered into [G, B, H_q, d] / [G, B, H_q] and
+ *      dsa_merge_partials combines them:
+ *        lse = log sum_g exp(lse_g),  out = sum_g exp(lse_g - lse) * out_g.
+ * Every shard must hold at least one position of every sequence
+ * (context_lens_g[b] >= 1); a zero length is reported as DSA_ERR_INVALID_ARG
+ * through dsa_stream_status, as in dsa_decode.
+ * One workspace of dsa_split_workspace_size(G, B, max_context, H_q, d, k_sel)
+ * bytes (max_context: the largest shard length) serves all four calls.
+ */
+size_t dsa_split_workspace_size(int G, int B, int64_t max_context, int H_q, int d, int k_sel);
+
+/*
+ * dsa_decode_select -- step 1 on one shard.  Inputs as dsa_decode's indexer
+ * half (q_idx, q_scale, w, kidx_cache, kscale_cache, block_table,
+ * context_lens, ... with the shard's local lengths, max_context the largest);
+ * pos_base int32 [B]: the global position of each sequence's first position
+ * on this shard.  Outputs cand_pos_out int32 [B, k_sel]: the shard's top-k as
+ * global positions, ascending, -1 padded; cand_score_out f32 [B, k_sel]:
+ * their indexer scores (-inf for -1).  A negative base or a global position
+ * past INT32_MAX is reported through dsa_stream_status.  Supported as
+ * dsa_decode.
+ */
+dsa_status dsa_decode_select(const void *q_idx, const float *q_scale, const void *w, const void *kidx_cache,
+                             const float *kscale_cache, const int32_t *block_table, const int32_t *context_lens,
+                             const int32_t *pos_base, int64_t num_pages, int max_pages_per_seq, int page_size,
+                             int B, int64_t max_context, int H_I, int d_I, int k_sel, int32_t *cand_pos_out,
+                             float *cand_score_out, void *workspace, size_t ws_bytes, void *stream);
+
+/*
+ * dsa_merge_selections -- step 3.  G candidate lists as dsa_decode_select
+ * wrote them, list g from shard g: positions int32 [B, k_sel] at
+ * cand_pos + g * list_stride and scores f32 [B, k_sel] at
+ * cand_score + g * list_stride (elements; 0 means B * k_sel, i.e. dense
+ * [G, B, k_sel] arrays).  A stride lets one all-gathered buffer of
+ * [G][positions | scores] serve both.  idx_out int32 [B, k_sel]: the k_sel
+ * best positions of the union (score descending, ties to the lower
+ * position), ascending, -1 padded.  Entries with position -1 never win.
+ */
+dsa_status dsa_merge_selections(const int32_t *cand_pos, const float *cand_score, int64_t list_stride, int G,
+                                int B, int k_sel, int32_t *idx_out, void *workspace, size_t ws_bytes, void *stream);
+
+/*
+ * dsa_decode_attend -- step 4 on one shard.  q bf16 [B, H_q, d]; the shard's
+ * caches, block_table, context_lens and pos_base as in dsa_decode_select;
+ * k_cache_scale / v_cache_scale NULL for bf16 K/V, or both given for FP8
+ * E4M3 K/V as in dsa_decode_kv8; idx int32 [B, k_sel]: the merged global
+ * selection.  Positions outside this shard are skipped.  Outputs out bf16
+ * [B, H_q, d] and lse_out f32 [B, H_q] (required): the attention over this
+ * shard's part of the selection.  Supported as dsa_decode (FP8: as
+ * dsa_decode_kv8).
+ */
+dsa_status dsa_decode_attend(const void *q, const void *k_cache, const float *k_cache_scale, const void *v_cache,
+                             const float *v_cache_scale, const int32_t *block_table, const int32_t *context_lens,
+                             const int32_t *pos_base, int64_t num_pages, int max_pages_per_seq, int page_size, int B,
+                             int H_q, int d, int k_sel, const int32_t *idx, float sm_scale, void *out,
+                             float *lse_out, void *workspace, size_t ws_bytes, void *stream);
+
+/*
+ * dsa_merge_partials -- step 5.  Partial g: out bf16 [B, H_q, d] at
+ * part_out + g * out_stride and lse f32 [B, H_q] at part_lse + g * lse_stride
+ * (elements of each type; 0 means dense [G, B, H_q, d] / [G, B, H_q]; a stride
+ * lets one all-gathered buffer of [G][out | lse] serve both; out_stride a
+ * multiple of 8).  out bf16 [B, H_q, d], lse_out f32 [B, H_q] (nullable).  A
+ * head whose every partial has lse -inf gets zeros and -inf.  d == 128.
+ * Needs no workspace; device errors are CUDA launch errors only.
+ */
+dsa_status dsa_merge_partials(const void *part_out, int64_t out_stride, const float *part_lse, int64_t lse_stride,
+                              int G, int B, int H_q, int d, void *out, float *lse_out, void *stream);
+
+/*
  * dsa_quantize_e4m3 -- FP8 E4M3 quantisation with one fp32 scale per row, the
  * storage of the indexer's query and key ("DeepSeek-V3.2-Exp DSA 技术深度解析",
  * section 1: FP8 indexer; the DeepSeek-V4 engineering page's FP8 decoding

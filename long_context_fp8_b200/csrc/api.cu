@@ -440,6 +440,72 @@ size_t dsa_decode_workspace_size(int B, int64_t max_context, int H_q, int d, int
 
 namespace {
 
+// The decode indexer's scores [B, max_context] and each row's top-k (plus the
+// window) into idx [B, k_sel + window].
+cudaError_t run_decode_select(const void *q_idx, const float *q_scale, const void *w, const void *kidx_cache,
+                              const float *kscale_cache, const int32_t *block_table, const int32_t *context_lens,
+                              int64_t num_pages, int max_pages_per_seq, int page_size, int B,
+                              int64_t max_context, int H_I, int k_sel, int window, float *scores, int32_t *idx,
+                              void *topk_ws, WsHeader *hdr, cudaStream_t st)
+{
+    cudaError_t e;
+    // tensor-core (tcgen05 + TMA) indexer where the shape allows, else mma.sync
+    if (decode_index_tc_supported(H_I, page_size) && B <= 4096 &&
+        (int64_t)num_pages * page_size < ((int64_t)1 << 31) && aligned16(kscale_cache))
+        e = launch_decode_index_tc((const uint8_t *)q_idx, q_scale, (const uint16_t *)w,
+                                   (const uint8_t *)kidx_cache, kscale_cache, block_table, context_lens,
+                                   num_pages, max_pages_per_seq, page_size, B, max_context, H_I, scores,
+                                   max_context, hdr, st);
+    else
+        e = launch_decode_index((const uint8_t *)q_idx, q_scale, (const uint16_t *)w,
+                                (const uint8_t *)kidx_cache, kscale_cache, block_table, context_lens,
+                                num_pages, max_pages_per_seq, page_size, B, max_context, H_I, scores,
+                                max_context, hdr, st);
+    if (e == cudaSuccess)   // each row split over 16K-position chunks (CTAs), then one CTA per row
+        e = launch_topk_split(scores, max_context, context_lens, max_context, B, k_sel, idx, topk_ws, hdr, st,
+                              window);
+    return e;
+}
+
+// The paged attention of B single-token queries over idx [B, kw] (tcgen05
+// kernel where the shape allows, else the mma.sync one; FP8 K/V when
+// k_cache_scale is given), split over the index list and merged.
+cudaError_t run_decode_attend(const void *q, const void *k_cache, const void *v_cache, const float *k_cache_scale,
+                              const float *v_cache_scale, const int32_t *block_table, const int32_t *context_lens,
+                              int64_t num_pages, int max_pages_per_seq, int page_size, int B, int H_q, int d,
+                              int kw, float sm_scale, const int32_t *idx, void *out, float *lse_out, float *part,
+                              WsHeader *hdr, cudaStream_t st)
+{
+    const int splits = sparse_attn_paged_splits(B, kw);
+    const int chunk = (int)(ceil_div(ceil_div(kw, splits), 128) * 128);
+    const int tc_splits = (int)ceil_div(kw, chunk);
+    cudaError_t e;
+    if (k_cache_scale) {
+        // tcgen05 kernel over the FP8 caches, the index list split in 128-row blocks
+        if ((int64_t)num_pages * page_size >= ((int64_t)1 << 31)) return cudaErrorNotSupported;
+        e = launch_sparse_attn_tc_kv8((const uint16_t *)q, (const uint8_t *)k_cache, k_cache_scale,
+                                      (const uint8_t *)v_cache, v_cache_scale, num_pages * page_size, block_table,
+                                      context_lens, num_pages, max_pages_per_seq, page_size, idx, B, H_q, d, kw,
+                                      sm_scale, (uint16_t *)out, lse_out, part, tc_splits, hdr, st,
+                                      /*chained=*/true);
+        if (e == cudaSuccess) e = launch_merge_splits(part, B, tc_splits, H_q, d, (uint16_t *)out, lse_out, st);
+        return e;
+    }
+    if (sparse_attn_tc_supported(H_q, d) && (int64_t)num_pages * page_size < ((int64_t)1 << 31)) {
+        // tcgen05 kernel over the paged caches, the index list split in 128-row blocks
+        e = launch_sparse_attn_tc((const uint16_t *)q, (const uint16_t *)k_cache, (const uint16_t *)v_cache,
+                                  num_pages * page_size, 0, block_table, context_lens, num_pages,
+                                  max_pages_per_seq, page_size, idx, B, H_q, d, kw, sm_scale, (uint16_t *)out,
+                                  lse_out, part, tc_splits, hdr, st, /*chained=*/true);
+        if (e == cudaSuccess) e = launch_merge_splits(part, B, tc_splits, H_q, d, (uint16_t *)out, lse_out, st);
+        if (e != cudaErrorNotSupported) return e;
+    }
+    PagedKV kv{(const uint16_t *)k_cache, (const uint16_t *)v_cache, block_table, context_lens,
+               num_pages, max_pages_per_seq, page_size};
+    return launch_sparse_attn_paged_bf16((const uint16_t *)q, kv, idx, B, H_q, d, kw, sm_scale, (uint16_t *)out,
+                                         lse_out, part, splits, hdr, st);
+}
+
 // dsa_decode with a sliding window of `window` positions (0: none); the
 // selection rows (and the attention's index lists) are k_sel + window wide.
 // k_cache_scale / v_cache_scale non-null: the K/V caches hold E4M3 codes with
@@ -488,60 +554,17 @@ dsa_status decode_impl(const void *q_idx, const float *q_scale, const void *w, c
     off += align_up(sparse_attn_paged_part_bytes(B, H_q, d, sparse_attn_paged_splits(B, kw)), 256);
     void *topk_ws = ws + off;
     if (idx_out) idx = idx_out;
-    const int splits = sparse_attn_paged_splits(B, kw);
 
     cudaError_t e = cudaMemsetAsync(hdr, 0, sizeof(WsHeader), st);
+    if (e == cudaSuccess)
+        e = run_decode_select(q_idx, q_scale, w, kidx_cache, kscale_cache, block_table, context_lens, num_pages,
+                              max_pages_per_seq, page_size, B, max_context, H_I, k_sel, window, scores, idx,
+                              topk_ws, hdr, st);
     if (e == cudaSuccess) {
-        // tensor-core (tcgen05 + TMA) indexer where the shape allows, else mma.sync
-        if (decode_index_tc_supported(H_I, page_size) && B <= 4096 &&
-            (int64_t)num_pages * page_size < ((int64_t)1 << 31) && aligned16(kscale_cache))
-            e = launch_decode_index_tc((const uint8_t *)q_idx, q_scale, (const uint16_t *)w,
-                                       (const uint8_t *)kidx_cache, kscale_cache, block_table,
-                                       context_lens, num_pages, max_pages_per_seq, page_size, B,
-                                       max_context, H_I, scores, max_context, hdr, st);
-        else
-            e = launch_decode_index((const uint8_t *)q_idx, q_scale, (const uint16_t *)w,
-                                    (const uint8_t *)kidx_cache, kscale_cache, block_table,
-                                    context_lens, num_pages, max_pages_per_seq, page_size, B,
-                                    max_context, H_I, scores, max_context, hdr, st);
-    }
-    if (e == cudaSuccess)   // each row split over 16K-position chunks (CTAs), then one CTA per row
-        e = launch_topk_split(scores, max_context, context_lens, max_context, B, k_sel, idx, topk_ws,
-                              hdr, st, window);
-    if (e == cudaSuccess && kv8) {
-        // tcgen05 kernel over the FP8 caches, the index list split in 128-row blocks
-        if ((int64_t)num_pages * page_size >= ((int64_t)1 << 31)) return DSA_ERR_UNSUPPORTED;
-        const int chunk = (int)(ceil_div(ceil_div(kw, splits), 128) * 128);
-        const int tc_splits = (int)ceil_div(kw, chunk);
-        e = launch_sparse_attn_tc_kv8((const uint16_t *)q, (const uint8_t *)k_cache, k_cache_scale,
-                                      (const uint8_t *)v_cache, v_cache_scale, num_pages * page_size,
-                                      block_table, context_lens, num_pages, max_pages_per_seq, page_size, idx,
-                                      B, H_q, d, kw, sm_scale, (uint16_t *)out, lse_out, part, tc_splits, hdr,
-                                      st, /*chained=*/true);
+        e = run_decode_attend(q, k_cache, v_cache, k_cache_scale, v_cache_scale, block_table, context_lens,
+                              num_pages, max_pages_per_seq, page_size, B, H_q, d, kw, sm_scale, idx, out, lse_out,
+                              part, hdr, st);
         if (e == cudaErrorNotSupported) return DSA_ERR_UNSUPPORTED;
-        if (e == cudaSuccess) e = launch_merge_splits(part, B, tc_splits, H_q, d, (uint16_t *)out, lse_out, st);
-        return cuda_status(e);
-    }
-    if (e == cudaSuccess) {
-        bool done = false;
-        if (sparse_attn_tc_supported(H_q, d) && (int64_t)num_pages * page_size < ((int64_t)1 << 31)) {
-            // tcgen05 kernel over the paged caches, the index list split in 128-row blocks
-            const int chunk = (int)(ceil_div(ceil_div(kw, splits), 128) * 128);
-            const int tc_splits = (int)ceil_div(kw, chunk);
-            e = launch_sparse_attn_tc((const uint16_t *)q, (const uint16_t *)k_cache,
-                                      (const uint16_t *)v_cache, num_pages * page_size, 0,
-                                      block_table, context_lens, num_pages, max_pages_per_seq,
-                                      page_size, idx, B, H_q, d, kw, sm_scale, (uint16_t *)out,
-                                      lse_out, part, tc_splits, hdr, st, /*chained=*/true);
-            if (e == cudaSuccess) e = launch_merge_splits(part, B, tc_splits, H_q, d, (uint16_t *)out, lse_out, st);
-            done = e != cudaErrorNotSupported;
-        }
-        if (!done) {
-            PagedKV kv{(const uint16_t *)k_cache, (const uint16_t *)v_cache, block_table, context_lens,
-                       num_pages, max_pages_per_seq, page_size};
-            e = launch_sparse_attn_paged_bf16((const uint16_t *)q, kv, idx, B, H_q, d, kw, sm_scale,
-                                              (uint16_t *)out, lse_out, part, splits, hdr, st);
-        }
     }
     return cuda_status(e);
 }
@@ -590,6 +613,133 @@ dsa_status dsa_decode_kv8(const void *q_idx, const float *q_scale, const void *w
                        context_lens, num_pages, max_pages_per_seq, page_size, B, max_context, H_I, d_I,
                        H_q, d, k_sel, window, sm_scale, out, lse_out, idx_out, workspace, ws_bytes,
                        stream, k_cache_scale, v_cache_scale);
+}
+
+size_t dsa_split_workspace_size(int G, int B, int64_t max_context, int H_q, int d, int k_sel)
+{
+    if (G <= 0 || B <= 0 || max_context <= 0 || H_q <= 0 || d <= 0 || k_sel <= 0) return 0;
+    const size_t select = align_up(sizeof(float) * (size_t)B * max_context, 256) + idx_bytes(B, k_sel) +
+                          align_up(topk_split_ws_bytes(B, max_context), 256);
+    const size_t attend = idx_bytes(B, k_sel) +
+                          align_up(sparse_attn_paged_part_bytes(B, H_q, d, sparse_attn_paged_splits(B, k_sel)), 256);
+    const size_t merge = align_up(merge_selections_ws_bytes(B, G, k_sel), 256);
+    size_t m = select > attend ? select : attend;
+    m = m > merge ? m : merge;
+    return kWsHeader + m;
+}
+
+dsa_status dsa_decode_select(const void *q_idx, const float *q_scale, const void *w, const void *kidx_cache,
+                             const float *kscale_cache, const int32_t *block_table, const int32_t *context_lens,
+                             const int32_t *pos_base, int64_t num_pages, int max_pages_per_seq, int page_size,
+                             int B, int64_t max_context, int H_I, int d_I, int k_sel, int32_t *cand_pos_out,
+                             float *cand_score_out, void *workspace, size_t ws_bytes, void *stream)
+{
+    if (!q_idx || !q_scale || !w || !kidx_cache || !kscale_cache || !block_table || !context_lens || !pos_base ||
+        !cand_pos_out || !cand_score_out)
+        return DSA_ERR_INVALID_ARG;
+    if (B <= 0 || max_context <= 0 || max_context > INT32_MAX || num_pages <= 0 || max_pages_per_seq <= 0 ||
+        page_size <= 0 || H_I <= 0 || k_sel <= 0 || k_sel > 65536)
+        return DSA_ERR_INVALID_ARG;
+    if (!aligned16(q_idx) || !aligned16(kidx_cache)) return DSA_ERR_INVALID_ARG;
+    if (d_I != 128 || H_I > 64 || H_I % 8 != 0 || page_size % 16 != 0) return DSA_ERR_UNSUPPORTED;
+    if (B > 65535) return DSA_ERR_UNSUPPORTED;
+    if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u)) return DSA_ERR_WORKSPACE;
+    const size_t need = kWsHeader + align_up(sizeof(float) * (size_t)B * max_context, 256) + idx_bytes(B, k_sel) +
+                        align_up(topk_split_ws_bytes(B, max_context), 256);
+    if (ws_bytes < need) return DSA_ERR_WORKSPACE;
+
+    cudaStream_t st = as_stream(stream);
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    WsHeader *hdr = reinterpret_cast<WsHeader *>(ws);
+    size_t off = kWsHeader;
+    float *scores = reinterpret_cast<float *>(ws + off);
+    off += align_up(sizeof(float) * (size_t)B * max_context, 256);
+    int32_t *idx_local = reinterpret_cast<int32_t *>(ws + off);
+    off += idx_bytes(B, k_sel);
+    cudaError_t e = cudaMemsetAsync(hdr, 0, sizeof(WsHeader), st);
+    if (e == cudaSuccess)
+        e = run_decode_select(q_idx, q_scale, w, kidx_cache, kscale_cache, block_table, context_lens, num_pages,
+                              max_pages_per_seq, page_size, B, max_context, H_I, k_sel, 0, scores, idx_local,
+                              ws + off, hdr, st);
+    if (e == cudaSuccess)
+        e = launch_gather_selected(scores, max_context, idx_local, pos_base, B, k_sel, cand_pos_out, cand_score_out,
+                                   hdr, st);
+    return cuda_status(e);
+}
+
+dsa_status dsa_merge_selections(const int32_t *cand_pos, const float *cand_score, int64_t list_stride, int G,
+                                int B, int k_sel, int32_t *idx_out, void *workspace, size_t ws_bytes, void *stream)
+{
+    if (!cand_pos || !cand_score || !idx_out || G <= 0 || B <= 0 || k_sel <= 0 || k_sel > 65536)
+        return DSA_ERR_INVALID_ARG;
+    if (list_stride == 0) list_stride = (int64_t)B * k_sel;
+    if (list_stride < (int64_t)B * k_sel && G > 1) return DSA_ERR_INVALID_ARG;
+    if ((int64_t)G * k_sel > INT32_MAX / 2) return DSA_ERR_UNSUPPORTED;
+    if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u)) return DSA_ERR_WORKSPACE;
+    if (ws_bytes < kWsHeader + align_up(merge_selections_ws_bytes(B, G, k_sel), 256)) return DSA_ERR_WORKSPACE;
+    cudaStream_t st = as_stream(stream);
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    WsHeader *hdr = reinterpret_cast<WsHeader *>(ws);
+    cudaError_t e = cudaMemsetAsync(hdr, 0, sizeof(WsHeader), st);
+    if (e == cudaSuccess)
+        e = launch_merge_selections(cand_pos, cand_score, list_stride, B, G, k_sel, idx_out, ws + kWsHeader, hdr,
+                                    st);
+    return cuda_status(e);
+}
+
+dsa_status dsa_decode_attend(const void *q, const void *k_cache, const float *k_cache_scale, const void *v_cache,
+                             const float *v_cache_scale, const int32_t *block_table, const int32_t *context_lens,
+                             const int32_t *pos_base, int64_t num_pages, int max_pages_per_seq, int page_size, int B,
+                             int H_q, int d, int k_sel, const int32_t *idx, float sm_scale, void *out,
+                             float *lse_out, void *workspace, size_t ws_bytes, void *stream)
+{
+    const bool kv8 = k_cache_scale != nullptr;
+    if (kv8 != (v_cache_scale != nullptr)) return DSA_ERR_INVALID_ARG;
+    if (kv8 && ((reinterpret_cast<uintptr_t>(k_cache_scale) & 3u) || (reinterpret_cast<uintptr_t>(v_cache_scale) & 3u)))
+        return DSA_ERR_INVALID_ARG;
+    if (!q || !k_cache || !v_cache || !block_table || !context_lens || !pos_base || !idx || !out || !lse_out)
+        return DSA_ERR_INVALID_ARG;
+    if (B <= 0 || num_pages <= 0 || max_pages_per_seq <= 0 || page_size <= 0 || H_q <= 0 || k_sel <= 0 ||
+        k_sel > 65536 || !std::isfinite(sm_scale))
+        return DSA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out)) return DSA_ERR_INVALID_ARG;
+    if (d != 128 || page_size % 16 != 0 || B > 65535) return DSA_ERR_UNSUPPORTED;
+    if (H_q > 128 && H_q % 128 != 0) return DSA_ERR_UNSUPPORTED;
+    if (kv8 && !sparse_attn_tc_supported(H_q, d)) return DSA_ERR_UNSUPPORTED;
+    if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u)) return DSA_ERR_WORKSPACE;
+    const size_t part_bytes = sparse_attn_paged_part_bytes(B, H_q, d, sparse_attn_paged_splits(B, k_sel));
+    if (ws_bytes < kWsHeader + idx_bytes(B, k_sel) + align_up(part_bytes, 256)) return DSA_ERR_WORKSPACE;
+
+    cudaStream_t st = as_stream(stream);
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    WsHeader *hdr = reinterpret_cast<WsHeader *>(ws);
+    int32_t *idx_local = reinterpret_cast<int32_t *>(ws + kWsHeader);
+    float *part = reinterpret_cast<float *>(ws + kWsHeader + idx_bytes(B, k_sel));
+    cudaError_t e = cudaMemsetAsync(hdr, 0, sizeof(WsHeader), st);
+    if (e == cudaSuccess) e = launch_local_idx(idx, pos_base, context_lens, B, k_sel, idx_local, st);
+    if (e == cudaSuccess) {
+        e = run_decode_attend(q, k_cache, v_cache, k_cache_scale, v_cache_scale, block_table, context_lens,
+                              num_pages, max_pages_per_seq, page_size, B, H_q, d, k_sel, sm_scale, idx_local, out,
+                              lse_out, part, hdr, st);
+        if (e == cudaErrorNotSupported) return DSA_ERR_UNSUPPORTED;
+    }
+    return cuda_status(e);
+}
+
+dsa_status dsa_merge_partials(const void *part_out, int64_t out_stride, const float *part_lse, int64_t lse_stride,
+                              int G, int B, int H_q, int d, void *out, float *lse_out, void *stream)
+{
+    if (!part_out || !part_lse || !out || G <= 0 || B <= 0 || H_q <= 0) return DSA_ERR_INVALID_ARG;
+    if (!aligned16(part_out) || !aligned16(out) || (reinterpret_cast<uintptr_t>(part_lse) & 3u))
+        return DSA_ERR_INVALID_ARG;
+    if (d != 128 || (int64_t)ceil_div(H_q, 8) > 65535) return DSA_ERR_UNSUPPORTED;
+    const int64_t n_out = (int64_t)B * H_q * d, n_lse = (int64_t)B * H_q;
+    if (out_stride == 0) out_stride = n_out;
+    if (lse_stride == 0) lse_stride = n_lse;
+    if (G > 1 && (out_stride < n_out || lse_stride < n_lse)) return DSA_ERR_INVALID_ARG;
+    if (out_stride % 8 != 0) return DSA_ERR_INVALID_ARG;          // keeps every partial 16-byte aligned
+    return cuda_status(launch_merge_partials((const uint16_t *)part_out, out_stride, part_lse, lse_stride, G, B, H_q,
+                                             d, (uint16_t *)out, lse_out, as_stream(stream)));
 }
 
 dsa_status dsa_quantize_e4m3(const void *x, dsa_dtype x_dtype, int64_t rows, int64_t cols,

@@ -127,4 +127,24 @@ cudaError_t launch_decode_index(const uint8_t *q8, const float *sq, const uint16
                                 int64_t max_context, int H, float *scores, int64_t ld,
                                 WsHeader *hdr, cudaStream_t st);
 
+// ---- context split over devices (split.cu) ----
+// Shard-local selections [B, k] -> global positions (+ base[b]) and their scores.
+cudaError_t launch_gather_selected(const float *scores, int64_t ld, const int32_t *idx_local, const int32_t *base,
+                                   int B, int k, int32_t *idx_out, float *score_out, WsHeader *hdr,
+                                   cudaStream_t st);
+// Exact top-k of the union of G candidate lists [B, k] (list g at g * stride
+// elements; positions ascending within a list, lists in position order),
+// positions out [B, k].
+size_t merge_selections_ws_bytes(int B, int G, int k);
+cudaError_t launch_merge_selections(const int32_t *cand_pos, const float *cand_score, int64_t stride, int B, int G,
+                                    int k, int32_t *idx_out, void *ws, WsHeader *hdr, cudaStream_t st);
+// Global positions -> this shard's positions [base[b], base[b] + lens[b]) - base[b], else -1.
+cudaError_t launch_local_idx(const int32_t *idx, const int32_t *base, const int32_t *lens, int B, int k,
+                             int32_t *idx_local, cudaStream_t st);
+// Log-sum-exp merge of G partial attentions (bf16 [B, H, d] and f32 [B, H]
+// each, partial g at g * out_stride / g * lse_stride elements); d == 128.
+cudaError_t launch_merge_partials(const uint16_t *part_out, int64_t out_stride, const float *part_lse,
+                                  int64_t lse_stride, int G, int B, int H, int d, uint16_t *out, float *lse,
+                                  cudaStream_t st);
+
 }  // namespace dsa

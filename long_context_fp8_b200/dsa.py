@@ -28,7 +28,8 @@ EXPORTS = ("dsa_status_string", "dsa_version", "dsa_index_scores", "dsa_topk_wor
            "dsa_prefill", "dsa_prefill_window", "dsa_prefill_host_workspace_size", "dsa_prefill_host",
            "dsa_decode_workspace_size", "dsa_decode", "dsa_decode_window", "dsa_decode_kv8",
            "dsa_quantize_e4m3", "dsa_cache_append", "dsa_cache_append_kv8", "dsa_decode_noalloc",
-           "dsa_stream_status")
+           "dsa_split_workspace_size", "dsa_decode_select", "dsa_merge_selections", "dsa_decode_attend",
+           "dsa_merge_partials", "dsa_stream_status")
 
 
 class DSAError(RuntimeError):
@@ -81,6 +82,13 @@ def load(path: str = LIB_PATH):
                                   P, P], I32),
         "dsa_cache_append": ([P, I32, P, P, P, P, I64, I32, P, I32, I64, I32, I32, I32, P, P, P, P, P, P],
                              I32),
+        "dsa_split_workspace_size": ([I32, I32, I64, I32, I32, I32], SZ),
+        "dsa_decode_select": ([P, P, P, P, P, P, P, P, I64, I32, I32, I32, I64, I32, I32, I32, P, P, P, SZ, P],
+                              I32),
+        "dsa_merge_selections": ([P, P, I64, I32, I32, I32, P, P, SZ, P], I32),
+        "dsa_decode_attend": ([P, P, P, P, P, P, P, P, I64, I32, I32, I32, I32, I32, I32, P, F, P, P, P, SZ, P],
+                              I32),
+        "dsa_merge_partials": ([P, I64, P, I64, I32, I32, I32, I32, P, P, P], I32),
         "dsa_stream_status": ([P, P], I32),
     }
     for name, (args, res) in sig.items():
@@ -443,6 +451,101 @@ def dsa_decode_noalloc(inp: dict, k_sel: int, max_context: int, sm_scale=None, o
                                    _p(out), _p(lse), _p(idx_out), _p(status_out), _stream(stream))
     _check("dsa_decode_noalloc", st)
     return out, lse, idx_out
+
+
+def _p_lists(t: torch.Tensor):
+    """Pointer and dim-0 stride (elements) of G lists whose inner dims are
+    dense (a [G, ...] view that may be a slice of a larger message)."""
+    if not t.is_cuda:
+        raise ValueError("DSA entry points take CUDA tensors")
+    if not t[0].is_contiguous():
+        raise ValueError("each list must be dense")
+    return ctypes.c_void_p(t.data_ptr()), int(t.stride(0))
+
+
+def split_workspace_size(G, B, max_context, H_q, d, k_sel) -> int:
+    return load().dsa_split_workspace_size(G, B, max_context, H_q, d, k_sel)
+
+
+def dsa_decode_select(shard: dict, pos_base, k_sel: int, max_context: int, cand_pos=None, cand_score=None,
+                      ws=None, stream=None):
+    """This shard's indexer scores and top-k as global positions (+ pos_base)
+    with their scores -> (cand_pos [B, k_sel], cand_score [B, k_sel])."""
+    B, H_I, d_I = shard["q_idx"].shape
+    P, ps, _ = shard["kidx_cache"].shape
+    max_pages = shard["block_table"].shape[1]
+    dev = shard["q_idx"].device
+    lib = load()
+    if ws is None:
+        ws = workspace(lib.dsa_split_workspace_size(1, B, max_context, 128, 128, k_sel), dev)
+    if cand_pos is None:
+        cand_pos = torch.empty((B, k_sel), dtype=torch.int32, device=dev)
+    if cand_score is None:
+        cand_score = torch.empty((B, k_sel), dtype=torch.float32, device=dev)
+    st = lib.dsa_decode_select(_p(shard["q_idx"]), _p(shard["q_scale"]), _p(shard["w"]), _p(shard["kidx_cache"]),
+                               _p(shard["kscale_cache"]), _p(shard["block_table"]), _p(shard["context_lens"]),
+                               _p(pos_base), P, max_pages, ps, B, max_context, H_I, d_I, k_sel, _p(cand_pos),
+                               _p(cand_score), _p(ws), ws.numel(), _stream(stream))
+    _check("dsa_decode_select", st)
+    return cand_pos, cand_score
+
+
+def dsa_merge_selections(cand_pos, cand_score, idx_out=None, ws=None, stream=None):
+    """Exact top-k of the union of G candidate lists (cand_pos/cand_score
+    [G, B, k_sel] views with a common dim-0 stride) -> idx [B, k_sel]."""
+    G, B, k_sel = cand_pos.shape
+    pp, sp = _p_lists(cand_pos)
+    ps_, ss = _p_lists(cand_score)
+    if sp != ss or cand_score.shape != cand_pos.shape:
+        raise ValueError("positions and scores must share shape and list stride")
+    lib = load()
+    if ws is None:
+        ws = workspace(lib.dsa_split_workspace_size(G, B, 1, 128, 128, k_sel), cand_pos.device)
+    if idx_out is None:
+        idx_out = torch.empty((B, k_sel), dtype=torch.int32, device=cand_pos.device)
+    st = lib.dsa_merge_selections(pp, ps_, sp, G, B, k_sel, _p(idx_out), _p(ws), ws.numel(), _stream(stream))
+    _check("dsa_merge_selections", st)
+    return idx_out
+
+
+def dsa_decode_attend(shard: dict, pos_base, idx, sm_scale=None, out=None, lse=None, ws=None, stream=None):
+    """Attention of each sequence's query over the selected positions this
+    shard holds -> partial (out [B, H_q, d], lse [B, H_q]).  FP8 K/V when
+    ``shard`` holds k_cache_scale/v_cache_scale."""
+    B, H_q, d = shard["q"].shape
+    P, ps, _ = shard["k_cache"].shape
+    max_pages = shard["block_table"].shape[1]
+    k_sel = idx.shape[1]
+    dev = shard["q"].device
+    sm_scale = 1.0 / math.sqrt(d) if sm_scale is None else sm_scale
+    lib = load()
+    if ws is None:
+        ws = workspace(lib.dsa_split_workspace_size(1, B, 1, H_q, d, k_sel), dev)
+    if out is None:
+        out = torch.empty_like(shard["q"])
+    if lse is None:
+        lse = torch.empty((B, H_q), dtype=torch.float32, device=dev)
+    st = lib.dsa_decode_attend(_p(shard["q"]), _p(shard["k_cache"]), _p(shard.get("k_cache_scale")),
+                               _p(shard["v_cache"]), _p(shard.get("v_cache_scale")), _p(shard["block_table"]),
+                               _p(shard["context_lens"]), _p(pos_base), P, max_pages, ps, B, H_q, d, k_sel, _p(idx),
+                               sm_scale, _p(out), _p(lse), _p(ws), ws.numel(), _stream(stream))
+    _check("dsa_decode_attend", st)
+    return out, lse
+
+
+def dsa_merge_partials(part_out, part_lse, out=None, lse=None, stream=None):
+    """Log-sum-exp merge of G partial attentions (part_out [G, B, H_q, d]
+    bf16, part_lse [G, B, H_q] f32; views with dense inner dims) -> (out, lse)."""
+    G, B, H_q, d = part_out.shape
+    po, so = _p_lists(part_out)
+    pl, sl = _p_lists(part_lse)
+    if out is None:
+        out = torch.empty((B, H_q, d), dtype=torch.bfloat16, device=part_out.device)
+    if lse is None:
+        lse = torch.empty((B, H_q), dtype=torch.float32, device=part_out.device)
+    st = load().dsa_merge_partials(po, so, pl, sl, G, B, H_q, d, _p(out), _p(lse), _stream(stream))
+    _check("dsa_merge_partials", st)
+    return out, lse
 
 
 def dsa_stream_status(ws: torch.Tensor, stream=None) -> int:

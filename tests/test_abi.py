@@ -162,3 +162,42 @@ def test_host_argument_errors_window_quantiser_kv8(lib):
     kv[17] = fake
     kv[13] = 264                                                 # d
     assert lib.dsa_cache_append_kv8(*kv) == UNSUP
+
+
+def test_host_argument_errors_split_decode(lib):
+    """The split-context entry points reject bad arguments on the host, before
+    any launch (no GPU needed)."""
+    P = ctypes.c_void_p
+    fake = P(0x1000)            # never dereferenced: every call below fails validation first
+    OK, INVALID, UNSUP, WS = 0, 1, 2, 3
+    ws = lib.dsa_split_workspace_size(8, 4, 131072, 128, 128, 512)
+    assert ws >= 256 + 4 * 131072 * 4 + 8 * 4 * 512 * 4
+    assert lib.dsa_split_workspace_size(0, 4, 131072, 128, 128, 512) == 0
+    # select: pos_base required; index shape; workspace size
+    sargs = [fake] * 8 + [100, 4, 64, 2, 256, 64, 128, 64, fake, fake, fake, 1 << 30, None]
+    bad = list(sargs); bad[7] = None
+    assert lib.dsa_decode_select(*bad) == INVALID
+    bad = list(sargs); bad[14] = 64                              # d_I
+    assert lib.dsa_decode_select(*bad) == UNSUP
+    bad = list(sargs); bad[15] = 0                               # k_sel
+    assert lib.dsa_decode_select(*bad) == INVALID
+    bad = list(sargs); bad[19] = 16                              # ws_bytes
+    assert lib.dsa_decode_select(*bad) == WS
+    # merge of selections: sizes, a list stride shorter than a list
+    assert lib.dsa_merge_selections(fake, fake, 0, 0, 4, 64, fake, fake, 1 << 30, None) == INVALID
+    assert lib.dsa_merge_selections(fake, fake, 100, 2, 4, 64, fake, fake, 1 << 30, None) == INVALID
+    assert lib.dsa_merge_selections(fake, fake, 0, 2, 4, 64, fake, fake, 16, None) == WS
+    # attend: lse required; one FP8 scale without the other; d
+    aargs = [fake, fake, None, fake, None, fake, fake, fake, 100, 4, 64, 2, 128, 128, 64, fake, 0.1, fake, fake,
+             fake, 1 << 30, None]
+    bad = list(aargs); bad[18] = None
+    assert lib.dsa_decode_attend(*bad) == INVALID
+    bad = list(aargs); bad[2] = fake
+    assert lib.dsa_decode_attend(*bad) == INVALID
+    bad = list(aargs); bad[13] = 64                              # d
+    assert lib.dsa_decode_attend(*bad) == UNSUP
+    # merge of partials: d, strides, alignment
+    assert lib.dsa_merge_partials(fake, 0, fake, 0, 2, 4, 128, 64, fake, None, None) == UNSUP
+    assert lib.dsa_merge_partials(fake, 100, fake, 0, 2, 4, 128, 128, fake, None, None) == INVALID
+    assert lib.dsa_merge_partials(fake, 0, P(0x1002), 0, 2, 4, 128, 128, fake, None, None) == INVALID
+    assert lib.dsa_merge_partials(fake, 65540, fake, 0, 2, 4, 128, 128, fake, None, None) == INVALID
