@@ -425,13 +425,40 @@ def bench_append(dsa, spec, inp, args, flush):
     return dict(us=1e3 * sum(ms) / len(ms), launches=2)
 
 
+GRAPH_FALLBACKS = []
+
+
+def graphed(fn):
+    """fn's launches captured once into a CUDA graph (after one eager call on a
+    side stream); returns the graph's replay, or fn itself (recorded in
+    GRAPH_FALLBACKS) if the capture is refused."""
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        fn()
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    try:
+        with torch.cuda.graph(g):
+            fn()
+    except RuntimeError as e:
+        GRAPH_FALLBACKS.append(str(e).splitlines()[0][:200])
+        torch.cuda.synchronize()
+        return fn
+    torch.cuda.synchronize()
+    return g.replay
+
+
 def bench_split(args, dsa, spec, shards_n, flush):
     """The decode of contexts split over `shards_n` devices (dsa_decode_select,
     dsa_merge_selections, dsa_decode_attend, dsa_merge_partials), the shards
-    run one after another on this GPU: each entry point's device time per
-    shard, the per-rank step (the slowest shard's select and attend plus the
-    two merges; the two all-gathers, which need several GPUs, are not
-    included) and the whole-context dsa_decode of the same input beside it."""
+    run one after another on this GPU.  Each rank's step (its select, the merge
+    of the gathered candidates, its attend, the merge of the gathered partials;
+    the two all-gathers, which need several GPUs, are not included) is
+    captured in a CUDA graph and timed per shard; the per-rank step is the
+    slowest shard's.  The whole-context dsa_decode of the same input, also
+    graph-replayed, is timed beside it."""
     from long_context_fp8_b200 import split_decode
     dev = torch.device("cuda")
     inp = dsa_synth.make_decode(spec, device=dev)
@@ -446,46 +473,72 @@ def bench_split(args, dsa, spec, shards_n, flush):
     idx = torch.empty((B, k), dtype=torch.int32, device=dev)
     out = torch.empty((B, H_q, d), dtype=torch.bfloat16, device=dev)
     lse = torch.empty((B, H_q), dtype=torch.float32, device=dev)
+    cpos, cscore = split_decode.candidate_views(recv)
+    po, pl = split_decode.partial_views(precv, B, H_q, d)
     steps = max(args.steps, 10)
 
-    def mean_ms(fn):
+    def mean_us(fn):
         ms = timed_steps(fn, steps, args.warmup, flush)
-        return sum(ms) / len(ms)
+        return 1e3 * sum(ms) / len(ms)
 
-    sel_ms, att_ms = [], []
-    for g, (sh, base) in enumerate(shards):
+    def select(g):
+        sh, base = shards[g]
         pos, score = split_decode.candidate_views(recv[g])
-        sel_ms.append(mean_ms(lambda: dsa.dsa_decode_select(sh, base, k, maxc, cand_pos=pos, cand_score=score,
-                                                            ws=ws)))
-    cpos, cscore = split_decode.candidate_views(recv)
-    mrg_ms = mean_ms(lambda: dsa.dsa_merge_selections(cpos, cscore, idx_out=idx, ws=ws))
-    for g, (sh, base) in enumerate(shards):
+        return lambda: dsa.dsa_decode_select(sh, base, k, maxc, cand_pos=pos, cand_score=score, ws=ws)
+
+    def attend(g):
+        sh, base = shards[g]
         o, l = split_decode.partial_views(precv[g], B, H_q, d)
-        att_ms.append(mean_ms(lambda: dsa.dsa_decode_attend(sh, base, idx, sm, out=o, lse=l, ws=ws)))
-    po, pl = split_decode.partial_views(precv, B, H_q, d)
-    mp_ms = mean_ms(lambda: dsa.dsa_merge_partials(po, pl, out=out, lse=lse))
+        return lambda: dsa.dsa_decode_attend(sh, base, idx, sm, out=o, lse=l, ws=ws)
+
+    merge_sel = lambda: dsa.dsa_merge_selections(cpos, cscore, idx_out=idx, ws=ws)
+    merge_part = lambda: dsa.dsa_merge_partials(po, pl, out=out, lse=lse)
+
+    # fill every shard's message slots once, eagerly
+    for g in range(shards_n):
+        select(g)()
+    merge_sel()
+    for g in range(shards_n):
+        attend(g)()
+    merge_part()
+    torch.cuda.synchronize()
     status = dsa.dsa_stream_status(ws)
+
+    def rank_step(g):
+        sel, att = select(g), attend(g)
+        def fn():
+            sel(); merge_sel(); att(); merge_part()
+        return fn
+
+    rank_us = [mean_us(graphed(rank_step(g))) for g in range(shards_n)]
+    sel_us = [mean_us(graphed(select(g))) for g in range(shards_n)]
+    att_us = [mean_us(graphed(attend(g))) for g in range(shards_n)]
+    mrg_us = mean_us(graphed(merge_sel))
+    mp_us = mean_us(graphed(merge_part))
+    status = status or dsa.dsa_stream_status(ws)
     del shards, ws
     torch.cuda.empty_cache()
     wws = dsa.workspace(dsa.decode_workspace_size(B, max(spec.context_lens), H_q, d, k), dev)
-    w_idx = torch.empty_like(idx)
-    whole_ms = mean_ms(lambda: dsa.dsa_decode(inp, k, max(spec.context_lens), sm, idx_out=w_idx, ws=wws))
+    w_idx, w_out, w_lse = torch.empty_like(idx), torch.empty_like(out), torch.empty_like(lse)
+    whole = lambda: dsa.dsa_decode(inp, k, max(spec.context_lens), sm, out=w_out, lse=w_lse, idx_out=w_idx,
+                                   ws=wws)
+    whole_us = mean_us(graphed(whole))
     same = bool(torch.equal(w_idx, idx))
-    rank_ms = max(a + b for a, b in zip(sel_ms, att_ms)) + mrg_ms + mp_ms
     del inp, wws
     torch.cuda.empty_cache()
     return {"shards": shards_n, "top_k": k,
             "workload": f"{B} sequences of {'/'.join(str(c) for c in spec.context_lens)} cached positions, "
                         f"each cut into {shards_n} contiguous shards",
-            "rank_step_us": round(rank_ms * 1e3, 2), "whole_context_decode_us": round(whole_ms * 1e3, 2),
-            "select_us": [round(x * 1e3, 2) for x in sel_ms],
-            "merge_selections_us": round(mrg_ms * 1e3, 2),
-            "attend_us": [round(x * 1e3, 2) for x in att_ms],
-            "merge_partials_us": round(mp_ms * 1e3, 2),
+            "rank_step_us": round(max(rank_us), 2), "rank_step_us_per_shard": [round(x, 2) for x in rank_us],
+            "whole_context_decode_us": round(whole_us, 2),
+            "select_us": [round(x, 2) for x in sel_us], "merge_selections_us": round(mrg_us, 2),
+            "attend_us": [round(x, 2) for x in att_us], "merge_partials_us": round(mp_us, 2),
             "message_bytes": {"candidates": shards_n * B * k * 8,
                               "partials": shards_n * 4 * split_decode.partial_words(B, H_q, d)},
             "selection_equals_whole_context": same, "device_status": status,
-            "note": "shards timed one after another on one GPU; the two all-gathers are not included"}
+            "graph_fallbacks": list(GRAPH_FALLBACKS),
+            "note": "CUDA-graph replays; shards timed one after another on one GPU; the two all-gathers "
+                    "are not included"}
 
 
 def bench_quantize(args, dsa, spec, peaks):

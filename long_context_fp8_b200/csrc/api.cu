@@ -674,7 +674,7 @@ dsa_status dsa_merge_selections(const int32_t *cand_pos, const float *cand_score
         return DSA_ERR_INVALID_ARG;
     if (list_stride == 0) list_stride = (int64_t)B * k_sel;
     if (list_stride < (int64_t)B * k_sel && G > 1) return DSA_ERR_INVALID_ARG;
-    if ((int64_t)G * k_sel > INT32_MAX / 2) return DSA_ERR_UNSUPPORTED;
+    if ((int64_t)G * k_sel > INT32_MAX / 2 || B > 65535) return DSA_ERR_UNSUPPORTED;
     if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u)) return DSA_ERR_WORKSPACE;
     if (ws_bytes < kWsHeader + align_up(merge_selections_ws_bytes(B, G, k_sel), 256)) return DSA_ERR_WORKSPACE;
     cudaStream_t st = as_stream(stream);

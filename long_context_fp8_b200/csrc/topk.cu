@@ -589,9 +589,14 @@ __device__ uint32_t sampled_threshold(TopkSmem<C> &sm, const float *row, int64_t
         for (int q = 0; q < C::NSAMP / C::NT; ++q) smp[tid + q * C::NT] = float_key(sv[q]);
     }
     __syncthreads();
-    // at least 8 samples above the threshold: a rank of 1 or 2 (long rows, small k)
-    // estimates the count so loosely that it often lands below k
-    const double want = 1.5 * (double)k * C::NSAMP / (double)n;
+    // lam = k * NSAMP / n samples are expected above the k-th largest key, about
+    // Poisson-distributed; the guess falls short of k when lam's count reaches the
+    // chosen rank.  1.5 lam leaves a wide margin for large lam, but for few samples
+    // (short shards of long rows, small k: lam = 8 fails about one row in ten at
+    // rank 12) the rank needs lam + 4 sqrt(lam) + 2 (a miss rate near 1e-4 at lam
+    // = 8), and at least 8.
+    const double lam = (double)k * C::NSAMP / (double)n;
+    const double want = fmax(1.5 * lam, lam + 4.0 * sqrt(lam) + 2.0);
     const uint32_t rank = (uint32_t)min((double)C::NSAMP, max(8.0, ceil(want)));
     uint32_t tau, unused;
     radix_select_smem(sm, smp, C::NSAMP, rank, &tau, &unused, 1, false);
