@@ -297,30 +297,54 @@ __global__ void merge_splits_kernel(const float *__restrict__ part, int rows, in
 // The same merge for D = 128 with one warp per (row, head): lane l owns
 // dimensions 4l .. 4l+3 (16-byte loads of each split's partial), eight heads
 // per 256-thread block, so a decode step's merge is a few waves of blocks.
+// Lane i holds split i's log-sum-exp and weight (32 splits a round), and the
+// splits' partial rows are loaded eight at a time, all in flight together: the
+// merge moves a few MB and is bound by memory latency.
 __global__ void __launch_bounds__(256)
 merge_splits_warp_kernel(const float *__restrict__ part, int rows, int splits, int H,
                          uint16_t *__restrict__ out, float *__restrict__ lse)
 {
-    constexpr int D = 128;
+    constexpr int D = 128, U = 8;
     grid_dep_wait();                                 // the attention's partials
     const int64_t row = blockIdx.x;
     const int h = blockIdx.y * 8 + (threadIdx.x >> 5);
     const int lane = threadIdx.x & 31;
     if (h >= H) return;
-    const float *pl = part + (int64_t)rows * splits * H * D;
+    const float *pl = part + (int64_t)rows * splits * H * D + row * splits * H + h;
+    const float *po = part + (row * splits * H + h) * (int64_t)D + lane * 4;
     float mx = -INFINITY;
-    for (int i = 0; i < splits; ++i) mx = fmaxf(mx, __ldg(pl + (row * splits + i) * H + h));
+    for (int i0 = 0; i0 < splits; i0 += 32)
+        if (i0 + lane < splits) mx = fmaxf(mx, __ldg(pl + (int64_t)(i0 + lane) * H));
+#pragma unroll
+    for (int o = 16; o; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    float den = 0.f;
+    float den = 0.f;                                 // this lane's splits' weights
     if (mx != -INFINITY) {
-        for (int i = 0; i < splits; ++i) {
-            const float li = __ldg(pl + (row * splits + i) * H + h);
-            const float wgt = li == -INFINITY ? 0.f : __expf(li - mx);
-            den += wgt;
-            const float4 o = __ldg(reinterpret_cast<const float4 *>(part + ((row * splits + i) * H + h) * (int64_t)D) + lane);
-            acc.x += wgt * o.x; acc.y += wgt * o.y; acc.z += wgt * o.z; acc.w += wgt * o.w;
+        for (int i0 = 0; i0 < splits; i0 += 32) {
+            const float li = i0 + lane < splits ? __ldg(pl + (int64_t)(i0 + lane) * H) : -INFINITY;
+            const float wl = li == -INFINITY ? 0.f : __expf(li - mx);
+            den += wl;
+            const int n = splits - i0 < 32 ? splits - i0 : 32;
+            for (int j0 = 0; j0 < n; j0 += U) {
+                float4 v[U];
+#pragma unroll
+                for (int u = 0; u < U; ++u)
+                    v[u] = j0 + u < n
+                               ? __ldg(reinterpret_cast<const float4 *>(po + (int64_t)(i0 + j0 + u) * H * D))
+                               : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+                for (int u = 0; u < U; ++u) {
+                    const float wgt = __shfl_sync(0xffffffffu, wl, (j0 + u) & 31);
+                    if (j0 + u < n && wgt != 0.f) {  // an empty split's partial is not read into the sum
+                        acc.x += wgt * v[u].x; acc.y += wgt * v[u].y;
+                        acc.z += wgt * v[u].z; acc.w += wgt * v[u].w;
+                    }
+                }
+            }
         }
     }
+#pragma unroll
+    for (int o = 16; o; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
     const float inv = den > 0.f ? 1.f / den : 0.f;
     uint2 packed;
     packed.x = pack_bf16x2(acc.x * inv, acc.y * inv);
