@@ -150,3 +150,59 @@ def test_messages_layout():
     l[2].fill_(-3.0)
     o2, l2 = split_decode.partial_views(precv[2], B, H, d)
     assert bool((o2 == 1.5).all()) and bool((l2 == -3.0).all())
+
+
+def test_union_of_shard_topk_holds_the_whole_topk():
+    """The exactness the split decode rests on, checked on the oracle's own
+    selector: the top-k of the union of the shards' top-k lists (score
+    descending, ties to the lower position) is the top-k of the whole row.
+    Scores are drawn from a few values so that ties are the rule, and shard
+    sizes range from below k to several times k."""
+    from oracle import oracle
+    rng = np.random.default_rng(21)
+    for trial in range(40):
+        n = int(rng.integers(1, 3000))
+        k = int(rng.integers(1, 300))
+        G = int(rng.integers(1, 9))
+        row = rng.integers(-6, 7, size=n).astype(np.float64) * 0.25
+        whole = oracle.topk(row[None], [n - 1], k)[0]
+        edges = [(g * n) // G for g in range(G + 1)]
+        cand_p, cand_s = [], []
+        for g in range(G):
+            a, b = edges[g], edges[g + 1]
+            if b == a:
+                continue
+            sel = oracle.topk(row[None, a:b], [b - a - 1], k)[0]
+            sel = sel[sel >= 0]
+            cand_p.append(sel + a)
+            cand_s.append(row[a:b][sel])
+        p, s = np.concatenate(cand_p), np.concatenate(cand_s)
+        merged = np.sort(p[np.lexsort((p, -s))[:k]])
+        want = whole[whole >= 0]
+        assert np.array_equal(merged, want), (trial, n, k, G)
+
+
+def test_partition_merge_equals_whole_attention():
+    """The partial-attention merge: the oracle's attention over a selection
+    equals the log-sum-exp merge of its attentions over any partition of the
+    selection (fp64, to rounding)."""
+    from oracle import oracle
+    g = torch.Generator().manual_seed(22)
+    H, d, n = 8, 64, 300
+    q = torch.randn((1, H, d), generator=g).to(torch.bfloat16)
+    K = torch.randn((n, d), generator=g).to(torch.bfloat16)
+    V = torch.randn((n, d), generator=g).to(torch.bfloat16)
+    o_all, l_all = oracle.sparse_attn(q, K, V, np.arange(n, dtype=np.int32)[None], [0], 0.125)
+    rng = np.random.default_rng(5)
+    for parts in (2, 3, 7):
+        cuts = np.sort(rng.choice(np.arange(1, n), size=parts - 1, replace=False))
+        bounds = [0, *cuts.tolist(), n]
+        outs, lses = [], []
+        for a, b in zip(bounds[:-1], bounds[1:]):
+            o, l = oracle.sparse_attn(q, K[a:b], V[a:b], np.arange(b - a, dtype=np.int32)[None], [0], 0.125)
+            outs.append(o[0]); lses.append(l[0])
+        L = np.stack(lses)                                      # [parts, H]
+        tot = np.logaddexp.reduce(L, axis=0)
+        merged = (np.exp(L - tot)[..., None] * np.stack(outs)).sum(0)
+        assert np.allclose(tot, l_all[0], rtol=0, atol=1e-12)
+        assert np.allclose(merged, o_all[0], rtol=0, atol=1e-12)
