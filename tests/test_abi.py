@@ -201,3 +201,16 @@ def test_host_argument_errors_split_decode(lib):
     assert lib.dsa_merge_partials(fake, 100, fake, 0, 2, 4, 128, 128, fake, None, None) == INVALID
     assert lib.dsa_merge_partials(fake, 0, P(0x1002), 0, 2, 4, 128, 128, fake, None, None) == INVALID
     assert lib.dsa_merge_partials(fake, 65540, fake, 0, 2, 4, 128, 128, fake, None, None) == INVALID
+
+
+def test_header_compiles_as_c_and_library_links(lib, tmp_path):
+    """A C99 program that includes include/dsa.h, links the shared library and
+    calls the entry points that need no GPU."""
+    exe = str(tmp_path / "abi_consumer")
+    src = os.path.join(ROOT, "tests", "abi_consumer.c")
+    libdir = os.path.dirname(dsa_build.LIB)
+    subprocess.run(["gcc", "-std=c99", "-Wall", "-Werror", "-pedantic", "-I", os.path.join(ROOT, "include"), src,
+                    "-o", exe, f"-L{libdir}", "-l:libdsa_b200.so", f"-Wl,-rpath,{libdir}"], check=True,
+                   capture_output=True, text=True)
+    r = subprocess.run([exe], capture_output=True, text=True)
+    assert r.returncode == 0 and r.stdout.strip() == "ok", (r.returncode, r.stdout, r.stderr)
