@@ -112,6 +112,9 @@ class CudaOps:
         dsa.dsa_merge_partials(part_out, part_lse, out=out, lse=lse)
 
 
+_default_ops: Optional[CudaOps] = None
+
+
 def split_decode_step(shard: dict, pos_base: torch.Tensor, k_sel: int, max_context: int, group=None,
                       sm_scale: Optional[float] = None, ops=None):
     """One decode step of B sequences whose contexts are split over the ranks
@@ -121,7 +124,11 @@ def split_decode_step(shard: dict, pos_base: torch.Tensor, k_sel: int, max_conte
     position of each sequence; max_context is the largest shard length on
     any rank.  Returns (out [B, H_q, d] bf16, lse [B, H_q], idx [B, k_sel]),
     identical on every rank."""
-    ops = ops or CudaOps()
+    global _default_ops
+    if ops is None:
+        if _default_ops is None:
+            _default_ops = CudaOps()              # one workspace, grown on demand, reused by every step
+        ops = _default_ops
     G = dist.get_world_size(group)
     B, H_q, d = shard["q"].shape
     dev = shard["q"].device
