@@ -192,3 +192,57 @@ def test_decode_select_reports_negative_base():
     pos, _ = dsa.dsa_decode_select(inp, base, 64, 300, ws=ws)
     assert dsa.dsa_stream_status(ws) == 1                           # DSA_ERR_INVALID_ARG
     assert int((pos[1] >= 0).sum()) == 0 and int((pos[0] >= 0).sum()) == 64
+
+
+def test_split_single_shard_equals_decode_bit_for_bit():
+    """G = 1: the merge of one candidate list is that list, the attention is the
+    whole-context decode's own, and the merge of one partial multiplies by
+    exp(0) = 1 -- every output equals dsa_decode's bit for bit."""
+    lens, k = (5000, 3000, 777), 512
+    inp = to_dev(dsa_synth.make_decode(_spec(lens, k, seed=97)))
+    sm = sm_of(128)
+    out, lse, idx, _ = _emulated_split(inp, 1, k, sm)
+    w_out, w_lse, w_idx = dsa.dsa_decode(inp, k, max(lens), sm)
+    torch.cuda.synchronize()
+    assert torch.equal(idx, w_idx) and torch.equal(out, w_out) and torch.equal(lse, w_lse)
+
+
+def test_split_shard_holding_none_of_the_selection():
+    """Shard 0's index keys are zeroed (their scores are 0 while the others'
+    are positive), so the merged selection holds none of its positions: its
+    partial is empty (lse -inf, zeros) and the merge must ignore it."""
+    lens, k, G = (6000, 4000, 9000), 256, 4
+    inp = dsa_synth.make_decode(_spec(lens, k, seed=98))
+    ps = inp["kidx_cache"].shape[1]
+    flat = inp["kidx_cache"].view(-1, inp["kidx_cache"].shape[2])
+    for b, n in enumerate(lens):
+        p = torch.arange(n // G)
+        flat[inp["block_table"][b, p // ps].long() * ps + p % ps] = 0
+    inp = to_dev(inp)
+    sm = sm_of(128)
+    out, lse, idx, (p_out, p_lse) = _emulated_split(inp, G, k, sm)
+    w_out, w_lse, w_idx = dsa.dsa_decode(inp, k, max(lens), sm)
+    torch.cuda.synchronize()
+    assert torch.equal(idx, w_idx)
+    for b, n in enumerate(lens):
+        sel = idx[b][idx[b] >= 0]
+        assert int(sel.numel()) == k and int((sel < n // G).sum()) == 0
+    assert bool(torch.isneginf(p_lse[0]).all()) and float(p_out[0].float().abs().max()) == 0.0
+    ro, rl = _attention_over(inp, idx.cpu().numpy(), sm)
+    assert_attn_close(out.float().cpu().numpy(), ro, lse.cpu().numpy(), rl, "shard without selection")
+
+
+def test_split_zero_length_shard_is_reported():
+    """A sequence shorter than G leaves some shards without positions: the
+    select reports DSA_ERR_INVALID_ARG and returns no candidates for it, the
+    other sequences' candidates are unaffected."""
+    lens, k, G = (2, 300), 64, 4
+    inp = to_dev(dsa_synth.make_decode(_spec(lens, k, seed=99)))
+    shards = dsa_synth.split_decode_input(inp, G)
+    sh, base = shards[0]
+    assert sh["context_lens"].tolist() == [0, 75]
+    ws = dsa.workspace(dsa.split_workspace_size(G, 2, 75, 128, 128, k), "cuda")
+    pos, score = dsa.dsa_decode_select(sh, base, k, 75, ws=ws)
+    assert dsa.dsa_stream_status(ws) == 1                           # DSA_ERR_INVALID_ARG
+    assert bool((pos[0] == -1).all()) and bool(torch.isneginf(score[0]).all())
+    assert int((pos[1] >= 0).sum()) == k and int(pos[1].max()) < 75
