@@ -206,3 +206,40 @@ def test_partition_merge_equals_whole_attention():
         merged = (np.exp(L - tot)[..., None] * np.stack(outs)).sum(0)
         assert np.allclose(tot, l_all[0], rtol=0, atol=1e-12)
         assert np.allclose(merged, o_all[0], rtol=0, atol=1e-12)
+
+
+def test_split_decode_input_repacks_rows_exactly():
+    """Every cached row of every sequence lands in exactly one shard, at its
+    local position, with the same bytes (index key, its scale, K, V and, for
+    FP8 K/V caches, their scales); shard tables point only at the shard's
+    own pages; the queries are shared."""
+    import dsa_synth
+    spec = dsa_synth.DecodeSpec("split_repack", context_lens=(1000, 64, 1, 2049, 130), H_I=8, d_I=64, k=32,
+                                H_q=8, d=64, page_size=64, needle_frac=0.0, needle_min_age=0, seed=31)
+    for inp in (dsa_synth.make_decode(spec), dsa_synth.decode_kv_to_fp8(dsa_synth.make_decode(spec))):
+        ps = spec.page_size
+        keys = [k for k in ("kidx_cache", "kscale_cache", "k_cache", "v_cache", "k_cache_scale", "v_cache_scale")
+                if k in inp]
+        for G in (1, 3, 4):
+            shards = dsa_synth.split_decode_input(inp, G)
+            seen = [np.zeros(n, dtype=np.int64) for n in spec.context_lens]
+            for sh, base in shards:
+                for k_ in ("q_idx", "q_scale", "w", "q"):
+                    assert sh[k_] is inp[k_]
+                P = sh["kidx_cache"].shape[0]
+                for b, n_all in enumerate(spec.context_lens):
+                    n, pb = int(sh["context_lens"][b]), int(base[b])
+                    pages = (n + ps - 1) // ps
+                    tab = sh["block_table"][b]
+                    assert bool((tab[:pages] >= 0).all()) and bool((tab[:pages] < P).all())
+                    assert bool((tab[pages:] == -1).all())
+                    for p in range(n):
+                        g_slot = int(inp["block_table"][b, (pb + p) // ps]) * ps + (pb + p) % ps
+                        l_slot = int(tab[p // ps]) * ps + p % ps
+                        for k_ in keys:
+                            full = inp[k_].reshape((-1,) + tuple(inp[k_].shape[2:]))
+                            part = sh[k_].reshape((-1,) + tuple(sh[k_].shape[2:]))
+                            assert torch.equal(full[g_slot], part[l_slot]), (k_, G, b, p)
+                        seen[b][pb + p] += 1
+            for b in range(len(seen)):
+                assert bool((seen[b] == 1).all()), (G, b)
