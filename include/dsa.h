@@ -438,12 +438,19 @@ dsa_status dsa_cache_append_kv8(const void *kidx_new, dsa_dtype kidx_dtype, cons
  * step's device status word (a dsa_status) on `stream` after the step.
  *
  * The scratch is a fixed device array of DSA_DECODE_NOALLOC_SCRATCH_BYTES
- * (64 MiB) inside the library; every GPU that loads the library holds it
- * until the process exits.  A problem whose dsa_decode_workspace_size()
- * exceeds that size is rejected with DSA_ERR_WORKSPACE before any launch
- * (64 sequences x 64K context x k 2048 x 128 heads needs about 33 MiB).
- * The first call on each device looks up the array's device address with
- * that device current; make that first call before any stream capture.
+ * (64 MiB) inside the library.  CUDA loads the library's device code lazily,
+ * so that array is reserved on a device by the FIRST call on that device
+ * (when the call looks up the array's device address with the device
+ * current); the reservation then lasts as long as the device's context.
+ * That first call can therefore fail with DSA_ERR_CUDA when the device has no
+ * 64 MiB left, and may synchronise the device: make it early, as a warm-up,
+ * before filling a memory pool or starting a stream capture.  Later calls on
+ * the same context reserve nothing.  A device reset (or a released and
+ * recreated primary context) loads the code again; the next call notices the
+ * new context and looks the address up again (that call reserves again).
+ * A problem whose dsa_decode_workspace_size() exceeds the array is rejected
+ * with DSA_ERR_WORKSPACE before any launch (64 sequences x 64K context x
+ * k 2048 x 128 heads needs about 33 MiB).
  * Every call on a device shares the one array and leaves its contents behind
  * (the status word is cleared at the start of each call): calls whose GPU
  * work overlaps -- on different streams, or from different host threads --

@@ -10,6 +10,7 @@ from __future__ import annotations
 import concurrent.futures as cf
 import glob
 import os
+import re
 import shutil
 import subprocess
 import sys
@@ -24,6 +25,57 @@ BUILD_DIR = os.path.join(ROOT, "_build")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 NVCC_FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "--expt-relaxed-constexpr",
               "-I", INCLUDE, "-I", CSRC]
+
+
+# Kernels whose warpgroups re-split their registers with setmaxnreg: the split
+# adds up to the launch's register file only when ptxas gives them exactly this
+# many registers per thread, so any other count fails the build (instead of a
+# launch that would wait forever in setmaxnreg, or a silent slower path).
+SETMAXNREG_KERNELS = {"index_tc_kernel": 168, "sparse_attn_tc_kernel": 168}
+
+
+def kernel_name(mangled: str) -> str:
+    """The unqualified function name of an Itanium-mangled nested name
+    (_ZN <len><component> ... E|I ...); the input itself if it is not one."""
+    if not mangled.startswith("_ZN"):
+        return mangled
+    i = 3
+    while i < len(mangled) and mangled[i].isdigit():
+        j = i
+        while mangled[j].isdigit():
+            j += 1
+        n = int(mangled[i:j])
+        comp = mangled[j:j + n]
+        i = j + n
+        if i >= len(mangled) or mangled[i] in "EI":
+            return comp
+    return mangled
+
+
+def check_registers(ptxas_log: str, src: str) -> list:
+    """Checks the ptxas -v report of one source file against
+    SETMAXNREG_KERNELS; returns (mangled name, registers, spill-store bytes)
+    per entry function."""
+    found, cur, spill = [], None, 0
+    for line in ptxas_log.splitlines():
+        m = re.search(r"Compiling entry function '([^']+)'", line)
+        if m:
+            cur, spill = m.group(1), 0
+            continue
+        m = re.search(r"(\d+) bytes spill stores", line)
+        if m and cur is not None:
+            spill = int(m.group(1))
+            continue
+        m = re.search(r"Used (\d+) registers", line)
+        if m and cur is not None:
+            found.append((cur, int(m.group(1)), spill))
+            cur = None
+    for name, regs, _ in found:
+        want = SETMAXNREG_KERNELS.get(kernel_name(name))
+        if want is not None and regs != want:
+            raise RuntimeError(f"{os.path.basename(src)}: {kernel_name(name)} built with {regs} registers "
+                               f"per thread, its setmaxnreg split needs exactly {want}")
+    return found
 
 
 def nvcc() -> str:
@@ -58,12 +110,13 @@ def build(force: bool = False, verbose: bool = False, extra_flags=()) -> str:
 
     def compile_one(src):
         obj = os.path.join(BUILD_DIR, os.path.basename(src) + ".o")
-        cmd = [cc, *ARCH, *NVCC_FLAGS, *extra_flags, "-c", src, "-o", obj]
+        cmd = [cc, *ARCH, *NVCC_FLAGS, *extra_flags, "-Xptxas", "-v", "-c", src, "-o", obj]
         if verbose:
             print(" ".join(cmd), flush=True)
         r = subprocess.run(cmd, capture_output=True, text=True)
         if r.returncode != 0:
             raise RuntimeError(f"nvcc failed for {src}:\n{r.stdout}\n{r.stderr}")
+        check_registers(r.stdout + r.stderr, src)
         if verbose and (r.stdout or r.stderr):
             print(r.stdout, r.stderr, flush=True)
         return obj

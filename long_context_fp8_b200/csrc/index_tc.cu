@@ -444,7 +444,8 @@ cudaError_t launch_index_tc(const uint8_t *q8, const float *sq, const uint8_t *k
     cudaFuncAttributes fa;
     cudaError_t e = cudaFuncGetAttributes(&fa, index_tc_kernel);
     if (e != cudaSuccess) return e;
-    if (fa.numRegs != IT_LAUNCH_REGS) return cudaErrorNotSupported;
+    // (the build checks this too; a mismatch is an error, not a silent slower path)
+    if (fa.numRegs != IT_LAUNCH_REGS) return cudaErrorInvalidKernelImage;
     e = cudaFuncSetAttribute(index_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     if (write_upper) {

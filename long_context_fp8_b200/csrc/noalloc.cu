@@ -4,8 +4,15 @@
 // process has reserved all device memory in its own pool, or code on a
 // latency-critical path where a device allocation (which can synchronise the
 // device) is not allowed.  dsa_decode_noalloc runs the same kernels as
-// dsa_decode, with the scratch in a fixed, file-scope device array that every
-// GPU loading this library holds until the process exits.
+// dsa_decode, with the scratch in a fixed, file-scope device array.
+//
+// CUDA loads modules lazily, so the array is backed by device memory when its
+// module is first needed on a device: the first call's address lookup below.
+// That first call therefore reserves the 64 MiB (and can fail with
+// DSA_ERR_CUDA when the device is full); later calls reserve nothing.  The
+// reservation lasts as long as the context that loaded the module.
+#include <cudaTypedefs.h>
+
 #include <mutex>
 
 #include "kernels.h"
@@ -16,24 +23,55 @@ static __device__ __align__(256) unsigned char dsa_decode_scratch[DSA_DECODE_NOA
 
 constexpr int kMaxDevices = 256;
 std::mutex g_scratch_mu;
-void *g_scratch_addr[kMaxDevices];
+struct ScratchSlot {
+    CUcontext ctx;       // the context the address belongs to
+    void *addr;
+};
+ScratchSlot g_scratch[kMaxDevices];
+
+PFN_cuCtxGetCurrent_v4000 ctx_get_current_fn()
+{
+    static PFN_cuCtxGetCurrent_v4000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(p);
+    });
+    return fn;
+}
 
 // Device address of the scratch array on the current device.  The symbol's
-// host-side name is not a device address, so it is looked up once per device
-// (with that device current) and cached.
+// host-side name is not a device address, so the address is looked up with
+// the device current and cached together with the context it belongs to: a
+// device reset (or a released and recreated primary context) loads the
+// module again, possibly at another address, and the lookup is redone.
 dsa_status scratch_on_current_device(void **out)
 {
     int dev = -1;
     if (cudaGetDevice(&dev) != cudaSuccess) return DSA_ERR_CUDA;
     if (dev < 0 || dev >= kMaxDevices) return DSA_ERR_UNSUPPORTED;
+    PFN_cuCtxGetCurrent_v4000 get_ctx = ctx_get_current_fn();
+    if (!get_ctx) return DSA_ERR_CUDA;
+    CUcontext ctx = nullptr;
+    if (get_ctx(&ctx) != CUDA_SUCCESS) return DSA_ERR_CUDA;
     std::lock_guard<std::mutex> lock(g_scratch_mu);
-    if (!g_scratch_addr[dev]) {
+    ScratchSlot &slot = g_scratch[dev];
+    if (ctx == nullptr || slot.addr == nullptr || slot.ctx != ctx) {
+        // (no context yet: the lookup makes the runtime create the device's primary one)
         void *p = nullptr;
         cudaError_t e = cudaGetSymbolAddress(&p, dsa_decode_scratch);
-        if (e != cudaSuccess || p == nullptr) return DSA_ERR_CUDA;
-        g_scratch_addr[dev] = p;
+        if (e != cudaSuccess || p == nullptr) {
+            (void)cudaGetLastError();        // reported through the return value, not left sticky
+            return DSA_ERR_CUDA;
+        }
+        if (ctx == nullptr && (get_ctx(&ctx) != CUDA_SUCCESS || ctx == nullptr)) return DSA_ERR_CUDA;
+        slot.ctx = ctx;
+        slot.addr = p;
     }
-    *out = g_scratch_addr[dev];
+    *out = slot.addr;
     return DSA_OK;
 }
 

@@ -758,7 +758,8 @@ cudaError_t launch_attn_tc_impl(const CUtensorMap &qmap, const CUtensorMap &kmap
     cudaFuncAttributes fa;
     cudaError_t e = cudaFuncGetAttributes(&fa, sparse_attn_tc_kernel<KV8>);
     if (e != cudaSuccess) return e;
-    if (fa.numRegs != AT_LAUNCH_REGS) return cudaErrorNotSupported;   // the register split assumes it
+    // the register split assumes it (the build checks it too): an error, not a silent slower path
+    if (fa.numRegs != AT_LAUNCH_REGS) return cudaErrorInvalidKernelImage;
     e = cudaFuncSetAttribute(sparse_attn_tc_kernel<KV8>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     const unsigned grid = (unsigned)std::min<int64_t>(a.items, sms);

@@ -68,3 +68,22 @@ def test_noalloc_reports_device_status():
     torch.cuda.synchronize()
     assert int(status.item()) == 1       # DSA_ERR_INVALID_ARG
     inp["block_table"][1, 2] = 0
+
+
+def test_noalloc_second_call_reserves_no_device_memory():
+    # The scratch array is reserved by the first call on a device (lazy module
+    # loading); every later call must leave the device's free memory unchanged.
+    spec, inp = _decode_inputs((1500, 400), 9, k=64)
+    maxc = max(spec.context_lens)
+    out = torch.empty_like(inp["q"])
+    lse = torch.empty((spec.B, spec.H_q), dtype=torch.float32, device="cuda")
+    idx = torch.empty((spec.B, spec.k), dtype=torch.int32, device="cuda")
+    status = torch.zeros((1,), dtype=torch.int32, device="cuda")
+    dsa.dsa_decode_noalloc(inp, spec.k, maxc, out=out, lse=lse, idx_out=idx, status_out=status)
+    torch.cuda.synchronize()
+    free_before, _ = torch.cuda.mem_get_info()
+    dsa.dsa_decode_noalloc(inp, spec.k, maxc, out=out, lse=lse, idx_out=idx, status_out=status)
+    torch.cuda.synchronize()
+    free_after, _ = torch.cuda.mem_get_info()
+    assert free_after == free_before, (free_before, free_after)
+    assert int(status.item()) == 0
