@@ -196,50 +196,22 @@ def count_launches(fn):
 
 # ----------------------------------------------------------------------------- prefill
 
-def prefill_stage_breakdown(dsa, inp, spec, ws, flush, reps=2):
-    """Per-kernel time of the prefill's stages, each stage entry point timed
-    with CUDA events on the current stream (same kernels, same row passes)."""
-    T, k = spec.L, spec.k
-    R = ws["rows_per_pass"]
-    scores = ws["scores"]
-    idx = ws["idx"]
-    stream = torch.cuda.current_stream()
-    idx_ms, topk_ms, attn_ms = 0.0, 0.0, 0.0
-    per_launch = []
-    for rep in range(reps):
-        flush.zero_()
-        for r0 in range(0, T, R):
-            n = min(R, T - r0)
-            ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
-            ev[0].record(stream)
-            dsa.dsa_index_scores(inp["q_idx"], inp["q_scale"], inp["k_idx"], inp["k_scale"], inp["w"],
-                                 row_begin=r0, row_count=n, out=scores[:n * T].view(n, T), ld=T,
-                                 fill_upper=False)
-            ev[1].record(stream)
-            dsa.dsa_topk(scores[:n * T].view(n, T), k, row_begin=r0, T=T, out=idx[r0:r0 + n])
-            ev[2].record(stream)
-            per_launch.append((ev, r0, n))
-        a = torch.cuda.Event(enable_timing=True)
-        b = torch.cuda.Event(enable_timing=True)
-        a.record(stream)
-        dsa.dsa_sparse_attn(inp["q"], inp["k"], inp["v"], idx, 1.0 / math.sqrt(spec.d),
-                            out=ws["out"], lse=ws["lse"])
-        b.record(stream)
-        per_launch.append(((a, b), None, None))
-    torch.cuda.synchronize()
-    idx_launch_ms, idx_launch_flop = [], []
-    for ev, r0, n in per_launch:
-        if r0 is None:
-            attn_ms += ev[0].elapsed_time(ev[1])
-        else:
-            t_i = ev[0].elapsed_time(ev[1])
-            idx_ms += t_i
-            topk_ms += ev[1].elapsed_time(ev[2])
-            idx_launch_ms.append(t_i)
-            pairs = sum_pairs(r0, n)
-            idx_launch_flop.append(2.0 * spec.H_I * spec.d_I * pairs)
-    return dict(indexer_ms=idx_ms / reps, topk_ms=topk_ms / reps, attn_ms=attn_ms / reps,
-                indexer_launch_ms=idx_launch_ms, indexer_launch_flop=idx_launch_flop)
+def prefill_stage_breakdown(dsa, step, flush, reps=2):
+    """Per-stage device time of dsa_prefill's own launches: the library's stage
+    timing records CUDA events on the call's stream around each stage (the
+    fused selection's sample scores, thresholds, select epilogue, finish and
+    repair; the attention), summed over the row passes, averaged over reps."""
+    dsa.profile_read()                      # drop anything recorded before
+    dsa.profile_enable(True)
+    try:
+        for _ in range(reps):
+            flush.zero_()
+            step()
+        torch.cuda.synchronize()
+    finally:
+        dsa.profile_enable(False)
+    st = dsa.profile_read()
+    return {name: (ms / reps, runs // reps) for name, (ms, runs) in st.items()}
 
 
 def sum_pairs(r0, n):
@@ -275,17 +247,14 @@ def bench_prefill(args, dsa, spec, peaks, peak_kind, ws_n, rank):
     step_ms = sum(ms) / len(ms)
     step_ms_max = max_over_ranks(step_ms, ws_n)
 
-    # stage breakdown (same kernels as dsa_prefill's passes) for the roofline
-    rows_per_pass = rows_per_pass_of(wsb, T, k)
-    scores_buf = torch.empty(rows_per_pass * T, dtype=torch.float32, device=dev)
-    br = prefill_stage_breakdown(dsa, inp, spec,
-                                 dict(rows_per_pass=rows_per_pass, scores=scores_buf, idx=idx,
-                                      out=out, lse=lse), flush)
-    del scores_buf
+    # stage breakdown of the same call, for the roofline of its dominant kernel
+    br = prefill_stage_breakdown(dsa, step, flush)
     flops = dsa_synth.prefill_flops(spec)
     fp8_peak = peaks["bf16_tflops"] * 2.0           # nominal fp8:bf16 ratio 2 on B200
-    idx_achieved = sum(br["indexer_launch_flop"]) / (sum(br["indexer_launch_ms"]) * 1e-3) / 1e12
-    attn_tflops = flops["attn_flop"] / (br["attn_ms"] * 1e-3) / 1e12
+    # the select epilogue's indexer scores every causal pair (and writes none of them)
+    idx_ms = br["select"][0] + br["scores"][0]
+    idx_achieved = flops["indexer_flop"] / (idx_ms * 1e-3) / 1e12
+    attn_tflops = flops["attn_flop"] / (br["attention"][0] * 1e-3) / 1e12
 
     e2e = None
     if not args.no_e2e:
@@ -295,13 +264,7 @@ def bench_prefill(args, dsa, spec, peaks, peak_kind, ws_n, rank):
     torch.cuda.empty_cache()
     return dict(step_ms=step_ms_max, ms=ms, clocks=clocks, launches=n_launch, per_kernel=per_kernel,
                 breakdown=br, flops=flops, fp8_peak=fp8_peak, idx_tflops=idx_achieved,
-                attn_tflops=attn_tflops, e2e=e2e, rows_per_pass=rows_per_pass)
-
-
-def rows_per_pass_of(wsb, T, k):
-    fixed = 256  # idx_out is passed, so only the header precedes the score buffer
-    R = ((wsb - fixed) // (4 * T)) // 64 * 64
-    return min(R, ((T + 63) // 64) * 64)
+                attn_tflops=attn_tflops, e2e=e2e, workspace_bytes=wsb)
 
 
 def replica_spec(spec, rank):
@@ -769,7 +732,7 @@ def main():
     value = whole_job_rate(ws_n, T, pre["step_ms"])
     br = pre["breakdown"]
     idx_peak = pre["fp8_peak"]
-    roofline = {"bound": "tensor", "kernel": "indexer (FP8 e4m3 x e4m3 -> fp32)",
+    roofline = {"bound": "tensor", "kernel": "indexer with the fused select epilogue (FP8 e4m3 x e4m3 -> fp32)",
                 "achieved": round(pre["idx_tflops"], 2), "peak": round(idx_peak, 1),
                 "unit": "TFLOP/s", "frac": round(pre["idx_tflops"] / idx_peak, 4),
                 "peak_source": f"{peak_kind} bf16 dense x 2 (fp8:bf16 nominal ratio), burst",
@@ -781,13 +744,16 @@ def main():
         sus = peaks["bf16_tflops_sustained"] * 2.0
         roofline["peak_sustained"] = round(sus, 1)
         roofline["frac_sustained"] = round(pre["idx_tflops"] / sus, 4)
+    sel_ms = sum(br[n][0] for n in ("sample", "tau", "finish", "repair", "topk"))
     stages = {
-        "indexer_ms": round(br["indexer_ms"], 3), "topk_ms": round(br["topk_ms"], 3),
-        "attention_ms": round(br["attn_ms"], 3),
+        "indexer_ms": round(br["select"][0] + br["scores"][0], 3),
+        "selection_ms": round(sel_ms, 3),
+        "attention_ms": round(br["attention"][0], 3),
         "attention_tflops": round(pre["attn_tflops"], 2),
         "attention_frac_bf16": round(pre["attn_tflops"] / peaks["bf16_tflops"], 4),
-        "topk_hbm_gbs": round((pre["flops"]["pairs"] * 4 + T * spec.k * 4) / (br["topk_ms"] * 1e-3) / 1e9, 1),
-        "indexer_passes": len(br["indexer_launch_ms"]), "rows_per_pass": pre["rows_per_pass"],
+        "per_stage_ms": {n: round(v[0], 3) for n, v in br.items() if v[1]},
+        "per_stage_runs": {n: v[1] for n, v in br.items() if v[1]},
+        "workspace_bytes": pre["workspace_bytes"],
     }
     line = {"metric": metric, "value": round(value, 1), "unit": "tokens/s", "n_gpus": ws_n,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(pre["step_ms"], 3),

@@ -152,8 +152,26 @@ dsa_status dsa_sparse_attn(const void *q, const void *k, const void *v, const in
  * three stage functions above; dtype DSA_E4M3 or DSA_F32).
  *   out [T, H_q, d]; lse_out [T, H_q] (nullable); idx_out int32 [T, k_sel]
  *   (nullable: the selection is then kept in the workspace only).
- * workspace: at least dsa_prefill_workspace_size(...) bytes.  A larger
- * workspace lets the indexer process more query rows per pass.
+ * With DSA_E4M3 index values, at most 64 index heads and k_sel <= 4096 the
+ * selection is fused into the indexer (the pages' indexer -> top-k selector
+ * flow, "DeepSeek-V3.2-Exp 稀疏注意力机制(DSA)技术深度解析", section 1; the
+ * sider.ai page's point that selection must stay cheap and cache-aware): the
+ * causal score matrix is never written.  Query rows go in passes of R rows:
+ * the indexer first scores a sample of the keys (one pseudo-random position
+ * per 64) to fix a per-row threshold, then scores every key and keeps only
+ * the (score, position) pairs at or above it, and an exact select finishes
+ * each row from those.  A row whose count of kept pairs is below k_sel or
+ * above the list's capacity (4 k_sel, at least 4096) -- for example when
+ * many scores tie -- is recomputed by the score epilogue and selected by the
+ * stand-alone top-k, so the result is always the exact top-k of the same
+ * fp32 scores that dsa_index_scores returns.  Otherwise (f32 inputs, more
+ * heads, larger k) the indexer writes row blocks of scores and dsa_topk's
+ * kernel selects from them.
+ * workspace: at least dsa_prefill_workspace_size(...) bytes; with a smaller
+ * one the call returns DSA_ERR_WORKSPACE.  The fused path's size is the
+ * selection (T x k_sel indices, unless idx_out is given) plus per-pass
+ * scratch of at most 4096 rows and 1 GiB of repair score rows: linear in T.
+ * A larger workspace lets a pass take more query rows.
  */
 size_t dsa_prefill_workspace_size(int64_t T, int H_I, int d_I, int H_q, int d, int k_sel,
                                   dsa_dtype dtype);
@@ -176,6 +194,35 @@ dsa_status dsa_prefill_window(const void *q_idx, const float *q_scale, const voi
                               int window, float sm_scale, void *out, float *lse_out,
                               int32_t *idx_out, dsa_dtype dtype, void *workspace, size_t ws_bytes,
                               void *stream);
+
+/*
+ * dsa_prefill_rows -- the fused prefill of the query rows [row_begin,
+ * row_begin + row_count) of a T-token sequence, for a split of one long
+ * prefill over devices: each device takes a set of query rows (a causal row
+ * costs in proportion to its position, so rows are dealt in a zigzag of 2G
+ * chunks, device g taking chunks g and 2G - 1 - g) and needs the key side of
+ * every earlier position.  None of the pages describes a multi-device
+ * prefill; the hotdry page's million-token setting motivates it.
+ *   Query side, row_count rows (row r is position row_begin + r):
+ *     q_idx u8 [row_count, H_I, d_I], q_scale f32 [row_count],
+ *     w bf16 [row_count, H_I], q bf16 [row_count, H_q, d].
+ *   Key side, positions 0..T-1: k_idx u8 [T, d_I], k_scale f32 [T],
+ *     k, v bf16 [T, d] (only positions < row_begin + row_count are read).
+ *   Outputs for those rows: out [row_count, H_q, d], lse_out [row_count, H_q]
+ *     (nullable), idx_out int32 [row_count, k_sel] (nullable: then kept in
+ *     the workspace).
+ * Row r's results equal, bit for bit, row row_begin + r of dsa_prefill on the
+ * whole sequence.  Requires dtype DSA_E4M3, H_I <= 64, k_sel <= 4096 (the
+ * fused selection); else DSA_ERR_UNSUPPORTED.  Workspace: at least
+ * dsa_prefill_rows_workspace_size(...) bytes (0 when unsupported).
+ */
+size_t dsa_prefill_rows_workspace_size(int64_t T, int64_t row_count, int H_I, int d_I, int H_q, int d,
+                                       int k_sel, dsa_dtype dtype);
+dsa_status dsa_prefill_rows(const void *q_idx, const float *q_scale, const void *k_idx, const float *k_scale,
+                            const void *w, const void *q, const void *k, const void *v, int64_t T,
+                            int64_t row_begin, int64_t row_count, int H_I, int d_I, int H_q, int d, int k_sel,
+                            float sm_scale, void *out, float *lse_out, int32_t *idx_out, dsa_dtype dtype,
+                            void *workspace, size_t ws_bytes, void *stream);
 
 /*
  * dsa_prefill_host -- dsa_prefill for inputs and outputs in HOST memory
@@ -465,6 +512,35 @@ dsa_status dsa_decode_noalloc(const void *q_idx, const float *q_scale, const voi
                               int64_t max_context, int H_I, int d_I, int H_q, int d, int k_sel,
                               float sm_scale, void *out, float *lse_out, int32_t *idx_out,
                               uint32_t *status_out, void *stream);
+
+/*
+ * Stage timing -- a tracing aid with no counterpart on the pages.  While
+ * enabled (process-wide), dsa_prefill and dsa_prefill_host record a pair of
+ * CUDA events on their stream around each stage's launches; the events are
+ * timed on the device, so enabling this does not synchronise the stream.
+ * dsa_profile_read waits for the recorded events, adds each stage's elapsed
+ * milliseconds into ms_out[stage] and the number of times the stage ran into
+ * launches_out[stage] (nullable), both arrays of DSA_STAGE_COUNT entries
+ * (the caller zeroes them), and forgets the records.  Do not enable it
+ * around a stream capture.  The events belong to
+ * the device that was current when they were recorded.
+ * Stages: the fused selection's sample scores, thresholds, select epilogue,
+ * finish and repair; the stand-alone indexer and top-k of the unfused
+ * prefill; the sparse attention.
+ */
+typedef enum dsa_stage {
+    DSA_STAGE_SAMPLE = 0,
+    DSA_STAGE_TAU = 1,
+    DSA_STAGE_SELECT = 2,
+    DSA_STAGE_FINISH = 3,
+    DSA_STAGE_REPAIR = 4,
+    DSA_STAGE_SCORES = 5,
+    DSA_STAGE_TOPK = 6,
+    DSA_STAGE_ATTN = 7,
+    DSA_STAGE_COUNT = 8
+} dsa_stage;
+dsa_status dsa_profile_enable(int on);
+dsa_status dsa_profile_read(double *ms_out, int64_t *launches_out);
 
 /*
  * dsa_stream_status -- waits for `stream`, then returns the device status

@@ -1,7 +1,9 @@
 // C entry points: argument validation, workspace carving, stage sequencing.
 // Everything numeric happens in the kernels; this file only checks and launches.
+#include <atomic>
 #include <cmath>
 #include <mutex>
+#include <vector>
 
 #include "kernels.h"
 
@@ -29,8 +31,195 @@ inline int64_t prefill_rows_default(int64_t T)
 
 inline size_t idx_bytes(int64_t rows, int k) { return align_up(sizeof(int32_t) * (size_t)rows * k, 256); }
 
+// ---- stage timing (dsa_profile_enable / dsa_profile_read)
+struct ProfRec {
+    int stage;
+    cudaEvent_t a, b;
+};
+struct Profiler {
+    std::mutex mu;
+    std::atomic<bool> on{false};
+    std::vector<ProfRec> recs;
+};
+Profiler &profiler()
+{
+    static Profiler p;
+    return p;
+}
+// Records an event pair on `st` around its scope when timing is enabled.
+class StageTimer {
+public:
+    StageTimer(int stage, cudaStream_t st) : stage_(stage), st_(st)
+    {
+        if (!profiler().on.load(std::memory_order_relaxed)) return;
+        if (cudaEventCreate(&a_) != cudaSuccess) { a_ = nullptr; return; }
+        if (cudaEventCreate(&b_) != cudaSuccess || cudaEventRecord(a_, st_) != cudaSuccess) {
+            cudaEventDestroy(a_);
+            if (b_) cudaEventDestroy(b_);
+            a_ = b_ = nullptr;
+        }
+    }
+    ~StageTimer()
+    {
+        if (!a_) return;
+        if (cudaEventRecord(b_, st_) != cudaSuccess) {
+            cudaEventDestroy(a_);
+            cudaEventDestroy(b_);
+            return;
+        }
+        std::lock_guard<std::mutex> g(profiler().mu);
+        profiler().recs.push_back({stage_, a_, b_});
+    }
+    StageTimer(const StageTimer &) = delete;
+    StageTimer &operator=(const StageTimer &) = delete;
+
+private:
+    int stage_;
+    cudaStream_t st_;
+    cudaEvent_t a_ = nullptr, b_ = nullptr;
+};
+
 // Largest sliding window (positions) the window entry points accept.
 constexpr int kMaxWindow = 1 << 24;
+
+// ---- fused prefill selection (the FP8 tcgen05 indexer with its select epilogue)
+// A pass of R query rows: sample scores -> per-row tau -> select epilogue
+// (candidates at or above tau) -> exact finish; rows whose candidate count
+// fell outside [k, cap] are recomputed by the score epilogue (only their row
+// blocks) and selected by the stand-alone top-k.  The repair's score rows
+// bound R: kRepairBudget bytes of them by default.
+constexpr int kSampleStride = 64;               // one sampled key per 64 positions
+constexpr int kFusedMaxK = 4096;                // larger k: the stand-alone top-k path
+constexpr size_t kRepairBudget = size_t(1) << 30;
+
+inline bool fused_ok(dsa_dtype dtype, int H_I, int64_t T, int k)
+{
+    return dtype == DSA_E4M3 && index_tc_supported(H_I) && T < ((int64_t)1 << 31) && k >= 1 && k <= kFusedMaxK;
+}
+inline int fused_cap(int k) { return 4 * k > 4096 ? 4 * k : 4096; }
+
+// The fused scratch for passes of R rows, carved after `base` bytes.
+struct FusedLayout {
+    int S = kSampleStride, cap = 0;
+    int64_t T = 0, M = 0, ldM = 0, R = 0;
+    size_t ks = 0, sks = 0, any = 0, ss = 0, tau = 0, cnt = 0, row_fail = 0, rb_fail = 0, cand = 0, scores = 0,
+           end = 0;
+    FusedLayout(int64_t T_, int k, int64_t R_, size_t base) : cap(fused_cap(k)), T(T_), R(R_)
+    {
+        M = sample_count(T, S);
+        ldM = (M + 3) / 4 * 4;
+        if (ldM < 4) ldM = 4;
+        size_t off = base;
+        auto take = [&](size_t bytes) { size_t o = off; off += align_up(bytes > 0 ? bytes : 1, 256); return o; };
+        ks = take((size_t)M * 128);
+        sks = take(sizeof(float) * (size_t)M);
+        any = take(sizeof(uint32_t));
+        ss = take(sizeof(float) * (size_t)R * ldM);
+        tau = take(sizeof(float) * (size_t)R);
+        cnt = take(sizeof(uint32_t) * (size_t)R * kCandCntStride);
+        row_fail = take(sizeof(uint32_t) * (size_t)R);
+        rb_fail = take(sizeof(uint32_t) * (size_t)ceil_div(R, 128));
+        cand = take(sizeof(uint2) * (size_t)R * cap);
+        scores = take(sizeof(float) * (size_t)R * T);
+        end = off;
+    }
+};
+
+inline int64_t fused_rows_max(int64_t T) { return ceil_div(T, 128) * 128; }
+// Default pass: at most kFusedRowsMax rows (the candidate lists take 32 KB
+// a row at k 2048) and kRepairBudget bytes of repair score rows.
+constexpr int64_t kFusedRowsMax = 4096;
+inline int64_t fused_rows_default(int64_t T)
+{
+    int64_t r = (int64_t)(kRepairBudget / (sizeof(float) * (size_t)T)) / 128 * 128;
+    if (r < 128) r = 128;
+    if (r > kFusedRowsMax) r = kFusedRowsMax;
+    return r < fused_rows_max(T) ? r : fused_rows_max(T);
+}
+// Largest R (a multiple of 128, at most T rounded up) whose layout fits ws_bytes; 0 if none.
+inline int64_t fused_rows_fitting(int64_t T, int k, size_t base, size_t ws_bytes)
+{
+    int64_t lo = 0, hi = fused_rows_max(T) / 128;        // in units of 128 rows
+    while (lo < hi) {
+        const int64_t mid = (lo + hi + 1) / 2;
+        if (FusedLayout(T, k, mid * 128, base).end <= ws_bytes) lo = mid; else hi = mid - 1;
+    }
+    return lo * 128;
+}
+
+// The sampled keys, once per sequence.
+cudaError_t fused_gather(const FusedLayout &L, uint8_t *ws, const void *k_idx, const float *k_scale, cudaStream_t st)
+{
+    return launch_gather_samples((const uint8_t *)k_idx, k_scale, L.M, L.S, ws + L.ks, (float *)(ws + L.sks), st);
+}
+
+// Selection of query rows [r0, r0 + n) (n <= L.R) into idx_rows (row r0 first,
+// k + window wide).  q_idx, q_scale and w hold positions [q_base, q_base +
+// q_rows) of the sequence; the key side holds positions [0, T).
+cudaError_t fused_select_pass(const FusedLayout &L, uint8_t *ws, const void *q_idx, const float *q_scale,
+                              const void *k_idx, const float *k_scale, const void *w, int64_t T, int H_I, int k,
+                              int window, int64_t r0, int64_t n, int32_t *idx_rows, WsHeader *hdr, cudaStream_t st,
+                              int64_t q_base = 0, int64_t q_rows = 0)
+{
+    float *ss = (float *)(ws + L.ss), *tau = (float *)(ws + L.tau), *scores = (float *)(ws + L.scores);
+    uint32_t *cnt = (uint32_t *)(ws + L.cnt), *row_fail = (uint32_t *)(ws + L.row_fail);
+    uint32_t *rb_fail = (uint32_t *)(ws + L.rb_fail), *any = (uint32_t *)(ws + L.any);
+    uint2 *cand = (uint2 *)(ws + L.cand);
+    const uint8_t *q8 = (const uint8_t *)q_idx, *k8 = (const uint8_t *)k_idx;
+    const uint16_t *wb = (const uint16_t *)w;
+    cudaError_t e = cudaSuccess;
+    // sample scores, needed only by rows with more competing positions than cap
+    if (r0 + n - window > L.cap) {
+        StageTimer tm(DSA_STAGE_SAMPLE, st);
+        IndexTcOpts o;
+        o.mode = IT_SAMPLE;
+        o.q_base = q_base;
+        o.q_rows = q_rows;
+        o.nkeys = L.M;
+        o.window = window;
+        o.sample_stride = L.S;
+        e = launch_index_tc(q8, q_scale, ws + L.ks, (const float *)(ws + L.sks), wb, T, H_I, r0, n, ss, L.ldM,
+                            false, hdr, st, &o);
+        if (e != cudaSuccess) return e;
+    }
+    {
+        StageTimer tm(DSA_STAGE_TAU, st);
+        e = launch_prefill_tau(ss, L.ldM, r0, n, k, window, L.S, L.cap, tau, cnt, row_fail, rb_fail, any, st);
+        if (e != cudaSuccess) return e;
+    }
+    {
+        StageTimer tm(DSA_STAGE_SELECT, st);
+        IndexTcOpts o;
+        o.mode = IT_SELECT;
+        o.q_base = q_base;
+        o.q_rows = q_rows;
+        o.window = window;
+        o.tau = tau;
+        o.cand = cand;
+        o.cand_cnt = cnt;
+        o.cap = L.cap;
+        e = launch_index_tc(q8, q_scale, k8, k_scale, wb, T, H_I, r0, n, nullptr, 0, false, hdr, st, &o);
+        if (e != cudaSuccess) return e;
+    }
+    {
+        StageTimer tm(DSA_STAGE_FINISH, st);
+        e = launch_prefill_finish(cand, L.cap, cnt, r0, n, k, window, idx_rows, row_fail, rb_fail, any, st);
+        if (e != cudaSuccess) return e;
+    }
+    // repair: scores of the flagged row blocks (nothing when none), stand-alone select of the flagged rows
+    StageTimer tm(DSA_STAGE_REPAIR, st);
+    {
+        IndexTcOpts o;
+        o.mode = IT_SCORES;
+        o.q_base = q_base;
+        o.q_rows = q_rows;
+        o.rb_mask = rb_fail;
+        o.any = any;
+        e = launch_index_tc(q8, q_scale, k8, k_scale, wb, T, H_I, r0, n, scores, T, false, hdr, st, &o);
+        if (e != cudaSuccess) return e;
+    }
+    return launch_topk_rows(scores, T, r0, nullptr, T, n, k, idx_rows, hdr, st, window, row_fail);
+}
 
 dsa_status check_index_args(const void *q_idx, const float *q_scale, const void *k_idx,
                             const float *k_scale, const void *w, int64_t T, int H_I, int d_I,
@@ -129,9 +318,12 @@ cudaError_t run_index(const void *q_idx, const float *q_scale, const void *k_idx
 struct HostPrefillLayout {
     size_t q_idx, q_scale, w, q, k_idx, k_scale, k, v, out, lse, idx, scores, total;
     int64_t R;
+    bool fused;                  // the fused selection's scratch follows the mirrors
+    FusedLayout F;
     HostPrefillLayout(int64_t T, int H_I, int d_I, int H_q, int d, int k_sel)
+        : fused(fused_ok(DSA_E4M3, H_I, T, k_sel)), F(1, 1, 0, 0)
     {
-        R = prefill_rows_default(T);
+        R = fused ? fused_rows_default(T) : prefill_rows_default(T);
         size_t off = kWsHeader;
         auto take = [&](size_t bytes) { size_t o = off; off += align_up(bytes, 256); return o; };
         q_idx = take((size_t)T * H_I * d_I);
@@ -145,8 +337,14 @@ struct HostPrefillLayout {
         out = take(2 * (size_t)T * H_q * d);
         lse = take(sizeof(float) * (size_t)T * H_q);
         idx = take(sizeof(int32_t) * (size_t)T * k_sel);
-        scores = take(sizeof(float) * (size_t)R * T);
-        total = off;
+        if (fused) {
+            F = FusedLayout(T, k_sel, R, off);
+            scores = F.scores;
+            total = F.end;
+        } else {
+            scores = take(sizeof(float) * (size_t)R * T);
+            total = off;
+        }
     }
 };
 
@@ -174,6 +372,29 @@ CopyEngine *copy_engine()
                cudaEventCreateWithFlags(&c.done, cudaEventDisableTiming) == cudaSuccess;
     });
     return engines[dev].ok ? &engines[dev] : nullptr;
+}
+
+// The fused prefill of query rows [row_begin, row_begin + rows) of a sequence
+// whose key side (k_idx, k_scale, k, v) holds positions [0, T): the query side
+// (q_idx, q_scale, w, q) and the outputs (out, lse, idx) hold those rows only.
+cudaError_t prefill_fused_rows(const FusedLayout &L, uint8_t *ws, const void *q_idx, const float *q_scale,
+                               const void *k_idx, const float *k_scale, const void *w, const void *q,
+                               const void *k, const void *v, int64_t T, int64_t row_begin, int64_t rows, int H_I,
+                               int H_q, int d, int k_sel, int window, float sm_scale, void *out, float *lse_out,
+                               int32_t *idx, WsHeader *hdr, cudaStream_t st)
+{
+    const int kw = k_sel + window;
+    cudaError_t e = fused_gather(L, ws, k_idx, k_scale, st);
+    for (int64_t r = 0; e == cudaSuccess && r < rows; r += L.R) {
+        const int64_t n = rows - r < L.R ? rows - r : L.R;
+        e = fused_select_pass(L, ws, q_idx, q_scale, k_idx, k_scale, w, T, H_I, k_sel, window, row_begin + r, n,
+                              idx + r * (int64_t)kw, hdr, st, row_begin, rows);
+    }
+    if (e == cudaSuccess) {
+        StageTimer tm(DSA_STAGE_ATTN, st);
+        e = run_attn_rows(q, k, v, idx, T, rows, H_q, d, kw, sm_scale, out, lse_out, st);
+    }
+    return e;
 }
 
 }  // namespace
@@ -257,8 +478,10 @@ dsa_status dsa_sparse_attn(const void *q, const void *k, const void *v, const in
 size_t dsa_prefill_workspace_size(int64_t T, int H_I, int d_I, int H_q, int d, int k_sel,
                                   dsa_dtype dtype)
 {
-    (void)H_I; (void)d_I; (void)H_q; (void)d; (void)dtype;
+    (void)d_I; (void)H_q; (void)d;
     if (T <= 0 || k_sel <= 0) return 0;
+    if (fused_ok(dtype, H_I, T, k_sel))
+        return FusedLayout(T, k_sel, fused_rows_default(T), kWsHeader + idx_bytes(T, k_sel)).end;
     int64_t R = prefill_rows_default(T);
     return kWsHeader + idx_bytes(T, k_sel) + align_up(sizeof(float) * (size_t)R * T, 256);
 }
@@ -286,6 +509,20 @@ dsa_status prefill_impl(const void *q_idx, const float *q_scale, const void *k_i
     if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u)) return DSA_ERR_WORKSPACE;
     const int kw = k_sel + window;                    // selection row width
     size_t fixed = kWsHeader + (idx_out ? 0 : idx_bytes(T, kw));
+    if (fused_ok(dtype, H_I, T, k_sel)) {
+        const int64_t R = fused_rows_fitting(T, k_sel, fixed, ws_bytes);
+        if (R < 128) return DSA_ERR_WORKSPACE;
+        const FusedLayout L(T, k_sel, R, fixed);
+        cudaStream_t st = as_stream(stream);
+        uint8_t *ws = static_cast<uint8_t *>(workspace);
+        WsHeader *hdr = reinterpret_cast<WsHeader *>(ws);
+        int32_t *idx = idx_out ? idx_out : reinterpret_cast<int32_t *>(ws + kWsHeader);
+        cudaError_t e = cudaMemsetAsync(hdr, 0, sizeof(WsHeader), st);
+        if (e == cudaSuccess)
+            e = prefill_fused_rows(L, ws, q_idx, q_scale, k_idx, k_scale, w, q, k, v, T, 0, T, H_I, H_q, d, k_sel,
+                                   window, sm_scale, out, lse_out, idx, hdr, st);
+        return cuda_status(e);
+    }
     if (ws_bytes < fixed + sizeof(float) * 64 * (size_t)T) return DSA_ERR_WORKSPACE;
     int64_t R = (int64_t)((ws_bytes - fixed) / (sizeof(float) * (size_t)T)) / 64 * 64;
     R = R < T ? R : ceil_div(T, 64) * 64;
@@ -298,14 +535,21 @@ dsa_status prefill_impl(const void *q_idx, const float *q_scale, const void *k_i
     cudaError_t e = cudaMemsetAsync(hdr, 0, sizeof(WsHeader), st);
     for (int64_t r0 = 0; e == cudaSuccess && r0 < T; r0 += R) {
         int64_t n = T - r0 < R ? T - r0 : R;
-        e = run_index(q_idx, q_scale, k_idx, k_scale, w, T, H_I, d_I, r0, n, scores, T, false,
-                      dtype, st);
-        if (e == cudaSuccess)
+        {
+            StageTimer tm(DSA_STAGE_SCORES, st);
+            e = run_index(q_idx, q_scale, k_idx, k_scale, w, T, H_I, d_I, r0, n, scores, T, false,
+                          dtype, st);
+        }
+        if (e == cudaSuccess) {
+            StageTimer tm(DSA_STAGE_TOPK, st);
             e = launch_topk_rows(scores, T, r0, nullptr, T, n, k_sel, idx + r0 * (int64_t)kw,
                                  hdr, st, window);
+        }
     }
-    if (e == cudaSuccess)
+    if (e == cudaSuccess) {
+        StageTimer tm(DSA_STAGE_ATTN, st);
         e = run_attn(q, k, v, idx, T, H_q, d, kw, sm_scale, out, lse_out, dtype, st);
+    }
     return cuda_status(e);
 }
 
@@ -332,6 +576,50 @@ dsa_status dsa_prefill_window(const void *q_idx, const float *q_scale, const voi
 {
     return prefill_impl(q_idx, q_scale, k_idx, k_scale, w, q, k, v, T, H_I, d_I, H_q, d, k_sel,
                         window, sm_scale, out, lse_out, idx_out, dtype, workspace, ws_bytes, stream);
+}
+
+size_t dsa_prefill_rows_workspace_size(int64_t T, int64_t row_count, int H_I, int d_I, int H_q, int d,
+                                       int k_sel, dsa_dtype dtype)
+{
+    (void)d_I; (void)H_q; (void)d;
+    if (T <= 0 || row_count <= 0 || row_count > T || !fused_ok(dtype, H_I, T, k_sel)) return 0;
+    const int64_t rmax = ceil_div(row_count, 128) * 128;
+    const int64_t R = fused_rows_default(T) < rmax ? fused_rows_default(T) : rmax;
+    return FusedLayout(T, k_sel, R, kWsHeader + idx_bytes(row_count, k_sel)).end;
+}
+
+dsa_status dsa_prefill_rows(const void *q_idx, const float *q_scale, const void *k_idx, const float *k_scale,
+                            const void *w, const void *q, const void *k, const void *v, int64_t T,
+                            int64_t row_begin, int64_t row_count, int H_I, int d_I, int H_q, int d, int k_sel,
+                            float sm_scale, void *out, float *lse_out, int32_t *idx_out, dsa_dtype dtype,
+                            void *workspace, size_t ws_bytes, void *stream)
+{
+    if (dtype != DSA_E4M3) return DSA_ERR_UNSUPPORTED;
+    if (row_begin < 0 || row_count < 0 || row_begin + row_count > T) return DSA_ERR_INVALID_ARG;
+    // the q-side arrays hold row_count rows: check them as a sequence of that length
+    dsa_status s = check_index_args(q_idx, q_scale, k_idx, k_scale, w, T, H_I, d_I, dtype);
+    if (s != DSA_OK) return s;
+    s = check_attn_args(q, k, v, reinterpret_cast<const int32_t *>(q), T, H_q, d, k_sel, out, dtype);
+    if (s != DSA_OK) return s;
+    if (k_sel > 65536 || !std::isfinite(sm_scale)) return DSA_ERR_INVALID_ARG;
+    if (!fused_ok(dtype, H_I, T, k_sel)) return DSA_ERR_UNSUPPORTED;
+    if (row_count == 0) return DSA_OK;
+    if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u)) return DSA_ERR_WORKSPACE;
+    const size_t fixed = kWsHeader + (idx_out ? 0 : idx_bytes(row_count, k_sel));
+    int64_t R = fused_rows_fitting(T, k_sel, fixed, ws_bytes);
+    const int64_t rmax = ceil_div(row_count, 128) * 128;
+    if (R > rmax) R = rmax;
+    if (R < 128) return DSA_ERR_WORKSPACE;
+    const FusedLayout L(T, k_sel, R, fixed);
+    cudaStream_t st = as_stream(stream);
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    WsHeader *hdr = reinterpret_cast<WsHeader *>(ws);
+    int32_t *idx = idx_out ? idx_out : reinterpret_cast<int32_t *>(ws + kWsHeader);
+    cudaError_t e = cudaMemsetAsync(hdr, 0, sizeof(WsHeader), st);
+    if (e == cudaSuccess)
+        e = prefill_fused_rows(L, ws, q_idx, q_scale, k_idx, k_scale, w, q, k, v, T, row_begin, row_count, H_I,
+                               H_q, d, k_sel, 0, sm_scale, out, lse_out, idx, hdr, st);
+    return cuda_status(e);
 }
 
 size_t dsa_prefill_host_workspace_size(int64_t T, int H_I, int d_I, int H_q, int d, int k_sel,
@@ -390,6 +678,12 @@ dsa_status dsa_prefill_host(const void *q_idx, const float *q_scale, const void 
     if (e == cudaSuccess) e = h2d(L.v, v, 2 * (size_t)T * d);
     if (e == cudaSuccess) e = h2d(L.q_scale, q_scale, sizeof(float) * (size_t)T);
     if (e == cudaSuccess) e = h2d(L.w, w, 2 * (size_t)T * H_I);
+    if (e == cudaSuccess && L.fused) {
+        // the sampled keys, once the keys have landed
+        e = cudaEventRecord(ce->in, ce->h2d);
+        if (e == cudaSuccess) e = cudaStreamWaitEvent(st, ce->in, 0);
+        if (e == cudaSuccess) e = fused_gather(L.F, ws, ws + L.k_idx, (const float *)(ws + L.k_scale), st);
+    }
     // Passes run from the last rows to the first: late rows carry the most work per
     // copied byte (their causal rows are longest), so the copies stay ahead of the
     // computation from the start, and the last pass's outputs are the cheapest.
@@ -401,16 +695,28 @@ dsa_status dsa_prefill_host(const void *q_idx, const float *q_scale, const void 
         if (e == cudaSuccess) e = h2d(L.q + r0 * q_row, static_cast<const uint8_t *>(q) + r0 * q_row, n * q_row);
         if (e == cudaSuccess) e = cudaEventRecord(ce->in, ce->h2d);
         if (e == cudaSuccess) e = cudaStreamWaitEvent(st, ce->in, 0);
-        if (e == cudaSuccess)
-            e = run_index(ws + L.q_idx, (const float *)(ws + L.q_scale), ws + L.k_idx,
-                          (const float *)(ws + L.k_scale), ws + L.w, T, H_I, d_I, r0, n, scores, T, false,
-                          dtype, st);
-        if (e == cudaSuccess)
-            e = launch_topk_rows(scores, T, r0, nullptr, T, n, k_sel, idx + r0 * (int64_t)k_sel, hdr, st);
-        if (e == cudaSuccess)
+        if (e == cudaSuccess && L.fused) {
+            e = fused_select_pass(L.F, ws, ws + L.q_idx, (const float *)(ws + L.q_scale), ws + L.k_idx,
+                                  (const float *)(ws + L.k_scale), ws + L.w, T, H_I, k_sel, 0, r0, n,
+                                  idx + r0 * (int64_t)k_sel, hdr, st);
+        } else {
+            if (e == cudaSuccess) {
+                StageTimer tm(DSA_STAGE_SCORES, st);
+                e = run_index(ws + L.q_idx, (const float *)(ws + L.q_scale), ws + L.k_idx,
+                              (const float *)(ws + L.k_scale), ws + L.w, T, H_I, d_I, r0, n, scores, T, false,
+                              dtype, st);
+            }
+            if (e == cudaSuccess) {
+                StageTimer tm(DSA_STAGE_TOPK, st);
+                e = launch_topk_rows(scores, T, r0, nullptr, T, n, k_sel, idx + r0 * (int64_t)k_sel, hdr, st);
+            }
+        }
+        if (e == cudaSuccess) {
+            StageTimer tm(DSA_STAGE_ATTN, st);
             e = run_attn_rows(ws + L.q + r0 * q_row, ws + L.k, ws + L.v, idx + r0 * (int64_t)k_sel, T, n, H_q,
                               d, k_sel, sm_scale, ws + L.out + r0 * q_row,
                               reinterpret_cast<float *>(ws + L.lse) + r0 * H_q, st);
+        }
         if (e == cudaSuccess) e = cudaEventRecord(ce->out, st);
         if (e == cudaSuccess) e = cudaStreamWaitEvent(ce->d2h, ce->out, 0);
         if (e == cudaSuccess)
@@ -807,6 +1113,35 @@ dsa_status dsa_cache_append_kv8(const void *kidx_new, dsa_dtype kidx_dtype, cons
                                            max_pages_per_seq, num_pages, page_size, d_I, d,
                                            (uint8_t *)kidx_cache, kscale_cache, k_cache, v_cache, k_cache_scale,
                                            v_cache_scale, status, as_stream(stream)));
+}
+
+dsa_status dsa_profile_enable(int on)
+{
+    profiler().on.store(on != 0);
+    return DSA_OK;
+}
+
+dsa_status dsa_profile_read(double *ms_out, int64_t *launches_out)
+{
+    if (!ms_out) return DSA_ERR_INVALID_ARG;
+    std::vector<ProfRec> recs;
+    {
+        std::lock_guard<std::mutex> g(profiler().mu);
+        recs.swap(profiler().recs);
+    }
+    dsa_status s = DSA_OK;
+    for (const ProfRec &r : recs) {
+        float ms = 0.f;
+        if (s == DSA_OK && (cudaEventSynchronize(r.b) != cudaSuccess || cudaEventElapsedTime(&ms, r.a, r.b) != cudaSuccess))
+            s = DSA_ERR_CUDA;
+        if (s == DSA_OK && r.stage >= 0 && r.stage < DSA_STAGE_COUNT) {
+            ms_out[r.stage] += ms;
+            if (launches_out) launches_out[r.stage] += 1;
+        }
+        cudaEventDestroy(r.a);
+        cudaEventDestroy(r.b);
+    }
+    return s;
 }
 
 dsa_status dsa_stream_status(void *workspace, void *stream)

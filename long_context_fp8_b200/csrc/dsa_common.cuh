@@ -59,6 +59,32 @@ inline cudaError_t launch_chained(void (*kernel)(KArgs...), dim3 grid, dim3 bloc
     return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
 }
 
+// Sampled key positions of the fused prefill selection's threshold estimate:
+// sample j sits at position j * S + (hash(j) mod S) (S a power of two), one
+// pseudo-random point of each block of S positions, so that no periodic
+// pattern in the keys lines up with the samples.  The hash is the 32-bit
+// finaliser of MurmurHash3 (Appleby), applied to j.
+__host__ __device__ inline uint32_t sample_hash(uint32_t j)
+{
+    j ^= j >> 16;
+    j *= 0x85ebca6bu;
+    j ^= j >> 13;
+    j *= 0xc2b2ae35u;
+    j ^= j >> 16;
+    return j;
+}
+__host__ __device__ inline int64_t sample_pos(int64_t j, int S)
+{
+    return j * S + (int64_t)(sample_hash((uint32_t)j) & (uint32_t)(S - 1));
+}
+// Number of samples at positions < n (positions increase with j).
+__host__ __device__ inline int64_t sample_count(int64_t n, int S)
+{
+    if (n <= 0) return 0;
+    const int64_t j = (n - 1) / S;
+    return j + ((int64_t)(sample_hash((uint32_t)j) & (uint32_t)(S - 1)) <= n - 1 - j * S ? 1 : 0);
+}
+
 __device__ __forceinline__ float bf16_to_f32(uint16_t b)
 {
     return __uint_as_float(((uint32_t)b) << 16);

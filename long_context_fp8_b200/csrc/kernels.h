@@ -17,10 +17,30 @@ cudaError_t launch_index_fp8(const uint8_t *q8, const float *sq, const uint8_t *
                              int64_t row_begin, int64_t row_count, float *out, int64_t ld,
                              bool write_upper, cudaStream_t st);
 bool index_tc_supported(int H);
+// Epilogue modes of the tcgen05 indexer (index_tc.cu).
+enum IndexTcMode { IT_SCORES = 0, IT_SAMPLE = 1, IT_SELECT = 2 };
+constexpr int kCandCntStride = 32;      // uint32 words per candidate counter (one per 128 bytes)
+struct IndexTcOpts {
+    int mode = IT_SCORES;
+    int64_t nkeys = 0;                  // keys of k8/sk (0: T); the sample count in IT_SAMPLE
+    int window = 0;                     // IT_SAMPLE, IT_SELECT: competing positions [0, t + 1 - window)
+    int sample_stride = 0;              // IT_SAMPLE: S (a power of two; see sample_pos)
+    const float *tau = nullptr;         // IT_SELECT: [row_count] thresholds
+    uint2 *cand = nullptr;              // IT_SELECT: [row_count][cap] (score bits, position)
+    uint32_t *cand_cnt = nullptr;       // IT_SELECT: [row_count * kCandCntStride], zero before
+    int cap = 0;
+    const uint32_t *rb_mask = nullptr;  // IT_SCORES: visit only row blocks (128 rows) flagged here
+    const uint32_t *any = nullptr;      // IT_SCORES: do nothing when *any == 0
+    int64_t q_base = 0;                 // q8, sq and w hold positions [q_base, q_base + q_rows)
+    int64_t q_rows = 0;                 // 0: T - q_base
+};
+// IT_SCORES writes out[(t-row_begin)*ld + s] for s <= t; IT_SAMPLE writes
+// out[(t-row_begin)*ld + j] for the samples j before the row's window (k8/sk
+// are the gathered samples); IT_SELECT appends candidates, out unused.
 cudaError_t launch_index_tc(const uint8_t *q8, const float *sq, const uint8_t *k8, const float *sk,
                             const uint16_t *w, int64_t T, int H, int64_t row_begin,
                             int64_t row_count, float *out, int64_t ld, bool write_upper,
-                            WsHeader *hdr, cudaStream_t st);
+                            WsHeader *hdr, cudaStream_t st, const IndexTcOpts *opts = nullptr);
 cudaError_t launch_index_f32(const float *q, const float *k, const float *w, int64_t T, int H,
                              int D, int64_t row_begin, int64_t row_count, float *out,
                              int64_t ld, bool write_upper, cudaStream_t st);
@@ -31,9 +51,27 @@ cudaError_t launch_index_f32(const float *q, const float *k, const float *w, int
 // ascending, -1 padded.  With window > 0 only s < n_r - window compete and
 // the window positions follow the selected ones.  Rows with lens[r] outside
 // [1, max_len] are skipped (set to -1) and reported in hdr.
+// row_mask (nullable): only rows r with row_mask[r] != 0 are selected.
 cudaError_t launch_topk_rows(const float *scores, int64_t ld, int64_t row_begin,
                              const int32_t *lens, int64_t max_len, int64_t row_count, int k,
-                             int32_t *idx, WsHeader *hdr, cudaStream_t st, int window = 0);
+                             int32_t *idx, WsHeader *hdr, cudaStream_t st, int window = 0,
+                             const uint32_t *row_mask = nullptr);
+
+// ---- fused prefill selection (index_tc.cu, topk.cu) ----
+// Gathers the M = sample_count(T, S) sampled index keys and their scales.
+cudaError_t launch_gather_samples(const uint8_t *k8, const float *sk, int64_t M, int S, uint8_t *ks,
+                                  float *sks, cudaStream_t st);
+// Per row of the pass: tau from the sample scores ss[r * ld + j], the
+// candidate counter zeroed, the repair flags cleared.
+cudaError_t launch_prefill_tau(const float *ss, int64_t ld, int64_t row_begin, int64_t rows, int k, int window,
+                               int S, int cap, float *tau, uint32_t *cnt, uint32_t *row_fail, uint32_t *rb_fail,
+                               uint32_t *any_fail, cudaStream_t st);
+// Per row: the exact selection from its candidates into idx[r * (k + window)],
+// or the row flagged in row_fail / rb_fail (per 128 rows) / any_fail.
+size_t prefill_finish_smem(int cap);
+cudaError_t launch_prefill_finish(const uint2 *cand, int cap, const uint32_t *cnt, int64_t row_begin, int64_t rows,
+                                  int k, int window, int32_t *idx, uint32_t *row_fail, uint32_t *rb_fail,
+                                  uint32_t *any_fail, cudaStream_t st);
 
 // Rows of lengths lens[r] (decode): each row split over CTAs of 16384
 // positions that share a sampled threshold and collect their candidates, then

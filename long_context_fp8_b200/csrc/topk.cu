@@ -648,7 +648,7 @@ __device__ __forceinline__ bool emit_whole_row(int32_t *out, int k, int window, 
 __global__ void __launch_bounds__(RowsCfg::NT, 2)
 topk_rows_kernel(const float *__restrict__ scores, int64_t ld, int64_t row_begin,
                  const int32_t *__restrict__ lens, int64_t max_len, int k, int window,
-                 int32_t *__restrict__ idx, WsHeader *hdr, int vec_ok)
+                 int32_t *__restrict__ idx, WsHeader *hdr, int vec_ok, const uint32_t *__restrict__ row_mask)
 {
     using C = RowsCfg;
     extern __shared__ __align__(16) uint8_t smem_raw[];
@@ -656,6 +656,7 @@ topk_rows_kernel(const float *__restrict__ scores, int64_t ld, int64_t row_begin
 
     const int64_t r = blockIdx.x;
     const int tid = threadIdx.x;
+    if (row_mask && row_mask[r] == 0u) return;        // only the rows flagged for repair
     const float *row = scores + r * ld;
     int32_t *out = idx + r * (int64_t)(k + window);
     int64_t n_all;
@@ -845,11 +846,204 @@ topk_split_final_kernel(const float *__restrict__ scores, int64_t ld, const int3
     }
 }
 
+// ---------------------------------------------------------------- fused prefill selection
+// The prefill indexer's select epilogue appends, for each query row, every
+// competing position whose score is at or above the row's threshold tau, as
+// (score bits, position), in no particular order.  tau comes from the scores
+// of a sample of the keys (one pseudo-random position per S): with m samples
+// before the row's window and n competing positions, lam = k m / n samples
+// are expected above the k-th largest score, and tau is the sample of rank
+// lam + 6 sqrt(lam) + 2, which leaves about that many times S candidates
+// and falls short of k only with probability near 2e-8 per row.  A row
+// whose count lies outside [k, cap] is flagged; the caller then recomputes
+// its scores and runs the stand-alone select on it, so every row is exact.
+
+// Rank of tau among the m samples of a row of n competing positions.
+__host__ __device__ inline uint32_t tau_rank(int k, int64_t m, int64_t n)
+{
+    const double lam = (double)k * (double)m / (double)n;
+    double r = ceil(lam + 6.0 * sqrt(lam) + 2.0);
+    if (r > (double)m) r = (double)m;
+    return r < 1.0 ? 1u : (uint32_t)r;
+}
+
+// One warp per row: tau (+inf when the whole row is selected without scores,
+// -inf when every competing position fits the candidate list), and the
+// row's candidate counter and repair flags cleared for the select pass.
+// The rank-th largest sample key is found by bisection over the key range:
+// 32 steps of a warp-wide count, the keys held in registers (m <= 2048) or
+// re-read from the sample scores.
+constexpr int TAU_WARPS = 8;
+constexpr int TAU_REG = 64;                      // keys per lane held in registers
+
+__global__ void __launch_bounds__(TAU_WARPS * 32)
+prefill_tau_kernel(const float *__restrict__ ss, int64_t ld, int64_t row_begin, int64_t rows, int k, int window,
+                   int S, int cap, float *__restrict__ tau, uint32_t *__restrict__ cnt,
+                   uint32_t *__restrict__ row_fail, uint32_t *__restrict__ rb_fail, uint32_t *__restrict__ any_fail)
+{
+    const int lane = threadIdx.x & 31;
+    const int64_t r = (int64_t)blockIdx.x * TAU_WARPS + (threadIdx.x >> 5);
+    if (r >= rows) return;
+    const int64_t t = row_begin + r;
+    const int64_t n = t + 1 - window > 0 ? t + 1 - window : 0;
+    float tv;
+    if (n <= k) {
+        tv = INFINITY;
+    } else if (n <= cap) {
+        tv = -INFINITY;
+    } else {
+        const int64_t m = sample_count(n, S);
+        const uint32_t rank = tau_rank(k, m, n);
+        const float *row = ss + r * ld;
+        uint32_t lo = 0u, hi = 0xffffffffu;              // count(key >= lo) >= rank throughout
+        if (m <= 32 * TAU_REG) {
+            uint32_t kv[TAU_REG];
+#pragma unroll
+            for (int i = 0; i < TAU_REG; ++i) {
+                const int64_t j = lane + 32 * i;
+                kv[i] = j < m ? float_key(row[j]) : 0u;      // key 0 is no score's key
+            }
+            while (lo < hi) {
+                const uint32_t mid = lo + ((hi - lo) >> 1) + 1u;
+                uint32_t c = 0;
+#pragma unroll
+                for (int i = 0; i < TAU_REG; ++i) c += kv[i] >= mid;
+                c = __reduce_add_sync(0xffffffffu, c);
+                if (c >= rank) lo = mid; else hi = mid - 1u;
+            }
+        } else {
+            while (lo < hi) {
+                const uint32_t mid = lo + ((hi - lo) >> 1) + 1u;
+                uint32_t c = 0;
+                for (int64_t j = lane; j < m; j += 32) c += float_key(row[j]) >= mid;
+                c = __reduce_add_sync(0xffffffffu, c);
+                if (c >= rank) lo = mid; else hi = mid - 1u;
+            }
+        }
+        tv = key_float(lo);
+    }
+    if (lane == 0) {
+        tau[r] = tv;
+        cnt[r * kCandCntStride] = 0u;
+        row_fail[r] = 0u;
+        if ((r & 127) == 0) rb_fail[r >> 7] = 0u;
+        if (r == 0) *any_fail = 0u;
+    }
+}
+
+// One CTA per row: the exact top-k of the row's candidates, emitted in
+// ascending position order (the window, if any, after them).  The k-th
+// largest key thr and the number `need` of keys equal to thr that rank
+// within the top k come from the radix select; the emit then marks the
+// positions of keys above thr, and of keys equal to thr, in two bitmaps of a
+// 65536-position window, takes the `need` lowest equal ones, and writes the
+// marked positions in order through block-wide prefix counts.
+using FinCfg = TopkCfg<256, 256, 8, false>;
+constexpr int FIN_WIN_WORDS = 2048;                  // 65536 positions per emit window
+
+__host__ __device__ inline size_t finish_smem_bytes(int cap)
+{
+    return align_up(sizeof(TopkSmem<FinCfg>), 16) + sizeof(uint32_t) * (FIN_WIN_WORDS + (size_t)cap);
+}
+
+__global__ void __launch_bounds__(FinCfg::NT)
+prefill_finish_kernel(const uint2 *__restrict__ cand, int cap, const uint32_t *__restrict__ cnt, int64_t row_begin,
+                      int k, int window, int32_t *__restrict__ idx, uint32_t *__restrict__ row_fail,
+                      uint32_t *__restrict__ rb_fail, uint32_t *__restrict__ any_fail)
+{
+    using C = FinCfg;
+    extern __shared__ __align__(16) uint8_t smem_raw[];
+    TopkSmem<C> &sm = *reinterpret_cast<TopkSmem<C> *>(smem_raw);
+    uint32_t *eqbm = reinterpret_cast<uint32_t *>(smem_raw + align_up(sizeof(TopkSmem<C>), 16));
+    uint32_t *keys = eqbm + FIN_WIN_WORDS;
+    uint32_t *gtbm = sm.hist;                        // free once the select is done
+    static_assert(sizeof(sm.hist) / sizeof(uint32_t) == FIN_WIN_WORDS, "bitmap window");
+
+    const int tid = threadIdx.x;
+    const int64_t r = blockIdx.x;
+    const int64_t n_all = row_begin + r + 1;
+    const int64_t n = before_window(n_all, window);
+    int32_t *out = idx + r * (int64_t)(k + window);
+    if (emit_whole_row<C>(out, k, window, n, n_all)) return;
+    emit_window<C>(out, k, window, n);
+    const uint32_t c = cnt[r * kCandCntStride];
+    if (c < (uint32_t)k || c > (uint32_t)cap) {
+        if (tid == 0) {                              // the repair pass takes this row
+            row_fail[r] = 1u;
+            atomicOr(rb_fail + (r >> 7), 1u);
+            atomicOr(any_fail, 1u);
+        }
+        return;
+    }
+    const uint2 *cr = cand + r * (int64_t)cap;
+    for (uint32_t i = tid; i < c; i += C::NT) keys[i] = float_key(__uint_as_float(cr[i].x));
+    __syncthreads();
+    uint32_t thr, need;
+    radix_select_smem(sm, keys, c, (uint32_t)k, &thr, &need);
+    __syncthreads();
+
+    uint32_t eq_base = 0, out_base = 0;              // block-uniform
+    for (int64_t w0 = 0; w0 < n; w0 += 32 * FIN_WIN_WORDS) {
+        for (int i = tid; i < FIN_WIN_WORDS; i += C::NT) { gtbm[i] = 0u; eqbm[i] = 0u; }
+        __syncthreads();
+        for (uint32_t i = tid; i < c; i += C::NT) {
+            const uint32_t key = keys[i];
+            if (key >= thr) {
+                const int64_t off = (int64_t)cr[i].y - w0;
+                if (off >= 0 && off < 32 * FIN_WIN_WORDS)
+                    atomicOr((key > thr ? gtbm : eqbm) + (off >> 5), 1u << (off & 31));
+            }
+        }
+        __syncthreads();
+        constexpr int WPT = FIN_WIN_WORDS / C::NT;   // words per thread, consecutive
+        uint32_t g[WPT], e[WPT], ecnt = 0;
+#pragma unroll
+        for (int q = 0; q < WPT; ++q) {
+            g[q] = gtbm[tid * WPT + q];
+            e[q] = eqbm[tid * WPT + q];
+            ecnt += (uint32_t)__popc(e[q]);
+        }
+        uint32_t etot;
+        uint32_t ebefore = eq_base + block_excl_scan<C>(ecnt, sm.warp_buf, &etot);
+        uint32_t scnt = 0;
+#pragma unroll
+        for (int q = 0; q < WPT; ++q) {
+            // the equal keys are taken in position order until `need` of them are
+            uint32_t x = e[q], taken = 0;
+            while (x && ebefore < need) {
+                const uint32_t lb = x & (0u - x);
+                taken |= lb;
+                x ^= lb;
+                ++ebefore;
+            }
+            ebefore += (uint32_t)__popc(x);
+            g[q] |= taken;
+            scnt += (uint32_t)__popc(g[q]);
+        }
+        uint32_t stot;
+        uint32_t o = out_base + block_excl_scan<C>(scnt, sm.warp_buf, &stot);
+#pragma unroll
+        for (int q = 0; q < WPT; ++q) {
+            uint32_t x = g[q];
+            while (x) {
+                const int b = __ffs(x) - 1;
+                x &= x - 1;
+                if (o < (uint32_t)k) out[o] = (int32_t)(w0 + (int64_t)(tid * WPT + q) * 32 + b);
+                ++o;
+            }
+        }
+        eq_base += etot;
+        out_base += stot;
+        __syncthreads();
+    }
+}
+
 }  // namespace
 
 cudaError_t launch_topk_rows(const float *scores, int64_t ld, int64_t row_begin,
                              const int32_t *lens, int64_t max_len, int64_t row_count, int k,
-                             int32_t *idx, WsHeader *hdr, cudaStream_t st, int window)
+                             int32_t *idx, WsHeader *hdr, cudaStream_t st, int window,
+                             const uint32_t *row_mask)
 {
     if (row_count <= 0) return cudaSuccess;
     const size_t smem = sizeof(TopkSmem<RowsCfg>);
@@ -858,7 +1052,8 @@ cudaError_t launch_topk_rows(const float *scores, int64_t ld, int64_t row_begin,
     if (e != cudaSuccess) return e;
     const int vec_ok = (ld % 4 == 0) && ((reinterpret_cast<uintptr_t>(scores) & 15u) == 0);
     topk_rows_kernel<<<(unsigned)row_count, RowsCfg::NT, smem, st>>>(scores, ld, row_begin, lens,
-                                                                     max_len, k, window, idx, hdr, vec_ok);
+                                                                     max_len, k, window, idx, hdr, vec_ok,
+                                                                     row_mask);
     return cudaGetLastError();
 }
 
@@ -896,6 +1091,33 @@ cudaError_t launch_topk_split(const float *scores, int64_t ld, const int32_t *le
     e = launch_chained(topk_split_final_kernel, dim3((unsigned)rows), dim3(SplitCfg::NT), smem, st, scores,
                        ld, lens, max_len, k, window, ws, idx, hdr, vec_ok);
     if (e != cudaSuccess) return e;
+    return cudaGetLastError();
+}
+
+
+cudaError_t launch_prefill_tau(const float *ss, int64_t ld, int64_t row_begin, int64_t rows, int k, int window,
+                               int S, int cap, float *tau, uint32_t *cnt, uint32_t *row_fail, uint32_t *rb_fail,
+                               uint32_t *any_fail, cudaStream_t st)
+{
+    if (rows <= 0) return cudaSuccess;
+    prefill_tau_kernel<<<(unsigned)ceil_div(rows, TAU_WARPS), TAU_WARPS * 32, 0, st>>>(
+        ss, ld, row_begin, rows, k, window, S, cap, tau, cnt, row_fail, rb_fail, any_fail);
+    return cudaGetLastError();
+}
+
+size_t prefill_finish_smem(int cap) { return finish_smem_bytes(cap); }
+
+cudaError_t launch_prefill_finish(const uint2 *cand, int cap, const uint32_t *cnt, int64_t row_begin, int64_t rows,
+                                  int k, int window, int32_t *idx, uint32_t *row_fail, uint32_t *rb_fail,
+                                  uint32_t *any_fail, cudaStream_t st)
+{
+    if (rows <= 0) return cudaSuccess;
+    const size_t smem = finish_smem_bytes(cap);
+    cudaError_t e = cudaFuncSetAttribute(prefill_finish_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem);
+    if (e != cudaSuccess) return e;
+    prefill_finish_kernel<<<(unsigned)rows, FinCfg::NT, smem, st>>>(cand, cap, cnt, row_begin, k, window, idx,
+                                                                   row_fail, rb_fail, any_fail);
     return cudaGetLastError();
 }
 

@@ -29,7 +29,8 @@ EXPORTS = ("dsa_status_string", "dsa_version", "dsa_index_scores", "dsa_topk_wor
            "dsa_decode_workspace_size", "dsa_decode", "dsa_decode_window", "dsa_decode_kv8",
            "dsa_quantize_e4m3", "dsa_cache_append", "dsa_cache_append_kv8", "dsa_decode_noalloc",
            "dsa_split_workspace_size", "dsa_decode_select", "dsa_merge_selections", "dsa_decode_attend",
-           "dsa_merge_partials", "dsa_stream_status")
+           "dsa_merge_partials", "dsa_stream_status", "dsa_profile_enable", "dsa_profile_read",
+           "dsa_prefill_rows_workspace_size", "dsa_prefill_rows")
 
 
 class DSAError(RuntimeError):
@@ -90,6 +91,11 @@ def load(path: str = LIB_PATH):
                               I32),
         "dsa_merge_partials": ([P, I64, P, I64, I32, I32, I32, I32, P, P, P], I32),
         "dsa_stream_status": ([P, P], I32),
+        "dsa_profile_enable": ([I32], I32),
+        "dsa_prefill_rows_workspace_size": ([I64, I64, I32, I32, I32, I32, I32, I32], SZ),
+        "dsa_prefill_rows": ([P, P, P, P, P, P, P, P, I64, I64, I64, I32, I32, I32, I32, I32, F, P, P, P, I32, P,
+                              SZ, P], I32),
+        "dsa_profile_read": ([P, P], I32),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -286,6 +292,39 @@ def dsa_prefill_window(inp: dict, k_sel: int, window: int, sm_scale=None, out=No
                                 k_sel, window, sm_scale, _p(out), _p(lse), _p(idx_out), dt, _p(ws),
                                 ws.numel(), _stream(stream))
     _check("dsa_prefill_window", st)
+    return out, lse, idx_out
+
+
+def prefill_rows_workspace_size(T, row_count, H_I, d_I, H_q, d, k_sel) -> int:
+    return load().dsa_prefill_rows_workspace_size(T, row_count, H_I, d_I, H_q, d, k_sel, DSA_E4M3)
+
+
+def dsa_prefill_rows(rows: dict, keys: dict, row_begin: int, k_sel: int, sm_scale=None, out=None, lse=None,
+                     idx_out=None, ws=None, stream=None):
+    """The fused prefill of query rows [row_begin, row_begin + n) of a sequence:
+    ``rows`` holds those rows' q_idx [n, H_I, d_I], q_scale [n], w [n, H_I] and
+    q [n, H_q, d]; ``keys`` the k_idx [T, d_I], k_scale [T], k and v [T, d] of
+    every position.  Returns (out, lse, idx) of the n rows."""
+    q_idx, q = rows["q_idx"], rows["q"]
+    n, H_I, d_I = q_idx.shape
+    _, H_q, d = q.shape
+    T = keys["k_idx"].shape[0]
+    sm_scale = 1.0 / math.sqrt(d) if sm_scale is None else sm_scale
+    lib = load()
+    if ws is None:
+        ws = workspace(max(1, lib.dsa_prefill_rows_workspace_size(T, n, H_I, d_I, H_q, d, k_sel, DSA_E4M3)),
+                       q.device)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((n, H_q), dtype=torch.float32, device=q.device)
+    if idx_out is None:
+        idx_out = torch.empty((n, k_sel), dtype=torch.int32, device=q.device)
+    st = lib.dsa_prefill_rows(_p(q_idx), _p(rows["q_scale"]), _p(keys["k_idx"]), _p(keys["k_scale"]),
+                              _p(rows["w"]), _p(q), _p(keys["k"]), _p(keys["v"]), T, row_begin, n, H_I, d_I,
+                              H_q, d, k_sel, sm_scale, _p(out), _p(lse), _p(idx_out), DSA_E4M3, _p(ws),
+                              ws.numel(), _stream(stream))
+    _check("dsa_prefill_rows", st)
     return out, lse, idx_out
 
 
@@ -551,3 +590,22 @@ def dsa_merge_partials(part_out, part_lse, out=None, lse=None, stream=None):
 def dsa_stream_status(ws: torch.Tensor, stream=None) -> int:
     """Synchronise the stream and return (and clear) the workspace's device status."""
     return load().dsa_stream_status(_p(ws), _stream(stream))
+
+
+# Stage names of dsa_profile_read, in dsa_stage order.
+STAGES = ("sample", "tau", "select", "finish", "repair", "scores", "topk", "attention")
+
+
+def profile_enable(on: bool = True):
+    """Turn the library's per-stage CUDA-event timing on or off (process-wide)."""
+    _check("dsa_profile_enable", load().dsa_profile_enable(1 if on else 0))
+
+
+def profile_read():
+    """Device milliseconds and run counts per stage recorded since the last
+    read (waits for the recorded events): {stage: (ms, runs)}."""
+    ms = (ctypes.c_double * len(STAGES))()
+    n = (ctypes.c_int64 * len(STAGES))()
+    _check("dsa_profile_read", load().dsa_profile_read(ctypes.cast(ms, ctypes.c_void_p),
+                                                       ctypes.cast(n, ctypes.c_void_p)))
+    return {name: (ms[i], n[i]) for i, name in enumerate(STAGES)}

@@ -214,3 +214,17 @@ def test_header_compiles_as_c_and_library_links(lib, tmp_path):
                    capture_output=True, text=True)
     r = subprocess.run([exe], capture_output=True, text=True)
     assert r.returncode == 0 and r.stdout.strip() == "ok", (r.returncode, r.stdout, r.stderr)
+
+
+def test_prefill_workspace_is_linear_in_the_sequence_length(lib):
+    """The fused selection keeps no T x T score matrix: beyond the selection
+    itself (T x k indices) the workspace stays within a fixed budget, so it
+    grows linearly with T instead of quadratically."""
+    from long_context_fp8_b200 import dsa
+    k = 2048
+    sizes = {T: lib.dsa_prefill_workspace_size(T, 64, 128, 128, 128, k, dsa.DSA_E4M3)
+             for T in (1 << 17, 1 << 18, 1 << 19)}
+    for T, size in sizes.items():
+        assert size - T * k * 4 < (3 << 29), (T, size)     # under 1.5 GiB besides the indices
+    assert sizes[1 << 18] < 2.2 * sizes[1 << 17]
+    assert sizes[1 << 19] < 2.2 * sizes[1 << 18]
