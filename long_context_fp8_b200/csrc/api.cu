@@ -91,6 +91,9 @@ constexpr int kMaxWindow = 1 << 24;
 constexpr int kSampleStride = 64;               // one sampled key per 64 positions
 constexpr int kFusedMaxK = 4096;                // larger k: the stand-alone top-k path
 constexpr size_t kRepairBudget = size_t(1) << 30;
+// Sample scores of up to kSampleBudget bytes of query rows are computed in one
+// launch (several passes' worth), which keeps that small launch's grid full.
+constexpr size_t kSampleBudget = size_t(128) << 20;
 
 inline bool fused_ok(dsa_dtype dtype, int H_I, int64_t T, int k)
 {
@@ -101,23 +104,29 @@ inline int fused_cap(int k) { return 4 * k > 4096 ? 4 * k : 4096; }
 // The fused scratch for passes of R rows, carved after `base` bytes.
 struct FusedLayout {
     int S = kSampleStride, cap = 0;
-    int64_t T = 0, M = 0, ldM = 0, R = 0;
-    size_t ks = 0, sks = 0, any = 0, ss = 0, tau = 0, cnt = 0, row_fail = 0, rb_fail = 0, cand = 0, scores = 0,
-           end = 0;
+    int64_t T = 0, M = 0, ldM = 0, R = 0, SG = 0;   // SG: rows of sample scores held (a multiple of R)
+    size_t ks = 0, sks = 0, fail_cnt = 0, ss = 0, tau = 0, cnt = 0, fail_list = 0, rb_fail = 0, cand = 0,
+           scores = 0, end = 0;
     FusedLayout(int64_t T_, int k, int64_t R_, size_t base) : cap(fused_cap(k)), T(T_), R(R_)
     {
         M = sample_count(T, S);
         ldM = (M + 3) / 4 * 4;
         if (ldM < 4) ldM = 4;
+        SG = R;
+        if (R > 0) {
+            const int64_t groups = (int64_t)(kSampleBudget / (sizeof(float) * (size_t)ldM)) / R;
+            const int64_t need = ceil_div(T, R);
+            SG = R * (groups < 1 ? 1 : (groups < need ? groups : need));
+        }
         size_t off = base;
         auto take = [&](size_t bytes) { size_t o = off; off += align_up(bytes > 0 ? bytes : 1, 256); return o; };
         ks = take((size_t)M * 128);
         sks = take(sizeof(float) * (size_t)M);
-        any = take(sizeof(uint32_t));
-        ss = take(sizeof(float) * (size_t)R * ldM);
+        fail_cnt = take(sizeof(uint32_t));
+        ss = take(sizeof(float) * (size_t)SG * ldM);
         tau = take(sizeof(float) * (size_t)R);
         cnt = take(sizeof(uint32_t) * (size_t)R * kCandCntStride);
-        row_fail = take(sizeof(uint32_t) * (size_t)R);
+        fail_list = take(sizeof(uint32_t) * (size_t)R);
         rb_fail = take(sizeof(uint32_t) * (size_t)ceil_div(R, 128));
         cand = take(sizeof(uint2) * (size_t)R * cap);
         scores = take(sizeof(float) * (size_t)R * T);
@@ -153,38 +162,45 @@ cudaError_t fused_gather(const FusedLayout &L, uint8_t *ws, const void *k_idx, c
     return launch_gather_samples((const uint8_t *)k_idx, k_scale, L.M, L.S, ws + L.ks, (float *)(ws + L.sks), st);
 }
 
+// Sample scores of query rows [g0, g0 + gn) (gn <= L.SG) into the sample-score
+// rows 0.. of the workspace, when any of those rows has more competing
+// positions than the candidate list holds (the others never read theirs).
+cudaError_t fused_sample(const FusedLayout &L, uint8_t *ws, const void *q_idx, const float *q_scale, const void *w,
+                         int64_t T, int H_I, int window, int64_t g0, int64_t gn, WsHeader *hdr, cudaStream_t st,
+                         int64_t q_base, int64_t q_rows)
+{
+    if (g0 + gn - window <= L.cap) return cudaSuccess;
+    StageTimer tm(DSA_STAGE_SAMPLE, st);
+    IndexTcOpts o;
+    o.mode = IT_SAMPLE;
+    o.q_base = q_base;
+    o.q_rows = q_rows;
+    o.nkeys = L.M;
+    o.window = window;
+    o.sample_stride = L.S;
+    return launch_index_tc((const uint8_t *)q_idx, q_scale, ws + L.ks, (const float *)(ws + L.sks),
+                           (const uint16_t *)w, T, H_I, g0, gn, (float *)(ws + L.ss), L.ldM, false, hdr, st, &o);
+}
+
 // Selection of query rows [r0, r0 + n) (n <= L.R) into idx_rows (row r0 first,
 // k + window wide).  q_idx, q_scale and w hold positions [q_base, q_base +
 // q_rows) of the sequence; the key side holds positions [0, T).
 cudaError_t fused_select_pass(const FusedLayout &L, uint8_t *ws, const void *q_idx, const float *q_scale,
                               const void *k_idx, const float *k_scale, const void *w, int64_t T, int H_I, int k,
                               int window, int64_t r0, int64_t n, int32_t *idx_rows, WsHeader *hdr, cudaStream_t st,
-                              int64_t q_base = 0, int64_t q_rows = 0)
+                              int64_t q_base, int64_t q_rows, int64_t ss_row0)
 {
     float *ss = (float *)(ws + L.ss), *tau = (float *)(ws + L.tau), *scores = (float *)(ws + L.scores);
-    uint32_t *cnt = (uint32_t *)(ws + L.cnt), *row_fail = (uint32_t *)(ws + L.row_fail);
-    uint32_t *rb_fail = (uint32_t *)(ws + L.rb_fail), *any = (uint32_t *)(ws + L.any);
+    uint32_t *cnt = (uint32_t *)(ws + L.cnt), *fail_list = (uint32_t *)(ws + L.fail_list);
+    uint32_t *rb_fail = (uint32_t *)(ws + L.rb_fail), *fail_cnt = (uint32_t *)(ws + L.fail_cnt);
     uint2 *cand = (uint2 *)(ws + L.cand);
     const uint8_t *q8 = (const uint8_t *)q_idx, *k8 = (const uint8_t *)k_idx;
     const uint16_t *wb = (const uint16_t *)w;
     cudaError_t e = cudaSuccess;
-    // sample scores, needed only by rows with more competing positions than cap
-    if (r0 + n - window > L.cap) {
-        StageTimer tm(DSA_STAGE_SAMPLE, st);
-        IndexTcOpts o;
-        o.mode = IT_SAMPLE;
-        o.q_base = q_base;
-        o.q_rows = q_rows;
-        o.nkeys = L.M;
-        o.window = window;
-        o.sample_stride = L.S;
-        e = launch_index_tc(q8, q_scale, ws + L.ks, (const float *)(ws + L.sks), wb, T, H_I, r0, n, ss, L.ldM,
-                            false, hdr, st, &o);
-        if (e != cudaSuccess) return e;
-    }
     {
         StageTimer tm(DSA_STAGE_TAU, st);
-        e = launch_prefill_tau(ss, L.ldM, r0, n, k, window, L.S, L.cap, tau, cnt, row_fail, rb_fail, any, st);
+        e = launch_prefill_tau(ss + ss_row0 * L.ldM, L.ldM, r0, n, k, window, L.S, L.cap, tau, cnt, rb_fail,
+                               fail_cnt, st);
         if (e != cudaSuccess) return e;
     }
     {
@@ -203,7 +219,7 @@ cudaError_t fused_select_pass(const FusedLayout &L, uint8_t *ws, const void *q_i
     }
     {
         StageTimer tm(DSA_STAGE_FINISH, st);
-        e = launch_prefill_finish(cand, L.cap, cnt, r0, n, k, window, idx_rows, row_fail, rb_fail, any, st);
+        e = launch_prefill_finish(cand, L.cap, cnt, r0, n, k, window, idx_rows, rb_fail, fail_cnt, fail_list, st);
         if (e != cudaSuccess) return e;
     }
     // repair: scores of the flagged row blocks (nothing when none), stand-alone select of the flagged rows
@@ -214,11 +230,11 @@ cudaError_t fused_select_pass(const FusedLayout &L, uint8_t *ws, const void *q_i
         o.q_base = q_base;
         o.q_rows = q_rows;
         o.rb_mask = rb_fail;
-        o.any = any;
+        o.any = fail_cnt;
         e = launch_index_tc(q8, q_scale, k8, k_scale, wb, T, H_I, r0, n, scores, T, false, hdr, st, &o);
         if (e != cudaSuccess) return e;
     }
-    return launch_topk_rows(scores, T, r0, nullptr, T, n, k, idx_rows, hdr, st, window, row_fail);
+    return launch_topk_rows_list(scores, T, r0, n, k, idx_rows, st, window, fail_list, fail_cnt);
 }
 
 dsa_status check_index_args(const void *q_idx, const float *q_scale, const void *k_idx,
@@ -387,8 +403,13 @@ cudaError_t prefill_fused_rows(const FusedLayout &L, uint8_t *ws, const void *q_
     cudaError_t e = fused_gather(L, ws, k_idx, k_scale, st);
     for (int64_t r = 0; e == cudaSuccess && r < rows; r += L.R) {
         const int64_t n = rows - r < L.R ? rows - r : L.R;
+        if (r % L.SG == 0) {                         // the sample scores of the next group of passes
+            e = fused_sample(L, ws, q_idx, q_scale, w, T, H_I, window, row_begin + r,
+                             rows - r < L.SG ? rows - r : L.SG, hdr, st, row_begin, rows);
+            if (e != cudaSuccess) break;
+        }
         e = fused_select_pass(L, ws, q_idx, q_scale, k_idx, k_scale, w, T, H_I, k_sel, window, row_begin + r, n,
-                              idx + r * (int64_t)kw, hdr, st, row_begin, rows);
+                              idx + r * (int64_t)kw, hdr, st, row_begin, rows, r % L.SG);
     }
     if (e == cudaSuccess) {
         StageTimer tm(DSA_STAGE_ATTN, st);
@@ -696,9 +717,14 @@ dsa_status dsa_prefill_host(const void *q_idx, const float *q_scale, const void 
         if (e == cudaSuccess) e = cudaEventRecord(ce->in, ce->h2d);
         if (e == cudaSuccess) e = cudaStreamWaitEvent(st, ce->in, 0);
         if (e == cudaSuccess && L.fused) {
-            e = fused_select_pass(L.F, ws, ws + L.q_idx, (const float *)(ws + L.q_scale), ws + L.k_idx,
-                                  (const float *)(ws + L.k_scale), ws + L.w, T, H_I, k_sel, 0, r0, n,
-                                  idx + r0 * (int64_t)k_sel, hdr, st);
+            // passes run last rows first, each after its own query rows landed: one
+            // pass's sample scores at a time
+            e = fused_sample(L.F, ws, ws + L.q_idx, (const float *)(ws + L.q_scale), ws + L.w, T, H_I, 0, r0, n,
+                             hdr, st, 0, T);
+            if (e == cudaSuccess)
+                e = fused_select_pass(L.F, ws, ws + L.q_idx, (const float *)(ws + L.q_scale), ws + L.k_idx,
+                                      (const float *)(ws + L.k_scale), ws + L.w, T, H_I, k_sel, 0, r0, n,
+                                      idx + r0 * (int64_t)k_sel, hdr, st, 0, T, 0);
         } else {
             if (e == cudaSuccess) {
                 StageTimer tm(DSA_STAGE_SCORES, st);

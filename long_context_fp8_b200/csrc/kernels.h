@@ -51,27 +51,14 @@ cudaError_t launch_index_f32(const float *q, const float *k, const float *w, int
 // ascending, -1 padded.  With window > 0 only s < n_r - window compete and
 // the window positions follow the selected ones.  Rows with lens[r] outside
 // [1, max_len] are skipped (set to -1) and reported in hdr.
-// row_mask (nullable): only rows r with row_mask[r] != 0 are selected.
 cudaError_t launch_topk_rows(const float *scores, int64_t ld, int64_t row_begin,
                              const int32_t *lens, int64_t max_len, int64_t row_count, int k,
-                             int32_t *idx, WsHeader *hdr, cudaStream_t st, int window = 0,
-                             const uint32_t *row_mask = nullptr);
-
-// ---- fused prefill selection (index_tc.cu, topk.cu) ----
-// Gathers the M = sample_count(T, S) sampled index keys and their scales.
-cudaError_t launch_gather_samples(const uint8_t *k8, const float *sk, int64_t M, int S, uint8_t *ks,
-                                  float *sks, cudaStream_t st);
-// Per row of the pass: tau from the sample scores ss[r * ld + j], the
-// candidate counter zeroed, the repair flags cleared.
-cudaError_t launch_prefill_tau(const float *ss, int64_t ld, int64_t row_begin, int64_t rows, int k, int window,
-                               int S, int cap, float *tau, uint32_t *cnt, uint32_t *row_fail, uint32_t *rb_fail,
-                               uint32_t *any_fail, cudaStream_t st);
-// Per row: the exact selection from its candidates into idx[r * (k + window)],
-// or the row flagged in row_fail / rb_fail (per 128 rows) / any_fail.
-size_t prefill_finish_smem(int cap);
-cudaError_t launch_prefill_finish(const uint2 *cand, int cap, const uint32_t *cnt, int64_t row_begin, int64_t rows,
-                                  int k, int window, int32_t *idx, uint32_t *row_fail, uint32_t *rb_fail,
-                                  uint32_t *any_fail, cudaStream_t st);
+                             int32_t *idx, WsHeader *hdr, cudaStream_t st, int window = 0);
+// The rows list[0, *count) of a pass of `rows` rows (row r is position
+// row_begin + r, its scores at scores[r * ld], its output at idx[r * (k + window)]).
+cudaError_t launch_topk_rows_list(const float *scores, int64_t ld, int64_t row_begin, int64_t rows, int k,
+                                  int32_t *idx, cudaStream_t st, int window, const uint32_t *list,
+                                  const uint32_t *count);
 
 // Rows of lengths lens[r] (decode): each row split over CTAs of 16384
 // positions that share a sampled threshold and collect their candidates, then
@@ -81,6 +68,22 @@ size_t topk_split_ws_bytes(int64_t rows, int64_t max_len);
 cudaError_t launch_topk_split(const float *scores, int64_t ld, const int32_t *lens, int64_t max_len,
                               int64_t rows, int k, int32_t *idx, void *ws_base, WsHeader *hdr,
                               cudaStream_t st, int window = 0);
+
+// ---- fused prefill selection (index_tc.cu, topk.cu) ----
+// Gathers the M = sample_count(T, S) sampled index keys and their scales.
+cudaError_t launch_gather_samples(const uint8_t *k8, const float *sk, int64_t M, int S, uint8_t *ks,
+                                  float *sks, cudaStream_t st);
+// Per row of the pass: tau from the sample scores ss[r * ld + j], the
+// candidate counter zeroed, the repair state (rb_fail, *fail_cnt) cleared.
+cudaError_t launch_prefill_tau(const float *ss, int64_t ld, int64_t row_begin, int64_t rows, int k, int window,
+                               int S, int cap, float *tau, uint32_t *cnt, uint32_t *rb_fail, uint32_t *fail_cnt,
+                               cudaStream_t st);
+// Per row: the exact selection from its candidates into idx[r * (k + window)],
+// or the row listed for repair (fail_list[*fail_cnt++], rb_fail per 128 rows).
+size_t prefill_finish_smem(int cap);
+cudaError_t launch_prefill_finish(const uint2 *cand, int cap, const uint32_t *cnt, int64_t row_begin, int64_t rows,
+                                  int k, int window, int32_t *idx, uint32_t *rb_fail, uint32_t *fail_cnt,
+                                  uint32_t *fail_list, cudaStream_t st);
 
 // ---- FP8 quantisation and cache append (quant.cu) ----
 // codes[r, :] / scale[r] of x[r, 0..cols) (bf16 or fp32), one scale per row;

@@ -21,6 +21,8 @@
 // section on the sliding-window KV cache: the most recent tokens keep their
 // full KV) only the positions before the window compete, and the W window
 // positions follow the selected ones in the output row of k + W entries.
+#include <algorithm>
+
 #include "kernels.h"
 
 namespace dsa {
@@ -645,10 +647,43 @@ __device__ __forceinline__ bool emit_whole_row(int32_t *out, int k, int window, 
     return true;
 }
 
+// The exact top-k of one row of n_all causal positions (the last `window`
+// of them always selected) into out[k + window].
+__device__ __forceinline__ void topk_one_row(TopkSmem<RowsCfg> &sm, const float *row, int64_t n_all, int k,
+                                             int window, int32_t *out, bool vec)
+{
+    using C = RowsCfg;
+    const int tid = threadIdx.x;
+    const int64_t n = n_all > window ? n_all - window : 0;     // positions before the window
+    if (emit_whole_row<C>(out, k, window, n, n_all)) return;
+    emit_window<C>(out, k, window, n);
+    if (tid == 0) { sm.sh_count = 0; sm.sh_overflow = 0; }
+
+    // ---- short rows: every key is a candidate ----
+    if (n <= C::CAP) {
+        const uint32_t c = collect_candidates(sm, row, n, vec, [](uint32_t) { return true; });
+        select_candidates(sm, c, k, out);
+        return;
+    }
+
+    // ---- guess a threshold from evenly spaced samples: about 1.5 k keys of the
+    // row should lie at or above it; then one ordered pass collects them ----
+    {
+        const uint32_t tau = sampled_threshold(sm, row, n, k, vec);
+        const uint32_t c = collect_above_warp(sm, row, n, vec, key_float(tau));
+        if (c >= (uint32_t)k && c <= C::CAP) {        // the selection lies among the candidates
+            select_candidates(sm, c, k, out);
+            return;
+        }
+    }
+    // ---- fallback: the exact histogram path ----
+    topk_row_histogram(sm, row, n, vec, k, out);
+}
+
 __global__ void __launch_bounds__(RowsCfg::NT, 2)
 topk_rows_kernel(const float *__restrict__ scores, int64_t ld, int64_t row_begin,
                  const int32_t *__restrict__ lens, int64_t max_len, int k, int window,
-                 int32_t *__restrict__ idx, WsHeader *hdr, int vec_ok, const uint32_t *__restrict__ row_mask)
+                 int32_t *__restrict__ idx, WsHeader *hdr, int vec_ok)
 {
     using C = RowsCfg;
     extern __shared__ __align__(16) uint8_t smem_raw[];
@@ -656,7 +691,6 @@ topk_rows_kernel(const float *__restrict__ scores, int64_t ld, int64_t row_begin
 
     const int64_t r = blockIdx.x;
     const int tid = threadIdx.x;
-    if (row_mask && row_mask[r] == 0u) return;        // only the rows flagged for repair
     const float *row = scores + r * ld;
     int32_t *out = idx + r * (int64_t)(k + window);
     int64_t n_all;
@@ -695,6 +729,26 @@ topk_rows_kernel(const float *__restrict__ scores, int64_t ld, int64_t row_begin
     }
     // ---- fallback: the exact histogram path ----
     topk_row_histogram(sm, row, n, vec, k, out);
+}
+
+// The rows listed in list[0, *count) (pass-relative, position row_begin + r),
+// shared out over a persistent grid: the prefill's repair of rows whose fused
+// selection failed, which is usually an empty list.
+__global__ void __launch_bounds__(RowsCfg::NT, 2)
+topk_rows_list_kernel(const float *__restrict__ scores, int64_t ld, int64_t row_begin, int k, int window,
+                      int32_t *__restrict__ idx, int vec_ok, const uint32_t *__restrict__ list,
+                      const uint32_t *__restrict__ count)
+{
+    using C = RowsCfg;
+    extern __shared__ __align__(16) uint8_t smem_raw[];
+    TopkSmem<C> &sm = *reinterpret_cast<TopkSmem<C> *>(smem_raw);
+    const uint32_t n = *count;
+    for (uint32_t i = blockIdx.x; i < n; i += gridDim.x) {
+        __syncthreads();                              // the previous row is done with shared memory
+        const int64_t r = list[i];
+        topk_one_row(sm, scores + r * ld, row_begin + r + 1, k, window, idx + r * (int64_t)(k + window),
+                     vec_ok != 0);
+    }
 }
 
 
@@ -869,20 +923,32 @@ __host__ __device__ inline uint32_t tau_rank(int k, int64_t m, int64_t n)
 
 // One warp per row: tau (+inf when the whole row is selected without scores,
 // -inf when every competing position fits the candidate list), and the
-// row's candidate counter and repair flags cleared for the select pass.
-// The rank-th largest sample key is found by bisection over the key range:
-// 32 steps of a warp-wide count, the keys held in registers (m <= 2048) or
-// re-read from the sample scores.
+// row's candidate counter and repair state cleared for the select pass.
+// The rank-th largest sample key: each lane keeps its own J = ceil(rank/32)
+// largest keys; the smallest of the lanes' J-th largest, L, has at least
+// 32 J >= rank keys at or above it, so only those are compacted (usually a
+// tenth of the samples) and searched by bisection over the key range [L, max].
+// Rows with more samples than the registers hold bisect over all of them.
 constexpr int TAU_WARPS = 8;
 constexpr int TAU_REG = 64;                      // keys per lane held in registers
+constexpr int TAU_TOP = 4;                       // per-lane top list: ranks up to 128
+constexpr int TAU_LIST = 1024;                   // compacted keys per warp
+
+__device__ __forceinline__ uint32_t warp_count_ge(const uint32_t *list, uint32_t n, uint32_t mid)
+{
+    uint32_t c = 0;
+    for (uint32_t j = threadIdx.x & 31; j < n; j += 32) c += list[j] >= mid;
+    return __reduce_add_sync(0xffffffffu, c);
+}
 
 __global__ void __launch_bounds__(TAU_WARPS * 32)
 prefill_tau_kernel(const float *__restrict__ ss, int64_t ld, int64_t row_begin, int64_t rows, int k, int window,
                    int S, int cap, float *__restrict__ tau, uint32_t *__restrict__ cnt,
-                   uint32_t *__restrict__ row_fail, uint32_t *__restrict__ rb_fail, uint32_t *__restrict__ any_fail)
+                   uint32_t *__restrict__ rb_fail, uint32_t *__restrict__ fail_cnt)
 {
-    const int lane = threadIdx.x & 31;
-    const int64_t r = (int64_t)blockIdx.x * TAU_WARPS + (threadIdx.x >> 5);
+    __shared__ uint32_t lists[TAU_WARPS][TAU_LIST];
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+    const int64_t r = (int64_t)blockIdx.x * TAU_WARPS + wid;
     if (r >= rows) return;
     const int64_t t = row_begin + r;
     const int64_t n = t + 1 - window > 0 ? t + 1 - window : 0;
@@ -896,20 +962,66 @@ prefill_tau_kernel(const float *__restrict__ ss, int64_t ld, int64_t row_begin, 
         const uint32_t rank = tau_rank(k, m, n);
         const float *row = ss + r * ld;
         uint32_t lo = 0u, hi = 0xffffffffu;              // count(key >= lo) >= rank throughout
-        if (m <= 32 * TAU_REG) {
+        if (m <= 32 * TAU_REG && rank <= 32 * TAU_TOP) {
             uint32_t kv[TAU_REG];
 #pragma unroll
             for (int i = 0; i < TAU_REG; ++i) {
                 const int64_t j = lane + 32 * i;
                 kv[i] = j < m ? float_key(row[j]) : 0u;      // key 0 is no score's key
             }
-            while (lo < hi) {
-                const uint32_t mid = lo + ((hi - lo) >> 1) + 1u;
-                uint32_t c = 0;
+            // this lane's TAU_TOP largest keys, descending
+            uint32_t top[TAU_TOP];
 #pragma unroll
-                for (int i = 0; i < TAU_REG; ++i) c += kv[i] >= mid;
-                c = __reduce_add_sync(0xffffffffu, c);
-                if (c >= rank) lo = mid; else hi = mid - 1u;
+            for (int q = 0; q < TAU_TOP; ++q) top[q] = 0u;
+            uint32_t mx = 0u;
+#pragma unroll
+            for (int i = 0; i < TAU_REG; ++i) {
+                uint32_t x = kv[i];
+                mx = max(mx, x);
+#pragma unroll
+                for (int q = 0; q < TAU_TOP; ++q) {
+                    const uint32_t hiq = max(top[q], x);
+                    x = min(top[q], x);
+                    top[q] = hiq;
+                }
+            }
+            const int J = (int)((rank + 31) / 32);
+            uint32_t lj = top[0];
+#pragma unroll
+            for (int q = 1; q < TAU_TOP; ++q)
+                if (q == J - 1) lj = top[q];
+            const uint32_t L = __reduce_min_sync(0xffffffffu, lj);
+            const uint32_t M = __reduce_max_sync(0xffffffffu, mx);
+            // compact the keys >= L (a key of 0 is padding and never counted)
+            uint32_t *list = lists[wid];
+            uint32_t base = 0;
+            const uint32_t lt = (1u << lane) - 1u;
+            bool fits = true;
+#pragma unroll
+            for (int i = 0; i < TAU_REG; ++i) {
+                const bool p = kv[i] >= L && kv[i] != 0u;
+                const uint32_t bal = __ballot_sync(0xffffffffu, p);
+                if (p && base + __popc(bal & lt) < (uint32_t)TAU_LIST) list[base + __popc(bal & lt)] = kv[i];
+                base += __popc(bal);
+            }
+            fits = base <= (uint32_t)TAU_LIST;
+            __syncwarp();
+            lo = L;
+            hi = M;
+            if (fits) {
+                while (lo < hi) {
+                    const uint32_t mid = lo + ((hi - lo) >> 1) + 1u;
+                    if (warp_count_ge(list, base, mid) >= rank) lo = mid; else hi = mid - 1u;
+                }
+            } else {
+                while (lo < hi) {
+                    const uint32_t mid = lo + ((hi - lo) >> 1) + 1u;
+                    uint32_t c = 0;
+#pragma unroll
+                    for (int i = 0; i < TAU_REG; ++i) c += kv[i] >= mid;
+                    c = __reduce_add_sync(0xffffffffu, c);
+                    if (c >= rank) lo = mid; else hi = mid - 1u;
+                }
             }
         } else {
             while (lo < hi) {
@@ -925,38 +1037,39 @@ prefill_tau_kernel(const float *__restrict__ ss, int64_t ld, int64_t row_begin, 
     if (lane == 0) {
         tau[r] = tv;
         cnt[r * kCandCntStride] = 0u;
-        row_fail[r] = 0u;
         if ((r & 127) == 0) rb_fail[r >> 7] = 0u;
-        if (r == 0) *any_fail = 0u;
+        if (r == 0) *fail_cnt = 0u;
     }
 }
 
 // One CTA per row: the exact top-k of the row's candidates, emitted in
 // ascending position order (the window, if any, after them).  The k-th
-// largest key thr and the number `need` of keys equal to thr that rank
-// within the top k come from the radix select; the emit then marks the
-// positions of keys above thr, and of keys equal to thr, in two bitmaps of a
-// 65536-position window, takes the `need` lowest equal ones, and writes the
-// marked positions in order through block-wide prefix counts.
-using FinCfg = TopkCfg<256, 256, 8, false>;
-constexpr int FIN_WIN_WORDS = 2048;                  // 65536 positions per emit window
+// largest key thr and the number `need` of keys equal to thr that rank within
+// the top k come from the radix select over the keys in shared memory (the
+// positions stay in registers).  When more keys than `need` equal thr, the
+// lowest positions win: a bisection over positions finds the cut.  The emit
+// then marks the selected positions in a bitmap of 65536 positions at a time
+// and writes them in order through one block-wide prefix count per window.
+constexpr int FIN_NT = 256;
+using FinCfg = TopkCfg<FIN_NT, 256, 8, false>;
+constexpr int FIN_WIN_WORDS = 2048;                  // 65536 positions per emit window (the histogram's words)
 
 __host__ __device__ inline size_t finish_smem_bytes(int cap)
 {
-    return align_up(sizeof(TopkSmem<FinCfg>), 16) + sizeof(uint32_t) * (FIN_WIN_WORDS + (size_t)cap);
+    return align_up(sizeof(TopkSmem<FinCfg>), 16) + sizeof(uint32_t) * (size_t)cap;
 }
 
-__global__ void __launch_bounds__(FinCfg::NT)
+template <int PER>                                   // candidates per thread: cap <= PER * FIN_NT
+__global__ void __launch_bounds__(FIN_NT, PER <= 32 ? 3 : 2)
 prefill_finish_kernel(const uint2 *__restrict__ cand, int cap, const uint32_t *__restrict__ cnt, int64_t row_begin,
-                      int k, int window, int32_t *__restrict__ idx, uint32_t *__restrict__ row_fail,
-                      uint32_t *__restrict__ rb_fail, uint32_t *__restrict__ any_fail)
+                      int k, int window, int32_t *__restrict__ idx, uint32_t *__restrict__ rb_fail,
+                      uint32_t *__restrict__ fail_cnt, uint32_t *__restrict__ fail_list)
 {
     using C = FinCfg;
     extern __shared__ __align__(16) uint8_t smem_raw[];
     TopkSmem<C> &sm = *reinterpret_cast<TopkSmem<C> *>(smem_raw);
-    uint32_t *eqbm = reinterpret_cast<uint32_t *>(smem_raw + align_up(sizeof(TopkSmem<C>), 16));
-    uint32_t *keys = eqbm + FIN_WIN_WORDS;
-    uint32_t *gtbm = sm.hist;                        // free once the select is done
+    uint32_t *keys = reinterpret_cast<uint32_t *>(smem_raw + align_up(sizeof(TopkSmem<C>), 16));
+    uint32_t *bm = sm.hist;                          // free once the select is done
     static_assert(sizeof(sm.hist) / sizeof(uint32_t) == FIN_WIN_WORDS, "bitmap window");
 
     const int tid = threadIdx.x;
@@ -969,55 +1082,76 @@ prefill_finish_kernel(const uint2 *__restrict__ cand, int cap, const uint32_t *_
     const uint32_t c = cnt[r * kCandCntStride];
     if (c < (uint32_t)k || c > (uint32_t)cap) {
         if (tid == 0) {                              // the repair pass takes this row
-            row_fail[r] = 1u;
+            fail_list[atomicAdd(fail_cnt, 1u)] = (uint32_t)r;
             atomicOr(rb_fail + (r >> 7), 1u);
-            atomicOr(any_fail, 1u);
         }
         return;
     }
     const uint2 *cr = cand + r * (int64_t)cap;
-    for (uint32_t i = tid; i < c; i += C::NT) keys[i] = float_key(__uint_as_float(cr[i].x));
+#pragma unroll 8
+    for (int j = 0; j < PER; ++j) {
+        const uint32_t i = tid + j * FIN_NT;
+        if (i < c) keys[i] = float_key(__uint_as_float(cr[i].x));
+    }
     __syncthreads();
     uint32_t thr, need;
     radix_select_smem(sm, keys, c, (uint32_t)k, &thr, &need);
     __syncthreads();
+    // the positions, read again (from L2) now that the select's registers are free
+    uint32_t pos[PER];
+#pragma unroll
+    for (int j = 0; j < PER; ++j) {
+        const uint32_t i = tid + j * FIN_NT;
+        pos[j] = i < c ? cr[i].y : 0u;
+    }
 
-    uint32_t eq_base = 0, out_base = 0;              // block-uniform
+    // ties at thr: the lowest `need` positions among them
+    uint32_t ecnt = 0;
+#pragma unroll
+    for (int j = 0; j < PER; ++j) {
+        const uint32_t i = tid + j * FIN_NT;
+        ecnt += i < c && keys[i] == thr;
+    }
+    uint32_t etot;
+    block_excl_scan<C>(ecnt, sm.warp_buf, &etot);
+    uint32_t pcut = 0xffffffffu;                     // every key equal to thr is taken
+    if (etot > need) {                               // block-uniform
+        uint32_t lo = 0, hi = (uint32_t)(n - 1);     // smallest p with count(eq, pos <= p) >= need
+        while (lo < hi) {
+            const uint32_t mid = lo + (hi - lo) / 2;
+            uint32_t e = 0;
+#pragma unroll
+            for (int j = 0; j < PER; ++j) {
+                const uint32_t i = tid + j * FIN_NT;
+                e += i < c && keys[i] == thr && pos[j] <= mid;
+            }
+            uint32_t tot;
+            block_excl_scan<C>(e, sm.warp_buf, &tot);
+            if (tot >= need) hi = mid; else lo = mid + 1;
+        }
+        pcut = lo;
+    }
+
+    uint32_t out_base = 0;                           // block-uniform
     for (int64_t w0 = 0; w0 < n; w0 += 32 * FIN_WIN_WORDS) {
-        for (int i = tid; i < FIN_WIN_WORDS; i += C::NT) { gtbm[i] = 0u; eqbm[i] = 0u; }
+        for (int i = tid; i < FIN_WIN_WORDS; i += FIN_NT) bm[i] = 0u;
         __syncthreads();
-        for (uint32_t i = tid; i < c; i += C::NT) {
-            const uint32_t key = keys[i];
-            if (key >= thr) {
-                const int64_t off = (int64_t)cr[i].y - w0;
-                if (off >= 0 && off < 32 * FIN_WIN_WORDS)
-                    atomicOr((key > thr ? gtbm : eqbm) + (off >> 5), 1u << (off & 31));
+#pragma unroll
+        for (int j = 0; j < PER; ++j) {
+            const uint32_t i = tid + j * FIN_NT;
+            if (i < c) {
+                const uint32_t key = keys[i];
+                const int64_t off = (int64_t)pos[j] - w0;
+                if ((key > thr || (key == thr && pos[j] <= pcut)) && off >= 0 && off < 32 * FIN_WIN_WORDS)
+                    atomicOr(bm + (off >> 5), 1u << (off & 31));
             }
         }
         __syncthreads();
-        constexpr int WPT = FIN_WIN_WORDS / C::NT;   // words per thread, consecutive
-        uint32_t g[WPT], e[WPT], ecnt = 0;
+        constexpr int WPT = FIN_WIN_WORDS / FIN_NT;  // words per thread, consecutive
+        uint32_t g[WPT], scnt = 0;
 #pragma unroll
         for (int q = 0; q < WPT; ++q) {
-            g[q] = gtbm[tid * WPT + q];
-            e[q] = eqbm[tid * WPT + q];
-            ecnt += (uint32_t)__popc(e[q]);
-        }
-        uint32_t etot;
-        uint32_t ebefore = eq_base + block_excl_scan<C>(ecnt, sm.warp_buf, &etot);
-        uint32_t scnt = 0;
-#pragma unroll
-        for (int q = 0; q < WPT; ++q) {
-            // the equal keys are taken in position order until `need` of them are
-            uint32_t x = e[q], taken = 0;
-            while (x && ebefore < need) {
-                const uint32_t lb = x & (0u - x);
-                taken |= lb;
-                x ^= lb;
-                ++ebefore;
-            }
-            ebefore += (uint32_t)__popc(x);
-            g[q] |= taken;
+            g[q] = bm[tid * WPT + q];
             scnt += (uint32_t)__popc(g[q]);
         }
         uint32_t stot;
@@ -1032,7 +1166,6 @@ prefill_finish_kernel(const uint2 *__restrict__ cand, int cap, const uint32_t *_
                 ++o;
             }
         }
-        eq_base += etot;
         out_base += stot;
         __syncthreads();
     }
@@ -1042,8 +1175,7 @@ prefill_finish_kernel(const uint2 *__restrict__ cand, int cap, const uint32_t *_
 
 cudaError_t launch_topk_rows(const float *scores, int64_t ld, int64_t row_begin,
                              const int32_t *lens, int64_t max_len, int64_t row_count, int k,
-                             int32_t *idx, WsHeader *hdr, cudaStream_t st, int window,
-                             const uint32_t *row_mask)
+                             int32_t *idx, WsHeader *hdr, cudaStream_t st, int window)
 {
     if (row_count <= 0) return cudaSuccess;
     const size_t smem = sizeof(TopkSmem<RowsCfg>);
@@ -1052,8 +1184,7 @@ cudaError_t launch_topk_rows(const float *scores, int64_t ld, int64_t row_begin,
     if (e != cudaSuccess) return e;
     const int vec_ok = (ld % 4 == 0) && ((reinterpret_cast<uintptr_t>(scores) & 15u) == 0);
     topk_rows_kernel<<<(unsigned)row_count, RowsCfg::NT, smem, st>>>(scores, ld, row_begin, lens,
-                                                                     max_len, k, window, idx, hdr, vec_ok,
-                                                                     row_mask);
+                                                                     max_len, k, window, idx, hdr, vec_ok);
     return cudaGetLastError();
 }
 
@@ -1096,28 +1227,61 @@ cudaError_t launch_topk_split(const float *scores, int64_t ld, const int32_t *le
 
 
 cudaError_t launch_prefill_tau(const float *ss, int64_t ld, int64_t row_begin, int64_t rows, int k, int window,
-                               int S, int cap, float *tau, uint32_t *cnt, uint32_t *row_fail, uint32_t *rb_fail,
-                               uint32_t *any_fail, cudaStream_t st)
+                               int S, int cap, float *tau, uint32_t *cnt, uint32_t *rb_fail, uint32_t *fail_cnt,
+                               cudaStream_t st)
 {
     if (rows <= 0) return cudaSuccess;
     prefill_tau_kernel<<<(unsigned)ceil_div(rows, TAU_WARPS), TAU_WARPS * 32, 0, st>>>(
-        ss, ld, row_begin, rows, k, window, S, cap, tau, cnt, row_fail, rb_fail, any_fail);
+        ss, ld, row_begin, rows, k, window, S, cap, tau, cnt, rb_fail, fail_cnt);
     return cudaGetLastError();
 }
 
 size_t prefill_finish_smem(int cap) { return finish_smem_bytes(cap); }
 
-cudaError_t launch_prefill_finish(const uint2 *cand, int cap, const uint32_t *cnt, int64_t row_begin, int64_t rows,
-                                  int k, int window, int32_t *idx, uint32_t *row_fail, uint32_t *rb_fail,
-                                  uint32_t *any_fail, cudaStream_t st)
+template <int PER>
+static cudaError_t launch_finish_per(const uint2 *cand, int cap, const uint32_t *cnt, int64_t row_begin, int64_t rows,
+                                     int k, int window, int32_t *idx, uint32_t *rb_fail, uint32_t *fail_cnt,
+                                     uint32_t *fail_list, cudaStream_t st)
 {
-    if (rows <= 0) return cudaSuccess;
     const size_t smem = finish_smem_bytes(cap);
-    cudaError_t e = cudaFuncSetAttribute(prefill_finish_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t e = cudaFuncSetAttribute(prefill_finish_kernel<PER>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)smem);
     if (e != cudaSuccess) return e;
-    prefill_finish_kernel<<<(unsigned)rows, FinCfg::NT, smem, st>>>(cand, cap, cnt, row_begin, k, window, idx,
-                                                                   row_fail, rb_fail, any_fail);
+    prefill_finish_kernel<PER><<<(unsigned)rows, FIN_NT, smem, st>>>(cand, cap, cnt, row_begin, k, window, idx,
+                                                                     rb_fail, fail_cnt, fail_list);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_prefill_finish(const uint2 *cand, int cap, const uint32_t *cnt, int64_t row_begin, int64_t rows,
+                                  int k, int window, int32_t *idx, uint32_t *rb_fail, uint32_t *fail_cnt,
+                                  uint32_t *fail_list, cudaStream_t st)
+{
+    if (rows <= 0) return cudaSuccess;
+    if (cap <= 16 * FIN_NT)
+        return launch_finish_per<16>(cand, cap, cnt, row_begin, rows, k, window, idx, rb_fail, fail_cnt, fail_list, st);
+    if (cap <= 32 * FIN_NT)
+        return launch_finish_per<32>(cand, cap, cnt, row_begin, rows, k, window, idx, rb_fail, fail_cnt, fail_list, st);
+    if (cap <= 64 * FIN_NT)
+        return launch_finish_per<64>(cand, cap, cnt, row_begin, rows, k, window, idx, rb_fail, fail_cnt, fail_list, st);
+    return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_topk_rows_list(const float *scores, int64_t ld, int64_t row_begin, int64_t rows, int k,
+                                  int32_t *idx, cudaStream_t st, int window, const uint32_t *list,
+                                  const uint32_t *count)
+{
+    if (rows <= 0) return cudaSuccess;
+    const size_t smem = sizeof(TopkSmem<RowsCfg>);
+    cudaError_t e = cudaFuncSetAttribute(topk_rows_list_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem);
+    if (e != cudaSuccess) return e;
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const unsigned grid = (unsigned)std::min<int64_t>(rows, 2 * (int64_t)sms);
+    const int vec_ok = (ld % 4 == 0) && ((reinterpret_cast<uintptr_t>(scores) & 15u) == 0);
+    topk_rows_list_kernel<<<grid, RowsCfg::NT, smem, st>>>(scores, ld, row_begin, k, window, idx, vec_ok, list,
+                                                          count);
     return cudaGetLastError();
 }
 
