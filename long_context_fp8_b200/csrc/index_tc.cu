@@ -206,32 +206,43 @@ index_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant_
             if (lane == 0) {
                 tma_prefetch_desc(&qmap);
                 tma_prefetch_desc(&kmap);
+                // The per-head path is kept to a few instructions (stage and phase
+                // advance incrementally; progress is published once, at the end): this
+                // warp shares its scheduler with two busy epilogue warps.
                 TileWalk<MODE> tw;
-                int lt = 0;
+                int lt = 0, qst = 0, qi = 0;
+                uint32_t qph = 0;
                 for (bool ok = tw.start(a, blockIdx.x); ok; ok = tw.next(a, gridDim.x), ++lt) {
                     const int kb = lt & 1;
                     if (!wait_or_abort(&kempty[kb], ((lt >> 1) & 1) ^ 1, &abort_flag)) break;
                     mbar_arrive_expect_tx(&kfull[kb], IT_KBYTES);
                     tma_load_2d(Ks + kb * IT_KBYTES, &kmap, &kfull[kb], 0, (int)(tw.kt * IT_BN));
                     k_issued = lt + 1;
-                    const int t0 = (int)(a.row_begin + tw.rb * IT_BM);
+                    const int tq = (int)(a.row_begin + tw.rb * IT_BM - a.q_base);
                     bool stop = false;
                     for (int h = 0; h < H; ++h) {
-                        const int g = lt * H + h, st = g % IT_QSTAGES;
-                        if (!wait_or_abort(&qempty[st], ((g / IT_QSTAGES) & 1) ^ 1, &abort_flag)) { stop = true; break; }
-                        mbar_arrive_expect_tx(&qfull[st], IT_QBYTES);
-                        tma_load_3d(Qs + st * IT_QBYTES, &qmap, &qfull[st], 0, h, (int)(t0 - a.q_base));
-                        q_issued = g + 1;
+                        if (!wait_or_abort(&qempty[qst], qph ^ 1, &abort_flag)) { stop = true; break; }
+                        mbar_arrive_expect_tx(&qfull[qst], IT_QBYTES);
+                        tma_load_3d(Qs + qst * IT_QBYTES, &qmap, &qfull[qst], 0, h, tq);
+                        ++qi;
+                        if (++qst == IT_QSTAGES) { qst = 0; qph ^= 1; }
                     }
                     if (stop) break;
                 }
+                q_issued = qi;
             }
         } else if (warp == 1) {
             // ------------------------------------------------ MMA issuer
             if (lane == 0) {
+                // Lean per-head path, as for the producer: stage, accumulator and
+                // phases advance incrementally, the query-tile descriptors are
+                // precomputed, and the progress for the abort drain is published once.
                 constexpr uint32_t idesc = umma_idesc_e4m3_f32(IT_BM, IT_BN);
+                const uint64_t qdesc0 = umma_desc_k_sw128(smem_u32(Qs));
+                constexpr uint64_t kQStep = (uint64_t)(IT_QBYTES >> 4);   // descriptor address units
                 TileWalk<MODE> tw;
-                int lt = 0;
+                int lt = 0, qst = 0, acc = 0, qdone = 0, issued = 0;
+                uint32_t qph = 0, aph = 0;
                 for (bool ok = tw.start(a, blockIdx.x); ok; ok = tw.next(a, gridDim.x), ++lt) {
                     const int kb = lt & 1;
                     if (!wait_or_abort(&kfull[kb], (lt >> 1) & 1, &abort_flag)) break;
@@ -239,22 +250,27 @@ index_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant_
                     const uint64_t bdesc = umma_desc_k_sw128(smem_u32(Ks + kb * IT_KBYTES));
                     bool stop = false;
                     for (int h = 0; h < H; ++h) {
-                        const int g = lt * H + h, st = g % IT_QSTAGES, acc = g & 1;
-                        if (!wait_or_abort(&qfull[st], (g / IT_QSTAGES) & 1, &abort_flag)) { stop = true; break; }
-                        q_consumed = g + 1;
-                        if (!wait_or_abort(&tempty[acc], ((g >> 1) & 1) ^ 1, &abort_flag)) { stop = true; break; }
+                        if (!wait_or_abort(&qfull[qst], qph, &abort_flag)) { stop = true; break; }
+                        ++qdone;
+                        if (!wait_or_abort(&tempty[acc], aph ^ 1, &abort_flag)) { stop = true; break; }
                         tc_fence_after();
-                        const uint64_t adesc = umma_desc_k_sw128(smem_u32(Qs + st * IT_QBYTES));
+                        const uint64_t adesc = qdesc0 + (uint64_t)qst * kQStep;
                         const uint32_t d = tmem + (uint32_t)(acc * IT_BN);
+                        umma_f8f6f4(d, adesc, bdesc, idesc, 0u);
     #pragma unroll
-                        for (int k = 0; k < 4; ++k) umma_f8f6f4(d, adesc + 2 * k, bdesc + 2 * k, idesc, k > 0);
-                        umma_commit(&qempty[st]);
+                        for (int k = 1; k < 4; ++k) umma_f8f6f4(d, adesc + 2 * k, bdesc + 2 * k, idesc, 1u);
+                        umma_commit(&qempty[qst]);
                         umma_commit(&tfull[acc]);
-                        mma_heads = g + 1;
+                        ++issued;
+                        if (++qst == IT_QSTAGES) { qst = 0; qph ^= 1; }
+                        acc ^= 1;
+                        aph ^= (uint32_t)(acc == 0);
                     }
                     if (stop) break;
                     umma_commit(&kempty[kb]);
                 }
+                q_consumed = qdone;
+                mma_heads = issued;
             }
         } else {
             // ------------------------------------------------ coefficient warps (2, 3)
