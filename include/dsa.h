@@ -543,6 +543,27 @@ dsa_status dsa_profile_enable(int on);
 dsa_status dsa_profile_read(double *ms_out, int64_t *launches_out);
 
 /*
+ * dsa_test_stall_next -- a test hook for the device-side bounded waits (no
+ * counterpart on the pages; off by default).  It arms a one-shot fault on the
+ * host side: the next launch of the named tcgen05 indexer (the prefill one,
+ * inside dsa_prefill / dsa_index_scores, or the decode one, inside
+ * dsa_decode) has its producer warp in CTA 0 stop early (before its second
+ * query copy in the prefill indexer, before its first copy in the decode
+ * one), so the CTA's consumer waits for data that never comes.  That wait gives up
+ * after its limit (2 s); the CTA records DSA_ERR_TIMEOUT in the workspace
+ * status word, lets the copies and MMAs it did issue land, frees its tensor
+ * memory and returns; the other CTAs finish normally, and the context stays
+ * usable (the call's outputs are then incomplete).  DSA_STALL_NONE disarms.
+ * Process-wide; not for production use.
+ */
+typedef enum dsa_stall_target {
+    DSA_STALL_NONE = 0,
+    DSA_STALL_PREFILL_INDEXER = 1,
+    DSA_STALL_DECODE_INDEXER = 2
+} dsa_stall_target;
+dsa_status dsa_test_stall_next(dsa_stall_target target);
+
+/*
  * dsa_stream_status -- waits for `stream`, then returns the device status
  * word of `workspace` (DSA_OK if no device-side error was recorded by the
  * last call that used this workspace) and resets it to DSA_OK.

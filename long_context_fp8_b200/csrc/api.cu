@@ -418,9 +418,26 @@ cudaError_t prefill_fused_rows(const FusedLayout &L, uint8_t *ws, const void *q_
     return e;
 }
 
+std::atomic<int> g_test_stall{0};               // 0: off, else 1 + the armed target
+
 }  // namespace
 
+bool dsa::consume_test_stall(int target)
+{
+    int want = target + 1;
+    return g_test_stall.load(std::memory_order_relaxed) == want &&
+           g_test_stall.compare_exchange_strong(want, 0);
+}
+
 extern "C" {
+
+dsa_status dsa_test_stall_next(dsa_stall_target target)
+{
+    if (target == DSA_STALL_NONE) { g_test_stall.store(0); return DSA_OK; }
+    if (target != DSA_STALL_PREFILL_INDEXER && target != DSA_STALL_DECODE_INDEXER) return DSA_ERR_INVALID_ARG;
+    g_test_stall.store(target == DSA_STALL_PREFILL_INDEXER ? 1 : 2);
+    return DSA_OK;
+}
 
 const char *dsa_status_string(dsa_status s)
 {

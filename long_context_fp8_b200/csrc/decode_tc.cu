@@ -61,6 +61,7 @@ struct DecTcArgs {
     float *scores;
     int64_t ld;
     WsHeader *hdr;
+    int64_t stall_at;        // test hook: CTA 0's producer stops before its item stall_at (-1: off)
 };
 
 constexpr size_t dt_smem_bytes()
@@ -164,7 +165,7 @@ decode_index_tc_kernel(const __grid_constant__ CUtensorMap kmap,
     int32_t *tab_n = reinterpret_cast<int32_t *>(cw + 128);                        // [DT_MAX_B]
     int32_t *tab_prefix = tab_n + DT_MAX_B;                                         // [DT_MAX_B + 1]
     __shared__ volatile int abort_flag;
-    __shared__ int k_issued, k_consumed, mma_items;
+    __shared__ int k_issued, k_consumed, mma_items, q_issued, q_consumed;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int ps = a.page_size;
@@ -213,7 +214,7 @@ decode_index_tc_kernel(const __grid_constant__ CUtensorMap kmap,
         for (int i = 0; i < 2; ++i) { mbar_init(&qfull[i], 1); mbar_init(&qempty[i], 1); }
         for (int i = 0; i < DT_ACC; ++i) { mbar_init(&tfull[i], 1); mbar_init(&tempty[i], DT_EPI_WARPS); }
         abort_flag = 0;
-        k_issued = k_consumed = mma_items = 0;
+        k_issued = k_consumed = mma_items = q_issued = q_consumed = 0;
         fence_mbar_init();
     }
     tc_fence_before();
@@ -276,6 +277,10 @@ decode_index_tc_kernel(const __grid_constant__ CUtensorMap kmap,
             const int nb = (int)min((int64_t)32, count - j0);
             for (int i = 0; i < nb; ++i) {
                 const int64_t j = j0 + i;
+                if (j == a.stall_at && blockIdx.x == 0) {    // test hook: leave a copy unissued
+                    stop = true;
+                    break;
+                }
                 const int s = (int)(j % DT_STAGES);
                 const uint32_t mask = pt_mask[t * 32 + i];
                 bool ok = true;
@@ -288,6 +293,7 @@ decode_index_tc_kernel(const __grid_constant__ CUtensorMap kmap,
                         if (ok) {
                             mbar_arrive_expect_tx(&qfull[seg & 1], H * 128);
                             tma_load_2d(qs + (seg & 1) * 8192, &qmap, &qfull[seg & 1], 0, b * H);
+                            q_issued = seg + 1;
                         }
                     }
                     if (ok) ok = wait_or_abort(&kempty[s], (uint32_t)((j / DT_STAGES) & 1) ^ 1, &abort_flag);
@@ -325,6 +331,7 @@ decode_index_tc_kernel(const __grid_constant__ CUtensorMap kmap,
                     ++seg;
                     prev_b = it.b;
                     if (!wait_or_abort(&qfull[seg & 1], (seg >> 1) & 1, &abort_flag)) break;
+                    q_consumed = seg + 1;
                     bdesc = umma_desc_k_sw128(smem_u32(qs + (seg & 1) * 8192));
                 }
                 const int s = j % DT_STAGES, acc = j % DT_ACC;
@@ -433,6 +440,7 @@ decode_index_tc_kernel(const __grid_constant__ CUtensorMap kmap,
         record_error(a.hdr, DSA_ERR_TIMEOUT, blockIdx.x);
         // let copies and MMAs still in flight land before shared and tensor memory go
         for (int j = k_consumed; j < k_issued; ++j) mbar_wait(&kfull[j % DT_STAGES], (j / DT_STAGES) & 1);
+        for (int q = q_consumed; q < q_issued; ++q) mbar_wait(&qfull[q & 1], (q >> 1) & 1);
         if (mma_items > 0) mbar_wait(&tfull[(mma_items - 1) % DT_ACC], ((mma_items - 1) / DT_ACC) & 1);
     }
     __syncthreads();
@@ -470,7 +478,7 @@ cudaError_t launch_decode_index_tc(const uint8_t *q8, const float *sq, const uin
     if (!make_tmap_u8(&kmap, kidx, 2, kd, kst, kb) || !make_tmap_u8(&qmap, q8, 2, qd, qst, qb))
         return cudaErrorNotSupported;
     DecTcArgs a{sq, w, kscale, block_table, context_lens, num_pages, max_pages, page_size, box_rows,
-                B, max_context, scores, ld, hdr};
+                B, max_context, scores, ld, hdr, consume_test_stall(1 /* decode indexer */) ? 0 : -1};
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);

@@ -86,6 +86,7 @@ struct IdxTcArgs {
     int vec_store;               // ld % 4 == 0 and out 16-byte aligned
     int tma_store;               // tiles wholly below the diagonal leave through TMA stores (omap)
     WsHeader *hdr;
+    int stall_at;                // test hook: CTA 0's producer stops before query copy stall_at (-1: off)
 };
 
 struct SmemLayout {
@@ -221,6 +222,7 @@ index_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant_
                     const int tq = (int)(a.row_begin + tw.rb * IT_BM - a.q_base);
                     bool stop = false;
                     for (int h = 0; h < H; ++h) {
+                        if (qi == a.stall_at && blockIdx.x == 0) { stop = true; break; }   // test hook
                         if (!wait_or_abort(&qempty[qst], qph ^ 1, &abort_flag)) { stop = true; break; }
                         mbar_arrive_expect_tx(&qfull[qst], IT_QBYTES);
                         tma_load_3d(Qs + qst * IT_QBYTES, &qmap, &qfull[qst], 0, h, tq);
@@ -596,6 +598,7 @@ cudaError_t launch_index_tc(const uint8_t *q8, const float *sq, const uint8_t *k
     a.tma_store = o.mode == IT_SCORES && a.vec_store && row_count < ((int64_t)1 << 31) &&
                   make_tmap_f32_2d(&omap, out, (uint64_t)T, (uint64_t)row_count, (uint64_t)ld * 4, 32, 32);
     a.hdr = hdr;
+    a.stall_at = -1;
     // number of work tiles, to size the persistent grid (a repair launch may visit fewer)
     int64_t tiles = 0;
     for (int64_t rb = 0; rb < a.n_rb; ++rb) {
@@ -626,6 +629,7 @@ cudaError_t launch_index_tc(const uint8_t *q8, const float *sq, const uint8_t *k
             fill_upper_kernel<<<dim3(8, (unsigned)n), 256, 0, st>>>(out + r0 * ld, ld, T, row_begin + r0);
         }
     }
+    if (consume_test_stall(0 /* prefill indexer */)) a.stall_at = 1;
     kern<<<grid, IT_THREADS, smem, st>>>(qmap, kmap, omap, a);
     return cudaGetLastError();
 }

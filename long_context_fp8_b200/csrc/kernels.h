@@ -9,6 +9,11 @@
 
 namespace dsa {
 
+// ---- test hook (api.cu): true once after dsa_test_stall_next armed `target`
+// (0: the prefill indexer, 1: the decode indexer); that launch leaves one copy
+// unissued so that a bounded wait runs out.
+bool consume_test_stall(int target);
+
 // ---- indexer (index.cu, index_tc.cu) ----
 // Scores of rows [row_begin, row_begin+row_count) into out[(t-row_begin)*ld + s].
 // write_upper: also write -inf for s in (t, T).

@@ -30,7 +30,7 @@ EXPORTS = ("dsa_status_string", "dsa_version", "dsa_index_scores", "dsa_topk_wor
            "dsa_quantize_e4m3", "dsa_cache_append", "dsa_cache_append_kv8", "dsa_decode_noalloc",
            "dsa_split_workspace_size", "dsa_decode_select", "dsa_merge_selections", "dsa_decode_attend",
            "dsa_merge_partials", "dsa_stream_status", "dsa_profile_enable", "dsa_profile_read",
-           "dsa_prefill_rows_workspace_size", "dsa_prefill_rows")
+           "dsa_prefill_rows_workspace_size", "dsa_prefill_rows", "dsa_test_stall_next")
 
 
 class DSAError(RuntimeError):
@@ -92,6 +92,7 @@ def load(path: str = LIB_PATH):
         "dsa_merge_partials": ([P, I64, P, I64, I32, I32, I32, I32, P, P, P], I32),
         "dsa_stream_status": ([P, P], I32),
         "dsa_profile_enable": ([I32], I32),
+        "dsa_test_stall_next": ([I32], I32),
         "dsa_prefill_rows_workspace_size": ([I64, I64, I32, I32, I32, I32, I32, I32], SZ),
         "dsa_prefill_rows": ([P, P, P, P, P, P, P, P, I64, I64, I64, I32, I32, I32, I32, I32, F, P, P, P, I32, P,
                               SZ, P], I32),
@@ -609,3 +610,12 @@ def profile_read():
     _check("dsa_profile_read", load().dsa_profile_read(ctypes.cast(ms, ctypes.c_void_p),
                                                        ctypes.cast(n, ctypes.c_void_p)))
     return {name: (ms[i], n[i]) for i, name in enumerate(STAGES)}
+
+
+STALL_NONE, STALL_PREFILL_INDEXER, STALL_DECODE_INDEXER = 0, 1, 2
+
+
+def test_stall_next(target: int):
+    """Arm the library's one-shot test hook: the next launch of the named
+    indexer leaves one copy unissued, so that its bounded wait runs out."""
+    _check("dsa_test_stall_next", load().dsa_test_stall_next(int(target)))
