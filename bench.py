@@ -36,6 +36,28 @@ import dsa_synth  # noqa: E402
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 L2_FLUSH_BYTES = 256 << 20
 
+# DRAM traffic of the dominant kernel (the indexer's select epilogue), from a
+# one-pass ncu capture (dram__bytes_read.sum + dram__bytes_write.sum) of every
+# select launch of one 128K prefill, averaged per launch.  The record holds the
+# SHA-256 of the kernel's source at capture time; once the source changes the
+# figure no longer describes the kernel and the bench reports null.
+SELECT_TRAFFIC = {"bytes_per_launch": 112211493, "launches": 35,
+                  "source_sha256": "8e161a9493f6366a2e3b93f20d265b27159c2acfc89c9d95f3d7d11712ae0429",
+                  "profile": "profiles/index_tc_select__prefill128k_and_16k.md"}
+
+
+def select_traffic():
+    """The recorded per-launch DRAM bytes of the select kernel, or None when no
+    capture is recorded or the kernel's source changed since."""
+    if not SELECT_TRAFFIC:
+        return None
+    import hashlib
+    src = os.path.join(ROOT, "long_context_fp8_b200", "csrc", "index_tc.cu")
+    with open(src, "rb") as f:
+        if hashlib.sha256(f.read()).hexdigest() != SELECT_TRAFFIC["source_sha256"]:
+            return None
+    return SELECT_TRAFFIC["bytes_per_launch"]
+
 
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
@@ -654,7 +676,7 @@ def main():
                 "steps": args.steps, "warmup": args.warmup,
                 "ms_per_step": 1000.0 * spec.L / v, "higher_is_better": True, "scaling": "weak",
                 "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-                "config": workload_config(spec, dspec), "impl": "reference",
+                "config": dict(workload_config(spec, dspec), parallelism="replicas1"), "impl": "reference",
                 "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": oracle_threads(),
                                  "kind": "oracle",
                                  "sample": f"{nrows} uniformly spaced query rows of the {spec.L}-token "
@@ -735,8 +757,8 @@ def main():
     roofline = {"bound": "tensor", "kernel": "indexer with the fused select epilogue (FP8 e4m3 x e4m3 -> fp32)",
                 "achieved": round(pre["idx_tflops"], 2), "peak": round(idx_peak, 1),
                 "unit": "TFLOP/s", "frac": round(pre["idx_tflops"] / idx_peak, 4),
-                "peak_source": f"{peak_kind} bf16 dense x 2 (fp8:bf16 nominal ratio), burst",
-                "traffic": None}
+                "peak_source": f"derived: {peak_kind} bf16 dense (cuBLAS, burst) x 2, the nominal fp8:bf16 ratio",
+                "traffic": select_traffic(), "traffic_unit": "bytes per launch"}
     if "bf16_tflops_sustained" in peaks:
         # the indexer runs inside a long step; the sustained figure was measured at
         # lower clocks (cuBLAS under the power cap), so it is reported beside the
