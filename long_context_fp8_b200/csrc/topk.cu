@@ -1045,11 +1045,14 @@ prefill_tau_kernel(const float *__restrict__ ss, int64_t ld, int64_t row_begin, 
 // One CTA per row: the exact top-k of the row's candidates, emitted in
 // ascending position order (the window, if any, after them).  The k-th
 // largest key thr and the number `need` of keys equal to thr that rank within
-// the top k come from the radix select over the keys in shared memory (the
-// positions stay in registers).  When more keys than `need` equal thr, the
-// lowest positions win: a bisection over positions finds the cut.  The emit
-// then marks the selected positions in a bitmap of 65536 positions at a time
-// and writes them in order through one block-wide prefix count per window.
+// the top k come from the radix select over the keys in shared memory.  When
+// more keys than `need` equal thr, the lowest positions win: a bisection over
+// positions finds the cut.  The emit then marks the selected positions in a
+// bitmap of 65536 positions at a time and writes them in order through one
+// block-wide prefix count per window.  Positions are read again from the
+// candidate list (L2) where needed rather than held in registers: the kernel
+// is bound by its barriers and latencies, so the registers buy more resident
+// rows (five CTAs per SM) instead.
 constexpr int FIN_NT = 256;
 using FinCfg = TopkCfg<FIN_NT, 256, 8, false>;
 constexpr int FIN_WIN_WORDS = 2048;                  // 65536 positions per emit window (the histogram's words)
@@ -1060,7 +1063,7 @@ __host__ __device__ inline size_t finish_smem_bytes(int cap)
 }
 
 template <int PER>                                   // candidates per thread: cap <= PER * FIN_NT
-__global__ void __launch_bounds__(FIN_NT, PER <= 32 ? 3 : 2)
+__global__ void __launch_bounds__(FIN_NT, PER <= 32 ? 5 : 4)
 prefill_finish_kernel(const uint2 *__restrict__ cand, int cap, const uint32_t *__restrict__ cnt, int64_t row_begin,
                       int k, int window, int32_t *__restrict__ idx, uint32_t *__restrict__ rb_fail,
                       uint32_t *__restrict__ fail_cnt, uint32_t *__restrict__ fail_list)
@@ -1097,13 +1100,6 @@ prefill_finish_kernel(const uint2 *__restrict__ cand, int cap, const uint32_t *_
     uint32_t thr, need;
     radix_select_smem(sm, keys, c, (uint32_t)k, &thr, &need);
     __syncthreads();
-    // the positions, read again (from L2) now that the select's registers are free
-    uint32_t pos[PER];
-#pragma unroll
-    for (int j = 0; j < PER; ++j) {
-        const uint32_t i = tid + j * FIN_NT;
-        pos[j] = i < c ? cr[i].y : 0u;
-    }
 
     // ties at thr: the lowest `need` positions among them
     uint32_t ecnt = 0;
@@ -1120,10 +1116,10 @@ prefill_finish_kernel(const uint2 *__restrict__ cand, int cap, const uint32_t *_
         while (lo < hi) {
             const uint32_t mid = lo + (hi - lo) / 2;
             uint32_t e = 0;
-#pragma unroll
+#pragma unroll 4
             for (int j = 0; j < PER; ++j) {
                 const uint32_t i = tid + j * FIN_NT;
-                e += i < c && keys[i] == thr && pos[j] <= mid;
+                e += i < c && keys[i] == thr && __ldg(&cr[i].y) <= mid;
             }
             uint32_t tot;
             block_excl_scan<C>(e, sm.warp_buf, &tot);
@@ -1136,14 +1132,17 @@ prefill_finish_kernel(const uint2 *__restrict__ cand, int cap, const uint32_t *_
     for (int64_t w0 = 0; w0 < n; w0 += 32 * FIN_WIN_WORDS) {
         for (int i = tid; i < FIN_WIN_WORDS; i += FIN_NT) bm[i] = 0u;
         __syncthreads();
-#pragma unroll
+#pragma unroll 4
         for (int j = 0; j < PER; ++j) {
             const uint32_t i = tid + j * FIN_NT;
             if (i < c) {
                 const uint32_t key = keys[i];
-                const int64_t off = (int64_t)pos[j] - w0;
-                if ((key > thr || (key == thr && pos[j] <= pcut)) && off >= 0 && off < 32 * FIN_WIN_WORDS)
-                    atomicOr(bm + (off >> 5), 1u << (off & 31));
+                if (key >= thr) {
+                    const uint32_t p = __ldg(&cr[i].y);
+                    const int64_t off = (int64_t)p - w0;
+                    if ((key > thr || p <= pcut) && off >= 0 && off < 32 * FIN_WIN_WORDS)
+                        atomicOr(bm + (off >> 5), 1u << (off & 31));
+                }
             }
         }
         __syncthreads();
