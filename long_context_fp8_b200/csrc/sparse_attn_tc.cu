@@ -238,9 +238,10 @@ sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_con
         }
         mbar_init(ofull, 1); mbar_init(oempty, 4);                // oempty: set 0 read O_0 and O_1
         mbar_init(mlfull, 4); mbar_init(mlempty, 4);              // set 1 -> set 0 hand-off of (m, l)
-        // kvfull: one asynchronous arrival per producer thread when its copies land,
-        // plus one ordinary arrival per producer warp publishing the validity bits
-        for (int i = 0; i < AT_STAGES; ++i) { mbar_init(&kvfull[i], AT_PRODUCERS + 2); mbar_init(&kvempty[i], 1); }
+        // kvfull: one asynchronous arrival per copying producer thread when its copies
+        // land (bf16: the one warp of the block; KV8: both warps), plus two ordinary
+        // arrivals publishing the validity bits
+        for (int i = 0; i < AT_STAGES; ++i) { mbar_init(&kvfull[i], (KV8 ? AT_PRODUCERS : 32) + 2); mbar_init(&kvempty[i], 1); }
         abort_flag = 0;
         kv_issued = kv_consumed = q_issued = q_consumed = pv_last = s_last = 0;
         fence_mbar_init();
@@ -293,20 +294,15 @@ sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_con
                 if (warp == 5) stop = stop || abort_flag;
                 ++qi;
                 const int32_t *irow = a.idx + item.row * a.ksel;
-                // warp (w - 4) copies rows 32 (w - 4) .. +31 of each block; lane l copies
-                // 16-byte chunk l % 16 of the row's K (l < 16) or V (l >= 16), so one
-                // instruction moves one whole row pair (two 256-byte runs).  Lane l also
-                // resolves row 32 (w - 4) + l of the block, broadcast by shuffles.
+                // bf16: producer warp w = warp - 4 takes blocks b = w, w + 2, ... of the item
+                // whole; lane l resolves rows l and 32 + l of its block (broadcast by shuffles)
+                // and copies 16-byte chunk l % 16 of each row's K (l < 16) or V (l >= 16), so
+                // one instruction moves one whole row pair (two 256-byte runs).  A warp's
+                // loop runs at the latency of the index reads for its next block, so the
+                // two warps taking alternate blocks issue a block in about half that time.
+                // KV8: warp w copies rows 32 w .. 32 w + 31 of every block (below).
                 const int rbase = (warp - 4) * 32;
                 const int32_t *brow = paged ? a.block_table + item.row * a.max_pages : nullptr;
-                // Lane l's selected position in blocks b + 1 and b + 2 and, for the
-                // paged caches, the page id of block b + 1: the index and block-table
-                // reads run ahead of the copies, so their latency is not paid per block.
-                int e = item.e0 + rbase + lane;
-                int p1 = e < item.e1 ? __ldg(irow + e) : -1;
-                int pg1 = paged && p1 >= 0 && p1 < ctx ? __ldg(brow + p1 / a.page_size) : -1;
-                e += AT_BLK;
-                int p2 = (1 < item.nblk && e < item.e1) ? __ldg(irow + e) : -1;
                 const int chunk = lane & 15;
                 const bool is_v = lane >= 16;
                 // K/V row of selected position p (page pg): lane l resolves row
@@ -375,37 +371,66 @@ sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_con
                     pgnx = page_of(pnx);
                     pnx2 = pos_of(AT_NSTG);
                 }
-                for (int b = 0; b < item.nblk && !stop; ++b, ++g) {
-                    const int st = g % AT_STAGES;
-                    const int p = p1, pg = pg1;
-                    if constexpr (!KV8) {
-                        p1 = p2;
-                        pg1 = paged && p1 >= 0 && p1 < ctx ? __ldg(brow + p1 / a.page_size) : -1;
-                        e += AT_BLK;
-                        p2 = (b + 2 < item.nblk && e < item.e1) ? __ldg(irow + e) : -1;
-                    }
-                    // warp-uniform outcome: the ballot and shuffles below need every lane
-                    const bool ok = __all_sync(0xffffffffu,
-                                               wait_or_abort(&kvempty[st], ((g / AT_STAGES) & 1) ^ 1, &abort_flag));
-                    if (!ok) { stop = true; break; }
-                    if constexpr (!KV8) {
-                        int r;
-                        bool v;
-                        resolve(p, pg, r, v);
-                        const unsigned vw = __ballot_sync(0xffffffffu, v);
+                if constexpr (!KV8) {
+                    const int w = warp - 4;
+                    auto pos_at = [&](int bb, int row) -> int {
+                        const int ee = item.e0 + bb * AT_BLK + row;
+                        return (bb < item.nblk && ee < item.e1) ? __ldg(irow + ee) : -1;
+                    };
+                    // positions of the warp's block b (rows l, 32 + l) and of its next block
+                    // b + 2, read one block of the warp ahead; paged: block b's page ids
+                    int qa0 = pos_at(w, lane), qa1 = pos_at(w, 32 + lane);
+                    int qb0 = pos_at(w + 2, lane), qb1 = pos_at(w + 2, 32 + lane);
+                    int pga0 = page_of(qa0), pga1 = page_of(qa1);
+                    for (int b = w; b < item.nblk && !stop; b += 2) {
+                        const int gb = g + b, st = gb % AT_STAGES;
+                        const int p0 = qa0, p1 = qa1, pg0 = pga0, pg1 = pga1;
+                        qa0 = qb0;
+                        qa1 = qb1;
+                        pga0 = page_of(qa0);
+                        pga1 = page_of(qa1);
+                        qb0 = pos_at(b + 4, lane);
+                        qb1 = pos_at(b + 4, 32 + lane);
+                        // warp-uniform outcome: the ballots and shuffles below need every lane
+                        const bool ok = __all_sync(0xffffffffu,
+                                                   wait_or_abort(&kvempty[st], ((gb / AT_STAGES) & 1) ^ 1, &abort_flag));
+                        if (!ok) { stop = true; break; }
+                        int r0, r1;
+                        bool v0, v1;
+                        resolve(p0, pg0, r0, v0);
+                        resolve(p1, pg1, r1, v1);
+                        const unsigned vw0 = __ballot_sync(0xffffffffu, v0);
+                        const unsigned vw1 = __ballot_sync(0xffffffffu, v1);
                         if (lane == 0) {
-                            valid[st * 2 + (warp - 4)] = vw;
+                            valid[st * 2] = vw0;
+                            valid[st * 2 + 1] = vw1;
                             mbar_arrive(&kvfull[st]);      // releases the validity bits
+                            mbar_arrive(&kvfull[st]);
                         }
-                        uint8_t *tile = KVs + st * AT_STAGE + (is_v ? AT_KTILE : 0) + (chunk >> 3) * AT_KHALF + rbase * 128;
+                        uint8_t *tile = KVs + st * AT_STAGE + (is_v ? AT_KTILE : 0) + (chunk >> 3) * AT_KHALF;
                         const uint16_t *base = (is_v ? a.v : a.k) + chunk * 8;
 #pragma unroll
-                        for (int i = 0; i < 32; ++i) {    // row rbase + i of the block (rbase % 8 == 0)
-                            const int ri = __shfl_sync(0xffffffffu, r, i);
-                            cp_async_16(tile + i * 128 + (((chunk ^ i) & 7) << 4), base + (int64_t)ri * AT_D, (vw >> i) & 1u);
+                        for (int i = 0; i < 32; ++i) {    // rows i and 32 + i of the block
+                            const int ri = __shfl_sync(0xffffffffu, r0, i);
+                            cp_async_16(tile + i * 128 + (((chunk ^ i) & 7) << 4), base + (int64_t)ri * AT_D, (vw0 >> i) & 1u);
+                        }
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) {
+                            const int ri = __shfl_sync(0xffffffffu, r1, i);
+                            cp_async_16(tile + (32 + i) * 128 + (((chunk ^ i) & 7) << 4), base + (int64_t)ri * AT_D,
+                                        (vw1 >> i) & 1u);
                         }
                         cp_async_arrive_noinc(&kvfull[st]);   // fires when this thread's copies land
-                    } else {
+                        if (lane == 0) atomicMax(&kv_issued, gb + 1);
+                    }
+                    g += item.nblk;
+                } else {
+                    for (int b = 0; b < item.nblk && !stop; ++b, ++g) {
+                        const int st = g % AT_STAGES;
+                        // warp-uniform outcome: the ballot and shuffles below need every lane
+                        const bool ok = __all_sync(0xffffffffu,
+                                                   wait_or_abort(&kvempty[st], ((g / AT_STAGES) & 1) ^ 1, &abort_flag));
+                        if (!ok) { stop = true; break; }
                         cp_async_wait<AT_NSTG - 2>();     // this lane's copies of block g have landed
                         __syncwarp();                     // and every lane's (scales, validity word)
                         const int buf = g % AT_NSTG;
@@ -438,8 +463,8 @@ sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_con
                         pnx = pnx2;
                         pgnx = page_of(pnx);
                         pnx2 = pos_of(b + AT_NSTG + 1);
+                        if (pt == 0) kv_issued = g + 1;
                     }
-                    if (pt == 0) kv_issued = g + 1;
                 }
             }
             cp_async_wait<0>();                           // nothing in flight when the CTA retires
