@@ -145,6 +145,16 @@ inline int64_t fused_rows_default(int64_t T)
     if (r > kFusedRowsMax) r = kFusedRowsMax;
     return r < fused_rows_max(T) ? r : fused_rows_max(T);
 }
+// The host-memory prefill's pass: twice the repair budget of the default (so, at
+// 128K positions, 4096 rows instead of 2048), since its workspace already mirrors
+// every input and output; fewer passes mean fewer small sample launches.
+inline int64_t fused_rows_host(int64_t T)
+{
+    int64_t r = (int64_t)(2 * kRepairBudget / (sizeof(float) * (size_t)T)) / 128 * 128;
+    if (r < 128) r = 128;
+    if (r > kFusedRowsMax) r = kFusedRowsMax;
+    return r < fused_rows_max(T) ? r : fused_rows_max(T);
+}
 // Largest R (a multiple of 128, at most T rounded up) whose layout fits ws_bytes; 0 if none.
 inline int64_t fused_rows_fitting(int64_t T, int k, size_t base, size_t ws_bytes)
 {
@@ -339,7 +349,7 @@ struct HostPrefillLayout {
     HostPrefillLayout(int64_t T, int H_I, int d_I, int H_q, int d, int k_sel)
         : fused(fused_ok(DSA_E4M3, H_I, T, k_sel)), F(1, 1, 0, 0)
     {
-        R = fused ? fused_rows_default(T) : prefill_rows_default(T);
+        R = fused ? fused_rows_host(T) : prefill_rows_default(T);
         size_t off = kWsHeader;
         auto take = [&](size_t bytes) { size_t o = off; off += align_up(bytes, 256); return o; };
         q_idx = take((size_t)T * H_I * d_I);
@@ -368,7 +378,7 @@ struct HostPrefillLayout {
 // use and kept for the life of the process.
 struct CopyEngine {
     cudaStream_t h2d = nullptr, d2h = nullptr;
-    cudaEvent_t start = nullptr, in = nullptr, out = nullptr, done = nullptr;
+    cudaEvent_t start = nullptr, in = nullptr, in_attn = nullptr, out = nullptr, done = nullptr;
     bool ok = false;
 };
 
@@ -384,6 +394,7 @@ CopyEngine *copy_engine()
                cudaStreamCreateWithFlags(&c.d2h, cudaStreamNonBlocking) == cudaSuccess &&
                cudaEventCreateWithFlags(&c.start, cudaEventDisableTiming) == cudaSuccess &&
                cudaEventCreateWithFlags(&c.in, cudaEventDisableTiming) == cudaSuccess &&
+               cudaEventCreateWithFlags(&c.in_attn, cudaEventDisableTiming) == cudaSuccess &&
                cudaEventCreateWithFlags(&c.out, cudaEventDisableTiming) == cudaSuccess &&
                cudaEventCreateWithFlags(&c.done, cudaEventDisableTiming) == cudaSuccess;
     });
@@ -689,13 +700,33 @@ dsa_status dsa_prefill_host(const void *q_idx, const float *q_scale, const void 
     s = check_attn_args(ws + L.q, ws + L.k, ws + L.v, (const int32_t *)(ws + L.idx), T, H_q, d, k_sel,
                         ws + L.out, dtype);
     if (s != DSA_OK) return s;
+    // Passes run from the last rows to the first: late rows carry the most work per
+    // copied byte (their causal rows are longest), so the copies stay ahead of the
+    // computation.  The first pass and the last are at most kHostEdgeRows rows: the
+    // computation starts as soon as that few query rows have landed, and the outputs
+    // left to copy after it has ended are that few rows'.
+    constexpr int64_t kHostEdgeRows = 512;
+    std::vector<std::pair<int64_t, int64_t>> passes;   // (first row, rows), in processing order
+    {
+        const int64_t edge = L.R < kHostEdgeRows ? L.R : kHostEdgeRows;
+        int64_t top = T;
+        const int64_t n0 = edge < top ? edge : top;
+        passes.emplace_back(top - n0, n0);
+        top -= n0;
+        const int64_t bottom = edge < top ? edge : top;
+        while (top > bottom) {
+            const int64_t n = L.R < top - bottom ? L.R : top - bottom;
+            passes.emplace_back(top - n, n);
+            top -= n;
+        }
+        if (bottom > 0) passes.emplace_back(0, bottom);
+    }
     CopyEngine *ce = copy_engine();
     if (!ce) return DSA_ERR_CUDA;
     cudaStream_t st = as_stream(stream);
     WsHeader *hdr = reinterpret_cast<WsHeader *>(ws);
     float *scores = reinterpret_cast<float *>(ws + L.scores);
     int32_t *idx = reinterpret_cast<int32_t *>(ws + L.idx);
-    const int64_t R = L.R;
     const size_t qi_row = (size_t)H_I * d_I, q_row = 2 * (size_t)H_q * d;
     auto h2d = [&](size_t off, const void *src, size_t bytes) {
         return cudaMemcpyAsync(ws + off, src, bytes, cudaMemcpyHostToDevice, ce->h2d);
@@ -710,32 +741,37 @@ dsa_status dsa_prefill_host(const void *q_idx, const float *q_scale, const void 
     if (e == cudaSuccess) e = cudaEventRecord(ce->start, st);
     if (e == cudaSuccess) e = cudaStreamWaitEvent(ce->h2d, ce->start, 0);
     if (e == cudaSuccess) e = cudaStreamWaitEvent(ce->d2h, ce->start, 0);
+    // The selection needs only the index keys, their scales, the query scales and
+    // the head weights: they go first, and K and V follow while the first pass
+    // selects.
     if (e == cudaSuccess) e = h2d(L.k_idx, k_idx, (size_t)T * d_I);
     if (e == cudaSuccess) e = h2d(L.k_scale, k_scale, sizeof(float) * (size_t)T);
-    if (e == cudaSuccess) e = h2d(L.k, k, 2 * (size_t)T * d);
-    if (e == cudaSuccess) e = h2d(L.v, v, 2 * (size_t)T * d);
     if (e == cudaSuccess) e = h2d(L.q_scale, q_scale, sizeof(float) * (size_t)T);
     if (e == cudaSuccess) e = h2d(L.w, w, 2 * (size_t)T * H_I);
-    if (e == cudaSuccess && L.fused) {
-        // the sampled keys, once the keys have landed
-        e = cudaEventRecord(ce->in, ce->h2d);
-        if (e == cudaSuccess) e = cudaStreamWaitEvent(st, ce->in, 0);
-        if (e == cudaSuccess) e = fused_gather(L.F, ws, ws + L.k_idx, (const float *)(ws + L.k_scale), st);
-    }
-    // Passes run from the last rows to the first: late rows carry the most work per
-    // copied byte (their causal rows are longest), so the copies stay ahead of the
-    // computation from the start, and the last pass's outputs are the cheapest.
-    const int64_t npass = ceil_div(T, R);
-    for (int64_t pi = npass - 1; e == cudaSuccess && pi >= 0; --pi) {
-        const int64_t r0 = pi * R;
-        const int64_t n = T - r0 < R ? T - r0 : R;
-        e = h2d(L.q_idx + r0 * qi_row, static_cast<const uint8_t *>(q_idx) + r0 * qi_row, n * qi_row);
+    if (e == cudaSuccess) e = cudaEventRecord(ce->in, ce->h2d);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(st, ce->in, 0);
+    if (e == cudaSuccess && L.fused)          // the sampled keys, once the keys have landed
+        e = fused_gather(L.F, ws, ws + L.k_idx, (const float *)(ws + L.k_scale), st);
+    // the first pass's index queries go ahead of K and V (the h2d stream is in order)
+    if (e == cudaSuccess)
+        e = h2d(L.q_idx + passes[0].first * qi_row, static_cast<const uint8_t *>(q_idx) + passes[0].first * qi_row,
+                passes[0].second * qi_row);
+    if (e == cudaSuccess) e = cudaEventRecord(ce->in, ce->h2d);
+    if (e == cudaSuccess) e = h2d(L.k, k, 2 * (size_t)T * d);
+    if (e == cudaSuccess) e = h2d(L.v, v, 2 * (size_t)T * d);
+    for (size_t pi = 0; e == cudaSuccess && pi < passes.size(); ++pi) {
+        const int64_t r0 = passes[pi].first, n = passes[pi].second;
+        // the pass's index queries for its selection (the first pass's went ahead of K
+        // and V), then its queries for its attention
+        if (pi > 0) {
+            e = h2d(L.q_idx + r0 * qi_row, static_cast<const uint8_t *>(q_idx) + r0 * qi_row, n * qi_row);
+            if (e == cudaSuccess) e = cudaEventRecord(ce->in, ce->h2d);
+        }
         if (e == cudaSuccess) e = h2d(L.q + r0 * q_row, static_cast<const uint8_t *>(q) + r0 * q_row, n * q_row);
-        if (e == cudaSuccess) e = cudaEventRecord(ce->in, ce->h2d);
+        if (e == cudaSuccess) e = cudaEventRecord(ce->in_attn, ce->h2d);
         if (e == cudaSuccess) e = cudaStreamWaitEvent(st, ce->in, 0);
         if (e == cudaSuccess && L.fused) {
-            // passes run last rows first, each after its own query rows landed: one
-            // pass's sample scores at a time
+            // one pass's sample scores at a time
             e = fused_sample(L.F, ws, ws + L.q_idx, (const float *)(ws + L.q_scale), ws + L.w, T, H_I, 0, r0, n,
                              hdr, st, 0, T);
             if (e == cudaSuccess)
@@ -754,6 +790,8 @@ dsa_status dsa_prefill_host(const void *q_idx, const float *q_scale, const void 
                 e = launch_topk_rows(scores, T, r0, nullptr, T, n, k_sel, idx + r0 * (int64_t)k_sel, hdr, st);
             }
         }
+        // the attention also needs K and V, copied before any pass's queries
+        if (e == cudaSuccess) e = cudaStreamWaitEvent(st, ce->in_attn, 0);
         if (e == cudaSuccess) {
             StageTimer tm(DSA_STAGE_ATTN, st);
             e = run_attn_rows(ws + L.q + r0 * q_row, ws + L.k, ws + L.v, idx + r0 * (int64_t)k_sel, T, n, H_q,

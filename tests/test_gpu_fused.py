@@ -176,3 +176,27 @@ def test_fused_repeat_calls_same_workspace():
     _, _, b = dsa.dsa_prefill(dev, k, sm_of(128), ws=ws)
     torch.cuda.synchronize()
     assert torch.equal(a, b)
+
+
+@pytest.mark.parametrize("L", [300, 700, 5000])
+def test_prefill_host_edge_passes_match_device(L):
+    """dsa_prefill_host runs a small first pass (the last rows) and a small last
+    pass (the first rows) around full ones; per-row results do not depend on
+    the pass split, so they equal dsa_prefill's bit for bit (one pass, two
+    passes, and edge passes around a middle one)."""
+    k = 256
+    spec = dsa_synth.PrefillSpec("host_edges", L=L, H_I=64, d_I=128, k=k, H_q=128, d=128, fp8=True,
+                                 n_needles=max(1, L // 200), seed=L)
+    inp = to_dev(dsa_synth.make_prefill(spec))
+    out_d, lse_d, idx_d = dsa.dsa_prefill(inp, k, sm_of(128))
+    torch.cuda.synchronize()
+    keys = ("q_idx", "q_scale", "k_idx", "k_scale", "w", "q", "k", "v")
+    host = {key: inp[key].cpu().pin_memory() for key in keys}
+    out_h = torch.empty(out_d.shape, dtype=out_d.dtype).pin_memory()
+    lse_h = torch.empty(lse_d.shape, dtype=lse_d.dtype).pin_memory()
+    idx_h = torch.empty(idx_d.shape, dtype=idx_d.dtype).pin_memory()
+    dsa.dsa_prefill_host(host, k, out_h, sm_of(128), lse=lse_h, idx_out=idx_h)
+    torch.cuda.synchronize()
+    assert torch.equal(idx_h, idx_d.cpu())
+    assert torch.equal(out_h.view(torch.int16), out_d.cpu().view(torch.int16))
+    assert torch.equal(lse_h, lse_d.cpu())
