@@ -234,8 +234,13 @@ dsa_status dsa_prefill_rows(const void *q_idx, const float *q_scale, const void 
  *   out, lse_out (nullable), idx_out (nullable): host outputs.
  * The query rows move to the device, and their outputs back, pass by pass on
  * two copy streams of the library's own (created once per device), while the
- * indexer, top-k and attention of the previous pass run on `stream`; the keys
- * and values move first.  The call is asynchronous: the outputs are complete
+ * indexer, top-k and attention of the previous pass run on `stream`.  The
+ * index keys, their scales, the query scales and the head weights move first,
+ * then the first pass's index queries, then K and V; each pass's selection
+ * waits only for its index queries, its attention also for its bf16 queries.
+ * Passes run from the last rows to the first, the first and the last of them
+ * at most 512 rows, so that the computation starts early and little output is
+ * left to copy after it.  The call is asynchronous: the outputs are complete
  * once `stream` reaches the point after the call (e.g. cudaStreamSynchronize).
  * Host buffers must stay valid until then.
  * workspace: device memory of at least dsa_prefill_host_workspace_size(...)
