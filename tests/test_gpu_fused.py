@@ -200,3 +200,17 @@ def test_prefill_host_edge_passes_match_device(L):
     assert torch.equal(idx_h, idx_d.cpu())
     assert torch.equal(out_h.view(torch.int16), out_d.cpu().view(torch.int16))
     assert torch.equal(lse_h, lse_d.cpu())
+
+
+@pytest.mark.parametrize("H_I", [1, 12, 32])
+def test_fused_other_index_head_counts_bit_exact(H_I):
+    """The fused selection with fewer index heads than 64: 32 (vector weight loads),
+    12 and 1 (the coefficient table's scalar path) select exactly what the oracle
+    selects on the GPU's own score rows, on sampled-threshold rows."""
+    L, k = 9000, 256
+    spec = _spec(L, k, seed=H_I + 17, H_I=H_I)
+    inp = dsa_synth.make_prefill(spec)
+    dev = to_dev(inp)
+    _, _, idx = dsa.dsa_prefill(dev, k, sm_of(128))
+    rows = np.concatenate([np.arange(0, 40), np.arange(L - 600, L)])
+    _check_rows(dev, idx, rows, k)

@@ -26,7 +26,8 @@ def fp8_spec(L, H_I=64, H_q=16, k=128, seed=11, n_needles=None, d=128):
 # ------------------------------------------------------------------ indexer
 
 @pytest.mark.parametrize("L,H_I,rows", [(1000, 64, (0, 1000)), (777, 64, (130, 333)),
-                                        (300, 8, (0, 300)), (1, 64, (0, 1)), (513, 128, (500, 13))])
+                                        (300, 8, (0, 300)), (1, 64, (0, 1)), (513, 128, (500, 13)),
+                                        (900, 12, (100, 700)), (700, 32, (0, 700)), (400, 1, (0, 400))])
 def test_index_scores_fp8(L, H_I, rows):
     inp = dsa_synth.make_prefill(fp8_spec(L, H_I=H_I, seed=L + H_I))
     dev = to_dev(inp)
