@@ -214,3 +214,23 @@ def test_fused_other_index_head_counts_bit_exact(H_I):
     _, _, idx = dsa.dsa_prefill(dev, k, sm_of(128))
     rows = np.concatenate([np.arange(0, 40), np.arange(L - 600, L)])
     _check_rows(dev, idx, rows, k)
+
+
+@pytest.mark.parametrize("k,W", [(3000, 1024), (4096, 0), (4097, 0)])
+def test_fused_large_k_bit_exact(k, W):
+    """k beyond 2048 takes the finish kernel's largest candidate capacity (4 k
+    candidates a row, 64 a thread); k = 4096 is the largest fused k and 4097
+    takes the score-writing path.  Rows where every position is taken, where
+    every competing position is a candidate, and where the sampled threshold
+    applies all select exactly what the oracle selects on the GPU's scores."""
+    L = 20000
+    spec = _spec(L, k, seed=k + W)
+    inp = dsa_synth.make_prefill(spec)
+    dev = to_dev(inp)
+    if W:
+        idx = dsa.dsa_prefill_window(dev, k, W, sm_of(128))[2]
+    else:
+        _, _, idx = dsa.dsa_prefill(dev, k, sm_of(128))
+    rows = np.concatenate([np.arange(k - 3, k + 3), np.arange(4 * k + W - 3, 4 * k + W + 3),
+                           np.arange(L - 200, L)])
+    _check_rows(dev, idx, rows, k, window=W)
