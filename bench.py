@@ -46,6 +46,13 @@ SELECT_TRAFFIC = {"bytes_per_launch": 112211493, "launches": 35,
                   "profile": "profiles/index_tc_select__prefill128k_and_16k.md"}
 
 
+# L2-to-SM gather ceiling for the attention's access pattern (random 512-byte K+V
+# row pairs of an L2-resident table, 16 bytes a lane, cp.async, 8 warps per SM),
+# measured on this machine's B200 with a stand-alone gather microbenchmark: the
+# denominator of the attention's L2 fraction.
+L2_GATHER_PEAK_TBS = 20.2
+
+
 def select_traffic():
     """The recorded per-launch DRAM bytes of the select kernel, or None when no
     capture is recorded or the kernel's source changed since."""
@@ -277,6 +284,13 @@ def bench_prefill(args, dsa, spec, peaks, peak_kind, ws_n, rank):
     idx_ms = br["select"][0] + br["scores"][0]
     idx_achieved = flops["indexer_flop"] / (idx_ms * 1e-3) / 1e12
     attn_tflops = flops["attn_flop"] / (br["attention"][0] * 1e-3) / 1e12
+    # the attention's other roofs: the K/V rows it gathers (from L2, where the K/V
+    # stay) and what it moves to and from HBM (Q, O, LSE and the index lists once)
+    attn_s = br["attention"][0] * 1e-3
+    attn_gather = flops["selected"] * 2 * d * 2
+    attn_hbm = 2 * T * H_q * d * 2 + T * H_q * 4 + T * k * 4 + 2 * T * d * 2
+    attn_roofs = dict(gather_tbs=attn_gather / attn_s / 1e12, hbm_gbs=attn_hbm / attn_s / 1e9,
+                      gather_bytes=attn_gather, hbm_bytes=attn_hbm)
 
     e2e = None
     if not args.no_e2e:
@@ -286,7 +300,7 @@ def bench_prefill(args, dsa, spec, peaks, peak_kind, ws_n, rank):
     torch.cuda.empty_cache()
     return dict(step_ms=step_ms_max, ms=ms, clocks=clocks, launches=n_launch, per_kernel=per_kernel,
                 breakdown=br, flops=flops, fp8_peak=fp8_peak, idx_tflops=idx_achieved,
-                attn_tflops=attn_tflops, e2e=e2e, workspace_bytes=wsb)
+                attn_tflops=attn_tflops, attn_roofs=attn_roofs, e2e=e2e, workspace_bytes=wsb)
 
 
 def replica_spec(spec, rank):
@@ -773,6 +787,12 @@ def main():
         "attention_ms": round(br["attention"][0], 3),
         "attention_tflops": round(pre["attn_tflops"], 2),
         "attention_frac_bf16": round(pre["attn_tflops"] / peaks["bf16_tflops"], 4),
+        "attention_l2_gather": {"TB/s": round(pre["attn_roofs"]["gather_tbs"], 2),
+                                "frac": round(pre["attn_roofs"]["gather_tbs"] / L2_GATHER_PEAK_TBS, 4),
+                                "peak": L2_GATHER_PEAK_TBS, "bytes": pre["attn_roofs"]["gather_bytes"]},
+        "attention_hbm": {"GB/s": round(pre["attn_roofs"]["hbm_gbs"], 1),
+                          "frac": round(pre["attn_roofs"]["hbm_gbs"] / peaks["hbm_gbs"], 4),
+                          "bytes": pre["attn_roofs"]["hbm_bytes"]},
         "per_stage_ms": {n: round(v[0], 3) for n, v in br.items() if v[1]},
         "per_stage_runs": {n: v[1] for n, v in br.items() if v[1]},
         "workspace_bytes": pre["workspace_bytes"],
